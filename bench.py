@@ -1,0 +1,493 @@
+#!/usr/bin/env python
+"""Benchmark of the DeltaLog decode step on B200.
+
+Workload (default): GDN decode, B=256 slots, H=32 heads, d_k=d_v=128, fp32
+state (537 MB), bf16 q/k/v, merge interval M=8, synthetic seeded inputs.
+One bench step = one pass of the whole hot path over the workload's 256-token
+decode sequence for all B slots: 256/M merge cycles, each M-1 append
+launches + 1 merge launch.  ``value`` = slot-tokens per second (B * tokens
+per step * steps / time) summed over all ranks, inputs resident in HBM.
+
+``--impl reference`` times the fp64 CPU oracle instead (rank 0 only).
+
+Prints ONE JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "state-update tokens/s (B*steps/s)"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["deltalog", "reference"], default="deltalog")
+    ap.add_argument("--op", choices=["gdn", "kda", "rwkv6"], default="gdn")
+    ap.add_argument("--B", type=int, default=256)
+    ap.add_argument("--H", type=int, default=32)
+    ap.add_argument("--d", type=int, default=128)
+    ap.add_argument("--M", type=int, default=8)
+    ap.add_argument("--tokens", type=int, default=256, help="decode tokens per bench step")
+    ap.add_argument("--pool", type=int, default=64, help="distinct input tokens kept on device")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-eager", action="store_true")
+    ap.add_argument("--sweep", default="", help="extra M values to time, e.g. 1,4,16")
+    args = ap.parse_args()
+    if args.tokens % args.M:
+        ap.error("--tokens must be a multiple of --M")
+    return args
+
+
+def workload_name(a):
+    return f"{a.op}_decode_b{a.B}_h{a.H}_d{a.d}_m{a.M}_bf16"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes (what the method must move; no cache effects)
+# ---------------------------------------------------------------------------
+
+def entry_bytes(op, dk, dv, es=2):
+    """Bytes of one log entry: a_i (input dtype) + b_i + Lam_i."""
+    a = dk * es
+    b = dv * (es if op == "rwkv6" else 4)
+    lam = 4 if op == "gdn" else 4 * dk
+    return a + b + lam
+
+
+def launch_bytes(op, kind, B, H, dk, dv, n=0, es=2):
+    """Algorithmic HBM bytes of one launch over all B*H (slot, head) units.
+
+    kind: "append" (n entries in the log), "merge" (n entries before the step),
+    "eager".  Per unit: state read 4*dk*dv (+ write on merge/eager), q/k/v in,
+    o out, gates, the n log entries read (deferred only) and the appended entry
+    (append only).  The RWKV6 bonus u[H, dk] is read once per launch.
+    """
+    unit = 4 * dk * dv
+    if kind in ("merge", "eager"):
+        unit += 4 * dk * dv
+    unit += (2 * dk + dv) * es + dv * es                      # q|r, k, v in; o out
+    unit += {"gdn": 8, "kda": 4 * dk + 4, "rwkv6": 4 * dk}[op]  # gates
+    if kind != "eager":
+        unit += n * entry_bytes(op, dk, dv, es)
+    if kind == "append":
+        unit += entry_bytes(op, dk, dv, es)
+    total = unit * B * H
+    if op == "rwkv6":
+        total += H * dk * 4
+    return total
+
+
+def step_bytes(op, B, H, d, M, tokens, es=2):
+    if M == 1:
+        return tokens * launch_bytes(op, "eager", B, H, d, d, 0, es)
+    per_cycle = sum(launch_bytes(op, "append", B, H, d, d, n, es) for n in range(M - 1))
+    per_cycle += launch_bytes(op, "merge", B, H, d, d, M - 1, es)
+    return per_cycle * (tokens // M)
+
+
+def write_bytes_per_token(op, B, H, d, M, es=2):
+    """Algorithmic HBM write bytes per slot-token (all heads), averaged over a cycle."""
+    state_w = 4 * d * d
+    io_w = d * es
+    if M == 1:
+        return H * (state_w + io_w)
+    ent = entry_bytes(op, d, d, es)
+    per_cycle = (M - 1) * (io_w + ent) + (io_w + state_w)
+    return H * per_cycle / M
+
+
+# ---------------------------------------------------------------------------
+# environment helpers
+# ---------------------------------------------------------------------------
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "recurrent_state_update_deltalog_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu summary,
+    or None when there is none or the kernel sources changed since."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d[workload]
+        if e.get("source_hash") != kernel_source_hash():
+            return None
+        return e["bytes_per_launch"]
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        self.gpu = gpu_index
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[4:8]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the fp64 CPU oracle
+# ---------------------------------------------------------------------------
+
+def oracle_sample(a, slots, tokens, t0=0):
+    """Run the oracle on `slots` slots (all H heads) for `tokens` tokens; returns seconds."""
+    import numpy as np
+    from oracle import eager
+    from synthetic import bonus, initial_state, sequence
+    S0 = initial_state(a.seed, a.B, a.H, a.d, a.d, slots=range(slots))
+    seq = sequence(a.seed, a.op, slots, a.H, a.d, a.d, tokens, bf16=True, t0=t0)
+    u = bonus(a.seed, a.H, a.d) if a.op == "rwkv6" else None
+    t = time.perf_counter()
+    o, _, _ = eager(a.op, S0, seq, u=u)
+    el = time.perf_counter() - t
+    assert np.isfinite(o).all()
+    return el
+
+
+def cpu_threads():
+    """Threads the oracle uses: its contractions are numpy einsum loops without
+    BLAS dispatch, and its elementwise work is numpy ufuncs -- one thread."""
+    return 1
+
+
+def cpu_baseline(a, budget_s=10.0):
+    """Oracle throughput on a bounded sample: 1 slot (H heads), growing token count."""
+    tokens, el = 8, 0.0
+    while True:
+        el = oracle_sample(a, 1, tokens)
+        if el >= budget_s or tokens >= a.tokens:
+            break
+        tokens = min(a.tokens, max(tokens * 2, int(tokens * budget_s / max(el, 1e-3))))
+    return {"value": tokens / el, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"1 slot x {a.H} heads x {tokens} tokens of {workload_name(a)} (fp64 eager)",
+            "seconds": round(el, 3)}
+
+
+def run_reference(a, rank):
+    if rank != 0:
+        return
+    per_step_tokens = a.M * 4
+    for _ in range(a.warmup):
+        oracle_sample(a, 1, per_step_tokens)
+    times = [oracle_sample(a, 1, per_step_tokens, t0=i * per_step_tokens) for i in range(a.steps)]
+    total = sum(times)
+    value = per_step_tokens * a.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * total / a.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": workload_name(a), "op": a.op, "B": a.B, "H": a.H, "d_k": a.d,
+                   "d_v": a.d, "M": a.M, "parallelism": "cpu"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                         "sample": f"each step: 1 slot x {a.H} heads x {per_step_tokens} tokens"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def run_gpu(a, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from recurrent_state_update_deltalog_b200 import DeltaLog
+    from synthetic import bonus, initial_state, sequence
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    op, B, H, d, M = a.op, a.B, a.H, a.d, a.M
+    seed = a.seed + 1000 * rank
+    es = 2
+
+    # inputs: a pool of distinct tokens resident in HBM (> L2), cycled
+    S0 = torch.from_numpy(initial_state(seed, B, H, d, d)).to(dev)
+    seq = sequence(seed, op, B, H, d, d, a.pool, bf16=True)
+    first = "r" if op == "rwkv6" else "q"
+    names = [first, "k", "v", "log_decay"] + ([] if op == "rwkv6" else ["beta"])
+    host = {}
+    dpool = {}
+    for nm in names:
+        t = torch.from_numpy(np.ascontiguousarray(seq[nm]))
+        t = t.to(torch.bfloat16) if nm in (first, "k", "v") else t.float()
+        host[nm] = t.pin_memory()
+        dpool[nm] = t.to(dev)
+    del seq
+    u = torch.from_numpy(bonus(seed, H, d)).to(dev) if op == "rwkv6" else None
+    out = torch.empty((a.pool, B, H, d), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def tok_args(pool, i):
+        return (pool[first][i], pool["k"][i], pool["v"][i], pool["log_decay"][i],
+                pool["beta"][i] if op != "rwkv6" else None)
+
+    def make_handle(m):
+        h = DeltaLog(B, H, d, d, m, op=op, dtype=torch.bfloat16)
+        h.load_state(S0)
+        if u is not None:
+            h.set_bonus(u)
+        return h
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    tok_counter = [0]
+
+    def run_step(h, m, eager=False, ev=None, rec=None):
+        """One bench step: a.tokens decode tokens through dl_step (or dl_eager_step).
+        With `ev`, every append launch is bracketed by a pair of events (kept in `rec`)."""
+        for j in range(a.tokens):
+            i = tok_counter[0] % a.pool
+            tok_counter[0] += 1
+            args = tok_args(dpool, i)
+            if eager:
+                h.eager_step(*args, out=out[i], stream=stream)
+            elif ev is not None and (j % m) != m - 1:
+                e0, e1 = ev.pop()
+                e0.record(stream)
+                h.step(*args, out=out[i], stream=stream)
+                e1.record(stream)
+                rec.append((e0, e1, j % m))
+            else:
+                h.step(*args, out=out[i], stream=stream)
+
+    def timed(m, eager=False, per_launch=False):
+        h = make_handle(m)
+        for _ in range(a.warmup):
+            run_step(h, m, eager)
+        nev = a.steps * a.tokens if per_launch else 0
+        rec = []
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(nev)]
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        start.record(stream)
+        for _ in range(a.steps):
+            run_step(h, m, eager, ev if per_launch else None, rec)
+        stop.record(stream)
+        barrier()
+        ms = start.elapsed_time(stop)
+        launches = None
+        if per_launch:
+            launches = [(e0.elapsed_time(e1), n) for e0, e1, n in rec]
+        h.check_device(stream)
+        h.close()
+        return max_over_ranks(ms), launches
+
+    peak, peak_kind = measured_peak()
+    result = {}
+
+    # headline: DeltaLog at M, with per-launch timing of the dominant (append) kernel
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    ms, launches = timed(M, per_launch=M > 1)
+    clocks = sampler.stop()
+    tokens_total = B * a.tokens * a.steps * world
+    value = tokens_total / (ms / 1e3)
+    sb = step_bytes(op, B, H, d, M, a.tokens)
+    result["value"] = value
+    result["ms"] = ms
+
+    if M > 1 and launches:
+        dur = sum(t for t, _ in launches) / len(launches)
+        alg = sum(launch_bytes(op, "append", B, H, d, d, n) for _, n in launches) / len(launches)
+        dominant = "deltalog_step_kernel (append)"
+    else:
+        dur = ms / (a.steps * a.tokens)
+        alg = launch_bytes(op, "eager" if M == 1 else "merge", B, H, d, d, 0)
+        dominant = "deltalog_step_kernel (merge, M=1)"
+    achieved = alg / (dur / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": profiled_traffic(workload_name(a)),
+                "kernel": dominant, "avg_launch_us": dur * 1e3,
+                "alg_bytes_per_launch": alg, "peak_source": peak_kind,
+                "step_gbs": sb / (ms / a.steps / 1e3) / 1e9}
+
+    extra = {}
+    if not a.no_eager:
+        ems, _ = timed(1, eager=True)
+        eb = step_bytes(op, B, H, d, 1, a.tokens)
+        extra["eager"] = {"value": B * a.tokens * a.steps * world / (ems / 1e3), "unit": UNIT,
+                          "ms_per_step": ems / a.steps,
+                          "gbs": eb / (ems / a.steps / 1e3) / 1e9,
+                          "frac": eb / (ems / a.steps / 1e3) / 1e9 / peak,
+                          "write_bytes_per_token": write_bytes_per_token(op, B, H, d, 1)}
+        extra["speedup_vs_eager"] = value / extra["eager"]["value"]
+    sweep = {}
+    for mv in [int(x) for x in a.sweep.split(",") if x.strip()]:
+        if a.tokens % mv:
+            continue
+        sms, _ = timed(mv)
+        sbb = step_bytes(op, B, H, d, mv, a.tokens)
+        sweep[str(mv)] = {"value": B * a.tokens * a.steps * world / (sms / 1e3),
+                          "gbs": sbb / (sms / a.steps / 1e3) / 1e9,
+                          "write_bytes_per_token": write_bytes_per_token(op, B, H, d, mv)}
+    if sweep:
+        extra["sweep"] = sweep
+
+    # end to end: host (pinned) inputs -> dl_step_host -> host outputs, every token
+    e2e = None
+    if not a.no_e2e:
+        h = make_handle(M)
+        hout = torch.empty((B, H, d), dtype=torch.bfloat16).pin_memory()
+
+        def host_step():
+            for j in range(a.tokens):
+                i = tok_counter[0] % a.pool
+                tok_counter[0] += 1
+                h.step_host(*tok_args(host, i), out=hout, stream=stream)
+
+        for _ in range(a.warmup):
+            host_step()
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        start.record(stream)
+        for _ in range(a.steps):
+            host_step()
+        stop.record(stream)
+        barrier()
+        e_ms = max_over_ranks(start.elapsed_time(stop))
+        h.close()
+        h2d = sum(host[nm][0].numel() * host[nm].element_size() for nm in names) * a.tokens
+        d2h = hout.numel() * hout.element_size() * a.tokens
+        e2e = {"value": B * a.tokens * a.steps * world / (e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "api": "dl_step_host (pinned host buffers, copies on the step's stream)"}
+
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": result["value"], "unit": UNIT, "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": result["ms"] / a.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": workload_name(a), "op": op, "B": B, "H": H, "d_k": d, "d_v": d,
+                   "M": M, "state": "fp32", "inputs": "bf16", "tokens_per_step": a.tokens,
+                   "input_pool_tokens": a.pool, "seed": a.seed,
+                   "l2": f"inputs larger than L2 (state {4 * B * H * d * d / 1e6:.0f} MB)",
+                   "parallelism": "replicas" if world == 1 else f"replicas x{world} (B per rank)"},
+        "roofline": roofline,
+        "gpu_launches": a.steps * a.tokens,
+        "write_bytes_per_token": write_bytes_per_token(op, B, H, d, M),
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    line.update(extra)
+    if not a.no_cpu and world == 1:
+        line["cpu_baseline"] = cpu_baseline(a)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    a = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if a.impl == "reference":
+        run_reference(a, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_gpu(a, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,136 @@
+/*
+ * deltalog.h -- C ABI of libdeltalog, the DeltaLog decode step for
+ * linear-attention recurrent state on NVIDIA B200 (sm_100a).
+ *
+ * What it computes.  Per (slot, head) the logical recurrent state
+ * S_t in R^{d_k x d_v} of one of three operators (DeltaLog technical summary,
+ * gist.science, section "Kernel implementation", operator list):
+ *   GDN    S_t = a_t S_{t-1} + k_t b_t^T,  b_t = beta_t (v_t - a_t S_{t-1}^T k_t),
+ *          o_t = S_t^T q_t                        (a_t scalar per head)
+ *   KDA    S_t = diag(a_t) S_{t-1} + k_t b_t^T,
+ *          b_t = beta_t (v_t - (diag(a_t) S_{t-1})^T k_t),  o_t = S_t^T q_t
+ *   RWKV6  o_t = (S_{t-1} + diag(u) k_t v_t^T)^T r_t,
+ *          S_t = diag(w_t) S_{t-1} + k_t v_t^T
+ * is kept as a dense fp32 base Sbar plus a bounded log of compact factors
+ * (a_i = k_i, b_i) with a log-decay snapshot Lam_i per entry (same summary,
+ * section "Method -- core mechanism: base + log").  Steps 1..M-1 of each
+ * cycle only append one entry; step M computes its output and writes the
+ * full state back into Sbar, emptying the log ("append phase" / "merge
+ * phase").  Every output equals the eager recurrence's up to rounding
+ * (arXiv 2608.15533 abstract: the model sees the same dense state as eager
+ * decoding).  dl_eager_step is the dense baseline that reads and writes the
+ * whole state every token (summary, section "Problem: the state-update tax").
+ *
+ * Layouts (all C-contiguous, row-major, last index fastest):
+ *   state      float  [B][H][d_k][d_v]     (d_v contiguous)
+ *   q / r, k   in_dtype [B][H][d_k]
+ *   v          in_dtype [B][H][d_v]
+ *   o          in_dtype [B][H][d_v]
+ *   log_decay  float  [B][H]       GDN: natural log of a_t (<= 0)
+ *              float  [B][H][d_k]  KDA: log a_t per key; RWKV6: log w_t per key
+ *   beta       float  [B][H]       GDN and KDA; must be NULL for RWKV6
+ *   u          float  [H][d_k]     RWKV6 bonus (dl_set_bonus)
+ * in_dtype is DL_F32 (float) or DL_BF16 (bfloat16, IEEE upper half).
+ * Decays enter as natural logs: the library never divides by a cumulative
+ * decay; every replay ratio is exp(Lam_t - Lam_i) <= 1.
+ *
+ * Ownership.  The caller owns every pointer it passes and the stream.  The
+ * handle owns Sbar, the log and small host-staging buffers, allocated by
+ * dl_create on the device current at that time and freed by dl_destroy.
+ * Every call runs on that device (the caller's current device is restored).
+ * All device-pointer calls are asynchronous on `stream` (a cudaStream_t, NULL
+ * = legacy default stream): inputs must stay valid and outputs must not be
+ * read until the stream reaches the call.  A handle must not be used from two
+ * host threads at once, nor on two streams whose work overlaps.
+ *
+ * Errors.  Every int-returning call returns DL_OK (0) or a negative
+ * dl_status; nothing aborts, throws or traps.  On an error the handle is
+ * unchanged, except DL_ERR_CUDA after work was already queued.
+ * dl_last_error() gives a message for the last failing call of this thread.
+ */
+#ifndef DELTALOG_H
+#define DELTALOG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct dl_handle* dl_t;
+
+enum dl_op { DL_GDN = 0, DL_KDA = 1, DL_RWKV6 = 2 };
+enum dl_dtype { DL_F32 = 0, DL_BF16 = 1 };
+
+enum dl_status {
+  DL_OK = 0,
+  DL_ERR_ARG = -1,          /* null handle/pointer, bad size, misaligned pointer */
+  DL_ERR_UNSUPPORTED = -2,  /* (op, d_k, d_v, dtype, M) not compiled in */
+  DL_ERR_CUDA = -3,         /* a CUDA runtime call or kernel launch failed */
+  DL_ERR_OOM = -4,          /* device or pinned allocation failed */
+  DL_ERR_DEVICE = -5,       /* a kernel raised the handle's device error word */
+  DL_ERR_STATE = -6         /* call not valid in the handle's current state */
+};
+
+/* Create a handle for B slots x H heads.  Supported: d_k, d_v in {64, 128},
+ * 1 <= M <= DL_MAX_M.  The base state starts at zero with an empty log; the
+ * RWKV6 bonus starts at zero.  Pointers passed later must be 16-byte aligned.
+ * M = 1 makes every step a merge step (the deferred path then performs the
+ * eager schedule). */
+#define DL_MAX_M 64
+int dl_create(dl_t* out, int B, int H, int d_k, int d_v, int M, int op, int in_dtype);
+
+/* Free everything the handle owns.  Synchronises the handle's device first.
+ * NULL is accepted and ignored. */
+int dl_destroy(dl_t h);
+
+/* Copy the dense state S [B][H][d_k][d_v] (device pointer) into Sbar and empty
+ * the log: the next step starts a new merge cycle. */
+int dl_load_state(dl_t h, const float* S, void* stream);
+
+/* RWKV6 only: copy the bonus u [H][d_k] (device pointer). */
+int dl_set_bonus(dl_t h, const float* u, void* stream);
+
+/* One DeltaLog decode token for all B slots and H heads.  q is r for RWKV6.
+ * With n entries in the log before the call: if n + 1 < M the step appends
+ * (Sbar is read, never written); if n + 1 == M it merges (Sbar <- S_t and the
+ * log empties).  Writes o [B][H][d_v].  All pointers are device pointers. */
+int dl_step(dl_t h, const void* q, const void* k, const void* v,
+            const float* log_decay, const float* beta, void* o, void* stream);
+
+/* Same as dl_step with HOST pointers (pinned or pageable): copies the inputs
+ * into handle-owned device buffers, runs the step and copies o back, all on
+ * `stream`.  o is valid once the stream has reached the call. */
+int dl_step_host(dl_t h, const void* q, const void* k, const void* v,
+                 const float* log_decay, const float* beta, void* o, void* stream);
+
+/* Eager dense baseline: read S_{t-1} from Sbar, write S_t back, every token.
+ * Requires an empty log (returns DL_ERR_STATE otherwise; call dl_merge). */
+int dl_eager_step(dl_t h, const void* q, const void* k, const void* v,
+                  const float* log_decay, const float* beta, void* o, void* stream);
+
+/* Fold the log into Sbar now (no output) and empty it; a no-op on an empty
+ * log.  For an explicit flush, slot eviction or a checkpoint. */
+int dl_merge(dl_t h, void* stream);
+
+/* Write the logical state (Sbar + replayed log) to S_out [B][H][d_k][d_v]
+ * (device pointer) without changing the handle. */
+int dl_read_state(dl_t h, float* S_out, void* stream);
+
+/* Number of entries currently in the log (host-side counter, exact in stream
+ * order). */
+int dl_log_len(dl_t h, int* n);
+
+/* Read and clear the handle's device error word (synchronises `stream`).
+ * Returns DL_OK or DL_ERR_DEVICE. */
+int dl_check_device(dl_t h, void* stream);
+
+/* Static text for a status code, and the last error message of this thread. */
+const char* dl_strerror(int status);
+const char* dl_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DELTALOG_H */

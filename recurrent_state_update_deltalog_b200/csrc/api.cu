@@ -1,0 +1,377 @@
+// C ABI of libdeltalog: handle lifetime, argument validation and launches.
+// The contract of every entry point is documented in include/deltalog.h.
+#include "deltalog.h"
+#include "launch.cuh"
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <new>
+#include <string>
+
+struct dl_handle {
+  int B, H, dk, dv, M, op, dtype, device;
+  int n;       // entries in the log (host counter; all slots step in lockstep)
+  int Mcap;    // log capacity per (slot, head): max(M - 1, 1)
+  size_t esize;
+  float* Sbar;
+  void* logA;
+  void* logB;
+  float* logLam;
+  float* u;
+  int* err;
+  // device staging for dl_step_host
+  void* sq;
+  void* sk;
+  void* sv;
+  void* so;
+  float* sld;
+  float* sbeta;
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(DL_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// Makes the handle's device current for the scope of a call and restores the
+// caller's device afterwards.
+class DeviceScope {
+ public:
+  explicit DeviceScope(int dev) {
+    ok_ = cudaGetDevice(&prev_) == cudaSuccess;
+    if (ok_ && prev_ != dev) {
+      ok_ = cudaSetDevice(dev) == cudaSuccess;
+      changed_ = ok_;
+    }
+  }
+  ~DeviceScope() {
+    if (changed_) cudaSetDevice(prev_);
+  }
+  bool ok() const { return ok_; }
+
+ private:
+  int prev_ = 0;
+  bool ok_ = false;
+  bool changed_ = false;
+};
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t lam_per_entry(const dl_handle* h) { return h->op == DL_GDN ? 1 : static_cast<size_t>(h->dk); }
+size_t logb_esize(const dl_handle* h) { return h->op == DL_RWKV6 ? h->esize : sizeof(float); }
+size_t bh(const dl_handle* h) { return static_cast<size_t>(h->B) * h->H; }
+size_t state_bytes(const dl_handle* h) { return bh(h) * h->dk * h->dv * sizeof(float); }
+size_t decay_elems(const dl_handle* h) { return bh(h) * lam_per_entry(h); }
+
+void free_all(dl_handle* h) {
+  void* ptrs[] = {h->Sbar, h->logA, h->logB, h->logLam, h->u, h->err,
+                  h->sq, h->sk, h->sv, h->so, h->sld, h->sbeta};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+}
+
+dl::LaunchShape shape_of(const dl_handle* h) {
+  return dl::LaunchShape{static_cast<int>(bh(h)), h->dk, h->dv, h->dtype};
+}
+
+int check_step_args(const dl_handle* h, const void* q, const void* k, const void* v,
+                    const float* log_decay, const float* beta, const void* o) {
+  if (!h) return fail(DL_ERR_ARG, "null handle");
+  if (!q || !k || !v || !log_decay || !o) return fail(DL_ERR_ARG, "null input/output pointer");
+  if (h->op == DL_RWKV6 && beta) return fail(DL_ERR_ARG, "beta must be NULL for RWKV6");
+  if (h->op != DL_RWKV6 && !beta) return fail(DL_ERR_ARG, "beta is required for GDN/KDA");
+  const void* tp[] = {q, k, v, o};
+  for (const void* p : tp)
+    if (!aligned(p, h->esize)) return fail(DL_ERR_ARG, "input/output pointer not aligned to its element size");
+  if (!aligned(log_decay, 4) || (beta && !aligned(beta, 4))) return fail(DL_ERR_ARG, "gate pointer not 4-byte aligned");
+  return DL_OK;
+}
+
+dl::StepArgs step_args(dl_handle* h, const void* q, const void* k, const void* v,
+                       const float* log_decay, const float* beta, void* o) {
+  dl::StepArgs a;
+  a.Sbar = h->Sbar;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.log_decay = log_decay;
+  a.beta = beta;
+  a.o = o;
+  a.logA = h->logA;
+  a.logB = h->logB;
+  a.logLam = h->logLam;
+  a.u = h->u;
+  a.H = h->H;
+  a.Mcap = h->Mcap;
+  a.n = h->n;
+  return a;
+}
+
+cudaError_t launch_step(const dl_handle* h, bool merge, const dl::StepArgs& a, cudaStream_t s) {
+  const dl::LaunchShape sh = shape_of(h);
+  switch (h->op) {
+    case DL_GDN: return dl::launch_step_op<dl::OP_GDN>(sh, merge, a, s);
+    case DL_KDA: return dl::launch_step_op<dl::OP_KDA>(sh, merge, a, s);
+    default: return dl::launch_step_op<dl::OP_RWKV6>(sh, merge, a, s);
+  }
+}
+
+cudaError_t launch_eager(const dl_handle* h, const dl::StepArgs& a, cudaStream_t s) {
+  const dl::LaunchShape sh = shape_of(h);
+  switch (h->op) {
+    case DL_GDN: return dl::launch_eager_op<dl::OP_GDN>(sh, a, s);
+    case DL_KDA: return dl::launch_eager_op<dl::OP_KDA>(sh, a, s);
+    default: return dl::launch_eager_op<dl::OP_RWKV6>(sh, a, s);
+  }
+}
+
+cudaError_t launch_materialize(const dl_handle* h, float* out, cudaStream_t s) {
+  dl::MaterializeArgs a;
+  a.Sin = h->Sbar;
+  a.Sout = out;
+  a.logA = h->logA;
+  a.logB = h->logB;
+  a.logLam = h->logLam;
+  a.Mcap = h->Mcap;
+  a.n = h->n;
+  const dl::LaunchShape sh = shape_of(h);
+  switch (h->op) {
+    case DL_GDN: return dl::launch_materialize_op<dl::OP_GDN>(sh, a, s);
+    case DL_KDA: return dl::launch_materialize_op<dl::OP_KDA>(sh, a, s);
+    default: return dl::launch_materialize_op<dl::OP_RWKV6>(sh, a, s);
+  }
+}
+
+int do_step(dl_handle* h, const void* q, const void* k, const void* v, const float* log_decay,
+            const float* beta, void* o, cudaStream_t s) {
+  const bool merge = h->n + 1 == h->M;
+  cudaError_t e = launch_step(h, merge, step_args(h, q, k, v, log_decay, beta, o), s);
+  if (e != cudaSuccess) return cuda_fail(e, "deltalog step launch");
+  h->n = merge ? 0 : h->n + 1;
+  return DL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dl_create(dl_t* out, int B, int H, int d_k, int d_v, int M, int op, int in_dtype) {
+  if (!out) return fail(DL_ERR_ARG, "null output handle pointer");
+  *out = nullptr;
+  if (B <= 0 || H <= 0) return fail(DL_ERR_ARG, "B and H must be positive (B=%d H=%d)", B, H);
+  if (M < 1 || M > DL_MAX_M) return fail(DL_ERR_UNSUPPORTED, "M=%d outside [1, %d]", M, DL_MAX_M);
+  if (op < DL_GDN || op > DL_RWKV6) return fail(DL_ERR_ARG, "unknown op %d", op);
+  if (in_dtype != DL_F32 && in_dtype != DL_BF16) return fail(DL_ERR_ARG, "unknown dtype %d", in_dtype);
+  const bool dk_ok = d_k == 64 || d_k == 128, dv_ok = d_v == 64 || d_v == 128;
+  if (!dk_ok || !dv_ok) return fail(DL_ERR_UNSUPPORTED, "d_k=%d d_v=%d not in {64,128}", d_k, d_v);
+  if (static_cast<long long>(B) * H > (1ll << 30)) return fail(DL_ERR_ARG, "B*H too large");
+
+  dl_handle* h = new (std::nothrow) dl_handle();
+  if (!h) return fail(DL_ERR_OOM, "host allocation failed");
+  h->B = B;
+  h->H = H;
+  h->dk = d_k;
+  h->dv = d_v;
+  h->M = M;
+  h->op = op;
+  h->dtype = in_dtype;
+  h->n = 0;
+  h->Mcap = M > 1 ? M - 1 : 1;
+  h->esize = in_dtype == DL_BF16 ? 2 : 4;
+  if (cudaGetDevice(&h->device) != cudaSuccess) {
+    delete h;
+    return fail(DL_ERR_CUDA, "no current CUDA device");
+  }
+  const size_t nbh = bh(h);
+  struct {
+    void** p;
+    size_t bytes;
+  } allocs[] = {
+      {reinterpret_cast<void**>(&h->Sbar), state_bytes(h)},
+      {&h->logA, nbh * h->Mcap * d_k * h->esize},
+      {&h->logB, nbh * h->Mcap * d_v * logb_esize(h)},
+      {reinterpret_cast<void**>(&h->logLam), nbh * h->Mcap * lam_per_entry(h) * sizeof(float)},
+      {reinterpret_cast<void**>(&h->u), static_cast<size_t>(H) * d_k * sizeof(float)},
+      {reinterpret_cast<void**>(&h->err), sizeof(int)},
+      {&h->sq, nbh * d_k * h->esize},
+      {&h->sk, nbh * d_k * h->esize},
+      {&h->sv, nbh * d_v * h->esize},
+      {&h->so, nbh * d_v * h->esize},
+      {reinterpret_cast<void**>(&h->sld), decay_elems(h) * sizeof(float)},
+      {reinterpret_cast<void**>(&h->sbeta), nbh * sizeof(float)},
+  };
+  for (auto& a : allocs) {
+    cudaError_t e = cudaMalloc(a.p, a.bytes);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      free_all(h);
+      delete h;
+      return fail(e == cudaErrorMemoryAllocation ? DL_ERR_OOM : DL_ERR_CUDA,
+                  "cudaMalloc of %zu bytes failed: %s", a.bytes, cudaGetErrorString(e));
+    }
+  }
+  cudaError_t e = cudaMemset(h->Sbar, 0, state_bytes(h));
+  if (e == cudaSuccess) e = cudaMemset(h->u, 0, static_cast<size_t>(H) * d_k * sizeof(float));
+  if (e == cudaSuccess) e = cudaMemset(h->err, 0, sizeof(int));
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    free_all(h);
+    delete h;
+    return cuda_fail(e, "dl_create initialisation");
+  }
+  *out = h;
+  return DL_OK;
+}
+
+int dl_destroy(dl_t h) {
+  if (!h) return DL_OK;
+  DeviceScope ds(h->device);
+  free_all(h);
+  delete h;
+  return ds.ok() ? DL_OK : fail(DL_ERR_CUDA, "could not select the handle's device");
+}
+
+int dl_load_state(dl_t h, const float* S, void* stream) {
+  if (!h) return fail(DL_ERR_ARG, "null handle");
+  if (!S || !aligned(S, 16)) return fail(DL_ERR_ARG, "state pointer null or not 16-byte aligned");
+  DeviceScope ds(h->device);
+  if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
+  cudaError_t e = cudaMemcpyAsync(h->Sbar, S, state_bytes(h), cudaMemcpyDeviceToDevice,
+                                  static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "dl_load_state copy");
+  h->n = 0;
+  return DL_OK;
+}
+
+int dl_set_bonus(dl_t h, const float* u, void* stream) {
+  if (!h) return fail(DL_ERR_ARG, "null handle");
+  if (h->op != DL_RWKV6) return fail(DL_ERR_STATE, "dl_set_bonus is for RWKV6 handles only");
+  if (!u || !aligned(u, 4)) return fail(DL_ERR_ARG, "bonus pointer null or misaligned");
+  DeviceScope ds(h->device);
+  if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
+  cudaError_t e = cudaMemcpyAsync(h->u, u, static_cast<size_t>(h->H) * h->dk * sizeof(float),
+                                  cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DL_OK : cuda_fail(e, "dl_set_bonus copy");
+}
+
+int dl_step(dl_t h, const void* q, const void* k, const void* v, const float* log_decay,
+            const float* beta, void* o, void* stream) {
+  int rc = check_step_args(h, q, k, v, log_decay, beta, o);
+  if (rc != DL_OK) return rc;
+  DeviceScope ds(h->device);
+  if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
+  return do_step(h, q, k, v, log_decay, beta, o, static_cast<cudaStream_t>(stream));
+}
+
+int dl_step_host(dl_t h, const void* q, const void* k, const void* v, const float* log_decay,
+                 const float* beta, void* o, void* stream) {
+  int rc = check_step_args(h, q, k, v, log_decay, beta, o);
+  if (rc != DL_OK) return rc;
+  DeviceScope ds(h->device);
+  if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t nbh = bh(h);
+  struct {
+    void* dst;
+    const void* src;
+    size_t bytes;
+  } in[] = {
+      {h->sq, q, nbh * h->dk * h->esize},
+      {h->sk, k, nbh * h->dk * h->esize},
+      {h->sv, v, nbh * h->dv * h->esize},
+      {h->sld, log_decay, decay_elems(h) * sizeof(float)},
+      {h->sbeta, beta, beta ? nbh * sizeof(float) : 0},
+  };
+  for (auto& c : in) {
+    if (!c.bytes) continue;
+    cudaError_t e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "dl_step_host input copy");
+  }
+  rc = do_step(h, h->sq, h->sk, h->sv, h->sld, beta ? h->sbeta : nullptr, h->so, s);
+  if (rc != DL_OK) return rc;
+  cudaError_t e = cudaMemcpyAsync(o, h->so, nbh * h->dv * h->esize, cudaMemcpyDeviceToHost, s);
+  return e == cudaSuccess ? DL_OK : cuda_fail(e, "dl_step_host output copy");
+}
+
+int dl_eager_step(dl_t h, const void* q, const void* k, const void* v, const float* log_decay,
+                  const float* beta, void* o, void* stream) {
+  int rc = check_step_args(h, q, k, v, log_decay, beta, o);
+  if (rc != DL_OK) return rc;
+  if (h->n != 0) return fail(DL_ERR_STATE, "eager step needs an empty log (n=%d); call dl_merge", h->n);
+  DeviceScope ds(h->device);
+  if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
+  cudaError_t e = launch_eager(h, step_args(h, q, k, v, log_decay, beta, o), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DL_OK : cuda_fail(e, "eager step launch");
+}
+
+int dl_merge(dl_t h, void* stream) {
+  if (!h) return fail(DL_ERR_ARG, "null handle");
+  if (h->n == 0) return DL_OK;
+  DeviceScope ds(h->device);
+  if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
+  cudaError_t e = launch_materialize(h, h->Sbar, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  h->n = 0;
+  return DL_OK;
+}
+
+int dl_read_state(dl_t h, float* S_out, void* stream) {
+  if (!h) return fail(DL_ERR_ARG, "null handle");
+  if (!S_out || !aligned(S_out, 16)) return fail(DL_ERR_ARG, "output pointer null or not 16-byte aligned");
+  DeviceScope ds(h->device);
+  if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = h->n == 0 ? cudaMemcpyAsync(S_out, h->Sbar, state_bytes(h), cudaMemcpyDeviceToDevice, s)
+                            : launch_materialize(h, S_out, s);
+  return e == cudaSuccess ? DL_OK : cuda_fail(e, "dl_read_state");
+}
+
+int dl_log_len(dl_t h, int* n) {
+  if (!h || !n) return fail(DL_ERR_ARG, "null argument");
+  *n = h->n;
+  return DL_OK;
+}
+
+int dl_check_device(dl_t h, void* stream) {
+  if (!h) return fail(DL_ERR_ARG, "null handle");
+  DeviceScope ds(h->device);
+  if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int flag = 0;
+  cudaError_t e = cudaMemcpyAsync(&flag, h->err, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess && flag) e = cudaMemsetAsync(h->err, 0, sizeof(int), s);
+  if (e != cudaSuccess) return cuda_fail(e, "dl_check_device");
+  return flag ? fail(DL_ERR_DEVICE, "device error word 0x%x", flag) : DL_OK;
+}
+
+const char* dl_strerror(int status) {
+  switch (status) {
+    case DL_OK: return "ok";
+    case DL_ERR_ARG: return "invalid argument";
+    case DL_ERR_UNSUPPORTED: return "unsupported configuration";
+    case DL_ERR_CUDA: return "CUDA error";
+    case DL_ERR_OOM: return "out of memory";
+    case DL_ERR_DEVICE: return "device-side error flag raised";
+    case DL_ERR_STATE: return "call not valid in the current handle state";
+    default: return "unknown status";
+  }
+}
+
+const char* dl_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

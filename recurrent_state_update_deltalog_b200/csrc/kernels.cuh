@@ -1,0 +1,540 @@
+// DeltaLog decode kernels for sm_100a: deferred step (append / merge-fused),
+// eager dense baseline, and log materialisation.
+//
+// Method (DeltaLog technical summary, gist.science, sections "Method -- core
+// mechanism: base + log" and "Kernel implementation"): the logical state of a
+// (slot, head) after step t is
+//     S_t = diag(e^{Lam_t}) Sbar + sum_{i in log} diag(e^{Lam_t - Lam_i}) a_i b_i^T
+// with a_i = k_i and Lam the cumulative natural-log decay since the last
+// merge (a scalar for GDN, a per-key vector for KDA and RWKV6).  Append steps
+// read Sbar and add one log entry; every M-th step writes S_t back to Sbar.
+//
+// Work decomposition on B200.  One CTA owns one (slot, head): the key-side
+// "ReplayPrep" coefficients (decay ratios, a_i.k_t, a_i.q_t) are computed once
+// per CTA by its warps and shared through shared memory with every value tile
+// of that head, so nothing key-side is recomputed per value tile.  Value tiles
+// are the float4 column groups of the CTA's threads: thread (rg, c4) holds
+// rows [rg*RPT, rg*RPT+RPT) x columns [4*c4, 4*c4+4) of the fp32 state in
+// registers.  All state loads of a CTA are issued up front as 128-bit
+// streaming loads (64 KB in flight per CTA at d = 128), the two contractions
+// Sbar^T k~ and Sbar^T q~ are formed in one pass over those registers, and the
+// d_k reduction crosses row groups through a small shared-memory stage.  On a
+// merge step the rank-(n+1) update is applied to the same registers and
+// stored back with 128-bit streaming stores, so Sbar crosses HBM once each
+// way.  No tensor cores: this is matrix-vector work at ~1 flop/byte.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <type_traits>
+
+namespace dl {
+
+enum { OP_GDN = 0, OP_KDA = 1, OP_RWKV6 = 2 };
+
+// Arguments of one deferred step (device pointers; sizes in elements).
+struct StepArgs {
+  float* Sbar;             // [BH][DK][DV]
+  const void* q;           // [BH][DK] (r for RWKV6), input dtype
+  const void* k;           // [BH][DK]
+  const void* v;           // [BH][DV]
+  const float* log_decay;  // [BH] (GDN) or [BH][DK]
+  const float* beta;       // [BH] (GDN/KDA)
+  void* o;                 // [BH][DV], input dtype
+  void* logA;              // [BH][Mcap][DK], input dtype (a_i = k_i)
+  void* logB;              // [BH][Mcap][DV], fp32 (GDN/KDA) or input dtype (RWKV6)
+  float* logLam;           // [BH][Mcap] (GDN) or [BH][Mcap][DK]
+  const float* u;          // [H][DK] (RWKV6)
+  int H;
+  int Mcap;                // log capacity per (slot, head), >= 1
+  int n;                   // entries in the log before this step
+};
+
+// Arguments of log materialisation: Sout = Sbar + replayed log (n >= 1).
+struct MaterializeArgs {
+  const float* Sin;
+  float* Sout;
+  const void* logA;
+  const void* logB;
+  const float* logLam;
+  int Mcap;
+  int n;
+};
+
+template <typename T>
+__device__ __forceinline__ float to_f(T x);
+template <>
+__device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f(float x);
+template <>
+__device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// 128-bit loads/stores of the state: streaming (evict-first) so the state,
+// which is far larger than L2, does not push the log and inputs out of L2.
+__device__ __forceinline__ float4 ld_state(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }
+__device__ __forceinline__ void st_state(float* p, float4 v) { __stcs(reinterpret_cast<float4*>(p), v); }
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+  return x;
+}
+
+__device__ __forceinline__ void fma4(float4& acc, float a, float4 b) {
+  acc.x = fmaf(a, b.x, acc.x);
+  acc.y = fmaf(a, b.y, acc.y);
+  acc.z = fmaf(a, b.z, acc.z);
+  acc.w = fmaf(a, b.w, acc.w);
+}
+
+template <int DK, int DV>
+struct Tile {
+  static constexpr int NT = 2 * DV;      // threads per CTA
+  static constexpr int TPR = DV / 4;     // threads that cover one state row with float4s
+  static constexpr int RG = NT / TPR;    // row groups (= 8)
+  static constexpr int RPT = DK / RG;    // rows held by each thread
+  static constexpr int NW = NT / 32;     // warps
+  static constexpr int KPL = DK / 32;    // keys per lane in warp-wide key loops
+  static constexpr int MINB = NT >= 256 ? 2 : 4;
+  static_assert(DV % 64 == 0 && DK % 32 == 0 && RG == 8 && RPT % 4 == 0, "tile shape");
+  static_assert(DK <= NT && DV <= NT, "one thread per key / value in setup phases");
+};
+
+// Prefetched log values per finalize thread (entries beyond this are loaded late).
+constexpr int kPrefetch = 8;
+
+// Largest supported merge interval M (log capacity M-1).
+constexpr int kMaxM = 64;
+
+// ---------------------------------------------------------------------------
+// Deferred step.  MERGE=false: append (Sbar read only).  MERGE=true: the step
+// with n+1 == M; it also writes S_t over Sbar.
+// ---------------------------------------------------------------------------
+template <int OP, int DK, int DV, typename TI, bool MERGE>
+__global__ void __launch_bounds__(Tile<DK, DV>::NT, Tile<DK, DV>::MINB)
+deltalog_step_kernel(const StepArgs a) {
+  using TL = Tile<DK, DV>;
+  using TB = typename std::conditional<OP == OP_RWKV6, TI, float>::type;
+  constexpr bool DELTA = OP != OP_RWKV6;
+  constexpr bool PERKEY = OP != OP_GDN;
+
+  __shared__ __align__(16) float s_kt[DK];       // k~ = e^{Lam_t} (.) k   (GDN/KDA)
+  __shared__ __align__(16) float s_qt[DK];       // q~ (GDN/KDA: e^{Lam_t}; RWKV6: e^{Lam_{t-1}})
+  __shared__ __align__(16) float s_dec[DK];      // e^{Lam_t} per row (merge)
+  __shared__ __align__(16) float s_red[2][TL::RG][DV];
+  __shared__ float s_ck[kMaxM], s_cq[kMaxM];
+  __shared__ float s_kappa;
+  extern __shared__ __align__(16) float s_dyn[];  // merge: As[(n+1)][DK], Bs[(n+1)][DV]
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int c4 = tid % TL::TPR, rg = tid / TL::TPR;
+  const long sh = blockIdx.x;
+  const int h = static_cast<int>(sh % a.H);
+  const int n = a.n;
+
+  // 1. Stream this head's Sbar tile into registers (all loads in flight).
+  float* Sp = a.Sbar + sh * (DK * DV);
+  float4 st[TL::RPT];
+#pragma unroll
+  for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + (rg * TL::RPT + j) * DV + 4 * c4);
+
+  // 2. Key-side values for this lane's keys j = lane + 32 m.
+  const TI* qg = static_cast<const TI*>(a.q) + sh * DK;
+  const TI* kg = static_cast<const TI*>(a.k) + sh * DK;
+  float kr[TL::KPL], qr[TL::KPL], lt[TL::KPL], lp[TL::KPL];
+  if (PERKEY) {
+    const float* lamp = a.logLam + (sh * a.Mcap + (n > 0 ? n - 1 : 0)) * DK;
+#pragma unroll
+    for (int m = 0; m < TL::KPL; ++m) {
+      const int j = lane + 32 * m;
+      kr[m] = to_f(kg[j]);
+      qr[m] = to_f(qg[j]);
+      lp[m] = n > 0 ? lamp[j] : 0.f;
+      lt[m] = lp[m] + a.log_decay[sh * DK + j];
+    }
+  } else {
+    const float lprev = n > 0 ? a.logLam[sh * a.Mcap + (n - 1)] : 0.f;
+    const float lcur = lprev + a.log_decay[sh];
+#pragma unroll
+    for (int m = 0; m < TL::KPL; ++m) {
+      const int j = lane + 32 * m;
+      kr[m] = to_f(kg[j]);
+      qr[m] = to_f(qg[j]);
+      lp[m] = lprev;
+      lt[m] = lcur;
+    }
+  }
+
+  // Finalize threads (one per value column) prefetch v, beta and early log b's.
+  const int c = tid;
+  float vc = 0.f, betac = 0.f;
+  float bpre[kPrefetch];
+  const TB* logBh = static_cast<const TB*>(a.logB) + sh * a.Mcap * DV;
+  if (c < DV) {
+    vc = to_f(static_cast<const TI*>(a.v)[sh * DV + c]);
+    if (DELTA) betac = a.beta[sh];
+    if (!MERGE) {
+#pragma unroll
+      for (int i = 0; i < kPrefetch; ++i) bpre[i] = i < n ? to_f(logBh[i * DV + c]) : 0.f;
+    }
+  }
+
+  float* As = s_dyn;                       // merge only
+  float* Bs = s_dyn + (n + 1) * DK;
+
+  // 3. ReplayPrep: per-entry coefficients once per (slot, head).  Warp w takes
+  // entries i = w, w+NW, ...; i == n is the current token (kappa).
+  const TI* logAh = static_cast<const TI*>(a.logA) + sh * a.Mcap * DK;
+  for (int i = warp; i <= n; i += TL::NW) {
+    float dk = 0.f, dq = 0.f;
+    if (i < n) {
+      float lam_i_s = 0.f;
+      if (!PERKEY) lam_i_s = a.logLam[sh * a.Mcap + i];
+#pragma unroll
+      for (int m = 0; m < TL::KPL; ++m) {
+        const int j = lane + 32 * m;
+        const float ai = to_f(logAh[i * DK + j]);
+        const float lam_i = PERKEY ? a.logLam[(sh * a.Mcap + i) * DK + j] : lam_i_s;
+        const float r_t = expf(lt[m] - lam_i);                 // ratio to Lam_t
+        if (DELTA) {
+          dk = fmaf(r_t * ai, kr[m], dk);
+          dq = fmaf(r_t * ai, qr[m], dq);
+        } else {
+          const float r_p = expf(lp[m] - lam_i);               // RWKV6 reads S_{t-1}
+          dq = fmaf(r_p * ai, qr[m], dq);
+        }
+        if (MERGE) As[i * DK + j] = r_t * ai;
+      }
+    } else {
+#pragma unroll
+      for (int m = 0; m < TL::KPL; ++m) {
+        const int j = lane + 32 * m;
+        if (DELTA) {
+          dq = fmaf(kr[m], qr[m], dq);                           // kappa = k . q
+        } else {
+          dq = fmaf(a.u[h * DK + j] * kr[m], qr[m], dq);         // kappa = (u (.) k) . r
+        }
+        if (MERGE) As[n * DK + j] = kr[m];                       // current entry, ratio 1
+      }
+    }
+    dk = warp_sum(dk);
+    dq = warp_sum(dq);
+    if (lane == 0) {
+      if (i < n) {
+        s_ck[i] = dk;
+        s_cq[i] = dq;
+      } else {
+        s_kappa = dq;
+      }
+    }
+  }
+  if (warp == 0) {
+#pragma unroll
+    for (int m = 0; m < TL::KPL; ++m) {
+      const int j = lane + 32 * m;
+      const float et = expf(lt[m]);
+      if (DELTA) {
+        s_kt[j] = et * kr[m];
+        s_qt[j] = et * qr[m];
+      } else {
+        s_qt[j] = expf(lp[m]) * qr[m];
+      }
+      if (MERGE) s_dec[j] = et;
+    }
+    if (!MERGE) {  // append: a_n = k_t and its log-decay snapshot
+      TI* dstA = static_cast<TI*>(a.logA) + (sh * a.Mcap + n) * DK;
+#pragma unroll
+      for (int m = 0; m < TL::KPL; ++m) {
+        const int j = lane + 32 * m;
+        dstA[j] = kg[j];
+        if (PERKEY) a.logLam[(sh * a.Mcap + n) * DK + j] = lt[m];
+      }
+      if (!PERKEY && lane == 0) a.logLam[sh * a.Mcap + n] = lt[0];
+    }
+  }
+  if (MERGE) {  // stage the log's value factors b_i for the rank-(n+1) update
+    for (int e = tid; e < n * DV; e += TL::NT) Bs[e] = to_f(logBh[e]);
+  }
+  __syncthreads();
+
+  // 4. One pass over the register tile: partial Sbar^T k~ and Sbar^T q~.
+  {
+    float4 p4 = make_float4(0.f, 0.f, 0.f, 0.f), s4 = p4;
+#pragma unroll
+    for (int j = 0; j < TL::RPT; ++j) {
+      const int row = rg * TL::RPT + j;
+      if (DELTA) fma4(p4, s_kt[row], st[j]);
+      fma4(s4, s_qt[row], st[j]);
+    }
+    if (DELTA) *reinterpret_cast<float4*>(&s_red[0][rg][4 * c4]) = p4;
+    *reinterpret_cast<float4*>(&s_red[1][rg][4 * c4]) = s4;
+  }
+  __syncthreads();
+
+  // 5. AppendDecode finalize for value column c: replay, delta correction, output.
+  if (c < DV) {
+    float p = 0.f, s = 0.f;
+#pragma unroll
+    for (int g = 0; g < TL::RG; ++g) {
+      if (DELTA) p += s_red[0][g][c];
+      s += s_red[1][g][c];
+    }
+    float oc = s, bt;
+    for (int i = 0; i < n; ++i) {
+      float bi;
+      if (MERGE) {
+        bi = Bs[i * DV + c];
+      } else {
+        bi = i < kPrefetch ? bpre[i] : to_f(logBh[i * DV + c]);
+      }
+      if (DELTA) p = fmaf(s_ck[i], bi, p);
+      oc = fmaf(s_cq[i], bi, oc);
+    }
+    if (DELTA) {
+      bt = betac * (vc - p);
+    } else {
+      bt = vc;
+    }
+    oc = fmaf(s_kappa, bt, oc);
+    static_cast<TI*>(a.o)[sh * DV + c] = from_f<TI>(oc);
+    if (MERGE) {
+      Bs[n * DV + c] = bt;
+    } else {
+      TB* dstB = static_cast<TB*>(a.logB) + (sh * a.Mcap + n) * DV;
+      if constexpr (DELTA) {
+        dstB[c] = bt;
+      } else {
+        dstB[c] = static_cast<const TI*>(a.v)[sh * DV + c];   // raw v, bit copy
+      }
+    }
+  }
+
+  // 6. Merge: S_t = diag(e^{Lam_t}) Sbar + sum_{i<=n} (ratio_i (.) a_i) b_i^T.
+  if (MERGE) {
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < TL::RPT; ++j) {
+      const float d = s_dec[rg * TL::RPT + j];
+      st[j].x *= d;
+      st[j].y *= d;
+      st[j].z *= d;
+      st[j].w *= d;
+    }
+    for (int i = 0; i <= n; ++i) {
+      const float4 b4 = *reinterpret_cast<const float4*>(&Bs[i * DV + 4 * c4]);
+      const float* ai = &As[i * DK + rg * TL::RPT];
+#pragma unroll
+      for (int j4 = 0; j4 < TL::RPT; j4 += 4) {
+        const float4 a4 = *reinterpret_cast<const float4*>(ai + j4);
+        fma4(st[j4 + 0], a4.x, b4);
+        fma4(st[j4 + 1], a4.y, b4);
+        fma4(st[j4 + 2], a4.z, b4);
+        fma4(st[j4 + 3], a4.w, b4);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < TL::RPT; ++j) st_state(Sp + (rg * TL::RPT + j) * DV + 4 * c4, st[j]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Eager dense baseline: S_{t-1} -> S_t read and written every token.
+// ---------------------------------------------------------------------------
+template <int OP, int DK, int DV, typename TI>
+__global__ void __launch_bounds__(Tile<DK, DV>::NT, Tile<DK, DV>::MINB)
+eager_step_kernel(const StepArgs a) {
+  using TL = Tile<DK, DV>;
+  constexpr bool DELTA = OP != OP_RWKV6;
+
+  __shared__ __align__(16) float s_kx[DK];   // contraction vector for p
+  __shared__ __align__(16) float s_qx[DK];   // contraction vector for s
+  __shared__ __align__(16) float s_dec[DK];  // per-row decay of S_{t-1}
+  __shared__ __align__(16) float s_k[DK];    // k_t (rank-1 update rows)
+  __shared__ __align__(16) float s_b[DV];    // b_t (rank-1 update columns)
+  __shared__ __align__(16) float s_red[2][TL::RG][DV];
+  __shared__ float s_kappa;
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int c4 = tid % TL::TPR, rg = tid / TL::TPR;
+  const long sh = blockIdx.x;
+  const int h = static_cast<int>(sh % a.H);
+
+  float* Sp = a.Sbar + sh * (DK * DV);
+  float4 st[TL::RPT];
+#pragma unroll
+  for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + (rg * TL::RPT + j) * DV + 4 * c4);
+
+  const int c = tid;
+  float vc = 0.f, betac = 0.f;
+  if (c < DV) {
+    vc = to_f(static_cast<const TI*>(a.v)[sh * DV + c]);
+    if (DELTA) betac = a.beta[sh];
+  }
+
+  if (warp == 0) {
+    const TI* qg = static_cast<const TI*>(a.q) + sh * DK;
+    const TI* kg = static_cast<const TI*>(a.k) + sh * DK;
+    float kap = 0.f;
+#pragma unroll
+    for (int m = 0; m < TL::KPL; ++m) {
+      const int j = lane + 32 * m;
+      const float kj = to_f(kg[j]), qj = to_f(qg[j]);
+      const float dec = expf(OP == OP_GDN ? a.log_decay[sh] : a.log_decay[sh * DK + j]);
+      s_dec[j] = dec;
+      s_k[j] = kj;
+      if (OP == OP_GDN) {          // p = S^T k, s = S^T q (alpha applied after)
+        s_kx[j] = kj;
+        s_qx[j] = qj;
+        kap = fmaf(kj, qj, kap);
+      } else if (OP == OP_KDA) {   // p = S^T (alpha (.) k), s = S^T (alpha (.) q)
+        s_kx[j] = dec * kj;
+        s_qx[j] = dec * qj;
+        kap = fmaf(kj, qj, kap);
+      } else {                     // RWKV6: s = S^T r, kappa = (u (.) k) . r
+        s_qx[j] = qj;
+        kap = fmaf(a.u[h * DK + j] * kj, qj, kap);
+      }
+    }
+    kap = warp_sum(kap);
+    if (lane == 0) s_kappa = kap;
+  }
+  __syncthreads();
+
+  {
+    float4 p4 = make_float4(0.f, 0.f, 0.f, 0.f), s4 = p4;
+#pragma unroll
+    for (int j = 0; j < TL::RPT; ++j) {
+      const int row = rg * TL::RPT + j;
+      if (DELTA) fma4(p4, s_kx[row], st[j]);
+      fma4(s4, s_qx[row], st[j]);
+    }
+    if (DELTA) *reinterpret_cast<float4*>(&s_red[0][rg][4 * c4]) = p4;
+    *reinterpret_cast<float4*>(&s_red[1][rg][4 * c4]) = s4;
+  }
+  __syncthreads();
+
+  if (c < DV) {
+    float p = 0.f, s = 0.f;
+#pragma unroll
+    for (int g = 0; g < TL::RG; ++g) {
+      if (DELTA) p += s_red[0][g][c];
+      s += s_red[1][g][c];
+    }
+    float oc, bt;
+    if (OP == OP_GDN) {
+      const float alpha = s_dec[0];
+      bt = betac * (vc - alpha * p);
+      oc = fmaf(s_kappa, bt, alpha * s);
+    } else if (OP == OP_KDA) {
+      bt = betac * (vc - p);
+      oc = fmaf(s_kappa, bt, s);
+    } else {
+      bt = vc;
+      oc = fmaf(s_kappa, vc, s);
+    }
+    s_b[c] = bt;
+    static_cast<TI*>(a.o)[sh * DV + c] = from_f<TI>(oc);
+  }
+  __syncthreads();
+
+  const float4 b4 = *reinterpret_cast<const float4*>(&s_b[4 * c4]);
+#pragma unroll
+  for (int j = 0; j < TL::RPT; ++j) {
+    const int row = rg * TL::RPT + j;
+    const float d = s_dec[row];
+    float4 x = st[j];
+    x.x *= d;
+    x.y *= d;
+    x.z *= d;
+    x.w *= d;
+    fma4(x, s_k[row], b4);
+    st_state(Sp + row * DV + 4 * c4, x);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Materialise base + log into Sout (dl_merge with Sout == Sin, dl_read_state
+// otherwise).  Lam_last = Lam_{n-1}, the newest snapshot.
+// ---------------------------------------------------------------------------
+template <int OP, int DK, int DV, typename TI>
+__global__ void __launch_bounds__(Tile<DK, DV>::NT, Tile<DK, DV>::MINB)
+materialize_kernel(const MaterializeArgs a) {
+  using TL = Tile<DK, DV>;
+  using TB = typename std::conditional<OP == OP_RWKV6, TI, float>::type;
+  constexpr bool PERKEY = OP != OP_GDN;
+  __shared__ __align__(16) float s_dec[DK];
+  extern __shared__ __align__(16) float s_dyn[];  // As[n][DK], Bs[n][DV]
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int c4 = tid % TL::TPR, rg = tid / TL::TPR;
+  const long sh = blockIdx.x;
+  const int n = a.n;
+
+  const float* Sp = a.Sin + sh * (DK * DV);
+  float4 st[TL::RPT];
+#pragma unroll
+  for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + (rg * TL::RPT + j) * DV + 4 * c4);
+
+  float* As = s_dyn;
+  float* Bs = s_dyn + n * DK;
+  const TI* logAh = static_cast<const TI*>(a.logA) + sh * a.Mcap * DK;
+  const TB* logBh = static_cast<const TB*>(a.logB) + sh * a.Mcap * DV;
+
+  float ll[TL::KPL];
+#pragma unroll
+  for (int m = 0; m < TL::KPL; ++m) {
+    const int j = lane + 32 * m;
+    ll[m] = PERKEY ? a.logLam[(sh * a.Mcap + (n - 1)) * DK + j] : a.logLam[sh * a.Mcap + (n - 1)];
+  }
+  for (int i = warp; i < n; i += TL::NW) {
+#pragma unroll
+    for (int m = 0; m < TL::KPL; ++m) {
+      const int j = lane + 32 * m;
+      const float lam_i = PERKEY ? a.logLam[(sh * a.Mcap + i) * DK + j] : a.logLam[sh * a.Mcap + i];
+      As[i * DK + j] = expf(ll[m] - lam_i) * to_f(logAh[i * DK + j]);
+    }
+  }
+  if (warp == 0) {
+#pragma unroll
+    for (int m = 0; m < TL::KPL; ++m) s_dec[lane + 32 * m] = expf(ll[m]);
+  }
+  for (int e = tid; e < n * DV; e += TL::NT) Bs[e] = to_f(logBh[e]);
+  __syncthreads();
+
+#pragma unroll
+  for (int j = 0; j < TL::RPT; ++j) {
+    const float d = s_dec[rg * TL::RPT + j];
+    st[j].x *= d;
+    st[j].y *= d;
+    st[j].z *= d;
+    st[j].w *= d;
+  }
+  for (int i = 0; i < n; ++i) {
+    const float4 b4 = *reinterpret_cast<const float4*>(&Bs[i * DV + 4 * c4]);
+    const float* ai = &As[i * DK + rg * TL::RPT];
+#pragma unroll
+    for (int j4 = 0; j4 < TL::RPT; j4 += 4) {
+      const float4 a4 = *reinterpret_cast<const float4*>(ai + j4);
+      fma4(st[j4 + 0], a4.x, b4);
+      fma4(st[j4 + 1], a4.y, b4);
+      fma4(st[j4 + 2], a4.z, b4);
+      fma4(st[j4 + 3], a4.w, b4);
+    }
+  }
+  float* Sq = a.Sout + sh * (DK * DV);
+#pragma unroll
+  for (int j = 0; j < TL::RPT; ++j) st_state(Sq + (rg * TL::RPT + j) * DV + 4 * c4, st[j]);
+}
+
+}  // namespace dl

@@ -1,0 +1,153 @@
+"""PyTorch-facing handle over libdeltalog (marshalling only).
+
+PyTorch supplies device memory and streams; every step of the decode path
+runs inside the CUDA library.  Shapes and dtypes are checked here only to
+turn a caller mistake into a Python exception before the pointer crosses the
+C ABI.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _native as N
+
+OPS = {"gdn": N.DL_GDN, "kda": N.DL_KDA, "rwkv6": N.DL_RWKV6}
+DTYPES = {torch.float32: N.DL_F32, torch.bfloat16: N.DL_BF16}
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+class DeltaLog:
+    """One library handle: B slots x H heads of d_k x d_v fp32 state, merge interval M.
+
+    ``op`` is ``"gdn"``, ``"kda"`` or ``"rwkv6"``; ``dtype`` is the dtype of
+    q/k/v/o (``torch.bfloat16`` or ``torch.float32``).  The handle lives on the
+    CUDA device that is current (or given) at construction.
+    """
+
+    def __init__(self, B, H, d_k, d_v, M, op="gdn", dtype=torch.bfloat16, device=None):
+        if op not in OPS:
+            raise ValueError(f"op must be one of {sorted(OPS)}")
+        if dtype not in DTYPES:
+            raise ValueError("dtype must be torch.bfloat16 or torch.float32")
+        self.B, self.H, self.d_k, self.d_v, self.M = B, H, d_k, d_v, M
+        self.op, self.dtype = op, dtype
+        self.device = torch.device("cuda", torch.cuda.current_device() if device is None
+                                   else torch.device(device).index or 0)
+        self._h = ctypes.c_void_p()
+        with torch.cuda.device(self.device):
+            N.call("dl_create", ctypes.byref(self._h), B, H, d_k, d_v, M, OPS[op], DTYPES[dtype])
+
+    # -- helpers -------------------------------------------------------------
+    def _stream(self, stream):
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        return ctypes.c_void_p(s.cuda_stream)
+
+    def _check(self, name, t, shape, dtype, cuda=True):
+        if t is None:
+            raise ValueError(f"{name} is required")
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+        if t.dtype != dtype:
+            raise ValueError(f"{name}: expected {dtype}, got {t.dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if cuda and t.device != self.device:
+            raise ValueError(f"{name} must live on {self.device}")
+        if not cuda and t.device.type != "cpu":
+            raise ValueError(f"{name} must be a host tensor")
+
+    def _decay_shape(self):
+        return (self.B, self.H) if self.op == "gdn" else (self.B, self.H, self.d_k)
+
+    def _check_step(self, q, k, v, log_decay, beta, out, cuda):
+        B, H = self.B, self.H
+        self._check("q", q, (B, H, self.d_k), self.dtype, cuda)
+        self._check("k", k, (B, H, self.d_k), self.dtype, cuda)
+        self._check("v", v, (B, H, self.d_v), self.dtype, cuda)
+        self._check("log_decay", log_decay, self._decay_shape(), torch.float32, cuda)
+        if self.op == "rwkv6":
+            if beta is not None:
+                raise ValueError("beta must be None for rwkv6")
+        else:
+            self._check("beta", beta, (B, H), torch.float32, cuda)
+        self._check("out", out, (B, H, self.d_v), self.dtype, cuda)
+
+    def _alloc_out(self, cuda):
+        if cuda:
+            return torch.empty((self.B, self.H, self.d_v), dtype=self.dtype, device=self.device)
+        return torch.empty((self.B, self.H, self.d_v), dtype=self.dtype, pin_memory=True)
+
+    # -- API -----------------------------------------------------------------
+    def load_state(self, S, stream=None):
+        self._check("S", S, (self.B, self.H, self.d_k, self.d_v), torch.float32)
+        N.call("dl_load_state", self._h, _ptr(S), self._stream(stream))
+
+    def set_bonus(self, u, stream=None):
+        self._check("u", u, (self.H, self.d_k), torch.float32)
+        N.call("dl_set_bonus", self._h, _ptr(u), self._stream(stream))
+
+    def step(self, q, k, v, log_decay, beta=None, out=None, stream=None):
+        """One DeltaLog decode token (append, or merge on the M-th step); returns o."""
+        out = self._alloc_out(True) if out is None else out
+        self._check_step(q, k, v, log_decay, beta, out, True)
+        N.call("dl_step", self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(beta),
+               _ptr(out), self._stream(stream))
+        return out
+
+    def step_host(self, q, k, v, log_decay, beta=None, out=None, stream=None):
+        """dl_step on host tensors (pinned for async copies); o is ready after a stream sync."""
+        out = self._alloc_out(False) if out is None else out
+        self._check_step(q, k, v, log_decay, beta, out, False)
+        N.call("dl_step_host", self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(beta),
+               _ptr(out), self._stream(stream))
+        return out
+
+    def eager_step(self, q, k, v, log_decay, beta=None, out=None, stream=None):
+        """Dense baseline: S_{t-1} read and S_t written every token (needs an empty log)."""
+        out = self._alloc_out(True) if out is None else out
+        self._check_step(q, k, v, log_decay, beta, out, True)
+        N.call("dl_eager_step", self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(beta),
+               _ptr(out), self._stream(stream))
+        return out
+
+    def merge(self, stream=None):
+        N.call("dl_merge", self._h, self._stream(stream))
+
+    def read_state(self, out=None, stream=None):
+        if out is None:
+            out = torch.empty((self.B, self.H, self.d_k, self.d_v), dtype=torch.float32,
+                              device=self.device)
+        self._check("out", out, (self.B, self.H, self.d_k, self.d_v), torch.float32)
+        N.call("dl_read_state", self._h, _ptr(out), self._stream(stream))
+        return out
+
+    @property
+    def log_len(self):
+        n = ctypes.c_int()
+        N.call("dl_log_len", self._h, ctypes.byref(n))
+        return n.value
+
+    def check_device(self, stream=None):
+        N.call("dl_check_device", self._h, self._stream(stream))
+
+    def close(self):
+        if self._h:
+            N.call("dl_destroy", self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()

@@ -1,0 +1,91 @@
+"""C-ABI checks that need no GPU: the library loads, exports every declared
+symbol, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from recurrent_state_update_deltalog_b200 import _native as N
+from recurrent_state_update_deltalog_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", f)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(dl_\w+)\s*\(", text, flags=re.M))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return N.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _declared()
+    assert {"dl_create", "dl_step", "dl_merge", "dl_eager_step", "dl_destroy"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert declared == set(N.SIGNATURES), declared ^ set(N.SIGNATURES)
+
+
+def test_build_targets_sm100a_only():
+    from recurrent_state_update_deltalog_b200 import build as B
+    assert B.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+    assert all("sm_" not in f or "sm_100a" in f for f in B.NVCC_FLAGS)
+
+
+def test_strerror(lib):
+    for code, name in N.STATUS.items():
+        assert lib.dl_strerror(code)
+    assert lib.dl_strerror(-99) == b"unknown status"
+
+
+@pytest.mark.parametrize("args,status", [
+    ((1, 1, 64, 64, 0, 0, 0), -2),      # M = 0
+    ((1, 1, 64, 64, 65, 0, 0), -2),     # M > DL_MAX_M
+    ((1, 1, 96, 64, 8, 0, 0), -2),      # unsupported d_k
+    ((1, 1, 64, 32, 8, 0, 0), -2),      # unsupported d_v
+    ((0, 1, 64, 64, 8, 0, 0), -1),      # B = 0
+    ((1, -2, 64, 64, 8, 0, 0), -1),     # H < 0
+    ((1, 1, 64, 64, 8, 3, 0), -1),      # unknown op
+    ((1, 1, 64, 64, 8, 0, 7), -1),      # unknown dtype
+])
+def test_create_rejects_bad_arguments(lib, args, status):
+    h = ctypes.c_void_p()
+    assert lib.dl_create(ctypes.byref(h), *args) == status
+    assert not h.value
+    assert lib.dl_last_error()
+
+
+def test_null_handle_paths(lib):
+    assert lib.dl_create(None, 1, 1, 64, 64, 8, 0, 0) == -1
+    p = ctypes.c_void_p(16)
+    for fn in ("dl_step", "dl_eager_step", "dl_step_host"):
+        assert getattr(lib, fn)(None, p, p, p, p, p, p, None) == -1
+    assert lib.dl_merge(None, None) == -1
+    assert lib.dl_read_state(None, p, None) == -1
+    assert lib.dl_load_state(None, p, None) == -1
+    assert lib.dl_set_bonus(None, p, None) == -1
+    assert lib.dl_check_device(None, None) == -1
+    n = ctypes.c_int()
+    assert lib.dl_log_len(None, ctypes.byref(n)) == -1
+    assert lib.dl_destroy(None) == 0
+
+
+def test_python_binding_fails_loudly_without_library(tmp_path):
+    import importlib
+    mod = importlib.reload(N)
+    try:
+        mod._lib = None
+        with pytest.raises(ImportError):
+            mod.load(str(tmp_path / "missing.so"))
+    finally:
+        importlib.reload(N)

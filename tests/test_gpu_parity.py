@@ -1,0 +1,187 @@
+"""GPU parity: libdeltalog (through the C ABI) against the fp64 oracle.
+
+Tolerances: max relative error 5e-3 for bf16 inputs/outputs and 1e-4 for fp32,
+per tensor (all outputs stacked; each merged base; the final logical state).
+"""
+import numpy as np
+import pytest
+import torch
+
+from _parity import TOL, make_inputs, relerr, run_gpu, run_oracle, step_args, to_device
+
+pytestmark = pytest.mark.gpu
+
+OPS = ["gdn", "kda", "rwkv6"]
+
+
+def _check_run(op, B, H, dk, dv, M, T, dtype, eager=False, seed=0):
+    S0, seq, u = make_inputs(op, B, H, dk, dv, T, dtype, seed)
+    merge_steps = [t for t in range(T) if (t + 1) % M == 0] if not eager else []
+    o_ref, S_ref, kept = run_oracle(op, S0, seq, u, record=set(merge_steps))
+    o, merges, final = run_gpu(op, S0, seq, u, M, dtype, eager=eager)
+    tol = TOL[dtype]
+    e_o = relerr(o, o_ref)
+    assert e_o < tol, f"outputs: {e_o:.3e}"
+    for t in merge_steps:
+        e = relerr(merges[t], kept[t])
+        assert e < tol, f"merged base at t={t}: {e:.3e}"
+    e_s = relerr(final, S_ref)
+    assert e_s < tol, f"final state: {e_s:.3e}"
+    return e_o, e_s
+
+
+@pytest.mark.parametrize("M", [8, 1])
+def test_gdn_single_head_fp32(M):
+    """B=H=1, d=64, fp32 inputs, 64 steps, seed 0."""
+    _check_run("gdn", 1, 1, 64, 64, M, 64, torch.float32)
+
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("dims", [(64, 64), (128, 128), (64, 128), (128, 64)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_deferred_shapes(op, dims, dtype):
+    """Ragged B*H, every shape, M=4 with a tail that ends mid-cycle."""
+    _check_run(op, 3, 5, dims[0], dims[1], 4, 11, dtype)
+
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 16, 32, 33, 64])
+def test_deferred_every_M(op, M):
+    _check_run(op, 2, 3, 128, 128, M, min(2 * M + 3, 70), torch.bfloat16)
+
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_eager_kernel(op, dtype):
+    _check_run(op, 3, 4, 128, 128, 1, 9, dtype, eager=True)
+    _check_run(op, 2, 3, 64, 64, 1, 9, dtype, eager=True)
+
+
+@pytest.mark.parametrize("op", OPS)
+def test_M1_deferred_matches_eager_kernel(op):
+    S0, seq, u = make_inputs(op, 4, 4, 128, 128, 10, torch.float32)
+    o_d, _, s_d = run_gpu(op, S0, seq, u, 1, torch.float32, record_merges=False)
+    o_e, _, s_e = run_gpu(op, S0, seq, u, 1, torch.float32, eager=True)
+    assert relerr(o_d, o_e) < 1e-5 and relerr(s_d, s_e) < 1e-5
+
+
+def _full_size_case(op, B, H, d, M, T, n_units=24):
+    """Full-size launch; sampled (slot, head) units checked against the oracle."""
+    dtype = torch.bfloat16
+    S0, seq, u = make_inputs(op, B, H, d, d, T, dtype)
+    rng = np.random.default_rng(1234)
+    flat = rng.choice(B * H, size=n_units, replace=False)
+    flat = np.unique(np.concatenate([flat, [0, B * H - 1]]))
+    bs, hs = flat // H, flat % H
+    S0_s = S0[bs, hs]
+    seq_s = {k: v[:, bs, hs] for k, v in seq.items()}
+    u_s = u[hs] if u is not None else None
+    merge_steps = [t for t in range(T) if (t + 1) % M == 0]
+    o_ref, S_ref, kept = run_oracle(op, S0_s, seq_s, u_s, record=set(merge_steps))
+    o, merges, final = run_gpu(op, S0, seq, u, M, dtype)
+    assert relerr(o[:, bs, hs], o_ref) < TOL[dtype]
+    for t in merge_steps:
+        assert relerr(merges[t][bs, hs], kept[t]) < TOL[dtype]
+    assert relerr(final[bs, hs], S_ref) < TOL[dtype]
+    # properties over every unit: finite outputs, untouched dtype range
+    assert np.isfinite(o).all() and np.isfinite(final).all()
+
+
+@pytest.mark.parametrize("M", [8, 4, 16, 1])
+def test_full_size_gdn_b256_h32_d128(M):
+    _full_size_case("gdn", 256, 32, 128, M, 2 * M + 3 if M > 1 else 6)
+
+
+def test_full_size_kda_b128_h32_d128():
+    _full_size_case("kda", 128, 32, 128, 8, 19)
+
+
+def test_full_size_rwkv6_b128_h64_d64():
+    _full_size_case("rwkv6", 128, 64, 64, 8, 19)
+
+
+# ---- handle semantics through the C ABI ---------------------------------------
+
+@pytest.mark.parametrize("op", OPS)
+def test_explicit_merge_and_read_state(op):
+    """dl_merge mid-cycle, dl_read_state leaves the handle untouched."""
+    from recurrent_state_update_deltalog_b200 import DeltaLog
+    B, H, d, M, T = 2, 3, 64, 8, 13
+    S0, seq, u = make_inputs(op, B, H, d, d, T, torch.float32)
+    o_ref, S_ref, kept = run_oracle(op, S0, seq, u, record=set(range(T)))
+    dseq = to_device(seq, torch.float32)
+    h = DeltaLog(B, H, d, d, M, op=op, dtype=torch.float32)
+    h.load_state(torch.from_numpy(S0).cuda())
+    if u is not None:
+        h.set_bonus(torch.from_numpy(u).cuda())
+    outs = []
+    for t in range(T):
+        outs.append(h.step(*step_args(op, dseq, t)).cpu().numpy())
+        s1 = h.read_state().cpu().numpy()
+        s2 = h.read_state().cpu().numpy()
+        assert np.array_equal(s1, s2)
+        assert relerr(s1, kept[t]) < 1e-4, t
+        if t == 4:
+            assert h.log_len == 5
+            h.merge()
+            assert h.log_len == 0
+            assert relerr(h.read_state().cpu().numpy(), kept[t]) < 1e-4
+    assert relerr(np.stack(outs), o_ref) < 1e-4
+    h.merge()
+    h.merge()                      # no-op on an empty log
+    assert relerr(h.read_state().cpu().numpy(), S_ref) < 1e-4
+    h.close()
+
+
+def test_eager_needs_empty_log_and_load_state_resets():
+    from recurrent_state_update_deltalog_b200 import DeltaLog, DeltaLogError
+    S0, seq, _ = make_inputs("gdn", 1, 2, 64, 64, 3, torch.float32)
+    dseq = to_device(seq, torch.float32)
+    h = DeltaLog(1, 2, 64, 64, 4, op="gdn", dtype=torch.float32)
+    h.load_state(torch.from_numpy(S0).cuda())
+    h.step(*step_args("gdn", dseq, 0))
+    with pytest.raises(DeltaLogError) as ei:
+        h.eager_step(*step_args("gdn", dseq, 1))
+    assert ei.value.status == -6
+    h.load_state(torch.from_numpy(S0).cuda())
+    assert h.log_len == 0
+    h.eager_step(*step_args("gdn", dseq, 0))
+    with pytest.raises(DeltaLogError):
+        DeltaLog(1, 2, 64, 64, 4, op="gdn").set_bonus(torch.zeros(2, 64, device="cuda"))
+    h.close()
+
+
+@pytest.mark.parametrize("op", OPS)
+def test_step_host_matches_device_step(op):
+    from recurrent_state_update_deltalog_b200 import DeltaLog
+    B, H, d, M, T = 4, 8, 128, 4, 6
+    S0, seq, u = make_inputs(op, B, H, d, d, T, torch.bfloat16)
+    dseq = to_device(seq, torch.bfloat16)
+    hseq = {k: v.cpu().pin_memory() for k, v in dseq.items()}
+    hd = DeltaLog(B, H, d, d, M, op=op)
+    hh = DeltaLog(B, H, d, d, M, op=op)
+    for h in (hd, hh):
+        h.load_state(torch.from_numpy(S0).cuda())
+        if u is not None:
+            h.set_bonus(torch.from_numpy(u).cuda())
+    for t in range(T):
+        od = hd.step(*step_args(op, dseq, t))
+        oh = hh.step_host(*step_args(op, hseq, t))
+        torch.cuda.synchronize()
+        assert torch.equal(od.cpu(), oh)
+    assert torch.equal(hd.read_state(), hh.read_state())
+    hd.close()
+    hh.close()
+
+
+def test_zero_log_decay_and_beta_zero_keep_state():
+    """beta = 0 and alpha = 1: the state never changes and o = S0^T q (GDN/KDA)."""
+    from recurrent_state_update_deltalog_b200 import DeltaLog
+    for op in ("gdn", "kda"):
+        S0, seq, _ = make_inputs(op, 2, 2, 64, 64, 9, torch.float32)
+        seq["beta"][:] = 0
+        seq["log_decay"][:] = 0
+        o, merges, final = run_gpu(op, S0, seq, None, 4, torch.float32)
+        assert np.array_equal(final, S0)
+        want = np.einsum("bhkv,tbhk->tbhv", S0.astype(np.float64), seq["q"].astype(np.float64))
+        assert relerr(o, want) < 1e-5
