@@ -115,6 +115,7 @@ dl::StepArgs step_args(dl_handle* h, const void* q, const void* k, const void* v
   a.logB = h->logB;
   a.logLam = h->logLam;
   a.u = h->u;
+  a.err = h->err;
   a.H = h->H;
   a.Mcap = h->Mcap;
   a.n = h->n;
@@ -146,6 +147,7 @@ cudaError_t launch_materialize(const dl_handle* h, float* out, cudaStream_t s) {
   a.logA = h->logA;
   a.logB = h->logB;
   a.logLam = h->logLam;
+  a.err = h->err;
   a.Mcap = h->Mcap;
   a.n = h->n;
   const dl::LaunchShape sh = shape_of(h);

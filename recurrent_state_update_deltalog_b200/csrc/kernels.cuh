@@ -16,7 +16,10 @@
 // are the float4 column groups of the CTA's threads: thread (rg, c4) holds
 // rows [rg*RPT, rg*RPT+RPT) x columns [4*c4, 4*c4+4) of the fp32 state in
 // registers.  All state loads of a CTA are issued up front as 128-bit
-// streaming loads (64 KB in flight per CTA at d = 128), the two contractions
+// streaming loads (64 KB in flight per CTA at d = 128) while one thread stages
+// the head's whole log (a_i, Lam_i, b_i) into shared memory with TMA bulk
+// copies on an mbarrier, so the log costs one round trip, not one per entry.
+// The two contractions
 // Sbar^T k~ and Sbar^T q~ are formed in one pass over those registers, and the
 // d_k reduction crosses row groups through a small shared-memory stage.  On a
 // merge step the rank-(n+1) update is applied to the same registers and
@@ -29,6 +32,8 @@
 #include <stdint.h>
 
 #include <type_traits>
+
+#include "ptx.cuh"
 
 namespace dl {
 
@@ -47,6 +52,7 @@ struct StepArgs {
   void* logB;              // [BH][Mcap][DV], fp32 (GDN/KDA) or input dtype (RWKV6)
   float* logLam;           // [BH][Mcap] (GDN) or [BH][Mcap][DK]
   const float* u;          // [H][DK] (RWKV6)
+  int* err;               // device error word (kErr* bits)
   int H;
   int Mcap;                // log capacity per (slot, head), >= 1
   int n;                   // entries in the log before this step
@@ -59,6 +65,7 @@ struct MaterializeArgs {
   const void* logA;
   const void* logB;
   const float* logLam;
+  int* err;
   int Mcap;
   int n;
 };
@@ -108,11 +115,74 @@ struct Tile {
   static_assert(DK <= NT && DV <= NT, "one thread per key / value in setup phases");
 };
 
-// Prefetched log values per finalize thread (entries beyond this are loaded late).
-constexpr int kPrefetch = 8;
-
 // Largest supported merge interval M (log capacity M-1).
 constexpr int kMaxM = 64;
+
+// Shared-memory image of a (slot, head)'s log, staged by TMA bulk copies.
+// Byte layout (every region starts 16-byte aligned):
+//   A   n x DK input dtype     a_i = k_i
+//   L   n x DK fp32            Lam_i (KDA / RWKV6 only; GDN keeps n scalars apart)
+//   B   n x DV (fp32 | input)  b_i (RWKV6: raw v_i in the input dtype)
+// followed, for merge-type launches, by the fp32 work arrays
+//   As  (n+1) x DK             ratio-scaled a_i, current entry last (ratio 1)
+//   Bc  DV                     the current entry's b_t
+template <int OP, int DK, int DV, typename TI>
+struct LogLayout {
+  using TB = typename std::conditional<OP == OP_RWKV6, TI, float>::type;
+  static constexpr bool PERKEY = OP != OP_GDN;
+  __host__ __device__ static constexpr size_t a_bytes(int n) { return size_t(n) * DK * sizeof(TI); }
+  __host__ __device__ static constexpr size_t l_bytes(int n) { return PERKEY ? size_t(n) * DK * 4 : 0; }
+  __host__ __device__ static constexpr size_t b_bytes(int n) { return size_t(n) * DV * sizeof(TB); }
+  __host__ __device__ static constexpr size_t staged(int n) { return a_bytes(n) + l_bytes(n) + b_bytes(n); }
+  __host__ __device__ static constexpr size_t step_smem(int n, bool merge) {
+    return staged(n) + (merge ? size_t(n + 1) * DK * 4 + size_t(DV) * 4 : 0);
+  }
+  __host__ __device__ static constexpr size_t materialize_smem(int n) { return staged(n) + size_t(n) * DK * 4; }
+};
+
+// Four consecutive log values as floats (fp32 or bf16 storage).
+__device__ __forceinline__ float4 load4f(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 load4f(const __nv_bfloat16* p) {
+  const uint2 r = *reinterpret_cast<const uint2*>(p);
+  const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&r.x);
+  const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&r.y);
+  const float2 a = __bfloat1622float2(lo), b = __bfloat1622float2(hi);
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+
+// Thread 0 starts the bulk copies of entries [0, n) of this (slot, head)'s log
+// into shared memory; completion arrives on `bar` (phase 0).
+template <int OP, int DK, int DV, typename TI>
+__device__ __forceinline__ void stage_log(unsigned char* smem, uint64_t* bar, const void* logA,
+                                          const float* logLam, const void* logB, long sh, int Mcap,
+                                          int n) {
+  using LL = LogLayout<OP, DK, DV, TI>;
+  using TB = typename LL::TB;
+  mbar_init(bar, 1);
+  fence_mbar_init();
+  if (n == 0) return;
+  mbar_arrive_expect_tx(bar, static_cast<uint32_t>(LL::staged(n)));
+  bulk_g2s(smem, static_cast<const TI*>(logA) + sh * Mcap * DK, static_cast<uint32_t>(LL::a_bytes(n)), bar);
+  if (LL::PERKEY)
+    bulk_g2s(smem + LL::a_bytes(n), logLam + sh * Mcap * DK, static_cast<uint32_t>(LL::l_bytes(n)), bar);
+  bulk_g2s(smem + LL::a_bytes(n) + LL::l_bytes(n), static_cast<const TB*>(logB) + sh * Mcap * DV,
+           static_cast<uint32_t>(LL::b_bytes(n)), bar);
+}
+
+// Every thread waits for the staged log.  On a timeout the whole CTA agrees to
+// stop: the error word is raised, copies still in flight get one more bounded
+// wait (the CTA must not exit while they target its shared memory), and the
+// caller returns.
+__device__ __forceinline__ bool wait_log(uint64_t* bar, int n, int* err) {
+  int ok = n == 0 ? 1 : static_cast<int>(mbar_wait_bounded(bar, 0));
+  if (__syncthreads_and(ok)) return true;
+  if (threadIdx.x == 0) {
+    atomicOr(err, kErrWaitTimeout);
+    mbar_wait_bounded(bar, 0);
+  }
+  __syncthreads();
+  return false;
+}
 
 // ---------------------------------------------------------------------------
 // Deferred step.  MERGE=false: append (Sbar read only).  MERGE=true: the step
@@ -122,7 +192,8 @@ template <int OP, int DK, int DV, typename TI, bool MERGE>
 __global__ void __launch_bounds__(Tile<DK, DV>::NT, Tile<DK, DV>::MINB)
 deltalog_step_kernel(const StepArgs a) {
   using TL = Tile<DK, DV>;
-  using TB = typename std::conditional<OP == OP_RWKV6, TI, float>::type;
+  using LL = LogLayout<OP, DK, DV, TI>;
+  using TB = typename LL::TB;
   constexpr bool DELTA = OP != OP_RWKV6;
   constexpr bool PERKEY = OP != OP_GDN;
 
@@ -131,8 +202,10 @@ deltalog_step_kernel(const StepArgs a) {
   __shared__ __align__(16) float s_dec[DK];      // e^{Lam_t} per row (merge)
   __shared__ __align__(16) float s_red[2][TL::RG][DV];
   __shared__ float s_ck[kMaxM], s_cq[kMaxM];
+  __shared__ float s_lam[kMaxM];                 // GDN: scalar Lam_i of the log entries
   __shared__ float s_kappa;
-  extern __shared__ __align__(16) float s_dyn[];  // merge: As[(n+1)][DK], Bs[(n+1)][DV]
+  __shared__ __align__(8) uint64_t s_bar;
+  extern __shared__ __align__(16) unsigned char s_dyn[];
 
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
@@ -141,13 +214,22 @@ deltalog_step_kernel(const StepArgs a) {
   const int h = static_cast<int>(sh % a.H);
   const int n = a.n;
 
-  // 1. Stream this head's Sbar tile into registers (all loads in flight).
+  const TI* sA = reinterpret_cast<const TI*>(s_dyn);
+  const float* sL = reinterpret_cast<const float*>(s_dyn + LL::a_bytes(n));
+  const TB* sB = reinterpret_cast<const TB*>(s_dyn + LL::a_bytes(n) + LL::l_bytes(n));
+  float* As = reinterpret_cast<float*>(s_dyn + LL::staged(n));      // merge only
+  float* Bc = As + (n + 1) * DK;                                      // merge only
+
+  // 1. Stream this head's Sbar tile into registers (all loads in flight), and
+  // let one thread start the TMA bulk copies of the log into shared memory.
   float* Sp = a.Sbar + sh * (DK * DV);
   float4 st[TL::RPT];
 #pragma unroll
   for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + (rg * TL::RPT + j) * DV + 4 * c4);
+  if (tid == 0) stage_log<OP, DK, DV, TI>(s_dyn, &s_bar, a.logA, a.logLam, a.logB, sh, a.Mcap, n);
 
-  // 2. Key-side values for this lane's keys j = lane + 32 m.
+  // 2. Key-side values for this lane's keys j = lane + 32 m; GDN's scalar
+  // snapshots; per-column v and beta for the finalize threads.
   const TI* qg = static_cast<const TI*>(a.q) + sh * DK;
   const TI* kg = static_cast<const TI*>(a.k) + sh * DK;
   float kr[TL::KPL], qr[TL::KPL], lt[TL::KPL], lp[TL::KPL];
@@ -162,6 +244,7 @@ deltalog_step_kernel(const StepArgs a) {
       lt[m] = lp[m] + a.log_decay[sh * DK + j];
     }
   } else {
+    if (tid < n) s_lam[tid] = a.logLam[sh * a.Mcap + tid];
     const float lprev = n > 0 ? a.logLam[sh * a.Mcap + (n - 1)] : 0.f;
     const float lcur = lprev + a.log_decay[sh];
 #pragma unroll
@@ -173,37 +256,25 @@ deltalog_step_kernel(const StepArgs a) {
       lt[m] = lcur;
     }
   }
-
-  // Finalize threads (one per value column) prefetch v, beta and early log b's.
   const int c = tid;
   float vc = 0.f, betac = 0.f;
-  float bpre[kPrefetch];
-  const TB* logBh = static_cast<const TB*>(a.logB) + sh * a.Mcap * DV;
   if (c < DV) {
     vc = to_f(static_cast<const TI*>(a.v)[sh * DV + c]);
     if (DELTA) betac = a.beta[sh];
-    if (!MERGE) {
-#pragma unroll
-      for (int i = 0; i < kPrefetch; ++i) bpre[i] = i < n ? to_f(logBh[i * DV + c]) : 0.f;
-    }
   }
-
-  float* As = s_dyn;                       // merge only
-  float* Bs = s_dyn + (n + 1) * DK;
+  __syncthreads();                              // barrier init and s_lam visible
+  if (!wait_log(&s_bar, n, a.err)) return;
 
   // 3. ReplayPrep: per-entry coefficients once per (slot, head).  Warp w takes
   // entries i = w, w+NW, ...; i == n is the current token (kappa).
-  const TI* logAh = static_cast<const TI*>(a.logA) + sh * a.Mcap * DK;
   for (int i = warp; i <= n; i += TL::NW) {
     float dk = 0.f, dq = 0.f;
     if (i < n) {
-      float lam_i_s = 0.f;
-      if (!PERKEY) lam_i_s = a.logLam[sh * a.Mcap + i];
 #pragma unroll
       for (int m = 0; m < TL::KPL; ++m) {
         const int j = lane + 32 * m;
-        const float ai = to_f(logAh[i * DK + j]);
-        const float lam_i = PERKEY ? a.logLam[(sh * a.Mcap + i) * DK + j] : lam_i_s;
+        const float ai = to_f(sA[i * DK + j]);
+        const float lam_i = PERKEY ? sL[i * DK + j] : s_lam[i];
         const float r_t = expf(lt[m] - lam_i);                 // ratio to Lam_t
         if (DELTA) {
           dk = fmaf(r_t * ai, kr[m], dk);
@@ -226,7 +297,7 @@ deltalog_step_kernel(const StepArgs a) {
         if (MERGE) As[n * DK + j] = kr[m];                       // current entry, ratio 1
       }
     }
-    dk = warp_sum(dk);
+    if (DELTA) dk = warp_sum(dk);
     dq = warp_sum(dq);
     if (lane == 0) {
       if (i < n) {
@@ -261,9 +332,6 @@ deltalog_step_kernel(const StepArgs a) {
       if (!PERKEY && lane == 0) a.logLam[sh * a.Mcap + n] = lt[0];
     }
   }
-  if (MERGE) {  // stage the log's value factors b_i for the rank-(n+1) update
-    for (int e = tid; e < n * DV; e += TL::NT) Bs[e] = to_f(logBh[e]);
-  }
   __syncthreads();
 
   // 4. One pass over the register tile: partial Sbar^T k~ and Sbar^T q~.
@@ -290,12 +358,7 @@ deltalog_step_kernel(const StepArgs a) {
     }
     float oc = s, bt;
     for (int i = 0; i < n; ++i) {
-      float bi;
-      if (MERGE) {
-        bi = Bs[i * DV + c];
-      } else {
-        bi = i < kPrefetch ? bpre[i] : to_f(logBh[i * DV + c]);
-      }
+      const float bi = to_f(sB[i * DV + c]);
       if (DELTA) p = fmaf(s_ck[i], bi, p);
       oc = fmaf(s_cq[i], bi, oc);
     }
@@ -307,7 +370,7 @@ deltalog_step_kernel(const StepArgs a) {
     oc = fmaf(s_kappa, bt, oc);
     static_cast<TI*>(a.o)[sh * DV + c] = from_f<TI>(oc);
     if (MERGE) {
-      Bs[n * DV + c] = bt;
+      Bc[c] = bt;
     } else {
       TB* dstB = static_cast<TB*>(a.logB) + (sh * a.Mcap + n) * DV;
       if constexpr (DELTA) {
@@ -330,7 +393,7 @@ deltalog_step_kernel(const StepArgs a) {
       st[j].w *= d;
     }
     for (int i = 0; i <= n; ++i) {
-      const float4 b4 = *reinterpret_cast<const float4*>(&Bs[i * DV + 4 * c4]);
+      const float4 b4 = i < n ? load4f(sB + i * DV + 4 * c4) : load4f(Bc + 4 * c4);
       const float* ai = &As[i * DK + rg * TL::RPT];
 #pragma unroll
       for (int j4 = 0; j4 < TL::RPT; j4 += 4) {
@@ -464,16 +527,19 @@ eager_step_kernel(const StepArgs a) {
 
 // ---------------------------------------------------------------------------
 // Materialise base + log into Sout (dl_merge with Sout == Sin, dl_read_state
-// otherwise).  Lam_last = Lam_{n-1}, the newest snapshot.
+// otherwise).  Lam_last = Lam_{n-1}, the newest snapshot.  Requires n >= 1.
 // ---------------------------------------------------------------------------
 template <int OP, int DK, int DV, typename TI>
 __global__ void __launch_bounds__(Tile<DK, DV>::NT, Tile<DK, DV>::MINB)
 materialize_kernel(const MaterializeArgs a) {
   using TL = Tile<DK, DV>;
-  using TB = typename std::conditional<OP == OP_RWKV6, TI, float>::type;
+  using LL = LogLayout<OP, DK, DV, TI>;
+  using TB = typename LL::TB;
   constexpr bool PERKEY = OP != OP_GDN;
   __shared__ __align__(16) float s_dec[DK];
-  extern __shared__ __align__(16) float s_dyn[];  // As[n][DK], Bs[n][DV]
+  __shared__ float s_lam[kMaxM];
+  __shared__ __align__(8) uint64_t s_bar;
+  extern __shared__ __align__(16) unsigned char s_dyn[];
 
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
@@ -481,15 +547,16 @@ materialize_kernel(const MaterializeArgs a) {
   const long sh = blockIdx.x;
   const int n = a.n;
 
+  const TI* sA = reinterpret_cast<const TI*>(s_dyn);
+  const float* sL = reinterpret_cast<const float*>(s_dyn + LL::a_bytes(n));
+  const TB* sB = reinterpret_cast<const TB*>(s_dyn + LL::a_bytes(n) + LL::l_bytes(n));
+  float* As = reinterpret_cast<float*>(s_dyn + LL::staged(n));
+
   const float* Sp = a.Sin + sh * (DK * DV);
   float4 st[TL::RPT];
 #pragma unroll
   for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + (rg * TL::RPT + j) * DV + 4 * c4);
-
-  float* As = s_dyn;
-  float* Bs = s_dyn + n * DK;
-  const TI* logAh = static_cast<const TI*>(a.logA) + sh * a.Mcap * DK;
-  const TB* logBh = static_cast<const TB*>(a.logB) + sh * a.Mcap * DV;
+  if (tid == 0) stage_log<OP, DK, DV, TI>(s_dyn, &s_bar, a.logA, a.logLam, a.logB, sh, a.Mcap, n);
 
   float ll[TL::KPL];
 #pragma unroll
@@ -497,19 +564,22 @@ materialize_kernel(const MaterializeArgs a) {
     const int j = lane + 32 * m;
     ll[m] = PERKEY ? a.logLam[(sh * a.Mcap + (n - 1)) * DK + j] : a.logLam[sh * a.Mcap + (n - 1)];
   }
+  if (!PERKEY && tid < n) s_lam[tid] = a.logLam[sh * a.Mcap + tid];
+  __syncthreads();
+  if (!wait_log(&s_bar, n, a.err)) return;
+
   for (int i = warp; i < n; i += TL::NW) {
 #pragma unroll
     for (int m = 0; m < TL::KPL; ++m) {
       const int j = lane + 32 * m;
-      const float lam_i = PERKEY ? a.logLam[(sh * a.Mcap + i) * DK + j] : a.logLam[sh * a.Mcap + i];
-      As[i * DK + j] = expf(ll[m] - lam_i) * to_f(logAh[i * DK + j]);
+      const float lam_i = PERKEY ? sL[i * DK + j] : s_lam[i];
+      As[i * DK + j] = expf(ll[m] - lam_i) * to_f(sA[i * DK + j]);
     }
   }
   if (warp == 0) {
 #pragma unroll
     for (int m = 0; m < TL::KPL; ++m) s_dec[lane + 32 * m] = expf(ll[m]);
   }
-  for (int e = tid; e < n * DV; e += TL::NT) Bs[e] = to_f(logBh[e]);
   __syncthreads();
 
 #pragma unroll
@@ -521,7 +591,7 @@ materialize_kernel(const MaterializeArgs a) {
     st[j].w *= d;
   }
   for (int i = 0; i < n; ++i) {
-    const float4 b4 = *reinterpret_cast<const float4*>(&Bs[i * DV + 4 * c4]);
+    const float4 b4 = load4f(sB + i * DV + 4 * c4);
     const float* ai = &As[i * DK + rg * TL::RPT];
 #pragma unroll
     for (int j4 = 0; j4 < TL::RPT; j4 += 4) {

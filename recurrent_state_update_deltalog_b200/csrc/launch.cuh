@@ -14,20 +14,34 @@ struct LaunchShape {
   int dtype;  // 0 = fp32, 1 = bf16 inputs
 };
 
+// Opt a kernel into more than the default 48 KB of shared memory (static +
+// dynamic) when a launch needs it; `worst` is the largest dynamic size any
+// launch of this kernel can ask for.
+template <typename K>
+cudaError_t allow_smem(K kern, size_t smem, size_t worst) {
+  if (smem <= 16 * 1024) return cudaSuccess;  // every kernel's static part is < 32 KB
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.sharedSizeBytes + smem <= 48 * 1024) return cudaSuccess;
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(worst));
+}
+
 template <int OP, int DK, int DV, typename TI>
 cudaError_t step_dims(const LaunchShape& s, bool merge, const StepArgs& a, cudaStream_t st) {
   using TL = Tile<DK, DV>;
+  using LL = LogLayout<OP, DK, DV, TI>;
+  const size_t smem = LL::step_smem(a.n, merge);
   if (merge) {
     auto kern = deltalog_step_kernel<OP, DK, DV, TI, true>;
-    const size_t smem = static_cast<size_t>(a.n + 1) * (DK + DV) * sizeof(float);
-    if (smem > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(kMaxM * (DK + DV) * sizeof(float)));
-      if (e != cudaSuccess) return e;
-    }
+    cudaError_t e = allow_smem(kern, smem, LL::step_smem(kMaxM - 1, true));
+    if (e != cudaSuccess) return e;
     kern<<<s.BH, TL::NT, smem, st>>>(a);
   } else {
-    deltalog_step_kernel<OP, DK, DV, TI, false><<<s.BH, TL::NT, 0, st>>>(a);
+    auto kern = deltalog_step_kernel<OP, DK, DV, TI, false>;
+    cudaError_t e = allow_smem(kern, smem, LL::step_smem(kMaxM - 1, false));
+    if (e != cudaSuccess) return e;
+    kern<<<s.BH, TL::NT, smem, st>>>(a);
   }
   return cudaGetLastError();
 }
@@ -40,13 +54,11 @@ cudaError_t eager_dims(const LaunchShape& s, const StepArgs& a, cudaStream_t st)
 
 template <int OP, int DK, int DV, typename TI>
 cudaError_t materialize_dims(const LaunchShape& s, const MaterializeArgs& a, cudaStream_t st) {
+  using LL = LogLayout<OP, DK, DV, TI>;
   auto kern = materialize_kernel<OP, DK, DV, TI>;
-  const size_t smem = static_cast<size_t>(a.n) * (DK + DV) * sizeof(float);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kMaxM * (DK + DV) * sizeof(float)));
-    if (e != cudaSuccess) return e;
-  }
+  const size_t smem = LL::materialize_smem(a.n);
+  cudaError_t e = allow_smem(kern, smem, LL::materialize_smem(kMaxM - 1));
+  if (e != cudaSuccess) return e;
   kern<<<s.BH, Tile<DK, DV>::NT, smem, st>>>(a);
   return cudaGetLastError();
 }
