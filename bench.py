@@ -226,15 +226,16 @@ def cpu_threads():
 
 
 def cpu_baseline(a, budget_s=10.0):
-    """Oracle throughput on a bounded sample: 1 slot (H heads), growing token count."""
-    tokens, el = 8, 0.0
-    while True:
-        el = oracle_sample(a, 1, tokens)
-        if el >= budget_s or tokens >= a.tokens:
-            break
-        tokens = min(a.tokens, max(tokens * 2, int(tokens * budget_s / max(el, 1e-3))))
-    return {"value": tokens / el, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"1 slot x {a.H} heads x {tokens} tokens of {workload_name(a)} (fp64 eager)",
+    """Oracle throughput on a bounded sample of the workload: the first `slots`
+    slots (all H heads) over one bench step of tokens, grown to ~budget_s."""
+    tokens = a.tokens
+    probe = min(a.tokens, 32)
+    el = oracle_sample(a, 1, probe)
+    slots = int(max(1, min(a.B, budget_s / max(el * tokens / probe, 1e-3))))
+    el = oracle_sample(a, slots, tokens)
+    return {"value": slots * tokens / el, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{slots} slots x {a.H} heads x {tokens} tokens of {workload_name(a)} "
+                      f"(fp64 eager recurrence)",
             "seconds": round(el, 3)}
 
 
