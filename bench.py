@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-eager", action="store_true")
     ap.add_argument("--sweep", default="", help="extra M values to time, e.g. 1,4,16")
+    ap.add_argument("--kernel", choices=["auto", "register", "stream"], default="auto",
+                    help="dl_step kernel variant")
     args = ap.parse_args()
     if args.tokens % args.M:
         ap.error("--tokens must be a multiple of --M")
@@ -302,6 +304,7 @@ def run_gpu(a, rank, world, local_rank):
 
     def make_handle(m):
         h = DeltaLog(B, H, d, d, m, op=op, dtype=torch.bfloat16)
+        h.set_step_kernel(a.kernel)
         h.load_state(S0)
         if u is not None:
             h.set_bonus(u)
@@ -320,6 +323,7 @@ def run_gpu(a, rank, world, local_rank):
         return float(t.item())
 
     tok_counter = [0]
+    used_kernel = [None]
 
     def run_step(h, m, eager=False, ev=None, rec=None):
         """One bench step: a.tokens decode tokens through dl_step (or dl_eager_step).
@@ -358,6 +362,7 @@ def run_gpu(a, rank, world, local_rank):
         launches = None
         if per_launch:
             launches = [(e0.elapsed_time(e1), n) for e0, e1, n in rec]
+        used_kernel[0] = h.last_step_kernel
         h.check_device(stream)
         h.close()
         return max_over_ranks(ms), launches
@@ -379,7 +384,8 @@ def run_gpu(a, rank, world, local_rank):
     if M > 1 and launches:
         dur = sum(t for t, _ in launches) / len(launches)
         alg = sum(launch_bytes(op, "append", B, H, d, d, n) for _, n in launches) / len(launches)
-        dominant = "deltalog_step_kernel (append)"
+        dominant = ("deltalog_stream_kernel" if used_kernel[0] == "stream"
+                    else "deltalog_step_kernel") + " (append)"
     else:
         dur = ms / (a.steps * a.tokens)
         alg = launch_bytes(op, "eager" if M == 1 else "merge", B, H, d, d, 0)
@@ -451,6 +457,7 @@ def run_gpu(a, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": workload_name(a), "op": op, "B": B, "H": H, "d_k": d, "d_v": d,
                    "M": M, "state": "fp32", "inputs": "bf16", "tokens_per_step": a.tokens,
+                   "step_kernel": used_kernel[0],
                    "input_pool_tokens": a.pool, "seed": a.seed,
                    "l2": f"inputs larger than L2 (state {4 * B * H * d * d / 1e6:.0f} MB)",
                    "parallelism": "replicas" if world == 1 else f"replicas x{world} (B per rank)"},

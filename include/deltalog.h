@@ -75,7 +75,9 @@ enum dl_status {
 
 /* Create a handle for B slots x H heads.  Supported: d_k, d_v in {64, 128},
  * 1 <= M <= DL_MAX_M.  The base state starts at zero with an empty log; the
- * RWKV6 bonus starts at zero.  Pointers passed later must be 16-byte aligned.
+ * RWKV6 bonus starts at zero.  Pointers passed later must be aligned to their
+ * element size (state pointers to 16 bytes); q, k, v (and per-key
+ * log_decay) aligned to 16 bytes let dl_step use its streaming kernel.
  * M = 1 makes every step a merge step (the deferred path then performs the
  * eager schedule). */
 #define DL_MAX_M 64
@@ -117,6 +119,23 @@ int dl_merge(dl_t h, void* stream);
 /* Write the logical state (Sbar + replayed log) to S_out [B][H][d_k][d_v]
  * (device pointer) without changing the handle. */
 int dl_read_state(dl_t h, float* S_out, void* stream);
+
+/* Tuning options.  DL_OPT_STEP_KERNEL picks the kernel behind dl_step; all
+ * variants compute the same result up to the order of fp32 summation.
+ *   DL_STEP_AUTO (default): the fastest kernel measured for the launch
+ *     (currently the register-tile kernel everywhere);
+ *   DL_STEP_REGISTER: always the register-tile kernel (one CTA per slot-head);
+ *   DL_STEP_STREAM: the persistent TMA-streaming kernel; needs q, k, v (and,
+ *     for KDA/RWKV6, log_decay) 16-byte aligned and a shared-memory plan that
+ *     fits the device, else dl_step returns DL_ERR_UNSUPPORTED.
+ * Returns DL_ERR_ARG for an unknown option or value. */
+enum dl_option { DL_OPT_STEP_KERNEL = 0 };
+enum dl_step_kernel { DL_STEP_AUTO = 0, DL_STEP_REGISTER = 1, DL_STEP_STREAM = 2 };
+int dl_set_option(dl_t h, int option, int value);
+
+/* Which kernel the most recent dl_step / dl_step_host launched:
+ * DL_STEP_REGISTER or DL_STEP_STREAM (DL_STEP_AUTO before the first step). */
+int dl_last_step_kernel(dl_t h, int* kind);
 
 /* Number of entries currently in the log (host-side counter, exact in stream
  * order). */

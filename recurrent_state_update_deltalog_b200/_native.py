@@ -15,6 +15,8 @@ DL_GDN, DL_KDA, DL_RWKV6 = 0, 1, 2
 DL_F32, DL_BF16 = 0, 1
 DL_OK = 0
 DL_MAX_M = 64
+DL_OPT_STEP_KERNEL = 0
+DL_STEP_AUTO, DL_STEP_REGISTER, DL_STEP_STREAM = 0, 1, 2
 STATUS = {0: "DL_OK", -1: "DL_ERR_ARG", -2: "DL_ERR_UNSUPPORTED", -3: "DL_ERR_CUDA",
           -4: "DL_ERR_OOM", -5: "DL_ERR_DEVICE", -6: "DL_ERR_STATE"}
 
@@ -31,6 +33,8 @@ SIGNATURES = {
     "dl_eager_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
     "dl_merge": (_I, [_P, _P]),
     "dl_read_state": (_I, [_P, _P, _P]),
+    "dl_set_option": (_I, [_P, _I, _I]),
+    "dl_last_step_kernel": (_I, [_P, ctypes.POINTER(_I)]),
     "dl_log_len": (_I, [_P, ctypes.POINTER(_I)]),
     "dl_check_device": (_I, [_P, _P]),
     "dl_strerror": (ctypes.c_char_p, [_I]),

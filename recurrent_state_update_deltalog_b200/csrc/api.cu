@@ -11,6 +11,9 @@
 
 struct dl_handle {
   int B, H, dk, dv, M, op, dtype, device;
+  int sms, smem_block_optin, smem_sm, smem_reserved;  // device limits
+  int step_kernel;                                    // DL_STEP_* requested
+  int last_kernel;                                    // DL_STEP_* used by the last dl_step
   int n;       // entries in the log (host counter; all slots step in lockstep)
   int Mcap;    // log capacity per (slot, head): max(M - 1, 1)
   size_t esize;
@@ -72,6 +75,9 @@ class DeviceScope {
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 size_t lam_per_entry(const dl_handle* h) { return h->op == DL_GDN ? 1 : static_cast<size_t>(h->dk); }
+size_t lam_unit_floats(const dl_handle* h) {
+  return h->op == DL_GDN ? static_cast<size_t>(dl::gdn_lam_stride(h->Mcap)) : static_cast<size_t>(h->Mcap) * h->dk;
+}
 size_t logb_esize(const dl_handle* h) { return h->op == DL_RWKV6 ? h->esize : sizeof(float); }
 size_t bh(const dl_handle* h) { return static_cast<size_t>(h->B) * h->H; }
 size_t state_bytes(const dl_handle* h) { return bh(h) * h->dk * h->dv * sizeof(float); }
@@ -84,8 +90,19 @@ void free_all(dl_handle* h) {
     if (p) cudaFree(p);
 }
 
-dl::LaunchShape shape_of(const dl_handle* h) {
-  return dl::LaunchShape{static_cast<int>(bh(h)), h->dk, h->dv, h->dtype};
+dl::LaunchShape shape_of(const dl_handle* h, bool aligned16 = false) {
+  dl::LaunchShape s;
+  s.BH = static_cast<int>(bh(h));
+  s.dk = h->dk;
+  s.dv = h->dv;
+  s.dtype = h->dtype;
+  s.sms = h->sms;
+  s.smem_block_optin = h->smem_block_optin;
+  s.smem_sm = h->smem_sm;
+  s.smem_reserved = h->smem_reserved;
+  s.variant = h->step_kernel;
+  s.aligned16 = aligned16;
+  return s;
 }
 
 int check_step_args(const dl_handle* h, const void* q, const void* k, const void* v,
@@ -122,12 +139,16 @@ dl::StepArgs step_args(dl_handle* h, const void* q, const void* k, const void* v
   return a;
 }
 
-cudaError_t launch_step(const dl_handle* h, bool merge, const dl::StepArgs& a, cudaStream_t s) {
-  const dl::LaunchShape sh = shape_of(h);
+cudaError_t launch_step(dl_handle* h, bool merge, const dl::StepArgs& a, cudaStream_t s) {
+  // bulk-copy sources of the streaming kernel (GDN's scalar gate is a plain load)
+  const bool al = aligned(a.q, 16) && aligned(a.k, 16) && aligned(a.v, 16) &&
+                  (h->op == DL_GDN || aligned(a.log_decay, 16));
+  const dl::LaunchShape sh = shape_of(h, al);
+  int* used = &h->last_kernel;
   switch (h->op) {
-    case DL_GDN: return dl::launch_step_op<dl::OP_GDN>(sh, merge, a, s);
-    case DL_KDA: return dl::launch_step_op<dl::OP_KDA>(sh, merge, a, s);
-    default: return dl::launch_step_op<dl::OP_RWKV6>(sh, merge, a, s);
+    case DL_GDN: return dl::launch_step_op<dl::OP_GDN>(sh, merge, a, s, used);
+    case DL_KDA: return dl::launch_step_op<dl::OP_KDA>(sh, merge, a, s, used);
+    default: return dl::launch_step_op<dl::OP_RWKV6>(sh, merge, a, s, used);
   }
 }
 
@@ -162,6 +183,8 @@ int do_step(dl_handle* h, const void* q, const void* k, const void* v, const flo
             const float* beta, void* o, cudaStream_t s) {
   const bool merge = h->n + 1 == h->M;
   cudaError_t e = launch_step(h, merge, step_args(h, q, k, v, log_decay, beta, o), s);
+  if (e == cudaErrorNotSupported)
+    return fail(DL_ERR_UNSUPPORTED, "the streaming step kernel cannot run this launch (alignment or shared memory)");
   if (e != cudaSuccess) return cuda_fail(e, "deltalog step launch");
   h->n = merge ? 0 : h->n + 1;
   return DL_OK;
@@ -194,9 +217,27 @@ int dl_create(dl_t* out, int B, int H, int d_k, int d_v, int M, int op, int in_d
   h->n = 0;
   h->Mcap = M > 1 ? M - 1 : 1;
   h->esize = in_dtype == DL_BF16 ? 2 : 4;
+  h->step_kernel = DL_STEP_AUTO;
+  h->last_kernel = DL_STEP_AUTO;
   if (cudaGetDevice(&h->device) != cudaSuccess) {
     delete h;
     return fail(DL_ERR_CUDA, "no current CUDA device");
+  }
+  {
+    const struct {
+      int* dst;
+      cudaDeviceAttr attr;
+    } q[] = {{&h->sms, cudaDevAttrMultiProcessorCount},
+             {&h->smem_block_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin},
+             {&h->smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor},
+             {&h->smem_reserved, cudaDevAttrReservedSharedMemoryPerBlock}};
+    for (auto& x : q) {
+      cudaError_t e = cudaDeviceGetAttribute(x.dst, x.attr, h->device);
+      if (e != cudaSuccess) {
+        delete h;
+        return cuda_fail(e, "device attribute query");
+      }
+    }
   }
   const size_t nbh = bh(h);
   struct {
@@ -206,7 +247,7 @@ int dl_create(dl_t* out, int B, int H, int d_k, int d_v, int M, int op, int in_d
       {reinterpret_cast<void**>(&h->Sbar), state_bytes(h)},
       {&h->logA, nbh * h->Mcap * d_k * h->esize},
       {&h->logB, nbh * h->Mcap * d_v * logb_esize(h)},
-      {reinterpret_cast<void**>(&h->logLam), nbh * h->Mcap * lam_per_entry(h) * sizeof(float)},
+      {reinterpret_cast<void**>(&h->logLam), nbh * lam_unit_floats(h) * sizeof(float)},
       {reinterpret_cast<void**>(&h->u), static_cast<size_t>(H) * d_k * sizeof(float)},
       {reinterpret_cast<void**>(&h->err), sizeof(int)},
       {&h->sq, nbh * d_k * h->esize},
@@ -340,6 +381,20 @@ int dl_read_state(dl_t h, float* S_out, void* stream) {
   cudaError_t e = h->n == 0 ? cudaMemcpyAsync(S_out, h->Sbar, state_bytes(h), cudaMemcpyDeviceToDevice, s)
                             : launch_materialize(h, S_out, s);
   return e == cudaSuccess ? DL_OK : cuda_fail(e, "dl_read_state");
+}
+
+int dl_set_option(dl_t h, int option, int value) {
+  if (!h) return fail(DL_ERR_ARG, "null handle");
+  if (option != DL_OPT_STEP_KERNEL) return fail(DL_ERR_ARG, "unknown option %d", option);
+  if (value < DL_STEP_AUTO || value > DL_STEP_STREAM) return fail(DL_ERR_ARG, "bad step-kernel value %d", value);
+  h->step_kernel = value;
+  return DL_OK;
+}
+
+int dl_last_step_kernel(dl_t h, int* kind) {
+  if (!h || !kind) return fail(DL_ERR_ARG, "null argument");
+  *kind = h->last_kernel;
+  return DL_OK;
 }
 
 int dl_log_len(dl_t h, int* n) {

@@ -50,7 +50,7 @@ struct StepArgs {
   void* o;                 // [BH][DV], input dtype
   void* logA;              // [BH][Mcap][DK], input dtype (a_i = k_i)
   void* logB;              // [BH][Mcap][DV], fp32 (GDN/KDA) or input dtype (RWKV6)
-  float* logLam;           // [BH][Mcap] (GDN) or [BH][Mcap][DK]
+  float* logLam;           // [BH][gdn_lam_stride(Mcap)] (GDN) or [BH][Mcap][DK]
   const float* u;          // [H][DK] (RWKV6)
   int* err;               // device error word (kErr* bits)
   int H;
@@ -117,6 +117,10 @@ struct Tile {
 
 // Largest supported merge interval M (log capacity M-1).
 constexpr int kMaxM = 64;
+
+// GDN keeps one scalar snapshot per entry; each head's row of snapshots is
+// padded to a multiple of 4 floats so that it can be staged by a bulk copy.
+__host__ __device__ constexpr int gdn_lam_stride(int Mcap) { return (Mcap + 3) & ~3; }
 
 // Shared-memory image of a (slot, head)'s log, staged by TMA bulk copies.
 // Byte layout (every region starts 16-byte aligned):
@@ -205,7 +209,7 @@ deltalog_step_kernel(const StepArgs a) {
   __shared__ float s_lam[kMaxM];                 // GDN: scalar Lam_i of the log entries
   __shared__ float s_kappa;
   __shared__ __align__(8) uint64_t s_bar;
-  extern __shared__ __align__(16) unsigned char s_dyn[];
+  extern __shared__ __align__(128) unsigned char s_dyn[];
 
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
@@ -244,8 +248,8 @@ deltalog_step_kernel(const StepArgs a) {
       lt[m] = lp[m] + a.log_decay[sh * DK + j];
     }
   } else {
-    if (tid < n) s_lam[tid] = a.logLam[sh * a.Mcap + tid];
-    const float lprev = n > 0 ? a.logLam[sh * a.Mcap + (n - 1)] : 0.f;
+    if (tid < n) s_lam[tid] = a.logLam[sh * gdn_lam_stride(a.Mcap) + tid];
+    const float lprev = n > 0 ? a.logLam[sh * gdn_lam_stride(a.Mcap) + (n - 1)] : 0.f;
     const float lcur = lprev + a.log_decay[sh];
 #pragma unroll
     for (int m = 0; m < TL::KPL; ++m) {
@@ -329,7 +333,7 @@ deltalog_step_kernel(const StepArgs a) {
         dstA[j] = kg[j];
         if (PERKEY) a.logLam[(sh * a.Mcap + n) * DK + j] = lt[m];
       }
-      if (!PERKEY && lane == 0) a.logLam[sh * a.Mcap + n] = lt[0];
+      if (!PERKEY && lane == 0) a.logLam[sh * gdn_lam_stride(a.Mcap) + n] = lt[0];
     }
   }
   __syncthreads();
@@ -539,7 +543,7 @@ materialize_kernel(const MaterializeArgs a) {
   __shared__ __align__(16) float s_dec[DK];
   __shared__ float s_lam[kMaxM];
   __shared__ __align__(8) uint64_t s_bar;
-  extern __shared__ __align__(16) unsigned char s_dyn[];
+  extern __shared__ __align__(128) unsigned char s_dyn[];
 
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
@@ -562,9 +566,10 @@ materialize_kernel(const MaterializeArgs a) {
 #pragma unroll
   for (int m = 0; m < TL::KPL; ++m) {
     const int j = lane + 32 * m;
-    ll[m] = PERKEY ? a.logLam[(sh * a.Mcap + (n - 1)) * DK + j] : a.logLam[sh * a.Mcap + (n - 1)];
+    ll[m] = PERKEY ? a.logLam[(sh * a.Mcap + (n - 1)) * DK + j]
+                   : a.logLam[sh * gdn_lam_stride(a.Mcap) + (n - 1)];
   }
-  if (!PERKEY && tid < n) s_lam[tid] = a.logLam[sh * a.Mcap + tid];
+  if (!PERKEY && tid < n) s_lam[tid] = a.logLam[sh * gdn_lam_stride(a.Mcap) + tid];
   __syncthreads();
   if (!wait_log(&s_bar, n, a.err)) return;
 

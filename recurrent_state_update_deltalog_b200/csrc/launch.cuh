@@ -4,15 +4,76 @@
 #pragma once
 
 #include "kernels.cuh"
+#include "stream.cuh"
 
 namespace dl {
 
+// Step-kernel variants (dl_set_option DL_OPT_STEP_KERNEL).
+enum { STEP_AUTO = 0, STEP_REGISTER = 1, STEP_STREAM = 2 };
+
 struct LaunchShape {
-  int BH;     // slots x heads = grid size
+  int BH;     // slots x heads
   int dk;
   int dv;
   int dtype;  // 0 = fp32, 1 = bf16 inputs
+  // device limits, queried once per handle
+  int sms;
+  int smem_block_optin;
+  int smem_sm;
+  int smem_reserved;
+  int variant;     // STEP_*
+  bool aligned16;  // q, k, v, log_decay all 16-byte aligned (bulk-copy sources)
 };
+
+// Ring/slot plan of the streaming kernel for one launch.
+struct StreamPlan {
+  bool ok;
+  int ctas_per_sm;
+  int ns;
+  size_t smem;
+};
+
+// Largest ring that fits: two CTAs per SM first (each one's finalize then
+// overlaps the other's streaming), else one CTA with a deeper ring.  A merge
+// launch keeps all of a unit's chunks resident until its write-back, so its
+// ring holds at least one chunk more than a unit.
+template <int OP, int DK, int DV, typename TI>
+StreamPlan plan_stream(const LaunchShape& s, int n, bool merge, size_t static_smem) {
+  using SG = StreamGeom<OP, DK, DV, TI>;
+  const int min_ns = merge ? SG::CPU + 1 : 2;
+  const int max_ns[2] = {6, kMaxStages};
+  for (int pass = 0; pass < 2; ++pass) {
+    const int ctas = pass == 0 ? 2 : 1;
+    for (int ns = max_ns[pass]; ns >= min_ns; --ns) {
+      const size_t dyn = SG::smem(n, merge, ns);
+      const size_t blk = dyn + static_smem;
+      if (blk > static_cast<size_t>(s.smem_block_optin)) continue;
+      if (static_cast<size_t>(ctas) * (blk + s.smem_reserved) > static_cast<size_t>(s.smem_sm)) continue;
+      return StreamPlan{true, ctas, ns, dyn};
+    }
+  }
+  return StreamPlan{false, 0, 0, 0};
+}
+
+template <int OP, int DK, int DV, typename TI, bool MERGE>
+cudaError_t stream_dims(const LaunchShape& s, const StepArgs& a, cudaStream_t st, bool* launched) {
+  auto kern = deltalog_stream_kernel<OP, DK, DV, TI, MERGE>;
+  *launched = false;
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  const StreamPlan p = plan_stream<OP, DK, DV, TI>(s, a.n, MERGE, fa.sharedSizeBytes);
+  if (!p.ok) return cudaSuccess;
+  if (p.smem + fa.sharedSizeBytes > 48 * 1024) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             s.smem_block_optin - static_cast<int>(fa.sharedSizeBytes));
+    if (e != cudaSuccess) return e;
+  }
+  const int grid = s.BH < p.ctas_per_sm * s.sms ? s.BH : p.ctas_per_sm * s.sms;
+  kern<<<grid, Tile<DK, DV>::NT, p.smem, st>>>(a, StreamCfg{s.BH, p.ns});
+  *launched = true;
+  return cudaGetLastError();
+}
 
 // Opt a kernel into more than the default 48 KB of shared memory (static +
 // dynamic) when a launch needs it; `worst` is the largest dynamic size any
@@ -28,9 +89,20 @@ cudaError_t allow_smem(K kern, size_t smem, size_t worst) {
 }
 
 template <int OP, int DK, int DV, typename TI>
-cudaError_t step_dims(const LaunchShape& s, bool merge, const StepArgs& a, cudaStream_t st) {
+cudaError_t step_dims(const LaunchShape& s, bool merge, const StepArgs& a, cudaStream_t st, int* used) {
   using TL = Tile<DK, DV>;
   using LL = LogLayout<OP, DK, DV, TI>;
+  // AUTO runs the register-tile kernel: it is the faster of the two on B200
+  // (GDN B=256 H=32 d=128: 92 vs 101 us per append launch); STREAM is opt-in.
+  if (s.variant == STEP_STREAM && s.aligned16) {
+    bool launched = false;
+    cudaError_t e = merge ? stream_dims<OP, DK, DV, TI, true>(s, a, st, &launched)
+                          : stream_dims<OP, DK, DV, TI, false>(s, a, st, &launched);
+    if (launched) *used = STEP_STREAM;
+    if (e != cudaSuccess || launched) return e;
+  }
+  if (s.variant == STEP_STREAM) return cudaErrorNotSupported;
+  *used = STEP_REGISTER;
   const size_t smem = LL::step_smem(a.n, merge);
   if (merge) {
     auto kern = deltalog_step_kernel<OP, DK, DV, TI, true>;
@@ -77,8 +149,8 @@ cudaError_t materialize_dims(const LaunchShape& s, const MaterializeArgs& a, cud
   } while (0)
 
 template <int OP>
-cudaError_t launch_step_op(const LaunchShape& s, bool merge, const StepArgs& a, cudaStream_t st) {
-  DL_DISPATCH_DIMS(step_dims, s, merge, a, st);
+cudaError_t launch_step_op(const LaunchShape& s, bool merge, const StepArgs& a, cudaStream_t st, int* used) {
+  DL_DISPATCH_DIMS(step_dims, s, merge, a, st, used);
 }
 
 template <int OP>
@@ -92,12 +164,12 @@ cudaError_t launch_materialize_op(const LaunchShape& s, const MaterializeArgs& a
 }
 
 #define DL_DECLARE_OP(OPV)                                                                      \
-  extern template cudaError_t launch_step_op<OPV>(const LaunchShape&, bool, const StepArgs&, cudaStream_t); \
+  extern template cudaError_t launch_step_op<OPV>(const LaunchShape&, bool, const StepArgs&, cudaStream_t, int*); \
   extern template cudaError_t launch_eager_op<OPV>(const LaunchShape&, const StepArgs&, cudaStream_t);      \
   extern template cudaError_t launch_materialize_op<OPV>(const LaunchShape&, const MaterializeArgs&, cudaStream_t);
 
 #define DL_INSTANTIATE_OP(OPV)                                                                  \
-  template cudaError_t launch_step_op<OPV>(const LaunchShape&, bool, const StepArgs&, cudaStream_t); \
+  template cudaError_t launch_step_op<OPV>(const LaunchShape&, bool, const StepArgs&, cudaStream_t, int*); \
   template cudaError_t launch_eager_op<OPV>(const LaunchShape&, const StepArgs&, cudaStream_t);      \
   template cudaError_t launch_materialize_op<OPV>(const LaunchShape&, const MaterializeArgs&, cudaStream_t);
 

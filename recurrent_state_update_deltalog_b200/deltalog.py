@@ -126,6 +126,18 @@ class DeltaLog:
         N.call("dl_read_state", self._h, _ptr(out), self._stream(stream))
         return out
 
+    def set_step_kernel(self, kind):
+        """``"auto"`` (default), ``"register"`` or ``"stream"``: which kernel runs dl_step."""
+        vals = {"auto": N.DL_STEP_AUTO, "register": N.DL_STEP_REGISTER, "stream": N.DL_STEP_STREAM}
+        N.call("dl_set_option", self._h, N.DL_OPT_STEP_KERNEL, vals[kind])
+
+    @property
+    def last_step_kernel(self):
+        """Kernel used by the most recent step: ``"register"``, ``"stream"`` or ``None``."""
+        k = ctypes.c_int()
+        N.call("dl_last_step_kernel", self._h, ctypes.byref(k))
+        return {N.DL_STEP_REGISTER: "register", N.DL_STEP_STREAM: "stream"}.get(k.value)
+
     @property
     def log_len(self):
         n = ctypes.c_int()

@@ -45,13 +45,16 @@ def step_args(op, dseq, t):
     return first[t], dseq["k"][t], dseq["v"][t], dseq["log_decay"][t], beta
 
 
-def run_gpu(op, S0, seq, u, M, dtype, eager=False, record_merges=True):
-    """Run T steps through the library; returns (o[T,B,H,dv], {t: Sbar}, final logical S)."""
+def run_gpu(op, S0, seq, u, M, dtype, eager=False, record_merges=True, kernel="auto"):
+    """Run T steps through the library; returns (o[T,B,H,dv], {t: Sbar}, final logical S).
+
+    ``kernel`` selects the dl_step kernel ("auto", "register" or "stream")."""
     from recurrent_state_update_deltalog_b200 import DeltaLog
     B, H, dk, dv = S0.shape
     T = seq["k"].shape[0]
     dseq = to_device(seq, dtype)
     h = DeltaLog(B, H, dk, dv, M, op=op, dtype=dtype)
+    h.set_step_kernel(kernel)
     try:
         h.load_state(torch.from_numpy(S0).cuda())
         if u is not None:

@@ -14,11 +14,14 @@ pytestmark = pytest.mark.gpu
 OPS = ["gdn", "kda", "rwkv6"]
 
 
-def _check_run(op, B, H, dk, dv, M, T, dtype, eager=False, seed=0):
+KERNELS = ["register", "stream"]
+
+
+def _check_run(op, B, H, dk, dv, M, T, dtype, eager=False, seed=0, kernel="auto"):
     S0, seq, u = make_inputs(op, B, H, dk, dv, T, dtype, seed)
     merge_steps = [t for t in range(T) if (t + 1) % M == 0] if not eager else []
     o_ref, S_ref, kept = run_oracle(op, S0, seq, u, record=set(merge_steps))
-    o, merges, final = run_gpu(op, S0, seq, u, M, dtype, eager=eager)
+    o, merges, final = run_gpu(op, S0, seq, u, M, dtype, eager=eager, kernel=kernel)
     tol = TOL[dtype]
     e_o = relerr(o, o_ref)
     assert e_o < tol, f"outputs: {e_o:.3e}"
@@ -30,24 +33,61 @@ def _check_run(op, B, H, dk, dv, M, T, dtype, eager=False, seed=0):
     return e_o, e_s
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("M", [8, 1])
-def test_gdn_single_head_fp32(M):
+def test_gdn_single_head_fp32(M, kernel):
     """B=H=1, d=64, fp32 inputs, 64 steps, seed 0."""
-    _check_run("gdn", 1, 1, 64, 64, M, 64, torch.float32)
+    _check_run("gdn", 1, 1, 64, 64, M, 64, torch.float32, kernel=kernel)
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("op", OPS)
 @pytest.mark.parametrize("dims", [(64, 64), (128, 128), (64, 128), (128, 64)])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-def test_deferred_shapes(op, dims, dtype):
+def test_deferred_shapes(op, dims, dtype, kernel):
     """Ragged B*H, every shape, M=4 with a tail that ends mid-cycle."""
-    _check_run(op, 3, 5, dims[0], dims[1], 4, 11, dtype)
+    _check_run(op, 3, 5, dims[0], dims[1], 4, 11, dtype, kernel=kernel)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 16, 32, 33, 64])
+def test_deferred_every_M(op, M, kernel):
+    T = min(2 * M + 3, 70)
+    if kernel == "stream" and M == 64 and op != "gdn":
+        # A 63-entry per-key log does not fit the streaming kernel's shared
+        # memory next to its ring: forcing it is refused, AUTO falls back.
+        from recurrent_state_update_deltalog_b200 import DeltaLogError
+        with pytest.raises(DeltaLogError) as ei:
+            _check_run(op, 2, 3, 128, 128, M, T, torch.bfloat16, kernel="stream")
+        assert ei.value.status == -2
+        kernel = "auto"
+    _check_run(op, 2, 3, 128, 128, M, T, torch.bfloat16, kernel=kernel)
+
+
+def test_step_kernel_selection_is_reported():
+    from recurrent_state_update_deltalog_b200 import DeltaLog
+    S0, seq, _ = make_inputs("gdn", 4, 8, 128, 128, 3, torch.bfloat16)
+    dseq = to_device(seq, torch.bfloat16)
+    h = DeltaLog(4, 8, 128, 128, 8, op="gdn")
+    assert h.last_step_kernel is None
+    h.step(*step_args("gdn", dseq, 0))
+    assert h.last_step_kernel in ("register", "stream")
+    h.set_step_kernel("stream")
+    h.step(*step_args("gdn", dseq, 1))
+    assert h.last_step_kernel == "stream"
+    h.set_step_kernel("register")
+    h.step(*step_args("gdn", dseq, 2))
+    assert h.last_step_kernel == "register"
+    h.close()
 
 
 @pytest.mark.parametrize("op", OPS)
-@pytest.mark.parametrize("M", [1, 2, 3, 8, 16, 32, 33, 64])
-def test_deferred_every_M(op, M):
-    _check_run(op, 2, 3, 128, 128, M, min(2 * M + 3, 70), torch.bfloat16)
+def test_stream_kernel_many_units_per_cta(op):
+    """More units than persistent CTAs: every CTA walks several units and the
+    ring wraps many times (B*H = 2000 > 2 x SM count)."""
+    _check_run(op, 125, 16, 64, 64, 4, 9, torch.bfloat16, kernel="stream")
+    _check_run(op, 40, 16, 128, 128, 3, 7, torch.bfloat16, kernel="stream")
 
 
 @pytest.mark.parametrize("op", OPS)
@@ -65,7 +105,7 @@ def test_M1_deferred_matches_eager_kernel(op):
     assert relerr(o_d, o_e) < 1e-5 and relerr(s_d, s_e) < 1e-5
 
 
-def _full_size_case(op, B, H, d, M, T, n_units=24):
+def _full_size_case(op, B, H, d, M, T, n_units=24, kernel="auto"):
     """Full-size launch; sampled (slot, head) units checked against the oracle."""
     dtype = torch.bfloat16
     S0, seq, u = make_inputs(op, B, H, d, d, T, dtype)
@@ -78,7 +118,7 @@ def _full_size_case(op, B, H, d, M, T, n_units=24):
     u_s = u[hs] if u is not None else None
     merge_steps = [t for t in range(T) if (t + 1) % M == 0]
     o_ref, S_ref, kept = run_oracle(op, S0_s, seq_s, u_s, record=set(merge_steps))
-    o, merges, final = run_gpu(op, S0, seq, u, M, dtype)
+    o, merges, final = run_gpu(op, S0, seq, u, M, dtype, kernel=kernel)
     assert relerr(o[:, bs, hs], o_ref) < TOL[dtype]
     for t in merge_steps:
         assert relerr(merges[t][bs, hs], kept[t]) < TOL[dtype]
@@ -90,6 +130,10 @@ def _full_size_case(op, B, H, d, M, T, n_units=24):
 @pytest.mark.parametrize("M", [8, 4, 16, 1])
 def test_full_size_gdn_b256_h32_d128(M):
     _full_size_case("gdn", 256, 32, 128, M, 2 * M + 3 if M > 1 else 6)
+
+
+def test_full_size_gdn_b256_h32_d128_register_kernel():
+    _full_size_case("gdn", 256, 32, 128, 8, 19, kernel="register")
 
 
 def test_full_size_kda_b128_h32_d128():
@@ -185,3 +229,30 @@ def test_zero_log_decay_and_beta_zero_keep_state():
         assert np.array_equal(final, S0)
         want = np.einsum("bhkv,tbhk->tbhv", S0.astype(np.float64), seq["q"].astype(np.float64))
         assert relerr(o, want) < 1e-5
+
+
+def test_unaligned_inputs_fall_back_or_refuse():
+    """q/k/v views offset by one element: AUTO runs the register kernel (same
+    result), STREAM refuses with DL_ERR_UNSUPPORTED."""
+    from recurrent_state_update_deltalog_b200 import DeltaLog, DeltaLogError
+    B, H, d, M, T = 2, 4, 64, 4, 6
+    S0, seq, _ = make_inputs("gdn", B, H, d, d, T, torch.bfloat16)
+    o_ref, S_ref, _ = run_oracle("gdn", S0, seq, None)
+    dseq = to_device(seq, torch.bfloat16)
+    shifted = {}
+    for key in ("q", "k", "v"):
+        flat = torch.zeros(dseq[key].numel() + 1, dtype=torch.bfloat16, device="cuda")
+        flat[1:] = dseq[key].reshape(-1)
+        shifted[key] = flat[1:].view(dseq[key].shape)
+    h = DeltaLog(B, H, d, d, M, op="gdn")
+    h.load_state(torch.from_numpy(S0).cuda())
+    outs = []
+    for t in range(T):
+        outs.append(h.step(shifted["q"][t], shifted["k"][t], shifted["v"][t],
+                           dseq["log_decay"][t], dseq["beta"][t]).float().cpu().numpy())
+    assert relerr(np.stack(outs), o_ref) < 5e-3
+    h.set_step_kernel("stream")
+    with pytest.raises(DeltaLogError) as ei:
+        h.step(shifted["q"][0], shifted["k"][0], shifted["v"][0], dseq["log_decay"][0], dseq["beta"][0])
+    assert ei.value.status == -2
+    h.close()
