@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--sweep", default="", help="extra M values to time, e.g. 1,4,16")
     ap.add_argument("--kernel", choices=["auto", "register", "stream"], default="auto",
                     help="dl_step kernel variant")
+    ap.add_argument("--no-pdl", action="store_true",
+                    help="launch every step with plain stream ordering")
     args = ap.parse_args()
     if args.tokens % args.M:
         ap.error("--tokens must be a multiple of --M")
@@ -305,6 +307,7 @@ def run_gpu(a, rank, world, local_rank):
     def make_handle(m):
         h = DeltaLog(B, H, d, d, m, op=op, dtype=torch.bfloat16)
         h.set_step_kernel(a.kernel)
+        h.set_pdl(not a.no_pdl)
         h.load_state(S0)
         if u is not None:
             h.set_bonus(u)
@@ -344,17 +347,21 @@ def run_gpu(a, rank, world, local_rank):
                 h.step(*args, out=out[i], stream=stream)
 
     def timed(m, eager=False, per_launch=False):
+        """Time a.steps bench steps (or, with per_launch, a shorter second pass in
+        which every append launch is bracketed by its own pair of events: those
+        events sit between launches, so each launch is timed in isolation)."""
         h = make_handle(m)
         for _ in range(a.warmup):
             run_step(h, m, eager)
-        nev = a.steps * a.tokens if per_launch else 0
+        steps = min(a.steps, 2) if per_launch else a.steps
+        nev = steps * a.tokens if per_launch else 0
         rec = []
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(nev)]
         start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
         start.record(stream)
-        for _ in range(a.steps):
+        for _ in range(steps):
             run_step(h, m, eager, ev if per_launch else None, rec)
         stop.record(stream)
         barrier()
@@ -362,7 +369,8 @@ def run_gpu(a, rank, world, local_rank):
         launches = None
         if per_launch:
             launches = [(e0.elapsed_time(e1), n) for e0, e1, n in rec]
-        used_kernel[0] = h.last_step_kernel
+        if not eager:
+            used_kernel[0] = h.last_step_kernel
         h.check_device(stream)
         h.close()
         return max_over_ranks(ms), launches
@@ -370,11 +378,13 @@ def run_gpu(a, rank, world, local_rank):
     peak, peak_kind = measured_peak()
     result = {}
 
-    # headline: DeltaLog at M, with per-launch timing of the dominant (append) kernel
+    # headline: DeltaLog at M over the timed region (no events between launches)
     sampler = ClockSampler(local_rank)
     sampler.start()
-    ms, launches = timed(M, per_launch=M > 1)
+    ms, _ = timed(M)
     clocks = sampler.stop()
+    # per-launch durations of the dominant (append) kernel, second pass
+    launches = timed(M, per_launch=True)[1] if M > 1 else None
     tokens_total = B * a.tokens * a.steps * world
     value = tokens_total / (ms / 1e3)
     sb = step_bytes(op, B, H, d, M, a.tokens)
@@ -423,6 +433,7 @@ def run_gpu(a, rank, world, local_rank):
     e2e = None
     if not a.no_e2e:
         h = make_handle(M)
+        h.set_host_prefetch(True)   # host inputs are ready when each call is made
         hout = torch.empty((B, H, d), dtype=torch.bfloat16).pin_memory()
 
         def host_step():
@@ -443,10 +454,11 @@ def run_gpu(a, rank, world, local_rank):
         e_ms = max_over_ranks(start.elapsed_time(stop))
         h.close()
         h2d = sum(host[nm][0].numel() * host[nm].element_size() for nm in names) * a.tokens
-        d2h = hout.numel() * hout.element_size() * a.tokens
+        d2h = hout.numel() * hout.element_size() * a.tokens   # written by the kernel over PCIe
         e2e = {"value": B * a.tokens * a.steps * world / (e_ms / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "api": "dl_step_host (pinned host buffers, copies on the step's stream)"}
+               "api": "dl_step_host, pinned host buffers: uploads prefetched on the handle's copy "
+                      "stream, o written by the kernel into pinned host memory"}
 
     if rank != 0:
         return
@@ -457,7 +469,7 @@ def run_gpu(a, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": workload_name(a), "op": op, "B": B, "H": H, "d_k": d, "d_v": d,
                    "M": M, "state": "fp32", "inputs": "bf16", "tokens_per_step": a.tokens,
-                   "step_kernel": used_kernel[0],
+                   "step_kernel": used_kernel[0], "pdl": not a.no_pdl,
                    "input_pool_tokens": a.pool, "seed": a.seed,
                    "l2": f"inputs larger than L2 (state {4 * B * H * d * d / 1e6:.0f} MB)",
                    "parallelism": "replicas" if world == 1 else f"replicas x{world} (B per rank)"},

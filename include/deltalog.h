@@ -35,8 +35,9 @@
  * decay; every replay ratio is exp(Lam_t - Lam_i) <= 1.
  *
  * Ownership.  The caller owns every pointer it passes and the stream.  The
- * handle owns Sbar, the log and small host-staging buffers, allocated by
- * dl_create on the device current at that time and freed by dl_destroy.
+ * handle owns Sbar, the log, two small device staging sets for dl_step_host
+ * and one copy stream, created by dl_create on the device current at that
+ * time and released by dl_destroy.
  * Every call runs on that device (the caller's current device is restored).
  * All device-pointer calls are asynchronous on `stream` (a cudaStream_t, NULL
  * = legacy default stream): inputs must stay valid and outputs must not be
@@ -76,7 +77,7 @@ enum dl_status {
 /* Create a handle for B slots x H heads.  Supported: d_k, d_v in {64, 128},
  * 1 <= M <= DL_MAX_M.  The base state starts at zero with an empty log; the
  * RWKV6 bonus starts at zero.  Pointers passed later must be aligned to their
- * element size (state pointers to 16 bytes); q, k, v (and per-key
+ * element size (state pointers to 16 bytes); q, k, v, o (and per-key
  * log_decay) aligned to 16 bytes let dl_step use its streaming kernel.
  * M = 1 makes every step a merge step (the deferred path then performs the
  * eager schedule). */
@@ -102,8 +103,16 @@ int dl_step(dl_t h, const void* q, const void* k, const void* v,
             const float* log_decay, const float* beta, void* o, void* stream);
 
 /* Same as dl_step with HOST pointers (pinned or pageable): copies the inputs
- * into handle-owned device buffers, runs the step and copies o back, all on
- * `stream`.  o is valid once the stream has reached the call. */
+ * into handle-owned device buffers, runs the step and copies o back.  Inputs
+ * must stay valid, and o is valid, once `stream` has reached the call.  By
+ * default every copy is ordered on `stream`.  With DL_OPT_HOST_PREFETCH set
+ * the uploads run on the handle's own copy stream as soon as the call is made
+ * (two staging sets alternate), overlapping the previous call's step and
+ * download; the caller then promises that the host inputs are completely
+ * written when it makes the call (not produced by work still queued on
+ * `stream`).  When o is pinned host memory mapped into the device's address
+ * space (cudaHostAlloc / cudaHostRegister with UVA), the step writes it
+ * directly and no separate download is made. */
 int dl_step_host(dl_t h, const void* q, const void* k, const void* v,
                  const float* log_decay, const float* beta, void* o, void* stream);
 
@@ -125,11 +134,20 @@ int dl_read_state(dl_t h, float* S_out, void* stream);
  *   DL_STEP_AUTO (default): the fastest kernel measured for the launch
  *     (currently the register-tile kernel everywhere);
  *   DL_STEP_REGISTER: always the register-tile kernel (one CTA per slot-head);
- *   DL_STEP_STREAM: the persistent TMA-streaming kernel; needs q, k, v (and,
- *     for KDA/RWKV6, log_decay) 16-byte aligned and a shared-memory plan that
- *     fits the device, else dl_step returns DL_ERR_UNSUPPORTED.
+ *   DL_STEP_STREAM: the persistent TMA-streaming kernel; needs q, k, v, o
+ *     (and, for KDA/RWKV6, log_decay) 16-byte aligned and a shared-memory
+ *     plan that fits the device, else dl_step returns DL_ERR_UNSUPPORTED.
  * Returns DL_ERR_ARG for an unknown option or value. */
-enum dl_option { DL_OPT_STEP_KERNEL = 0 };
+/* DL_OPT_HOST_PREFETCH (0 or 1, default 0): see dl_step_host.
+ * DL_OPT_PDL (0 or 1, default 1): a register-tile step that follows an append
+ * step of the same handle is launched as a programmatic dependent of the
+ * previous kernel in the stream, so it starts streaming Sbar (which an append
+ * never writes) while that kernel drains; it reads the log and its inputs
+ * only once the previous kernel has completed.  Append steps allow their
+ * successor to launch early; merge steps, dl_eager_step and dl_merge never
+ * do.  Disable if other kernels in the stream trigger their dependents early
+ * while still writing memory that a later dl_step reads as input. */
+enum dl_option { DL_OPT_STEP_KERNEL = 0, DL_OPT_HOST_PREFETCH = 1, DL_OPT_PDL = 2 };
 enum dl_step_kernel { DL_STEP_AUTO = 0, DL_STEP_REGISTER = 1, DL_STEP_STREAM = 2 };
 int dl_set_option(dl_t h, int option, int value);
 

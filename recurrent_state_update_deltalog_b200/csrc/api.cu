@@ -23,13 +23,23 @@ struct dl_handle {
   float* logLam;
   float* u;
   int* err;
-  // device staging for dl_step_host
-  void* sq;
-  void* sk;
-  void* sv;
-  void* so;
-  float* sld;
-  float* sbeta;
+  // device staging for dl_step_host: two sets, so that with host prefetch the
+  // inputs of call t+1 upload (on copy_stream) while call t computes
+  struct Staging {
+    void* q;
+    void* k;
+    void* v;
+    void* o;
+    float* ld;
+    float* beta;
+  } st[2];
+  cudaStream_t copy_stream;
+  cudaEvent_t in_ready[2];  // recorded on copy_stream after a set's uploads
+  cudaEvent_t set_free[2];  // recorded on the caller's stream after a set's download
+  bool set_used[2];
+  int host_calls;
+  int host_prefetch;        // DL_OPT_HOST_PREFETCH
+  int pdl;                  // DL_OPT_PDL
 };
 
 namespace {
@@ -84,10 +94,19 @@ size_t state_bytes(const dl_handle* h) { return bh(h) * h->dk * h->dv * sizeof(f
 size_t decay_elems(const dl_handle* h) { return bh(h) * lam_per_entry(h); }
 
 void free_all(dl_handle* h) {
-  void* ptrs[] = {h->Sbar, h->logA, h->logB, h->logLam, h->u, h->err,
-                  h->sq, h->sk, h->sv, h->so, h->sld, h->sbeta};
+  void* ptrs[] = {h->Sbar, h->logA, h->logB, h->logLam, h->u, h->err};
   for (void* p : ptrs)
     if (p) cudaFree(p);
+  for (auto& st : h->st) {
+    void* sp[] = {st.q, st.k, st.v, st.o, st.ld, st.beta};
+    for (void* p : sp)
+      if (p) cudaFree(p);
+  }
+  for (int j = 0; j < 2; ++j) {
+    if (h->in_ready[j]) cudaEventDestroy(h->in_ready[j]);
+    if (h->set_free[j]) cudaEventDestroy(h->set_free[j]);
+  }
+  if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
 }
 
 dl::LaunchShape shape_of(const dl_handle* h, bool aligned16 = false) {
@@ -102,6 +121,8 @@ dl::LaunchShape shape_of(const dl_handle* h, bool aligned16 = false) {
   s.smem_reserved = h->smem_reserved;
   s.variant = h->step_kernel;
   s.aligned16 = aligned16;
+  // Only after an append of this handle: the previous step did not write Sbar.
+  s.pdl = h->pdl && h->n > 0;
   return s;
 }
 
@@ -141,7 +162,7 @@ dl::StepArgs step_args(dl_handle* h, const void* q, const void* k, const void* v
 
 cudaError_t launch_step(dl_handle* h, bool merge, const dl::StepArgs& a, cudaStream_t s) {
   // bulk-copy sources of the streaming kernel (GDN's scalar gate is a plain load)
-  const bool al = aligned(a.q, 16) && aligned(a.k, 16) && aligned(a.v, 16) &&
+  const bool al = aligned(a.q, 16) && aligned(a.k, 16) && aligned(a.v, 16) && aligned(a.o, 16) &&
                   (h->op == DL_GDN || aligned(a.log_decay, 16));
   const dl::LaunchShape sh = shape_of(h, al);
   int* used = &h->last_kernel;
@@ -219,6 +240,7 @@ int dl_create(dl_t* out, int B, int H, int d_k, int d_v, int M, int op, int in_d
   h->esize = in_dtype == DL_BF16 ? 2 : 4;
   h->step_kernel = DL_STEP_AUTO;
   h->last_kernel = DL_STEP_AUTO;
+  h->pdl = 1;
   if (cudaGetDevice(&h->device) != cudaSuccess) {
     delete h;
     return fail(DL_ERR_CUDA, "no current CUDA device");
@@ -250,12 +272,18 @@ int dl_create(dl_t* out, int B, int H, int d_k, int d_v, int M, int op, int in_d
       {reinterpret_cast<void**>(&h->logLam), nbh * lam_unit_floats(h) * sizeof(float)},
       {reinterpret_cast<void**>(&h->u), static_cast<size_t>(H) * d_k * sizeof(float)},
       {reinterpret_cast<void**>(&h->err), sizeof(int)},
-      {&h->sq, nbh * d_k * h->esize},
-      {&h->sk, nbh * d_k * h->esize},
-      {&h->sv, nbh * d_v * h->esize},
-      {&h->so, nbh * d_v * h->esize},
-      {reinterpret_cast<void**>(&h->sld), decay_elems(h) * sizeof(float)},
-      {reinterpret_cast<void**>(&h->sbeta), nbh * sizeof(float)},
+      {&h->st[0].q, nbh * d_k * h->esize},
+      {&h->st[0].k, nbh * d_k * h->esize},
+      {&h->st[0].v, nbh * d_v * h->esize},
+      {&h->st[0].o, nbh * d_v * h->esize},
+      {reinterpret_cast<void**>(&h->st[0].ld), decay_elems(h) * sizeof(float)},
+      {reinterpret_cast<void**>(&h->st[0].beta), nbh * sizeof(float)},
+      {&h->st[1].q, nbh * d_k * h->esize},
+      {&h->st[1].k, nbh * d_k * h->esize},
+      {&h->st[1].v, nbh * d_v * h->esize},
+      {&h->st[1].o, nbh * d_v * h->esize},
+      {reinterpret_cast<void**>(&h->st[1].ld), decay_elems(h) * sizeof(float)},
+      {reinterpret_cast<void**>(&h->st[1].beta), nbh * sizeof(float)},
   };
   for (auto& a : allocs) {
     cudaError_t e = cudaMalloc(a.p, a.bytes);
@@ -267,7 +295,12 @@ int dl_create(dl_t* out, int B, int H, int d_k, int d_v, int M, int op, int in_d
                   "cudaMalloc of %zu bytes failed: %s", a.bytes, cudaGetErrorString(e));
     }
   }
-  cudaError_t e = cudaMemset(h->Sbar, 0, state_bytes(h));
+  cudaError_t e = cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking);
+  for (int j = 0; j < 2 && e == cudaSuccess; ++j) {
+    e = cudaEventCreateWithFlags(&h->in_ready[j], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->set_free[j], cudaEventDisableTiming);
+  }
+  if (e == cudaSuccess) e = cudaMemset(h->Sbar, 0, state_bytes(h));
   if (e == cudaSuccess) e = cudaMemset(h->u, 0, static_cast<size_t>(H) * d_k * sizeof(float));
   if (e == cudaSuccess) e = cudaMemset(h->err, 0, sizeof(int));
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
@@ -328,26 +361,53 @@ int dl_step_host(dl_t h, const void* q, const void* k, const void* v, const floa
   if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t nbh = bh(h);
+  // Without prefetch the uploads are ordered on the caller's stream like any
+  // other work there; with it they run on the handle's copy stream, gated
+  // only by the reuse of their staging set, and the caller's stream waits for
+  // them before the step.
+  const int j = h->host_prefetch ? (h->host_calls & 1) : 0;
+  dl_handle::Staging& st = h->st[j];
+  cudaStream_t cs = h->host_prefetch ? h->copy_stream : s;
+  cudaError_t e = cudaSuccess;
+  if (h->host_prefetch && h->set_used[j]) e = cudaStreamWaitEvent(cs, h->set_free[j], 0);
   struct {
     void* dst;
     const void* src;
     size_t bytes;
   } in[] = {
-      {h->sq, q, nbh * h->dk * h->esize},
-      {h->sk, k, nbh * h->dk * h->esize},
-      {h->sv, v, nbh * h->dv * h->esize},
-      {h->sld, log_decay, decay_elems(h) * sizeof(float)},
-      {h->sbeta, beta, beta ? nbh * sizeof(float) : 0},
+      {st.q, q, nbh * h->dk * h->esize},
+      {st.k, k, nbh * h->dk * h->esize},
+      {st.v, v, nbh * h->dv * h->esize},
+      {st.ld, log_decay, decay_elems(h) * sizeof(float)},
+      {st.beta, beta, beta ? nbh * sizeof(float) : 0},
   };
   for (auto& c : in) {
-    if (!c.bytes) continue;
-    cudaError_t e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, s);
-    if (e != cudaSuccess) return cuda_fail(e, "dl_step_host input copy");
+    if (e != cudaSuccess) break;
+    if (c.bytes) e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, cs);
   }
-  rc = do_step(h, h->sq, h->sk, h->sv, h->sld, beta ? h->sbeta : nullptr, h->so, s);
+  if (e == cudaSuccess && h->host_prefetch) {
+    e = cudaEventRecord(h->in_ready[j], cs);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, h->in_ready[j], 0);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "dl_step_host input upload");
+  // A pinned, device-mapped output buffer is written by the kernel itself
+  // (its stores cross PCIe while the step streams the state); anything else
+  // goes through the staging set and one download.
+  void* o_dev = nullptr;
+  cudaPointerAttributes pa;
+  if (cudaPointerGetAttributes(&pa, o) == cudaSuccess && pa.type == cudaMemoryTypeHost && pa.devicePointer &&
+      aligned(pa.devicePointer, 16))
+    o_dev = pa.devicePointer;
+  else
+    cudaGetLastError();  // pageable memory reports an error on some drivers
+  rc = do_step(h, st.q, st.k, st.v, st.ld, beta ? st.beta : nullptr, o_dev ? o_dev : st.o, s);
   if (rc != DL_OK) return rc;
-  cudaError_t e = cudaMemcpyAsync(o, h->so, nbh * h->dv * h->esize, cudaMemcpyDeviceToHost, s);
-  return e == cudaSuccess ? DL_OK : cuda_fail(e, "dl_step_host output copy");
+  if (!o_dev) e = cudaMemcpyAsync(o, st.o, nbh * h->dv * h->esize, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && h->host_prefetch) e = cudaEventRecord(h->set_free[j], s);
+  if (e != cudaSuccess) return cuda_fail(e, "dl_step_host output download");
+  h->set_used[j] = true;
+  ++h->host_calls;
+  return DL_OK;
 }
 
 int dl_eager_step(dl_t h, const void* q, const void* k, const void* v, const float* log_decay,
@@ -385,10 +445,22 @@ int dl_read_state(dl_t h, float* S_out, void* stream) {
 
 int dl_set_option(dl_t h, int option, int value) {
   if (!h) return fail(DL_ERR_ARG, "null handle");
-  if (option != DL_OPT_STEP_KERNEL) return fail(DL_ERR_ARG, "unknown option %d", option);
-  if (value < DL_STEP_AUTO || value > DL_STEP_STREAM) return fail(DL_ERR_ARG, "bad step-kernel value %d", value);
-  h->step_kernel = value;
-  return DL_OK;
+  switch (option) {
+    case DL_OPT_STEP_KERNEL:
+      if (value < DL_STEP_AUTO || value > DL_STEP_STREAM) return fail(DL_ERR_ARG, "bad step-kernel value %d", value);
+      h->step_kernel = value;
+      return DL_OK;
+    case DL_OPT_HOST_PREFETCH:
+      if (value != 0 && value != 1) return fail(DL_ERR_ARG, "bad host-prefetch value %d", value);
+      h->host_prefetch = value;
+      return DL_OK;
+    case DL_OPT_PDL:
+      if (value != 0 && value != 1) return fail(DL_ERR_ARG, "bad PDL value %d", value);
+      h->pdl = value;
+      return DL_OK;
+    default:
+      return fail(DL_ERR_ARG, "unknown option %d", option);
+  }
 }
 
 int dl_last_step_kernel(dl_t h, int* kind) {

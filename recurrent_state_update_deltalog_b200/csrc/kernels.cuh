@@ -224,12 +224,18 @@ deltalog_step_kernel(const StepArgs a) {
   float* As = reinterpret_cast<float*>(s_dyn + LL::staged(n));      // merge only
   float* Bc = As + (n + 1) * DK;                                      // merge only
 
-  // 1. Stream this head's Sbar tile into registers (all loads in flight), and
-  // let one thread start the TMA bulk copies of the log into shared memory.
+  // 1. Stream this head's Sbar tile into registers (all loads in flight).  The
+  // state is never written by the preceding kernel when this one is launched
+  // as a programmatic dependent (the host only does so after an append step),
+  // so these loads may overlap that kernel's tail; everything it may have
+  // written (log, inputs) is read after griddep_wait.  An append lets the next
+  // step launch early; a merge, which writes Sbar, does not.
   float* Sp = a.Sbar + sh * (DK * DV);
   float4 st[TL::RPT];
 #pragma unroll
   for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + (rg * TL::RPT + j) * DV + 4 * c4);
+  if (!MERGE) griddep_launch_dependents();
+  griddep_wait();
   if (tid == 0) stage_log<OP, DK, DV, TI>(s_dyn, &s_bar, a.logA, a.logLam, a.logB, sh, a.Mcap, n);
 
   // 2. Key-side values for this lane's keys j = lane + 32 m; GDN's scalar

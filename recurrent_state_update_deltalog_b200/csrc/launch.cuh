@@ -22,8 +22,26 @@ struct LaunchShape {
   int smem_sm;
   int smem_reserved;
   int variant;     // STEP_*
-  bool aligned16;  // q, k, v, log_decay all 16-byte aligned (bulk-copy sources)
+  bool aligned16;  // q, k, v, o (and per-key log_decay) 16-byte aligned (bulk-copy sources)
+  bool pdl;        // launch the step as a programmatic dependent of the previous kernel
 };
+
+// Launch with the programmatic-stream-serialisation attribute when `pdl`.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_maybe_pdl(void (*kern)(KArgs...), int grid, int block, size_t smem, cudaStream_t st, bool pdl,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
 
 // Ring/slot plan of the streaming kernel for one launch.
 struct StreamPlan {
@@ -68,9 +86,12 @@ cudaError_t stream_dims(const LaunchShape& s, const StepArgs& a, cudaStream_t st
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              s.smem_block_optin - static_cast<int>(fa.sharedSizeBytes));
     if (e != cudaSuccess) return e;
+    // the whole unified L1/shared array as shared memory, so the planned CTAs fit
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
   }
   const int grid = s.BH < p.ctas_per_sm * s.sms ? s.BH : p.ctas_per_sm * s.sms;
-  kern<<<grid, Tile<DK, DV>::NT, p.smem, st>>>(a, StreamCfg{s.BH, p.ns});
+  kern<<<grid, StreamGeom<OP, DK, DV, TI>::NT, p.smem, st>>>(a, StreamCfg{s.BH, p.ns});
   *launched = true;
   return cudaGetLastError();
 }
@@ -108,14 +129,12 @@ cudaError_t step_dims(const LaunchShape& s, bool merge, const StepArgs& a, cudaS
     auto kern = deltalog_step_kernel<OP, DK, DV, TI, true>;
     cudaError_t e = allow_smem(kern, smem, LL::step_smem(kMaxM - 1, true));
     if (e != cudaSuccess) return e;
-    kern<<<s.BH, TL::NT, smem, st>>>(a);
-  } else {
-    auto kern = deltalog_step_kernel<OP, DK, DV, TI, false>;
-    cudaError_t e = allow_smem(kern, smem, LL::step_smem(kMaxM - 1, false));
-    if (e != cudaSuccess) return e;
-    kern<<<s.BH, TL::NT, smem, st>>>(a);
+    return launch_maybe_pdl(kern, s.BH, TL::NT, smem, st, s.pdl, a);
   }
-  return cudaGetLastError();
+  auto kern = deltalog_step_kernel<OP, DK, DV, TI, false>;
+  cudaError_t e = allow_smem(kern, smem, LL::step_smem(kMaxM - 1, false));
+  if (e != cudaSuccess) return e;
+  return launch_maybe_pdl(kern, s.BH, TL::NT, smem, st, s.pdl, a);
 }
 
 template <int OP, int DK, int DV, typename TI>

@@ -131,6 +131,15 @@ class DeltaLog:
         vals = {"auto": N.DL_STEP_AUTO, "register": N.DL_STEP_REGISTER, "stream": N.DL_STEP_STREAM}
         N.call("dl_set_option", self._h, N.DL_OPT_STEP_KERNEL, vals[kind])
 
+    def set_host_prefetch(self, on):
+        """Let step_host upload inputs on the handle's copy stream ahead of the
+        caller's stream (the host inputs must be ready when step_host is called)."""
+        N.call("dl_set_option", self._h, N.DL_OPT_HOST_PREFETCH, 1 if on else 0)
+
+    def set_pdl(self, on):
+        """Programmatic dependent launch of steps that follow an append (default on)."""
+        N.call("dl_set_option", self._h, N.DL_OPT_PDL, 1 if on else 0)
+
     @property
     def last_step_kernel(self):
         """Kernel used by the most recent step: ``"register"``, ``"stream"`` or ``None``."""
