@@ -147,7 +147,17 @@ int dl_read_state(dl_t h, float* S_out, void* stream);
  * successor to launch early; merge steps, dl_eager_step and dl_merge never
  * do.  Disable if other kernels in the stream trigger their dependents early
  * while still writing memory that a later dl_step reads as input. */
-enum dl_option { DL_OPT_STEP_KERNEL = 0, DL_OPT_HOST_PREFETCH = 1, DL_OPT_PDL = 2 };
+/* DL_OPT_VALUE_TILES (0 = automatic, 1, 2 or 4): value tiles per head of the
+ * register-tile step kernel, i.e. how many CTAs split a head's d_v columns
+ * (a split below 32 columns per tile falls back to fewer tiles; each tile
+ * recomputes the head's key-side coefficients).  Automatic: 2 for d_v = 128
+ * while the log holds fewer than 16 entries, else 1. */
+enum dl_option {
+  DL_OPT_STEP_KERNEL = 0,
+  DL_OPT_HOST_PREFETCH = 1,
+  DL_OPT_PDL = 2,
+  DL_OPT_VALUE_TILES = 3
+};
 enum dl_step_kernel { DL_STEP_AUTO = 0, DL_STEP_REGISTER = 1, DL_STEP_STREAM = 2 };
 int dl_set_option(dl_t h, int option, int value);
 

@@ -40,6 +40,7 @@ struct dl_handle {
   int host_calls;
   int host_prefetch;        // DL_OPT_HOST_PREFETCH
   int pdl;                  // DL_OPT_PDL
+  int value_tiles;          // DL_OPT_VALUE_TILES (0 = automatic)
 };
 
 namespace {
@@ -123,6 +124,13 @@ dl::LaunchShape shape_of(const dl_handle* h, bool aligned16 = false) {
   s.aligned16 = aligned16;
   // Only after an append of this handle: the previous step did not write Sbar.
   s.pdl = h->pdl && h->n > 0;
+  if (h->value_tiles == 0) {
+    // measured on B200: two 64-column tiles per head win for d_v = 128 while
+    // the log is short (each tile recomputes the key-side coefficients)
+    s.split = h->dv == 128 && h->n < 16 ? 2 : 1;
+  } else {
+    s.split = h->dv / h->value_tiles >= 32 ? h->value_tiles : 1;
+  }
   return s;
 }
 
@@ -457,6 +465,11 @@ int dl_set_option(dl_t h, int option, int value) {
     case DL_OPT_PDL:
       if (value != 0 && value != 1) return fail(DL_ERR_ARG, "bad PDL value %d", value);
       h->pdl = value;
+      return DL_OK;
+    case DL_OPT_VALUE_TILES:
+      if (value != 0 && value != 1 && value != 2 && value != 4)
+        return fail(DL_ERR_ARG, "bad value-tile count %d", value);
+      h->value_tiles = value;
       return DL_OK;
     default:
       return fail(DL_ERR_ARG, "unknown option %d", option);

@@ -95,12 +95,25 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
+// acc += a * b on a float4, as two packed fp32x2 FMAs (sm_100 FFMA2; each
+// lane rounds exactly like fmaf).
 __device__ __forceinline__ void fma4(float4& acc, float a, float4 b) {
-  acc.x = fmaf(a, b.x, acc.x);
-  acc.y = fmaf(a, b.y, acc.y);
-  acc.z = fmaf(a, b.z, acc.z);
-  acc.w = fmaf(a, b.w, acc.w);
+  const float2 aa = make_float2(a, a);
+  const float2 lo = __ffma2_rn(aa, make_float2(b.x, b.y), make_float2(acc.x, acc.y));
+  const float2 hi = __ffma2_rn(aa, make_float2(b.z, b.w), make_float2(acc.z, acc.w));
+  acc = make_float4(lo.x, lo.y, hi.x, hi.y);
 }
+
+// v *= d on a float4 (two packed fp32x2 multiplies).
+__device__ __forceinline__ void scale4(float4& v, float d) {
+  const float2 dd = make_float2(d, d);
+  const float2 lo = __fmul2_rn(dd, make_float2(v.x, v.y));
+  const float2 hi = __fmul2_rn(dd, make_float2(v.z, v.w));
+  v = make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
+// Largest supported merge interval M (log capacity M-1).
+constexpr int kMaxM = 64;
 
 template <int DK, int DV>
 struct Tile {
@@ -110,13 +123,11 @@ struct Tile {
   static constexpr int RPT = DK / RG;    // rows held by each thread
   static constexpr int NW = NT / 32;     // warps
   static constexpr int KPL = DK / 32;    // keys per lane in warp-wide key loops
-  static constexpr int MINB = NT >= 256 ? 2 : 4;
-  static_assert(DV % 64 == 0 && DK % 32 == 0 && RG == 8 && RPT % 4 == 0, "tile shape");
-  static_assert(DK <= NT && DV <= NT, "one thread per key / value in setup phases");
+  static constexpr int MINB = NT >= 256 ? 2 : (NT >= 128 ? 4 : 8);
+  static_assert(DV % 32 == 0 && DK % 32 == 0 && RG == 8 && RPT % 4 == 0, "tile shape");
+  static_assert(NT >= kMaxM - 1 && DV <= NT, "one thread per log entry / value column in setup phases");
 };
 
-// Largest supported merge interval M (log capacity M-1).
-constexpr int kMaxM = 64;
 
 // GDN keeps one scalar snapshot per entry; each head's row of snapshots is
 // padded to a multiple of 4 floats so that it can be staged by a bulk copy.
@@ -190,12 +201,16 @@ __device__ __forceinline__ bool wait_log(uint64_t* bar, int n, int* err) {
 
 // ---------------------------------------------------------------------------
 // Deferred step.  MERGE=false: append (Sbar read only).  MERGE=true: the step
-// with n+1 == M; it also writes S_t over Sbar.
+// with n+1 == M; it also writes S_t over Sbar.  NSPLIT > 1 splits each head's
+// d_v columns into NSPLIT value tiles, one CTA each (grid B*H*NSPLIT); every
+// tile recomputes the head's ReplayPrep coefficients and the first tile
+// appends the key-side entry.
 // ---------------------------------------------------------------------------
-template <int OP, int DK, int DV, typename TI, bool MERGE>
-__global__ void __launch_bounds__(Tile<DK, DV>::NT, Tile<DK, DV>::MINB)
+template <int OP, int DK, int DV, typename TI, bool MERGE, int NSPLIT>
+__global__ void __launch_bounds__(Tile<DK, DV / NSPLIT>::NT, Tile<DK, DV / NSPLIT>::MINB)
 deltalog_step_kernel(const StepArgs a) {
-  using TL = Tile<DK, DV>;
+  constexpr int DVT = DV / NSPLIT;  // value-tile width owned by this CTA
+  using TL = Tile<DK, DVT>;
   using LL = LogLayout<OP, DK, DV, TI>;
   using TB = typename LL::TB;
   constexpr bool DELTA = OP != OP_RWKV6;
@@ -204,7 +219,7 @@ deltalog_step_kernel(const StepArgs a) {
   __shared__ __align__(16) float s_kt[DK];       // k~ = e^{Lam_t} (.) k   (GDN/KDA)
   __shared__ __align__(16) float s_qt[DK];       // q~ (GDN/KDA: e^{Lam_t}; RWKV6: e^{Lam_{t-1}})
   __shared__ __align__(16) float s_dec[DK];      // e^{Lam_t} per row (merge)
-  __shared__ __align__(16) float s_red[2][TL::RG][DV];
+  __shared__ __align__(16) float s_red[2][TL::RG][DVT];
   __shared__ float s_ck[kMaxM], s_cq[kMaxM];
   __shared__ float s_lam[kMaxM];                 // GDN: scalar Lam_i of the log entries
   __shared__ float s_kappa;
@@ -214,7 +229,8 @@ deltalog_step_kernel(const StepArgs a) {
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const int c4 = tid % TL::TPR, rg = tid / TL::TPR;
-  const long sh = blockIdx.x;
+  const long sh = blockIdx.x / NSPLIT;
+  const int col0 = (blockIdx.x % NSPLIT) * DVT;  // first value column of this tile
   const int h = static_cast<int>(sh % a.H);
   const int n = a.n;
 
@@ -233,7 +249,7 @@ deltalog_step_kernel(const StepArgs a) {
   float* Sp = a.Sbar + sh * (DK * DV);
   float4 st[TL::RPT];
 #pragma unroll
-  for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + (rg * TL::RPT + j) * DV + 4 * c4);
+  for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + (rg * TL::RPT + j) * DV + col0 + 4 * c4);
   if (!MERGE) griddep_launch_dependents();
   griddep_wait();
   if (tid == 0) stage_log<OP, DK, DV, TI>(s_dyn, &s_bar, a.logA, a.logLam, a.logB, sh, a.Mcap, n);
@@ -268,8 +284,8 @@ deltalog_step_kernel(const StepArgs a) {
   }
   const int c = tid;
   float vc = 0.f, betac = 0.f;
-  if (c < DV) {
-    vc = to_f(static_cast<const TI*>(a.v)[sh * DV + c]);
+  if (c < DVT) {
+    vc = to_f(static_cast<const TI*>(a.v)[sh * DV + col0 + c]);
     if (DELTA) betac = a.beta[sh];
   }
   __syncthreads();                              // barrier init and s_lam visible
@@ -331,7 +347,7 @@ deltalog_step_kernel(const StepArgs a) {
       }
       if (MERGE) s_dec[j] = et;
     }
-    if (!MERGE) {  // append: a_n = k_t and its log-decay snapshot
+    if (!MERGE && col0 == 0) {  // append (first value tile): a_n = k_t and its snapshot
       TI* dstA = static_cast<TI*>(a.logA) + (sh * a.Mcap + n) * DK;
 #pragma unroll
       for (int m = 0; m < TL::KPL; ++m) {
@@ -359,7 +375,7 @@ deltalog_step_kernel(const StepArgs a) {
   __syncthreads();
 
   // 5. AppendDecode finalize for value column c: replay, delta correction, output.
-  if (c < DV) {
+  if (c < DVT) {
     float p = 0.f, s = 0.f;
 #pragma unroll
     for (int g = 0; g < TL::RG; ++g) {
@@ -368,7 +384,7 @@ deltalog_step_kernel(const StepArgs a) {
     }
     float oc = s, bt;
     for (int i = 0; i < n; ++i) {
-      const float bi = to_f(sB[i * DV + c]);
+      const float bi = to_f(sB[i * DV + col0 + c]);
       if (DELTA) p = fmaf(s_ck[i], bi, p);
       oc = fmaf(s_cq[i], bi, oc);
     }
@@ -378,15 +394,15 @@ deltalog_step_kernel(const StepArgs a) {
       bt = vc;
     }
     oc = fmaf(s_kappa, bt, oc);
-    static_cast<TI*>(a.o)[sh * DV + c] = from_f<TI>(oc);
+    static_cast<TI*>(a.o)[sh * DV + col0 + c] = from_f<TI>(oc);
     if (MERGE) {
       Bc[c] = bt;
     } else {
-      TB* dstB = static_cast<TB*>(a.logB) + (sh * a.Mcap + n) * DV;
+      TB* dstB = static_cast<TB*>(a.logB) + (sh * a.Mcap + n) * DV + col0;
       if constexpr (DELTA) {
         dstB[c] = bt;
       } else {
-        dstB[c] = static_cast<const TI*>(a.v)[sh * DV + c];   // raw v, bit copy
+        dstB[c] = static_cast<const TI*>(a.v)[sh * DV + col0 + c];   // raw v, bit copy
       }
     }
   }
@@ -396,14 +412,10 @@ deltalog_step_kernel(const StepArgs a) {
     __syncthreads();
 #pragma unroll
     for (int j = 0; j < TL::RPT; ++j) {
-      const float d = s_dec[rg * TL::RPT + j];
-      st[j].x *= d;
-      st[j].y *= d;
-      st[j].z *= d;
-      st[j].w *= d;
+      scale4(st[j], s_dec[rg * TL::RPT + j]);
     }
     for (int i = 0; i <= n; ++i) {
-      const float4 b4 = i < n ? load4f(sB + i * DV + 4 * c4) : load4f(Bc + 4 * c4);
+      const float4 b4 = i < n ? load4f(sB + i * DV + col0 + 4 * c4) : load4f(Bc + 4 * c4);
       const float* ai = &As[i * DK + rg * TL::RPT];
 #pragma unroll
       for (int j4 = 0; j4 < TL::RPT; j4 += 4) {
@@ -415,7 +427,7 @@ deltalog_step_kernel(const StepArgs a) {
       }
     }
 #pragma unroll
-    for (int j = 0; j < TL::RPT; ++j) st_state(Sp + (rg * TL::RPT + j) * DV + 4 * c4, st[j]);
+    for (int j = 0; j < TL::RPT; ++j) st_state(Sp + (rg * TL::RPT + j) * DV + col0 + 4 * c4, st[j]);
   }
 }
 
@@ -524,12 +536,8 @@ eager_step_kernel(const StepArgs a) {
 #pragma unroll
   for (int j = 0; j < TL::RPT; ++j) {
     const int row = rg * TL::RPT + j;
-    const float d = s_dec[row];
     float4 x = st[j];
-    x.x *= d;
-    x.y *= d;
-    x.z *= d;
-    x.w *= d;
+    scale4(x, s_dec[row]);
     fma4(x, s_k[row], b4);
     st_state(Sp + row * DV + 4 * c4, x);
   }
@@ -595,11 +603,7 @@ materialize_kernel(const MaterializeArgs a) {
 
 #pragma unroll
   for (int j = 0; j < TL::RPT; ++j) {
-    const float d = s_dec[rg * TL::RPT + j];
-    st[j].x *= d;
-    st[j].y *= d;
-    st[j].z *= d;
-    st[j].w *= d;
+    scale4(st[j], s_dec[rg * TL::RPT + j]);
   }
   for (int i = 0; i < n; ++i) {
     const float4 b4 = load4f(sB + i * DV + 4 * c4);

@@ -24,6 +24,7 @@ struct LaunchShape {
   int variant;     // STEP_*
   bool aligned16;  // q, k, v, o (and per-key log_decay) 16-byte aligned (bulk-copy sources)
   bool pdl;        // launch the step as a programmatic dependent of the previous kernel
+  int split;       // value tiles per head for the register-tile step kernel (1, 2 or 4)
 };
 
 // Launch with the programmatic-stream-serialisation attribute when `pdl`.
@@ -109,12 +110,28 @@ cudaError_t allow_smem(K kern, size_t smem, size_t worst) {
   return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(worst));
 }
 
+template <int OP, int DK, int DV, typename TI, int NSPLIT>
+cudaError_t register_step(const LaunchShape& s, bool merge, const StepArgs& a, cudaStream_t st) {
+  using TL = Tile<DK, DV / NSPLIT>;
+  using LL = LogLayout<OP, DK, DV, TI>;
+  const size_t smem = LL::step_smem(a.n, merge);
+  const int grid = s.BH * NSPLIT;
+  if (merge) {
+    auto kern = deltalog_step_kernel<OP, DK, DV, TI, true, NSPLIT>;
+    cudaError_t e = allow_smem(kern, smem, LL::step_smem(kMaxM - 1, true));
+    if (e != cudaSuccess) return e;
+    return launch_maybe_pdl(kern, grid, TL::NT, smem, st, s.pdl, a);
+  }
+  auto kern = deltalog_step_kernel<OP, DK, DV, TI, false, NSPLIT>;
+  cudaError_t e = allow_smem(kern, smem, LL::step_smem(kMaxM - 1, false));
+  if (e != cudaSuccess) return e;
+  return launch_maybe_pdl(kern, grid, TL::NT, smem, st, s.pdl, a);
+}
+
 template <int OP, int DK, int DV, typename TI>
 cudaError_t step_dims(const LaunchShape& s, bool merge, const StepArgs& a, cudaStream_t st, int* used) {
-  using TL = Tile<DK, DV>;
-  using LL = LogLayout<OP, DK, DV, TI>;
-  // AUTO runs the register-tile kernel: it is the faster of the two on B200
-  // (GDN B=256 H=32 d=128: 92 vs 101 us per append launch); STREAM is opt-in.
+  // AUTO runs the register-tile kernel, the faster of the two on B200 for
+  // every operator's merge launches and for d_v = 64; STREAM is opt-in.
   if (s.variant == STEP_STREAM && s.aligned16) {
     bool launched = false;
     cudaError_t e = merge ? stream_dims<OP, DK, DV, TI, true>(s, a, st, &launched)
@@ -124,17 +141,13 @@ cudaError_t step_dims(const LaunchShape& s, bool merge, const StepArgs& a, cudaS
   }
   if (s.variant == STEP_STREAM) return cudaErrorNotSupported;
   *used = STEP_REGISTER;
-  const size_t smem = LL::step_smem(a.n, merge);
-  if (merge) {
-    auto kern = deltalog_step_kernel<OP, DK, DV, TI, true>;
-    cudaError_t e = allow_smem(kern, smem, LL::step_smem(kMaxM - 1, true));
-    if (e != cudaSuccess) return e;
-    return launch_maybe_pdl(kern, s.BH, TL::NT, smem, st, s.pdl, a);
+  if constexpr (DV >= 128) {
+    if (s.split == 4) return register_step<OP, DK, DV, TI, 4>(s, merge, a, st);
   }
-  auto kern = deltalog_step_kernel<OP, DK, DV, TI, false>;
-  cudaError_t e = allow_smem(kern, smem, LL::step_smem(kMaxM - 1, false));
-  if (e != cudaSuccess) return e;
-  return launch_maybe_pdl(kern, s.BH, TL::NT, smem, st, s.pdl, a);
+  if constexpr (DV >= 64) {
+    if (s.split == 2) return register_step<OP, DK, DV, TI, 2>(s, merge, a, st);
+  }
+  return register_step<OP, DK, DV, TI, 1>(s, merge, a, st);
 }
 
 template <int OP, int DK, int DV, typename TI>

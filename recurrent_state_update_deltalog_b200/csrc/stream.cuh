@@ -413,12 +413,8 @@ deltalog_stream_kernel(const StepArgs a, const StreamCfg cfg) {
           float4 x[RPC];
 #pragma unroll
           for (int j = 0; j < RPC; ++j) {
-            const float d = dec_w[ri0 + j];
             x[j] = *reinterpret_cast<const float4*>(ch + (rg * RPC + j) * DV + 4 * c4);
-            x[j].x *= d;
-            x[j].y *= d;
-            x[j].z *= d;
-            x[j].w *= d;
+            scale4(x[j], dec_w[ri0 + j]);
           }
           for (int i = 0; i <= n; ++i) {
             const float4 b4 = i < n ? load4f(sB + i * DV + 4 * c4) : bt;

@@ -140,6 +140,10 @@ class DeltaLog:
         """Programmatic dependent launch of steps that follow an append (default on)."""
         N.call("dl_set_option", self._h, N.DL_OPT_PDL, 1 if on else 0)
 
+    def set_value_tiles(self, n):
+        """0 (automatic), 1 or 2 value tiles (CTAs) per head in the register-tile step kernel."""
+        N.call("dl_set_option", self._h, N.DL_OPT_VALUE_TILES, int(n))
+
     @property
     def last_step_kernel(self):
         """Kernel used by the most recent step: ``"register"``, ``"stream"`` or ``None``."""

@@ -17,11 +17,11 @@ OPS = ["gdn", "kda", "rwkv6"]
 KERNELS = ["register", "stream"]
 
 
-def _check_run(op, B, H, dk, dv, M, T, dtype, eager=False, seed=0, kernel="auto"):
+def _check_run(op, B, H, dk, dv, M, T, dtype, eager=False, seed=0, kernel="auto", tiles=0):
     S0, seq, u = make_inputs(op, B, H, dk, dv, T, dtype, seed)
     merge_steps = [t for t in range(T) if (t + 1) % M == 0] if not eager else []
     o_ref, S_ref, kept = run_oracle(op, S0, seq, u, record=set(merge_steps))
-    o, merges, final = run_gpu(op, S0, seq, u, M, dtype, eager=eager, kernel=kernel)
+    o, merges, final = run_gpu(op, S0, seq, u, M, dtype, eager=eager, kernel=kernel, tiles=tiles)
     tol = TOL[dtype]
     e_o = relerr(o, o_ref)
     assert e_o < tol, f"outputs: {e_o:.3e}"
@@ -80,6 +80,23 @@ def test_step_kernel_selection_is_reported():
     h.step(*step_args("gdn", dseq, 2))
     assert h.last_step_kernel == "register"
     h.close()
+
+
+@pytest.mark.parametrize("tiles", [1, 2, 4])
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("dims", [(64, 64), (128, 128), (64, 128), (128, 64)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_value_tiles(op, dims, dtype, tiles):
+    """Register-tile kernel with each head's d_v columns split over 1, 2 or 4
+    CTAs (a split that would leave fewer than 32 columns falls back to fewer)."""
+    _check_run(op, 3, 5, dims[0], dims[1], 4, 11, dtype, kernel="register", tiles=tiles)
+
+
+@pytest.mark.parametrize("tiles", [2, 4])
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("M", [2, 8, 33, 64])
+def test_value_tiles_every_M(op, M, tiles):
+    _check_run(op, 2, 3, 128, 128, M, min(2 * M + 3, 70), torch.bfloat16, kernel="register", tiles=tiles)
 
 
 @pytest.mark.parametrize("op", OPS)
