@@ -432,37 +432,40 @@ deltalog_step_kernel(const StepArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Eager dense baseline: S_{t-1} -> S_t read and written every token.
+// Eager dense baseline: S_{t-1} -> S_t read and written every token.  Same
+// tile mapping (and value-tile split) as the deferred step.
 // ---------------------------------------------------------------------------
-template <int OP, int DK, int DV, typename TI>
-__global__ void __launch_bounds__(Tile<DK, DV>::NT, Tile<DK, DV>::MINB)
+template <int OP, int DK, int DV, typename TI, int NSPLIT>
+__global__ void __launch_bounds__(Tile<DK, DV / NSPLIT>::NT, Tile<DK, DV / NSPLIT>::MINB)
 eager_step_kernel(const StepArgs a) {
-  using TL = Tile<DK, DV>;
+  constexpr int DVT = DV / NSPLIT;  // value-tile width owned by this CTA
+  using TL = Tile<DK, DVT>;
   constexpr bool DELTA = OP != OP_RWKV6;
 
   __shared__ __align__(16) float s_kx[DK];   // contraction vector for p
   __shared__ __align__(16) float s_qx[DK];   // contraction vector for s
   __shared__ __align__(16) float s_dec[DK];  // per-row decay of S_{t-1}
   __shared__ __align__(16) float s_k[DK];    // k_t (rank-1 update rows)
-  __shared__ __align__(16) float s_b[DV];    // b_t (rank-1 update columns)
-  __shared__ __align__(16) float s_red[2][TL::RG][DV];
+  __shared__ __align__(16) float s_b[DVT];   // b_t (rank-1 update columns)
+  __shared__ __align__(16) float s_red[2][TL::RG][DVT];
   __shared__ float s_kappa;
 
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const int c4 = tid % TL::TPR, rg = tid / TL::TPR;
-  const long sh = blockIdx.x;
+  const long sh = blockIdx.x / NSPLIT;
+  const int col0 = (blockIdx.x % NSPLIT) * DVT;
   const int h = static_cast<int>(sh % a.H);
 
   float* Sp = a.Sbar + sh * (DK * DV);
   float4 st[TL::RPT];
 #pragma unroll
-  for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + (rg * TL::RPT + j) * DV + 4 * c4);
+  for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + (rg * TL::RPT + j) * DV + col0 + 4 * c4);
 
   const int c = tid;
   float vc = 0.f, betac = 0.f;
-  if (c < DV) {
-    vc = to_f(static_cast<const TI*>(a.v)[sh * DV + c]);
+  if (c < DVT) {
+    vc = to_f(static_cast<const TI*>(a.v)[sh * DV + col0 + c]);
     if (DELTA) betac = a.beta[sh];
   }
 
@@ -508,7 +511,7 @@ eager_step_kernel(const StepArgs a) {
   }
   __syncthreads();
 
-  if (c < DV) {
+  if (c < DVT) {
     float p = 0.f, s = 0.f;
 #pragma unroll
     for (int g = 0; g < TL::RG; ++g) {
@@ -528,7 +531,7 @@ eager_step_kernel(const StepArgs a) {
       oc = fmaf(s_kappa, vc, s);
     }
     s_b[c] = bt;
-    static_cast<TI*>(a.o)[sh * DV + c] = from_f<TI>(oc);
+    static_cast<TI*>(a.o)[sh * DV + col0 + c] = from_f<TI>(oc);
   }
   __syncthreads();
 
@@ -539,7 +542,7 @@ eager_step_kernel(const StepArgs a) {
     float4 x = st[j];
     scale4(x, s_dec[row]);
     fma4(x, s_k[row], b4);
-    st_state(Sp + row * DV + 4 * c4, x);
+    st_state(Sp + row * DV + col0 + 4 * c4, x);
   }
 }
 

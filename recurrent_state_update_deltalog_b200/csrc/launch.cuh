@@ -152,7 +152,13 @@ cudaError_t step_dims(const LaunchShape& s, bool merge, const StepArgs& a, cudaS
 
 template <int OP, int DK, int DV, typename TI>
 cudaError_t eager_dims(const LaunchShape& s, const StepArgs& a, cudaStream_t st) {
-  eager_step_kernel<OP, DK, DV, TI><<<s.BH, Tile<DK, DV>::NT, 0, st>>>(a);
+  if constexpr (DV >= 64) {
+    if (s.split == 2) {
+      eager_step_kernel<OP, DK, DV, TI, 2><<<s.BH * 2, Tile<DK, DV / 2>::NT, 0, st>>>(a);
+      return cudaGetLastError();
+    }
+  }
+  eager_step_kernel<OP, DK, DV, TI, 1><<<s.BH, Tile<DK, DV>::NT, 0, st>>>(a);
   return cudaGetLastError();
 }
 
