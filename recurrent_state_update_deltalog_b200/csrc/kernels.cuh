@@ -123,7 +123,10 @@ struct Tile {
   static constexpr int RPT = DK / RG;    // rows held by each thread
   static constexpr int NW = NT / 32;     // warps
   static constexpr int KPL = DK / 32;    // keys per lane in warp-wide key loops
-  static constexpr int MINB = NT >= 256 ? 2 : (NT >= 128 ? 4 : 8);
+  // CTAs per SM the register budget is sized for: d_k = 64 tiles keep only
+  // 32 state registers per thread, so eight 128-thread CTAs (64 registers
+  // each) fit and keep 128 KB of state loads in flight per SM.
+  static constexpr int MINB = NT >= 256 ? 2 : (NT >= 128 ? (DK == 64 ? 8 : 4) : 8);
   static_assert(DV % 32 == 0 && DK % 32 == 0 && RG == 8 && RPT % 4 == 0, "tile shape");
   static_assert(NT >= kMaxM - 1 && DV <= NT, "one thread per log entry / value column in setup phases");
 };
