@@ -55,7 +55,14 @@ def parse():
                     help="dl_step kernel variant")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch every step with plain stream ordering")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay each M-token cycle from a CUDA graph instead of launching from Python")
+    ap.add_argument("--grid", default="",
+                    help="B x M sweep, e.g. '1,16,64,256,1024x1,2,4,8,16,32': one JSON line per "
+                         "point (CUDA graphs; M=1 is the eager kernel)")
     args = ap.parse_args()
+    if args.grid:
+        return args
     if args.tokens % args.M:
         ap.error("--tokens must be a multiple of --M")
     return args
@@ -346,11 +353,53 @@ def run_gpu(a, rank, world, local_rank):
             else:
                 h.step(*args, out=out[i], stream=stream)
 
+    def build_graphs(h, m, eager):
+        """One CUDA graph per m-token cycle of the input pool (8 tokens for the
+        eager kernel); the log is empty at every cycle boundary, so each graph
+        replays a complete append...merge cycle."""
+        cyc = 8 if eager else m
+        gs = torch.cuda.Stream(dev)
+        graphs = []
+        with torch.cuda.stream(gs):
+            for c in range(max(1, a.pool // cyc)):
+                gr = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gr, stream=gs):
+                    for j in range(cyc):
+                        i = (c * cyc + j) % a.pool
+                        fn = h.eager_step if eager else h.step
+                        fn(*tok_args(dpool, i), out=out[i], stream=gs)
+                graphs.append(gr)
+        torch.cuda.synchronize(dev)
+        return graphs, cyc
+
+    def run_graph_step(graphs, cyc):
+        for _ in range(a.tokens // cyc):
+            graphs[tok_counter[0] % len(graphs)].replay()
+            tok_counter[0] += 1
+
     def timed(m, eager=False, per_launch=False):
         """Time a.steps bench steps (or, with per_launch, a shorter second pass in
         which every append launch is bracketed by its own pair of events: those
         events sit between launches, so each launch is timed in isolation)."""
         h = make_handle(m)
+        if a.graph and not per_launch:
+            graphs, cyc = build_graphs(h, m, eager)
+            for _ in range(a.warmup):
+                run_graph_step(graphs, cyc)
+            start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            barrier()
+            start.record(stream)
+            for _ in range(a.steps):
+                run_graph_step(graphs, cyc)
+            stop.record(stream)
+            barrier()
+            ms = start.elapsed_time(stop)
+            if not eager:
+                used_kernel[0] = h.last_step_kernel
+            h.check_device(stream)
+            del graphs
+            h.close()
+            return max_over_ranks(ms), None
         for _ in range(a.warmup):
             run_step(h, m, eager)
         steps = min(a.steps, 2) if per_launch else a.steps
@@ -378,28 +427,30 @@ def run_gpu(a, rank, world, local_rank):
     peak, peak_kind = measured_peak()
     result = {}
 
-    # headline: DeltaLog at M over the timed region (no events between launches)
+    # headline: DeltaLog at M over the timed region (no events between launches);
+    # in a B x M grid, M = 1 stands for the eager kernel
+    eager_head = bool(getattr(a, "eager_headline", False))
     sampler = ClockSampler(local_rank)
     sampler.start()
-    ms, _ = timed(M)
+    ms, _ = timed(M, eager=eager_head)
     clocks = sampler.stop()
     # per-launch durations of the dominant (append) kernel, second pass
-    launches = timed(M, per_launch=True)[1] if M > 1 else None
+    launches = timed(M, per_launch=True)[1] if M > 1 and not a.graph else None
     tokens_total = B * a.tokens * a.steps * world
     value = tokens_total / (ms / 1e3)
     sb = step_bytes(op, B, H, d, M, a.tokens)
     result["value"] = value
     result["ms"] = ms
 
-    if M > 1 and launches:
+    if launches:
         dur = sum(t for t, _ in launches) / len(launches)
         alg = sum(launch_bytes(op, "append", B, H, d, d, n) for _, n in launches) / len(launches)
         dominant = ("deltalog_stream_kernel" if used_kernel[0] == "stream"
                     else "deltalog_step_kernel") + " (append)"
-    else:
+    else:   # average over every launch of the step (graph replay or M = 1)
         dur = ms / (a.steps * a.tokens)
-        alg = launch_bytes(op, "eager" if M == 1 else "merge", B, H, d, d, 0)
-        dominant = "deltalog_step_kernel (merge, M=1)"
+        alg = sb / a.tokens
+        dominant = "eager_step_kernel" if eager_head else "deltalog_step_kernel (all launches)"
     achieved = alg / (dur / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "traffic": profiled_traffic(workload_name(a)),
@@ -461,7 +512,7 @@ def run_gpu(a, rank, world, local_rank):
                       "stream, o written by the kernel into pinned host memory"}
 
     if rank != 0:
-        return
+        return None
     line = {
         "metric": METRIC, "value": result["value"], "unit": UNIT, "n_gpus": world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": result["ms"] / a.steps,
@@ -470,8 +521,11 @@ def run_gpu(a, rank, world, local_rank):
         "config": {"workload": workload_name(a), "op": op, "B": B, "H": H, "d_k": d, "d_v": d,
                    "M": M, "state": "fp32", "inputs": "bf16", "tokens_per_step": a.tokens,
                    "step_kernel": used_kernel[0], "pdl": not a.no_pdl,
+                   "launch": "cuda graph per cycle" if a.graph else "python loop",
                    "input_pool_tokens": a.pool, "seed": a.seed,
-                   "l2": f"inputs larger than L2 (state {4 * B * H * d * d / 1e6:.0f} MB)",
+                   "l2": (f"inputs larger than L2 (state {4 * B * H * d * d / 1e6:.0f} MB)"
+                          if 4 * B * H * d * d > L2_BYTES else
+                          f"state {4 * B * H * d * d / 1e6:.1f} MB fits in L2: HBM figures undercount"),
                    "parallelism": "replicas" if world == 1 else f"replicas x{world} (B per rank)"},
         "roofline": roofline,
         "gpu_launches": a.steps * a.tokens,
@@ -482,7 +536,27 @@ def run_gpu(a, rank, world, local_rank):
     line.update(extra)
     if not a.no_cpu and world == 1:
         line["cpu_baseline"] = cpu_baseline(a)
-    print(json.dumps(line), flush=True)
+    return line
+
+
+def run_grid(a, rank, world, local_rank):
+    """B x M sweep (one JSON line per point): CUDA-graph replay, 512-token
+    steps by default, M = 1 timed on the eager kernel."""
+    import copy
+    bs, ms = a.grid.split("x")
+    for B in [int(x) for x in bs.split(",")]:
+        for M in [int(x) for x in ms.split(",")]:
+            p = copy.copy(a)
+            p.B, p.M, p.graph = B, M, True
+            p.no_e2e, p.no_cpu, p.no_eager, p.sweep = True, True, True, ""
+            p.eager_headline = M == 1
+            if p.tokens % M:
+                continue
+            line = run_gpu(p, rank, world, local_rank)
+            if line is not None:
+                line["config"]["grid_point"] = {"B": B, "M": M, "kernel": "eager" if M == 1 else "deltalog"}
+                line["step_gbs"] = line["roofline"]["step_gbs"]
+                print(json.dumps(line), flush=True)
 
 
 def main():
@@ -502,7 +576,12 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_gpu(a, rank, world, local_rank)
+        if a.grid:
+            run_grid(a, rank, world, local_rank)
+        else:
+            line = run_gpu(a, rank, world, local_rank)
+            if line is not None:
+                print(json.dumps(line), flush=True)
     finally:
         if world > 1:
             import torch.distributed as dist
