@@ -42,7 +42,7 @@ def parse():
     ap.add_argument("--op", choices=["gdn", "kda", "rwkv6"], default="gdn")
     ap.add_argument("--B", type=int, default=256)
     ap.add_argument("--H", type=int, default=32)
-    ap.add_argument("--d", type=int, default=128)
+    ap.add_argument("--dk", dest="d", type=int, default=128, help="d_k = d_v")
     ap.add_argument("--M", type=int, default=8)
     ap.add_argument("--tokens", type=int, default=256, help="decode tokens per bench step")
     ap.add_argument("--pool", type=int, default=64, help="distinct input tokens kept on device")
@@ -124,6 +124,31 @@ def write_bytes_per_token(op, B, H, d, M, es=2):
     ent = entry_bytes(op, d, d, es)
     per_cycle = (M - 1) * (io_w + ent) + (io_w + state_w)
     return H * per_cycle / M
+
+
+# ---------------------------------------------------------------------------
+# multi-rank plumbing (one process per GPU; replicas, weak scaling)
+# ---------------------------------------------------------------------------
+
+def rank_seed(seed, rank):
+    """Each rank is an independent replica with its own B slots and inputs."""
+    return seed + 1000 * rank
+
+
+def reduce_max(x, world, device):
+    """Max of a per-rank float over all ranks (the job's time is its slowest rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(B, tokens, steps, world, max_ms):
+    """Whole-job throughput: every rank's slot-tokens over the slowest rank's time."""
+    return B * tokens * steps * world / (max_ms / 1e3)
 
 
 # ---------------------------------------------------------------------------
@@ -287,7 +312,7 @@ def run_gpu(a, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     op, B, H, d, M = a.op, a.B, a.H, a.d, a.M
-    seed = a.seed + 1000 * rank
+    seed = rank_seed(a.seed, rank)
     es = 2
 
     # inputs: a pool of distinct tokens resident in HBM (> L2), cycled
@@ -326,11 +351,7 @@ def run_gpu(a, rank, world, local_rank):
         torch.cuda.synchronize(dev)
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, dev)
 
     tok_counter = [0]
     used_kernel = [None]
@@ -436,8 +457,7 @@ def run_gpu(a, rank, world, local_rank):
     clocks = sampler.stop()
     # per-launch durations of the dominant (append) kernel, second pass
     launches = timed(M, per_launch=True)[1] if M > 1 and not a.graph else None
-    tokens_total = B * a.tokens * a.steps * world
-    value = tokens_total / (ms / 1e3)
+    value = job_tokens_per_s(B, a.tokens, a.steps, world, ms)
     sb = step_bytes(op, B, H, d, M, a.tokens)
     result["value"] = value
     result["ms"] = ms
