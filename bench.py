@@ -55,6 +55,9 @@ def parse():
                     help="dl_step kernel variant")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch every step with plain stream ordering")
+    ap.add_argument("--stagger", action="store_true",
+                    help="offset slot b's merge cycle by b mod M (every launch ragged: 1/M of "
+                         "the slots merge each token)")
     ap.add_argument("--graph", action="store_true",
                     help="replay each M-token cycle from a CUDA graph instead of launching from Python")
     ap.add_argument("--grid", default="",
@@ -63,6 +66,8 @@ def parse():
     args = ap.parse_args()
     if args.grid:
         return args
+    if args.stagger and args.graph:
+        ap.error("--stagger runs the Python launch loop")
     if args.tokens % args.M:
         ap.error("--tokens must be a multiple of --M")
     return args
@@ -403,6 +408,14 @@ def run_gpu(a, rank, world, local_rank):
         which every append launch is bracketed by its own pair of events: those
         events sit between launches, so each launch is timed in isolation)."""
         h = make_handle(m)
+        if a.stagger and not eager and m > 1:
+            # re-admit slot b at token (b mod m) so that every slot runs its own cycle
+            for j in range(m):
+                for b in range(j, B, m):
+                    h.slot_load(b, S0[b])
+                i = tok_counter[0] % a.pool
+                tok_counter[0] += 1
+                h.step(*tok_args(dpool, i), out=out[i], stream=stream)
         if a.graph and not per_launch:
             graphs, cyc = build_graphs(h, m, eager)
             for _ in range(a.warmup):
@@ -542,6 +555,7 @@ def run_gpu(a, rank, world, local_rank):
                    "M": M, "state": "fp32", "inputs": "bf16", "tokens_per_step": a.tokens,
                    "step_kernel": used_kernel[0], "pdl": not a.no_pdl,
                    "launch": "cuda graph per cycle" if a.graph else "python loop",
+                   "slot_cycles": "staggered (slot b offset by b mod M)" if a.stagger else "lockstep",
                    "input_pool_tokens": a.pool, "seed": a.seed,
                    "l2": (f"inputs larger than L2 (state {4 * B * H * d * d / 1e6:.0f} MB)"
                           if 4 * B * H * d * d > L2_BYTES else

@@ -96,9 +96,12 @@ int dl_load_state(dl_t h, const float* S, void* stream);
 int dl_set_bonus(dl_t h, const float* u, void* stream);
 
 /* One DeltaLog decode token for all B slots and H heads.  q is r for RWKV6.
- * With n entries in the log before the call: if n + 1 < M the step appends
- * (Sbar is read, never written); if n + 1 == M it merges (Sbar <- S_t and the
- * log empties).  Writes o [B][H][d_v].  All pointers are device pointers. */
+ * Per slot, with n entries in its log before the call: if n + 1 < M the step
+ * appends (Sbar is read, never written); if n + 1 == M it merges (Sbar <- S_t
+ * and the log empties).  Slots normally move in lockstep; after dl_slot_load
+ * or dl_slot_merge they may sit at different points of their cycles, and each
+ * slot then follows its own.  Writes o [B][H][d_v].  All pointers are device
+ * pointers. */
 int dl_step(dl_t h, const void* q, const void* k, const void* v,
             const float* log_decay, const float* beta, void* o, void* stream);
 
@@ -117,12 +120,13 @@ int dl_step_host(dl_t h, const void* q, const void* k, const void* v,
                  const float* log_decay, const float* beta, void* o, void* stream);
 
 /* Eager dense baseline: read S_{t-1} from Sbar, write S_t back, every token.
- * Requires an empty log (returns DL_ERR_STATE otherwise; call dl_merge). */
+ * Requires every slot's log to be empty (DL_ERR_STATE otherwise; call
+ * dl_merge). */
 int dl_eager_step(dl_t h, const void* q, const void* k, const void* v,
                   const float* log_decay, const float* beta, void* o, void* stream);
 
-/* Fold the log into Sbar now (no output) and empty it; a no-op on an empty
- * log.  For an explicit flush, slot eviction or a checkpoint. */
+/* Fold every slot's log into Sbar now (no output) and empty them; a no-op
+ * when all logs are empty.  For an explicit flush or a checkpoint. */
 int dl_merge(dl_t h, void* stream);
 
 /* Write the logical state (Sbar + replayed log) to S_out [B][H][d_k][d_v]
@@ -165,9 +169,26 @@ int dl_set_option(dl_t h, int option, int value);
  * DL_STEP_REGISTER or DL_STEP_STREAM (DL_STEP_AUTO before the first step). */
 int dl_last_step_kernel(dl_t h, int* kind);
 
-/* Number of entries currently in the log (host-side counter, exact in stream
- * order). */
+/* Number of entries currently in the log when every slot holds the same
+ * number (host-side counter, exact in stream order); DL_ERR_STATE when slots
+ * differ (see dl_slot_log_len). */
 int dl_log_len(dl_t h, int* n);
+
+/* Per-slot lifecycle for serving (admission, eviction, checkpoint of one
+ * sequence while the other slots keep decoding).
+ *   dl_slot_load: set slot `slot`'s state to S [H][d_k][d_v] (device pointer;
+ *     NULL = zeros, e.g. a fresh sequence) and empty its log, so it starts a
+ *     new merge cycle while the other slots continue theirs.
+ *   dl_slot_merge: fold slot `slot`'s log into its base now (no output) and
+ *     empty it; a no-op on an empty log.
+ *   dl_slot_read: write slot `slot`'s logical state (base + replayed log) to
+ *     S_out [H][d_k][d_v] (device pointer) without changing the handle.
+ *   dl_slot_log_len: entries in slot `slot`'s log.
+ * All are asynchronous on `stream`; DL_ERR_ARG for a slot outside [0, B). */
+int dl_slot_load(dl_t h, int slot, const float* S, void* stream);
+int dl_slot_merge(dl_t h, int slot, void* stream);
+int dl_slot_read(dl_t h, int slot, float* S_out, void* stream);
+int dl_slot_log_len(dl_t h, int slot, int* n);
 
 /* Read and clear the handle's device error word (synchronises `stream`).
  * Returns DL_OK or DL_ERR_DEVICE. */

@@ -39,6 +39,10 @@ SIGNATURES = {
     "dl_set_option": (_I, [_P, _I, _I]),
     "dl_last_step_kernel": (_I, [_P, ctypes.POINTER(_I)]),
     "dl_log_len": (_I, [_P, ctypes.POINTER(_I)]),
+    "dl_slot_load": (_I, [_P, _I, _P, _P]),
+    "dl_slot_merge": (_I, [_P, _I, _P]),
+    "dl_slot_read": (_I, [_P, _I, _P, _P]),
+    "dl_slot_log_len": (_I, [_P, _I, ctypes.POINTER(_I)]),
     "dl_check_device": (_I, [_P, _P]),
     "dl_strerror": (ctypes.c_char_p, [_I]),
     "dl_last_error": (ctypes.c_char_p, []),

@@ -53,12 +53,20 @@ struct StepArgs {
   float* logLam;           // [BH][gdn_lam_stride(Mcap)] (GDN) or [BH][Mcap][DK]
   const float* u;          // [H][DK] (RWKV6)
   int* err;               // device error word (kErr* bits)
+  const int* n_in;         // ragged launches: log length per slot before this step [B]
+  int* n_out;              // ragged launches: log length per slot after this step [B]
   int H;
+  int M;                   // merge interval
   int Mcap;                // log capacity per (slot, head), >= 1
-  int n;                   // entries in the log before this step
+  int n;                   // entries in the log before this step (lockstep launches)
 };
 
-// Arguments of log materialisation: Sout = Sbar + replayed log (n >= 1).
+// Step kernel modes: every slot appends, every slot merges, or each slot
+// decides from its own log length (slots admitted at different times).
+enum { MODE_APPEND = 0, MODE_MERGE = 1, MODE_RAGGED = 2 };
+
+// Arguments of log materialisation: Sout = Sbar + replayed log, for the
+// units [unit0, unit0 + gridDim.x); Sout points at the first of them.
 struct MaterializeArgs {
   const float* Sin;
   float* Sout;
@@ -66,6 +74,9 @@ struct MaterializeArgs {
   const void* logB;
   const float* logLam;
   int* err;
+  const int* n_slot;   // per-slot log length, or null: every unit has n entries
+  long unit0;
+  int H;
   int Mcap;
   int n;
 };
@@ -203,13 +214,16 @@ __device__ __forceinline__ bool wait_log(uint64_t* bar, int n, int* err) {
 }
 
 // ---------------------------------------------------------------------------
-// Deferred step.  MERGE=false: append (Sbar read only).  MERGE=true: the step
-// with n+1 == M; it also writes S_t over Sbar.  NSPLIT > 1 splits each head's
+// Deferred step.  MODE_APPEND: every slot appends (Sbar read only).
+// MODE_MERGE: every slot is at n+1 == M; it also writes S_t over Sbar.
+// MODE_RAGGED: slots sit at different points of their cycles; each CTA reads
+// its slot's n, merges when n+1 == M, and the slot's first CTA records the
+// slot's new log length.  NSPLIT > 1 splits each head's
 // d_v columns into NSPLIT value tiles, one CTA each (grid B*H*NSPLIT); every
 // tile recomputes the head's ReplayPrep coefficients and the first tile
 // appends the key-side entry.
 // ---------------------------------------------------------------------------
-template <int OP, int DK, int DV, typename TI, bool MERGE, int NSPLIT>
+template <int OP, int DK, int DV, typename TI, int MODE, int NSPLIT>
 __global__ void __launch_bounds__(Tile<DK, DV / NSPLIT>::NT, Tile<DK, DV / NSPLIT>::MINB)
 deltalog_step_kernel(const StepArgs a) {
   constexpr int DVT = DV / NSPLIT;  // value-tile width owned by this CTA
@@ -235,7 +249,9 @@ deltalog_step_kernel(const StepArgs a) {
   const long sh = blockIdx.x / NSPLIT;
   const int col0 = (blockIdx.x % NSPLIT) * DVT;  // first value column of this tile
   const int h = static_cast<int>(sh % a.H);
-  const int n = a.n;
+  const int n = MODE == MODE_RAGGED ? a.n_in[sh / a.H] : a.n;
+  const bool MERGE = MODE == MODE_MERGE || (MODE == MODE_RAGGED && n + 1 == a.M);
+  if (MODE == MODE_RAGGED && h == 0 && col0 == 0 && threadIdx.x == 0) a.n_out[sh / a.H] = MERGE ? 0 : n + 1;
 
   const TI* sA = reinterpret_cast<const TI*>(s_dyn);
   const float* sL = reinterpret_cast<const float*>(s_dyn + LL::a_bytes(n));
@@ -253,7 +269,7 @@ deltalog_step_kernel(const StepArgs a) {
   float4 st[TL::RPT];
 #pragma unroll
   for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + (rg * TL::RPT + j) * DV + col0 + 4 * c4);
-  if (!MERGE) griddep_launch_dependents();
+  if (MODE == MODE_APPEND) griddep_launch_dependents();
   griddep_wait();
   if (tid == 0) stage_log<OP, DK, DV, TI>(s_dyn, &s_bar, a.logA, a.logLam, a.logB, sh, a.Mcap, n);
 
@@ -551,7 +567,8 @@ eager_step_kernel(const StepArgs a) {
 
 // ---------------------------------------------------------------------------
 // Materialise base + log into Sout (dl_merge with Sout == Sin, dl_read_state
-// otherwise).  Lam_last = Lam_{n-1}, the newest snapshot.  Requires n >= 1.
+// otherwise).  Lam_last = Lam_{n-1}, the newest snapshot; a unit with an
+// empty log is copied through.
 // ---------------------------------------------------------------------------
 template <int OP, int DK, int DV, typename TI>
 __global__ void __launch_bounds__(Tile<DK, DV>::NT, Tile<DK, DV>::MINB)
@@ -568,8 +585,8 @@ materialize_kernel(const MaterializeArgs a) {
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const int c4 = tid % TL::TPR, rg = tid / TL::TPR;
-  const long sh = blockIdx.x;
-  const int n = a.n;
+  const long sh = a.unit0 + blockIdx.x;
+  const int n = a.n_slot ? a.n_slot[sh / a.H] : a.n;
 
   const TI* sA = reinterpret_cast<const TI*>(s_dyn);
   const float* sL = reinterpret_cast<const float*>(s_dyn + LL::a_bytes(n));
@@ -586,8 +603,9 @@ materialize_kernel(const MaterializeArgs a) {
 #pragma unroll
   for (int m = 0; m < TL::KPL; ++m) {
     const int j = lane + 32 * m;
-    ll[m] = PERKEY ? a.logLam[(sh * a.Mcap + (n - 1)) * DK + j]
-                   : a.logLam[sh * gdn_lam_stride(a.Mcap) + (n - 1)];
+    ll[m] = n == 0 ? 0.f
+            : PERKEY ? a.logLam[(sh * a.Mcap + (n - 1)) * DK + j]
+                     : a.logLam[sh * gdn_lam_stride(a.Mcap) + (n - 1)];
   }
   if (!PERKEY && tid < n) s_lam[tid] = a.logLam[sh * gdn_lam_stride(a.Mcap) + tid];
   __syncthreads();
@@ -623,7 +641,7 @@ materialize_kernel(const MaterializeArgs a) {
       fma4(st[j4 + 3], a4.w, b4);
     }
   }
-  float* Sq = a.Sout + sh * (DK * DV);
+  float* Sq = a.Sout + blockIdx.x * (DK * DV);
 #pragma unroll
   for (int j = 0; j < TL::RPT; ++j) st_state(Sq + (rg * TL::RPT + j) * DV + 4 * c4, st[j]);
 }

@@ -25,6 +25,8 @@ struct LaunchShape {
   bool aligned16;  // q, k, v, o (and per-key log_decay) 16-byte aligned (bulk-copy sources)
   bool pdl;        // launch the step as a programmatic dependent of the previous kernel
   int split;       // value tiles per head for the register-tile step kernel (1, 2 or 4)
+  int max_n;       // longest log of any launched unit (shared-memory sizing)
+  int units;       // materialisation: units in the launch
 };
 
 // Launch with the programmatic-stream-serialisation attribute when `pdl`.
@@ -110,44 +112,46 @@ cudaError_t allow_smem(K kern, size_t smem, size_t worst) {
   return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(worst));
 }
 
-template <int OP, int DK, int DV, typename TI, int NSPLIT>
-cudaError_t register_step(const LaunchShape& s, bool merge, const StepArgs& a, cudaStream_t st) {
+template <int OP, int DK, int DV, typename TI, int MODE, int NSPLIT>
+cudaError_t register_step_mode(const LaunchShape& s, const StepArgs& a, cudaStream_t st) {
   using TL = Tile<DK, DV / NSPLIT>;
   using LL = LogLayout<OP, DK, DV, TI>;
-  const size_t smem = LL::step_smem(a.n, merge);
-  const int grid = s.BH * NSPLIT;
-  if (merge) {
-    auto kern = deltalog_step_kernel<OP, DK, DV, TI, true, NSPLIT>;
-    cudaError_t e = allow_smem(kern, smem, LL::step_smem(kMaxM - 1, true));
-    if (e != cudaSuccess) return e;
-    return launch_maybe_pdl(kern, grid, TL::NT, smem, st, s.pdl, a);
-  }
-  auto kern = deltalog_step_kernel<OP, DK, DV, TI, false, NSPLIT>;
-  cudaError_t e = allow_smem(kern, smem, LL::step_smem(kMaxM - 1, false));
+  // a ragged launch sizes shared memory for its longest log, as a merge
+  const size_t smem = MODE == MODE_RAGGED ? LL::step_smem(s.max_n, true) : LL::step_smem(a.n, MODE == MODE_MERGE);
+  auto kern = deltalog_step_kernel<OP, DK, DV, TI, MODE, NSPLIT>;
+  cudaError_t e = allow_smem(kern, smem, LL::step_smem(kMaxM - 1, MODE != MODE_APPEND));
   if (e != cudaSuccess) return e;
-  return launch_maybe_pdl(kern, grid, TL::NT, smem, st, s.pdl, a);
+  return launch_maybe_pdl(kern, s.BH * NSPLIT, TL::NT, smem, st, s.pdl, a);
+}
+
+template <int OP, int DK, int DV, typename TI, int NSPLIT>
+cudaError_t register_step(const LaunchShape& s, int mode, const StepArgs& a, cudaStream_t st) {
+  if (mode == MODE_APPEND) return register_step_mode<OP, DK, DV, TI, MODE_APPEND, NSPLIT>(s, a, st);
+  if (mode == MODE_MERGE) return register_step_mode<OP, DK, DV, TI, MODE_MERGE, NSPLIT>(s, a, st);
+  return register_step_mode<OP, DK, DV, TI, MODE_RAGGED, NSPLIT>(s, a, st);
 }
 
 template <int OP, int DK, int DV, typename TI>
-cudaError_t step_dims(const LaunchShape& s, bool merge, const StepArgs& a, cudaStream_t st, int* used) {
+cudaError_t step_dims(const LaunchShape& s, int mode, const StepArgs& a, cudaStream_t st, int* used) {
   // AUTO runs the register-tile kernel, the faster of the two on B200 for
-  // every operator's merge launches and for d_v = 64; STREAM is opt-in.
-  if (s.variant == STEP_STREAM && s.aligned16) {
+  // every operator's merge launches and for d_v = 64; STREAM is opt-in and
+  // runs lockstep launches only.
+  if (s.variant == STEP_STREAM && s.aligned16 && mode != MODE_RAGGED) {
     bool launched = false;
-    cudaError_t e = merge ? stream_dims<OP, DK, DV, TI, true>(s, a, st, &launched)
-                          : stream_dims<OP, DK, DV, TI, false>(s, a, st, &launched);
+    cudaError_t e = mode == MODE_MERGE ? stream_dims<OP, DK, DV, TI, true>(s, a, st, &launched)
+                                       : stream_dims<OP, DK, DV, TI, false>(s, a, st, &launched);
     if (launched) *used = STEP_STREAM;
     if (e != cudaSuccess || launched) return e;
   }
   if (s.variant == STEP_STREAM) return cudaErrorNotSupported;
   *used = STEP_REGISTER;
   if constexpr (DV >= 128) {
-    if (s.split == 4) return register_step<OP, DK, DV, TI, 4>(s, merge, a, st);
+    if (s.split == 4) return register_step<OP, DK, DV, TI, 4>(s, mode, a, st);
   }
   if constexpr (DV >= 64) {
-    if (s.split == 2) return register_step<OP, DK, DV, TI, 2>(s, merge, a, st);
+    if (s.split == 2) return register_step<OP, DK, DV, TI, 2>(s, mode, a, st);
   }
-  return register_step<OP, DK, DV, TI, 1>(s, merge, a, st);
+  return register_step<OP, DK, DV, TI, 1>(s, mode, a, st);
 }
 
 template <int OP, int DK, int DV, typename TI>
@@ -166,10 +170,10 @@ template <int OP, int DK, int DV, typename TI>
 cudaError_t materialize_dims(const LaunchShape& s, const MaterializeArgs& a, cudaStream_t st) {
   using LL = LogLayout<OP, DK, DV, TI>;
   auto kern = materialize_kernel<OP, DK, DV, TI>;
-  const size_t smem = LL::materialize_smem(a.n);
+  const size_t smem = LL::materialize_smem(s.max_n);
   cudaError_t e = allow_smem(kern, smem, LL::materialize_smem(kMaxM - 1));
   if (e != cudaSuccess) return e;
-  kern<<<s.BH, Tile<DK, DV>::NT, smem, st>>>(a);
+  kern<<<s.units, Tile<DK, DV>::NT, smem, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -187,8 +191,8 @@ cudaError_t materialize_dims(const LaunchShape& s, const MaterializeArgs& a, cud
   } while (0)
 
 template <int OP>
-cudaError_t launch_step_op(const LaunchShape& s, bool merge, const StepArgs& a, cudaStream_t st, int* used) {
-  DL_DISPATCH_DIMS(step_dims, s, merge, a, st, used);
+cudaError_t launch_step_op(const LaunchShape& s, int mode, const StepArgs& a, cudaStream_t st, int* used) {
+  DL_DISPATCH_DIMS(step_dims, s, mode, a, st, used);
 }
 
 template <int OP>
@@ -202,12 +206,12 @@ cudaError_t launch_materialize_op(const LaunchShape& s, const MaterializeArgs& a
 }
 
 #define DL_DECLARE_OP(OPV)                                                                      \
-  extern template cudaError_t launch_step_op<OPV>(const LaunchShape&, bool, const StepArgs&, cudaStream_t, int*); \
+  extern template cudaError_t launch_step_op<OPV>(const LaunchShape&, int, const StepArgs&, cudaStream_t, int*); \
   extern template cudaError_t launch_eager_op<OPV>(const LaunchShape&, const StepArgs&, cudaStream_t);      \
   extern template cudaError_t launch_materialize_op<OPV>(const LaunchShape&, const MaterializeArgs&, cudaStream_t);
 
 #define DL_INSTANTIATE_OP(OPV)                                                                  \
-  template cudaError_t launch_step_op<OPV>(const LaunchShape&, bool, const StepArgs&, cudaStream_t, int*); \
+  template cudaError_t launch_step_op<OPV>(const LaunchShape&, int, const StepArgs&, cudaStream_t, int*); \
   template cudaError_t launch_eager_op<OPV>(const LaunchShape&, const StepArgs&, cudaStream_t);      \
   template cudaError_t launch_materialize_op<OPV>(const LaunchShape&, const MaterializeArgs&, cudaStream_t);
 

@@ -153,8 +153,36 @@ class DeltaLog:
 
     @property
     def log_len(self):
+        """Common log length of all slots (raises DeltaLogError when slots differ)."""
         n = ctypes.c_int()
         N.call("dl_log_len", self._h, ctypes.byref(n))
+        return n.value
+
+    # -- per-slot lifecycle (serving) ------------------------------------------
+    def _slot_state_shape(self):
+        return (self.H, self.d_k, self.d_v)
+
+    def slot_load(self, slot, S=None, stream=None):
+        """Admit a sequence into `slot`: state S [H, d_k, d_v] (None = zeros), empty log."""
+        if S is not None:
+            self._check("S", S, self._slot_state_shape(), torch.float32)
+        N.call("dl_slot_load", self._h, int(slot), _ptr(S), self._stream(stream))
+
+    def slot_merge(self, slot, stream=None):
+        """Fold `slot`'s log into its base now (eviction / checkpoint)."""
+        N.call("dl_slot_merge", self._h, int(slot), self._stream(stream))
+
+    def slot_read(self, slot, out=None, stream=None):
+        """Logical state of `slot` as [H, d_k, d_v] fp32 (the handle is unchanged)."""
+        if out is None:
+            out = torch.empty(self._slot_state_shape(), dtype=torch.float32, device=self.device)
+        self._check("out", out, self._slot_state_shape(), torch.float32)
+        N.call("dl_slot_read", self._h, int(slot), _ptr(out), self._stream(stream))
+        return out
+
+    def slot_log_len(self, slot):
+        n = ctypes.c_int()
+        N.call("dl_slot_log_len", self._h, int(slot), ctypes.byref(n))
         return n.value
 
     def check_device(self, stream=None):

@@ -302,3 +302,83 @@ def test_programmatic_launch_gives_identical_results(op):
         res.append((torch.stack(outs).cpu(), h.read_state().cpu()))
         h.close()
     assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
+
+
+# ---- per-slot cycles (serving: admit / evict / flush one slot) -----------------
+
+def _oracle_step(op, S, seq, t, u):
+    """One eager step of every unit (fp64): returns (o_t, S_t)."""
+    one = {key: val[t:t + 1] for key, val in seq.items()}
+    o, S_next, _ = run_oracle(op, S, one, u)
+    return o[0], S_next
+
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("dims,M", [((64, 64), 3), ((128, 128), 4), ((128, 128), 8), ((64, 128), 5)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_ragged_slots(op, dims, M, dtype):
+    """Slots admitted and flushed at different times follow their own cycles."""
+    from recurrent_state_update_deltalog_b200 import DeltaLog, DeltaLogError
+    from synthetic import initial_state
+    B, H, T = 6, 3, 20
+    dk, dv = dims
+    S0, seq, u = make_inputs(op, B, H, dk, dv, T, dtype)
+    fresh = initial_state(7, B, H, dk, dv)                       # states of admitted sequences
+    dseq = to_device(seq, dtype)
+    tol = TOL[dtype]
+    h = DeltaLog(B, H, dk, dv, M, op=op, dtype=dtype)
+    h.load_state(torch.from_numpy(S0).cuda())
+    if u is not None:
+        h.set_bonus(torch.from_numpy(u).cuda())
+    S_ref = S0.astype(np.float64)
+    expect_n = [0] * B
+    events = {2: ("load", 2), 5: ("merge", 4), 7: ("zero", 0), 11: ("load", 1), 13: ("flush", None),
+              15: ("load", 5)}
+    outs, refs = [], []
+    for t in range(T):
+        ev = events.get(t)
+        if ev:
+            kind, b = ev
+            if kind == "load":
+                h.slot_load(b, torch.from_numpy(fresh[b]).cuda())
+                S_ref[b] = fresh[b]
+                expect_n[b] = 0
+            elif kind == "zero":
+                h.slot_load(b)
+                S_ref[b] = 0
+                expect_n[b] = 0
+            elif kind == "merge":
+                h.slot_merge(b)
+                expect_n[b] = 0
+            else:
+                got = h.read_state().cpu().numpy()
+                assert relerr(got, S_ref) < tol
+                h.merge()
+                expect_n = [0] * B
+        assert [h.slot_log_len(b) for b in range(B)] == expect_n
+        if len(set(expect_n)) > 1:
+            with pytest.raises(DeltaLogError):
+                h.log_len
+        o = h.step(*step_args(op, dseq, t))
+        outs.append(o.float().cpu().numpy())
+        o_ref, S_ref = _oracle_step(op, S_ref, seq, t, u)
+        refs.append(o_ref)
+        expect_n = [0 if n + 1 == M else n + 1 for n in expect_n]
+        if t in (8, 16):
+            for b in (0, 3):
+                assert relerr(h.slot_read(b).cpu().numpy(), S_ref[b]) < tol, (t, b)
+    assert relerr(np.stack(outs), np.stack(refs)) < tol
+    assert relerr(h.read_state().cpu().numpy(), S_ref) < tol
+    h.check_device()
+    h.close()
+
+
+def test_slot_arguments_rejected():
+    from recurrent_state_update_deltalog_b200 import DeltaLog, DeltaLogError
+    h = DeltaLog(2, 2, 64, 64, 4, op="gdn")
+    for bad in (-1, 2):
+        with pytest.raises(DeltaLogError):
+            h.slot_merge(bad)
+        with pytest.raises(DeltaLogError):
+            h.slot_load(bad)
+    h.close()
