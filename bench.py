@@ -55,9 +55,9 @@ def parse():
                     help="dl_step kernel variant")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch every step with plain stream ordering")
-    ap.add_argument("--stagger", action="store_true",
-                    help="offset slot b's merge cycle by b mod M (every launch ragged: 1/M of "
-                         "the slots merge each token)")
+    ap.add_argument("--admit-every", type=int, default=0, metavar="K",
+                    help="re-admit one slot (dl_slot_load of a fresh state, round robin) every K "
+                         "tokens inside the timed region (serving churn; 0 = off)")
     ap.add_argument("--graph", action="store_true",
                     help="replay each M-token cycle from a CUDA graph instead of launching from Python")
     ap.add_argument("--grid", default="",
@@ -66,8 +66,8 @@ def parse():
     args = ap.parse_args()
     if args.grid:
         return args
-    if args.stagger and args.graph:
-        ap.error("--stagger runs the Python launch loop")
+    if args.admit_every and args.graph:
+        ap.error("--admit-every runs the Python launch loop")
     if args.tokens % args.M:
         ap.error("--tokens must be a multiple of --M")
     return args
@@ -378,6 +378,9 @@ def run_gpu(a, rank, world, local_rank):
                 rec.append((e0, e1, j % m))
             else:
                 h.step(*args, out=out[i], stream=stream)
+            if a.admit_every and not eager and tok_counter[0] % a.admit_every == 0:
+                b = (tok_counter[0] // a.admit_every) % B
+                h.slot_load(b, S0[b], stream=stream)
 
     def build_graphs(h, m, eager):
         """One CUDA graph per m-token cycle of the input pool (8 tokens for the
@@ -408,14 +411,6 @@ def run_gpu(a, rank, world, local_rank):
         which every append launch is bracketed by its own pair of events: those
         events sit between launches, so each launch is timed in isolation)."""
         h = make_handle(m)
-        if a.stagger and not eager and m > 1:
-            # re-admit slot b at token (b mod m) so that every slot runs its own cycle
-            for j in range(m):
-                for b in range(j, B, m):
-                    h.slot_load(b, S0[b])
-                i = tok_counter[0] % a.pool
-                tok_counter[0] += 1
-                h.step(*tok_args(dpool, i), out=out[i], stream=stream)
         if a.graph and not per_launch:
             graphs, cyc = build_graphs(h, m, eager)
             for _ in range(a.warmup):
@@ -555,7 +550,7 @@ def run_gpu(a, rank, world, local_rank):
                    "M": M, "state": "fp32", "inputs": "bf16", "tokens_per_step": a.tokens,
                    "step_kernel": used_kernel[0], "pdl": not a.no_pdl,
                    "launch": "cuda graph per cycle" if a.graph else "python loop",
-                   "slot_cycles": "staggered (slot b offset by b mod M)" if a.stagger else "lockstep",
+                   "admit_every_tokens": a.admit_every or None,
                    "input_pool_tokens": a.pool, "seed": a.seed,
                    "l2": (f"inputs larger than L2 (state {4 * B * H * d * d / 1e6:.0f} MB)"
                           if 4 * B * H * d * d > L2_BYTES else

@@ -96,12 +96,10 @@ int dl_load_state(dl_t h, const float* S, void* stream);
 int dl_set_bonus(dl_t h, const float* u, void* stream);
 
 /* One DeltaLog decode token for all B slots and H heads.  q is r for RWKV6.
- * Per slot, with n entries in its log before the call: if n + 1 < M the step
- * appends (Sbar is read, never written); if n + 1 == M it merges (Sbar <- S_t
- * and the log empties).  Slots normally move in lockstep; after dl_slot_load
- * or dl_slot_merge they may sit at different points of their cycles, and each
- * slot then follows its own.  Writes o [B][H][d_v].  All pointers are device
- * pointers. */
+ * With n entries in the log before the call (every slot holds n; see
+ * dl_slot_load): if n + 1 < M the step appends (Sbar is read, never
+ * written); if n + 1 == M it merges (Sbar <- S_t and the log empties).
+ * Writes o [B][H][d_v].  All pointers are device pointers. */
 int dl_step(dl_t h, const void* q, const void* k, const void* v,
             const float* log_decay, const float* beta, void* o, void* stream);
 
@@ -169,26 +167,30 @@ int dl_set_option(dl_t h, int option, int value);
  * DL_STEP_REGISTER or DL_STEP_STREAM (DL_STEP_AUTO before the first step). */
 int dl_last_step_kernel(dl_t h, int* kind);
 
-/* Number of entries currently in the log when every slot holds the same
- * number (host-side counter, exact in stream order); DL_ERR_STATE when slots
- * differ (see dl_slot_log_len). */
+/* Number of entries currently in every slot's log (host-side counter, exact
+ * in stream order). */
 int dl_log_len(dl_t h, int* n);
 
 /* Per-slot lifecycle for serving (admission, eviction, checkpoint of one
- * sequence while the other slots keep decoding).
+ * sequence while the other slots keep decoding).  Every slot keeps the
+ * handle's log length n: instead of starting a cycle of its own, a slot that
+ * is loaded or merged while n > 0 has its n log entries set to a_i = 0,
+ * b_i = 0, Lam_i = 0.  Such entries add nothing to S_t, and Lam_i = 0 makes
+ * the cumulative decay of the following entries and of the base start at
+ * that point, so the slot's logical state is exactly the loaded (or merged)
+ * one and every later dl_step stays one lockstep launch.  At the handle's
+ * next merge step the slot merges with the rest, possibly after fewer than
+ * M tokens of its own.
  *   dl_slot_load: set slot `slot`'s state to S [H][d_k][d_v] (device pointer;
- *     NULL = zeros, e.g. a fresh sequence) and empty its log, so it starts a
- *     new merge cycle while the other slots continue theirs.
+ *     NULL = zeros, e.g. a fresh sequence) and clear its log entries.
  *   dl_slot_merge: fold slot `slot`'s log into its base now (no output) and
- *     empty it; a no-op on an empty log.
+ *     clear its log entries; a no-op when n = 0.
  *   dl_slot_read: write slot `slot`'s logical state (base + replayed log) to
  *     S_out [H][d_k][d_v] (device pointer) without changing the handle.
- *   dl_slot_log_len: entries in slot `slot`'s log.
  * All are asynchronous on `stream`; DL_ERR_ARG for a slot outside [0, B). */
 int dl_slot_load(dl_t h, int slot, const float* S, void* stream);
 int dl_slot_merge(dl_t h, int slot, void* stream);
 int dl_slot_read(dl_t h, int slot, float* S_out, void* stream);
-int dl_slot_log_len(dl_t h, int slot, int* n);
 
 /* Read and clear the handle's device error word (synchronises `stream`).
  * Returns DL_OK or DL_ERR_DEVICE. */

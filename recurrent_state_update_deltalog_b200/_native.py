@@ -42,7 +42,6 @@ SIGNATURES = {
     "dl_slot_load": (_I, [_P, _I, _P, _P]),
     "dl_slot_merge": (_I, [_P, _I, _P]),
     "dl_slot_read": (_I, [_P, _I, _P, _P]),
-    "dl_slot_log_len": (_I, [_P, _I, ctypes.POINTER(_I)]),
     "dl_check_device": (_I, [_P, _P]),
     "dl_strerror": (ctypes.c_char_p, [_I]),
     "dl_last_error": (ctypes.c_char_p, []),

@@ -6,28 +6,18 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
-#include <algorithm>
 #include <new>
 #include <string>
-#include <vector>
 
 struct dl_handle {
   int B, H, dk, dv, M, op, dtype, device;
   int sms, smem_block_optin, smem_sm, smem_reserved;  // device limits
   int step_kernel;                                    // DL_STEP_* requested
   int last_kernel;                                    // DL_STEP_* used by the last dl_step
-  // Log length per slot, tracked on the host in stream order.  n is their
-  // common value while every slot is at the same point of its cycle (the
-  // lockstep kernels take it as an argument), or -1 once slots differ; a
-  // ragged launch then reads them from n_dev[cur] and writes n_dev[cur ^ 1].
-  std::vector<int> nslot;
+  // Entries in every slot's log, tracked on the host in stream order.  All
+  // slots share it: a slot loaded or merged mid-cycle keeps its n positions,
+  // zeroed, so every step is one lockstep launch.
   int n;
-  int max_n;
-  int* n_dev[2];
-  int cur;
-  bool n_dev_valid;    // n_dev[cur] holds nslot
-  int* n_pinned;       // upload staging for nslot
-  cudaEvent_t n_uploaded;
   bool wrote_state;    // the last launch on this handle may have written Sbar
   int Mcap;    // log capacity per (slot, head): max(M - 1, 1)
   size_t esize;
@@ -109,11 +99,9 @@ size_t state_bytes(const dl_handle* h) { return bh(h) * h->dk * h->dv * sizeof(f
 size_t decay_elems(const dl_handle* h) { return bh(h) * lam_per_entry(h); }
 
 void free_all(dl_handle* h) {
-  void* ptrs[] = {h->Sbar, h->logA, h->logB, h->logLam, h->u, h->err, h->n_dev[0], h->n_dev[1]};
+  void* ptrs[] = {h->Sbar, h->logA, h->logB, h->logLam, h->u, h->err};
   for (void* p : ptrs)
     if (p) cudaFree(p);
-  if (h->n_pinned) cudaFreeHost(h->n_pinned);
-  if (h->n_uploaded) cudaEventDestroy(h->n_uploaded);
   for (auto& st : h->st) {
     void* sp[] = {st.q, st.k, st.v, st.o, st.ld, st.beta};
     for (void* p : sp)
@@ -126,22 +114,8 @@ void free_all(dl_handle* h) {
   if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
 }
 
-// Recompute the common log length (or -1) and the longest log after nslot changed.
-void refresh_n(dl_handle* h) {
-  const int first = h->nslot.empty() ? 0 : h->nslot[0];
-  bool same = true;
-  int mx = 0;
-  for (int v : h->nslot) {
-    same = same && v == first;
-    mx = std::max(mx, v);
-  }
-  h->n = same ? first : -1;
-  h->max_n = mx;
-}
-
-// Launch geometry and policies.  `n_policy` is the log length that picks the
-// value-tile split (the common length, or the longest one of a ragged launch).
-dl::LaunchShape shape_of(const dl_handle* h, bool aligned16 = false, int n_policy = 0) {
+// Launch geometry and policies for the handle's current log length.
+dl::LaunchShape shape_of(const dl_handle* h, bool aligned16 = false) {
   dl::LaunchShape s;
   s.BH = static_cast<int>(bh(h));
   s.dk = h->dk;
@@ -159,11 +133,11 @@ dl::LaunchShape shape_of(const dl_handle* h, bool aligned16 = false, int n_polic
   if (h->value_tiles == 0) {
     // measured on B200: two 64-column tiles per head win for d_v = 128 while
     // the log is short (each tile recomputes the key-side coefficients)
-    s.split = h->dv == 128 && n_policy < 16 ? 2 : 1;
+    s.split = h->dv == 128 && h->n < 16 ? 2 : 1;
   } else {
     s.split = h->dv / h->value_tiles >= 32 ? h->value_tiles : 1;
   }
-  s.max_n = h->max_n;
+  s.max_n = h->n;
   s.units = s.BH;
   return s;
 }
@@ -196,8 +170,6 @@ dl::StepArgs step_args(dl_handle* h, const void* q, const void* k, const void* v
   a.logLam = h->logLam;
   a.u = h->u;
   a.err = h->err;
-  a.n_in = h->n_dev[h->cur];
-  a.n_out = h->n_dev[h->cur ^ 1];
   a.H = h->H;
   a.M = h->M;
   a.Mcap = h->Mcap;
@@ -205,33 +177,27 @@ dl::StepArgs step_args(dl_handle* h, const void* q, const void* k, const void* v
   return a;
 }
 
-// Make n_dev[cur] equal to the host's per-slot log lengths (after slots were
-// admitted or flushed individually).
-cudaError_t upload_n(dl_handle* h, cudaStream_t s) {
-  if (h->n_dev_valid) return cudaSuccess;
-  cudaError_t e = cudaEventSynchronize(h->n_uploaded);  // the staging buffer is free again
-  if (e != cudaSuccess) return e;
-  std::copy(h->nslot.begin(), h->nslot.end(), h->n_pinned);
-  e = cudaMemcpyAsync(h->n_dev[h->cur], h->n_pinned, h->nslot.size() * sizeof(int), cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess) e = cudaEventRecord(h->n_uploaded, s);
-  if (e == cudaSuccess) h->n_dev_valid = true;
+// Empty slot `b`'s log without changing its logical state: zero factors
+// contribute nothing, and Lam_i = 0 restarts its cumulative decay at the
+// present token.  Only positions [0, n) are ever read; the whole slot is
+// cleared.
+cudaError_t zero_slot_log(const dl_handle* h, int b, cudaStream_t s) {
+  const size_t units = static_cast<size_t>(h->H), first = static_cast<size_t>(b) * units;
+  const size_t a_unit = static_cast<size_t>(h->Mcap) * h->dk * h->esize;
+  const size_t b_unit = static_cast<size_t>(h->Mcap) * h->dv * logb_esize(h);
+  const size_t l_unit = lam_unit_floats(h) * sizeof(float);
+  cudaError_t e = cudaMemsetAsync(static_cast<char*>(h->logA) + first * a_unit, 0, units * a_unit, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(static_cast<char*>(h->logB) + first * b_unit, 0, units * b_unit, s);
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(reinterpret_cast<char*>(h->logLam) + first * l_unit, 0, units * l_unit, s);
   return e;
-}
-
-// Slot `b` has just emptied its log: mirror it on the host and on the device.
-cudaError_t reset_slot_n(dl_handle* h, int b, cudaStream_t s) {
-  h->nslot[b] = 0;
-  refresh_n(h);
-  if (!h->n_dev_valid) return cudaSuccess;
-  return cudaMemsetAsync(h->n_dev[h->cur] + b, 0, sizeof(int), s);
 }
 
 cudaError_t launch_step(dl_handle* h, int mode, const dl::StepArgs& a, cudaStream_t s) {
   // bulk-copy sources of the streaming kernel (GDN's scalar gate is a plain load)
   const bool al = aligned(a.q, 16) && aligned(a.k, 16) && aligned(a.v, 16) && aligned(a.o, 16) &&
                   (h->op == DL_GDN || aligned(a.log_decay, 16));
-  dl::LaunchShape sh = shape_of(h, al, mode == dl::MODE_RAGGED ? h->max_n : h->n);
-  if (mode == dl::MODE_RAGGED) sh.pdl = false;  // some slots of the previous step may have merged
+  const dl::LaunchShape sh = shape_of(h, al);
   int* used = &h->last_kernel;
   switch (h->op) {
     case DL_GDN: return dl::launch_step_op<dl::OP_GDN>(sh, mode, a, s, used);
@@ -241,7 +207,7 @@ cudaError_t launch_step(dl_handle* h, int mode, const dl::StepArgs& a, cudaStrea
 }
 
 cudaError_t launch_eager(const dl_handle* h, const dl::StepArgs& a, cudaStream_t s) {
-  const dl::LaunchShape sh = shape_of(h, false, 0);
+  const dl::LaunchShape sh = shape_of(h);
   switch (h->op) {
     case DL_GDN: return dl::launch_eager_op<dl::OP_GDN>(sh, a, s);
     case DL_KDA: return dl::launch_eager_op<dl::OP_KDA>(sh, a, s);
@@ -250,9 +216,8 @@ cudaError_t launch_eager(const dl_handle* h, const dl::StepArgs& a, cudaStream_t
 }
 
 // Base + log of units [unit0, unit0 + units) into `out` (which points at the
-// first of them).  n >= 0: every unit has n log entries; n < 0: per-slot
-// lengths from the device (ragged).
-cudaError_t launch_materialize(dl_handle* h, float* out, cudaStream_t s, long unit0, int units, int n) {
+// first of them).
+cudaError_t launch_materialize(const dl_handle* h, float* out, cudaStream_t s, long unit0, int units) {
   dl::MaterializeArgs a;
   a.Sin = h->Sbar;
   a.Sout = out;
@@ -263,16 +228,9 @@ cudaError_t launch_materialize(dl_handle* h, float* out, cudaStream_t s, long un
   a.unit0 = unit0;
   a.H = h->H;
   a.Mcap = h->Mcap;
-  a.n = n;
-  a.n_slot = nullptr;
-  if (n < 0) {
-    cudaError_t e = upload_n(h, s);
-    if (e != cudaSuccess) return e;
-    a.n_slot = h->n_dev[h->cur];
-  }
+  a.n = h->n;
   dl::LaunchShape sh = shape_of(h);
   sh.units = units;
-  sh.max_n = n < 0 ? h->max_n : n;
   switch (h->op) {
     case DL_GDN: return dl::launch_materialize_op<dl::OP_GDN>(sh, a, s);
     case DL_KDA: return dl::launch_materialize_op<dl::OP_KDA>(sh, a, s);
@@ -282,32 +240,14 @@ cudaError_t launch_materialize(dl_handle* h, float* out, cudaStream_t s, long un
 
 int do_step(dl_handle* h, const void* q, const void* k, const void* v, const float* log_decay,
             const float* beta, void* o, cudaStream_t s) {
-  int mode;
-  if (h->n >= 0) {
-    mode = h->n + 1 == h->M ? dl::MODE_MERGE : dl::MODE_APPEND;
-  } else {
-    mode = dl::MODE_RAGGED;
-    cudaError_t e = upload_n(h, s);
-    if (e != cudaSuccess) return cuda_fail(e, "per-slot log length upload");
-  }
-  cudaError_t e = launch_step(h, mode, step_args(h, q, k, v, log_decay, beta, o), s);
+  const bool merge = h->n + 1 == h->M;
+  cudaError_t e = launch_step(h, merge ? dl::MODE_MERGE : dl::MODE_APPEND,
+                              step_args(h, q, k, v, log_decay, beta, o), s);
   if (e == cudaErrorNotSupported)
-    return fail(DL_ERR_UNSUPPORTED, "the streaming step kernel cannot run this launch (alignment, shared memory "
-                                    "or slots at different points of their cycles)");
+    return fail(DL_ERR_UNSUPPORTED, "the streaming step kernel cannot run this launch (alignment or shared memory)");
   if (e != cudaSuccess) return cuda_fail(e, "deltalog step launch");
-  bool any_merge = false;
-  for (int& nb : h->nslot) {
-    const bool merge = nb + 1 == h->M;
-    any_merge = any_merge || merge;
-    nb = merge ? 0 : nb + 1;
-  }
-  h->wrote_state = any_merge;
-  if (mode == dl::MODE_RAGGED) {
-    h->cur ^= 1;  // the kernel wrote the new lengths into the other buffer
-  } else {
-    h->n_dev_valid = false;
-  }
-  refresh_n(h);
+  h->n = merge ? 0 : h->n + 1;
+  h->wrote_state = merge;
   return DL_OK;
 }
 
@@ -336,7 +276,6 @@ int dl_create(dl_t* out, int B, int H, int d_k, int d_v, int M, int op, int in_d
   h->op = op;
   h->dtype = in_dtype;
   h->n = 0;
-  h->max_n = 0;
   h->wrote_state = true;
   h->Mcap = M > 1 ? M - 1 : 1;
   h->esize = in_dtype == DL_BF16 ? 2 : 4;
@@ -374,8 +313,6 @@ int dl_create(dl_t* out, int B, int H, int d_k, int d_v, int M, int op, int in_d
       {reinterpret_cast<void**>(&h->logLam), nbh * lam_unit_floats(h) * sizeof(float)},
       {reinterpret_cast<void**>(&h->u), static_cast<size_t>(H) * d_k * sizeof(float)},
       {reinterpret_cast<void**>(&h->err), sizeof(int)},
-      {reinterpret_cast<void**>(&h->n_dev[0]), static_cast<size_t>(B) * sizeof(int)},
-      {reinterpret_cast<void**>(&h->n_dev[1]), static_cast<size_t>(B) * sizeof(int)},
       {&h->st[0].q, nbh * d_k * h->esize},
       {&h->st[0].k, nbh * d_k * h->esize},
       {&h->st[0].v, nbh * d_v * h->esize},
@@ -399,16 +336,7 @@ int dl_create(dl_t* out, int B, int H, int d_k, int d_v, int M, int op, int in_d
                   "cudaMalloc of %zu bytes failed: %s", a.bytes, cudaGetErrorString(e));
     }
   }
-  try {
-    h->nslot.assign(B, 0);
-  } catch (...) {
-    free_all(h);
-    delete h;
-    return fail(DL_ERR_OOM, "host allocation failed");
-  }
-  cudaError_t e = cudaMallocHost(reinterpret_cast<void**>(&h->n_pinned), static_cast<size_t>(B) * sizeof(int));
-  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->n_uploaded, cudaEventDisableTiming);
-  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking);
+  cudaError_t e = cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking);
   for (int j = 0; j < 2 && e == cudaSuccess; ++j) {
     e = cudaEventCreateWithFlags(&h->in_ready[j], cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->set_free[j], cudaEventDisableTiming);
@@ -442,9 +370,7 @@ int dl_load_state(dl_t h, const float* S, void* stream) {
   cudaError_t e = cudaMemcpyAsync(h->Sbar, S, state_bytes(h), cudaMemcpyDeviceToDevice,
                                   static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "dl_load_state copy");
-  std::fill(h->nslot.begin(), h->nslot.end(), 0);
-  refresh_n(h);
-  h->n_dev_valid = false;
+  h->n = 0;
   h->wrote_state = true;
   return DL_OK;
 }
@@ -544,12 +470,9 @@ int dl_merge(dl_t h, void* stream) {
   if (h->n == 0) return DL_OK;
   DeviceScope ds(h->device);
   if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
-  cudaError_t e = launch_materialize(h, h->Sbar, static_cast<cudaStream_t>(stream), 0,
-                                     static_cast<int>(bh(h)), h->n);
+  cudaError_t e = launch_materialize(h, h->Sbar, static_cast<cudaStream_t>(stream), 0, static_cast<int>(bh(h)));
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
-  std::fill(h->nslot.begin(), h->nslot.end(), 0);
-  refresh_n(h);
-  h->n_dev_valid = false;
+  h->n = 0;
   h->wrote_state = true;
   return DL_OK;
 }
@@ -561,7 +484,7 @@ int dl_read_state(dl_t h, float* S_out, void* stream) {
   if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = h->n == 0 ? cudaMemcpyAsync(S_out, h->Sbar, state_bytes(h), cudaMemcpyDeviceToDevice, s)
-                            : launch_materialize(h, S_out, s, 0, static_cast<int>(bh(h)), h->n);
+                            : launch_materialize(h, S_out, s, 0, static_cast<int>(bh(h)));
   return e == cudaSuccess ? DL_OK : cuda_fail(e, "dl_read_state");
 }
 
@@ -575,7 +498,7 @@ int dl_slot_load(dl_t h, int slot, const float* S, void* stream) {
   const size_t bytes = static_cast<size_t>(h->H) * h->dk * h->dv * sizeof(float);
   float* dst = h->Sbar + static_cast<size_t>(slot) * h->H * h->dk * h->dv;
   cudaError_t e = S ? cudaMemcpyAsync(dst, S, bytes, cudaMemcpyDeviceToDevice, s) : cudaMemsetAsync(dst, 0, bytes, s);
-  if (e == cudaSuccess) e = reset_slot_n(h, slot, s);
+  if (e == cudaSuccess && h->n > 0) e = zero_slot_log(h, slot, s);
   if (e != cudaSuccess) return cuda_fail(e, "dl_slot_load");
   h->wrote_state = true;
   return DL_OK;
@@ -584,14 +507,13 @@ int dl_slot_load(dl_t h, int slot, const float* S, void* stream) {
 int dl_slot_merge(dl_t h, int slot, void* stream) {
   if (!h) return fail(DL_ERR_ARG, "null handle");
   if (slot < 0 || slot >= h->B) return fail(DL_ERR_ARG, "slot %d outside [0, %d)", slot, h->B);
-  const int n = h->nslot[slot];
-  if (n == 0) return DL_OK;
+  if (h->n == 0) return DL_OK;
   DeviceScope ds(h->device);
   if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const long unit0 = static_cast<long>(slot) * h->H;
-  cudaError_t e = launch_materialize(h, h->Sbar + unit0 * h->dk * h->dv, s, unit0, h->H, n);
-  if (e == cudaSuccess) e = reset_slot_n(h, slot, s);
+  cudaError_t e = launch_materialize(h, h->Sbar + unit0 * h->dk * h->dv, s, unit0, h->H);
+  if (e == cudaSuccess) e = zero_slot_log(h, slot, s);
   if (e != cudaSuccess) return cuda_fail(e, "dl_slot_merge");
   h->wrote_state = true;
   return DL_OK;
@@ -605,19 +527,11 @@ int dl_slot_read(dl_t h, int slot, float* S_out, void* stream) {
   if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const long unit0 = static_cast<long>(slot) * h->H;
-  const int n = h->nslot[slot];
-  cudaError_t e = n == 0 ? cudaMemcpyAsync(S_out, h->Sbar + unit0 * h->dk * h->dv,
+  cudaError_t e = h->n == 0 ? cudaMemcpyAsync(S_out, h->Sbar + unit0 * h->dk * h->dv,
                                            static_cast<size_t>(h->H) * h->dk * h->dv * sizeof(float),
                                            cudaMemcpyDeviceToDevice, s)
-                         : launch_materialize(h, S_out, s, unit0, h->H, n);
+                            : launch_materialize(h, S_out, s, unit0, h->H);
   return e == cudaSuccess ? DL_OK : cuda_fail(e, "dl_slot_read");
-}
-
-int dl_slot_log_len(dl_t h, int slot, int* n) {
-  if (!h || !n) return fail(DL_ERR_ARG, "null argument");
-  if (slot < 0 || slot >= h->B) return fail(DL_ERR_ARG, "slot %d outside [0, %d)", slot, h->B);
-  *n = h->nslot[slot];
-  return DL_OK;
 }
 
 int dl_set_option(dl_t h, int option, int value) {
@@ -653,7 +567,6 @@ int dl_last_step_kernel(dl_t h, int* kind) {
 
 int dl_log_len(dl_t h, int* n) {
   if (!h || !n) return fail(DL_ERR_ARG, "null argument");
-  if (h->n < 0) return fail(DL_ERR_STATE, "slots hold logs of different lengths; use dl_slot_log_len");
   *n = h->n;
   return DL_OK;
 }

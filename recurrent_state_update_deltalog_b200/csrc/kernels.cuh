@@ -53,17 +53,14 @@ struct StepArgs {
   float* logLam;           // [BH][gdn_lam_stride(Mcap)] (GDN) or [BH][Mcap][DK]
   const float* u;          // [H][DK] (RWKV6)
   int* err;               // device error word (kErr* bits)
-  const int* n_in;         // ragged launches: log length per slot before this step [B]
-  int* n_out;              // ragged launches: log length per slot after this step [B]
   int H;
   int M;                   // merge interval
   int Mcap;                // log capacity per (slot, head), >= 1
   int n;                   // entries in the log before this step (lockstep launches)
 };
 
-// Step kernel modes: every slot appends, every slot merges, or each slot
-// decides from its own log length (slots admitted at different times).
-enum { MODE_APPEND = 0, MODE_MERGE = 1, MODE_RAGGED = 2 };
+// Step kernel modes: every slot appends, or every slot merges.
+enum { MODE_APPEND = 0, MODE_MERGE = 1 };
 
 // Arguments of log materialisation: Sout = Sbar + replayed log, for the
 // units [unit0, unit0 + gridDim.x); Sout points at the first of them.
@@ -74,7 +71,6 @@ struct MaterializeArgs {
   const void* logB;
   const float* logLam;
   int* err;
-  const int* n_slot;   // per-slot log length, or null: every unit has n entries
   long unit0;
   int H;
   int Mcap;
@@ -215,10 +211,7 @@ __device__ __forceinline__ bool wait_log(uint64_t* bar, int n, int* err) {
 
 // ---------------------------------------------------------------------------
 // Deferred step.  MODE_APPEND: every slot appends (Sbar read only).
-// MODE_MERGE: every slot is at n+1 == M; it also writes S_t over Sbar.
-// MODE_RAGGED: slots sit at different points of their cycles; each CTA reads
-// its slot's n, merges when n+1 == M, and the slot's first CTA records the
-// slot's new log length.  NSPLIT > 1 splits each head's
+// MODE_MERGE: every slot is at n+1 == M; it also writes S_t over Sbar.  NSPLIT > 1 splits each head's
 // d_v columns into NSPLIT value tiles, one CTA each (grid B*H*NSPLIT); every
 // tile recomputes the head's ReplayPrep coefficients and the first tile
 // appends the key-side entry.
@@ -249,9 +242,8 @@ deltalog_step_kernel(const StepArgs a) {
   const long sh = blockIdx.x / NSPLIT;
   const int col0 = (blockIdx.x % NSPLIT) * DVT;  // first value column of this tile
   const int h = static_cast<int>(sh % a.H);
-  const int n = MODE == MODE_RAGGED ? a.n_in[sh / a.H] : a.n;
-  const bool MERGE = MODE == MODE_MERGE || (MODE == MODE_RAGGED && n + 1 == a.M);
-  if (MODE == MODE_RAGGED && h == 0 && col0 == 0 && threadIdx.x == 0) a.n_out[sh / a.H] = MERGE ? 0 : n + 1;
+  const int n = a.n;
+  constexpr bool MERGE = MODE == MODE_MERGE;
 
   const TI* sA = reinterpret_cast<const TI*>(s_dyn);
   const float* sL = reinterpret_cast<const float*>(s_dyn + LL::a_bytes(n));
@@ -586,7 +578,7 @@ materialize_kernel(const MaterializeArgs a) {
   const int lane = tid & 31, warp = tid >> 5;
   const int c4 = tid % TL::TPR, rg = tid / TL::TPR;
   const long sh = a.unit0 + blockIdx.x;
-  const int n = a.n_slot ? a.n_slot[sh / a.H] : a.n;
+  const int n = a.n;
 
   const TI* sA = reinterpret_cast<const TI*>(s_dyn);
   const float* sL = reinterpret_cast<const float*>(s_dyn + LL::a_bytes(n));

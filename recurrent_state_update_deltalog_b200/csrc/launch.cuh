@@ -25,7 +25,7 @@ struct LaunchShape {
   bool aligned16;  // q, k, v, o (and per-key log_decay) 16-byte aligned (bulk-copy sources)
   bool pdl;        // launch the step as a programmatic dependent of the previous kernel
   int split;       // value tiles per head for the register-tile step kernel (1, 2 or 4)
-  int max_n;       // longest log of any launched unit (shared-memory sizing)
+  int max_n;       // log length of the launched units (shared-memory sizing)
   int units;       // materialisation: units in the launch
 };
 
@@ -116,8 +116,7 @@ template <int OP, int DK, int DV, typename TI, int MODE, int NSPLIT>
 cudaError_t register_step_mode(const LaunchShape& s, const StepArgs& a, cudaStream_t st) {
   using TL = Tile<DK, DV / NSPLIT>;
   using LL = LogLayout<OP, DK, DV, TI>;
-  // a ragged launch sizes shared memory for its longest log, as a merge
-  const size_t smem = MODE == MODE_RAGGED ? LL::step_smem(s.max_n, true) : LL::step_smem(a.n, MODE == MODE_MERGE);
+  const size_t smem = LL::step_smem(a.n, MODE == MODE_MERGE);
   auto kern = deltalog_step_kernel<OP, DK, DV, TI, MODE, NSPLIT>;
   cudaError_t e = allow_smem(kern, smem, LL::step_smem(kMaxM - 1, MODE != MODE_APPEND));
   if (e != cudaSuccess) return e;
@@ -126,17 +125,15 @@ cudaError_t register_step_mode(const LaunchShape& s, const StepArgs& a, cudaStre
 
 template <int OP, int DK, int DV, typename TI, int NSPLIT>
 cudaError_t register_step(const LaunchShape& s, int mode, const StepArgs& a, cudaStream_t st) {
-  if (mode == MODE_APPEND) return register_step_mode<OP, DK, DV, TI, MODE_APPEND, NSPLIT>(s, a, st);
   if (mode == MODE_MERGE) return register_step_mode<OP, DK, DV, TI, MODE_MERGE, NSPLIT>(s, a, st);
-  return register_step_mode<OP, DK, DV, TI, MODE_RAGGED, NSPLIT>(s, a, st);
+  return register_step_mode<OP, DK, DV, TI, MODE_APPEND, NSPLIT>(s, a, st);
 }
 
 template <int OP, int DK, int DV, typename TI>
 cudaError_t step_dims(const LaunchShape& s, int mode, const StepArgs& a, cudaStream_t st, int* used) {
   // AUTO runs the register-tile kernel, the faster of the two on B200 for
-  // every operator's merge launches and for d_v = 64; STREAM is opt-in and
-  // runs lockstep launches only.
-  if (s.variant == STEP_STREAM && s.aligned16 && mode != MODE_RAGGED) {
+  // every operator's merge launches and for d_v = 64; STREAM is opt-in.
+  if (s.variant == STEP_STREAM && s.aligned16) {
     bool launched = false;
     cudaError_t e = mode == MODE_MERGE ? stream_dims<OP, DK, DV, TI, true>(s, a, st, &launched)
                                        : stream_dims<OP, DK, DV, TI, false>(s, a, st, &launched);

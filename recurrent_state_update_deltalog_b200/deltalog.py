@@ -180,11 +180,6 @@ class DeltaLog:
         N.call("dl_slot_read", self._h, int(slot), _ptr(out), self._stream(stream))
         return out
 
-    def slot_log_len(self, slot):
-        n = ctypes.c_int()
-        N.call("dl_slot_log_len", self._h, int(slot), ctypes.byref(n))
-        return n.value
-
     def check_device(self, stream=None):
         N.call("dl_check_device", self._h, self._stream(stream))
 

@@ -78,7 +78,6 @@ def test_null_handle_paths(lib):
     assert lib.dl_slot_load(None, 0, p, None) == -1
     assert lib.dl_slot_merge(None, 0, None) == -1
     assert lib.dl_slot_read(None, 0, p, None) == -1
-    assert lib.dl_slot_log_len(None, 0, ctypes.byref(ctypes.c_int())) == -1
     n = ctypes.c_int()
     assert lib.dl_log_len(None, ctypes.byref(n)) == -1
     assert lib.dl_destroy(None) == 0

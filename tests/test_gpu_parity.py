@@ -304,7 +304,7 @@ def test_programmatic_launch_gives_identical_results(op):
     assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
 
 
-# ---- per-slot cycles (serving: admit / evict / flush one slot) -----------------
+# ---- per-slot admission (serving: admit / evict / flush one slot) ---------------
 
 def _oracle_step(op, S, seq, t, u):
     """One eager step of every unit (fp64): returns (o_t, S_t)."""
@@ -316,9 +316,11 @@ def _oracle_step(op, S, seq, t, u):
 @pytest.mark.parametrize("op", OPS)
 @pytest.mark.parametrize("dims,M", [((64, 64), 3), ((128, 128), 4), ((128, 128), 8), ((64, 128), 5)])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-def test_ragged_slots(op, dims, M, dtype):
-    """Slots admitted and flushed at different times follow their own cycles."""
-    from recurrent_state_update_deltalog_b200 import DeltaLog, DeltaLogError
+def test_slot_admission(op, dims, M, dtype):
+    """Slots loaded, merged and zeroed mid-cycle keep the handle's log length
+    (their entries are cleared), and every output and state follows the eager
+    recurrence restarted from the loaded state."""
+    from recurrent_state_update_deltalog_b200 import DeltaLog
     from synthetic import initial_state
     B, H, T = 6, 3, 20
     dk, dv = dims
@@ -331,7 +333,7 @@ def test_ragged_slots(op, dims, M, dtype):
     if u is not None:
         h.set_bonus(torch.from_numpy(u).cuda())
     S_ref = S0.astype(np.float64)
-    expect_n = [0] * B
+    n = 0
     events = {2: ("load", 2), 5: ("merge", 4), 7: ("zero", 0), 11: ("load", 1), 13: ("flush", None),
               15: ("load", 5)}
     outs, refs = [], []
@@ -342,28 +344,24 @@ def test_ragged_slots(op, dims, M, dtype):
             if kind == "load":
                 h.slot_load(b, torch.from_numpy(fresh[b]).cuda())
                 S_ref[b] = fresh[b]
-                expect_n[b] = 0
             elif kind == "zero":
                 h.slot_load(b)
                 S_ref[b] = 0
-                expect_n[b] = 0
             elif kind == "merge":
                 h.slot_merge(b)
-                expect_n[b] = 0
             else:
                 got = h.read_state().cpu().numpy()
                 assert relerr(got, S_ref) < tol
                 h.merge()
-                expect_n = [0] * B
-        assert [h.slot_log_len(b) for b in range(B)] == expect_n
-        if len(set(expect_n)) > 1:
-            with pytest.raises(DeltaLogError):
-                h.log_len
+                n = 0
+            if b is not None:                                  # the slot reads back as set
+                assert relerr(h.slot_read(b).cpu().numpy(), S_ref[b]) < tol, (t, b)
+        assert h.log_len == n
         o = h.step(*step_args(op, dseq, t))
         outs.append(o.float().cpu().numpy())
         o_ref, S_ref = _oracle_step(op, S_ref, seq, t, u)
         refs.append(o_ref)
-        expect_n = [0 if n + 1 == M else n + 1 for n in expect_n]
+        n = 0 if n + 1 == M else n + 1
         if t in (8, 16):
             for b in (0, 3):
                 assert relerr(h.slot_read(b).cpu().numpy(), S_ref[b]) < tol, (t, b)
