@@ -55,6 +55,9 @@ def parse():
                     help="dl_step kernel variant")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch every step with plain stream ordering")
+    ap.add_argument("--slot-map", action="store_true",
+                    help="run every token through the slot index map: batch row r on slot perm_t[r], "
+                         "a fresh random permutation of the B slots per pool token")
     ap.add_argument("--admit-every", type=int, default=0, metavar="K",
                     help="re-admit one slot (dl_slot_load of a fresh state, round robin) every K "
                          "tokens inside the timed region (serving churn; 0 = off)")
@@ -341,6 +344,13 @@ def run_gpu(a, rank, world, local_rank):
         return (pool[first][i], pool["k"][i], pool["v"][i], pool["log_decay"][i],
                 pool["beta"][i] if op != "rwkv6" else None)
 
+    perm_rng = np.random.default_rng(seed + 17)
+    sidx = ([torch.from_numpy(perm_rng.permutation(B).astype(np.int32)).to(dev) for _ in range(a.pool)]
+            if a.slot_map else None)
+
+    def tok_map(i):
+        return {"slot_idx": sidx[i]} if sidx else {}
+
     def make_handle(m):
         h = DeltaLog(B, H, d, d, m, op=op, dtype=torch.bfloat16)
         h.set_step_kernel(a.kernel)
@@ -369,15 +379,15 @@ def run_gpu(a, rank, world, local_rank):
             tok_counter[0] += 1
             args = tok_args(dpool, i)
             if eager:
-                h.eager_step(*args, out=out[i], stream=stream)
+                h.eager_step(*args, out=out[i], stream=stream, **tok_map(i))
             elif ev is not None and (j % m) != m - 1:
                 e0, e1 = ev.pop()
                 e0.record(stream)
-                h.step(*args, out=out[i], stream=stream)
+                h.step(*args, out=out[i], stream=stream, **tok_map(i))
                 e1.record(stream)
                 rec.append((e0, e1, j % m))
             else:
-                h.step(*args, out=out[i], stream=stream)
+                h.step(*args, out=out[i], stream=stream, **tok_map(i))
             if a.admit_every and not eager and tok_counter[0] % a.admit_every == 0:
                 b = (tok_counter[0] // a.admit_every) % B
                 h.slot_load(b, S0[b], stream=stream)
@@ -396,7 +406,7 @@ def run_gpu(a, rank, world, local_rank):
                     for j in range(cyc):
                         i = (c * cyc + j) % a.pool
                         fn = h.eager_step if eager else h.step
-                        fn(*tok_args(dpool, i), out=out[i], stream=gs)
+                        fn(*tok_args(dpool, i), out=out[i], stream=gs, **tok_map(i))
                 graphs.append(gr)
         torch.cuda.synchronize(dev)
         return graphs, cyc
@@ -551,6 +561,7 @@ def run_gpu(a, rank, world, local_rank):
                    "step_kernel": used_kernel[0], "pdl": not a.no_pdl,
                    "launch": "cuda graph per cycle" if a.graph else "python loop",
                    "admit_every_tokens": a.admit_every or None,
+                   "slot_map": "random permutation per token" if a.slot_map else None,
                    "input_pool_tokens": a.pool, "seed": a.seed,
                    "l2": (f"inputs larger than L2 (state {4 * B * H * d * d / 1e6:.0f} MB)"
                           if 4 * B * H * d * d > L2_BYTES else

@@ -103,6 +103,23 @@ int dl_set_bonus(dl_t h, const float* u, void* stream);
 int dl_step(dl_t h, const void* q, const void* k, const void* v,
             const float* log_decay, const float* beta, void* o, void* stream);
 
+/* dl_step over a subset of the slots, in any order (a serving batch over a
+ * state pool of B slots).  Batch row r (0 <= r < rows <= B) runs on slot
+ * slot_idx[r]: q, k, v, o, log_decay and beta are [rows][H][...] in the
+ * layouts above, slot_idx is a device int32 array [rows].  A negative index
+ * marks a padding row: nothing is read or written for it, o included.  An
+ * index >= B is skipped the same way and sets DL_DEVERR_SLOT_INDEX in the
+ * device error word (dl_check_device).  Rows must name distinct slots (undefined otherwise).
+ * The step appends or merges every named slot exactly like dl_step.  A slot
+ * that a step does not name receives no log entry, so from then on its state
+ * is undefined until dl_slot_load; every live sequence must be in every step
+ * (one handle per state pool and step sequence).  rows == 0 is a no-op.
+ * DL_STEP_STREAM does not take an index map, and a map has at most 65535
+ * rows (DL_ERR_UNSUPPORTED otherwise). */
+int dl_step_indexed(dl_t h, const int* slot_idx, int rows, const void* q, const void* k,
+                    const void* v, const float* log_decay, const float* beta, void* o,
+                    void* stream);
+
 /* Same as dl_step with HOST pointers (pinned or pageable): copies the inputs
  * into handle-owned device buffers, runs the step and copies o back.  Inputs
  * must stay valid, and o is valid, once `stream` has reached the call.  By
@@ -122,6 +139,13 @@ int dl_step_host(dl_t h, const void* q, const void* k, const void* v,
  * dl_merge). */
 int dl_eager_step(dl_t h, const void* q, const void* k, const void* v,
                   const float* log_decay, const float* beta, void* o, void* stream);
+
+/* dl_eager_step over batch rows on the slots slot_idx[0..rows), with the
+ * conventions of dl_step_indexed (padding rows, index errors, distinct
+ * slots).  Slots not named keep their state. */
+int dl_eager_step_indexed(dl_t h, const int* slot_idx, int rows, const void* q, const void* k,
+                          const void* v, const float* log_decay, const float* beta, void* o,
+                          void* stream);
 
 /* Fold every slot's log into Sbar now (no output) and empty them; a no-op
  * when all logs are empty.  For an explicit flush or a checkpoint. */
@@ -192,8 +216,14 @@ int dl_slot_load(dl_t h, int slot, const float* S, void* stream);
 int dl_slot_merge(dl_t h, int slot, void* stream);
 int dl_slot_read(dl_t h, int slot, float* S_out, void* stream);
 
+/* Bits of the device error word. */
+enum dl_device_error {
+  DL_DEVERR_WAIT_TIMEOUT = 1,  /* a bounded wait on a log copy gave up; that unit wrote nothing */
+  DL_DEVERR_SLOT_INDEX = 2     /* dl_step_indexed / dl_eager_step_indexed: slot index >= B */
+};
+
 /* Read and clear the handle's device error word (synchronises `stream`).
- * Returns DL_OK or DL_ERR_DEVICE. */
+ * Returns DL_OK, or DL_ERR_DEVICE with the word's bits in the message. */
 int dl_check_device(dl_t h, void* stream);
 
 /* Static text for a status code, and the last error message of this thread. */

@@ -32,8 +32,10 @@ SIGNATURES = {
     "dl_load_state": (_I, [_P, _P, _P]),
     "dl_set_bonus": (_I, [_P, _P, _P]),
     "dl_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
+    "dl_step_indexed": (_I, [_P, _P, _I, _P, _P, _P, _P, _P, _P, _P]),
     "dl_step_host": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
     "dl_eager_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
+    "dl_eager_step_indexed": (_I, [_P, _P, _I, _P, _P, _P, _P, _P, _P, _P]),
     "dl_merge": (_I, [_P, _P]),
     "dl_read_state": (_I, [_P, _P, _P]),
     "dl_set_option": (_I, [_P, _I, _I]),

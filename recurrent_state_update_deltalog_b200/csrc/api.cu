@@ -9,6 +9,9 @@
 #include <new>
 #include <string>
 
+static_assert(DL_DEVERR_WAIT_TIMEOUT == dl::kErrWaitTimeout, "device error bits");
+static_assert(DL_DEVERR_SLOT_INDEX == dl::kErrSlotIndex, "device error bits");
+
 struct dl_handle {
   int B, H, dk, dv, M, op, dtype, device;
   int sms, smem_block_optin, smem_sm, smem_reserved;  // device limits
@@ -118,6 +121,7 @@ void free_all(dl_handle* h) {
 dl::LaunchShape shape_of(const dl_handle* h, bool aligned16 = false) {
   dl::LaunchShape s;
   s.BH = static_cast<int>(bh(h));
+  s.H = h->H;
   s.dk = h->dk;
   s.dv = h->dv;
   s.dtype = h->dtype;
@@ -155,6 +159,16 @@ int check_step_args(const dl_handle* h, const void* q, const void* k, const void
   return DL_OK;
 }
 
+// A slot index map of `rows` rows; rows == 0 needs no pointer at all.
+int check_slot_map(const dl_handle* h, const int* slot_idx, int rows) {
+  if (!h) return fail(DL_ERR_ARG, "null handle");
+  if (rows < 0 || rows > h->B) return fail(DL_ERR_ARG, "rows=%d outside [0, %d]", rows, h->B);
+  if (rows > 65535) return fail(DL_ERR_UNSUPPORTED, "slot index maps take at most 65535 rows (grid y)");
+  if (rows > 0 && (!slot_idx || !aligned(slot_idx, 4)))
+    return fail(DL_ERR_ARG, "slot index pointer null or not 4-byte aligned");
+  return DL_OK;
+}
+
 dl::StepArgs step_args(dl_handle* h, const void* q, const void* k, const void* v,
                        const float* log_decay, const float* beta, void* o) {
   dl::StepArgs a;
@@ -165,6 +179,8 @@ dl::StepArgs step_args(dl_handle* h, const void* q, const void* k, const void* v
   a.log_decay = log_decay;
   a.beta = beta;
   a.o = o;
+  a.slot_idx = nullptr;
+  a.slots = h->B;
   a.logA = h->logA;
   a.logB = h->logB;
   a.logLam = h->logLam;
@@ -193,11 +209,13 @@ cudaError_t zero_slot_log(const dl_handle* h, int b, cudaStream_t s) {
   return e;
 }
 
-cudaError_t launch_step(dl_handle* h, int mode, const dl::StepArgs& a, cudaStream_t s) {
+// `rows` batch rows of H units each are launched (B without an index map).
+cudaError_t launch_step(dl_handle* h, int mode, const dl::StepArgs& a, int rows, cudaStream_t s) {
   // bulk-copy sources of the streaming kernel (GDN's scalar gate is a plain load)
   const bool al = aligned(a.q, 16) && aligned(a.k, 16) && aligned(a.v, 16) && aligned(a.o, 16) &&
                   (h->op == DL_GDN || aligned(a.log_decay, 16));
-  const dl::LaunchShape sh = shape_of(h, al);
+  dl::LaunchShape sh = shape_of(h, al);
+  sh.BH = rows * h->H;
   int* used = &h->last_kernel;
   switch (h->op) {
     case DL_GDN: return dl::launch_step_op<dl::OP_GDN>(sh, mode, a, s, used);
@@ -206,8 +224,9 @@ cudaError_t launch_step(dl_handle* h, int mode, const dl::StepArgs& a, cudaStrea
   }
 }
 
-cudaError_t launch_eager(const dl_handle* h, const dl::StepArgs& a, cudaStream_t s) {
-  const dl::LaunchShape sh = shape_of(h);
+cudaError_t launch_eager(const dl_handle* h, const dl::StepArgs& a, int rows, cudaStream_t s) {
+  dl::LaunchShape sh = shape_of(h);
+  sh.BH = rows * h->H;
   switch (h->op) {
     case DL_GDN: return dl::launch_eager_op<dl::OP_GDN>(sh, a, s);
     case DL_KDA: return dl::launch_eager_op<dl::OP_KDA>(sh, a, s);
@@ -238,13 +257,17 @@ cudaError_t launch_materialize(const dl_handle* h, float* out, cudaStream_t s, l
   }
 }
 
-int do_step(dl_handle* h, const void* q, const void* k, const void* v, const float* log_decay,
-            const float* beta, void* o, cudaStream_t s) {
+// One token: `rows` batch rows, row r on slot idx[r] (row r itself when idx
+// is null).
+int do_step(dl_handle* h, const int* idx, int rows, const void* q, const void* k, const void* v,
+            const float* log_decay, const float* beta, void* o, cudaStream_t s) {
   const bool merge = h->n + 1 == h->M;
-  cudaError_t e = launch_step(h, merge ? dl::MODE_MERGE : dl::MODE_APPEND,
-                              step_args(h, q, k, v, log_decay, beta, o), s);
+  dl::StepArgs a = step_args(h, q, k, v, log_decay, beta, o);
+  a.slot_idx = idx;
+  cudaError_t e = launch_step(h, merge ? dl::MODE_MERGE : dl::MODE_APPEND, a, rows, s);
   if (e == cudaErrorNotSupported)
-    return fail(DL_ERR_UNSUPPORTED, "the streaming step kernel cannot run this launch (alignment or shared memory)");
+    return fail(DL_ERR_UNSUPPORTED, "the streaming step kernel cannot run this launch (alignment, shared memory "
+                                    "or a slot index map)");
   if (e != cudaSuccess) return cuda_fail(e, "deltalog step launch");
   h->n = merge ? 0 : h->n + 1;
   h->wrote_state = merge;
@@ -392,7 +415,18 @@ int dl_step(dl_t h, const void* q, const void* k, const void* v, const float* lo
   if (rc != DL_OK) return rc;
   DeviceScope ds(h->device);
   if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
-  return do_step(h, q, k, v, log_decay, beta, o, static_cast<cudaStream_t>(stream));
+  return do_step(h, nullptr, h->B, q, k, v, log_decay, beta, o, static_cast<cudaStream_t>(stream));
+}
+
+int dl_step_indexed(dl_t h, const int* slot_idx, int rows, const void* q, const void* k, const void* v,
+                    const float* log_decay, const float* beta, void* o, void* stream) {
+  int rc = check_slot_map(h, slot_idx, rows);
+  if (rc != DL_OK || rows == 0) return rc;
+  rc = check_step_args(h, q, k, v, log_decay, beta, o);
+  if (rc != DL_OK) return rc;
+  DeviceScope ds(h->device);
+  if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
+  return do_step(h, slot_idx, rows, q, k, v, log_decay, beta, o, static_cast<cudaStream_t>(stream));
 }
 
 int dl_step_host(dl_t h, const void* q, const void* k, const void* v, const float* log_decay,
@@ -442,7 +476,7 @@ int dl_step_host(dl_t h, const void* q, const void* k, const void* v, const floa
     o_dev = pa.devicePointer;
   else
     cudaGetLastError();  // pageable memory reports an error on some drivers
-  rc = do_step(h, st.q, st.k, st.v, st.ld, beta ? st.beta : nullptr, o_dev ? o_dev : st.o, s);
+  rc = do_step(h, nullptr, h->B, st.q, st.k, st.v, st.ld, beta ? st.beta : nullptr, o_dev ? o_dev : st.o, s);
   if (rc != DL_OK) return rc;
   if (!o_dev) e = cudaMemcpyAsync(o, st.o, nbh * h->dv * h->esize, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess && h->host_prefetch) e = cudaEventRecord(h->set_free[j], s);
@@ -459,7 +493,26 @@ int dl_eager_step(dl_t h, const void* q, const void* k, const void* v, const flo
   if (h->n != 0) return fail(DL_ERR_STATE, "eager step needs every slot's log empty; call dl_merge");
   DeviceScope ds(h->device);
   if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
-  cudaError_t e = launch_eager(h, step_args(h, q, k, v, log_decay, beta, o), static_cast<cudaStream_t>(stream));
+  cudaError_t e =
+      launch_eager(h, step_args(h, q, k, v, log_decay, beta, o), h->B, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "eager step launch");
+  h->wrote_state = true;
+  return DL_OK;
+}
+
+int dl_eager_step_indexed(dl_t h, const int* slot_idx, int rows, const void* q, const void* k, const void* v,
+                          const float* log_decay, const float* beta, void* o, void* stream) {
+  int rc = check_slot_map(h, slot_idx, rows);
+  if (rc != DL_OK) return rc;
+  if (h->n != 0) return fail(DL_ERR_STATE, "eager step needs every slot's log empty; call dl_merge");
+  if (rows == 0) return DL_OK;
+  rc = check_step_args(h, q, k, v, log_decay, beta, o);
+  if (rc != DL_OK) return rc;
+  DeviceScope ds(h->device);
+  if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
+  dl::StepArgs a = step_args(h, q, k, v, log_decay, beta, o);
+  a.slot_idx = slot_idx;
+  cudaError_t e = launch_eager(h, a, rows, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "eager step launch");
   h->wrote_state = true;
   return DL_OK;

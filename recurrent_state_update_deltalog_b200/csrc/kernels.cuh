@@ -40,14 +40,18 @@ namespace dl {
 enum { OP_GDN = 0, OP_KDA = 1, OP_RWKV6 = 2 };
 
 // Arguments of one deferred step (device pointers; sizes in elements).
+// Units: a pool unit (slot, head) owns Sbar and log storage; a batch unit
+// (row, head) owns inputs and outputs.  Without an index map, row b is slot b.
 struct StepArgs {
-  float* Sbar;             // [BH][DK][DV]
-  const void* q;           // [BH][DK] (r for RWKV6), input dtype
-  const void* k;           // [BH][DK]
-  const void* v;           // [BH][DV]
-  const float* log_decay;  // [BH] (GDN) or [BH][DK]
-  const float* beta;       // [BH] (GDN/KDA)
-  void* o;                 // [BH][DV], input dtype
+  float* Sbar;             // [BH][DK][DV]                 pool units
+  const void* q;           // [rows*H][DK] (r for RWKV6), input dtype   batch units
+  const void* k;           // [rows*H][DK]
+  const void* v;           // [rows*H][DV]
+  const float* log_decay;  // [rows*H] (GDN) or [rows*H][DK]
+  const float* beta;       // [rows*H] (GDN/KDA)
+  void* o;                 // [rows*H][DV], input dtype
+  const int* slot_idx;     // [rows] pool slot of each batch row (< 0: padding), or null
+  int slots;               // pool slots B (bound of slot_idx)
   void* logA;              // [BH][Mcap][DK], input dtype (a_i = k_i)
   void* logB;              // [BH][Mcap][DV], fp32 (GDN/KDA) or input dtype (RWKV6)
   float* logLam;           // [BH][gdn_lam_stride(Mcap)] (GDN) or [BH][Mcap][DK]
@@ -61,6 +65,43 @@ struct StepArgs {
 
 // Step kernel modes: every slot appends, or every slot merges.
 enum { MODE_APPEND = 0, MODE_MERGE = 1 };
+
+// Device error bit: a slot index at or past the pool size (the row is skipped).
+constexpr int kErrSlotIndex = 2;
+
+// Which unit a CTA of a step kernel serves.  `bu` (row * H + head) indexes
+// inputs and outputs, `sh` (slot * H + head) the state and the log, `col0` is
+// the tile's first value column.  Unmapped launches: a 1-D grid of
+// B * H * NSPLIT CTAs and sh == bu.  Mapped launches (template switch, so the
+// unmapped kernels carry none of it): grid (H * NSPLIT, rows), row r on slot
+// slot_idx[r]; ok is false for a padding row (negative index) and for an
+// index past the pool, which also raises kErrSlotIndex.
+struct UnitIx {
+  long bu, sh;
+  int h, col0;
+  bool ok;
+};
+
+template <int NSPLIT, int DVT, bool MAP>
+__device__ __forceinline__ UnitIx unit_of(const StepArgs& a) {
+  UnitIx u;
+  if constexpr (MAP) {
+    u.h = static_cast<int>(blockIdx.x) / NSPLIT;
+    u.col0 = (static_cast<int>(blockIdx.x) % NSPLIT) * DVT;
+    u.bu = static_cast<long>(blockIdx.y) * a.H + u.h;
+    const int slot = __ldg(a.slot_idx + blockIdx.y);
+    u.ok = slot >= 0 && slot < a.slots;
+    if (slot >= a.slots && threadIdx.x == 0) atomicOr(a.err, kErrSlotIndex);
+    u.sh = static_cast<long>(slot) * a.H + u.h;
+  } else {
+    u.bu = blockIdx.x / NSPLIT;
+    u.col0 = (blockIdx.x % NSPLIT) * DVT;
+    u.h = static_cast<int>(u.bu % a.H);  // only RWKV6 reads it
+    u.sh = u.bu;
+    u.ok = true;
+  }
+  return u;
+}
 
 // Arguments of log materialisation: Sout = Sbar + replayed log, for the
 // units [unit0, unit0 + gridDim.x); Sout points at the first of them.
@@ -216,7 +257,7 @@ __device__ __forceinline__ bool wait_log(uint64_t* bar, int n, int* err) {
 // tile recomputes the head's ReplayPrep coefficients and the first tile
 // appends the key-side entry.
 // ---------------------------------------------------------------------------
-template <int OP, int DK, int DV, typename TI, int MODE, int NSPLIT>
+template <int OP, int DK, int DV, typename TI, int MODE, int NSPLIT, bool MAP>
 __global__ void __launch_bounds__(Tile<DK, DV / NSPLIT>::NT, Tile<DK, DV / NSPLIT>::MINB)
 deltalog_step_kernel(const StepArgs a) {
   constexpr int DVT = DV / NSPLIT;  // value-tile width owned by this CTA
@@ -239,9 +280,12 @@ deltalog_step_kernel(const StepArgs a) {
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const int c4 = tid % TL::TPR, rg = tid / TL::TPR;
-  const long sh = blockIdx.x / NSPLIT;
-  const int col0 = (blockIdx.x % NSPLIT) * DVT;  // first value column of this tile
-  const int h = static_cast<int>(sh % a.H);
+  const UnitIx ux = unit_of<NSPLIT, DVT, MAP>(a);
+  if (!ux.ok) return;
+  const long bu = ux.bu;      // batch unit: inputs and output
+  const long sh = ux.sh;      // pool unit: Sbar and the log
+  const int col0 = ux.col0;   // first value column of this tile
+  const int h = ux.h;
   const int n = a.n;
   constexpr bool MERGE = MODE == MODE_MERGE;
 
@@ -267,8 +311,8 @@ deltalog_step_kernel(const StepArgs a) {
 
   // 2. Key-side values for this lane's keys j = lane + 32 m; GDN's scalar
   // snapshots; per-column v and beta for the finalize threads.
-  const TI* qg = static_cast<const TI*>(a.q) + sh * DK;
-  const TI* kg = static_cast<const TI*>(a.k) + sh * DK;
+  const TI* qg = static_cast<const TI*>(a.q) + bu * DK;
+  const TI* kg = static_cast<const TI*>(a.k) + bu * DK;
   float kr[TL::KPL], qr[TL::KPL], lt[TL::KPL], lp[TL::KPL];
   if (PERKEY) {
     const float* lamp = a.logLam + (sh * a.Mcap + (n > 0 ? n - 1 : 0)) * DK;
@@ -278,12 +322,12 @@ deltalog_step_kernel(const StepArgs a) {
       kr[m] = to_f(kg[j]);
       qr[m] = to_f(qg[j]);
       lp[m] = n > 0 ? lamp[j] : 0.f;
-      lt[m] = lp[m] + a.log_decay[sh * DK + j];
+      lt[m] = lp[m] + a.log_decay[bu * DK + j];
     }
   } else {
     if (tid < n) s_lam[tid] = a.logLam[sh * gdn_lam_stride(a.Mcap) + tid];
     const float lprev = n > 0 ? a.logLam[sh * gdn_lam_stride(a.Mcap) + (n - 1)] : 0.f;
-    const float lcur = lprev + a.log_decay[sh];
+    const float lcur = lprev + a.log_decay[bu];
 #pragma unroll
     for (int m = 0; m < TL::KPL; ++m) {
       const int j = lane + 32 * m;
@@ -296,8 +340,8 @@ deltalog_step_kernel(const StepArgs a) {
   const int c = tid;
   float vc = 0.f, betac = 0.f;
   if (c < DVT) {
-    vc = to_f(static_cast<const TI*>(a.v)[sh * DV + col0 + c]);
-    if (DELTA) betac = a.beta[sh];
+    vc = to_f(static_cast<const TI*>(a.v)[bu * DV + col0 + c]);
+    if (DELTA) betac = a.beta[bu];
   }
   __syncthreads();                              // barrier init and s_lam visible
   if (!wait_log(&s_bar, n, a.err)) return;
@@ -405,7 +449,7 @@ deltalog_step_kernel(const StepArgs a) {
       bt = vc;
     }
     oc = fmaf(s_kappa, bt, oc);
-    static_cast<TI*>(a.o)[sh * DV + col0 + c] = from_f<TI>(oc);
+    static_cast<TI*>(a.o)[bu * DV + col0 + c] = from_f<TI>(oc);
     if (MERGE) {
       Bc[c] = bt;
     } else {
@@ -413,7 +457,7 @@ deltalog_step_kernel(const StepArgs a) {
       if constexpr (DELTA) {
         dstB[c] = bt;
       } else {
-        dstB[c] = static_cast<const TI*>(a.v)[sh * DV + col0 + c];   // raw v, bit copy
+        dstB[c] = static_cast<const TI*>(a.v)[bu * DV + col0 + c];   // raw v, bit copy
       }
     }
   }
@@ -446,7 +490,7 @@ deltalog_step_kernel(const StepArgs a) {
 // Eager dense baseline: S_{t-1} -> S_t read and written every token.  Same
 // tile mapping (and value-tile split) as the deferred step.
 // ---------------------------------------------------------------------------
-template <int OP, int DK, int DV, typename TI, int NSPLIT>
+template <int OP, int DK, int DV, typename TI, int NSPLIT, bool MAP>
 __global__ void __launch_bounds__(Tile<DK, DV / NSPLIT>::NT, Tile<DK, DV / NSPLIT>::MINB)
 eager_step_kernel(const StepArgs a) {
   constexpr int DVT = DV / NSPLIT;  // value-tile width owned by this CTA
@@ -464,9 +508,12 @@ eager_step_kernel(const StepArgs a) {
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const int c4 = tid % TL::TPR, rg = tid / TL::TPR;
-  const long sh = blockIdx.x / NSPLIT;
-  const int col0 = (blockIdx.x % NSPLIT) * DVT;
-  const int h = static_cast<int>(sh % a.H);
+  const UnitIx ux = unit_of<NSPLIT, DVT, MAP>(a);
+  if (!ux.ok) return;
+  const long bu = ux.bu;      // batch unit: inputs and output
+  const long sh = ux.sh;      // pool unit: the state
+  const int col0 = ux.col0;
+  const int h = ux.h;
 
   float* Sp = a.Sbar + sh * (DK * DV);
   float4 st[TL::RPT];
@@ -476,19 +523,19 @@ eager_step_kernel(const StepArgs a) {
   const int c = tid;
   float vc = 0.f, betac = 0.f;
   if (c < DVT) {
-    vc = to_f(static_cast<const TI*>(a.v)[sh * DV + col0 + c]);
-    if (DELTA) betac = a.beta[sh];
+    vc = to_f(static_cast<const TI*>(a.v)[bu * DV + col0 + c]);
+    if (DELTA) betac = a.beta[bu];
   }
 
   if (warp == 0) {
-    const TI* qg = static_cast<const TI*>(a.q) + sh * DK;
-    const TI* kg = static_cast<const TI*>(a.k) + sh * DK;
+    const TI* qg = static_cast<const TI*>(a.q) + bu * DK;
+    const TI* kg = static_cast<const TI*>(a.k) + bu * DK;
     float kap = 0.f;
 #pragma unroll
     for (int m = 0; m < TL::KPL; ++m) {
       const int j = lane + 32 * m;
       const float kj = to_f(kg[j]), qj = to_f(qg[j]);
-      const float dec = expf(OP == OP_GDN ? a.log_decay[sh] : a.log_decay[sh * DK + j]);
+      const float dec = expf(OP == OP_GDN ? a.log_decay[bu] : a.log_decay[bu * DK + j]);
       s_dec[j] = dec;
       s_k[j] = kj;
       if (OP == OP_GDN) {          // p = S^T k, s = S^T q (alpha applied after)
@@ -542,7 +589,7 @@ eager_step_kernel(const StepArgs a) {
       oc = fmaf(s_kappa, vc, s);
     }
     s_b[c] = bt;
-    static_cast<TI*>(a.o)[sh * DV + col0 + c] = from_f<TI>(oc);
+    static_cast<TI*>(a.o)[bu * DV + col0 + c] = from_f<TI>(oc);
   }
   __syncthreads();
 

@@ -12,7 +12,8 @@ namespace dl {
 enum { STEP_AUTO = 0, STEP_REGISTER = 1, STEP_STREAM = 2 };
 
 struct LaunchShape {
-  int BH;     // slots x heads
+  int BH;     // launched (slot or batch row) x heads
+  int H;      // heads
   int dk;
   int dv;
   int dtype;  // 0 = fp32, 1 = bf16 inputs
@@ -31,10 +32,10 @@ struct LaunchShape {
 
 // Launch with the programmatic-stream-serialisation attribute when `pdl`.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_maybe_pdl(void (*kern)(KArgs...), int grid, int block, size_t smem, cudaStream_t st, bool pdl,
+cudaError_t launch_maybe_pdl(void (*kern)(KArgs...), dim3 grid, int block, size_t smem, cudaStream_t st, bool pdl,
                              Args... args) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
+  cfg.gridDim = grid;
   cfg.blockDim = dim3(block);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -112,28 +113,40 @@ cudaError_t allow_smem(K kern, size_t smem, size_t worst) {
   return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(worst));
 }
 
-template <int OP, int DK, int DV, typename TI, int MODE, int NSPLIT>
+// Grid of a step kernel: unmapped B * H * NSPLIT CTAs; mapped (H * NSPLIT, rows).
+template <int NSPLIT, bool MAP>
+dim3 step_grid(const LaunchShape& s) {
+  if (MAP) return dim3(s.H * NSPLIT, s.BH / s.H);
+  return dim3(s.BH * NSPLIT);
+}
+
+template <int OP, int DK, int DV, typename TI, int MODE, int NSPLIT, bool MAP>
 cudaError_t register_step_mode(const LaunchShape& s, const StepArgs& a, cudaStream_t st) {
   using TL = Tile<DK, DV / NSPLIT>;
   using LL = LogLayout<OP, DK, DV, TI>;
   const size_t smem = LL::step_smem(a.n, MODE == MODE_MERGE);
-  auto kern = deltalog_step_kernel<OP, DK, DV, TI, MODE, NSPLIT>;
+  auto kern = deltalog_step_kernel<OP, DK, DV, TI, MODE, NSPLIT, MAP>;
   cudaError_t e = allow_smem(kern, smem, LL::step_smem(kMaxM - 1, MODE != MODE_APPEND));
   if (e != cudaSuccess) return e;
-  return launch_maybe_pdl(kern, s.BH * NSPLIT, TL::NT, smem, st, s.pdl, a);
+  return launch_maybe_pdl(kern, step_grid<NSPLIT, MAP>(s), TL::NT, smem, st, s.pdl, a);
 }
 
 template <int OP, int DK, int DV, typename TI, int NSPLIT>
 cudaError_t register_step(const LaunchShape& s, int mode, const StepArgs& a, cudaStream_t st) {
-  if (mode == MODE_MERGE) return register_step_mode<OP, DK, DV, TI, MODE_MERGE, NSPLIT>(s, a, st);
-  return register_step_mode<OP, DK, DV, TI, MODE_APPEND, NSPLIT>(s, a, st);
+  if (a.slot_idx) {
+    if (mode == MODE_MERGE) return register_step_mode<OP, DK, DV, TI, MODE_MERGE, NSPLIT, true>(s, a, st);
+    return register_step_mode<OP, DK, DV, TI, MODE_APPEND, NSPLIT, true>(s, a, st);
+  }
+  if (mode == MODE_MERGE) return register_step_mode<OP, DK, DV, TI, MODE_MERGE, NSPLIT, false>(s, a, st);
+  return register_step_mode<OP, DK, DV, TI, MODE_APPEND, NSPLIT, false>(s, a, st);
 }
 
 template <int OP, int DK, int DV, typename TI>
 cudaError_t step_dims(const LaunchShape& s, int mode, const StepArgs& a, cudaStream_t st, int* used) {
   // AUTO runs the register-tile kernel, the faster of the two on B200 for
-  // every operator's merge launches and for d_v = 64; STREAM is opt-in.
-  if (s.variant == STEP_STREAM && s.aligned16) {
+  // every operator's merge launches and for d_v = 64; STREAM is opt-in and
+  // takes no slot index map.
+  if (s.variant == STEP_STREAM && s.aligned16 && !a.slot_idx) {
     bool launched = false;
     cudaError_t e = mode == MODE_MERGE ? stream_dims<OP, DK, DV, TI, true>(s, a, st, &launched)
                                        : stream_dims<OP, DK, DV, TI, false>(s, a, st, &launched);
@@ -151,16 +164,21 @@ cudaError_t step_dims(const LaunchShape& s, int mode, const StepArgs& a, cudaStr
   return register_step<OP, DK, DV, TI, 1>(s, mode, a, st);
 }
 
-template <int OP, int DK, int DV, typename TI>
-cudaError_t eager_dims(const LaunchShape& s, const StepArgs& a, cudaStream_t st) {
+template <int OP, int DK, int DV, typename TI, bool MAP>
+cudaError_t eager_map(const LaunchShape& s, const StepArgs& a, cudaStream_t st) {
   if constexpr (DV >= 64) {
     if (s.split == 2) {
-      eager_step_kernel<OP, DK, DV, TI, 2><<<s.BH * 2, Tile<DK, DV / 2>::NT, 0, st>>>(a);
+      eager_step_kernel<OP, DK, DV, TI, 2, MAP><<<step_grid<2, MAP>(s), Tile<DK, DV / 2>::NT, 0, st>>>(a);
       return cudaGetLastError();
     }
   }
-  eager_step_kernel<OP, DK, DV, TI, 1><<<s.BH, Tile<DK, DV>::NT, 0, st>>>(a);
+  eager_step_kernel<OP, DK, DV, TI, 1, MAP><<<step_grid<1, MAP>(s), Tile<DK, DV>::NT, 0, st>>>(a);
   return cudaGetLastError();
+}
+
+template <int OP, int DK, int DV, typename TI>
+cudaError_t eager_dims(const LaunchShape& s, const StepArgs& a, cudaStream_t st) {
+  return a.slot_idx ? eager_map<OP, DK, DV, TI, true>(s, a, st) : eager_map<OP, DK, DV, TI, false>(s, a, st);
 }
 
 template <int OP, int DK, int DV, typename TI>

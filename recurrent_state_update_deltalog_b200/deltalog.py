@@ -64,12 +64,12 @@ class DeltaLog:
     def _decay_shape(self):
         return (self.B, self.H) if self.op == "gdn" else (self.B, self.H, self.d_k)
 
-    def _check_step(self, q, k, v, log_decay, beta, out, cuda):
-        B, H = self.B, self.H
+    def _check_step(self, q, k, v, log_decay, beta, out, cuda, rows=None):
+        B, H = self.B if rows is None else rows, self.H
         self._check("q", q, (B, H, self.d_k), self.dtype, cuda)
         self._check("k", k, (B, H, self.d_k), self.dtype, cuda)
         self._check("v", v, (B, H, self.d_v), self.dtype, cuda)
-        self._check("log_decay", log_decay, self._decay_shape(), torch.float32, cuda)
+        self._check("log_decay", log_decay, (B,) + self._decay_shape()[1:], torch.float32, cuda)
         if self.op == "rwkv6":
             if beta is not None:
                 raise ValueError("beta must be None for rwkv6")
@@ -77,10 +77,19 @@ class DeltaLog:
             self._check("beta", beta, (B, H), torch.float32, cuda)
         self._check("out", out, (B, H, self.d_v), self.dtype, cuda)
 
-    def _alloc_out(self, cuda):
+    def _alloc_out(self, cuda, rows=None):
+        shape = (self.B if rows is None else rows, self.H, self.d_v)
         if cuda:
-            return torch.empty((self.B, self.H, self.d_v), dtype=self.dtype, device=self.device)
-        return torch.empty((self.B, self.H, self.d_v), dtype=self.dtype, pin_memory=True)
+            return torch.empty(shape, dtype=self.dtype, device=self.device)
+        return torch.empty(shape, dtype=self.dtype, pin_memory=True)
+
+    def _slot_map(self, slot_idx):
+        if slot_idx is None:
+            return None
+        if not isinstance(slot_idx, torch.Tensor) or slot_idx.dim() != 1 or slot_idx.numel() > self.B:
+            raise ValueError(f"slot_idx must be 1-D with at most B={self.B} entries")
+        self._check("slot_idx", slot_idx, (slot_idx.numel(),), torch.int32)
+        return slot_idx.numel()
 
     # -- API -----------------------------------------------------------------
     def load_state(self, S, stream=None):
@@ -91,12 +100,21 @@ class DeltaLog:
         self._check("u", u, (self.H, self.d_k), torch.float32)
         N.call("dl_set_bonus", self._h, _ptr(u), self._stream(stream))
 
-    def step(self, q, k, v, log_decay, beta=None, out=None, stream=None):
-        """One DeltaLog decode token (append, or merge on the M-th step); returns o."""
-        out = self._alloc_out(True) if out is None else out
-        self._check_step(q, k, v, log_decay, beta, out, True)
-        N.call("dl_step", self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(beta),
-               _ptr(out), self._stream(stream))
+    def step(self, q, k, v, log_decay, beta=None, out=None, stream=None, slot_idx=None):
+        """One DeltaLog decode token (append, or merge on the M-th step); returns o.
+
+        With ``slot_idx`` (int32 [rows] on the device), inputs and output have
+        ``rows`` batch rows and row r runs on slot ``slot_idx[r]`` (negative:
+        padding row, left untouched); every live slot must be named."""
+        rows = self._slot_map(slot_idx)
+        out = self._alloc_out(True, rows) if out is None else out
+        self._check_step(q, k, v, log_decay, beta, out, True, rows)
+        if rows is None:
+            N.call("dl_step", self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(beta),
+                   _ptr(out), self._stream(stream))
+        else:
+            N.call("dl_step_indexed", self._h, _ptr(slot_idx), rows, _ptr(q), _ptr(k), _ptr(v),
+                   _ptr(log_decay), _ptr(beta), _ptr(out), self._stream(stream))
         return out
 
     def step_host(self, q, k, v, log_decay, beta=None, out=None, stream=None):
@@ -107,12 +125,18 @@ class DeltaLog:
                _ptr(out), self._stream(stream))
         return out
 
-    def eager_step(self, q, k, v, log_decay, beta=None, out=None, stream=None):
-        """Dense baseline: S_{t-1} read and S_t written every token (needs an empty log)."""
-        out = self._alloc_out(True) if out is None else out
-        self._check_step(q, k, v, log_decay, beta, out, True)
-        N.call("dl_eager_step", self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(beta),
-               _ptr(out), self._stream(stream))
+    def eager_step(self, q, k, v, log_decay, beta=None, out=None, stream=None, slot_idx=None):
+        """Dense baseline: S_{t-1} read and S_t written every token (needs an empty log).
+        ``slot_idx`` as in :meth:`step`; slots not named keep their state."""
+        rows = self._slot_map(slot_idx)
+        out = self._alloc_out(True, rows) if out is None else out
+        self._check_step(q, k, v, log_decay, beta, out, True, rows)
+        if rows is None:
+            N.call("dl_eager_step", self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(beta),
+                   _ptr(out), self._stream(stream))
+        else:
+            N.call("dl_eager_step_indexed", self._h, _ptr(slot_idx), rows, _ptr(q), _ptr(k), _ptr(v),
+                   _ptr(log_decay), _ptr(beta), _ptr(out), self._stream(stream))
         return out
 
     def merge(self, stream=None):

@@ -70,6 +70,9 @@ def test_null_handle_paths(lib):
     p = ctypes.c_void_p(16)
     for fn in ("dl_step", "dl_eager_step", "dl_step_host"):
         assert getattr(lib, fn)(None, p, p, p, p, p, p, None) == -1
+    for fn in ("dl_step_indexed", "dl_eager_step_indexed"):
+        assert getattr(lib, fn)(None, p, 1, p, p, p, p, p, p, None) == -1
+        assert getattr(lib, fn)(None, None, 0, None, None, None, None, None, None, None) == -1
     assert lib.dl_merge(None, None) == -1
     assert lib.dl_read_state(None, p, None) == -1
     assert lib.dl_load_state(None, p, None) == -1

@@ -380,3 +380,119 @@ def test_slot_arguments_rejected():
         with pytest.raises(DeltaLogError):
             h.slot_load(bad)
     h.close()
+
+
+# ---- slot index map (serving batch over a state pool) ---------------------------
+
+def _batch(seq, t, idx):
+    """Inputs of step t gathered into batch rows (padding and out-of-range rows
+    take the nearest slot's)."""
+    return {key: val[t:t + 1, np.clip(np.asarray(idx), 0, val.shape[1] - 1)] for key, val in seq.items()}
+
+
+def _run_indexed(op, dims, M, dtype, eager=False):
+    from recurrent_state_update_deltalog_b200 import DeltaLog
+    from synthetic import initial_state
+    B, H, T = 8, 3, 18
+    dk, dv = dims
+    S0, seq, u = make_inputs(op, B, H, dk, dv, T, dtype, seed=3)
+    fresh = initial_state(11, B, H, dk, dv)
+    tol = TOL[dtype]
+    rng = np.random.default_rng(5)
+    h = DeltaLog(B, H, dk, dv, M, op=op, dtype=dtype)
+    h.load_state(torch.from_numpy(S0).cuda())
+    if u is not None:
+        h.set_bonus(torch.from_numpy(u).cuda())
+    S_ref = S0.astype(np.float64)
+    live = [0, 1, 2, 3, 4, 5]
+    events = {4: ("evict", 2), 6: ("admit", 6), 9: ("admit", 2), 11: ("admit", 7), 14: ("evict", 0)}
+    for t in range(T):
+        ev = events.get(t)
+        if ev and ev[0] == "evict":
+            live.remove(ev[1])
+        elif ev:
+            b = ev[1]
+            if eager:   # the dense kernel keeps absent slots as they are; load like a new sequence
+                h.load_state(h.read_state().index_copy_(0, torch.tensor([b], device="cuda"),
+                                                       torch.from_numpy(fresh[b:b + 1]).cuda()))
+            else:
+                h.slot_load(b, torch.from_numpy(fresh[b]).cuda())
+            S_ref[b] = fresh[b]
+            live.append(b)
+        pad = int(rng.integers(0, 3))
+        idx = list(rng.permutation(live)) + [-1] * pad
+        idx = idx[:B]
+        one = _batch(seq, t, idx)
+        dseq = to_device(one, dtype)
+        sentinel = 7.0
+        out = torch.full((len(idx), H, dv), sentinel, dtype=dtype, device="cuda")
+        args = step_args(op, dseq, 0)
+        d_idx = torch.tensor(idx, dtype=torch.int32, device="cuda")
+        (h.eager_step if eager else h.step)(*args, out=out, slot_idx=d_idx)
+        o_all, S_all = _oracle_step(op, S_ref, seq, t, u)
+        got = out.float().cpu().numpy()
+        for r, b in enumerate(idx):
+            if b < 0:
+                assert np.all(got[r] == sentinel), (t, r)
+            else:
+                assert relerr(got[r], o_all[b]) < tol, (t, r, b)
+        S_ref[live] = S_all[live]
+    for b in live:
+        assert relerr(h.slot_read(b).cpu().numpy(), S_ref[b]) < tol, b
+    h.check_device()
+    h.close()
+
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("dims,M", [((64, 64), 3), ((128, 128), 8), ((64, 128), 5)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_slot_index_map(op, dims, M, dtype):
+    """Batch rows on pool slots given by an index map: permuted every token,
+    padding rows untouched, slots evicted (left out) and admitted mid-cycle."""
+    _run_indexed(op, dims, M, dtype)
+
+
+@pytest.mark.parametrize("op", OPS)
+def test_slot_index_map_eager(op):
+    _run_indexed(op, (128, 128), 1, torch.bfloat16, eager=True)
+
+
+def test_slot_index_out_of_range_raises_device_flag():
+    """An index past the pool skips its row and raises the device error word;
+    the other rows are computed as usual."""
+    from recurrent_state_update_deltalog_b200 import DeltaLog, DeltaLogError
+    op, B, H, dk, dv = "gdn", 4, 2, 64, 64
+    S0, seq, u = make_inputs(op, B, H, dk, dv, 1, torch.float32)
+    h = DeltaLog(B, H, dk, dv, 4, op=op, dtype=torch.float32)
+    h.load_state(torch.from_numpy(S0).cuda())
+    idx = [1, 9, 3]
+    dseq = to_device(_batch(seq, 0, idx), torch.float32)
+    out = torch.zeros((3, H, dv), device="cuda")
+    h.step(*step_args(op, dseq, 0), out=out, slot_idx=torch.tensor(idx, dtype=torch.int32, device="cuda"))
+    with pytest.raises(DeltaLogError, match="0x2"):
+        h.check_device()
+    h.check_device()                                   # the word was cleared
+    o_all, _ = _oracle_step(op, S0.astype(np.float64), seq, 0, u)
+    got = out.cpu().numpy()
+    assert relerr(got[0], o_all[1]) < 1e-4 and relerr(got[2], o_all[3]) < 1e-4
+    assert np.all(got[1] == 0)
+    h.close()
+
+
+def test_slot_index_map_arguments():
+    from recurrent_state_update_deltalog_b200 import DeltaLog, DeltaLogError
+    h = DeltaLog(2, 2, 64, 64, 4, op="gdn", dtype=torch.float32)
+    z = torch.zeros((3, 2, 64), device="cuda")
+    g = torch.zeros((3, 2), device="cuda")
+    with pytest.raises(ValueError):                    # more rows than slots
+        h.step(z, z, z, g, g, slot_idx=torch.zeros(3, dtype=torch.int32, device="cuda"))
+    e = torch.empty((0, 2, 64), device="cuda")
+    ge = torch.empty((0, 2), device="cuda")
+    h.step(e, e, e, ge, ge, slot_idx=torch.empty(0, dtype=torch.int32, device="cuda"))  # no-op
+    assert h.log_len == 0
+    h.set_step_kernel("stream")
+    one = torch.zeros((1, 2, 64), device="cuda")
+    with pytest.raises(DeltaLogError):
+        h.step(one, one, one, torch.zeros((1, 2), device="cuda"), torch.zeros((1, 2), device="cuda"),
+               slot_idx=torch.zeros(1, dtype=torch.int32, device="cuda"))
+    h.close()
