@@ -43,7 +43,8 @@ def parse():
     ap.add_argument("--B", type=int, default=256)
     ap.add_argument("--H", type=int, default=32)
     ap.add_argument("--dk", dest="d", type=int, default=128, help="d_k = d_v")
-    ap.add_argument("--M", type=int, default=8)
+    ap.add_argument("--M", type=int, default=8,
+                    help="merge interval; 0 = the library's choice for the op and shape (dl_suggest_m)")
     ap.add_argument("--tokens", type=int, default=256, help="decode tokens per bench step")
     ap.add_argument("--pool", type=int, default=64, help="distinct input tokens kept on device")
     ap.add_argument("--seed", type=int, default=0)
@@ -71,6 +72,11 @@ def parse():
         return args
     if args.admit_every and args.graph:
         ap.error("--admit-every runs the Python launch loop")
+    args.m_auto = args.M == 0
+    if args.m_auto:
+        from recurrent_state_update_deltalog_b200 import suggest_m
+        args.M = suggest_m(args.op, args.d, args.d)
+        args.tokens = -(-args.tokens // args.M) * args.M
     if args.tokens % args.M:
         ap.error("--tokens must be a multiple of --M")
     return args
@@ -560,6 +566,7 @@ def run_gpu(a, rank, world, local_rank):
                    "M": M, "state": "fp32", "inputs": "bf16", "tokens_per_step": a.tokens,
                    "step_kernel": used_kernel[0], "pdl": not a.no_pdl,
                    "launch": "cuda graph per cycle" if a.graph else "python loop",
+                   "m_choice": "dl_suggest_m" if getattr(a, "m_auto", False) else "given",
                    "admit_every_tokens": a.admit_every or None,
                    "slot_map": "random permutation per token" if a.slot_map else None,
                    "input_pool_tokens": a.pool, "seed": a.seed,
@@ -590,8 +597,7 @@ def run_grid(a, rank, world, local_rank):
             p.B, p.M, p.graph = B, M, True
             p.no_e2e, p.no_cpu, p.no_eager, p.sweep = True, True, True, ""
             p.eager_headline = M == 1
-            if p.tokens % M:
-                continue
+            p.tokens = -(-a.tokens // M) * M   # whole merge cycles per step
             line = run_gpu(p, rank, world, local_rank)
             if line is not None:
                 line["config"]["grid_point"] = {"B": B, "M": M, "kernel": "eager" if M == 1 else "deltalog"}

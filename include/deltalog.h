@@ -75,14 +75,34 @@ enum dl_status {
 };
 
 /* Create a handle for B slots x H heads.  Supported: d_k, d_v in {64, 128},
- * 1 <= M <= DL_MAX_M.  The base state starts at zero with an empty log; the
- * RWKV6 bonus starts at zero.  Pointers passed later must be aligned to their
- * element size (state pointers to 16 bytes); q, k, v, o (and per-key
- * log_decay) aligned to 16 bytes let dl_step use its streaming kernel.
- * M = 1 makes every step a merge step (the deferred path then performs the
- * eager schedule). */
+ * 1 <= M <= DL_MAX_M, or M = DL_M_AUTO for dl_suggest_m's choice (read it
+ * back with dl_merge_interval).  The base state starts at zero with an empty
+ * log; the RWKV6 bonus starts at zero.  Pointers passed later must be aligned
+ * to their element size (state pointers to 16 bytes); q, k, v, o (and
+ * per-key log_decay) aligned to 16 bytes let dl_step use its streaming
+ * kernel.  M = 1 makes every step a merge step (the deferred path then
+ * performs the eager schedule). */
 #define DL_MAX_M 64
+#define DL_M_AUTO 0
 int dl_create(dl_t* out, int B, int H, int d_k, int d_v, int M, int op, int in_dtype);
+
+/* Merge interval for an operator and head shape (no handle, no device).
+ * The pages put the best M where the replay reads of a growing log balance
+ * the saved dense writes (DeltaLog technical summary, gist.science, traffic
+ * model).  Per (slot, head) and token, with S = 4 d_k d_v state bytes and e
+ * log-entry bytes (a_i, b_i, Lam_i in their stored types), a cycle of M
+ * tokens costs about
+ *     f(M) = S/M + e (M-1)/M + rho (M-1)/2      (plus terms without M)
+ * bytes: the merge write, the appended entries, and the replay of
+ * 0 + 1 + ... + (M-1) entries at rho byte-equivalents each.  rho = e
+ * c(op, d_k, d_v), where c is the replay cost per entry over its bytes as
+ * measured on B200 for the square shapes (c = 1, pure traffic, for d_k !=
+ * d_v).  Writes the M in [2, DL_MAX_M] that minimises f.  DL_ERR_ARG for an
+ * unsupported op, shape or dtype, or a NULL M. */
+int dl_suggest_m(int op, int d_k, int d_v, int in_dtype, int* M);
+
+/* The handle's merge interval (the one chosen when created with DL_M_AUTO). */
+int dl_merge_interval(dl_t h, int* M);
 
 /* Free everything the handle owns.  Synchronises the handle's device first.
  * NULL is accepted and ignored. */

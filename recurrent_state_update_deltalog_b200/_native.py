@@ -15,6 +15,7 @@ DL_GDN, DL_KDA, DL_RWKV6 = 0, 1, 2
 DL_F32, DL_BF16 = 0, 1
 DL_OK = 0
 DL_MAX_M = 64
+DL_M_AUTO = 0
 DL_OPT_STEP_KERNEL = 0
 DL_OPT_HOST_PREFETCH = 1
 DL_OPT_PDL = 2
@@ -31,6 +32,8 @@ SIGNATURES = {
     "dl_destroy": (_I, [_P]),
     "dl_load_state": (_I, [_P, _P, _P]),
     "dl_set_bonus": (_I, [_P, _P, _P]),
+    "dl_suggest_m": (_I, [_I, _I, _I, _I, ctypes.POINTER(_I)]),
+    "dl_merge_interval": (_I, [_P, ctypes.POINTER(_I)]),
     "dl_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
     "dl_step_indexed": (_I, [_P, _P, _I, _P, _P, _P, _P, _P, _P, _P]),
     "dl_step_host": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),

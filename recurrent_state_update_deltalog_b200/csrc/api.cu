@@ -274,19 +274,77 @@ int do_step(dl_handle* h, const int* idx, int rows, const void* q, const void* k
   return DL_OK;
 }
 
+// Replay cost of one log entry over its bytes, c(op, d_k, d_v), measured on
+// B200 for the square shapes: a fine M sweep (4..16) per shape, fitted with
+// the cost model of dl_suggest_m (residuals under 1%).  It exceeds 1 where the
+// replay's arithmetic, repeated per value tile, outweighs its bytes.  Mixed
+// shapes take the pure traffic model (1).
+double replay_cost_ratio(int op, int dk, int dv) {
+  if (dk != dv) return 1.0;
+  const bool big = dk == 128;
+  switch (op) {
+    case DL_GDN: return big ? 2.17 : 1.06;
+    case DL_KDA: return big ? 1.48 : 1.16;
+    default: return big ? 1.39 : 1.0;
+  }
+}
+
+// Bytes of one log entry: a_i (input dtype), b_i (fp32, raw v for RWKV6), Lam_i.
+double entry_bytes(int op, int dk, int dv, int esize) {
+  const double a = static_cast<double>(dk) * esize;
+  const double b = static_cast<double>(dv) * (op == DL_RWKV6 ? esize : 4);
+  const double lam = op == DL_GDN ? 4.0 : 4.0 * dk;
+  return a + b + lam;
+}
+
+int suggest_m(int op, int dk, int dv, int esize) {
+  const double S = 4.0 * dk * dv;
+  const double e = entry_bytes(op, dk, dv, esize);
+  const double rho = e * replay_cost_ratio(op, dk, dv);
+  int best = 2;
+  double fbest = 0.0;
+  for (int M = 2; M <= DL_MAX_M; ++M) {
+    const double f = S / M + e * (M - 1) / M + rho * (M - 1) / 2.0;
+    if (M == 2 || f < fbest) {
+      best = M;
+      fbest = f;
+    }
+  }
+  return best;
+}
+
 }  // namespace
 
 extern "C" {
+
+int dl_suggest_m(int op, int d_k, int d_v, int in_dtype, int* M) {
+  if (!M) return fail(DL_ERR_ARG, "null output pointer");
+  if (op < DL_GDN || op > DL_RWKV6) return fail(DL_ERR_ARG, "unknown op %d", op);
+  if (in_dtype != DL_F32 && in_dtype != DL_BF16) return fail(DL_ERR_ARG, "unknown dtype %d", in_dtype);
+  if ((d_k != 64 && d_k != 128) || (d_v != 64 && d_v != 128))
+    return fail(DL_ERR_ARG, "d_k=%d d_v=%d not in {64,128}", d_k, d_v);
+  *M = suggest_m(op, d_k, d_v, in_dtype == DL_BF16 ? 2 : 4);
+  return DL_OK;
+}
+
+int dl_merge_interval(dl_t h, int* M) {
+  if (!h || !M) return fail(DL_ERR_ARG, "null argument");
+  *M = h->M;
+  return DL_OK;
+}
+
 
 int dl_create(dl_t* out, int B, int H, int d_k, int d_v, int M, int op, int in_dtype) {
   if (!out) return fail(DL_ERR_ARG, "null output handle pointer");
   *out = nullptr;
   if (B <= 0 || H <= 0) return fail(DL_ERR_ARG, "B and H must be positive (B=%d H=%d)", B, H);
-  if (M < 1 || M > DL_MAX_M) return fail(DL_ERR_UNSUPPORTED, "M=%d outside [1, %d]", M, DL_MAX_M);
+  if (M != DL_M_AUTO && (M < 1 || M > DL_MAX_M))
+    return fail(DL_ERR_UNSUPPORTED, "M=%d outside [1, %d] and not DL_M_AUTO", M, DL_MAX_M);
   if (op < DL_GDN || op > DL_RWKV6) return fail(DL_ERR_ARG, "unknown op %d", op);
   if (in_dtype != DL_F32 && in_dtype != DL_BF16) return fail(DL_ERR_ARG, "unknown dtype %d", in_dtype);
   const bool dk_ok = d_k == 64 || d_k == 128, dv_ok = d_v == 64 || d_v == 128;
   if (!dk_ok || !dv_ok) return fail(DL_ERR_UNSUPPORTED, "d_k=%d d_v=%d not in {64,128}", d_k, d_v);
+  if (M == DL_M_AUTO) M = suggest_m(op, d_k, d_v, in_dtype == DL_BF16 ? 2 : 4);
   if (static_cast<long long>(B) * H > (1ll << 30)) return fail(DL_ERR_ARG, "B*H too large");
 
   dl_handle* h = new (std::nothrow) dl_handle();

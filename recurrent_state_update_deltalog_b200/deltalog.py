@@ -21,8 +21,17 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
 
+def suggest_m(op, d_k, d_v, dtype=torch.bfloat16):
+    """Merge interval the library's cost model picks for this operator and
+    head shape (``dl_suggest_m``; no device needed)."""
+    m = ctypes.c_int()
+    N.call("dl_suggest_m", OPS[op], int(d_k), int(d_v), DTYPES[dtype], ctypes.byref(m))
+    return m.value
+
+
 class DeltaLog:
-    """One library handle: B slots x H heads of d_k x d_v fp32 state, merge interval M.
+    """One library handle: B slots x H heads of d_k x d_v fp32 state, merge interval M
+    (``"auto"`` or 0: the library's choice, see :func:`suggest_m`; read back as ``.M``).
 
     ``op`` is ``"gdn"``, ``"kda"`` or ``"rwkv6"``; ``dtype`` is the dtype of
     q/k/v/o (``torch.bfloat16`` or ``torch.float32``).  The handle lives on the
@@ -34,13 +43,17 @@ class DeltaLog:
             raise ValueError(f"op must be one of {sorted(OPS)}")
         if dtype not in DTYPES:
             raise ValueError("dtype must be torch.bfloat16 or torch.float32")
-        self.B, self.H, self.d_k, self.d_v, self.M = B, H, d_k, d_v, M
+        M = N.DL_M_AUTO if M == "auto" else int(M)
+        self.B, self.H, self.d_k, self.d_v = B, H, d_k, d_v
         self.op, self.dtype = op, dtype
         self.device = torch.device("cuda", torch.cuda.current_device() if device is None
                                    else torch.device(device).index or 0)
         self._h = ctypes.c_void_p()
         with torch.cuda.device(self.device):
             N.call("dl_create", ctypes.byref(self._h), B, H, d_k, d_v, M, OPS[op], DTYPES[dtype])
+        m = ctypes.c_int()
+        N.call("dl_merge_interval", self._h, ctypes.byref(m))
+        self.M = m.value
 
     # -- helpers -------------------------------------------------------------
     def _stream(self, stream):

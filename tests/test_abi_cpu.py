@@ -49,7 +49,7 @@ def test_strerror(lib):
 
 
 @pytest.mark.parametrize("args,status", [
-    ((1, 1, 64, 64, 0, 0, 0), -2),      # M = 0
+    ((1, 1, 64, 64, -1, 0, 0), -2),     # M < 0 (0 is DL_M_AUTO)
     ((1, 1, 64, 64, 65, 0, 0), -2),     # M > DL_MAX_M
     ((1, 1, 96, 64, 8, 0, 0), -2),      # unsupported d_k
     ((1, 1, 64, 32, 8, 0, 0), -2),      # unsupported d_v
@@ -95,3 +95,57 @@ def test_python_binding_fails_loudly_without_library(tmp_path):
             mod.load(str(tmp_path / "missing.so"))
     finally:
         importlib.reload(N)
+
+
+# ---- merge-interval choice (host only) ----------------------------------------
+
+def _suggest(lib, op, dk, dv, dtype=1):
+    m = ctypes.c_int(-1)
+    assert lib.dl_suggest_m(op, dk, dv, dtype, ctypes.byref(m)) == 0
+    return m.value
+
+
+def test_suggest_m_rejects_bad_arguments(lib):
+    m = ctypes.c_int()
+    assert lib.dl_suggest_m(3, 64, 64, 1, ctypes.byref(m)) == -1
+    assert lib.dl_suggest_m(0, 96, 64, 1, ctypes.byref(m)) == -1
+    assert lib.dl_suggest_m(0, 64, 64, 5, ctypes.byref(m)) == -1
+    assert lib.dl_suggest_m(0, 64, 64, 1, None) == -1
+    assert lib.dl_merge_interval(None, ctypes.byref(m)) == -1
+
+
+@pytest.mark.parametrize("op", [0, 1, 2])
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64), (128, 128)])
+@pytest.mark.parametrize("dtype", [0, 1])
+def test_suggest_m_near_stationary_point(lib, op, dk, dv, dtype):
+    """The chosen M sits next to the stationary point of the per-token cost
+    S/M + e(M-1)/M + rho(M-1)/2, i.e. M* = sqrt(2(S - e)/rho), for rho between
+    the entry's bytes (pure traffic) and three times that."""
+    import math
+    M = _suggest(lib, op, dk, dv, dtype)
+    es = 2 if dtype == 1 else 4
+    e = dk * es + dv * (es if op == 2 else 4) + (4 if op == 0 else 4 * dk)
+    S = 4 * dk * dv
+    lo, hi = math.sqrt(2 * (S - e) / (3 * e)), math.sqrt(2 * (S - e) / e)
+    assert 2 <= M <= 64
+    assert math.floor(lo) <= M <= math.ceil(hi), (M, lo, hi)
+    if dk != dv:                                    # uncalibrated shapes: pure traffic
+        assert M in (math.floor(hi), math.ceil(hi))
+
+
+@pytest.mark.parametrize("op,d,band", [
+    (0, 128, (7, 12)), (1, 128, (7, 12)), (2, 64, (6, 11)),
+    (0, 64, (8, 12)), (1, 64, (5, 9)), (2, 128, (7, 12)),
+])
+def test_suggest_m_inside_measured_band(lib, op, d, band):
+    """Within the band of M whose measured B200 throughput is within 1% of
+    the best point of a fine sweep (M = 4..16, bf16 inputs, large batch)."""
+    M = _suggest(lib, op, d, d)
+    assert band[0] <= M <= band[1], M
+
+
+def test_suggest_m_orders(lib):
+    """More state per entry favours longer cycles; fatter entries shorter ones."""
+    for op in (0, 1, 2):
+        assert _suggest(lib, op, 128, 128) >= _suggest(lib, op, 64, 64) - 1
+        assert _suggest(lib, op, 128, 128, 0) <= _suggest(lib, op, 128, 128, 1)

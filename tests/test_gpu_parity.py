@@ -496,3 +496,26 @@ def test_slot_index_map_arguments():
         h.step(one, one, one, torch.zeros((1, 2), device="cuda"), torch.zeros((1, 2), device="cuda"),
                slot_idx=torch.zeros(1, dtype=torch.int32, device="cuda"))
     h.close()
+
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("d", [64, 128])
+def test_auto_merge_interval(op, d):
+    """A handle created with M = "auto" takes dl_suggest_m's interval and its
+    outputs and state follow the oracle across two merges."""
+    from recurrent_state_update_deltalog_b200 import DeltaLog, suggest_m
+    B, H = 3, 2
+    h = DeltaLog(B, H, d, d, "auto", op=op, dtype=torch.bfloat16)
+    assert h.M == suggest_m(op, d, d) and 2 <= h.M <= 64
+    T = 2 * h.M + 3
+    S0, seq, u = make_inputs(op, B, H, d, d, T, torch.bfloat16, seed=4)
+    dseq = to_device(seq, torch.bfloat16)
+    h.load_state(torch.from_numpy(S0).cuda())
+    if u is not None:
+        h.set_bonus(torch.from_numpy(u).cuda())
+    outs = [h.step(*step_args(op, dseq, t)).float().cpu().numpy() for t in range(T)]
+    assert h.log_len == T % h.M
+    o_ref, S_ref, _ = run_oracle(op, S0, seq, u)
+    assert relerr(np.stack(outs), o_ref) < TOL[torch.bfloat16]
+    assert relerr(h.read_state().cpu().numpy(), S_ref) < TOL[torch.bfloat16]
+    h.close()
