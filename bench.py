@@ -56,6 +56,8 @@ def parse():
                     help="dl_step kernel variant")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch every step with plain stream ordering")
+    ap.add_argument("--log-b-bf16", action="store_true",
+                    help="store GDN/KDA log value factors b_i in bf16 (DL_OPT_LOG_B_BF16)")
     ap.add_argument("--slot-map", action="store_true",
                     help="run every token through the slot index map: batch row r on slot perm_t[r], "
                          "a fresh random permutation of the B slots per pool token")
@@ -83,22 +85,24 @@ def parse():
 
 
 def workload_name(a):
-    return f"{a.op}_decode_b{a.B}_h{a.H}_d{a.d}_m{a.M}_bf16"
+    tail = "_logb_bf16" if getattr(a, "log_b_bf16", False) and a.op != "rwkv6" else ""
+    return f"{a.op}_decode_b{a.B}_h{a.H}_d{a.d}_m{a.M}_bf16{tail}"
 
 
 # ---------------------------------------------------------------------------
 # algorithmic bytes (what the method must move; no cache effects)
 # ---------------------------------------------------------------------------
 
-def entry_bytes(op, dk, dv, es=2):
-    """Bytes of one log entry: a_i (input dtype) + b_i + Lam_i."""
+def entry_bytes(op, dk, dv, es=2, bb=None):
+    """Bytes of one log entry: a_i (input dtype) + b_i + Lam_i.  bb: bytes of
+    one b_i element (default: the input dtype for RWKV6, fp32 otherwise)."""
     a = dk * es
-    b = dv * (es if op == "rwkv6" else 4)
+    b = dv * (bb or (es if op == "rwkv6" else 4))
     lam = 4 if op == "gdn" else 4 * dk
     return a + b + lam
 
 
-def launch_bytes(op, kind, B, H, dk, dv, n=0, es=2):
+def launch_bytes(op, kind, B, H, dk, dv, n=0, es=2, bb=None):
     """Algorithmic HBM bytes of one launch over all B*H (slot, head) units.
 
     kind: "append" (n entries in the log), "merge" (n entries before the step),
@@ -112,30 +116,30 @@ def launch_bytes(op, kind, B, H, dk, dv, n=0, es=2):
     unit += (2 * dk + dv) * es + dv * es                      # q|r, k, v in; o out
     unit += {"gdn": 8, "kda": 4 * dk + 4, "rwkv6": 4 * dk}[op]  # gates
     if kind != "eager":
-        unit += n * entry_bytes(op, dk, dv, es)
+        unit += n * entry_bytes(op, dk, dv, es, bb)
     if kind == "append":
-        unit += entry_bytes(op, dk, dv, es)
+        unit += entry_bytes(op, dk, dv, es, bb)
     total = unit * B * H
     if op == "rwkv6":
         total += H * dk * 4
     return total
 
 
-def step_bytes(op, B, H, d, M, tokens, es=2):
+def step_bytes(op, B, H, d, M, tokens, es=2, bb=None):
     if M == 1:
         return tokens * launch_bytes(op, "eager", B, H, d, d, 0, es)
-    per_cycle = sum(launch_bytes(op, "append", B, H, d, d, n, es) for n in range(M - 1))
-    per_cycle += launch_bytes(op, "merge", B, H, d, d, M - 1, es)
+    per_cycle = sum(launch_bytes(op, "append", B, H, d, d, n, es, bb) for n in range(M - 1))
+    per_cycle += launch_bytes(op, "merge", B, H, d, d, M - 1, es, bb)
     return per_cycle * (tokens // M)
 
 
-def write_bytes_per_token(op, B, H, d, M, es=2):
+def write_bytes_per_token(op, B, H, d, M, es=2, bb=None):
     """Algorithmic HBM write bytes per slot-token (all heads), averaged over a cycle."""
     state_w = 4 * d * d
     io_w = d * es
     if M == 1:
         return H * (state_w + io_w)
-    ent = entry_bytes(op, d, d, es)
+    ent = entry_bytes(op, d, d, es, bb)
     per_cycle = (M - 1) * (io_w + ent) + (io_w + state_w)
     return H * per_cycle / M
 
@@ -327,6 +331,7 @@ def run_gpu(a, rank, world, local_rank):
     torch.cuda.set_device(dev)
     op, B, H, d, M = a.op, a.B, a.H, a.d, a.M
     seed = rank_seed(a.seed, rank)
+    bb = 2 if a.log_b_bf16 else None           # b_i element bytes in the log
     es = 2
 
     # inputs: a pool of distinct tokens resident in HBM (> L2), cycled
@@ -361,6 +366,8 @@ def run_gpu(a, rank, world, local_rank):
         h = DeltaLog(B, H, d, d, m, op=op, dtype=torch.bfloat16)
         h.set_step_kernel(a.kernel)
         h.set_pdl(not a.no_pdl)
+        if a.log_b_bf16 and m > 1:
+            h.set_log_b_bf16(True)
         h.load_state(S0)
         if u is not None:
             h.set_bonus(u)
@@ -482,13 +489,13 @@ def run_gpu(a, rank, world, local_rank):
     # per-launch durations of the dominant (append) kernel, second pass
     launches = timed(M, per_launch=True)[1] if M > 1 and not a.graph else None
     value = job_tokens_per_s(B, a.tokens, a.steps, world, ms)
-    sb = step_bytes(op, B, H, d, M, a.tokens)
+    sb = step_bytes(op, B, H, d, M, a.tokens, bb=bb)
     result["value"] = value
     result["ms"] = ms
 
     if launches:
         dur = sum(t for t, _ in launches) / len(launches)
-        alg = sum(launch_bytes(op, "append", B, H, d, d, n) for _, n in launches) / len(launches)
+        alg = sum(launch_bytes(op, "append", B, H, d, d, n, bb=bb) for _, n in launches) / len(launches)
         dominant = ("deltalog_stream_kernel" if used_kernel[0] == "stream"
                     else "deltalog_step_kernel") + " (append)"
     else:   # average over every launch of the step (graph replay or M = 1)
@@ -517,10 +524,10 @@ def run_gpu(a, rank, world, local_rank):
         if a.tokens % mv:
             continue
         sms, _ = timed(mv)
-        sbb = step_bytes(op, B, H, d, mv, a.tokens)
+        sbb = step_bytes(op, B, H, d, mv, a.tokens, bb=bb)
         sweep[str(mv)] = {"value": B * a.tokens * a.steps * world / (sms / 1e3),
                           "gbs": sbb / (sms / a.steps / 1e3) / 1e9,
-                          "write_bytes_per_token": write_bytes_per_token(op, B, H, d, mv)}
+                          "write_bytes_per_token": write_bytes_per_token(op, B, H, d, mv, bb=bb)}
     if sweep:
         extra["sweep"] = sweep
 
@@ -569,6 +576,7 @@ def run_gpu(a, rank, world, local_rank):
                    "m_choice": "dl_suggest_m" if getattr(a, "m_auto", False) else "given",
                    "admit_every_tokens": a.admit_every or None,
                    "slot_map": "random permutation per token" if a.slot_map else None,
+                   "log_b": "bf16" if (a.log_b_bf16 or op == "rwkv6") else "fp32",
                    "input_pool_tokens": a.pool, "seed": a.seed,
                    "l2": (f"inputs larger than L2 (state {4 * B * H * d * d / 1e6:.0f} MB)"
                           if 4 * B * H * d * d > L2_BYTES else
@@ -576,7 +584,7 @@ def run_gpu(a, rank, world, local_rank):
                    "parallelism": "replicas" if world == 1 else f"replicas x{world} (B per rank)"},
         "roofline": roofline,
         "gpu_launches": a.steps * a.tokens,
-        "write_bytes_per_token": write_bytes_per_token(op, B, H, d, M),
+        "write_bytes_per_token": write_bytes_per_token(op, B, H, d, M, bb=bb),
         "clocks": clocks,
         "e2e": e2e,
     }

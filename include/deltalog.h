@@ -198,11 +198,23 @@ int dl_read_state(dl_t h, float* S_out, void* stream);
  * (a split below 32 columns per tile falls back to fewer tiles; each tile
  * recomputes the head's key-side coefficients).  Automatic: 2 for d_v = 128
  * while the log holds fewer than 16 entries, else 1. */
+/* DL_OPT_LOG_B_BF16 (0 or 1, default 0): store the GDN/KDA value factors
+ * b_i of the log in bf16 instead of fp32, 516 instead of 772 bytes per entry
+ * for GDN d = 128 and 1024 instead of 1280 for KDA.  b_i is rounded to
+ * nearest-even when appended; the current token's b_t enters its own output
+ * and merge unrounded.  Every replayed or merged entry then carries a
+ * relative error of at most 2^-9 in b_i, which feeds into later outputs and
+ * into Sbar at each merge (outputs no longer equal the eager recurrence's up
+ * to fp32 rounding only).  bf16-input handles only (DL_ERR_UNSUPPORTED
+ * otherwise); a no-op for RWKV6, whose log already holds raw bf16 v_i.
+ * Changeable only while the log is empty (DL_ERR_STATE otherwise).  The
+ * streaming kernel does not take it (DL_ERR_UNSUPPORTED). */
 enum dl_option {
   DL_OPT_STEP_KERNEL = 0,
   DL_OPT_HOST_PREFETCH = 1,
   DL_OPT_PDL = 2,
-  DL_OPT_VALUE_TILES = 3
+  DL_OPT_VALUE_TILES = 3,
+  DL_OPT_LOG_B_BF16 = 4
 };
 enum dl_step_kernel { DL_STEP_AUTO = 0, DL_STEP_REGISTER = 1, DL_STEP_STREAM = 2 };
 int dl_set_option(dl_t h, int option, int value);

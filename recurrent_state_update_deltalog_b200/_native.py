@@ -20,6 +20,7 @@ DL_OPT_STEP_KERNEL = 0
 DL_OPT_HOST_PREFETCH = 1
 DL_OPT_PDL = 2
 DL_OPT_VALUE_TILES = 3
+DL_OPT_LOG_B_BF16 = 4
 DL_STEP_AUTO, DL_STEP_REGISTER, DL_STEP_STREAM = 0, 1, 2
 STATUS = {0: "DL_OK", -1: "DL_ERR_ARG", -2: "DL_ERR_UNSUPPORTED", -3: "DL_ERR_CUDA",
           -4: "DL_ERR_OOM", -5: "DL_ERR_DEVICE", -6: "DL_ERR_STATE"}

@@ -48,6 +48,7 @@ struct dl_handle {
   int host_prefetch;        // DL_OPT_HOST_PREFETCH
   int pdl;                  // DL_OPT_PDL
   int value_tiles;          // DL_OPT_VALUE_TILES (0 = automatic)
+  int log_b_bf16;           // DL_OPT_LOG_B_BF16
 };
 
 namespace {
@@ -96,7 +97,11 @@ size_t lam_per_entry(const dl_handle* h) { return h->op == DL_GDN ? 1 : static_c
 size_t lam_unit_floats(const dl_handle* h) {
   return h->op == DL_GDN ? static_cast<size_t>(dl::gdn_lam_stride(h->Mcap)) : static_cast<size_t>(h->Mcap) * h->dk;
 }
-size_t logb_esize(const dl_handle* h) { return h->op == DL_RWKV6 ? h->esize : sizeof(float); }
+// Element size of b_i in the log: RWKV6 keeps raw v_i in the input dtype;
+// GDN/KDA keep fp32, or bf16 with DL_OPT_LOG_B_BF16.  The buffer is sized
+// for fp32 (logb_alloc_esize) so that the option needs no reallocation.
+size_t logb_esize(const dl_handle* h) { return h->op == DL_RWKV6 || h->log_b_bf16 ? h->esize : sizeof(float); }
+size_t logb_alloc_esize(const dl_handle* h) { return h->op == DL_RWKV6 ? h->esize : sizeof(float); }
 size_t bh(const dl_handle* h) { return static_cast<size_t>(h->B) * h->H; }
 size_t state_bytes(const dl_handle* h) { return bh(h) * h->dk * h->dv * sizeof(float); }
 size_t decay_elems(const dl_handle* h) { return bh(h) * lam_per_entry(h); }
@@ -143,6 +148,7 @@ dl::LaunchShape shape_of(const dl_handle* h, bool aligned16 = false) {
   }
   s.max_n = h->n;
   s.units = s.BH;
+  s.blow = h->log_b_bf16 && h->op != DL_RWKV6;
   return s;
 }
 
@@ -390,7 +396,7 @@ int dl_create(dl_t* out, int B, int H, int d_k, int d_v, int M, int op, int in_d
   } allocs[] = {
       {reinterpret_cast<void**>(&h->Sbar), state_bytes(h)},
       {&h->logA, nbh * h->Mcap * d_k * h->esize},
-      {&h->logB, nbh * h->Mcap * d_v * logb_esize(h)},
+      {&h->logB, nbh * h->Mcap * d_v * logb_alloc_esize(h)},
       {reinterpret_cast<void**>(&h->logLam), nbh * lam_unit_floats(h) * sizeof(float)},
       {reinterpret_cast<void**>(&h->u), static_cast<size_t>(H) * d_k * sizeof(float)},
       {reinterpret_cast<void**>(&h->err), sizeof(int)},
@@ -659,6 +665,13 @@ int dl_set_option(dl_t h, int option, int value) {
     case DL_OPT_PDL:
       if (value != 0 && value != 1) return fail(DL_ERR_ARG, "bad PDL value %d", value);
       h->pdl = value;
+      return DL_OK;
+    case DL_OPT_LOG_B_BF16:
+      if (value != 0 && value != 1) return fail(DL_ERR_ARG, "bad log-b-bf16 value %d", value);
+      if (value && h->dtype != DL_BF16) return fail(DL_ERR_UNSUPPORTED, "a bf16 b-log needs bf16 inputs");
+      if (value != h->log_b_bf16 && h->n != 0)
+        return fail(DL_ERR_STATE, "change the b-log precision only with an empty log (call dl_merge)");
+      h->log_b_bf16 = value;
       return DL_OK;
     case DL_OPT_VALUE_TILES:
       if (value != 0 && value != 1 && value != 2 && value != 4)

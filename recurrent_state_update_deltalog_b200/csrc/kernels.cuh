@@ -188,13 +188,16 @@ __host__ __device__ constexpr int gdn_lam_stride(int Mcap) { return (Mcap + 3) &
 // Byte layout (every region starts 16-byte aligned):
 //   A   n x DK input dtype     a_i = k_i
 //   L   n x DK fp32            Lam_i (KDA / RWKV6 only; GDN keeps n scalars apart)
-//   B   n x DV (fp32 | input)  b_i (RWKV6: raw v_i in the input dtype)
+//   B   n x DV (fp32 | input)  b_i (RWKV6: raw v_i in the input dtype; BLOW:
+//                              GDN/KDA b_i rounded to bf16)
 // followed, for merge-type launches, by the fp32 work arrays
 //   As  (n+1) x DK             ratio-scaled a_i, current entry last (ratio 1)
 //   Bc  DV                     the current entry's b_t
-template <int OP, int DK, int DV, typename TI>
+template <int OP, int DK, int DV, typename TI, bool BLOW = false>
 struct LogLayout {
-  using TB = typename std::conditional<OP == OP_RWKV6, TI, float>::type;
+  static_assert(!BLOW || (OP != OP_RWKV6 && std::is_same<TI, __nv_bfloat16>::value),
+                "a bf16 b-log is an option of bf16-input GDN/KDA handles");
+  using TB = typename std::conditional<OP == OP_RWKV6 || BLOW, TI, float>::type;
   static constexpr bool PERKEY = OP != OP_GDN;
   __host__ __device__ static constexpr size_t a_bytes(int n) { return size_t(n) * DK * sizeof(TI); }
   __host__ __device__ static constexpr size_t l_bytes(int n) { return PERKEY ? size_t(n) * DK * 4 : 0; }
@@ -218,11 +221,11 @@ __device__ __forceinline__ float4 load4f(const __nv_bfloat16* p) {
 
 // Thread 0 starts the bulk copies of entries [0, n) of this (slot, head)'s log
 // into shared memory; completion arrives on `bar` (phase 0).
-template <int OP, int DK, int DV, typename TI>
+template <int OP, int DK, int DV, typename TI, bool BLOW>
 __device__ __forceinline__ void stage_log(unsigned char* smem, uint64_t* bar, const void* logA,
                                           const float* logLam, const void* logB, long sh, int Mcap,
                                           int n) {
-  using LL = LogLayout<OP, DK, DV, TI>;
+  using LL = LogLayout<OP, DK, DV, TI, BLOW>;
   using TB = typename LL::TB;
   mbar_init(bar, 1);
   fence_mbar_init();
@@ -257,12 +260,12 @@ __device__ __forceinline__ bool wait_log(uint64_t* bar, int n, int* err) {
 // tile recomputes the head's ReplayPrep coefficients and the first tile
 // appends the key-side entry.
 // ---------------------------------------------------------------------------
-template <int OP, int DK, int DV, typename TI, int MODE, int NSPLIT, bool MAP>
+template <int OP, int DK, int DV, typename TI, int MODE, int NSPLIT, bool MAP, bool BLOW>
 __global__ void __launch_bounds__(Tile<DK, DV / NSPLIT>::NT, Tile<DK, DV / NSPLIT>::MINB)
 deltalog_step_kernel(const StepArgs a) {
   constexpr int DVT = DV / NSPLIT;  // value-tile width owned by this CTA
   using TL = Tile<DK, DVT>;
-  using LL = LogLayout<OP, DK, DV, TI>;
+  using LL = LogLayout<OP, DK, DV, TI, BLOW>;
   using TB = typename LL::TB;
   constexpr bool DELTA = OP != OP_RWKV6;
   constexpr bool PERKEY = OP != OP_GDN;
@@ -307,7 +310,7 @@ deltalog_step_kernel(const StepArgs a) {
   for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + (rg * TL::RPT + j) * DV + col0 + 4 * c4);
   if (MODE == MODE_APPEND) griddep_launch_dependents();
   griddep_wait();
-  if (tid == 0) stage_log<OP, DK, DV, TI>(s_dyn, &s_bar, a.logA, a.logLam, a.logB, sh, a.Mcap, n);
+  if (tid == 0) stage_log<OP, DK, DV, TI, BLOW>(s_dyn, &s_bar, a.logA, a.logLam, a.logB, sh, a.Mcap, n);
 
   // 2. Key-side values for this lane's keys j = lane + 32 m; GDN's scalar
   // snapshots; per-column v and beta for the finalize threads.
@@ -455,7 +458,7 @@ deltalog_step_kernel(const StepArgs a) {
     } else {
       TB* dstB = static_cast<TB*>(a.logB) + (sh * a.Mcap + n) * DV + col0;
       if constexpr (DELTA) {
-        dstB[c] = bt;
+        dstB[c] = from_f<TB>(bt);
       } else {
         dstB[c] = static_cast<const TI*>(a.v)[bu * DV + col0 + c];   // raw v, bit copy
       }
@@ -609,11 +612,11 @@ eager_step_kernel(const StepArgs a) {
 // otherwise).  Lam_last = Lam_{n-1}, the newest snapshot; a unit with an
 // empty log is copied through.
 // ---------------------------------------------------------------------------
-template <int OP, int DK, int DV, typename TI>
+template <int OP, int DK, int DV, typename TI, bool BLOW>
 __global__ void __launch_bounds__(Tile<DK, DV>::NT, Tile<DK, DV>::MINB)
 materialize_kernel(const MaterializeArgs a) {
   using TL = Tile<DK, DV>;
-  using LL = LogLayout<OP, DK, DV, TI>;
+  using LL = LogLayout<OP, DK, DV, TI, BLOW>;
   using TB = typename LL::TB;
   constexpr bool PERKEY = OP != OP_GDN;
   __shared__ __align__(16) float s_dec[DK];
@@ -636,7 +639,7 @@ materialize_kernel(const MaterializeArgs a) {
   float4 st[TL::RPT];
 #pragma unroll
   for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + (rg * TL::RPT + j) * DV + 4 * c4);
-  if (tid == 0) stage_log<OP, DK, DV, TI>(s_dyn, &s_bar, a.logA, a.logLam, a.logB, sh, a.Mcap, n);
+  if (tid == 0) stage_log<OP, DK, DV, TI, BLOW>(s_dyn, &s_bar, a.logA, a.logLam, a.logB, sh, a.Mcap, n);
 
   float ll[TL::KPL];
 #pragma unroll

@@ -28,6 +28,7 @@ struct LaunchShape {
   int split;       // value tiles per head for the register-tile step kernel (1, 2 or 4)
   int max_n;       // log length of the launched units (shared-memory sizing)
   int units;       // materialisation: units in the launch
+  bool blow;       // GDN/KDA b_i stored in bf16 (bf16-input handles only)
 };
 
 // Launch with the programmatic-stream-serialisation attribute when `pdl`.
@@ -120,25 +121,38 @@ dim3 step_grid(const LaunchShape& s) {
   return dim3(s.BH * NSPLIT);
 }
 
-template <int OP, int DK, int DV, typename TI, int MODE, int NSPLIT, bool MAP>
+template <int OP, int DK, int DV, typename TI, int MODE, int NSPLIT, bool MAP, bool BLOW>
 cudaError_t register_step_mode(const LaunchShape& s, const StepArgs& a, cudaStream_t st) {
   using TL = Tile<DK, DV / NSPLIT>;
-  using LL = LogLayout<OP, DK, DV, TI>;
+  using LL = LogLayout<OP, DK, DV, TI, BLOW>;
   const size_t smem = LL::step_smem(a.n, MODE == MODE_MERGE);
-  auto kern = deltalog_step_kernel<OP, DK, DV, TI, MODE, NSPLIT, MAP>;
+  auto kern = deltalog_step_kernel<OP, DK, DV, TI, MODE, NSPLIT, MAP, BLOW>;
   cudaError_t e = allow_smem(kern, smem, LL::step_smem(kMaxM - 1, MODE != MODE_APPEND));
   if (e != cudaSuccess) return e;
   return launch_maybe_pdl(kern, step_grid<NSPLIT, MAP>(s), TL::NT, smem, st, s.pdl, a);
 }
 
+template <int OP, int DK, int DV, typename TI, int NSPLIT, bool BLOW>
+cudaError_t register_step_log(const LaunchShape& s, int mode, const StepArgs& a, cudaStream_t st) {
+  if (a.slot_idx) {
+    if (mode == MODE_MERGE) return register_step_mode<OP, DK, DV, TI, MODE_MERGE, NSPLIT, true, BLOW>(s, a, st);
+    return register_step_mode<OP, DK, DV, TI, MODE_APPEND, NSPLIT, true, BLOW>(s, a, st);
+  }
+  if (mode == MODE_MERGE) return register_step_mode<OP, DK, DV, TI, MODE_MERGE, NSPLIT, false, BLOW>(s, a, st);
+  return register_step_mode<OP, DK, DV, TI, MODE_APPEND, NSPLIT, false, BLOW>(s, a, st);
+}
+
+// A bf16 b-log exists for bf16-input GDN/KDA handles; other instantiations
+// are never built.
+template <int OP, typename TI>
+constexpr bool kHasBlow = OP != OP_RWKV6 && std::is_same<TI, __nv_bfloat16>::value;
+
 template <int OP, int DK, int DV, typename TI, int NSPLIT>
 cudaError_t register_step(const LaunchShape& s, int mode, const StepArgs& a, cudaStream_t st) {
-  if (a.slot_idx) {
-    if (mode == MODE_MERGE) return register_step_mode<OP, DK, DV, TI, MODE_MERGE, NSPLIT, true>(s, a, st);
-    return register_step_mode<OP, DK, DV, TI, MODE_APPEND, NSPLIT, true>(s, a, st);
+  if constexpr (kHasBlow<OP, TI>) {
+    if (s.blow) return register_step_log<OP, DK, DV, TI, NSPLIT, true>(s, mode, a, st);
   }
-  if (mode == MODE_MERGE) return register_step_mode<OP, DK, DV, TI, MODE_MERGE, NSPLIT, false>(s, a, st);
-  return register_step_mode<OP, DK, DV, TI, MODE_APPEND, NSPLIT, false>(s, a, st);
+  return register_step_log<OP, DK, DV, TI, NSPLIT, false>(s, mode, a, st);
 }
 
 template <int OP, int DK, int DV, typename TI>
@@ -146,7 +160,7 @@ cudaError_t step_dims(const LaunchShape& s, int mode, const StepArgs& a, cudaStr
   // AUTO runs the register-tile kernel, the faster of the two on B200 for
   // every operator's merge launches and for d_v = 64; STREAM is opt-in and
   // takes no slot index map.
-  if (s.variant == STEP_STREAM && s.aligned16 && !a.slot_idx) {
+  if (s.variant == STEP_STREAM && s.aligned16 && !a.slot_idx && !s.blow) {
     bool launched = false;
     cudaError_t e = mode == MODE_MERGE ? stream_dims<OP, DK, DV, TI, true>(s, a, st, &launched)
                                        : stream_dims<OP, DK, DV, TI, false>(s, a, st, &launched);
@@ -181,15 +195,23 @@ cudaError_t eager_dims(const LaunchShape& s, const StepArgs& a, cudaStream_t st)
   return a.slot_idx ? eager_map<OP, DK, DV, TI, true>(s, a, st) : eager_map<OP, DK, DV, TI, false>(s, a, st);
 }
 
-template <int OP, int DK, int DV, typename TI>
-cudaError_t materialize_dims(const LaunchShape& s, const MaterializeArgs& a, cudaStream_t st) {
-  using LL = LogLayout<OP, DK, DV, TI>;
-  auto kern = materialize_kernel<OP, DK, DV, TI>;
+template <int OP, int DK, int DV, typename TI, bool BLOW>
+cudaError_t materialize_log(const LaunchShape& s, const MaterializeArgs& a, cudaStream_t st) {
+  using LL = LogLayout<OP, DK, DV, TI, BLOW>;
+  auto kern = materialize_kernel<OP, DK, DV, TI, BLOW>;
   const size_t smem = LL::materialize_smem(s.max_n);
   cudaError_t e = allow_smem(kern, smem, LL::materialize_smem(kMaxM - 1));
   if (e != cudaSuccess) return e;
   kern<<<s.units, Tile<DK, DV>::NT, smem, st>>>(a);
   return cudaGetLastError();
+}
+
+template <int OP, int DK, int DV, typename TI>
+cudaError_t materialize_dims(const LaunchShape& s, const MaterializeArgs& a, cudaStream_t st) {
+  if constexpr (kHasBlow<OP, TI>) {
+    if (s.blow) return materialize_log<OP, DK, DV, TI, true>(s, a, st);
+  }
+  return materialize_log<OP, DK, DV, TI, false>(s, a, st);
 }
 
 #define DL_DISPATCH_DIMS(FN, ...)                                                          \

@@ -177,6 +177,10 @@ class DeltaLog:
         """Programmatic dependent launch of steps that follow an append (default on)."""
         N.call("dl_set_option", self._h, N.DL_OPT_PDL, 1 if on else 0)
 
+    def set_log_b_bf16(self, on):
+        """Store GDN/KDA log value factors b_i in bf16 (bf16 handles, empty log)."""
+        N.call("dl_set_option", self._h, N.DL_OPT_LOG_B_BF16, 1 if on else 0)
+
     def set_value_tiles(self, n):
         """0 (automatic), 1 or 2 value tiles (CTAs) per head in the register-tile step kernel."""
         N.call("dl_set_option", self._h, N.DL_OPT_VALUE_TILES, int(n))

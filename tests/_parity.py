@@ -45,7 +45,8 @@ def step_args(op, dseq, t):
     return first[t], dseq["k"][t], dseq["v"][t], dseq["log_decay"][t], beta
 
 
-def run_gpu(op, S0, seq, u, M, dtype, eager=False, record_merges=True, kernel="auto", tiles=0):
+def run_gpu(op, S0, seq, u, M, dtype, eager=False, record_merges=True, kernel="auto", tiles=0,
+            log_b_bf16=False):
     """Run T steps through the library; returns (o[T,B,H,dv], {t: Sbar}, final logical S).
 
     ``kernel`` selects the dl_step kernel ("auto", "register" or "stream")."""
@@ -56,6 +57,8 @@ def run_gpu(op, S0, seq, u, M, dtype, eager=False, record_merges=True, kernel="a
     h = DeltaLog(B, H, dk, dv, M, op=op, dtype=dtype)
     h.set_step_kernel(kernel)
     h.set_value_tiles(tiles)
+    if log_b_bf16:
+        h.set_log_b_bf16(True)
     try:
         h.load_state(torch.from_numpy(S0).cuda())
         if u is not None:
