@@ -56,6 +56,9 @@ def parse():
                     help="dl_step kernel variant")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch every step with plain stream ordering")
+    ap.add_argument("--prefill", type=int, default=0, metavar="L",
+                    help="time the prefill hand-off (dl_prefill) of B prompts of L tokens instead "
+                         "of decode; one JSON line, ALU roofline")
     ap.add_argument("--log-b-bf16", action="store_true",
                     help="store GDN/KDA log value factors b_i in bf16 (DL_OPT_LOG_B_BF16)")
     ap.add_argument("--slot-map", action="store_true",
@@ -70,7 +73,7 @@ def parse():
                     help="B x M sweep, e.g. '1,16,64,256,1024x1,2,4,8,16,32': one JSON line per "
                          "point (CUDA graphs; M=1 is the eager kernel)")
     args = ap.parse_args()
-    if args.grid:
+    if args.grid or args.prefill:
         return args
     if args.admit_every and args.graph:
         ap.error("--admit-every runs the Python launch loop")
@@ -613,6 +616,107 @@ def run_grid(a, rank, world, local_rank):
                 print(json.dumps(line), flush=True)
 
 
+def prefill_flops(op, dk, dv):
+    """fp32 flops of one prefill token per head: the contraction pass (S^T k and
+    S^T q for GDN/KDA, S^T r for RWKV6; one FMA = 2 flops per state element
+    each) and the update pass (decay multiply, 1 flop, and rank-1 FMA, 2)."""
+    return (4 if op != "rwkv6" else 2) * dk * dv + 3 * dk * dv
+
+
+def fp32_peak_tflops(sm_mhz, sms=148):
+    """fp32 SIMT peak: 128 FP32 lanes per SM, one FMA (2 flops) per lane per clock."""
+    return sms * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def run_prefill(a, rank, world, local_rank):
+    """Prefill hand-off: B prompts of L tokens packed token-major, every row
+    from a zero state into its own slot; tokens/s = B * L / time.  Beside it,
+    the same tokens pushed one by one through the eager decode kernel."""
+    import numpy as np
+    import torch
+    from recurrent_state_update_deltalog_b200 import DeltaLog
+    from synthetic import bonus, sequence
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    op, B, H, d, L = a.op, a.B, a.H, a.d, a.prefill
+    seed = rank_seed(a.seed, rank)
+    seq = sequence(seed, op, B, H, d, d, L, bf16=True)
+    first = "r" if op == "rwkv6" else "q"
+    names = [first, "k", "v", "log_decay"] + ([] if op == "rwkv6" else ["beta"])
+    packed = {}
+    for nm in names:        # [L, B, H, ...] -> rows one after another: [B * L, H, ...]
+        arr = np.ascontiguousarray(np.swapaxes(seq[nm], 0, 1)).reshape((B * L,) + seq[nm].shape[2:])
+        packed[nm] = torch.from_numpy(arr).to(dev, torch.bfloat16 if nm in (first, "k", "v") else torch.float32)
+    cu = torch.arange(0, (B + 1) * L, L, dtype=torch.int32, device=dev)
+    u = torch.from_numpy(bonus(seed, H, d)).to(dev) if op == "rwkv6" else None
+    h = DeltaLog(B, H, d, d, a.M, op=op, dtype=torch.bfloat16)
+    if u is not None:
+        h.set_bonus(u)
+    o = torch.empty((B * L, H, d), dtype=torch.bfloat16, device=dev)
+    args = tuple(packed[nm] for nm in (first, "k", "v", "log_decay")) + (packed.get("beta"),)
+    stream = torch.cuda.current_stream(dev)
+
+    def once():
+        h.prefill(*args, cu_seqlens=cu, zero_state=True, out=o, stream=stream)
+
+    for _ in range(max(a.warmup, 3)):
+        once()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(a.steps):
+        once()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1) / a.steps
+    h.check_device()
+    tok_s = B * L / (ms / 1e3)
+    flops = prefill_flops(op, d, d) * H * B * L / (ms / 1e3) / 1e12
+    sm = (clocks or {}).get("sm_mhz") or 1965.0
+    peak = fp32_peak_tflops(1965.0)
+
+    # baseline: the same prompts token by token through the eager decode kernel
+    he = DeltaLog(B, H, d, d, 1, op=op, dtype=torch.bfloat16)
+    if u is not None:
+        he.set_bonus(u)
+    dseq = {nm: torch.from_numpy(np.ascontiguousarray(seq[nm])).to(
+        dev, torch.bfloat16 if nm in (first, "k", "v") else torch.float32) for nm in names}
+    oe = torch.empty((B, H, d), dtype=torch.bfloat16, device=dev)
+
+    def eager_all():
+        for t in range(L):
+            he.eager_step(dseq[first][t], dseq["k"][t], dseq["v"][t], dseq["log_decay"][t],
+                          dseq["beta"][t] if op != "rwkv6" else None, out=oe, stream=stream)
+
+    eager_all()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    eager_all()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    eager_ms = e0.elapsed_time(e1)
+    line = {
+        "metric": "prefill tokens/s (B*L/s)", "value": tok_s, "unit": "tokens/s", "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"{op}_prefill_b{B}_l{L}_h{H}_d{d}_bf16", "op": op, "B": B, "L": L,
+                   "H": H, "d_k": d, "d_v": d, "state": "fp32", "inputs": "bf16",
+                   "start": "zero state", "kernel": "prefill_kernel (64 threads, 32 value columns)"},
+        "roofline": {"bound": "alu", "achieved": flops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": flops / peak, "traffic": None,
+                     "peak_note": "fp32 SIMT at the 1965 MHz max clock: 148 SMs x 128 lanes x 2 flops",
+                     "flops_per_token_head": prefill_flops(op, d, d), "sm_mhz": sm},
+        "eager_tokenwise": {"value": B * L / (eager_ms / 1e3), "unit": "tokens/s", "ms": eager_ms},
+        "clocks": clocks, "gpu_launches": a.steps,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     a = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -632,6 +736,8 @@ def main():
     try:
         if a.grid:
             run_grid(a, rank, world, local_rank)
+        elif a.prefill:
+            run_prefill(a, rank, world, local_rank)
         else:
             line = run_gpu(a, rank, world, local_rank)
             if line is not None:

@@ -140,6 +140,37 @@ int dl_step_indexed(dl_t h, const int* slot_idx, int rows, const void* q, const 
                     const void* v, const float* log_decay, const float* beta, void* o,
                     void* stream);
 
+/* Prefill -> decode hand-off: run the operator's recurrence over a packed
+ * batch of prompts and write each prompt's final state as its slot's base.
+ * The pages' decode path starts from a dense base that holds the history up
+ * to the last merge point (DeltaLog technical summary, gist.science,
+ * "Method -- core mechanism: base + log"); the end of a prompt is such a
+ * point.
+ *   rows        prompts in the batch (0 <= rows <= B, at most 65535);
+ *   slot_idx    device int32 [rows]: slot of row r (negative: skip the row),
+ *               or NULL: row r runs on slot r; rows must name distinct slots;
+ *   cu_seqlens  device int32 [rows + 1]: row r owns tokens
+ *               [cu_seqlens[r], cu_seqlens[r + 1]) of the packed inputs
+ *               (0 <= start <= end <= total, else the row is skipped and
+ *               DL_DEVERR_SEQLEN is raised);
+ *   total       tokens in the packed inputs;
+ *   q, k, v, o  [total][H][d] in the input dtype, log_decay [total][H] (GDN)
+ *               or [total][H][d_k], beta [total][H] (GDN/KDA, NULL for
+ *               RWKV6): the layouts of dl_step with tokens in place of slots;
+ *               o receives every token's output;
+ *   flags       DL_PREFILL_ZERO_STATE: every row starts from S = 0 (a new
+ *               sequence); 0: from the slot's current logical state (a
+ *               continued or chunked prompt, or a state loaded from a cache).
+ * Afterwards each named slot's base holds the state after its last token and
+ * its log entries are cleared (dl_slot_load's convention), so dl_step
+ * continues from it.  Other slots are untouched.  The outputs equal the
+ * eager recurrence's token by token up to fp32 rounding.  With total == 0
+ * the input pointers may be NULL. */
+#define DL_PREFILL_ZERO_STATE 1
+int dl_prefill(dl_t h, const int* slot_idx, int rows, const int* cu_seqlens, long long total, int flags,
+               const void* q, const void* k, const void* v, const float* log_decay,
+               const float* beta, void* o, void* stream);
+
 /* Same as dl_step with HOST pointers (pinned or pageable): copies the inputs
  * into handle-owned device buffers, runs the step and copies o back.  Inputs
  * must stay valid, and o is valid, once `stream` has reached the call.  By
@@ -251,7 +282,8 @@ int dl_slot_read(dl_t h, int slot, float* S_out, void* stream);
 /* Bits of the device error word. */
 enum dl_device_error {
   DL_DEVERR_WAIT_TIMEOUT = 1,  /* a bounded wait on a log copy gave up; that unit wrote nothing */
-  DL_DEVERR_SLOT_INDEX = 2     /* dl_step_indexed / dl_eager_step_indexed: slot index >= B */
+  DL_DEVERR_SLOT_INDEX = 2,    /* a slot index >= B (indexed steps, dl_prefill) */
+  DL_DEVERR_SEQLEN = 4         /* dl_prefill: a row's cu_seqlens range is invalid */
 };
 
 /* Read and clear the handle's device error word (synchronises `stream`).

@@ -16,6 +16,7 @@ DL_F32, DL_BF16 = 0, 1
 DL_OK = 0
 DL_MAX_M = 64
 DL_M_AUTO = 0
+DL_PREFILL_ZERO_STATE = 1
 DL_OPT_STEP_KERNEL = 0
 DL_OPT_HOST_PREFETCH = 1
 DL_OPT_PDL = 2
@@ -35,6 +36,7 @@ SIGNATURES = {
     "dl_set_bonus": (_I, [_P, _P, _P]),
     "dl_suggest_m": (_I, [_I, _I, _I, _I, ctypes.POINTER(_I)]),
     "dl_merge_interval": (_I, [_P, ctypes.POINTER(_I)]),
+    "dl_prefill": (_I, [_P, _P, _I, _P, ctypes.c_longlong, _I, _P, _P, _P, _P, _P, _P, _P]),
     "dl_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
     "dl_step_indexed": (_I, [_P, _P, _I, _P, _P, _P, _P, _P, _P, _P]),
     "dl_step_host": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),

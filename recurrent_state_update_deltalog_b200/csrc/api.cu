@@ -2,6 +2,7 @@
 // The contract of every entry point is documented in include/deltalog.h.
 #include "deltalog.h"
 #include "launch.cuh"
+#include "prefill.cuh"
 
 #include <cstdarg>
 #include <cstdio>
@@ -11,6 +12,7 @@
 
 static_assert(DL_DEVERR_WAIT_TIMEOUT == dl::kErrWaitTimeout, "device error bits");
 static_assert(DL_DEVERR_SLOT_INDEX == dl::kErrSlotIndex, "device error bits");
+static_assert(DL_DEVERR_SEQLEN == dl::kErrSeqlen, "device error bits");
 
 struct dl_handle {
   int B, H, dk, dv, M, op, dtype, device;
@@ -251,6 +253,8 @@ cudaError_t launch_materialize(const dl_handle* h, float* out, cudaStream_t s, l
   a.logLam = h->logLam;
   a.err = h->err;
   a.unit0 = unit0;
+  a.slot_idx = nullptr;
+  a.slots = h->B;
   a.H = h->H;
   a.Mcap = h->Mcap;
   a.n = h->n;
@@ -260,6 +264,40 @@ cudaError_t launch_materialize(const dl_handle* h, float* out, cudaStream_t s, l
     case DL_GDN: return dl::launch_materialize_op<dl::OP_GDN>(sh, a, s);
     case DL_KDA: return dl::launch_materialize_op<dl::OP_KDA>(sh, a, s);
     default: return dl::launch_materialize_op<dl::OP_RWKV6>(sh, a, s);
+  }
+}
+
+// Fold the logs of slots slot_idx[0..rows) into their bases, in place.
+cudaError_t materialize_slots(const dl_handle* h, const int* slot_idx, int rows, cudaStream_t s) {
+  dl::MaterializeArgs a;
+  a.Sin = h->Sbar;
+  a.Sout = h->Sbar;
+  a.logA = h->logA;
+  a.logB = h->logB;
+  a.logLam = h->logLam;
+  a.err = h->err;
+  a.unit0 = 0;
+  a.slot_idx = slot_idx;
+  a.slots = h->B;
+  a.H = h->H;
+  a.Mcap = h->Mcap;
+  a.n = h->n;
+  dl::LaunchShape sh = shape_of(h);
+  sh.units = slot_idx ? rows : rows * h->H;
+  switch (h->op) {
+    case DL_GDN: return dl::launch_materialize_op<dl::OP_GDN>(sh, a, s);
+    case DL_KDA: return dl::launch_materialize_op<dl::OP_KDA>(sh, a, s);
+    default: return dl::launch_materialize_op<dl::OP_RWKV6>(sh, a, s);
+  }
+}
+
+cudaError_t launch_prefill(const dl_handle* h, const dl::PrefillArgs& a, int rows, cudaStream_t s) {
+  dl::LaunchShape sh = shape_of(h);
+  sh.units = rows;
+  switch (h->op) {
+    case DL_GDN: return dl::launch_prefill_op<dl::OP_GDN>(sh, a, s);
+    case DL_KDA: return dl::launch_prefill_op<dl::OP_KDA>(sh, a, s);
+    default: return dl::launch_prefill_op<dl::OP_RWKV6>(sh, a, s);
   }
 }
 
@@ -491,6 +529,57 @@ int dl_step_indexed(dl_t h, const int* slot_idx, int rows, const void* q, const 
   DeviceScope ds(h->device);
   if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
   return do_step(h, slot_idx, rows, q, k, v, log_decay, beta, o, static_cast<cudaStream_t>(stream));
+}
+
+int dl_prefill(dl_t h, const int* slot_idx, int rows, const int* cu_seqlens, long long total, int flags,
+               const void* q, const void* k, const void* v, const float* log_decay, const float* beta, void* o,
+               void* stream) {
+  if (!h) return fail(DL_ERR_ARG, "null handle");
+  if (rows < 0 || rows > h->B) return fail(DL_ERR_ARG, "rows=%d outside [0, %d]", rows, h->B);
+  if (rows > 65535) return fail(DL_ERR_UNSUPPORTED, "a prefill takes at most 65535 rows (grid y)");
+  if (flags & ~DL_PREFILL_ZERO_STATE) return fail(DL_ERR_ARG, "unknown prefill flags 0x%x", flags);
+  if (total < 0) return fail(DL_ERR_ARG, "negative token count");
+  if (rows == 0) return DL_OK;
+  if (!cu_seqlens || !aligned(cu_seqlens, 4)) return fail(DL_ERR_ARG, "cu_seqlens null or not 4-byte aligned");
+  if (slot_idx && !aligned(slot_idx, 4)) return fail(DL_ERR_ARG, "slot index pointer not 4-byte aligned");
+  if (total > 0) {
+    int rc = check_step_args(h, q, k, v, log_decay, beta, o);
+    if (rc != DL_OK) return rc;
+  }
+  DeviceScope ds(h->device);
+  if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool zero = flags & DL_PREFILL_ZERO_STATE;
+  if (!zero && h->n > 0) {  // start from the logical state: fold the rows' logs first
+    cudaError_t e = materialize_slots(h, slot_idx, rows, s);
+    if (e != cudaSuccess) return cuda_fail(e, "prefill: log fold");
+  }
+  dl::PrefillArgs a;
+  a.Sbar = h->Sbar;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.log_decay = log_decay;
+  a.beta = beta;
+  a.o = o;
+  a.u = h->u;
+  a.slot_idx = slot_idx;
+  a.cu_seqlens = cu_seqlens;
+  a.logA = h->logA;
+  a.logB = h->logB;
+  a.logLam = h->logLam;
+  a.err = h->err;
+  a.total = static_cast<long>(total);
+  a.H = h->H;
+  a.slots = h->B;
+  a.Mcap = h->Mcap;
+  a.n = h->n;
+  a.b_esize = static_cast<int>(logb_esize(h));
+  a.zero_state = zero ? 1 : 0;
+  cudaError_t e = launch_prefill(h, a, rows, s);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+  h->wrote_state = true;
+  return DL_OK;
 }
 
 int dl_step_host(dl_t h, const void* q, const void* k, const void* v, const float* log_decay,

@@ -113,6 +113,10 @@ struct MaterializeArgs {
   const float* logLam;
   int* err;
   long unit0;
+  const int* slot_idx;  // null: units [unit0, unit0 + gridDim.x) into Sout;
+                        // else grid (H, rows): slot slot_idx[r]'s heads, in place
+                        // (Sout == Sin), rows with a negative index skipped
+  int slots;            // pool slots (bound of slot_idx)
   int H;
   int Mcap;
   int n;
@@ -627,7 +631,18 @@ materialize_kernel(const MaterializeArgs a) {
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const int c4 = tid % TL::TPR, rg = tid / TL::TPR;
-  const long sh = a.unit0 + blockIdx.x;
+  long sh = a.unit0 + blockIdx.x;
+  float* Sq = a.Sout + blockIdx.x * (DK * DV);
+  if (a.slot_idx) {
+    const int slot = __ldg(a.slot_idx + blockIdx.y);
+    if (slot < 0) return;
+    if (slot >= a.slots) {
+      if (tid == 0) atomicOr(a.err, kErrSlotIndex);
+      return;
+    }
+    sh = static_cast<long>(slot) * a.H + blockIdx.x;
+    Sq = a.Sout + sh * (DK * DV);
+  }
   const int n = a.n;
 
   const TI* sA = reinterpret_cast<const TI*>(s_dyn);
@@ -683,7 +698,6 @@ materialize_kernel(const MaterializeArgs a) {
       fma4(st[j4 + 3], a4.w, b4);
     }
   }
-  float* Sq = a.Sout + blockIdx.x * (DK * DV);
 #pragma unroll
   for (int j = 0; j < TL::RPT; ++j) st_state(Sq + (rg * TL::RPT + j) * DV + 4 * c4, st[j]);
 }

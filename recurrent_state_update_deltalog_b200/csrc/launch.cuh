@@ -202,7 +202,8 @@ cudaError_t materialize_log(const LaunchShape& s, const MaterializeArgs& a, cuda
   const size_t smem = LL::materialize_smem(s.max_n);
   cudaError_t e = allow_smem(kern, smem, LL::materialize_smem(kMaxM - 1));
   if (e != cudaSuccess) return e;
-  kern<<<s.units, Tile<DK, DV>::NT, smem, st>>>(a);
+  const dim3 grid = a.slot_idx ? dim3(s.H, s.units) : dim3(s.units);  // mapped: (heads, rows)
+  kern<<<grid, Tile<DK, DV>::NT, smem, st>>>(a);
   return cudaGetLastError();
 }
 

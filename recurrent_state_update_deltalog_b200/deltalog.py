@@ -130,6 +130,31 @@ class DeltaLog:
                    _ptr(log_decay), _ptr(beta), _ptr(out), self._stream(stream))
         return out
 
+    def prefill(self, q, k, v, log_decay, beta=None, cu_seqlens=None, slot_idx=None,
+                zero_state=False, out=None, stream=None):
+        """Prefill -> decode hand-off over packed prompts (``dl_prefill``).
+
+        q, k, v, log_decay, beta hold ``total`` tokens in dl_step's per-slot
+        layouts ([total, H, ...]); ``cu_seqlens`` (int32 [rows + 1], device)
+        splits them into rows; row r runs on slot ``slot_idx[r]`` (int32
+        [rows], device; default: slot r).  Each named slot's base then holds
+        the state after its last token.  Returns o [total, H, d_v]."""
+        if cu_seqlens is None:
+            raise ValueError("cu_seqlens is required")
+        total = q.shape[0]
+        rows = cu_seqlens.numel() - 1
+        if rows < 0 or rows > self.B:
+            raise ValueError(f"cu_seqlens must hold rows + 1 offsets with rows <= B={self.B}")
+        self._check("cu_seqlens", cu_seqlens, (rows + 1,), torch.int32)
+        if slot_idx is not None:
+            self._check("slot_idx", slot_idx, (rows,), torch.int32)
+        out = self._alloc_out(True, total) if out is None else out
+        self._check_step(q, k, v, log_decay, beta, out, True, total)
+        flags = N.DL_PREFILL_ZERO_STATE if zero_state else 0
+        N.call("dl_prefill", self._h, _ptr(slot_idx), rows, _ptr(cu_seqlens), total, flags,
+               _ptr(q), _ptr(k), _ptr(v), _ptr(log_decay), _ptr(beta), _ptr(out), self._stream(stream))
+        return out
+
     def step_host(self, q, k, v, log_decay, beta=None, out=None, stream=None):
         """dl_step on host tensors (pinned for async copies); o is ready after a stream sync."""
         out = self._alloc_out(False) if out is None else out

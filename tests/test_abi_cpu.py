@@ -73,6 +73,7 @@ def test_null_handle_paths(lib):
     for fn in ("dl_step_indexed", "dl_eager_step_indexed"):
         assert getattr(lib, fn)(None, p, 1, p, p, p, p, p, p, None) == -1
         assert getattr(lib, fn)(None, None, 0, None, None, None, None, None, None, None) == -1
+    assert lib.dl_prefill(None, None, 1, p, 1, 0, p, p, p, p, p, p, None) == -1
     assert lib.dl_merge(None, None) == -1
     assert lib.dl_read_state(None, p, None) == -1
     assert lib.dl_load_state(None, p, None) == -1

@@ -1,0 +1,164 @@
+"""Prefill -> decode hand-off (dl_prefill) against the fp64 oracle.
+
+Packed prompts of ragged lengths (0, 1, and several tiles of tokens) run on
+pool slots given by an index map; every token's output and each slot's
+final state must match the eager recurrence from the prompt's initial state,
+and decoding must continue from the handed-off state across merges.
+"""
+import numpy as np
+import pytest
+import torch
+
+from _parity import TOL, make_inputs, relerr, run_oracle, step_args, to_device
+from synthetic import initial_state, sequence
+
+pytestmark = pytest.mark.gpu
+
+OPS = ["gdn", "kda", "rwkv6"]
+
+
+def _pack(seq, lens):
+    """Rows of a [T, R, H, ...] sequence packed token-major: row r's first
+    lens[r] tokens, rows one after another."""
+    out = {}
+    for key, arr in seq.items():
+        out[key] = np.concatenate([arr[:n, r] for r, n in enumerate(lens)], axis=0)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    return out, cu
+
+
+def _device_packed(packed, dtype):
+    return {key: torch.from_numpy(np.ascontiguousarray(a)).to(
+        device="cuda", dtype=dtype if key in ("q", "r", "k", "v") else torch.float32)
+        for key, a in packed.items()}
+
+
+def _prefill_args(op, d):
+    first = d["r"] if op == "rwkv6" else d["q"]
+    return first, d["k"], d["v"], d["log_decay"], (None if op == "rwkv6" else d["beta"])
+
+
+def _oracle_row(op, S_init, seq, r, n, u):
+    """Eager oracle of row r over its first n tokens from state S_init [H, dk, dv]."""
+    one = {key: val[:n, r:r + 1] for key, val in seq.items()}
+    if n == 0:
+        return np.zeros((0, 1) + seq["v"].shape[2:]), S_init[None].astype(np.float64)
+    o, S, _ = run_oracle(op, S_init[None], one, u)
+    return o, S
+
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("dims", [(64, 64), (128, 128), (64, 128), (128, 64)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_prefill_then_decode(op, dims, dtype):
+    from recurrent_state_update_deltalog_b200 import DeltaLog
+    dk, dv = dims
+    B, H, M, T_dec = 8, 3, 4, 7
+    lens = [37, 0, 1, 64, 5]
+    slots = [6, 0, 3, 1, 4]
+    rows = len(lens)
+    bf16 = dtype == torch.bfloat16
+    seq = sequence(21, op, rows, H, dk, dv, max(lens), bf16=bf16)
+    u = make_inputs(op, 1, H, dk, dv, 1, dtype, seed=21)[2]
+    packed, cu = _pack(seq, lens)
+    tol = TOL[dtype]
+
+    S_pool = initial_state(5, B, H, dk, dv)             # other slots keep this
+    h = DeltaLog(B, H, dk, dv, M, op=op, dtype=dtype)
+    h.load_state(torch.from_numpy(S_pool).cuda())
+    if u is not None:
+        h.set_bonus(torch.from_numpy(u).cuda())
+    # two decode tokens first, so that the log holds entries at the hand-off
+    warm = make_inputs(op, B, H, dk, dv, 2, dtype, seed=22)[1]
+    dwarm = to_device(warm, dtype)
+    for t in range(2):
+        h.step(*step_args(op, dwarm, t))
+    _, S_ref, _ = run_oracle(op, S_pool, warm, u)
+
+    d = _device_packed(packed, dtype)
+    o = h.prefill(*_prefill_args(op, d), cu_seqlens=torch.from_numpy(cu).cuda(),
+                  slot_idx=torch.tensor(slots, dtype=torch.int32, device="cuda"), zero_state=True)
+    assert h.log_len == 2                                # the handle's cycle is unchanged
+    got = o.float().cpu().numpy()
+    zero = np.zeros((H, dk, dv))
+    for r, (n, b) in enumerate(zip(lens, slots)):
+        o_r, S_r = _oracle_row(op, zero, seq, r, n, u)
+        if n:
+            assert relerr(got[cu[r]:cu[r + 1]], o_r[:, 0]) < tol, r
+        S_ref[b] = S_r[0]
+        assert relerr(h.slot_read(b).cpu().numpy(), S_ref[b]) < tol, (r, b)
+    for b in (2, 5, 7):                                  # slots not named are untouched
+        assert relerr(h.slot_read(b).cpu().numpy(), S_ref[b]) < tol, b
+
+    # decode continues from the handed-off states, across a merge
+    dec = make_inputs(op, B, H, dk, dv, T_dec, dtype, seed=23)[1]
+    ddec = to_device(dec, dtype)
+    outs = [h.step(*step_args(op, ddec, t)).float().cpu().numpy() for t in range(T_dec)]
+    o_ref, S_fin, _ = run_oracle(op, S_ref, dec, u)
+    assert relerr(np.stack(outs), o_ref) < tol
+    assert relerr(h.read_state().cpu().numpy(), S_fin) < tol
+    h.check_device()
+    h.close()
+
+
+@pytest.mark.parametrize("op", OPS)
+def test_prefill_continues_logical_state(op):
+    """Without DL_PREFILL_ZERO_STATE a prompt continues from the slot's
+    logical state (base + log), e.g. the second chunk of a long prompt."""
+    from recurrent_state_update_deltalog_b200 import DeltaLog
+    dtype, dk, dv, B, H, M = torch.bfloat16, 128, 128, 4, 2, 8
+    S0, warm, u = make_inputs(op, B, H, dk, dv, 5, dtype, seed=31)
+    h = DeltaLog(B, H, dk, dv, M, op=op, dtype=dtype)
+    h.load_state(torch.from_numpy(S0).cuda())
+    if u is not None:
+        h.set_bonus(torch.from_numpy(u).cuda())
+    dwarm = to_device(warm, dtype)
+    for t in range(5):
+        h.step(*step_args(op, dwarm, t))
+    _, S_ref, _ = run_oracle(op, S0, warm, u)
+    lens = [20, 33, 0, 9]
+    seq = sequence(32, op, B, H, dk, dv, max(lens), bf16=True)
+    packed, cu = _pack(seq, lens)
+    d = _device_packed(packed, dtype)
+    o = h.prefill(*_prefill_args(op, d), cu_seqlens=torch.from_numpy(cu).cuda())   # row r = slot r
+    got = o.float().cpu().numpy()
+    for r, n in enumerate(lens):
+        o_r, S_r = _oracle_row(op, S_ref[r], seq, r, n, u)
+        if n:
+            assert relerr(got[cu[r]:cu[r + 1]], o_r[:, 0]) < TOL[dtype], r
+        assert relerr(h.slot_read(r).cpu().numpy(), S_r[0]) < TOL[dtype], r
+    h.check_device()
+    h.close()
+
+
+def test_prefill_bad_seqlen_raises_device_flag():
+    from recurrent_state_update_deltalog_b200 import DeltaLog, DeltaLogError
+    op, dtype, d, B, H = "gdn", torch.float32, 64, 3, 2
+    lens = [4, 6, 3]
+    seq = sequence(41, op, B, H, d, d, 6, bf16=False)
+    packed, cu = _pack(seq, lens)
+    bad = cu.copy()
+    bad[2] = 99                                          # row 1 ends past the batch, row 2 starts there
+    h = DeltaLog(B, H, d, d, 4, op=op, dtype=dtype)
+    dd = _device_packed(packed, dtype)
+    o = torch.zeros((int(cu[-1]), H, d), device="cuda")
+    h.prefill(*_prefill_args(op, dd), cu_seqlens=torch.from_numpy(bad).cuda(), zero_state=True, out=o)
+    with pytest.raises(DeltaLogError, match="0x4"):
+        h.check_device()
+    o_r, S_r = _oracle_row(op, np.zeros((H, d, d)), seq, 0, 4, None)
+    assert relerr(o[:4].cpu().numpy(), o_r[:, 0]) < TOL[dtype]          # row 0 ran
+    assert np.all(o[4:].cpu().numpy() == 0)                              # rows 1 and 2 skipped
+    h.close()
+
+
+def test_prefill_arguments():
+    from recurrent_state_update_deltalog_b200 import DeltaLog, DeltaLogError
+    h = DeltaLog(2, 2, 64, 64, 4, op="gdn", dtype=torch.float32)
+    e3 = torch.empty((0, 2, 64), device="cuda")
+    e2 = torch.empty((0, 2), device="cuda")
+    cu = torch.zeros(3, dtype=torch.int32, device="cuda")
+    h.prefill(e3, e3, e3, e2, e2, cu_seqlens=cu, zero_state=True)      # two empty prompts
+    assert np.all(h.read_state().cpu().numpy() == 0)
+    with pytest.raises(ValueError):
+        h.prefill(e3, e3, e3, e2, e2, cu_seqlens=torch.zeros(4, dtype=torch.int32, device="cuda"))
+    h.close()
