@@ -15,7 +15,6 @@ Prints ONE JSON line on rank 0.
 from __future__ import annotations
 
 import argparse
-import glob
 import hashlib
 import json
 import os
@@ -186,9 +185,14 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# the sources that define the decode step kernels and their launch geometry
+STEP_KERNEL_SOURCES = ("kernels.cuh", "launch.cuh", "ptx.cuh", "stream.cuh")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "recurrent_state_update_deltalog_b200", "csrc", "*"))):
+    csrc = os.path.join(ROOT, "recurrent_state_update_deltalog_b200", "csrc")
+    for f in sorted(os.path.join(csrc, name) for name in STEP_KERNEL_SOURCES):
         with open(f, "rb") as fh:
             h.update(os.path.basename(f).encode())
             h.update(fh.read())

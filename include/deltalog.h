@@ -219,8 +219,8 @@ int dl_read_state(dl_t h, float* S_out, void* stream);
  * DL_OPT_PDL (0 or 1, default 1): a register-tile step that follows an append
  * step of the same handle is launched as a programmatic dependent of the
  * previous kernel in the stream, so it starts streaming Sbar (which an append
- * never writes) while that kernel drains; it reads the log and its inputs
- * only once the previous kernel has completed.  Append steps allow their
+ * never writes) and reading its inputs while that kernel drains; it reads the
+ * log only once the previous kernel has completed.  Append steps allow their
  * successor to launch early; merge steps, dl_eager_step and dl_merge never
  * do.  Disable if other kernels in the stream trigger their dependents early
  * while still writing memory that a later dl_step reads as input. */
