@@ -514,6 +514,7 @@ def run_gpu(a, rank, world, local_rank):
                 "frac": achieved / peak, "traffic": profiled_traffic(workload_name(a)),
                 "kernel": dominant, "avg_launch_us": dur * 1e3,
                 "alg_bytes_per_launch": alg, "peak_source": peak_kind,
+                "frac_of_nominal_8000": achieved / 8000.0,
                 "step_gbs": sb / (ms / a.steps / 1e3) / 1e9}
 
     extra = {}
