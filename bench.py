@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--sweep", default="", help="extra M values to time, e.g. 1,4,16")
     ap.add_argument("--kernel", choices=["auto", "register", "stream"], default="auto",
                     help="dl_step kernel variant")
+    ap.add_argument("--tiles", type=int, default=0, choices=[0, 1, 2, 4],
+                    help="value tiles per head of the register step kernel (0 = automatic)")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch every step with plain stream ordering")
     ap.add_argument("--prefill", type=int, default=0, metavar="L",
@@ -373,6 +375,7 @@ def run_gpu(a, rank, world, local_rank):
         h = DeltaLog(B, H, d, d, m, op=op, dtype=torch.bfloat16)
         h.set_step_kernel(a.kernel)
         h.set_pdl(not a.no_pdl)
+        h.set_value_tiles(a.tiles)
         if a.log_b_bf16 and m > 1:
             h.set_log_b_bf16(True)
         h.load_state(S0)
@@ -579,7 +582,7 @@ def run_gpu(a, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": workload_name(a), "op": op, "B": B, "H": H, "d_k": d, "d_v": d,
                    "M": M, "state": "fp32", "inputs": "bf16", "tokens_per_step": a.tokens,
-                   "step_kernel": used_kernel[0], "pdl": not a.no_pdl,
+                   "step_kernel": used_kernel[0], "pdl": not a.no_pdl, "value_tiles": a.tiles or "auto",
                    "launch": "cuda graph per cycle" if a.graph else "python loop",
                    "m_choice": "dl_suggest_m" if getattr(a, "m_auto", False) else "given",
                    "admit_every_tokens": a.admit_every or None,

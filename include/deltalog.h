@@ -228,7 +228,8 @@ int dl_read_state(dl_t h, float* S_out, void* stream);
  * register-tile step kernel, i.e. how many CTAs split a head's d_v columns
  * (a split below 32 columns per tile falls back to fewer tiles; each tile
  * recomputes the head's key-side coefficients).  Automatic: 2 for d_v = 128
- * while the log holds fewer than 16 entries, else 1. */
+ * while the log holds fewer than 16 entries and the launch has at least two
+ * (slot, head) units per SM, else 1. */
 /* DL_OPT_LOG_B_BF16 (0 or 1, default 0): store the GDN/KDA value factors
  * b_i of the log in bf16 instead of fp32, 516 instead of 772 bytes per entry
  * for GDN d = 128 and 1024 instead of 1280 for KDA.  b_i is rounded to

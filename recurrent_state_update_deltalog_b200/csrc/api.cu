@@ -124,10 +124,11 @@ void free_all(dl_handle* h) {
   if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
 }
 
-// Launch geometry and policies for the handle's current log length.
-dl::LaunchShape shape_of(const dl_handle* h, bool aligned16 = false) {
+// Launch geometry and policies for the handle's current log length and
+// `units` launched (slot, head) units (0: every slot).
+dl::LaunchShape shape_of(const dl_handle* h, bool aligned16 = false, long units = 0) {
   dl::LaunchShape s;
-  s.BH = static_cast<int>(bh(h));
+  s.BH = static_cast<int>(units > 0 ? units : bh(h));
   s.H = h->H;
   s.dk = h->dk;
   s.dv = h->dv;
@@ -143,8 +144,10 @@ dl::LaunchShape shape_of(const dl_handle* h, bool aligned16 = false) {
   s.pdl = h->pdl && !h->wrote_state;
   if (h->value_tiles == 0) {
     // measured on B200: two 64-column tiles per head win for d_v = 128 while
-    // the log is short (each tile recomputes the key-side coefficients)
-    s.split = h->dv == 128 && h->n < 16 ? 2 : 1;
+    // the log is short (each tile recomputes the key-side coefficients) and
+    // the launch has at least two units per SM; below that (GDN B=4, H=32:
+    // 128 units) one tile is 7.7% faster
+    s.split = h->dv == 128 && h->n < 16 && s.BH >= 2 * h->sms ? 2 : 1;
   } else {
     s.split = h->dv / h->value_tiles >= 32 ? h->value_tiles : 1;
   }
@@ -222,8 +225,7 @@ cudaError_t launch_step(dl_handle* h, int mode, const dl::StepArgs& a, int rows,
   // bulk-copy sources of the streaming kernel (GDN's scalar gate is a plain load)
   const bool al = aligned(a.q, 16) && aligned(a.k, 16) && aligned(a.v, 16) && aligned(a.o, 16) &&
                   (h->op == DL_GDN || aligned(a.log_decay, 16));
-  dl::LaunchShape sh = shape_of(h, al);
-  sh.BH = rows * h->H;
+  const dl::LaunchShape sh = shape_of(h, al, static_cast<long>(rows) * h->H);
   int* used = &h->last_kernel;
   switch (h->op) {
     case DL_GDN: return dl::launch_step_op<dl::OP_GDN>(sh, mode, a, s, used);
@@ -233,8 +235,10 @@ cudaError_t launch_step(dl_handle* h, int mode, const dl::StepArgs& a, int rows,
 }
 
 cudaError_t launch_eager(const dl_handle* h, const dl::StepArgs& a, int rows, cudaStream_t s) {
-  dl::LaunchShape sh = shape_of(h);
-  sh.BH = rows * h->H;
+  dl::LaunchShape sh = shape_of(h, false, static_cast<long>(rows) * h->H);
+  // the eager kernel has no per-tile ReplayPrep to repeat: two tiles for
+  // d_v = 128 at every batch size measured (B = 1..1024)
+  if (h->value_tiles == 0) sh.split = h->dv == 128 ? 2 : 1;
   switch (h->op) {
     case DL_GDN: return dl::launch_eager_op<dl::OP_GDN>(sh, a, s);
     case DL_KDA: return dl::launch_eager_op<dl::OP_KDA>(sh, a, s);

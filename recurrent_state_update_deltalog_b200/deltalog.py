@@ -207,7 +207,7 @@ class DeltaLog:
         N.call("dl_set_option", self._h, N.DL_OPT_LOG_B_BF16, 1 if on else 0)
 
     def set_value_tiles(self, n):
-        """0 (automatic), 1 or 2 value tiles (CTAs) per head in the register-tile step kernel."""
+        """0 (automatic), 1, 2 or 4 value tiles (CTAs) per head in the register-tile step kernel."""
         N.call("dl_set_option", self._h, N.DL_OPT_VALUE_TILES, int(n))
 
     @property
