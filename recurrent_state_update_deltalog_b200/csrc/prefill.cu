@@ -6,7 +6,7 @@ namespace dl {
 
 template <int OP, int DK, int DV, typename TI>
 cudaError_t prefill_dims(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st) {
-  prefill_kernel<OP, DK, DV, TI><<<dim3(s.H * (DV / 32), s.units), Tile<DK, 32>::NT, 0, st>>>(a);
+  prefill_kernel<OP, DK, DV, TI><<<dim3(s.H * (DV / PrefillTile<DK>::CW), s.units), 32, 0, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -8,13 +8,15 @@
 // straight into Sbar and clears the slot's log entries; decode steps then
 // append to it like to any merged base.
 //
-// One CTA per (row, head, 32-column value tile) keeps its d_k x 32 slice of
+// One warp per (row, head, 16-column value tile) keeps its d_k x 16 slice of
 // the state in registers for the row's whole prompt; only q, k, v, gates and
 // o stream through HBM (state read once, written once).  Each token runs the
-// eager update of the operator (same arithmetic as the eager step kernel),
+// eager update of the operator (same arithmetic as the eager step kernel)
 // with the next token's inputs prefetched into registers during the current
-// one, so the per-token chain is three block barriers and no global-memory
-// latency.
+// one.  The per-row key-side values pass through double-buffered shared
+// memory behind one __syncwarp, the cross-row reduction is three xor
+// shuffles, and each lane finalises its own four columns: no block barrier
+// on the per-token chain.
 #pragma once
 
 #include "launch.cuh"
@@ -68,156 +70,196 @@ __device__ __forceinline__ void clear_log_tile(const PrefillArgs& a, long sh, in
   }
 }
 
-// d_k = 128 tiles hold 64 state registers per thread next to the prefetched
-// inputs: six CTAs per SM leave them 170 registers without spills.
+// Geometry of the one-warp prefill tile: 16 value columns, lane = 4 x row
+// group + column group; each lane holds RPT rows x 4 columns of the state.
+// Rows are interleaved so that a lane's rows come in runs of four
+// (row = 32 jb + 4 rg + i): its shared-memory reads of per-row values are
+// 128-bit and the eight row groups hit eight different bank quads.
 template <int DK>
-constexpr int kPrefillMinBlocks = DK == 128 ? 6 : 8;
+struct PrefillTile {
+  static constexpr int CW = 16;          // value columns per CTA
+  static constexpr int RG = 8;           // row groups
+  static constexpr int RPT = DK / RG;    // rows per lane
+  static constexpr int KPL = DK / 32;    // keys per lane when loading
+  // resident warps per SM the register budget is sized for (measured on
+  // B200: 16 warps of <= 128 registers beat 12 warps with a two-token input
+  // lookahead by 25% at d_k = 128)
+  static constexpr int MINB = DK == 128 ? 16 : 24;
+  __device__ static int row(int jj, int rg) { return (jj >> 2) * 32 + rg * 4 + (jj & 3); }
+};
 
 template <int OP, int DK, int DV, typename TI>
-__global__ void __launch_bounds__(Tile<DK, 32>::NT, kPrefillMinBlocks<DK>)
+__global__ void __launch_bounds__(32, PrefillTile<DK>::MINB)
 prefill_kernel(const PrefillArgs a) {
-  constexpr int DVT = 32;                 // value columns per CTA
-  constexpr int NSPLIT = DV / DVT;
-  using TL = Tile<DK, DVT>;
+  using PT = PrefillTile<DK>;
+  constexpr int CW = PT::CW, RPT = PT::RPT, KPL = PT::KPL;
+  constexpr int NSPLIT = DV / CW;
   constexpr bool DELTA = OP != OP_RWKV6;
-  static_assert(TL::NT == 64 && TL::KPL * 32 == DK, "prefill tile: two warps, warp 0 owns keys and columns");
+  static_assert(RPT % 4 == 0 && KPL * 32 == DK, "prefill tile shape");
 
-  __shared__ __align__(16) float s_kx[DK];      // contraction vector for p
-  __shared__ __align__(16) float s_qx[DK];      // contraction vector for s
-  __shared__ __align__(16) float s_dec[2][DK];  // per-row decay (double-buffered: read after the last barrier)
-  __shared__ __align__(16) float s_k[2][DK];    // k_t rows of the rank-1 update (double-buffered)
-  __shared__ __align__(16) float s_b[DVT];      // b_t columns of the rank-1 update
-  __shared__ __align__(16) float s_red[2][TL::RG][DVT];
+  // per-row key-side values of a token, double-buffered across tokens
+  __shared__ __align__(16) float s_kx[2][DK];   // contraction vector for p
+  __shared__ __align__(16) float s_qx[2][DK];   // contraction vector for s
+  __shared__ __align__(16) float s_dec[2][DK];  // per-row decay
+  __shared__ __align__(16) float s_k[2][DK];    // k_t rows of the rank-1 update
 
-  const int tid = threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5;
-  const int c4 = tid % TL::TPR, rg = tid / TL::TPR;
+  const int lane = threadIdx.x;
+  const int c4 = lane & 3, rg = lane >> 2;
   const int h = static_cast<int>(blockIdx.x) / NSPLIT;
-  const int col0 = (static_cast<int>(blockIdx.x) % NSPLIT) * DVT;
+  const int col0 = (static_cast<int>(blockIdx.x) % NSPLIT) * CW;
   const int r = blockIdx.y;
 
   const int slot = a.slot_idx ? __ldg(a.slot_idx + r) : r;
   if (slot < 0) return;
   if (slot >= a.slots) {
-    if (tid == 0) atomicOr(a.err, kErrSlotIndex);
+    if (lane == 0) atomicOr(a.err, kErrSlotIndex);
     return;
   }
   const long t0 = __ldg(a.cu_seqlens + r), t1 = __ldg(a.cu_seqlens + r + 1);
   if (t0 < 0 || t1 < t0 || t1 > a.total) {
-    if (tid == 0) atomicOr(a.err, kErrSeqlen);
+    if (lane == 0) atomicOr(a.err, kErrSeqlen);
     return;
   }
   const long sh = static_cast<long>(slot) * a.H + h;
-  float* Sp = a.Sbar + sh * (DK * DV);
+  float* Sp = a.Sbar + sh * (DK * DV) + col0 + 4 * c4;
 
-  float4 st[TL::RPT];
+  float4 st[RPT];
 #pragma unroll
-  for (int j = 0; j < TL::RPT; ++j)
-    st[j] = a.zero_state ? make_float4(0.f, 0.f, 0.f, 0.f) : ld_state(Sp + (rg * TL::RPT + j) * DV + col0 + 4 * c4);
+  for (int jj = 0; jj < RPT; ++jj)
+    st[jj] = a.zero_state ? make_float4(0.f, 0.f, 0.f, 0.f) : ld_state(Sp + PT::row(jj, rg) * DV);
 
-  // Warp 0 holds the next token's inputs: keys j = lane + 32 m, and value
-  // column `lane` of this tile.
-  float kn[TL::KPL], qn[TL::KPL], gn[TL::KPL], vn = 0.f, bn = 0.f;
+  // The next token's inputs, in registers: keys j = lane + 32 m, and this
+  // lane's four value columns (scalar accesses: inputs need only element
+  // alignment).
+  float kn[KPL], qn[KPL], gn[KPL], vn[4], bn = 0.f;
   auto fetch = [&](long t) {
     const long bu = t * a.H + h;
     const TI* qg = static_cast<const TI*>(a.q) + bu * DK;
     const TI* kg = static_cast<const TI*>(a.k) + bu * DK;
 #pragma unroll
-    for (int m = 0; m < TL::KPL; ++m) {
+    for (int m = 0; m < KPL; ++m) {
       const int j = lane + 32 * m;
       kn[m] = to_f(kg[j]);
       qn[m] = to_f(qg[j]);
-      gn[m] = OP == OP_GDN ? (m == 0 ? a.log_decay[bu] : 0.f) : a.log_decay[bu * DK + j];
+      gn[m] = OP == OP_GDN ? 0.f : a.log_decay[bu * DK + j];
     }
-    vn = to_f(static_cast<const TI*>(a.v)[bu * DV + col0 + lane]);
+    if (OP == OP_GDN) gn[0] = a.log_decay[bu];
+    const TI* vg = static_cast<const TI*>(a.v) + bu * DV + col0 + 4 * c4;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) vn[i] = to_f(vg[i]);
     if (DELTA) bn = a.beta[bu];
   };
-  if (warp == 0 && t0 < t1) fetch(t0);
-  float ur[TL::KPL];
+  if (t0 < t1) fetch(t0);
+  float ur[KPL];
 #pragma unroll
-  for (int m = 0; m < TL::KPL; ++m) ur[m] = OP == OP_RWKV6 && warp == 0 ? a.u[h * DK + lane + 32 * m] : 0.f;
+  for (int m = 0; m < KPL; ++m) ur[m] = OP == OP_RWKV6 ? a.u[h * DK + lane + 32 * m] : 0.f;
 
   for (long t = t0; t < t1; ++t) {
     const int buf = static_cast<int>(t & 1);
-    float kap = 0.f, alpha = 1.f;
-    const float vc = vn, betac = bn;
-    if (warp == 0) {
-      if (OP == OP_GDN) alpha = expf(__shfl_sync(0xffffffffu, gn[0], 0));
+    const float4 vc = make_float4(vn[0], vn[1], vn[2], vn[3]);
+    const float betac = bn;
+    const float alpha = OP == OP_GDN ? expf(gn[0]) : 1.f;
+    float kap = 0.f;
 #pragma unroll
-      for (int m = 0; m < TL::KPL; ++m) {
-        const int j = lane + 32 * m;
-        const float dec = OP == OP_GDN ? alpha : expf(gn[m]);
-        s_dec[buf][j] = dec;
-        s_k[buf][j] = kn[m];
-        if (OP == OP_GDN) {          // p = S^T k, s = S^T q (alpha applied after)
-          s_kx[j] = kn[m];
-          s_qx[j] = qn[m];
-          kap = fmaf(kn[m], qn[m], kap);
-        } else if (OP == OP_KDA) {   // p = S^T (alpha (.) k), s = S^T (alpha (.) q)
-          s_kx[j] = dec * kn[m];
-          s_qx[j] = dec * qn[m];
-          kap = fmaf(kn[m], qn[m], kap);
-        } else {                     // RWKV6: s = S^T r, kappa = (u (.) k) . r
-          s_qx[j] = qn[m];
-          kap = fmaf(ur[m] * kn[m], qn[m], kap);
-        }
+    for (int m = 0; m < KPL; ++m) {
+      const int j = lane + 32 * m;
+      const float dec = OP == OP_GDN ? alpha : expf(gn[m]);
+      s_dec[buf][j] = dec;
+      s_k[buf][j] = kn[m];
+      if (OP == OP_GDN) {          // p = S^T k, s = S^T q (alpha applied after)
+        s_kx[buf][j] = kn[m];
+        s_qx[buf][j] = qn[m];
+        kap = fmaf(kn[m], qn[m], kap);
+      } else if (OP == OP_KDA) {   // p = S^T (alpha (.) k), s = S^T (alpha (.) q)
+        s_kx[buf][j] = dec * kn[m];
+        s_qx[buf][j] = dec * qn[m];
+        kap = fmaf(kn[m], qn[m], kap);
+      } else {                     // RWKV6: s = S^T r, kappa = (u (.) k) . r
+        s_qx[buf][j] = qn[m];
+        kap = fmaf(ur[m] * kn[m], qn[m], kap);
       }
-      kap = warp_sum(kap);
-      if (t + 1 < t1) fetch(t + 1);  // in flight during this token's passes
     }
-    __syncthreads();
+    kap = warp_sum(kap);
+    if (t + 1 < t1) fetch(t + 1);  // in flight during this token's passes
+    __syncwarp();
 
-    {
-      float4 p4 = make_float4(0.f, 0.f, 0.f, 0.f), s4 = p4;
+    // contraction over this lane's rows, then over the eight row groups
+    float4 p4 = make_float4(0.f, 0.f, 0.f, 0.f), s4 = p4;
 #pragma unroll
-      for (int j = 0; j < TL::RPT; ++j) {
-        const int row = rg * TL::RPT + j;
-        if (DELTA) fma4(p4, s_kx[row], st[j]);
-        fma4(s4, s_qx[row], st[j]);
+    for (int jb = 0; jb < RPT / 4; ++jb) {
+      const int base = jb * 32 + rg * 4;
+      const float4 qx = *reinterpret_cast<const float4*>(&s_qx[buf][base]);
+      fma4(s4, qx.x, st[4 * jb + 0]);
+      fma4(s4, qx.y, st[4 * jb + 1]);
+      fma4(s4, qx.z, st[4 * jb + 2]);
+      fma4(s4, qx.w, st[4 * jb + 3]);
+      if (DELTA) {
+        const float4 kx = *reinterpret_cast<const float4*>(&s_kx[buf][base]);
+        fma4(p4, kx.x, st[4 * jb + 0]);
+        fma4(p4, kx.y, st[4 * jb + 1]);
+        fma4(p4, kx.z, st[4 * jb + 2]);
+        fma4(p4, kx.w, st[4 * jb + 3]);
       }
-      if (DELTA) *reinterpret_cast<float4*>(&s_red[0][rg][4 * c4]) = p4;
-      *reinterpret_cast<float4*>(&s_red[1][rg][4 * c4]) = s4;
     }
-    __syncthreads();
-
-    if (warp == 0) {  // value column `lane` of the tile
-      float p = 0.f, s = 0.f;
 #pragma unroll
-      for (int g = 0; g < TL::RG; ++g) {
-        if (DELTA) p += s_red[0][g][lane];
-        s += s_red[1][g][lane];
+    for (int off = 4; off < 32; off <<= 1) {
+      s4.x += __shfl_xor_sync(0xffffffffu, s4.x, off);
+      s4.y += __shfl_xor_sync(0xffffffffu, s4.y, off);
+      s4.z += __shfl_xor_sync(0xffffffffu, s4.z, off);
+      s4.w += __shfl_xor_sync(0xffffffffu, s4.w, off);
+      if (DELTA) {
+        p4.x += __shfl_xor_sync(0xffffffffu, p4.x, off);
+        p4.y += __shfl_xor_sync(0xffffffffu, p4.y, off);
+        p4.z += __shfl_xor_sync(0xffffffffu, p4.z, off);
+        p4.w += __shfl_xor_sync(0xffffffffu, p4.w, off);
       }
-      float oc, bt;
+    }
+
+    // this lane's four columns: b_t and o_t (every row group holds the same)
+    float bt[4], oc[4];
+    const float pv[4] = {p4.x, p4.y, p4.z, p4.w}, sv[4] = {s4.x, s4.y, s4.z, s4.w};
+    const float vv[4] = {vc.x, vc.y, vc.z, vc.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
       if (OP == OP_GDN) {
-        bt = betac * (vc - alpha * p);
-        oc = fmaf(kap, bt, alpha * s);
+        bt[i] = betac * (vv[i] - alpha * pv[i]);
+        oc[i] = fmaf(kap, bt[i], alpha * sv[i]);
       } else if (OP == OP_KDA) {
-        bt = betac * (vc - p);
-        oc = fmaf(kap, bt, s);
+        bt[i] = betac * (vv[i] - pv[i]);
+        oc[i] = fmaf(kap, bt[i], sv[i]);
       } else {
-        bt = vc;
-        oc = fmaf(kap, vc, s);
+        bt[i] = vv[i];
+        oc[i] = fmaf(kap, vv[i], sv[i]);
       }
-      s_b[lane] = bt;
-      static_cast<TI*>(a.o)[(t * a.H + h) * DV + col0 + lane] = from_f<TI>(oc);
     }
-    __syncthreads();
-
-    const float4 b4 = *reinterpret_cast<const float4*>(&s_b[4 * c4]);
+    if (rg == 0) {
+      TI* og = static_cast<TI*>(a.o) + (t * a.H + h) * DV + col0 + 4 * c4;
 #pragma unroll
-    for (int j = 0; j < TL::RPT; ++j) {
-      const int row = rg * TL::RPT + j;
-      scale4(st[j], s_dec[buf][row]);
-      fma4(st[j], s_k[buf][row], b4);
+      for (int i = 0; i < 4; ++i) og[i] = from_f<TI>(oc[i]);
+    }
+
+    // S_t = diag(dec) S_{t-1} + k_t b_t^T on this lane's rows and columns
+    const float4 b4 = make_float4(bt[0], bt[1], bt[2], bt[3]);
+#pragma unroll
+    for (int jb = 0; jb < RPT / 4; ++jb) {
+      const int base = jb * 32 + rg * 4;
+      const float4 d4 = *reinterpret_cast<const float4*>(&s_dec[buf][base]);
+      const float4 k4 = *reinterpret_cast<const float4*>(&s_k[buf][base]);
+      const float dd[4] = {d4.x, d4.y, d4.z, d4.w}, kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        scale4(st[4 * jb + i], dd[i]);
+        fma4(st[4 * jb + i], kk[i], b4);
+      }
     }
   }
 
 #pragma unroll
-  for (int j = 0; j < TL::RPT; ++j) st_state(Sp + (rg * TL::RPT + j) * DV + col0 + 4 * c4, st[j]);
-  clear_log_tile<OP, DK, DV, TI>(a, sh, col0, DVT);
+  for (int jj = 0; jj < RPT; ++jj) st_state(Sp + PT::row(jj, rg) * DV, st[jj]);
+  clear_log_tile<OP, DK, DV, TI>(a, sh, col0, CW);
 }
 
-// Grid (H * d_v/32, rows), 64 threads.  Instantiated in prefill.cu.
+// Grid (H * d_v/16, rows), one warp per CTA.  Instantiated in prefill.cu.
 template <int OP>
 cudaError_t launch_prefill_op(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st);
 extern template cudaError_t launch_prefill_op<OP_GDN>(const LaunchShape&, const PrefillArgs&, cudaStream_t);
