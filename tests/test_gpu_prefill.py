@@ -162,3 +162,29 @@ def test_prefill_arguments():
     with pytest.raises(ValueError):
         h.prefill(e3, e3, e3, e2, e2, cu_seqlens=torch.zeros(4, dtype=torch.int32, device="cuda"))
     h.close()
+
+
+@pytest.mark.parametrize("op,H,d", [("gdn", 32, 128), ("kda", 32, 128), ("rwkv6", 64, 64)])
+def test_prefill_full_size_sampled(op, H, d):
+    """The launch bench.py --prefill times (B = 64 prompts of L = 512 tokens,
+    every row from zero): two sampled rows checked token by token, with their
+    final states, against the oracle."""
+    from recurrent_state_update_deltalog_b200 import DeltaLog
+    from synthetic import bonus
+    B, L, dtype = 64, 512, torch.bfloat16
+    seq = sequence(0, op, B, H, d, d, L, bf16=True)
+    u = bonus(0, H, d) if op == "rwkv6" else None
+    packed, cu = _pack(seq, [L] * B)
+    dev = _device_packed(packed, dtype)
+    del packed
+    h = DeltaLog(B, H, d, d, 8, op=op, dtype=dtype)
+    if u is not None:
+        h.set_bonus(torch.from_numpy(u).cuda())
+    o = h.prefill(*_prefill_args(op, dev), cu_seqlens=torch.from_numpy(cu).cuda(), zero_state=True)
+    zero = np.zeros((H, d, d))
+    for r in (0, 37):
+        o_r, S_r = _oracle_row(op, zero, seq, r, L, u)
+        assert relerr(o[r * L:(r + 1) * L].float().cpu().numpy(), o_r[:, 0]) < TOL[dtype], r
+        assert relerr(h.slot_read(r).cpu().numpy(), S_r[0]) < TOL[dtype], r
+    h.check_device()
+    h.close()
