@@ -57,6 +57,9 @@ def parse():
                     help="value tiles per head of the register step kernel (0 = automatic)")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch every step with plain stream ordering")
+    ap.add_argument("--pcie", action="store_true",
+                    help="measure pinned host<->device copy bandwidth (the bound of the e2e line) "
+                         "and print one JSON line")
     ap.add_argument("--prefill", type=int, default=0, metavar="L",
                     help="time the prefill hand-off (dl_prefill) of B prompts of L tokens instead "
                          "of decode; one JSON line, ALU roofline")
@@ -74,7 +77,7 @@ def parse():
                     help="B x M sweep, e.g. '1,16,64,256,1024x1,2,4,8,16,32': one JSON line per "
                          "point (CUDA graphs; M=1 is the eager kernel)")
     args = ap.parse_args()
-    if args.grid or args.prefill:
+    if args.grid or args.prefill or args.pcie:
         return args
     if args.admit_every and args.graph:
         ap.error("--admit-every runs the Python launch loop")
@@ -725,6 +728,32 @@ def run_prefill(a, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def run_pcie(a, local_rank):
+    """Pinned host <-> device copy bandwidth for the copy sizes the e2e line
+    moves (20 back-to-back copies per size, CUDA events)."""
+    import torch
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    out = {}
+    for nbytes in (256 << 10, 2 << 20, 6 << 20, 64 << 20):
+        hb = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+        db = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        res = {}
+        for name, dst, src in (("h2d", db, hb), ("d2h", hb, db)):
+            for _ in range(3):
+                dst.copy_(src, non_blocking=True)
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(20):
+                dst.copy_(src, non_blocking=True)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            res[name + "_gbs"] = nbytes * 20 / (e0.elapsed_time(e1) / 1e3) / 1e9
+        out[f"{nbytes / 1e6:.2f}MB"] = res
+    print(json.dumps({"metric": "pinned copy GB/s", "copies": out}), flush=True)
+
+
 def main():
     a = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -746,6 +775,9 @@ def main():
             run_grid(a, rank, world, local_rank)
         elif a.prefill:
             run_prefill(a, rank, world, local_rank)
+        elif a.pcie:
+            if rank == 0:
+                run_pcie(a, local_rank)
         else:
             line = run_gpu(a, rank, world, local_rank)
             if line is not None:
