@@ -399,21 +399,27 @@ def run_gpu(a, rank, world, local_rank):
 
     def run_step(h, m, eager=False, ev=None, rec=None):
         """One bench step: a.tokens decode tokens through dl_step (or dl_eager_step).
-        With `ev`, every append launch is bracketed by a pair of events (kept in `rec`)."""
+        With `ev`, each cycle's run of append launches (log lengths 0 .. m-2) is
+        bracketed by one pair of events, kept in `rec`: the appends keep their
+        programmatic-launch overlap inside the run, and the run ends where the
+        merge (which never overlaps its predecessor's state) begins."""
+        seg = None
         for j in range(a.tokens):
             i = tok_counter[0] % a.pool
             tok_counter[0] += 1
             args = tok_args(dpool, i)
             if eager:
                 h.eager_step(*args, out=out[i], stream=stream, **tok_map(i))
-            elif ev is not None and (j % m) != m - 1:
-                e0, e1 = ev.pop()
-                e0.record(stream)
-                h.step(*args, out=out[i], stream=stream, **tok_map(i))
-                e1.record(stream)
-                rec.append((e0, e1, j % m))
-            else:
-                h.step(*args, out=out[i], stream=stream, **tok_map(i))
+                continue
+            n = j % m
+            if ev is not None and n == 0 and m > 1:
+                seg = ev.pop()
+                seg[0].record(stream)
+            h.step(*args, out=out[i], stream=stream, **tok_map(i))
+            if seg is not None and n == m - 2:
+                seg[1].record(stream)
+                rec.append((seg[0], seg[1], list(range(m - 1))))
+                seg = None
             if a.admit_every and not eager and tok_counter[0] % a.admit_every == 0:
                 b = (tok_counter[0] // a.admit_every) % B
                 h.slot_load(b, S0[b], stream=stream)
@@ -444,8 +450,8 @@ def run_gpu(a, rank, world, local_rank):
 
     def timed(m, eager=False, per_launch=False):
         """Time a.steps bench steps (or, with per_launch, a shorter second pass in
-        which every append launch is bracketed by its own pair of events: those
-        events sit between launches, so each launch is timed in isolation)."""
+        which each cycle's run of append launches is bracketed by one pair of
+        events: the average append duration of the dominant kernel)."""
         h = make_handle(m)
         if a.graph and not per_launch:
             graphs, cyc = build_graphs(h, m, eager)
@@ -468,7 +474,7 @@ def run_gpu(a, rank, world, local_rank):
         for _ in range(a.warmup):
             run_step(h, m, eager)
         steps = min(a.steps, 2) if per_launch else a.steps
-        nev = steps * a.tokens if per_launch else 0
+        nev = steps * (a.tokens // m + 1) if per_launch else 0
         rec = []
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(nev)]
@@ -482,7 +488,7 @@ def run_gpu(a, rank, world, local_rank):
         ms = start.elapsed_time(stop)
         launches = None
         if per_launch:
-            launches = [(e0.elapsed_time(e1), n) for e0, e1, n in rec]
+            launches = [(e0.elapsed_time(e1), ns) for e0, e1, ns in rec]
         if not eager:
             used_kernel[0] = h.last_step_kernel
         h.check_device(stream)
@@ -507,8 +513,9 @@ def run_gpu(a, rank, world, local_rank):
     result["ms"] = ms
 
     if launches:
-        dur = sum(t for t, _ in launches) / len(launches)
-        alg = sum(launch_bytes(op, "append", B, H, d, d, n, bb=bb) for _, n in launches) / len(launches)
+        count = sum(len(ns) for _, ns in launches)
+        dur = sum(t for t, _ in launches) / count
+        alg = sum(launch_bytes(op, "append", B, H, d, d, n, bb=bb) for _, ns in launches for n in ns) / count
         dominant = ("deltalog_stream_kernel" if used_kernel[0] == "stream"
                     else "deltalog_step_kernel") + " (append)"
     else:   # average over every launch of the step (graph replay or M = 1)
