@@ -252,6 +252,51 @@ def test_zero_log_decay_and_beta_zero_keep_state():
         assert relerr(o, want) < 1e-5
 
 
+def _extreme_gates(op, seq, levels, seed):
+    """Overwrite the gates with a seeded mix of extreme log-decays (per head
+    for GDN, per key otherwise) and betas of 0, 1/2 and 1."""
+    rng = np.random.default_rng(seed)
+    ld = seq["log_decay"]
+    seq["log_decay"] = rng.choice(np.asarray(levels, np.float32), size=ld.shape).astype(np.float32)
+    if "beta" in seq:
+        seq["beta"] = rng.choice(np.asarray([0.0, 0.5, 1.0], np.float32), size=seq["beta"].shape)
+    return seq
+
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("dims", [(64, 64), (128, 128)])
+@pytest.mark.parametrize("M", [8, 64])
+def test_extreme_gates(op, dims, M):
+    """Decays of 0 (no decay), -1e-7, -2 and -40 per step, mixed across keys
+    and steps, and betas of 0, 1/2 and 1: over cycles of up to 64 steps the
+    cumulative log-decay reaches about -2500, where exp(Lam_t) underflows
+    while ratios of recent entries stay near 1."""
+    dk, dv = dims
+    T = 2 * M + 3
+    S0, seq, u = make_inputs(op, 3, 2, dk, dv, T, torch.bfloat16, seed=13)
+    seq = _extreme_gates(op, seq, [0.0, -1e-7, -2.0, -40.0], seed=14)
+    o, merges, final = run_gpu(op, S0, seq, u, M, torch.bfloat16)
+    o_ref, S_ref, rec = run_oracle(op, S0, seq, u, record=tuple(merges))
+    assert np.isfinite(o).all() and np.isfinite(final).all()
+    assert relerr(o, o_ref) < TOL[torch.bfloat16]
+    for t, S in merges.items():
+        assert relerr(S, rec[t]) < TOL[torch.bfloat16], t
+    assert relerr(final, S_ref) < TOL[torch.bfloat16]
+
+
+@pytest.mark.parametrize("op", OPS)
+def test_extreme_gates_fp32(op):
+    """fp32 inputs with decays of 0, -1e-7, -2 and -20 at M = 8: the fp32
+    snapshots (|Lam| <= 140) keep the replay ratios inside the fp32 tolerance."""
+    M, T = 8, 19
+    S0, seq, u = make_inputs(op, 3, 2, 128, 128, T, torch.float32, seed=15)
+    seq = _extreme_gates(op, seq, [0.0, -1e-7, -2.0, -20.0], seed=16)
+    o, merges, final = run_gpu(op, S0, seq, u, M, torch.float32)
+    o_ref, S_ref, _ = run_oracle(op, S0, seq, u)
+    assert relerr(o, o_ref) < TOL[torch.float32]
+    assert relerr(final, S_ref) < TOL[torch.float32]
+
+
 def test_unaligned_inputs_fall_back_or_refuse():
     """q/k/v views offset by one element: AUTO runs the register kernel (same
     result), STREAM refuses with DL_ERR_UNSUPPORTED."""
