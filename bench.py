@@ -57,6 +57,8 @@ def parse():
                     help="value tiles per head of the register step kernel (0 = automatic)")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch every step with plain stream ordering")
+    ap.add_argument("--prefill-kernel", choices=["auto", "recurrent", "chunked"], default="auto",
+                    help="kernel behind dl_prefill (with --prefill)")
     ap.add_argument("--pcie", action="store_true",
                     help="measure pinned host<->device copy bandwidth (the bound of the e2e line) "
                          "and print one JSON line")
@@ -669,6 +671,7 @@ def run_prefill(a, rank, world, local_rank):
     cu = torch.arange(0, (B + 1) * L, L, dtype=torch.int32, device=dev)
     u = torch.from_numpy(bonus(seed, H, d)).to(dev) if op == "rwkv6" else None
     h = DeltaLog(B, H, d, d, a.M, op=op, dtype=torch.bfloat16)
+    h.set_prefill_kernel(a.prefill_kernel)
     if u is not None:
         h.set_bonus(u)
     o = torch.empty((B * L, H, d), dtype=torch.bfloat16, device=dev)
@@ -723,7 +726,7 @@ def run_prefill(a, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": f"{op}_prefill_b{B}_l{L}_h{H}_d{d}_bf16", "op": op, "B": B, "L": L,
                    "H": H, "d_k": d, "d_v": d, "state": "fp32", "inputs": "bf16",
-                   "start": "zero state", "kernel": "prefill_kernel (64 threads, 32 value columns)"},
+                   "start": "zero state", "kernel": h.last_prefill_kernel},
         "roofline": {"bound": "alu", "achieved": flops, "peak": peak, "unit": "TFLOP/s",
                      "frac": flops / peak, "traffic": None,
                      "peak_note": "fp32 SIMT at the 1965 MHz max clock: 148 SMs x 128 lanes x 2 flops",

@@ -241,19 +241,37 @@ int dl_read_state(dl_t h, float* S_out, void* stream);
  * otherwise); a no-op for RWKV6, whose log already holds raw bf16 v_i.
  * Changeable only while the log is empty (DL_ERR_STATE otherwise).  The
  * streaming kernel does not take it (DL_ERR_UNSUPPORTED). */
+/* DL_OPT_PREFILL_KERNEL picks the kernel behind dl_prefill:
+ *   DL_PREFILL_AUTO (default): the chunked kernel for bf16-input GDN handles
+ *     when the batch is too small to fill the GPU with the recurrent kernel
+ *     (rows x H x d_v/16 < 8 x SMs), the recurrent kernel otherwise;
+ *   DL_PREFILL_RECURRENT: the recurrence token by token, state in registers
+ *     (every operator and dtype; outputs equal the eager recurrence's up to
+ *     fp32 rounding);
+ *   DL_PREFILL_CHUNKED: 64-token chunks in the WY form of the delta rule on
+ *     tensor cores (bf16 products of the inputs, tf32 products with the
+ *     state; bf16-input GDN handles only, DL_ERR_UNSUPPORTED otherwise).
+ *     Its tf32 products round to 2^-11 relative, inside the bf16-input
+ *     tolerance. */
 enum dl_option {
   DL_OPT_STEP_KERNEL = 0,
   DL_OPT_HOST_PREFETCH = 1,
   DL_OPT_PDL = 2,
   DL_OPT_VALUE_TILES = 3,
-  DL_OPT_LOG_B_BF16 = 4
+  DL_OPT_LOG_B_BF16 = 4,
+  DL_OPT_PREFILL_KERNEL = 5
 };
+enum dl_prefill_kernel { DL_PREFILL_AUTO = 0, DL_PREFILL_RECURRENT = 1, DL_PREFILL_CHUNKED = 2 };
 enum dl_step_kernel { DL_STEP_AUTO = 0, DL_STEP_REGISTER = 1, DL_STEP_STREAM = 2 };
 int dl_set_option(dl_t h, int option, int value);
 
 /* Which kernel the most recent dl_step / dl_step_host launched:
  * DL_STEP_REGISTER or DL_STEP_STREAM (DL_STEP_AUTO before the first step). */
 int dl_last_step_kernel(dl_t h, int* kind);
+
+/* Which kernel the most recent dl_prefill launched: DL_PREFILL_RECURRENT or
+ * DL_PREFILL_CHUNKED (DL_PREFILL_AUTO before the first prefill). */
+int dl_last_prefill_kernel(dl_t h, int* kind);
 
 /* Number of entries currently in every slot's log (host-side counter, exact
  * in stream order). */

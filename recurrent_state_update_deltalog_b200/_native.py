@@ -22,6 +22,8 @@ DL_OPT_HOST_PREFETCH = 1
 DL_OPT_PDL = 2
 DL_OPT_VALUE_TILES = 3
 DL_OPT_LOG_B_BF16 = 4
+DL_OPT_PREFILL_KERNEL = 5
+DL_PREFILL_AUTO, DL_PREFILL_RECURRENT, DL_PREFILL_CHUNKED = 0, 1, 2
 DL_STEP_AUTO, DL_STEP_REGISTER, DL_STEP_STREAM = 0, 1, 2
 STATUS = {0: "DL_OK", -1: "DL_ERR_ARG", -2: "DL_ERR_UNSUPPORTED", -3: "DL_ERR_CUDA",
           -4: "DL_ERR_OOM", -5: "DL_ERR_DEVICE", -6: "DL_ERR_STATE"}
@@ -37,6 +39,7 @@ SIGNATURES = {
     "dl_suggest_m": (_I, [_I, _I, _I, _I, ctypes.POINTER(_I)]),
     "dl_merge_interval": (_I, [_P, ctypes.POINTER(_I)]),
     "dl_prefill": (_I, [_P, _P, _I, _P, ctypes.c_longlong, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "dl_last_prefill_kernel": (_I, [_P, ctypes.POINTER(_I)]),
     "dl_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
     "dl_step_indexed": (_I, [_P, _P, _I, _P, _P, _P, _P, _P, _P, _P]),
     "dl_step_host": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),

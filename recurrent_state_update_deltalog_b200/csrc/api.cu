@@ -51,6 +51,8 @@ struct dl_handle {
   int pdl;                  // DL_OPT_PDL
   int value_tiles;          // DL_OPT_VALUE_TILES (0 = automatic)
   int log_b_bf16;           // DL_OPT_LOG_B_BF16
+  int prefill_kernel;       // DL_OPT_PREFILL_KERNEL (DL_PREFILL_*)
+  int last_prefill;         // DL_PREFILL_* used by the last dl_prefill
 };
 
 namespace {
@@ -295,9 +297,27 @@ cudaError_t materialize_slots(const dl_handle* h, const int* slot_idx, int rows,
   }
 }
 
-cudaError_t launch_prefill(const dl_handle* h, const dl::PrefillArgs& a, int rows, cudaStream_t s) {
+// The chunked tensor-core prefill serves bf16-input GDN handles.  AUTO picks
+// it there when the recurrent kernel's warps (rows x H x d_v/16) would not
+// fill the GPU: B200 measured GDN d=128, 4 prompts of 4096 tokens 4.25 vs
+// 3.76 M tokens/s for the chunked kernel, 64 prompts of 512 tokens 4.84 vs
+// 7.30 for the recurrent one.
+bool chunked_prefill(const dl_handle* h, int rows) {
+  const bool ok = h->op == DL_GDN && h->dtype == DL_BF16;
+  const long recurrent_warps = static_cast<long>(rows) * h->H * (h->dv / 16);
+  return h->prefill_kernel == DL_PREFILL_CHUNKED ||
+         (h->prefill_kernel == DL_PREFILL_AUTO && ok && recurrent_warps < 8L * h->sms);
+}
+
+cudaError_t launch_prefill(dl_handle* h, const dl::PrefillArgs& a, int rows, cudaStream_t s) {
   dl::LaunchShape sh = shape_of(h);
   sh.units = rows;
+  if (chunked_prefill(h, rows)) {
+    if (h->op != DL_GDN || h->dtype != DL_BF16) return cudaErrorNotSupported;
+    h->last_prefill = DL_PREFILL_CHUNKED;
+    return dl::launch_gdn_chunk_prefill_dims(sh, a, s);
+  }
+  h->last_prefill = DL_PREFILL_RECURRENT;
   switch (h->op) {
     case DL_GDN: return dl::launch_prefill_op<dl::OP_GDN>(sh, a, s);
     case DL_KDA: return dl::launch_prefill_op<dl::OP_KDA>(sh, a, s);
@@ -581,6 +601,8 @@ int dl_prefill(dl_t h, const int* slot_idx, int rows, const int* cu_seqlens, lon
   a.b_esize = static_cast<int>(logb_esize(h));
   a.zero_state = zero ? 1 : 0;
   cudaError_t e = launch_prefill(h, a, rows, s);
+  if (e == cudaErrorNotSupported)
+    return fail(DL_ERR_UNSUPPORTED, "the chunked prefill serves bf16-input GDN handles that fit its shared memory");
   if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
   h->wrote_state = true;
   return DL_OK;
@@ -759,6 +781,11 @@ int dl_set_option(dl_t h, int option, int value) {
       if (value != 0 && value != 1) return fail(DL_ERR_ARG, "bad PDL value %d", value);
       h->pdl = value;
       return DL_OK;
+    case DL_OPT_PREFILL_KERNEL:
+      if (value < DL_PREFILL_AUTO || value > DL_PREFILL_CHUNKED)
+        return fail(DL_ERR_ARG, "bad prefill-kernel value %d", value);
+      h->prefill_kernel = value;
+      return DL_OK;
     case DL_OPT_LOG_B_BF16:
       if (value != 0 && value != 1) return fail(DL_ERR_ARG, "bad log-b-bf16 value %d", value);
       if (value && h->dtype != DL_BF16) return fail(DL_ERR_UNSUPPORTED, "a bf16 b-log needs bf16 inputs");
@@ -779,6 +806,12 @@ int dl_set_option(dl_t h, int option, int value) {
 int dl_last_step_kernel(dl_t h, int* kind) {
   if (!h || !kind) return fail(DL_ERR_ARG, "null argument");
   *kind = h->last_kernel;
+  return DL_OK;
+}
+
+int dl_last_prefill_kernel(dl_t h, int* kind) {
+  if (!h || !kind) return fail(DL_ERR_ARG, "null argument");
+  *kind = h->last_prefill;
   return DL_OK;
 }
 

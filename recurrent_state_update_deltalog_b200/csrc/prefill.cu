@@ -1,6 +1,7 @@
 // Instantiations of the prefill hand-off kernel (every operator, shape and
 // input dtype) in a translation unit of their own.
 #include "prefill.cuh"
+#include "prefill_chunk.cuh"
 
 namespace dl {
 
@@ -13,6 +14,25 @@ cudaError_t prefill_dims(const LaunchShape& s, const PrefillArgs& a, cudaStream_
 template <int OP>
 cudaError_t launch_prefill_op(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st) {
   DL_DISPATCH_DIMS(prefill_dims, s, a, st);
+}
+
+template <int DK, int DV>
+cudaError_t launch_gdn_chunk_prefill(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st) {
+  using G = ChunkGeom<DK>;
+  auto kern = gdn_chunk_prefill_kernel<DK, DV>;
+  if (G::BYTES + 8 * 1024 > static_cast<size_t>(s.smem_block_optin)) return cudaErrorNotSupported;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(G::BYTES));
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(s.H * (DV / G::VT), s.units), G::NT, G::BYTES, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gdn_chunk_prefill_dims(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st) {
+  if (s.dk == 64 && s.dv == 64) return launch_gdn_chunk_prefill<64, 64>(s, a, st);
+  if (s.dk == 128 && s.dv == 128) return launch_gdn_chunk_prefill<128, 128>(s, a, st);
+  if (s.dk == 64 && s.dv == 128) return launch_gdn_chunk_prefill<64, 128>(s, a, st);
+  if (s.dk == 128 && s.dv == 64) return launch_gdn_chunk_prefill<128, 64>(s, a, st);
+  return cudaErrorInvalidValue;
 }
 
 template cudaError_t launch_prefill_op<OP_GDN>(const LaunchShape&, const PrefillArgs&, cudaStream_t);

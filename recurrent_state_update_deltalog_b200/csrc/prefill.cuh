@@ -259,6 +259,11 @@ prefill_kernel(const PrefillArgs a) {
   clear_log_tile<OP, DK, DV, TI>(a, sh, col0, CW);
 }
 
+// Chunked tensor-core GDN prefill (bf16 inputs; prefill_chunk.cuh), any
+// supported d_k x d_v.  cudaErrorNotSupported when its shared memory does not
+// fit the device.
+cudaError_t launch_gdn_chunk_prefill_dims(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st);
+
 // Grid (H * d_v/16, rows), one warp per CTA.  Instantiated in prefill.cu.
 template <int OP>
 cudaError_t launch_prefill_op(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st);

@@ -202,6 +202,18 @@ class DeltaLog:
         """Programmatic dependent launch of steps that follow an append (default on)."""
         N.call("dl_set_option", self._h, N.DL_OPT_PDL, 1 if on else 0)
 
+    def set_prefill_kernel(self, kind):
+        """``"auto"`` (default), ``"recurrent"`` or ``"chunked"``: which kernel runs prefill."""
+        vals = {"auto": N.DL_PREFILL_AUTO, "recurrent": N.DL_PREFILL_RECURRENT, "chunked": N.DL_PREFILL_CHUNKED}
+        N.call("dl_set_option", self._h, N.DL_OPT_PREFILL_KERNEL, vals[kind])
+
+    @property
+    def last_prefill_kernel(self):
+        """Kernel used by the most recent prefill: ``"recurrent"``, ``"chunked"`` or ``None``."""
+        k = ctypes.c_int()
+        N.call("dl_last_prefill_kernel", self._h, ctypes.byref(k))
+        return {N.DL_PREFILL_RECURRENT: "recurrent", N.DL_PREFILL_CHUNKED: "chunked"}.get(k.value)
+
     def set_log_b_bf16(self, on):
         """Store GDN/KDA log value factors b_i in bf16 (bf16 handles, empty log)."""
         N.call("dl_set_option", self._h, N.DL_OPT_LOG_B_BF16, 1 if on else 0)

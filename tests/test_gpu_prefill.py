@@ -50,11 +50,13 @@ def _oracle_row(op, S_init, seq, r, n, u):
 @pytest.mark.parametrize("op", OPS)
 @pytest.mark.parametrize("dims", [(64, 64), (128, 128), (64, 128), (128, 64)])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-def test_prefill_then_decode(op, dims, dtype):
+@pytest.mark.parametrize("kernel", ["auto", "recurrent", "chunked"])
+def test_prefill_then_decode(op, dims, dtype, kernel):
+    """Prompts of 37, 0, 1, 64 + 66 (two chunks and a ragged tail) and 5 tokens."""
     from recurrent_state_update_deltalog_b200 import DeltaLog
     dk, dv = dims
     B, H, M, T_dec = 8, 3, 4, 7
-    lens = [37, 0, 1, 64, 5]
+    lens = [37, 0, 1, 130, 5]
     slots = [6, 0, 3, 1, 4]
     rows = len(lens)
     bf16 = dtype == torch.bfloat16
@@ -64,7 +66,10 @@ def test_prefill_then_decode(op, dims, dtype):
     tol = TOL[dtype]
 
     S_pool = initial_state(5, B, H, dk, dv)             # other slots keep this
+    if kernel == "chunked" and not (op == "gdn" and dtype == torch.bfloat16):
+        pytest.skip("the chunked prefill serves bf16-input GDN handles (refusal tested below)")
     h = DeltaLog(B, H, dk, dv, M, op=op, dtype=dtype)
+    h.set_prefill_kernel(kernel)
     h.load_state(torch.from_numpy(S_pool).cuda())
     if u is not None:
         h.set_bonus(torch.from_numpy(u).cuda())
@@ -79,6 +84,8 @@ def test_prefill_then_decode(op, dims, dtype):
     o = h.prefill(*_prefill_args(op, d), cu_seqlens=torch.from_numpy(cu).cuda(),
                   slot_idx=torch.tensor(slots, dtype=torch.int32, device="cuda"), zero_state=True)
     assert h.log_len == 2                                # the handle's cycle is unchanged
+    applies = op == "gdn" and dtype == torch.bfloat16
+    assert h.last_prefill_kernel == ("chunked" if kernel != "recurrent" and applies else "recurrent")
     got = o.float().cpu().numpy()
     zero = np.zeros((H, dk, dv))
     for r, (n, b) in enumerate(zip(lens, slots)):
@@ -102,13 +109,17 @@ def test_prefill_then_decode(op, dims, dtype):
 
 
 @pytest.mark.parametrize("op", OPS)
-def test_prefill_continues_logical_state(op):
+@pytest.mark.parametrize("kernel", ["auto", "recurrent", "chunked"])
+def test_prefill_continues_logical_state(op, kernel):
     """Without DL_PREFILL_ZERO_STATE a prompt continues from the slot's
     logical state (base + log), e.g. the second chunk of a long prompt."""
     from recurrent_state_update_deltalog_b200 import DeltaLog
     dtype, dk, dv, B, H, M = torch.bfloat16, 128, 128, 4, 2, 8
+    if kernel == "chunked" and op != "gdn":
+        pytest.skip("the chunked prefill serves bf16-input GDN handles (refusal tested below)")
     S0, warm, u = make_inputs(op, B, H, dk, dv, 5, dtype, seed=31)
     h = DeltaLog(B, H, dk, dv, M, op=op, dtype=dtype)
+    h.set_prefill_kernel(kernel)
     h.load_state(torch.from_numpy(S0).cuda())
     if u is not None:
         h.set_bonus(torch.from_numpy(u).cuda())
@@ -116,7 +127,7 @@ def test_prefill_continues_logical_state(op):
     for t in range(5):
         h.step(*step_args(op, dwarm, t))
     _, S_ref, _ = run_oracle(op, S0, warm, u)
-    lens = [20, 33, 0, 9]
+    lens = [20, 97, 0, 9]
     seq = sequence(32, op, B, H, dk, dv, max(lens), bf16=True)
     packed, cu = _pack(seq, lens)
     d = _device_packed(packed, dtype)
@@ -164,8 +175,9 @@ def test_prefill_arguments():
     h.close()
 
 
-@pytest.mark.parametrize("op,H,d", [("gdn", 32, 128), ("kda", 32, 128), ("rwkv6", 64, 64)])
-def test_prefill_full_size_sampled(op, H, d):
+@pytest.mark.parametrize("op,H,d,kernel", [("gdn", 32, 128, "chunked"), ("gdn", 32, 128, "recurrent"),
+                                           ("kda", 32, 128, "auto"), ("rwkv6", 64, 64, "auto")])
+def test_prefill_full_size_sampled(op, H, d, kernel):
     """The launch bench.py --prefill times (B = 64 prompts of L = 512 tokens,
     every row from zero): two sampled rows checked token by token, with their
     final states, against the oracle."""
@@ -178,6 +190,7 @@ def test_prefill_full_size_sampled(op, H, d):
     dev = _device_packed(packed, dtype)
     del packed
     h = DeltaLog(B, H, d, d, 8, op=op, dtype=dtype)
+    h.set_prefill_kernel(kernel)
     if u is not None:
         h.set_bonus(torch.from_numpy(u).cuda())
     o = h.prefill(*_prefill_args(op, dev), cu_seqlens=torch.from_numpy(cu).cuda(), zero_state=True)
@@ -188,3 +201,18 @@ def test_prefill_full_size_sampled(op, H, d):
         assert relerr(h.slot_read(r).cpu().numpy(), S_r[0]) < TOL[dtype], r
     h.check_device()
     h.close()
+
+
+def test_chunked_prefill_refused_where_it_does_not_apply():
+    """The chunked kernel serves bf16-input GDN handles only."""
+    from recurrent_state_update_deltalog_b200 import DeltaLog, DeltaLogError
+    for op, dtype in (("kda", torch.bfloat16), ("rwkv6", torch.bfloat16), ("gdn", torch.float32)):
+        h = DeltaLog(2, 2, 64, 64, 4, op=op, dtype=dtype)
+        h.set_prefill_kernel("chunked")
+        x = torch.zeros((3, 2, 64), device="cuda", dtype=dtype)
+        g = torch.zeros((3, 2) if op == "gdn" else (3, 2, 64), device="cuda")
+        b = None if op == "rwkv6" else torch.zeros((3, 2), device="cuda")
+        cu = torch.tensor([0, 3, 3], dtype=torch.int32, device="cuda")
+        with pytest.raises(DeltaLogError):
+            h.prefill(x, x, x, g, b, cu_seqlens=cu, zero_state=True)
+        h.close()
