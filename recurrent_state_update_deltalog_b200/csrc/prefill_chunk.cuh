@@ -54,7 +54,7 @@ struct ChunkGeom {
   static constexpr size_t W_OFF = al(A_OFF + size_t(C) * LDA * 4);
   static constexpr size_t U_OFF = al(W_OFF + size_t(C) * LDW * 4);
   static constexpr size_t G_OFF = al(U_OFF + size_t(C) * LDS * 4);
-  static constexpr size_t BYTES = al(G_OFF + 2 * C * 4);   // Gamma and beta
+  static constexpr size_t BYTES = al(G_OFF + 5 * C * 4);   // Gamma, beta and three per-row factors
 };
 
 namespace wm = nvcuda::wmma;
@@ -136,6 +136,9 @@ __global__ void __launch_bounds__(256, 1) gdn_chunk_prefill_kernel(const Prefill
   float* sU = reinterpret_cast<float*>(smem + G::U_OFF);                  // [C][LDS] U, then B
   float* sG = reinterpret_cast<float*>(smem + G::G_OFF);                  // [C] Gamma
   float* sBeta = sG + C;                                                  // [C] beta
+  float* sEG = sG + 2 * C;    // [C] e^{Gamma_t}
+  float* sBEG = sG + 3 * C;   // [C] beta_t e^{Gamma_t}
+  float* sEnd = sG + 4 * C;   // [C] e^{Gamma_end - Gamma_t} (0 past the prompt)
   __shared__ __align__(32) float s_patch[8][16 * 16];                     // per-warp output tile
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -241,10 +244,19 @@ __global__ void __launch_bounds__(256, 1) gdn_chunk_prefill_kernel(const Prefill
         if (lane >= off) incl += y;
       }
       const float excl = incl - pair;
-      sG[ta] = excl + g0;
-      sG[tb] = excl + pair;
+      const float Ga = excl + g0, Gb = excl + pair;
+      sG[ta] = Ga;
+      sG[tb] = Gb;
       sBeta[ta] = bn0;
       sBeta[tb] = bn1;
+      const float ea = expf(Ga), eb = expf(Gb);
+      sEG[ta] = ea;
+      sEG[tb] = eb;
+      sBEG[ta] = bn0 * ea;
+      sBEG[tb] = bn1 * eb;
+      const float gend = __shfl_sync(0xffffffffu, (n - 1) & 1 ? Gb : Ga, (n - 1) >> 1);
+      sEnd[ta] = ta < n ? expf(gend - Ga) : 0.f;
+      sEnd[tb] = tb < n ? expf(gend - Gb) : 0.f;
       if (has_next) fetch_gates(c0 + C);
     }
     __syncthreads();
@@ -260,7 +272,7 @@ __global__ void __launch_bounds__(256, 1) gdn_chunk_prefill_kernel(const Prefill
     // right-hand sides: beta e^{G} K into W, beta V into U
     for (int idx = tid; idx < C * DK; idx += G::NT) {
       const int t = idx / DK, j = idx % DK;
-      sW[t * G::LDW + j] = sBeta[t] * expf(sG[t]) * __bfloat162float(sK[t * G::LDK + j]);
+      sW[t * G::LDW + j] = sBEG[t] * __bfloat162float(sK[t * G::LDK + j]);
     }
     for (int idx = tid; idx < C * VT; idx += G::NT) {
       const int t = idx / VT, c = idx % VT;
@@ -269,21 +281,28 @@ __global__ void __launch_bounds__(256, 1) gdn_chunk_prefill_kernel(const Prefill
     __syncthreads();
 
     // 3. (I + A) X = R, one right-hand-side column per thread
+    // (W is a tf32 operand later and is stored tf32-rounded; U stays fp32.)
     if (tid < DK + VT) {
-      float* col = tid < DK ? sW + tid : sU + (tid - DK);
-      const int ld = tid < DK ? G::LDW : G::LDS;
+      const bool isw = tid < DK;
+      float* col = isw ? sW + tid : sU + (tid - DK);
+      const int ld = isw ? G::LDW : G::LDS;
       float x[C];
 #pragma unroll
       for (int t = 0; t < C; ++t) {
         float acc0 = col[t * ld], acc1 = 0.f;
+        const float* arow = sA + t * G::LDA;
 #pragma unroll
-        for (int s = 0; s + 1 < t; s += 2) {
-          acc0 = fmaf(-sA[t * G::LDA + s], x[s], acc0);
-          acc1 = fmaf(-sA[t * G::LDA + s + 1], x[s + 1], acc1);
+        for (int s = 0; s + 3 < t; s += 4) {
+          const float4 a4 = *reinterpret_cast<const float4*>(arow + s);
+          acc0 = fmaf(-a4.x, x[s], acc0);
+          acc1 = fmaf(-a4.y, x[s + 1], acc1);
+          acc0 = fmaf(-a4.z, x[s + 2], acc0);
+          acc1 = fmaf(-a4.w, x[s + 3], acc1);
         }
-        if (t & 1) acc0 = fmaf(-sA[t * G::LDA + t - 1], x[t - 1], acc0);
+#pragma unroll
+        for (int s = t & ~3; s < t; ++s) acc0 = fmaf(-arow[s], x[s], acc0);
         x[t] = acc0 + acc1;
-        col[t * ld] = x[t];
+        col[t * ld] = isw ? wm::__float_to_tf32(x[t]) : x[t];
       }
     }
     __syncthreads();
@@ -296,9 +315,8 @@ __global__ void __launch_bounds__(256, 1) gdn_chunk_prefill_kernel(const Prefill
       for (int kk = 0; kk < DK; kk += 8) {
         TfA fa;
         TfB fb;
-        wm::load_matrix_sync(fa, sW + (16 * i) * G::LDW + kk, G::LDW);
+        wm::load_matrix_sync(fa, sW + (16 * i) * G::LDW + kk, G::LDW);   // tf32-rounded already
         wm::load_matrix_sync(fb, sS + kk * G::LDS + 16 * j, G::LDS);
-        to_tf32(fa);
         to_tf32(fb);
         wm::mma_sync(acc, fa, fb, acc);
       }
@@ -306,7 +324,7 @@ __global__ void __launch_bounds__(256, 1) gdn_chunk_prefill_kernel(const Prefill
       float* p = sU + (16 * i) * G::LDS + 16 * j;
       wm::load_matrix_sync(u, p, G::LDS, wm::mem_row_major);
 #pragma unroll
-      for (int e = 0; e < u.num_elements; ++e) u.x[e] -= acc.x[e];
+      for (int e = 0; e < u.num_elements; ++e) u.x[e] = wm::__float_to_tf32(u.x[e] - acc.x[e]);   // B, a tf32 operand
       wm::store_matrix_sync(p, u, G::LDS, wm::mem_row_major);
     });
     __syncthreads();
@@ -315,13 +333,13 @@ __global__ void __launch_bounds__(256, 1) gdn_chunk_prefill_kernel(const Prefill
     lower_xyt<DK, G::LDK, G::LDA>(sQ, sK, sA);
     for (int idx = tid; idx < C * DK; idx += G::NT) {
       const int t = idx / DK, j = idx % DK;
-      sW[t * G::LDW + j] = expf(sG[t]) * __bfloat162float(sQ[t * G::LDK + j]);
+      sW[t * G::LDW + j] = wm::__float_to_tf32(sEG[t] * __bfloat162float(sQ[t * G::LDK + j]));
     }
     __syncthreads();
     for (int idx = tid; idx < C * C; idx += G::NT) {
       const int t = idx / C, s = idx % C;
       float& x = sA[t * G::LDA + s];
-      x = s <= t ? expf(sG[t] - sG[s]) * x : 0.f;
+      x = s <= t ? wm::__float_to_tf32(expf(sG[t] - sG[s]) * x) : 0.f;
     }
     __syncthreads();
 
@@ -333,19 +351,16 @@ __global__ void __launch_bounds__(256, 1) gdn_chunk_prefill_kernel(const Prefill
       for (int kk = 0; kk < DK; kk += 8) {
         TfA fa;
         TfB fb;
-        wm::load_matrix_sync(fa, sW + (16 * i) * G::LDW + kk, G::LDW);
+        wm::load_matrix_sync(fa, sW + (16 * i) * G::LDW + kk, G::LDW);   // e^G Q, tf32-rounded
         wm::load_matrix_sync(fb, sS + kk * G::LDS + 16 * j, G::LDS);
-        to_tf32(fa);
         to_tf32(fb);
         wm::mma_sync(acc, fa, fb, acc);
       }
       for (int kk = 0; kk < 16 * (i + 1); kk += 8) {   // P is lower triangular
         TfA fa;
         TfB fb;
-        wm::load_matrix_sync(fa, sA + (16 * i) * G::LDA + kk, G::LDA);
-        wm::load_matrix_sync(fb, sU + kk * G::LDS + 16 * j, G::LDS);
-        to_tf32(fa);
-        to_tf32(fb);
+        wm::load_matrix_sync(fa, sA + (16 * i) * G::LDA + kk, G::LDA);   // P, tf32-rounded
+        wm::load_matrix_sync(fb, sU + kk * G::LDS + 16 * j, G::LDS);     // B, tf32-rounded
         wm::mma_sync(acc, fa, fb, acc);
       }
       float* patch = s_patch[warp];
@@ -360,13 +375,12 @@ __global__ void __launch_bounds__(256, 1) gdn_chunk_prefill_kernel(const Prefill
     __syncthreads();
 
     // 7. S <- e^{G_end} S + (e^{G_end - G} K)^T B
-    const float gend = sG[n > 0 ? n - 1 : 0];
     for (int idx = tid; idx < C * DK; idx += G::NT) {
       const int t = idx / DK, j = idx % DK;
-      sW[t * G::LDW + j] = t < n ? expf(gend - sG[t]) * __bfloat162float(sK[t * G::LDK + j]) : 0.f;
+      sW[t * G::LDW + j] = wm::__float_to_tf32(sEnd[t] * __bfloat162float(sK[t * G::LDK + j]));
     }
     __syncthreads();
-    const float dend = expf(gend);
+    const float dend = sEG[n - 1];
     for_tiles<DK, VT>([&](int i, int j) {
       AccTf acc;
       float* p = sS + (16 * i) * G::LDS + 16 * j;
@@ -377,10 +391,8 @@ __global__ void __launch_bounds__(256, 1) gdn_chunk_prefill_kernel(const Prefill
       for (int kk = 0; kk < C; kk += 8) {
         TfAc fa;
         TfB fb;
-        wm::load_matrix_sync(fa, sW + kk * G::LDW + 16 * i, G::LDW);   // (e^{..} K)^T, col-major
-        wm::load_matrix_sync(fb, sU + kk * G::LDS + 16 * j, G::LDS);
-        to_tf32(fa);
-        to_tf32(fb);
+        wm::load_matrix_sync(fa, sW + kk * G::LDW + 16 * i, G::LDW);   // (e^{..} K)^T, col-major, tf32
+        wm::load_matrix_sync(fb, sU + kk * G::LDS + 16 * j, G::LDS);     // B, tf32
         wm::mma_sync(acc, fa, fb, acc);
       }
       wm::store_matrix_sync(p, acc, G::LDS, wm::mem_row_major);
