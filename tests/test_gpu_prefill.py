@@ -47,10 +47,14 @@ def _oracle_row(op, S_init, seq, r, n, u):
     return o, S
 
 
-@pytest.mark.parametrize("op", OPS)
+# the chunked kernel serves bf16-input GDN handles only (its refusal elsewhere
+# is tested below)
+_KERNELS = [(op, dt, k) for op in OPS for dt in (torch.bfloat16, torch.float32)
+            for k in ("auto", "recurrent", "chunked") if k != "chunked" or (op == "gdn" and dt == torch.bfloat16)]
+
+
+@pytest.mark.parametrize("op,dtype,kernel", _KERNELS)
 @pytest.mark.parametrize("dims", [(64, 64), (128, 128), (64, 128), (128, 64)])
-@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-@pytest.mark.parametrize("kernel", ["auto", "recurrent", "chunked"])
 def test_prefill_then_decode(op, dims, dtype, kernel):
     """Prompts of 37, 0, 1, 64 + 66 (two chunks and a ragged tail) and 5 tokens."""
     from recurrent_state_update_deltalog_b200 import DeltaLog
@@ -66,8 +70,6 @@ def test_prefill_then_decode(op, dims, dtype, kernel):
     tol = TOL[dtype]
 
     S_pool = initial_state(5, B, H, dk, dv)             # other slots keep this
-    if kernel == "chunked" and not (op == "gdn" and dtype == torch.bfloat16):
-        pytest.skip("the chunked prefill serves bf16-input GDN handles (refusal tested below)")
     h = DeltaLog(B, H, dk, dv, M, op=op, dtype=dtype)
     h.set_prefill_kernel(kernel)
     h.load_state(torch.from_numpy(S_pool).cuda())
@@ -108,15 +110,13 @@ def test_prefill_then_decode(op, dims, dtype, kernel):
     h.close()
 
 
-@pytest.mark.parametrize("op", OPS)
-@pytest.mark.parametrize("kernel", ["auto", "recurrent", "chunked"])
+@pytest.mark.parametrize("op,kernel", [(op, k) for op in OPS for k in ("auto", "recurrent", "chunked")
+                                       if k != "chunked" or op == "gdn"])
 def test_prefill_continues_logical_state(op, kernel):
     """Without DL_PREFILL_ZERO_STATE a prompt continues from the slot's
     logical state (base + log), e.g. the second chunk of a long prompt."""
     from recurrent_state_update_deltalog_b200 import DeltaLog
     dtype, dk, dv, B, H, M = torch.bfloat16, 128, 128, 4, 2, 8
-    if kernel == "chunked" and op != "gdn":
-        pytest.skip("the chunked prefill serves bf16-input GDN handles (refusal tested below)")
     S0, warm, u = make_inputs(op, B, H, dk, dv, 5, dtype, seed=31)
     h = DeltaLog(B, H, dk, dv, M, op=op, dtype=dtype)
     h.set_prefill_kernel(kernel)
