@@ -33,7 +33,7 @@ namespace dl {
 
 template <int DK>
 struct ChunkGeom {
-  static constexpr int C = 64;           // tokens per chunk
+  static constexpr int C = 32;           // tokens per chunk
   static constexpr int VT = 64;          // value columns per CTA
   static constexpr int NT = 256;         // threads (8 warps)
   static constexpr int LDK = DK + 8;     // bf16 row stride of K and Q (16-byte multiple)
@@ -43,13 +43,13 @@ struct ChunkGeom {
   static constexpr int LDW = DK + 4;     // fp32 row stride of W, e^Gamma Q and e^{..} K
   // shared-memory carve-up (bytes; every region 128-byte aligned)
   static constexpr size_t al(size_t x) { return (x + 127) & ~size_t(127); }
-  // K, Q and the V tile are double-buffered: chunk c + 1 streams in while
-  // chunk c computes
+  // K and the V tile are double-buffered (chunk c + 1 streams in while chunk
+  // c computes); Q streams in during the chunk's first steps
   static constexpr size_t KQ_BYTES = al(size_t(C) * LDK * 2), V_BYTES = al(size_t(C) * LDV * 2);
   static constexpr size_t S_OFF = 0;
   static constexpr size_t K_OFF = al(S_OFF + size_t(DK) * LDS * 4);
   static constexpr size_t Q_OFF = K_OFF + 2 * KQ_BYTES;
-  static constexpr size_t V_OFF = Q_OFF + 2 * KQ_BYTES;
+  static constexpr size_t V_OFF = Q_OFF + KQ_BYTES;
   static constexpr size_t A_OFF = V_OFF + 2 * V_BYTES;
   static constexpr size_t W_OFF = al(A_OFF + size_t(C) * LDA * 4);
   static constexpr size_t U_OFF = al(W_OFF + size_t(C) * LDW * 4);
@@ -78,9 +78,9 @@ using BfBc = wm::fragment<wm::matrix_b, 16, 16, 16, __nv_bfloat16, wm::col_major
 
 // X Y^T of two bf16 row-major [C][LDK] blocks (rows 16i.. of X, 16j.. of Y)
 // into an fp32 [C][LDA] block; tiles above the diagonal are zero.
-template <int DK, int LDK, int LDA>
+template <int C, int DK, int LDK, int LDA>
 __device__ __forceinline__ void lower_xyt(const __nv_bfloat16* X, const __nv_bfloat16* Y, float* out) {
-  for_tiles<64, 64>([&](int i, int j) {
+  for_tiles<C, C>([&](int i, int j) {
     AccBf acc;
     wm::fill_fragment(acc, 0.f);
     if (j <= i) {
@@ -121,7 +121,7 @@ __device__ __forceinline__ void to_tf32(Frag& f) {
 }
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(256, 1) gdn_chunk_prefill_kernel(const PrefillArgs a) {
+__global__ void __launch_bounds__(256, 2) gdn_chunk_prefill_kernel(const PrefillArgs a) {
   using G = ChunkGeom<DK>;
   constexpr int C = G::C, VT = G::VT, NSPLIT = DV / VT;
   static_assert(DV % VT == 0 && DK % 16 == 0, "chunk tile shape");
@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(256, 1) gdn_chunk_prefill_kernel(const Prefill
   float* sS = reinterpret_cast<float*>(smem + G::S_OFF);                  // [DK][LDS] state slice
   // [2][C][LDK] K and Q, [2][C][LDV] V tile: buffer (chunk index & 1)
   auto kbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem + G::K_OFF + b * G::KQ_BYTES); };
-  auto qbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem + G::Q_OFF + b * G::KQ_BYTES); };
+  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem + G::Q_OFF);
   auto vbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem + G::V_OFF + b * G::V_BYTES); };
   float* sA = reinterpret_cast<float*>(smem + G::A_OFF);                  // [C][LDA] A, then P
   float* sW = reinterpret_cast<float*>(smem + G::W_OFF);                  // [C][LDW] W, then e^G Q, then e^{..} K
@@ -173,96 +173,97 @@ __global__ void __launch_bounds__(256, 1) gdn_chunk_prefill_kernel(const Prefill
   __nv_bfloat16* Og = static_cast<__nv_bfloat16*>(a.o);
   const __nv_bfloat16 zero_bf = __float2bfloat16_rn(0.f);
 
-  // Stage chunk [c, c + C) of K, Q and the V tile into buffer b; rows past the
-  // prompt are zeros.  16-byte async copies when the inputs allow them.
+  // Stage chunk [c, c + C) of K and the V tile into buffer b, or of Q; rows
+  // past the prompt are zeros.  16-byte async copies when the inputs allow.
   const bool async_ok = aligned_to(a.q, 16) && aligned_to(a.k, 16) && aligned_to(a.v, 16);
-  auto stage = [&](int b, long c) {
+  auto stage_rows = [&](__nv_bfloat16* dst, const __nv_bfloat16* src, long c, int width, int ld, int stride,
+                        int off) {
     const int nv = static_cast<int>(t1 - c < C ? t1 - c : C);
-    __nv_bfloat16 *dK = kbuf(b), *dQ = qbuf(b), *dV = vbuf(b);
     if (async_ok) {
-      constexpr int SEGK = DK / 8, SEGV = VT / 8;   // 16-byte segments per row
-      for (int idx = tid; idx < C * SEGK; idx += G::NT) {
-        const int t = idx / SEGK, seg = idx % SEGK;
-        const long row = ((c + (t < nv ? t : nv - 1)) * a.H + h) * DK + 8 * seg;
-        const uint32_t bytes = t < nv ? 16u : 0u;
-        cp_async16(dK + t * G::LDK + 8 * seg, Kg + row, bytes);
-        cp_async16(dQ + t * G::LDK + 8 * seg, Qg + row, bytes);
-      }
-      for (int idx = tid; idx < C * SEGV; idx += G::NT) {
-        const int t = idx / SEGV, seg = idx % SEGV;
-        const long row = ((c + (t < nv ? t : nv - 1)) * a.H + h) * DV + col0 + 8 * seg;
-        cp_async16(dV + t * G::LDV + 8 * seg, Vg + row, t < nv ? 16u : 0u);
+      const int seg_per_row = width / 8;   // 16-byte segments
+      for (int idx = tid; idx < C * seg_per_row; idx += G::NT) {
+        const int t = idx / seg_per_row, seg = idx % seg_per_row;
+        const long row = ((c + (t < nv ? t : nv - 1)) * a.H + h) * stride + off + 8 * seg;
+        cp_async16(dst + t * ld + 8 * seg, src + row, t < nv ? 16u : 0u);
       }
     } else {
-      for (int idx = tid; idx < C * DK; idx += G::NT) {
-        const int t = idx / DK, j = idx % DK;
-        const long bu = (c + t) * a.H + h;
-        dK[t * G::LDK + j] = t < nv ? Kg[bu * DK + j] : zero_bf;
-        dQ[t * G::LDK + j] = t < nv ? Qg[bu * DK + j] : zero_bf;
-      }
-      for (int idx = tid; idx < C * VT; idx += G::NT) {
-        const int t = idx / VT, cc = idx % VT;
-        dV[t * G::LDV + cc] = t < nv ? Vg[((c + t) * a.H + h) * DV + col0 + cc] : zero_bf;
+      for (int idx = tid; idx < C * width; idx += G::NT) {
+        const int t = idx / width, j = idx % width;
+        dst[t * ld + j] = t < nv ? src[((c + t) * a.H + h) * stride + off + j] : zero_bf;
       }
     }
   };
-  // warp 0 keeps the next chunk's log-gates and betas in registers
-  float gn0 = 0.f, gn1 = 0.f, bn0 = 0.f, bn1 = 0.f;
+  auto stage_kv = [&](int b, long c) {
+    stage_rows(kbuf(b), Kg, c, DK, G::LDK, DK, 0);
+    stage_rows(vbuf(b), Vg, c, VT, G::LDV, DV, col0);
+  };
+  constexpr int EPL = C / 32;   // chunk rows per lane of warp 0
+  float gn[EPL], bnv[EPL];
   auto fetch_gates = [&](long c) {
     const int nv = static_cast<int>(t1 - c < C ? t1 - c : C);
-    const int ta = 2 * lane, tb = 2 * lane + 1;
-    gn0 = ta < nv ? a.log_decay[(c + ta) * a.H + h] : 0.f;
-    gn1 = tb < nv ? a.log_decay[(c + tb) * a.H + h] : 0.f;
-    bn0 = ta < nv ? a.beta[(c + ta) * a.H + h] : 0.f;
-    bn1 = tb < nv ? a.beta[(c + tb) * a.H + h] : 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      const int t = EPL * lane + e;
+      gn[e] = t < nv ? a.log_decay[(c + t) * a.H + h] : 0.f;
+      bnv[e] = t < nv ? a.beta[(c + t) * a.H + h] : 0.f;
+    }
   };
   if (t0 < t1) {
-    stage(0, t0);
+    stage_kv(0, t0);
     if (warp == 0) fetch_gates(t0);
   }
   cp_async_commit();
 
+  // Copy groups, in commit order: K/V of chunk c (committed one chunk ahead),
+  // then at chunk c: Q of chunk c, K/V of chunk c + 1 (possibly empty).
   int buf = 0;
   for (long c0 = t0; c0 < t1; c0 += C, buf ^= 1) {
     const int n = static_cast<int>(t1 - c0 < C ? t1 - c0 : C);   // valid rows of this chunk
     const bool has_next = c0 + C < t1;
     __syncthreads();   // the previous chunk is done with every buffer
-    if (has_next) stage(buf ^ 1, c0 + C);
+    stage_rows(sQ, Qg, c0, DK, G::LDK, DK, 0);
     cp_async_commit();
-    cp_async_wait<1>();   // this chunk's copies have landed (the next one's may be in flight)
-    __nv_bfloat16 *sK = kbuf(buf), *sQ = qbuf(buf), *sV = vbuf(buf);
+    if (has_next) stage_kv(buf ^ 1, c0 + C);
+    cp_async_commit();
+    cp_async_wait<2>();   // K/V of this chunk have landed (Q and the next K/V may be in flight)
+    __nv_bfloat16 *sK = kbuf(buf), *sV = vbuf(buf);
 
     // 1. Gamma = inclusive prefix sum of the chunk's log-gates (rows past the
     // prompt: 0), and beta; then the next chunk's gates
     if (warp == 0) {
-      const int ta = 2 * lane, tb = 2 * lane + 1;
-      const float g0 = gn0, g1 = gn1;
-      float pair = g0 + g1, incl = pair;
+      float loc[EPL], run = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) loc[e] = (run += gn[e]);
+      float incl = run;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const float y = __shfl_up_sync(0xffffffffu, incl, off);
         if (lane >= off) incl += y;
       }
-      const float excl = incl - pair;
-      const float Ga = excl + g0, Gb = excl + pair;
-      sG[ta] = Ga;
-      sG[tb] = Gb;
-      sBeta[ta] = bn0;
-      sBeta[tb] = bn1;
-      const float ea = expf(Ga), eb = expf(Gb);
-      sEG[ta] = ea;
-      sEG[tb] = eb;
-      sBEG[ta] = bn0 * ea;
-      sBEG[tb] = bn1 * eb;
-      const float gend = __shfl_sync(0xffffffffu, (n - 1) & 1 ? Gb : Ga, (n - 1) >> 1);
-      sEnd[ta] = ta < n ? expf(gend - Ga) : 0.f;
-      sEnd[tb] = tb < n ? expf(gend - Gb) : 0.f;
+      const float excl = incl - run;
+      float sel = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        loc[e] += excl;
+        if (e == (n - 1) % EPL) sel = loc[e];
+      }
+      const float gend = __shfl_sync(0xffffffffu, sel, (n - 1) / EPL);
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        const int t = EPL * lane + e;
+        const float eg = expf(loc[e]);
+        sG[t] = loc[e];
+        sBeta[t] = bnv[e];
+        sEG[t] = eg;
+        sBEG[t] = bnv[e] * eg;
+        sEnd[t] = t < n ? expf(gend - loc[e]) : 0.f;
+      }
       if (has_next) fetch_gates(c0 + C);
     }
     __syncthreads();
 
     // 2. A = strictly lower (beta_t e^{G_t - G_s} k_t . k_s)
-    lower_xyt<DK, G::LDK, G::LDA>(sK, sK, sA);
+    lower_xyt<C, DK, G::LDK, G::LDA>(sK, sK, sA);
     __syncthreads();
     for (int idx = tid; idx < C * C; idx += G::NT) {
       const int t = idx / C, s = idx % C;
@@ -330,7 +331,9 @@ __global__ void __launch_bounds__(256, 1) gdn_chunk_prefill_kernel(const Prefill
     __syncthreads();
 
     // 5. P = Q K^T (.) [e^{G_t - G_s}]_{s <= t} into A;  e^{G} Q into W
-    lower_xyt<DK, G::LDK, G::LDA>(sQ, sK, sA);
+    cp_async_wait<1>();   // Q of this chunk has landed
+    __syncthreads();
+    lower_xyt<C, DK, G::LDK, G::LDA>(sQ, sK, sA);
     for (int idx = tid; idx < C * DK; idx += G::NT) {
       const int t = idx / DK, j = idx % DK;
       sW[t * G::LDW + j] = wm::__float_to_tf32(sEG[t] * __bfloat162float(sQ[t * G::LDK + j]));
