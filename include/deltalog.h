@@ -243,12 +243,12 @@ int dl_read_state(dl_t h, float* S_out, void* stream);
  * streaming kernel does not take it (DL_ERR_UNSUPPORTED). */
 /* DL_OPT_PREFILL_KERNEL picks the kernel behind dl_prefill:
  *   DL_PREFILL_AUTO (default): the chunked kernel for bf16-input GDN handles
- *     when the batch is too small to fill the GPU with the recurrent kernel
- *     (rows x H x d_v/16 < 8 x SMs), the recurrent kernel otherwise;
+ *     whose prompts average at least 64 tokens (total >= 64 rows), the
+ *     recurrent kernel otherwise;
  *   DL_PREFILL_RECURRENT: the recurrence token by token, state in registers
  *     (every operator and dtype; outputs equal the eager recurrence's up to
  *     fp32 rounding);
- *   DL_PREFILL_CHUNKED: 64-token chunks in the WY form of the delta rule on
+ *   DL_PREFILL_CHUNKED: 32-token chunks in the WY form of the delta rule on
  *     tensor cores (bf16 products of the inputs, tf32 products with the
  *     state; bf16-input GDN handles only, DL_ERR_UNSUPPORTED otherwise).
  *     Its tf32 products round to 2^-11 relative, inside the bf16-input

@@ -298,21 +298,20 @@ cudaError_t materialize_slots(const dl_handle* h, const int* slot_idx, int rows,
 }
 
 // The chunked tensor-core prefill serves bf16-input GDN handles.  AUTO picks
-// it there when the recurrent kernel's warps (rows x H x d_v/16) would not
-// fill the GPU: B200 measured GDN d=128, 4 prompts of 4096 tokens 4.25 vs
-// 3.76 M tokens/s for the chunked kernel, 64 prompts of 512 tokens 4.84 vs
-// 7.30 for the recurrent one.
-bool chunked_prefill(const dl_handle* h, int rows) {
+// it there unless the prompts are short (fewer than 64 tokens on average):
+// on B200 it measured 1.00-2.40x the recurrent kernel from 64-token prompts
+// up (B=256 L=64 1.00, B=64 L=512 1.05, B=4 L=4096 1.76, B=1 L=8192 2.40,
+// d=64 1.22) and 0.97x on 32-token prompts.
+bool chunked_prefill(const dl_handle* h, int rows, long long total) {
   const bool ok = h->op == DL_GDN && h->dtype == DL_BF16;
-  const long recurrent_warps = static_cast<long>(rows) * h->H * (h->dv / 16);
   return h->prefill_kernel == DL_PREFILL_CHUNKED ||
-         (h->prefill_kernel == DL_PREFILL_AUTO && ok && recurrent_warps < 8L * h->sms);
+         (h->prefill_kernel == DL_PREFILL_AUTO && ok && total >= 64LL * rows);
 }
 
 cudaError_t launch_prefill(dl_handle* h, const dl::PrefillArgs& a, int rows, cudaStream_t s) {
   dl::LaunchShape sh = shape_of(h);
   sh.units = rows;
-  if (chunked_prefill(h, rows)) {
+  if (chunked_prefill(h, rows, a.total)) {
     if (h->op != DL_GDN || h->dtype != DL_BF16) return cudaErrorNotSupported;
     h->last_prefill = DL_PREFILL_CHUNKED;
     return dl::launch_gdn_chunk_prefill_dims(sh, a, s);

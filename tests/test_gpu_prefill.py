@@ -87,7 +87,9 @@ def test_prefill_then_decode(op, dims, dtype, kernel):
                   slot_idx=torch.tensor(slots, dtype=torch.int32, device="cuda"), zero_state=True)
     assert h.log_len == 2                                # the handle's cycle is unchanged
     applies = op == "gdn" and dtype == torch.bfloat16
-    assert h.last_prefill_kernel == ("chunked" if kernel != "recurrent" and applies else "recurrent")
+    auto_chunked = applies and sum(lens) >= 64 * rows                 # the automatic rule
+    want = "chunked" if kernel == "chunked" or (kernel == "auto" and auto_chunked) else "recurrent"
+    assert h.last_prefill_kernel == want
     got = o.float().cpu().numpy()
     zero = np.zeros((H, dk, dv))
     for r, (n, b) in enumerate(zip(lens, slots)):
