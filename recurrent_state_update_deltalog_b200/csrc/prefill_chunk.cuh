@@ -38,9 +38,11 @@ struct ChunkGeom {
   static constexpr int NT = 256;         // threads (8 warps)
   static constexpr int LDK = DK + 8;     // bf16 row stride of K and Q (16-byte multiple)
   static constexpr int LDV = VT + 8;     // bf16 row stride of the V tile
-  static constexpr int LDS = VT + 4;     // fp32 row stride of the state tile, B and U
+  static constexpr int LDS = VT + 8;     // fp32 row stride of the state tile, B and U (8 banks:
+                                         // conflict-free tf32 B-operand reads)
   static constexpr int LDA = C + 4;      // fp32 row stride of A and P
-  static constexpr int LDW = DK + 4;     // fp32 row stride of W, e^Gamma Q and e^{..} K
+  static constexpr int LDW = DK + 4;     // fp32 row stride of W and e^Gamma Q
+  static constexpr int LDT = C + 4;      // fp32 row stride of (e^{..} K)^T, stored transposed
   // shared-memory carve-up (bytes; every region 128-byte aligned)
   static constexpr size_t al(size_t x) { return (x + 127) & ~size_t(127); }
   // K and the V tile are double-buffered (chunk c + 1 streams in while chunk
@@ -52,7 +54,8 @@ struct ChunkGeom {
   static constexpr size_t V_OFF = Q_OFF + KQ_BYTES;
   static constexpr size_t A_OFF = V_OFF + 2 * V_BYTES;
   static constexpr size_t W_OFF = al(A_OFF + size_t(C) * LDA * 4);
-  static constexpr size_t U_OFF = al(W_OFF + size_t(C) * LDW * 4);
+  static constexpr size_t W_FLOATS = size_t(C) * LDW > size_t(DK) * LDT ? size_t(C) * LDW : size_t(DK) * LDT;
+  static constexpr size_t U_OFF = al(W_OFF + W_FLOATS * 4);
   static constexpr size_t G_OFF = al(U_OFF + size_t(C) * LDS * 4);
   static constexpr size_t BYTES = al(G_OFF + 5 * C * 4);   // Gamma, beta and three per-row factors
 };
@@ -132,7 +135,7 @@ __global__ void __launch_bounds__(256, 2) gdn_chunk_prefill_kernel(const Prefill
   __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem + G::Q_OFF);
   auto vbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem + G::V_OFF + b * G::V_BYTES); };
   float* sA = reinterpret_cast<float*>(smem + G::A_OFF);                  // [C][LDA] A, then P
-  float* sW = reinterpret_cast<float*>(smem + G::W_OFF);                  // [C][LDW] W, then e^G Q, then e^{..} K
+  float* sW = reinterpret_cast<float*>(smem + G::W_OFF);                  // [C][LDW] W, then e^G Q; [DK][LDT] (e^{..} K)^T
   float* sU = reinterpret_cast<float*>(smem + G::U_OFF);                  // [C][LDS] U, then B
   float* sG = reinterpret_cast<float*>(smem + G::G_OFF);                  // [C] Gamma
   float* sBeta = sG + C;                                                  // [C] beta
@@ -378,9 +381,9 @@ __global__ void __launch_bounds__(256, 2) gdn_chunk_prefill_kernel(const Prefill
     __syncthreads();
 
     // 7. S <- e^{G_end} S + (e^{G_end - G} K)^T B
-    for (int idx = tid; idx < C * DK; idx += G::NT) {
-      const int t = idx / DK, j = idx % DK;
-      sW[t * G::LDW + j] = wm::__float_to_tf32(sEnd[t] * __bfloat162float(sK[t * G::LDK + j]));
+    for (int idx = tid; idx < C * DK; idx += G::NT) {   // transposed, rows of keys
+      const int j = idx / C, t = idx % C;
+      sW[j * G::LDT + t] = wm::__float_to_tf32(sEnd[t] * __bfloat162float(sK[t * G::LDK + j]));
     }
     __syncthreads();
     const float dend = sEG[n - 1];
@@ -392,9 +395,9 @@ __global__ void __launch_bounds__(256, 2) gdn_chunk_prefill_kernel(const Prefill
       for (int e = 0; e < acc.num_elements; ++e) acc.x[e] *= dend;
 #pragma unroll 4
       for (int kk = 0; kk < C; kk += 8) {
-        TfAc fa;
+        TfA fa;
         TfB fb;
-        wm::load_matrix_sync(fa, sW + kk * G::LDW + 16 * i, G::LDW);   // (e^{..} K)^T, col-major, tf32
+        wm::load_matrix_sync(fa, sW + (16 * i) * G::LDT + kk, G::LDT);  // (e^{..} K)^T, tf32
         wm::load_matrix_sync(fb, sU + kk * G::LDS + 16 * j, G::LDS);     // B, tf32
         wm::mma_sync(acc, fa, fb, acc);
       }
