@@ -242,17 +242,19 @@ int dl_read_state(dl_t h, float* S_out, void* stream);
  * Changeable only while the log is empty (DL_ERR_STATE otherwise).  The
  * streaming kernel does not take it (DL_ERR_UNSUPPORTED). */
 /* DL_OPT_PREFILL_KERNEL picks the kernel behind dl_prefill:
- *   DL_PREFILL_AUTO (default): the chunked kernel for bf16-input GDN handles
- *     whose prompts average at least 64 tokens (total >= 64 rows), the
- *     recurrent kernel otherwise;
+ *   DL_PREFILL_AUTO (default): the chunked kernel for bf16-input handles
+ *     whose prompts average at least 64 tokens (total >= 64 rows) and, for
+ *     KDA, whose rows x H x d_v/16 is below 12 per SM; the recurrent kernel
+ *     otherwise;
  *   DL_PREFILL_RECURRENT: the recurrence token by token, state in registers
  *     (every operator and dtype; outputs equal the eager recurrence's up to
  *     fp32 rounding);
- *   DL_PREFILL_CHUNKED: 32-token chunks in the WY form of the delta rule on
- *     tensor cores (bf16 products of the inputs, tf32 products with the
- *     state; bf16-input GDN handles only, DL_ERR_UNSUPPORTED otherwise).
- *     Its tf32 products round to 2^-11 relative, inside the bf16-input
- *     tolerance. */
+ *   DL_PREFILL_CHUNKED: the chunk form on tensor cores (bf16-input handles
+ *     only, DL_ERR_UNSUPPORTED otherwise).  GDN: 32-token chunks in the WY
+ *     form of the delta rule, bf16 products of the inputs.  KDA and RWKV6:
+ *     chunks of 16 tokens (d_k = 128) or 32 (d_k = 64) whose per-key pair
+ *     weights are formed exactly on the SIMT lanes.  The products with the
+ *     state are tf32 (2^-11 relative), inside the bf16-input tolerance. */
 enum dl_option {
   DL_OPT_STEP_KERNEL = 0,
   DL_OPT_HOST_PREFETCH = 1,

@@ -297,24 +297,33 @@ cudaError_t materialize_slots(const dl_handle* h, const int* slot_idx, int rows,
   }
 }
 
-// The chunked tensor-core prefill serves bf16-input GDN handles.  AUTO picks
-// it there unless the prompts are short (fewer than 64 tokens on average):
-// on B200 it measured 1.00-2.40x the recurrent kernel from 64-token prompts
-// up (B=256 L=64 1.00, B=64 L=512 1.05, B=4 L=4096 1.76, B=1 L=8192 2.40,
-// d=64 1.22) and 0.97x on 32-token prompts.
+// The chunked tensor-core prefills serve bf16-input handles.  AUTO picks them
+// unless the prompts are short (fewer than 64 tokens on average); for KDA only
+// while the recurrent kernel's one-warp tiles (rows x heads x d_v/16) number
+// fewer than 12 per SM.  Measured on B200 against the recurrent kernel:
+//   GDN:   1.00-2.40x from 64-token prompts up (B=256 L=64 1.00, B=64 L=512
+//          1.05, B=4 L=4096 1.76, B=1 L=8192 2.40, d=64 1.22), 0.97x at L=32;
+//   RWKV6 (H=64, d=64): B=256 L=64 0.98, B=64 L=512 1.05, B=4 L=4096 2.58,
+//          B=1 L=8192 3.56;
+//   KDA:   B=4 L=4096 1.38, B=1 L=8192 1.80, but B=64 L=512 0.85 and B=256
+//          L=64 0.81 once the recurrent kernel fills the GPU.
 bool chunked_prefill(const dl_handle* h, int rows, long long total) {
-  const bool ok = h->op == DL_GDN && h->dtype == DL_BF16;
-  return h->prefill_kernel == DL_PREFILL_CHUNKED ||
-         (h->prefill_kernel == DL_PREFILL_AUTO && ok && total >= 64LL * rows);
+  if (h->prefill_kernel != DL_PREFILL_AUTO) return h->prefill_kernel == DL_PREFILL_CHUNKED;
+  if (h->dtype != DL_BF16 || total < 64LL * rows) return false;
+  return h->op != DL_KDA || static_cast<long long>(rows) * h->H * (h->dv / 16) < 12LL * h->sms;
 }
 
 cudaError_t launch_prefill(dl_handle* h, const dl::PrefillArgs& a, int rows, cudaStream_t s) {
   dl::LaunchShape sh = shape_of(h);
   sh.units = rows;
   if (chunked_prefill(h, rows, a.total)) {
-    if (h->op != DL_GDN || h->dtype != DL_BF16) return cudaErrorNotSupported;
+    if (h->dtype != DL_BF16) return cudaErrorNotSupported;
     h->last_prefill = DL_PREFILL_CHUNKED;
-    return dl::launch_gdn_chunk_prefill_dims(sh, a, s);
+    switch (h->op) {
+      case DL_GDN: return dl::launch_gdn_chunk_prefill_dims(sh, a, s);
+      case DL_KDA: return dl::launch_key_chunk_prefill_dims<dl::OP_KDA>(sh, a, s);
+      default: return dl::launch_key_chunk_prefill_dims<dl::OP_RWKV6>(sh, a, s);
+    }
   }
   h->last_prefill = DL_PREFILL_RECURRENT;
   switch (h->op) {
@@ -601,7 +610,7 @@ int dl_prefill(dl_t h, const int* slot_idx, int rows, const int* cu_seqlens, lon
   a.zero_state = zero ? 1 : 0;
   cudaError_t e = launch_prefill(h, a, rows, s);
   if (e == cudaErrorNotSupported)
-    return fail(DL_ERR_UNSUPPORTED, "the chunked prefill serves bf16-input GDN handles that fit its shared memory");
+    return fail(DL_ERR_UNSUPPORTED, "the chunked prefill serves bf16-input handles that fit its shared memory");
   if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
   h->wrote_state = true;
   return DL_OK;

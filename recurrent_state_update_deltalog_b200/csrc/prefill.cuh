@@ -264,6 +264,14 @@ prefill_kernel(const PrefillArgs a) {
 // fit the device.
 cudaError_t launch_gdn_chunk_prefill_dims(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st);
 
+// Chunked tensor-core KDA / RWKV6 prefill (bf16 inputs; prefill_chunk_key.cuh):
+// grid (H * d_v/64, rows), 256 threads.  cudaErrorNotSupported when its shared
+// memory does not fit the device.
+template <int OP>
+cudaError_t launch_key_chunk_prefill_dims(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st);
+extern template cudaError_t launch_key_chunk_prefill_dims<OP_KDA>(const LaunchShape&, const PrefillArgs&, cudaStream_t);
+extern template cudaError_t launch_key_chunk_prefill_dims<OP_RWKV6>(const LaunchShape&, const PrefillArgs&, cudaStream_t);
+
 // Grid (H * d_v/16, rows), one warp per CTA.  Instantiated in prefill.cu.
 template <int OP>
 cudaError_t launch_prefill_op(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st);

@@ -47,16 +47,16 @@ def _oracle_row(op, S_init, seq, r, n, u):
     return o, S
 
 
-# the chunked kernel serves bf16-input GDN handles only (its refusal elsewhere
-# is tested below)
+# the chunked kernels serve bf16-input handles only (their refusal for fp32
+# inputs is tested below)
 _KERNELS = [(op, dt, k) for op in OPS for dt in (torch.bfloat16, torch.float32)
-            for k in ("auto", "recurrent", "chunked") if k != "chunked" or (op == "gdn" and dt == torch.bfloat16)]
+            for k in ("auto", "recurrent", "chunked") if k != "chunked" or dt == torch.bfloat16]
 
 
 @pytest.mark.parametrize("op,dtype,kernel", _KERNELS)
 @pytest.mark.parametrize("dims", [(64, 64), (128, 128), (64, 128), (128, 64)])
 def test_prefill_then_decode(op, dims, dtype, kernel):
-    """Prompts of 37, 0, 1, 64 + 66 (two chunks and a ragged tail) and 5 tokens."""
+    """Prompts of 37, 0, 1, 130 (several chunks and a ragged tail) and 5 tokens."""
     from recurrent_state_update_deltalog_b200 import DeltaLog
     dk, dv = dims
     B, H, M, T_dec = 8, 3, 4, 7
@@ -86,8 +86,9 @@ def test_prefill_then_decode(op, dims, dtype, kernel):
     o = h.prefill(*_prefill_args(op, d), cu_seqlens=torch.from_numpy(cu).cuda(),
                   slot_idx=torch.tensor(slots, dtype=torch.int32, device="cuda"), zero_state=True)
     assert h.log_len == 2                                # the handle's cycle is unchanged
-    applies = op == "gdn" and dtype == torch.bfloat16
-    auto_chunked = applies and sum(lens) >= 64 * rows                 # the automatic rule
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    auto_chunked = (dtype == torch.bfloat16 and sum(lens) >= 64 * rows       # the automatic rule
+                    and (op != "kda" or rows * H * (dv // 16) < 12 * sms))
     want = "chunked" if kernel == "chunked" or (kernel == "auto" and auto_chunked) else "recurrent"
     assert h.last_prefill_kernel == want
     got = o.float().cpu().numpy()
@@ -112,8 +113,7 @@ def test_prefill_then_decode(op, dims, dtype, kernel):
     h.close()
 
 
-@pytest.mark.parametrize("op,kernel", [(op, k) for op in OPS for k in ("auto", "recurrent", "chunked")
-                                       if k != "chunked" or op == "gdn"])
+@pytest.mark.parametrize("op,kernel", [(op, k) for op in OPS for k in ("auto", "recurrent", "chunked")])
 def test_prefill_continues_logical_state(op, kernel):
     """Without DL_PREFILL_ZERO_STATE a prompt continues from the slot's
     logical state (base + log), e.g. the second chunk of a long prompt."""
@@ -177,8 +177,9 @@ def test_prefill_arguments():
     h.close()
 
 
-@pytest.mark.parametrize("op,H,d,kernel", [("gdn", 32, 128, "chunked"), ("gdn", 32, 128, "recurrent"),
-                                           ("kda", 32, 128, "auto"), ("rwkv6", 64, 64, "auto")])
+@pytest.mark.parametrize("op,H,d,kernel", [(op, H, d, k) for op, H, d in (("gdn", 32, 128), ("kda", 32, 128),
+                                                                         ("rwkv6", 64, 64))
+                                           for k in ("chunked", "recurrent")])
 def test_prefill_full_size_sampled(op, H, d, kernel):
     """The launch bench.py --prefill times (B = 64 prompts of L = 512 tokens,
     every row from zero): two sampled rows checked token by token, with their
@@ -206,9 +207,9 @@ def test_prefill_full_size_sampled(op, H, d, kernel):
 
 
 def test_chunked_prefill_refused_where_it_does_not_apply():
-    """The chunked kernel serves bf16-input GDN handles only."""
+    """The chunked kernels serve bf16-input handles only."""
     from recurrent_state_update_deltalog_b200 import DeltaLog, DeltaLogError
-    for op, dtype in (("kda", torch.bfloat16), ("rwkv6", torch.bfloat16), ("gdn", torch.float32)):
+    for op, dtype in (("gdn", torch.float32), ("kda", torch.float32), ("rwkv6", torch.float32)):
         h = DeltaLog(2, 2, 64, 64, 4, op=op, dtype=dtype)
         h.set_prefill_kernel("chunked")
         x = torch.zeros((3, 2, 64), device="cuda", dtype=dtype)
