@@ -17,11 +17,17 @@ cudaError_t launch_prefill_op(const LaunchShape& s, const PrefillArgs& a, cudaSt
   DL_DISPATCH_DIMS(prefill_dims, s, a, st);
 }
 
-template <int DK, int DV>
+// Whole-head CTAs (VT = 128) for d_k = d_v = 128 once they cover at least
+// half the SMs (rows x heads), 64-column tiles below that.  Measured on B200
+// for the KDA kernel (H=32): whole-head CTAs 1.18x at B=64 L=512, 1.21x at
+// B=4 L=4096, but 0.83x at B=1 L=8192 (32 CTAs).
+inline bool whole_head_tiles(const LaunchShape& s) { return 2LL * s.units * s.H > s.sms; }
+
+template <int DK, int DV, int VT>
 cudaError_t launch_gdn_chunk_prefill(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st) {
-  using G = ChunkGeom<DK>;
-  auto kern = gdn_chunk_prefill_kernel<DK, DV>;
-  if (G::BYTES + 8 * 1024 > static_cast<size_t>(s.smem_block_optin)) return cudaErrorNotSupported;
+  using G = ChunkGeom<DK, VT>;
+  auto kern = gdn_chunk_prefill_kernel<DK, DV, VT>;
+  if (G::BYTES + G::NW * 1024 > static_cast<size_t>(s.smem_block_optin)) return cudaErrorNotSupported;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(G::BYTES));
   if (e != cudaSuccess) return e;
   kern<<<dim3(s.H * (DV / G::VT), s.units), G::NT, G::BYTES, st>>>(a);
@@ -29,30 +35,34 @@ cudaError_t launch_gdn_chunk_prefill(const LaunchShape& s, const PrefillArgs& a,
 }
 
 cudaError_t launch_gdn_chunk_prefill_dims(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st) {
-  if (s.dk == 64 && s.dv == 64) return launch_gdn_chunk_prefill<64, 64>(s, a, st);
-  if (s.dk == 128 && s.dv == 128) return launch_gdn_chunk_prefill<128, 128>(s, a, st);
-  if (s.dk == 64 && s.dv == 128) return launch_gdn_chunk_prefill<64, 128>(s, a, st);
-  if (s.dk == 128 && s.dv == 64) return launch_gdn_chunk_prefill<128, 64>(s, a, st);
+  if (s.dk == 64 && s.dv == 64) return launch_gdn_chunk_prefill<64, 64, 64>(s, a, st);
+  if (s.dk == 128 && s.dv == 128)
+    return whole_head_tiles(s) ? launch_gdn_chunk_prefill<128, 128, 128>(s, a, st)
+                               : launch_gdn_chunk_prefill<128, 128, 64>(s, a, st);
+  if (s.dk == 64 && s.dv == 128) return launch_gdn_chunk_prefill<64, 128, 64>(s, a, st);
+  if (s.dk == 128 && s.dv == 64) return launch_gdn_chunk_prefill<128, 64, 64>(s, a, st);
   return cudaErrorInvalidValue;
 }
 
-template <int OP, int DK, int DV>
+template <int OP, int DK, int DV, int VT>
 cudaError_t launch_key_chunk_prefill(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st) {
-  using G = KeyChunkGeom<DK>;
-  auto kern = key_chunk_prefill_kernel<OP, DK, DV>;
-  if (G::BYTES + 8 * 1024 > static_cast<size_t>(s.smem_block_optin)) return cudaErrorNotSupported;
+  using G = KeyChunkGeom<DK, VT>;
+  auto kern = key_chunk_prefill_kernel<OP, DK, DV, VT>;
+  if (G::BYTES + G::NW * 1024 > static_cast<size_t>(s.smem_block_optin)) return cudaErrorNotSupported;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(G::BYTES));
   if (e != cudaSuccess) return e;
-  kern<<<dim3(s.H * (DV / G::VT), s.units), G::NT, G::BYTES, st>>>(a);
+  kern<<<dim3(s.H * (DV / VT), s.units), G::NT, G::BYTES, st>>>(a);
   return cudaGetLastError();
 }
 
 template <int OP>
 cudaError_t launch_key_chunk_prefill_dims(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st) {
-  if (s.dk == 64 && s.dv == 64) return launch_key_chunk_prefill<OP, 64, 64>(s, a, st);
-  if (s.dk == 128 && s.dv == 128) return launch_key_chunk_prefill<OP, 128, 128>(s, a, st);
-  if (s.dk == 64 && s.dv == 128) return launch_key_chunk_prefill<OP, 64, 128>(s, a, st);
-  if (s.dk == 128 && s.dv == 64) return launch_key_chunk_prefill<OP, 128, 64>(s, a, st);
+  if (s.dk == 64 && s.dv == 64) return launch_key_chunk_prefill<OP, 64, 64, 64>(s, a, st);
+  if (s.dk == 128 && s.dv == 128)
+    return whole_head_tiles(s) ? launch_key_chunk_prefill<OP, 128, 128, 128>(s, a, st)
+                               : launch_key_chunk_prefill<OP, 128, 128, 64>(s, a, st);
+  if (s.dk == 64 && s.dv == 128) return launch_key_chunk_prefill<OP, 64, 128, 64>(s, a, st);
+  if (s.dk == 128 && s.dv == 64) return launch_key_chunk_prefill<OP, 128, 64, 64>(s, a, st);
   return cudaErrorInvalidValue;
 }
 

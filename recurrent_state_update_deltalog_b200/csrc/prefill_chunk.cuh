@@ -31,11 +31,13 @@
 
 namespace dl {
 
-template <int DK>
+template <int DK, int VT_>
 struct ChunkGeom {
   static constexpr int C = 32;           // tokens per chunk
-  static constexpr int VT = 64;          // value columns per CTA
-  static constexpr int NT = 256;         // threads (8 warps)
+  static constexpr int VT = VT_;         // value columns per CTA (64 or 128)
+  static constexpr int NT = 4 * VT;      // threads (8 or 16 warps)
+  static constexpr int NW = NT / 32;
+  static constexpr int MINB = VT == 128 ? 1 : 2;   // resident CTAs per SM
   static constexpr int LDK = DK + 8;     // bf16 row stride of K and Q (16-byte multiple)
   static constexpr int LDV = VT + 8;     // bf16 row stride of the V tile
   static constexpr int LDS = VT + 8;     // fp32 row stride of the state tile, B and U (8 banks:
@@ -123,9 +125,10 @@ __device__ __forceinline__ void to_tf32(Frag& f) {
   for (int e = 0; e < f.num_elements; ++e) f.x[e] = wm::__float_to_tf32(f.x[e]);
 }
 
-template <int DK, int DV>
-__global__ void __launch_bounds__(256, 2) gdn_chunk_prefill_kernel(const PrefillArgs a) {
-  using G = ChunkGeom<DK>;
+template <int DK, int DV, int VT_>
+__global__ void __launch_bounds__(ChunkGeom<DK, VT_>::NT, ChunkGeom<DK, VT_>::MINB)
+    gdn_chunk_prefill_kernel(const PrefillArgs a) {
+  using G = ChunkGeom<DK, VT_>;
   constexpr int C = G::C, VT = G::VT, NSPLIT = DV / VT;
   static_assert(DV % VT == 0 && DK % 16 == 0, "chunk tile shape");
   extern __shared__ __align__(128) unsigned char smem[];
@@ -142,7 +145,7 @@ __global__ void __launch_bounds__(256, 2) gdn_chunk_prefill_kernel(const Prefill
   float* sEG = sG + 2 * C;    // [C] e^{Gamma_t}
   float* sBEG = sG + 3 * C;   // [C] beta_t e^{Gamma_t}
   float* sEnd = sG + 4 * C;   // [C] e^{Gamma_end - Gamma_t} (0 past the prompt)
-  __shared__ __align__(32) float s_patch[8][16 * 16];                     // per-warp output tile
+  __shared__ __align__(32) float s_patch[G::NW][16 * 16];                 // per-warp output tile
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = static_cast<int>(blockIdx.x) / NSPLIT;
@@ -414,9 +417,9 @@ __global__ void __launch_bounds__(256, 2) gdn_chunk_prefill_kernel(const Prefill
   clear_log_tile<OP_GDN, DK, DV, __nv_bfloat16>(a, sh, col0, VT);
 }
 
-// Grid (H * d_v/64, rows), 256 threads, ChunkGeom<DK>::BYTES of dynamic shared
-// memory.  Instantiated in prefill.cu.
-template <int DK, int DV>
+// Grid (H * d_v/VT, rows), 4 VT threads, ChunkGeom<DK, VT>::BYTES of dynamic
+// shared memory.  Instantiated in prefill.cu.
+template <int DK, int DV, int VT>
 cudaError_t launch_gdn_chunk_prefill(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st);
 
 }  // namespace dl

@@ -28,12 +28,15 @@
 // exp2 per (pair, key), shared by A and P for KDA; only the products with the
 // state, W and B run on the tensor cores (tf32 operands, fp32 accumulation).
 //
-// One CTA per (row, head, 64-column value tile) keeps its d_k x 64 state slice
-// in shared memory for the whole prompt.  Chunks are 16 tokens at d_k = 128
-// and 32 at d_k = 64, so that K, Q, V and the gates of the next chunk stream
-// in (cp.async, double-buffered) while two CTAs share each SM.  Where a C x 64
-// product has fewer 16 x 16 output tiles than the CTA has warps, its
-// contraction is split between two warps per tile.
+// One CTA per (row, head, value tile) keeps its d_k x VT state slice in shared
+// memory for the whole prompt, with K, Q, V and the gates of the next chunk
+// streaming in (cp.async, double-buffered).  Two geometries:
+//   VT = 128: a whole 128 x 128 head per 512-thread CTA, 32-token chunks, one
+//     CTA per SM (the key-side work is done once per head);
+//   VT = 64: 256-thread CTAs, two per SM; 32-token chunks at d_k = 64, 16 at
+//     d_k = 128 (to fit two CTAs).  Where a C x 64 product has fewer 16 x 16
+//     output tiles than the CTA has warps, its contraction is split between
+//     two warps per tile.
 #pragma once
 
 #include <type_traits>
@@ -42,11 +45,14 @@
 
 namespace dl {
 
-template <int DK>
+template <int DK, int VT_>
 struct KeyChunkGeom {
-  static constexpr int C = DK == 128 ? 16 : 32;   // tokens per chunk
-  static constexpr int VT = 64;                   // value columns per CTA
-  static constexpr int NT = 256, NW = NT / 32;    // threads, warps
+  // value columns per CTA: 128 (a whole d_v = 128 head, 512 threads, one CTA
+  // per SM) or 64 (256 threads, two CTAs per SM)
+  static constexpr int VT = VT_;
+  static constexpr int C = DK == 128 && VT == 64 ? 16 : 32;   // tokens per chunk
+  static constexpr int NT = VT == 128 ? 512 : 256, NW = NT / 32;   // threads, warps
+  static constexpr int MINB = NT == 512 ? 1 : 2;                    // resident CTAs per SM
   static constexpr int LDK = DK + 8;    // bf16 row stride of K and Q (16-byte multiple)
   static constexpr int LDV = VT + 8;    // bf16 row stride of the V tile
   static constexpr int LDS = VT + 8;    // fp32 row stride of the state tile, U and B
@@ -94,6 +100,15 @@ __device__ __forceinline__ void bf16x8_to_f32(const __nv_bfloat16* p, float (&f)
   }
 }
 
+// Four bf16 of an 8-byte-aligned shared row as floats.
+__device__ __forceinline__ void bf16x4_to_f32(const __nv_bfloat16* p, float (&f)[4]) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  f[0] = __uint_as_float(u.x << 16);
+  f[1] = __uint_as_float(u.x & 0xffff0000u);
+  f[2] = __uint_as_float(u.y << 16);
+  f[3] = __uint_as_float(u.y & 0xffff0000u);
+}
+
 // (t, s) of strict lower-triangle pair p = t (t - 1) / 2 + s, 0 <= s < t.
 __device__ __forceinline__ void strict_pair(int p, int& t, int& s) {
   t = static_cast<int>((1.f + sqrtf(8.f * static_cast<float>(p) + 1.f)) * 0.5f);
@@ -102,9 +117,10 @@ __device__ __forceinline__ void strict_pair(int p, int& t, int& s) {
   s = p - t * (t - 1) / 2;
 }
 
-template <int OP, int DK, int DV>
-__global__ void __launch_bounds__(256, 2) key_chunk_prefill_kernel(const PrefillArgs a) {
-  using G = KeyChunkGeom<DK>;
+template <int OP, int DK, int DV, int VT_>
+__global__ void __launch_bounds__(KeyChunkGeom<DK, VT_>::NT, KeyChunkGeom<DK, VT_>::MINB)
+    key_chunk_prefill_kernel(const PrefillArgs a) {
+  using G = KeyChunkGeom<DK, VT_>;
   constexpr int C = G::C, VT = G::VT, NSPLIT = DV / VT;
   constexpr bool DELTA = OP == OP_KDA;
   constexpr float LOG2E = 1.4426950408889634f;
@@ -224,25 +240,34 @@ __global__ void __launch_bounds__(256, 2) key_chunk_prefill_kernel(const Prefill
     }
     __syncthreads();
 
-    // 2. A and P pair by pair; the upper triangles zero; right-hand sides
+    // 2. A and P pair by pair; the upper triangles zero; right-hand sides.
+    // When twice the strict pairs plus the diagonal make exactly one item per
+    // thread (C = 16), each strict pair is split between two adjacent lanes,
+    // one half of the keys each.
     constexpr int NSTRICT = C * (C - 1) / 2;
-    for (int p = tid; p < NSTRICT + C; p += G::NT) {
+    constexpr bool SPLIT = 2 * NSTRICT + C == G::NT;
+    constexpr int NITEMS = SPLIT ? G::NT : NSTRICT + C;
+    for (int p = tid; p < NITEMS; p += G::NT) {
+      const int nstr = SPLIT ? 2 * NSTRICT : NSTRICT;   // strict items come first
+      const bool strict = p < nstr;
       int t, s;
-      if (p < NSTRICT) {
-        strict_pair(p, t, s);
+      if (strict) {
+        strict_pair(SPLIT ? p >> 1 : p, t, s);
       } else {
-        t = s = p - NSTRICT;
+        t = s = p - nstr;
       }
+      const int j0 = SPLIT && strict ? (p & 1) * (DK / 2) : 0;
+      const int j1 = SPLIT && strict ? j0 + DK / 2 : DK;
       const __nv_bfloat16* kt = sK + t * G::LDK;
       const __nv_bfloat16* ks = sK + s * G::LDK;
       const __nv_bfloat16* qt = sQ + t * G::LDK;
       float accA = 0.f, accP = 0.f;
-      if (s < t) {
+      if (strict) {
         // exponent rows: Gamma_t (KDA) or Gamma_{t-1} (RWKV6), against Gamma_s
         const float* gt = sG + (OP == OP_RWKV6 ? t - 1 : t) * G::LDG;
         const float* gs = sG + s * G::LDG;
 #pragma unroll 2
-        for (int j = 0; j < DK; j += 8) {
+        for (int j = j0; j < j1; j += 8) {
           float fks[8], fqt[8], fkt[8];
           bf16x8_to_f32(ks + j, fks);
           bf16x8_to_f32(qt + j, fqt);
@@ -260,7 +285,6 @@ __global__ void __launch_bounds__(256, 2) key_chunk_prefill_kernel(const Prefill
             accP = fmaf(fqt[e], m, accP);
           }
         }
-        if (DELTA) sA[t * G::LDA + s] = sBeta[t] * accA;
       } else {
         // diagonal: q_t . k_t (KDA), (u (.) k_t) . r_t (RWKV6)
 #pragma unroll 2
@@ -272,27 +296,49 @@ __global__ void __launch_bounds__(256, 2) key_chunk_prefill_kernel(const Prefill
           for (int e = 0; e < 8; ++e) accP = fmaf(fqt[e], OP == OP_RWKV6 ? sBonus[j + e] * fkt[e] : fkt[e], accP);
         }
       }
-      sP[t * G::LDA + s] = wm::__float_to_tf32(accP);
+      if (SPLIT) {   // one item per thread: every lane of the warp reaches the shuffles
+        const float oA = __shfl_xor_sync(0xffffffffu, accA, 1), oP = __shfl_xor_sync(0xffffffffu, accP, 1);
+        if (strict) {
+          accA += oA;
+          accP += oP;
+        }
+      }
+      if (!SPLIT || !strict || (p & 1) == 0) {
+        if (DELTA && strict) sA[t * G::LDA + s] = sBeta[t] * accA;
+        sP[t * G::LDA + s] = wm::__float_to_tf32(accP);
+      }
     }
     for (int idx = tid; idx < C * C; idx += G::NT) {
       const int t = idx / C, s = idx % C;
       if (s > t) sP[t * G::LDA + s] = 0.f;
       if (DELTA && s >= t) sA[t * G::LDA + s] = 0.f;
     }
+    // four consecutive columns per thread in the element-wise passes below
     if (DELTA) {
       // beta (e^{Gamma} (.) K) into W, beta V into U
-      for (int idx = tid; idx < C * DK; idx += G::NT) {
-        const int t = idx / DK, j = idx % DK;
-        sW[t * G::LDW + j] = sBeta[t] * ex2_approx(sG[t * G::LDG + j]) * __bfloat162float(sK[t * G::LDK + j]);
+      for (int idx = tid; idx < C * DK / 4; idx += G::NT) {
+        const int t = idx / (DK / 4), j = 4 * (idx % (DK / 4));
+        const float4 g = *reinterpret_cast<const float4*>(sG + t * G::LDG + j);
+        float k4[4];
+        bf16x4_to_f32(sK + t * G::LDK + j, k4);
+        const float bt = sBeta[t];
+        *reinterpret_cast<float4*>(sW + t * G::LDW + j) =
+            make_float4(bt * ex2_approx(g.x) * k4[0], bt * ex2_approx(g.y) * k4[1], bt * ex2_approx(g.z) * k4[2],
+                        bt * ex2_approx(g.w) * k4[3]);
       }
-      for (int idx = tid; idx < C * VT; idx += G::NT) {
-        const int t = idx / VT, c = idx % VT;
-        sU[t * G::LDS + c] = sBeta[t] * __bfloat162float(sV[t * G::LDV + c]);
+      for (int idx = tid; idx < C * VT / 4; idx += G::NT) {
+        const int t = idx / (VT / 4), c = 4 * (idx % (VT / 4));
+        float v4[4];
+        bf16x4_to_f32(sV + t * G::LDV + c, v4);
+        const float bt = sBeta[t];
+        *reinterpret_cast<float4*>(sU + t * G::LDS + c) = make_float4(bt * v4[0], bt * v4[1], bt * v4[2], bt * v4[3]);
       }
     } else {
-      for (int idx = tid; idx < C * VT; idx += G::NT) {   // B = V, a tf32 operand
-        const int t = idx / VT, c = idx % VT;
-        sU[t * G::LDS + c] = wm::__float_to_tf32(__bfloat162float(sV[t * G::LDV + c]));
+      for (int idx = tid; idx < C * VT / 4; idx += G::NT) {   // B = V, a tf32 operand (bf16 is tf32-exact)
+        const int t = idx / (VT / 4), c = 4 * (idx % (VT / 4));
+        float v4[4];
+        bf16x4_to_f32(sV + t * G::LDV + c, v4);
+        *reinterpret_cast<float4*>(sU + t * G::LDS + c) = make_float4(v4[0], v4[1], v4[2], v4[3]);
       }
     }
     __syncthreads();
@@ -364,10 +410,15 @@ __global__ void __launch_bounds__(256, 2) key_chunk_prefill_kernel(const Prefill
     }
 
     // 5. the scaled queries e^{Gamma_t} (.) q_t (KDA), e^{Gamma_{t-1}} (.) r_t (RWKV6) into W
-    for (int idx = tid; idx < C * DK; idx += G::NT) {
-      const int t = idx / DK, j = idx % DK;
-      const float g = OP == OP_KDA ? sG[t * G::LDG + j] : (t > 0 ? sG[(t - 1) * G::LDG + j] : 0.f);
-      sW[t * G::LDW + j] = wm::__float_to_tf32(ex2_approx(g) * __bfloat162float(sQ[t * G::LDK + j]));
+    for (int idx = tid; idx < C * DK / 4; idx += G::NT) {
+      const int t = idx / (DK / 4), j = 4 * (idx % (DK / 4));
+      const int tg = OP == OP_KDA ? t : t - 1;
+      const float4 g = tg >= 0 ? *reinterpret_cast<const float4*>(sG + tg * G::LDG + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      float q4[4];
+      bf16x4_to_f32(sQ + t * G::LDK + j, q4);
+      *reinterpret_cast<float4*>(sW + t * G::LDW + j) =
+          make_float4(wm::__float_to_tf32(ex2_approx(g.x) * q4[0]), wm::__float_to_tf32(ex2_approx(g.y) * q4[1]),
+                      wm::__float_to_tf32(ex2_approx(g.z) * q4[2]), wm::__float_to_tf32(ex2_approx(g.w) * q4[3]));
     }
     __syncthreads();
 
@@ -416,10 +467,15 @@ __global__ void __launch_bounds__(256, 2) key_chunk_prefill_kernel(const Prefill
     __syncthreads();
 
     // 7. (e^{Gamma_end - Gamma} (.) K)^T into W, transposed; S rows scaled by e^{Gamma_end}
-    for (int idx = tid; idx < C * DK; idx += G::NT) {
-      const int j = idx / C, t = idx % C;
-      sW[j * G::LDT + t] = wm::__float_to_tf32(ex2_approx(sG[(C - 1) * G::LDG + j] - sG[t * G::LDG + j]) *
-                                               __bfloat162float(sK[t * G::LDK + j]));
+    for (int idx = tid; idx < C * DK / 4; idx += G::NT) {   // four rows t of one key j
+      const int j = idx / (C / 4), t = 4 * (idx % (C / 4));
+      const float gend = sG[(C - 1) * G::LDG + j];
+      float w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        w[e] = wm::__float_to_tf32(ex2_approx(gend - sG[(t + e) * G::LDG + j]) *
+                                   __bfloat162float(sK[(t + e) * G::LDK + j]));
+      *reinterpret_cast<float4*>(sW + j * G::LDT + t) = make_float4(w[0], w[1], w[2], w[3]);
     }
     for (int idx = tid; idx < DK * VT / 4; idx += G::NT) {
       const int row = idx / (VT / 4), c4 = idx % (VT / 4);

@@ -57,9 +57,20 @@ _KERNELS = [(op, dt, k) for op in OPS for dt in (torch.bfloat16, torch.float32)
 @pytest.mark.parametrize("dims", [(64, 64), (128, 128), (64, 128), (128, 64)])
 def test_prefill_then_decode(op, dims, dtype, kernel):
     """Prompts of 37, 0, 1, 130 (several chunks and a ragged tail) and 5 tokens."""
+    _prefill_then_decode(op, dims, dtype, kernel, H=3)
+
+
+@pytest.mark.parametrize("op", OPS)
+def test_prefill_then_decode_whole_head_tiles(op):
+    """The same with 5 rows x 16 heads at d_k = d_v = 128: enough CTAs that the
+    chunked kernels take whole-head tiles (rows x heads above half the SMs)."""
+    _prefill_then_decode(op, (128, 128), torch.bfloat16, "chunked", H=16)
+
+
+def _prefill_then_decode(op, dims, dtype, kernel, H):
     from recurrent_state_update_deltalog_b200 import DeltaLog
     dk, dv = dims
-    B, H, M, T_dec = 8, 3, 4, 7
+    B, M, T_dec = 8, 4, 7
     lens = [37, 0, 1, 130, 5]
     slots = [6, 0, 3, 1, 4]
     rows = len(lens)
