@@ -648,6 +648,36 @@ def fp32_peak_tflops(sm_mhz, sms=148):
     return sms * 128 * 2 * sm_mhz * 1e6 / 1e12
 
 
+def eager_tokenwise(a, seq, names, first, u, stream, dev):
+    """The prefill's prompts token by token through the eager decode kernel:
+    tokens/s and ms of one pass (after one untimed pass)."""
+    import numpy as np
+    import torch
+    from recurrent_state_update_deltalog_b200 import DeltaLog
+    op, B, H, d, L = a.op, a.B, a.H, a.d, a.prefill
+    he = DeltaLog(B, H, d, d, 1, op=op, dtype=torch.bfloat16)
+    if u is not None:
+        he.set_bonus(u)
+    dseq = {nm: torch.from_numpy(np.ascontiguousarray(seq[nm])).to(
+        dev, torch.bfloat16 if nm in (first, "k", "v") else torch.float32) for nm in names}
+    oe = torch.empty((B, H, d), dtype=torch.bfloat16, device=dev)
+
+    def eager_all():
+        for t in range(L):
+            he.eager_step(dseq[first][t], dseq["k"][t], dseq["v"][t], dseq["log_decay"][t],
+                          dseq["beta"][t] if op != "rwkv6" else None, out=oe, stream=stream)
+
+    eager_all()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    eager_all()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    eager_ms = e0.elapsed_time(e1)
+    return {"value": B * L / (eager_ms / 1e3), "unit": "tokens/s", "ms": eager_ms}
+
+
 def run_prefill(a, rank, world, local_rank):
     """Prefill hand-off: B prompts of L tokens packed token-major, every row
     from a zero state into its own slot; tokens/s = B * L / time.  Beside it,
@@ -701,25 +731,10 @@ def run_prefill(a, rank, world, local_rank):
     peak = fp32_peak_tflops(1965.0)
 
     # baseline: the same prompts token by token through the eager decode kernel
-    he = DeltaLog(B, H, d, d, 1, op=op, dtype=torch.bfloat16)
-    if u is not None:
-        he.set_bonus(u)
-    dseq = {nm: torch.from_numpy(np.ascontiguousarray(seq[nm])).to(
-        dev, torch.bfloat16 if nm in (first, "k", "v") else torch.float32) for nm in names}
-    oe = torch.empty((B, H, d), dtype=torch.bfloat16, device=dev)
-
-    def eager_all():
-        for t in range(L):
-            he.eager_step(dseq[first][t], dseq["k"][t], dseq["v"][t], dseq["log_decay"][t],
-                          dseq["beta"][t] if op != "rwkv6" else None, out=oe, stream=stream)
-
-    eager_all()
-    torch.cuda.synchronize(dev)
-    e0.record(stream)
-    eager_all()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    eager_ms = e0.elapsed_time(e1)
+    # (skipped with --no-eager)
+    eager = None
+    if not a.no_eager:
+        eager = eager_tokenwise(a, seq, names, first, u, stream, dev)
     line = {
         "metric": "prefill tokens/s (B*L/s)", "value": tok_s, "unit": "tokens/s", "n_gpus": world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -731,7 +746,7 @@ def run_prefill(a, rank, world, local_rank):
                      "frac": flops / peak, "traffic": None,
                      "peak_note": "fp32 SIMT at the 1965 MHz max clock: 148 SMs x 128 lanes x 2 flops",
                      "flops_per_token_head": prefill_flops(op, d, d), "sm_mhz": sm},
-        "eager_tokenwise": {"value": B * L / (eager_ms / 1e3), "unit": "tokens/s", "ms": eager_ms},
+        "eager_tokenwise": eager,
         "clocks": clocks, "gpu_launches": a.steps,
     }
     if rank == 0:

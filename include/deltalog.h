@@ -244,7 +244,7 @@ int dl_read_state(dl_t h, float* S_out, void* stream);
 /* DL_OPT_PREFILL_KERNEL picks the kernel behind dl_prefill:
  *   DL_PREFILL_AUTO (default): the chunked kernel for bf16-input handles
  *     whose prompts average at least 64 tokens (total >= 64 rows) and, for
- *     KDA, whose rows x H x d_v/16 is below 12 per SM; the recurrent kernel
+ *     KDA, whose rows x H x d_v/16 is below 16 per SM; the recurrent kernel
  *     otherwise;
  *   DL_PREFILL_RECURRENT: the recurrence token by token, state in registers
  *     (every operator and dtype; outputs equal the eager recurrence's up to

@@ -99,7 +99,7 @@ def _prefill_then_decode(op, dims, dtype, kernel, H):
     assert h.log_len == 2                                # the handle's cycle is unchanged
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     auto_chunked = (dtype == torch.bfloat16 and sum(lens) >= 64 * rows       # the automatic rule
-                    and (op != "kda" or rows * H * (dv // 16) < 12 * sms))
+                    and (op != "kda" or rows * H * (dv // 16) < 16 * sms))
     want = "chunked" if kernel == "chunked" or (kernel == "auto" and auto_chunked) else "recurrent"
     assert h.last_prefill_kernel == want
     got = o.float().cpu().numpy()
