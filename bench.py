@@ -30,6 +30,7 @@ METRIC = "state-update tokens/s (B*steps/s)"
 UNIT = "tokens/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0   # burst cuBLAS bf16 GEMM, an earlier B200 measurement
 
 
 def parse():
@@ -643,6 +644,33 @@ def prefill_flops(op, dk, dv):
     return (4 if op != "rwkv6" else 2) * dk * dv + 3 * dk * dv
 
 
+def chunk_prefill_flops(op, d, C):
+    """Flops of the chunk form per token and head (d_k = d_v = d, chunks of C
+    tokens; a multiply-add counts 2).  Tensor-core products with the state,
+    2 d^2 each: W S, (scaled Q) S and the state update for GDN/KDA; (scaled R)
+    S and the update for RWKV6.  Per chunk, the C x C blocks: for GDN/KDA the
+    strictly lower A (C(C-1)/2 dot products of length d), the lower P
+    (C(C+1)/2), the forward substitution for the 2d columns of W and U
+    (C(C-1)/2 multiply-adds each) and P B (C(C+1)/2 d); for RWKV6 the strictly
+    lower P, its diagonal (u (.) k_t) . r_t (2 flops per key) and P V."""
+    if op == "rwkv6":
+        return 4 * d * d + 2 * (C + 1) * d
+    return 6 * d * d + (5 * C - 1) * d
+
+
+# dense tf32 : dense bf16 tensor throughput, nominal (1.1 and 2.25 PFLOP/s)
+TF32_PER_BF16 = 1.1 / 2.25
+
+
+def measured_bf16_tflops():
+    """Burst bf16 GEMM TFLOP/s from the measured peaks, else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
 def fp32_peak_tflops(sm_mhz, sms=148):
     """fp32 SIMT peak: 128 FP32 lanes per SM, one FMA (2 flops) per lane per clock."""
     return sms * 128 * 2 * sm_mhz * 1e6 / 1e12
@@ -726,9 +754,20 @@ def run_prefill(a, rank, world, local_rank):
     ms = e0.elapsed_time(e1) / a.steps
     h.check_device()
     tok_s = B * L / (ms / 1e3)
-    flops = prefill_flops(op, d, d) * H * B * L / (ms / 1e3) / 1e12
     sm = (clocks or {}).get("sm_mhz") or 1965.0
-    peak = fp32_peak_tflops(1965.0)
+    if h.last_prefill_kernel == "chunked":
+        # 16-token chunks only for d = 128 heads split into 64-column tiles
+        C = 16 if op != "gdn" and d == 128 and 2 * B * H <= 148 else 32
+        per_th = chunk_prefill_flops(op, d, C)
+        bf16, kind = measured_bf16_tflops()
+        peak = bf16 * TF32_PER_BF16
+        roof = {"bound": "tensor", "peak_note": f"tf32 dense: {kind} bf16 GEMM x {TF32_PER_BF16:.3f} "
+                "(nominal 1.1 / 2.25 PFLOP/s)", "chunk_tokens": C}
+    else:
+        per_th = prefill_flops(op, d, d)
+        peak = fp32_peak_tflops(1965.0)
+        roof = {"bound": "alu", "peak_note": "fp32 SIMT at the 1965 MHz max clock: 148 SMs x 128 lanes x 2 flops"}
+    flops = per_th * H * B * L / (ms / 1e3) / 1e12
 
     # baseline: the same prompts token by token through the eager decode kernel
     # (skipped with --no-eager)
@@ -742,10 +781,9 @@ def run_prefill(a, rank, world, local_rank):
         "config": {"workload": f"{op}_prefill_b{B}_l{L}_h{H}_d{d}_bf16", "op": op, "B": B, "L": L,
                    "H": H, "d_k": d, "d_v": d, "state": "fp32", "inputs": "bf16",
                    "start": "zero state", "kernel": h.last_prefill_kernel},
-        "roofline": {"bound": "alu", "achieved": flops, "peak": peak, "unit": "TFLOP/s",
-                     "frac": flops / peak, "traffic": None,
-                     "peak_note": "fp32 SIMT at the 1965 MHz max clock: 148 SMs x 128 lanes x 2 flops",
-                     "flops_per_token_head": prefill_flops(op, d, d), "sm_mhz": sm},
+        "roofline": {"bound": roof["bound"], "achieved": flops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": flops / peak, "traffic": None, **{k: v for k, v in roof.items() if k != "bound"},
+                     "flops_per_token_head": per_th, "sm_mhz": sm},
         "eager_tokenwise": eager,
         "clocks": clocks, "gpu_launches": a.steps,
     }

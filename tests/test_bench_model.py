@@ -56,3 +56,32 @@ def test_write_bytes_per_token(op, d, M):
         e = 2 * d + d * (2 if op == "rwkv6" else 4) + (4 if op == "gdn" else 4 * d)
         want = ((M - 1) * (o + e) + (o + 4 * d * d)) / M
     assert bench.write_bytes_per_token(op, 1, H, d, M) == pytest.approx(H * want, rel=1e-12)
+
+
+def _count_chunk_flops(op, d, C):
+    """Flops of one C-token chunk of one head, counted operation by operation
+    with loops (a multiply-add counts 2), divided by C."""
+    f = 0
+    # dense products with the state: [C x d] times [d x d], and the update
+    # [d x C] times [C x d]
+    dense = 3 if op != "rwkv6" else 2
+    f += dense * C * d * d * 2
+    for t in range(C):
+        for s in range(t + 1):
+            if op == "rwkv6":
+                f += 2 * d                       # P[t][s]: a dot product, or the diagonal's u (.) k . r
+                f += 2 * d                       # P V: row t takes P[t][s] v_s
+            else:
+                if s < t:
+                    f += 2 * d                   # A[t][s]
+                f += 2 * d                       # P[t][s]
+                f += 2 * d                       # P B
+        if op != "rwkv6":
+            f += 2 * t * (2 * d)                 # forward substitution, 2d right-hand-side columns
+    return f / C
+
+
+@pytest.mark.parametrize("op", ["gdn", "kda", "rwkv6"])
+@pytest.mark.parametrize("d,C", [(64, 32), (128, 16), (128, 32), (8, 4)])
+def test_chunk_prefill_flops(op, d, C):
+    assert bench.chunk_prefill_flops(op, d, C) == _count_chunk_flops(op, d, C)
