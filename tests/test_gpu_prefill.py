@@ -230,3 +230,37 @@ def test_chunked_prefill_refused_where_it_does_not_apply():
         with pytest.raises(DeltaLogError):
             h.prefill(x, x, x, g, b, cu_seqlens=cu, zero_state=True)
         h.close()
+
+
+@pytest.mark.parametrize("op,kernel", [(op, k) for op in OPS for k in ("recurrent", "chunked")])
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_strong_decay(op, kernel, d):
+    """Log-decays of -40 per token (on three keys for KDA/RWKV6, on every
+    tenth token for GDN): cumulative decays far past fp32 range inside a
+    chunk, which no kernel may divide by."""
+    from recurrent_state_update_deltalog_b200 import DeltaLog
+    dtype, H, lens = torch.bfloat16, 2, [100, 37]
+    rows = len(lens)
+    seq = sequence(51, op, rows, H, d, d, max(lens), bf16=True)
+    seq["log_decay"] = seq["log_decay"].copy()
+    if op == "gdn":
+        seq["log_decay"][::10] = -40.0
+    else:
+        seq["log_decay"][..., :3] = -40.0
+    u = make_inputs(op, 1, H, d, d, 1, dtype, seed=51)[2]
+    packed, cu = _pack(seq, lens)
+    h = DeltaLog(rows, H, d, d, 4, op=op, dtype=dtype)
+    h.set_prefill_kernel(kernel)
+    if u is not None:
+        h.set_bonus(torch.from_numpy(u).cuda())
+    o = h.prefill(*_prefill_args(op, _device_packed(packed, dtype)), cu_seqlens=torch.from_numpy(cu).cuda(),
+                  zero_state=True)
+    got = o.float().cpu().numpy()
+    assert np.all(np.isfinite(got))
+    zero = np.zeros((H, d, d))
+    for r, n in enumerate(lens):
+        o_r, S_r = _oracle_row(op, zero, seq, r, n, u)
+        assert relerr(got[cu[r]:cu[r + 1]], o_r[:, 0]) < TOL[dtype], r
+        assert relerr(h.slot_read(r).cpu().numpy(), S_r[0]) < TOL[dtype], r
+    h.check_device()
+    h.close()
