@@ -3,6 +3,7 @@
 #include "prefill.cuh"
 #include "prefill_chunk.cuh"
 #include "prefill_chunk_key.cuh"
+#include "prefill_chunk_tc.cuh"
 
 namespace dl {
 
@@ -34,10 +35,20 @@ cudaError_t launch_gdn_chunk_prefill(const LaunchShape& s, const PrefillArgs& a,
   return cudaGetLastError();
 }
 
+cudaError_t launch_gdn_chunk_prefill_tc(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st) {
+  using G = TcChunkGeom;
+  auto kern = gdn_chunk_prefill_tc_kernel<0>;
+  if (G::BYTES + 1024 > static_cast<size_t>(s.smem_block_optin)) return cudaErrorNotSupported;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(G::BYTES));
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(s.H, s.units), G::NT, G::BYTES, st>>>(a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gdn_chunk_prefill_dims(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st) {
   if (s.dk == 64 && s.dv == 64) return launch_gdn_chunk_prefill<64, 64, 64>(s, a, st);
   if (s.dk == 128 && s.dv == 128)
-    return whole_head_tiles(s) ? launch_gdn_chunk_prefill<128, 128, 128>(s, a, st)
+    return whole_head_tiles(s) ? launch_gdn_chunk_prefill_tc(s, a, st)
                                : launch_gdn_chunk_prefill<128, 128, 64>(s, a, st);
   if (s.dk == 64 && s.dv == 128) return launch_gdn_chunk_prefill<64, 128, 64>(s, a, st);
   if (s.dk == 128 && s.dv == 64) return launch_gdn_chunk_prefill<128, 64, 64>(s, a, st);

@@ -1,0 +1,493 @@
+// Chunked GDN prefill with the state in tensor memory: the WY chunk form of
+// gdn_chunk_prefill_kernel (prefill_chunk.cuh), with its three products with
+// the state issued as 5th-generation tensor-core MMAs (tcgen05, tf32 operands,
+// fp32 accumulation) on a whole 128 x 128 head per CTA.
+//
+// The state is kept transposed, S^T (value column c on TMEM lane c, key j on
+// column j), so that it serves directly as the A operand of
+//   B^T = U^T - S^T W^T                  (M = 128 value columns, N = C tokens)
+//   O^T = S^T (e^{Gamma} Q)^T + B^T P^T
+//   S^T <- e^{Gamma_end} S^T + B^T (e^{Gamma_end - Gamma} K)
+// and receives the last as its accumulator; it never leaves tensor memory
+// between the prompt's first and last chunk.  W, the scaled queries, P and
+// the scaled keys are written by the SIMT lanes into shared memory in the
+// K-major no-swizzle operand layout (8-row x 16-byte core matrices).  One
+// thread issues the MMAs; their completion is tracked by mbarriers (bounded
+// waits: a wait that runs out raises DL_DEVERR_WAIT_TIMEOUT and the CTA
+// stops).  The state update of chunk i runs while chunk i + 1 computes its
+// gates, A and the triangular solve.
+#pragma once
+
+#include "prefill_chunk.cuh"
+
+namespace dl {
+
+// ---- tcgen05 / tensor-memory wrappers --------------------------------------
+
+// Byte offset of element (r, k) of an R x KT tf32 operand stored K-major with
+// no swizzle: 8-row x 4-element core matrices of 128 contiguous bytes, the
+// core matrices of one 8-row group adjacent along k, groups KT/4 x 128 bytes
+// apart.
+__device__ __forceinline__ uint32_t kmajor_off(int r, int k, int kt) {
+  return static_cast<uint32_t>((r >> 3) * (kt >> 2) * 128 + (k >> 2) * 128 + (r & 7) * 16 + (k & 3) * 4);
+}
+
+// Shared-memory matrix descriptor of such an operand: start address, leading
+// byte offset 128 (next core matrix along k), stride byte offset `sbo` (next
+// 8-row group), descriptor version 1, no swizzle.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t addr, uint32_t sbo) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3fff) | (static_cast<uint64_t>(128 >> 4) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3fff) << 32) | (static_cast<uint64_t>(1) << 46);
+}
+
+// Instruction descriptor: kind::tf32, fp32 accumulator, both operands K-major.
+template <int M, int N>
+__host__ __device__ constexpr uint32_t umma_idesc_tf32() {
+  static_assert(M == 128 && N % 16 == 0 && N >= 16 && N <= 256, "tcgen05 tf32 tile shape");
+  return (1u << 4) | (2u << 7) | (2u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[tmem] B[smem desc]; one thread issues.
+__device__ __forceinline__ void umma_tf32_ts(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+      ::"r"(d), "r"(a), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
+      : "memory");
+}
+
+// Arrive once on `bar` when every MMA this thread issued so far has completed.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// Make this thread's shared-memory writes visible to the tensor cores' reads.
+__device__ __forceinline__ void fence_smem_to_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Warp-collective 32 lanes x 8 / x 32 columns of 32 bits (lane i of the warp
+// gets TMEM lane (address lane + i)).
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+               "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+               "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])),
+      "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+      "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])),
+      "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// ---- geometry ----------------------------------------------------------------
+
+constexpr size_t tc_align128(size_t x) { return (x + 127) & ~size_t(127); }
+
+struct TcChunkGeom {
+  static constexpr int DK = 128, DV = 128;   // a whole head per CTA
+  static constexpr int C = 32;               // tokens per chunk
+  static constexpr int NT = 512, NW = 16;    // threads, warps (four per TMEM lane quarter)
+  static constexpr int LDK = DK + 8;         // bf16 row stride of K and Q
+  static constexpr int LDV = DV + 8;         // bf16 row stride of V
+  static constexpr int LDA = C + 4;          // fp32 row stride of A and P (WMMA outputs)
+  static constexpr int LDU = DV + 4;         // fp32 row stride of U
+  static constexpr size_t KQ_BYTES = tc_align128(size_t(C) * LDK * 2), V_BYTES = tc_align128(size_t(C) * LDV * 2);
+  static constexpr size_t K_OFF = 0;                                  // [2][C][LDK] bf16
+  static constexpr size_t Q_OFF = K_OFF + 2 * KQ_BYTES;               // [C][LDK] bf16
+  static constexpr size_t V_OFF = Q_OFF + KQ_BYTES;                   // [2][C][LDV] bf16
+  static constexpr size_t A_OFF = V_OFF + 2 * V_BYTES;                // [C][LDA] fp32
+  static constexpr size_t WC_OFF = tc_align128(A_OFF + size_t(C) * LDA * 4);   // W, K-major C x DK
+  static constexpr size_t QC_OFF = WC_OFF + size_t(C) * DK * 4;       // e^G Q, K-major C x DK
+  static constexpr size_t PC_OFF = QC_OFF + size_t(C) * DK * 4;       // P, K-major C x C
+  static constexpr size_t KC_OFF = PC_OFF + size_t(C) * C * 4;        // (e^{..} K)^T, K-major DK x C
+  static constexpr size_t U_OFF = KC_OFF + size_t(DK) * C * 4;        // [C][LDU] fp32
+  static constexpr size_t G_OFF = tc_align128(U_OFF + size_t(C) * LDU * 4);    // 5 x [C] per-row factors
+  static constexpr size_t BAR_OFF = tc_align128(G_OFF + 5 * C * 4);            // 3 mbarriers, TMEM base, abort flag
+  static constexpr size_t BYTES = BAR_OFF + 64;
+  // tensor-memory columns
+  static constexpr uint32_t TM_COLS = 256;   // allocation (power of two)
+  static constexpr uint32_t TM_S = 0;        // S^T: 128 columns (keys)
+  static constexpr uint32_t TM_B = 128;      // W S, then B^T: C columns (tokens)
+  static constexpr uint32_t TM_O = 160;      // O^T: C columns
+};
+
+template <int DUMMY = 0>
+__global__ void __launch_bounds__(512, 1) gdn_chunk_prefill_tc_kernel(const PrefillArgs a) {
+  using G = TcChunkGeom;
+  constexpr int C = G::C, DK = G::DK, DV = G::DV;
+  extern __shared__ __align__(128) unsigned char smem[];
+  auto kbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem + G::K_OFF + b * G::KQ_BYTES); };
+  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem + G::Q_OFF);
+  auto vbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem + G::V_OFF + b * G::V_BYTES); };
+  float* sA = reinterpret_cast<float*>(smem + G::A_OFF);
+  unsigned char* sWc = smem + G::WC_OFF;
+  unsigned char* sQc = smem + G::QC_OFF;
+  unsigned char* sPc = smem + G::PC_OFF;
+  unsigned char* sKc = smem + G::KC_OFF;
+  float* sU = reinterpret_cast<float*>(smem + G::U_OFF);
+  float* sG = reinterpret_cast<float*>(smem + G::G_OFF);
+  float* sBeta = sG + C;
+  float* sEG = sG + 2 * C;
+  float* sBEG = sG + 3 * C;
+  float* sEnd = sG + 4 * C;
+  uint64_t* barB = reinterpret_cast<uint64_t*>(smem + G::BAR_OFF);   // W S done
+  uint64_t* barO = barB + 1;                                          // O^T done
+  uint64_t* barS = barB + 2;                                          // state update done
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(barB + 3);
+  volatile int* sAbort = reinterpret_cast<volatile int*>(sTmem + 1);
+  auto fp = [](unsigned char* base, uint32_t off) { return reinterpret_cast<float*>(base + off); };
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int quarter = warp & 3, group = warp >> 2;   // TMEM lanes 32 quarter .., column group
+  const int h = blockIdx.x;
+  const int r = blockIdx.y;
+
+  const int slot = a.slot_idx ? __ldg(a.slot_idx + r) : r;
+  if (slot < 0) return;
+  if (slot >= a.slots) {
+    if (tid == 0) atomicOr(a.err, kErrSlotIndex);
+    return;
+  }
+  const long t0 = __ldg(a.cu_seqlens + r), t1 = __ldg(a.cu_seqlens + r + 1);
+  if (t0 < 0 || t1 < t0 || t1 > a.total) {
+    if (tid == 0) atomicOr(a.err, kErrSeqlen);
+    return;
+  }
+  const long sh = static_cast<long>(slot) * a.H + h;
+  float* Sg = a.Sbar + sh * (DK * DV);
+
+  if (tid == 0) {
+    mbar_init(barB, 1);
+    mbar_init(barO, 1);
+    mbar_init(barS, 1);
+    fence_mbar_init();
+    *sAbort = 0;
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(sTmem)),
+                 "r"(G::TM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sTmem;
+  const uint32_t lane_base = static_cast<uint32_t>(32 * quarter) << 16;
+  const int c_own = 32 * quarter + lane;   // this thread's value column in TMEM epilogues
+
+  // S^T into tensor memory: this warp's 32 lanes (value columns), keys 32 group ..
+  {
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = a.zero_state ? 0.f : __ldcs(Sg + (32 * group + i) * DV + c_own);
+    tmem_st32(tmem + lane_base + G::TM_S + 32 * group, v);
+    tmem_wait_st();
+  }
+
+  const __nv_bfloat16* Kg = static_cast<const __nv_bfloat16*>(a.k);
+  const __nv_bfloat16* Qg = static_cast<const __nv_bfloat16*>(a.q);
+  const __nv_bfloat16* Vg = static_cast<const __nv_bfloat16*>(a.v);
+  __nv_bfloat16* Og = static_cast<__nv_bfloat16*>(a.o);
+  const __nv_bfloat16 zero_bf = __float2bfloat16_rn(0.f);
+
+  // Stage rows [c, c + C) of a [total][H][width] bf16 input into dst (row
+  // stride ld); rows past the prompt are zeros.
+  const bool async_ok = aligned_to(a.q, 16) && aligned_to(a.k, 16) && aligned_to(a.v, 16);
+  auto stage_rows = [&](__nv_bfloat16* dst, const __nv_bfloat16* src, long c, int width, int ld) {
+    const int nv = static_cast<int>(t1 - c < C ? t1 - c : C);
+    if (async_ok) {
+      const int seg_per_row = width / 8;
+      for (int idx = tid; idx < C * seg_per_row; idx += G::NT) {
+        const int t = idx / seg_per_row, seg = idx % seg_per_row;
+        const long row = ((c + (t < nv ? t : nv - 1)) * a.H + h) * width + 8 * seg;
+        cp_async16(dst + t * ld + 8 * seg, src + row, t < nv ? 16u : 0u);
+      }
+    } else {
+      for (int idx = tid; idx < C * width; idx += G::NT) {
+        const int t = idx / width, j = idx % width;
+        dst[t * ld + j] = t < nv ? src[((c + t) * a.H + h) * width + j] : zero_bf;
+      }
+    }
+  };
+  auto stage_kv = [&](int b, long c) {
+    stage_rows(kbuf(b), Kg, c, DK, G::LDK);
+    stage_rows(vbuf(b), Vg, c, DV, G::LDV);
+  };
+  float gn = 0.f, bnv = 0.f;   // warp 0, lane t: gate and beta of row t of the next chunk
+  auto fetch_gates = [&](long c) {
+    const int nv = static_cast<int>(t1 - c < C ? t1 - c : C);
+    gn = lane < nv ? a.log_decay[(c + lane) * a.H + h] : 0.f;
+    bnv = lane < nv ? a.beta[(c + lane) * a.H + h] : 0.f;
+  };
+  if (t0 < t1) {
+    stage_kv(0, t0);
+    if (warp == 0) fetch_gates(t0);
+  }
+  cp_async_commit();
+
+  // (r, k) of element e of a K-major operand with kt columns, enumerated in
+  // storage order (e * 4 is its byte offset)
+  auto kmajor_rk = [](int e, int kt, int& rr, int& kk) {
+    const int core = e >> 5, within = e & 31;
+    rr = (core / (kt >> 2)) * 8 + (within >> 2);
+    kk = (core % (kt >> 2)) * 4 + (within & 3);
+  };
+  float* sWt = reinterpret_cast<float*>(smem + G::QC_OFF);   // W row-major [C][DK + 4] during the solve
+  constexpr int LDW = DK + 4;
+  static_assert(size_t(C) * LDW * 4 <= G::KC_OFF - G::QC_OFF, "row-major W fits the Q and P operand space");
+
+  int buf = 0, ci = 0;
+  for (long c0 = t0; c0 < t1; c0 += C, buf ^= 1, ++ci) {
+    const int n = static_cast<int>(t1 - c0 < C ? t1 - c0 : C);
+    const bool has_next = c0 + C < t1;
+    const uint32_t par = static_cast<uint32_t>(ci & 1);
+    __syncthreads();   // the previous chunk is done with every buffer
+    stage_rows(sQ, Qg, c0, DK, G::LDK);
+    cp_async_commit();
+    if (has_next) stage_kv(buf ^ 1, c0 + C);
+    cp_async_commit();
+    cp_async_wait<2>();   // K/V of this chunk have landed
+    __nv_bfloat16 *sK = kbuf(buf), *sV = vbuf(buf);
+
+    // 1. Gamma (inclusive prefix of the log-gates), beta and per-row factors
+    if (warp == 0) {
+      float incl = gn;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      const float gend = __shfl_sync(0xffffffffu, incl, n - 1);
+      const float eg = expf(incl);
+      sG[lane] = incl;
+      sBeta[lane] = bnv;
+      sEG[lane] = eg;
+      sBEG[lane] = bnv * eg;
+      sEnd[lane] = lane < n ? expf(gend - incl) : 0.f;
+      if (has_next) fetch_gates(c0 + C);
+    }
+    __syncthreads();
+
+    // 2. A = strictly lower (beta_t e^{G_t - G_s} k_t . k_s); right-hand sides
+    lower_xyt<C, DK, G::LDK, G::LDA>(sK, sK, sA);
+    __syncthreads();
+    for (int idx = tid; idx < C * C; idx += G::NT) {
+      const int t = idx / C, s = idx % C;
+      float& x = sA[t * G::LDA + s];
+      x = s < t ? sBeta[t] * expf(sG[t] - sG[s]) * x : 0.f;
+    }
+    for (int idx = tid; idx < C * DK; idx += G::NT) {
+      const int t = idx / DK, j = idx % DK;
+      sWt[t * LDW + j] = sBEG[t] * __bfloat162float(sK[t * G::LDK + j]);
+    }
+    for (int idx = tid; idx < C * DV; idx += G::NT) {
+      const int t = idx / DV, c = idx % DV;
+      sU[t * G::LDU + c] = sBeta[t] * __bfloat162float(sV[t * G::LDV + c]);
+    }
+    __syncthreads();
+
+    // 3. (I + A) X = R, one right-hand-side column per thread
+    if (tid < DK + DV) {
+      const bool isw = tid < DK;
+      float* col = isw ? sWt + tid : sU + (tid - DK);
+      const int ld = isw ? LDW : G::LDU;
+      float x[C];
+#pragma unroll
+      for (int t = 0; t < C; ++t) {
+        float acc0 = col[t * ld], acc1 = 0.f;
+        const float* arow = sA + t * G::LDA;
+#pragma unroll
+        for (int s = 0; s + 3 < t; s += 4) {
+          const float4 a4 = *reinterpret_cast<const float4*>(arow + s);
+          acc0 = fmaf(-a4.x, x[s], acc0);
+          acc1 = fmaf(-a4.y, x[s + 1], acc1);
+          acc0 = fmaf(-a4.z, x[s + 2], acc0);
+          acc1 = fmaf(-a4.w, x[s + 3], acc1);
+        }
+#pragma unroll
+        for (int s = t & ~3; s < t; ++s) acc0 = fmaf(-arow[s], x[s], acc0);
+        x[t] = acc0 + acc1;
+        col[t * ld] = x[t];
+      }
+    }
+    __syncthreads();
+    // W into its K-major operand layout, tf32-rounded
+    for (int e = tid; e < C * DK; e += G::NT) {
+      int t, j;
+      kmajor_rk(e, DK, t, j);
+      fp(sWc, 4 * e)[0] = wm::__float_to_tf32(sWt[t * LDW + j]);
+    }
+    fence_smem_to_async();
+
+    // 4. the previous chunk's state update must be complete before S^T is read
+    if (ci > 0 && !mbar_wait_abortable(barS, par ^ 1u, sAbort) && tid == 0) atomicOr(a.err, kErrWaitTimeout);
+    tc_fence_before();
+    __syncthreads();
+    if (*sAbort) break;
+    tc_fence_after();
+    if (tid == 0) {   // W S  (M = 128 value columns, N = C tokens, K = DK)
+      constexpr uint32_t ID = umma_idesc_tf32<128, C>();
+      const uint32_t w0 = smem_u32(sWc);
+#pragma unroll
+      for (int s = 0; s < DK / 8; ++s)
+        umma_tf32_ts(tmem + G::TM_B, tmem + G::TM_S + 8 * s, umma_desc(w0 + 256 * s, (DK / 4) * 128), ID, s > 0);
+      umma_commit(barB);
+    }
+
+    // 5. P = Q K^T (.) [e^{G_t - G_s}]_{s <= t}, e^G Q and (e^{G_end - G} K)^T as operands
+    cp_async_wait<1>();   // Q of this chunk has landed
+    __syncthreads();
+    lower_xyt<C, DK, G::LDK, G::LDA>(sQ, sK, sA);
+    __syncthreads();
+    for (int e = tid; e < C * C; e += G::NT) {
+      int t, s;
+      kmajor_rk(e, C, t, s);
+      fp(sPc, 4 * e)[0] = s <= t ? wm::__float_to_tf32(expf(sG[t] - sG[s]) * sA[t * G::LDA + s]) : 0.f;
+    }
+    for (int e = tid; e < C * DK; e += G::NT) {
+      int t, j;
+      kmajor_rk(e, DK, t, j);
+      fp(sQc, 4 * e)[0] = wm::__float_to_tf32(sEG[t] * __bfloat162float(sQ[t * G::LDK + j]));
+    }
+    for (int e = tid; e < DK * C; e += G::NT) {
+      int j, t;
+      kmajor_rk(e, C, j, t);
+      fp(sKc, 4 * e)[0] = wm::__float_to_tf32(sEnd[t] * __bfloat162float(sK[t * G::LDK + j]));
+    }
+    fence_smem_to_async();
+    __syncthreads();
+    if (tid == 0) {   // O^T = S^T (e^G Q)^T, first term
+      tc_fence_after();
+      constexpr uint32_t ID = umma_idesc_tf32<128, C>();
+      const uint32_t q0 = smem_u32(sQc);
+#pragma unroll
+      for (int s = 0; s < DK / 8; ++s)
+        umma_tf32_ts(tmem + G::TM_O, tmem + G::TM_S + 8 * s, umma_desc(q0 + 256 * s, (DK / 4) * 128), ID, s > 0);
+    }
+
+    // 6. B^T = U^T - (W S)^T in tensor memory, tf32-rounded (columns 8 group ..)
+    if (!mbar_wait_abortable(barB, par, sAbort) && tid == 0) atomicOr(a.err, kErrWaitTimeout);
+    tc_fence_after();
+    if (!*sAbort) {
+      float v[8];
+      const uint32_t ta = tmem + lane_base + G::TM_B + 8 * group;
+      tmem_ld8(ta, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = wm::__float_to_tf32(sU[(8 * group + i) * G::LDU + c_own] - v[i]);
+      tmem_st8(ta, v);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*sAbort) break;
+    if (tid == 0) {   // O^T += B^T P^T
+      tc_fence_after();
+      constexpr uint32_t ID = umma_idesc_tf32<128, C>();
+      const uint32_t p0 = smem_u32(sPc);
+#pragma unroll
+      for (int s = 0; s < C / 8; ++s)
+        umma_tf32_ts(tmem + G::TM_O, tmem + G::TM_B + 8 * s, umma_desc(p0 + 256 * s, (C / 4) * 128), ID, 1u);
+      umma_commit(barO);
+    }
+
+    // 7. O rows < n to global; S^T scaled by e^{G_end} (every MMA reading it is done)
+    if (!mbar_wait_abortable(barO, par, sAbort) && tid == 0) atomicOr(a.err, kErrWaitTimeout);
+    tc_fence_after();
+    if (!*sAbort) {
+      float v[8];
+      tmem_ld8(tmem + lane_base + G::TM_O + 8 * group, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int t = 8 * group + i;
+        if (t < n) Og[((c0 + t) * a.H + h) * DV + c_own] = __float2bfloat16_rn(v[i]);
+      }
+      const float dend = sEG[n - 1];
+      float sv[32];
+      const uint32_t ts = tmem + lane_base + G::TM_S + 32 * group;
+      tmem_ld32(ts, sv);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) sv[i] *= dend;
+      tmem_st32(ts, sv);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*sAbort) break;
+    if (tid == 0) {   // S^T += B^T (e^{G_end - G} K)   (N = DK keys, K = C tokens)
+      tc_fence_after();
+      constexpr uint32_t ID = umma_idesc_tf32<128, DK>();
+      const uint32_t k0 = smem_u32(sKc);
+#pragma unroll
+      for (int s = 0; s < C / 8; ++s)
+        umma_tf32_ts(tmem + G::TM_S, tmem + G::TM_B + 8 * s, umma_desc(k0 + 256 * s, (C / 4) * 128), ID, 1u);
+      umma_commit(barS);
+    }
+  }
+
+  // the last state update, then S^T back to Sbar
+  if (ci > 0 && !*sAbort && !mbar_wait_abortable(barS, static_cast<uint32_t>((ci - 1) & 1), sAbort) && tid == 0)
+    atomicOr(a.err, kErrWaitTimeout);
+  cp_async_wait<0>();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const bool ok = !*sAbort;
+  if (ok) {
+    float v[32];
+    tmem_ld32(tmem + lane_base + G::TM_S + 32 * group, v);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) __stcs(Sg + (32 * group + i) * DV + c_own, v[i]);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(G::TM_COLS) : "memory");
+  }
+  if (ok) clear_log_tile<OP_GDN, DK, DV, __nv_bfloat16>(a, sh, 0, DV);
+}
+
+// Grid (H, rows), 512 threads, TcChunkGeom::BYTES of dynamic shared memory;
+// d_k = d_v = 128, bf16 inputs.  Instantiated in prefill.cu.
+cudaError_t launch_gdn_chunk_prefill_tc(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st);
+
+}  // namespace dl
