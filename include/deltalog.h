@@ -243,18 +243,20 @@ int dl_read_state(dl_t h, float* S_out, void* stream);
  * streaming kernel does not take it (DL_ERR_UNSUPPORTED). */
 /* DL_OPT_PREFILL_KERNEL picks the kernel behind dl_prefill:
  *   DL_PREFILL_AUTO (default): the chunked kernel for bf16-input handles
- *     whose prompts average at least 64 tokens (total >= 64 rows) and, for
- *     KDA, whose rows x H x d_v/16 is below 16 per SM; the recurrent kernel
- *     otherwise;
+ *     whose prompts average at least 64 tokens (total >= 64 rows), the
+ *     recurrent kernel otherwise;
  *   DL_PREFILL_RECURRENT: the recurrence token by token, state in registers
  *     (every operator and dtype; outputs equal the eager recurrence's up to
  *     fp32 rounding);
  *   DL_PREFILL_CHUNKED: the chunk form on tensor cores (bf16-input handles
- *     only, DL_ERR_UNSUPPORTED otherwise).  GDN: 32-token chunks in the WY
- *     form of the delta rule, bf16 products of the inputs.  KDA and RWKV6:
- *     chunks of 16 tokens (d_k = 128) or 32 (d_k = 64) whose per-key pair
- *     weights are formed exactly on the SIMT lanes.  The products with the
- *     state are tf32 (2^-11 relative), inside the bf16-input tolerance. */
+ *     only, DL_ERR_UNSUPPORTED otherwise): 32-token chunks, the WY form of
+ *     the delta rule for GDN and KDA, per-key pair weights of KDA and RWKV6
+ *     formed exactly on the SIMT lanes.  At d_k = d_v = 128, once rows x H
+ *     reach half the SM count, each CTA keeps a whole head's state in tensor
+ *     memory and runs the products with it as tcgen05 MMAs; otherwise
+ *     64-column tiles (16-token chunks for per-key decay at d_k = 128) use
+ *     warp-level MMAs.  The products with the state are tf32, inside the
+ *     bf16-input tolerance. */
 enum dl_option {
   DL_OPT_STEP_KERNEL = 0,
   DL_OPT_HOST_PREFETCH = 1,

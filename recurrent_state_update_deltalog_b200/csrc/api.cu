@@ -298,21 +298,17 @@ cudaError_t materialize_slots(const dl_handle* h, const int* slot_idx, int rows,
 }
 
 // The chunked tensor-core prefills serve bf16-input handles.  AUTO picks them
-// unless the prompts are short (fewer than 64 tokens on average); for KDA only
-// while the recurrent kernel's one-warp tiles (rows x heads x d_v/16) do not
-// fill the GPU (16 resident per SM).  Measured on B200 against the recurrent
-// kernel, bf16, d = 128, H = 32 unless stated:
-//   GDN:   B=256 L=64 1.04, B=64 L=512 1.16, B=4 L=4096 1.98, B=1 L=8192 2.5,
-//          d=64 1.22; 0.97 at L=32;
-//   RWKV6 (H=64, d=64): B=512 L=32 0.98, B=256 L=64 1.03, B=64 L=512 1.10,
-//          B=16 L=1024 1.58, B=4 L=4096 2.70, B=1 L=8192 3.79;
-//   KDA:   B=1 L=8192 1.89, B=4 L=4096 1.66, B=8 L=2048 1.06, but B=16
-//          L=1024 0.94, B=64 L=512 1.00 and B=256 L=64 0.93 once the recurrent
-//          kernel fills the GPU.
+// unless the prompts are short (fewer than 64 tokens on average).  Measured
+// on B200 against the recurrent kernel (bf16, H = 32, d = 128 unless
+// stated), with whole-head tcgen05 CTAs where rows x heads cover half the SMs:
+//   GDN:   B=256 L=64 2.0, B=64 L=512 2.4, B=4 L=4096 4.1, B=1 L=8192 2.5
+//          (64-column tiles); 0.97 on 32-token prompts (before tcgen05);
+//   KDA:   B=256 L=64 1.49, B=64 L=512 1.68, B=4 L=4096 2.80, B=1 L=8192 1.89;
+//   RWKV6 (H=64, d=64, tensor-core WMMA): B=512 L=32 0.98, B=256 L=64 1.03,
+//          B=64 L=512 1.10, B=4 L=4096 2.70, B=1 L=8192 3.79.
 bool chunked_prefill(const dl_handle* h, int rows, long long total) {
   if (h->prefill_kernel != DL_PREFILL_AUTO) return h->prefill_kernel == DL_PREFILL_CHUNKED;
-  if (h->dtype != DL_BF16 || total < 64LL * rows) return false;
-  return h->op != DL_KDA || static_cast<long long>(rows) * h->H * (h->dv / 16) < 16LL * h->sms;
+  return h->dtype == DL_BF16 && total >= 64LL * rows;
 }
 
 cudaError_t launch_prefill(dl_handle* h, const dl::PrefillArgs& a, int rows, cudaStream_t s) {

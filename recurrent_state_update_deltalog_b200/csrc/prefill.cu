@@ -67,10 +67,21 @@ cudaError_t launch_key_chunk_prefill(const LaunchShape& s, const PrefillArgs& a,
 }
 
 template <int OP>
+cudaError_t launch_key_chunk_prefill_tc(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st) {
+  using G = KeyTcChunkGeom;
+  auto kern = key_chunk_prefill_tc_kernel<OP>;
+  if (G::BYTES + 1024 > static_cast<size_t>(s.smem_block_optin)) return cudaErrorNotSupported;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(G::BYTES));
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(s.H, s.units), G::NT, G::BYTES, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int OP>
 cudaError_t launch_key_chunk_prefill_dims(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st) {
   if (s.dk == 64 && s.dv == 64) return launch_key_chunk_prefill<OP, 64, 64, 64>(s, a, st);
   if (s.dk == 128 && s.dv == 128)
-    return whole_head_tiles(s) ? launch_key_chunk_prefill<OP, 128, 128, 128>(s, a, st)
+    return whole_head_tiles(s) ? launch_key_chunk_prefill_tc<OP>(s, a, st)
                                : launch_key_chunk_prefill<OP, 128, 128, 64>(s, a, st);
   if (s.dk == 64 && s.dv == 128) return launch_key_chunk_prefill<OP, 64, 128, 64>(s, a, st);
   if (s.dk == 128 && s.dv == 64) return launch_key_chunk_prefill<OP, 128, 64, 64>(s, a, st);

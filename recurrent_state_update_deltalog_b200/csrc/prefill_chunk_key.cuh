@@ -117,6 +117,88 @@ __device__ __forceinline__ void strict_pair(int p, int& t, int& s) {
   s = p - t * (t - 1) / 2;
 }
 
+// A (KDA: beta_t-weighted, strictly lower) and P (lower; RWKV6: strictly
+// lower plus the bonus diagonal) of one chunk, pair by pair with one exp2 per
+// (pair, key) from Gamma in log2 units; the upper triangles zero.  P is stored
+// tf32-rounded.  When twice the strict pairs plus the diagonal make exactly
+// one item per thread, each strict pair is split between two adjacent lanes,
+// one half of the keys each.
+template <int OP, int DK, int C, int NT, int LDK, int LDG, int LDA>
+__device__ __forceinline__ void key_pair_phase(const __nv_bfloat16* sK, const __nv_bfloat16* sQ, const float* sG,
+                                               const float* sBeta, const float* sBonus, float* sA, float* sP) {
+  constexpr bool DELTA = OP == OP_KDA;
+  const int tid = threadIdx.x;
+  constexpr int NSTRICT = C * (C - 1) / 2;
+  constexpr bool SPLIT = 2 * NSTRICT + C == NT;
+  constexpr int NITEMS = SPLIT ? NT : NSTRICT + C;
+  for (int p = tid; p < NITEMS; p += NT) {
+    const int nstr = SPLIT ? 2 * NSTRICT : NSTRICT;   // strict items come first
+    const bool strict = p < nstr;
+    int t, s;
+    if (strict) {
+      strict_pair(SPLIT ? p >> 1 : p, t, s);
+    } else {
+      t = s = p - nstr;
+    }
+    const int j0 = SPLIT && strict ? (p & 1) * (DK / 2) : 0;
+    const int j1 = SPLIT && strict ? j0 + DK / 2 : DK;
+    const __nv_bfloat16* kt = sK + t * LDK;
+    const __nv_bfloat16* ks = sK + s * LDK;
+    const __nv_bfloat16* qt = sQ + t * LDK;
+    float accA = 0.f, accP = 0.f;
+    if (strict) {
+      // exponent rows: Gamma_t (KDA) or Gamma_{t-1} (RWKV6), against Gamma_s
+      const float* gt = sG + (OP == OP_RWKV6 ? t - 1 : t) * LDG;
+      const float* gs = sG + s * LDG;
+#pragma unroll 2
+      for (int j = j0; j < j1; j += 8) {
+        float fks[8], fqt[8], fkt[8];
+        bf16x8_to_f32(ks + j, fks);
+        bf16x8_to_f32(qt + j, fqt);
+        if (DELTA) bf16x8_to_f32(kt + j, fkt);
+        const float4 gt0 = *reinterpret_cast<const float4*>(gt + j);
+        const float4 gt1 = *reinterpret_cast<const float4*>(gt + j + 4);
+        const float4 gs0 = *reinterpret_cast<const float4*>(gs + j);
+        const float4 gs1 = *reinterpret_cast<const float4*>(gs + j + 4);
+        const float d[8] = {gt0.x - gs0.x, gt0.y - gs0.y, gt0.z - gs0.z, gt0.w - gs0.w,
+                            gt1.x - gs1.x, gt1.y - gs1.y, gt1.z - gs1.z, gt1.w - gs1.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float m = fks[e] * ex2_approx(d[e]);
+          if (DELTA) accA = fmaf(fkt[e], m, accA);
+          accP = fmaf(fqt[e], m, accP);
+        }
+      }
+    } else {
+      // diagonal: q_t . k_t (KDA), (u (.) k_t) . r_t (RWKV6)
+#pragma unroll 2
+      for (int j = 0; j < DK; j += 8) {
+        float fkt[8], fqt[8];
+        bf16x8_to_f32(kt + j, fkt);
+        bf16x8_to_f32(qt + j, fqt);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) accP = fmaf(fqt[e], OP == OP_RWKV6 ? sBonus[j + e] * fkt[e] : fkt[e], accP);
+      }
+    }
+    if (SPLIT) {   // one item per thread: every lane of the warp reaches the shuffles
+      const float oA = __shfl_xor_sync(0xffffffffu, accA, 1), oP = __shfl_xor_sync(0xffffffffu, accP, 1);
+      if (strict) {
+        accA += oA;
+        accP += oP;
+      }
+    }
+    if (!SPLIT || !strict || (p & 1) == 0) {
+      if (DELTA && strict) sA[t * LDA + s] = sBeta[t] * accA;
+      sP[t * LDA + s] = wm::__float_to_tf32(accP);
+    }
+  }
+  for (int idx = tid; idx < C * C; idx += NT) {
+    const int t = idx / C, s = idx % C;
+    if (s > t) sP[t * LDA + s] = 0.f;
+    if (DELTA && s >= t) sA[t * LDA + s] = 0.f;
+  }
+}
+
 template <int OP, int DK, int DV, int VT_>
 __global__ void __launch_bounds__(KeyChunkGeom<DK, VT_>::NT, KeyChunkGeom<DK, VT_>::MINB)
     key_chunk_prefill_kernel(const PrefillArgs a) {
@@ -240,79 +322,8 @@ __global__ void __launch_bounds__(KeyChunkGeom<DK, VT_>::NT, KeyChunkGeom<DK, VT
     }
     __syncthreads();
 
-    // 2. A and P pair by pair; the upper triangles zero; right-hand sides.
-    // When twice the strict pairs plus the diagonal make exactly one item per
-    // thread (C = 16), each strict pair is split between two adjacent lanes,
-    // one half of the keys each.
-    constexpr int NSTRICT = C * (C - 1) / 2;
-    constexpr bool SPLIT = 2 * NSTRICT + C == G::NT;
-    constexpr int NITEMS = SPLIT ? G::NT : NSTRICT + C;
-    for (int p = tid; p < NITEMS; p += G::NT) {
-      const int nstr = SPLIT ? 2 * NSTRICT : NSTRICT;   // strict items come first
-      const bool strict = p < nstr;
-      int t, s;
-      if (strict) {
-        strict_pair(SPLIT ? p >> 1 : p, t, s);
-      } else {
-        t = s = p - nstr;
-      }
-      const int j0 = SPLIT && strict ? (p & 1) * (DK / 2) : 0;
-      const int j1 = SPLIT && strict ? j0 + DK / 2 : DK;
-      const __nv_bfloat16* kt = sK + t * G::LDK;
-      const __nv_bfloat16* ks = sK + s * G::LDK;
-      const __nv_bfloat16* qt = sQ + t * G::LDK;
-      float accA = 0.f, accP = 0.f;
-      if (strict) {
-        // exponent rows: Gamma_t (KDA) or Gamma_{t-1} (RWKV6), against Gamma_s
-        const float* gt = sG + (OP == OP_RWKV6 ? t - 1 : t) * G::LDG;
-        const float* gs = sG + s * G::LDG;
-#pragma unroll 2
-        for (int j = j0; j < j1; j += 8) {
-          float fks[8], fqt[8], fkt[8];
-          bf16x8_to_f32(ks + j, fks);
-          bf16x8_to_f32(qt + j, fqt);
-          if (DELTA) bf16x8_to_f32(kt + j, fkt);
-          const float4 gt0 = *reinterpret_cast<const float4*>(gt + j);
-          const float4 gt1 = *reinterpret_cast<const float4*>(gt + j + 4);
-          const float4 gs0 = *reinterpret_cast<const float4*>(gs + j);
-          const float4 gs1 = *reinterpret_cast<const float4*>(gs + j + 4);
-          const float d[8] = {gt0.x - gs0.x, gt0.y - gs0.y, gt0.z - gs0.z, gt0.w - gs0.w,
-                              gt1.x - gs1.x, gt1.y - gs1.y, gt1.z - gs1.z, gt1.w - gs1.w};
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float m = fks[e] * ex2_approx(d[e]);
-            if (DELTA) accA = fmaf(fkt[e], m, accA);
-            accP = fmaf(fqt[e], m, accP);
-          }
-        }
-      } else {
-        // diagonal: q_t . k_t (KDA), (u (.) k_t) . r_t (RWKV6)
-#pragma unroll 2
-        for (int j = 0; j < DK; j += 8) {
-          float fkt[8], fqt[8];
-          bf16x8_to_f32(kt + j, fkt);
-          bf16x8_to_f32(qt + j, fqt);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) accP = fmaf(fqt[e], OP == OP_RWKV6 ? sBonus[j + e] * fkt[e] : fkt[e], accP);
-        }
-      }
-      if (SPLIT) {   // one item per thread: every lane of the warp reaches the shuffles
-        const float oA = __shfl_xor_sync(0xffffffffu, accA, 1), oP = __shfl_xor_sync(0xffffffffu, accP, 1);
-        if (strict) {
-          accA += oA;
-          accP += oP;
-        }
-      }
-      if (!SPLIT || !strict || (p & 1) == 0) {
-        if (DELTA && strict) sA[t * G::LDA + s] = sBeta[t] * accA;
-        sP[t * G::LDA + s] = wm::__float_to_tf32(accP);
-      }
-    }
-    for (int idx = tid; idx < C * C; idx += G::NT) {
-      const int t = idx / C, s = idx % C;
-      if (s > t) sP[t * G::LDA + s] = 0.f;
-      if (DELTA && s >= t) sA[t * G::LDA + s] = 0.f;
-    }
+    // 2. A and P pair by pair; the upper triangles zero; right-hand sides
+    key_pair_phase<OP, DK, C, G::NT, G::LDK, G::LDG, G::LDA>(sK, sQ, sG, sBeta, sBonus, sA, sP);
     // four consecutive columns per thread in the element-wise passes below
     if (DELTA) {
       // beta (e^{Gamma} (.) K) into W, beta V into U

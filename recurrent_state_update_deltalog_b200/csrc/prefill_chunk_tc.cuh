@@ -19,6 +19,7 @@
 #pragma once
 
 #include "prefill_chunk.cuh"
+#include "prefill_chunk_key.cuh"
 
 namespace dl {
 
@@ -489,5 +490,398 @@ __global__ void __launch_bounds__(512, 1) gdn_chunk_prefill_tc_kernel(const Pref
 // Grid (H, rows), 512 threads, TcChunkGeom::BYTES of dynamic shared memory;
 // d_k = d_v = 128, bf16 inputs.  Instantiated in prefill.cu.
 cudaError_t launch_gdn_chunk_prefill_tc(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st);
+
+// ---- KDA and RWKV6 (per-key decay) ---------------------------------------------
+//
+// The chunk form of key_chunk_prefill_kernel (prefill_chunk_key.cuh) with the
+// same tensor-memory state: A and P pair by pair on the SIMT lanes, the three
+// products with the state on tcgen05.  RWKV6 has no W S product: its B^T is
+// V^T, written straight into tensor memory.  The per-key decay of the state
+// update scales the columns of S^T.
+
+struct KeyTcChunkGeom {
+  static constexpr int DK = 128, DV = 128, C = 32, NT = 512, NW = 16;
+  static constexpr int LDK = DK + 8, LDV = DV + 8, LDG = DK + 4, LDA = C + 4, LDU = DV + 4;
+  static constexpr size_t KQ_BYTES = tc_align128(size_t(C) * LDK * 2), V_BYTES = tc_align128(size_t(C) * LDV * 2);
+  static constexpr size_t G_BYTES = tc_align128(size_t(C) * LDG * 4);
+  static constexpr size_t K_OFF = 0;                                   // [2][C][LDK] bf16
+  static constexpr size_t Q_OFF = K_OFF + 2 * KQ_BYTES;                // [2][C][LDK] bf16
+  static constexpr size_t V_OFF = Q_OFF + 2 * KQ_BYTES;                // [2][C][LDV] bf16
+  static constexpr size_t G_OFF = V_OFF + 2 * V_BYTES;                 // [2][C][LDG] gates, then Gamma
+  static constexpr size_t A_OFF = G_OFF + 2 * G_BYTES;                 // [C][LDA] A (KDA)
+  static constexpr size_t P_OFF = tc_align128(A_OFF + size_t(C) * LDA * 4);   // [C][LDA] P
+  static constexpr size_t WC_OFF = tc_align128(P_OFF + size_t(C) * LDA * 4);  // W, K-major C x DK
+  static constexpr size_t QC_OFF = WC_OFF + size_t(C) * DK * 4;        // scaled queries, K-major C x DK
+  static constexpr size_t PC_OFF = QC_OFF + size_t(C) * DK * 4;        // P, K-major C x C
+  static constexpr size_t KC_OFF = PC_OFF + size_t(C) * C * 4;         // scaled keys^T, K-major DK x C
+  static constexpr size_t U_OFF = KC_OFF + size_t(DK) * C * 4;         // [C][LDU] U (KDA)
+  static constexpr size_t E_OFF = tc_align128(U_OFF + size_t(C) * LDU * 4);   // e^{G_end} [DK], u [DK], beta [C]
+  static constexpr size_t BAR_OFF = tc_align128(E_OFF + (2 * DK + C) * 4);
+  static constexpr size_t BYTES = BAR_OFF + 64;
+  static constexpr uint32_t TM_COLS = 256, TM_S = 0, TM_B = 128, TM_O = 160;
+};
+
+template <int OP>
+__global__ void __launch_bounds__(512, 1) key_chunk_prefill_tc_kernel(const PrefillArgs a) {
+  using G = KeyTcChunkGeom;
+  constexpr int C = G::C, DK = G::DK, DV = G::DV;
+  constexpr bool DELTA = OP == OP_KDA;
+  constexpr float LOG2E = 1.4426950408889634f;
+  static_assert(OP == OP_KDA || OP == OP_RWKV6, "per-key decay operators");
+  extern __shared__ __align__(128) unsigned char smem[];
+  auto kbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem + G::K_OFF + b * G::KQ_BYTES); };
+  auto qbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem + G::Q_OFF + b * G::KQ_BYTES); };
+  auto vbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem + G::V_OFF + b * G::V_BYTES); };
+  auto gbuf = [&](int b) { return reinterpret_cast<float*>(smem + G::G_OFF + b * G::G_BYTES); };
+  float* sA = reinterpret_cast<float*>(smem + G::A_OFF);
+  float* sP = reinterpret_cast<float*>(smem + G::P_OFF);
+  unsigned char* sWc = smem + G::WC_OFF;
+  unsigned char* sQc = smem + G::QC_OFF;
+  unsigned char* sPc = smem + G::PC_OFF;
+  unsigned char* sKc = smem + G::KC_OFF;
+  float* sU = reinterpret_cast<float*>(smem + G::U_OFF);
+  float* sE = reinterpret_cast<float*>(smem + G::E_OFF);
+  float* sBonus = sE + DK;
+  float* sBeta = sE + 2 * DK;
+  uint64_t* barB = reinterpret_cast<uint64_t*>(smem + G::BAR_OFF);
+  uint64_t* barO = barB + 1;
+  uint64_t* barS = barB + 2;
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(barB + 3);
+  volatile int* sAbort = reinterpret_cast<volatile int*>(sTmem + 1);
+  auto fp = [](unsigned char* base, uint32_t off) { return reinterpret_cast<float*>(base + off); };
+  float* sWt = reinterpret_cast<float*>(smem + G::QC_OFF);   // W row-major [C][DK + 4] during the solve
+  constexpr int LDW = DK + 4;
+  static_assert(size_t(C) * LDW * 4 <= G::KC_OFF - G::QC_OFF, "row-major W fits the Q and P operand space");
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int quarter = warp & 3, group = warp >> 2;
+  const int h = blockIdx.x;
+  const int r = blockIdx.y;
+
+  const int slot = a.slot_idx ? __ldg(a.slot_idx + r) : r;
+  if (slot < 0) return;
+  if (slot >= a.slots) {
+    if (tid == 0) atomicOr(a.err, kErrSlotIndex);
+    return;
+  }
+  const long t0 = __ldg(a.cu_seqlens + r), t1 = __ldg(a.cu_seqlens + r + 1);
+  if (t0 < 0 || t1 < t0 || t1 > a.total) {
+    if (tid == 0) atomicOr(a.err, kErrSeqlen);
+    return;
+  }
+  const long sh = static_cast<long>(slot) * a.H + h;
+  float* Sg = a.Sbar + sh * (DK * DV);
+
+  if (tid == 0) {
+    mbar_init(barB, 1);
+    mbar_init(barO, 1);
+    mbar_init(barS, 1);
+    fence_mbar_init();
+    *sAbort = 0;
+  }
+  if (OP == OP_RWKV6)
+    for (int j = tid; j < DK; j += G::NT) sBonus[j] = a.u[h * DK + j];
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(sTmem)),
+                 "r"(G::TM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sTmem;
+  const uint32_t lane_base = static_cast<uint32_t>(32 * quarter) << 16;
+  const int c_own = 32 * quarter + lane;
+  {
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = a.zero_state ? 0.f : __ldcs(Sg + (32 * group + i) * DV + c_own);
+    tmem_st32(tmem + lane_base + G::TM_S + 32 * group, v);
+    tmem_wait_st();
+  }
+
+  const __nv_bfloat16* Kg = static_cast<const __nv_bfloat16*>(a.k);
+  const __nv_bfloat16* Qg = static_cast<const __nv_bfloat16*>(a.q);
+  const __nv_bfloat16* Vg = static_cast<const __nv_bfloat16*>(a.v);
+  __nv_bfloat16* Og = static_cast<__nv_bfloat16*>(a.o);
+  const bool async_ok = aligned_to(a.q, 16) && aligned_to(a.k, 16) && aligned_to(a.v, 16) &&
+                        aligned_to(a.log_decay, 16);
+  auto stage_rows = [&](auto* dst, const auto* src, long c, int width, int ld) {
+    using T = typename std::remove_const<typename std::remove_pointer<decltype(src)>::type>::type;
+    constexpr int PER_SEG = 16 / static_cast<int>(sizeof(T));
+    const int nv = static_cast<int>(t1 - c < C ? t1 - c : C);
+    if (async_ok) {
+      const int seg_per_row = width / PER_SEG;
+      for (int idx = tid; idx < C * seg_per_row; idx += G::NT) {
+        const int t = idx / seg_per_row, seg = idx % seg_per_row;
+        const long row = ((c + (t < nv ? t : nv - 1)) * a.H + h) * width + PER_SEG * seg;
+        cp_async16(dst + t * ld + PER_SEG * seg, src + row, t < nv ? 16u : 0u);
+      }
+    } else {
+      for (int idx = tid; idx < C * width; idx += G::NT) {
+        const int t = idx / width, j = idx % width;
+        dst[t * ld + j] = t < nv ? src[((c + t) * a.H + h) * width + j] : T(0.f);
+      }
+    }
+  };
+  auto stage = [&](int b, long c) {
+    stage_rows(kbuf(b), Kg, c, DK, G::LDK);
+    stage_rows(qbuf(b), Qg, c, DK, G::LDK);
+    stage_rows(vbuf(b), Vg, c, DV, G::LDV);
+    stage_rows(gbuf(b), a.log_decay, c, DK, G::LDG);
+  };
+  float bnext = 0.f;
+  if (t0 < t1) {
+    stage(0, t0);
+    if (DELTA && tid < C && t0 + tid < t1) bnext = a.beta[(t0 + tid) * a.H + h];
+  }
+  cp_async_commit();
+  auto kmajor_rk = [](int e, int kt, int& rr, int& kk) {
+    const int core = e >> 5, within = e & 31;
+    rr = (core / (kt >> 2)) * 8 + (within >> 2);
+    kk = (core % (kt >> 2)) * 4 + (within & 3);
+  };
+
+  int buf = 0, ci = 0;
+  for (long c0 = t0; c0 < t1; c0 += C, buf ^= 1, ++ci) {
+    const int n = static_cast<int>(t1 - c0 < C ? t1 - c0 : C);
+    const bool has_next = c0 + C < t1;
+    const uint32_t par = static_cast<uint32_t>(ci & 1);
+    __syncthreads();   // the previous chunk is done with buffer buf ^ 1 and every work buffer
+    if (has_next) stage(buf ^ 1, c0 + C);
+    cp_async_commit();
+    if (DELTA && tid < C) {
+      sBeta[tid] = bnext;
+      bnext = has_next && c0 + C + tid < t1 ? a.beta[(c0 + C + tid) * a.H + h] : 0.f;
+    }
+    cp_async_wait<1>();   // this chunk's inputs have landed
+    __syncthreads();
+    const __nv_bfloat16 *sK = kbuf(buf), *sQ = qbuf(buf), *sV = vbuf(buf);
+    float* sG = gbuf(buf);
+
+    // 1. Gamma in log2 units, per key, in place; e^{Gamma_end}
+    for (int j = tid; j < DK; j += G::NT) {
+      float run = 0.f;
+#pragma unroll 4
+      for (int t = 0; t < C; ++t) {
+        run = fmaf(sG[t * G::LDG + j], LOG2E, run);
+        sG[t * G::LDG + j] = run;
+      }
+      sE[j] = ex2_approx(run);
+    }
+    __syncthreads();
+
+    // 2. A and P pair by pair; right-hand sides (KDA)
+    key_pair_phase<OP, DK, C, G::NT, G::LDK, G::LDG, G::LDA>(sK, sQ, sG, sBeta, sBonus, sA, sP);
+    for (int idx = tid; idx < C * C; idx += G::NT) {
+      const int t = idx / C, s = idx % C;
+      if (s > t) sP[t * G::LDA + s] = 0.f;
+      if (DELTA && s >= t) sA[t * G::LDA + s] = 0.f;
+    }
+    if (DELTA) {
+      for (int idx = tid; idx < C * DK / 4; idx += G::NT) {
+        const int t = idx / (DK / 4), j = 4 * (idx % (DK / 4));
+        const float4 g = *reinterpret_cast<const float4*>(sG + t * G::LDG + j);
+        float k4[4];
+        bf16x4_to_f32(sK + t * G::LDK + j, k4);
+        const float bt = sBeta[t];
+        *reinterpret_cast<float4*>(sWt + t * LDW + j) =
+            make_float4(bt * ex2_approx(g.x) * k4[0], bt * ex2_approx(g.y) * k4[1], bt * ex2_approx(g.z) * k4[2],
+                        bt * ex2_approx(g.w) * k4[3]);
+      }
+      for (int idx = tid; idx < C * DV / 4; idx += G::NT) {
+        const int t = idx / (DV / 4), c = 4 * (idx % (DV / 4));
+        float v4[4];
+        bf16x4_to_f32(sV + t * G::LDV + c, v4);
+        const float bt = sBeta[t];
+        *reinterpret_cast<float4*>(sU + t * G::LDU + c) = make_float4(bt * v4[0], bt * v4[1], bt * v4[2], bt * v4[3]);
+      }
+    }
+    __syncthreads();
+
+    if (DELTA) {
+      // 3. (I + A) X = R, one right-hand-side column per thread; W to its operand layout
+      if (tid < DK + DV) {
+        const bool isw = tid < DK;
+        float* col = isw ? sWt + tid : sU + (tid - DK);
+        const int ld = isw ? LDW : G::LDU;
+        float x[C];
+#pragma unroll
+        for (int t = 0; t < C; ++t) {
+          float acc0 = col[t * ld], acc1 = 0.f;
+          const float* arow = sA + t * G::LDA;
+#pragma unroll
+          for (int s = 0; s + 3 < t; s += 4) {
+            const float4 a4 = *reinterpret_cast<const float4*>(arow + s);
+            acc0 = fmaf(-a4.x, x[s], acc0);
+            acc1 = fmaf(-a4.y, x[s + 1], acc1);
+            acc0 = fmaf(-a4.z, x[s + 2], acc0);
+            acc1 = fmaf(-a4.w, x[s + 3], acc1);
+          }
+#pragma unroll
+          for (int s = t & ~3; s < t; ++s) acc0 = fmaf(-arow[s], x[s], acc0);
+          x[t] = acc0 + acc1;
+          col[t * ld] = x[t];
+        }
+      }
+      __syncthreads();
+      for (int e = tid; e < C * DK; e += G::NT) {
+        int t, j;
+        kmajor_rk(e, DK, t, j);
+        fp(sWc, 4 * e)[0] = wm::__float_to_tf32(sWt[t * LDW + j]);
+      }
+      fence_smem_to_async();
+    }
+
+    // 4. the previous chunk's state update must be complete (it reads B^T and
+    // the scaled keys, and writes S^T)
+    if (ci > 0 && !mbar_wait_abortable(barS, par ^ 1u, sAbort) && tid == 0) atomicOr(a.err, kErrWaitTimeout);
+    tc_fence_before();
+    __syncthreads();
+    if (*sAbort) break;
+    tc_fence_after();
+    if (DELTA) {
+      if (tid == 0) {   // W S
+        constexpr uint32_t ID = umma_idesc_tf32<128, C>();
+        const uint32_t w0 = smem_u32(sWc);
+#pragma unroll
+        for (int s = 0; s < DK / 8; ++s)
+          umma_tf32_ts(tmem + G::TM_B, tmem + G::TM_S + 8 * s, umma_desc(w0 + 256 * s, (DK / 4) * 128), ID, s > 0);
+        umma_commit(barB);
+      }
+    } else {
+      // B^T = V^T (bf16 values are tf32-exact), columns 8 group ..
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = __bfloat162float(sV[(8 * group + i) * G::LDV + c_own]);
+      tmem_st8(tmem + lane_base + G::TM_B + 8 * group, v);
+      tmem_wait_st();
+    }
+
+    // 5. P, the scaled queries and the scaled keys^T into their operand layouts
+    for (int e = tid; e < C * C; e += G::NT) {
+      int t, s;
+      kmajor_rk(e, C, t, s);
+      fp(sPc, 4 * e)[0] = sP[t * G::LDA + s];   // tf32-rounded, zero above the diagonal
+    }
+    for (int e = tid; e < C * DK; e += G::NT) {
+      int t, j;
+      kmajor_rk(e, DK, t, j);
+      const int tg = DELTA ? t : t - 1;   // Gamma_t (KDA), Gamma_{t-1} (RWKV6)
+      const float g = tg >= 0 ? sG[tg * G::LDG + j] : 0.f;
+      fp(sQc, 4 * e)[0] = wm::__float_to_tf32(ex2_approx(g) * __bfloat162float(sQ[t * G::LDK + j]));
+    }
+    for (int e = tid; e < DK * C; e += G::NT) {
+      int j, t;
+      kmajor_rk(e, C, j, t);
+      fp(sKc, 4 * e)[0] = wm::__float_to_tf32(ex2_approx(sG[(C - 1) * G::LDG + j] - sG[t * G::LDG + j]) *
+                                               __bfloat162float(sK[t * G::LDK + j]));
+    }
+    fence_smem_to_async();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {   // O^T = S^T (scaled Q)^T  (+ B^T P^T at once for RWKV6)
+      tc_fence_after();
+      constexpr uint32_t ID = umma_idesc_tf32<128, C>();
+      const uint32_t q0 = smem_u32(sQc);
+#pragma unroll
+      for (int s = 0; s < DK / 8; ++s)
+        umma_tf32_ts(tmem + G::TM_O, tmem + G::TM_S + 8 * s, umma_desc(q0 + 256 * s, (DK / 4) * 128), ID, s > 0);
+      if (!DELTA) {
+        const uint32_t p0 = smem_u32(sPc);
+#pragma unroll
+        for (int s = 0; s < C / 8; ++s)
+          umma_tf32_ts(tmem + G::TM_O, tmem + G::TM_B + 8 * s, umma_desc(p0 + 256 * s, (C / 4) * 128), ID, 1u);
+        umma_commit(barO);
+      }
+    }
+
+    if (DELTA) {
+      // 6. B^T = U^T - (W S)^T, tf32-rounded, then O^T += B^T P^T
+      if (!mbar_wait_abortable(barB, par, sAbort) && tid == 0) atomicOr(a.err, kErrWaitTimeout);
+      tc_fence_after();
+      if (!*sAbort) {
+        float v[8];
+        const uint32_t ta = tmem + lane_base + G::TM_B + 8 * group;
+        tmem_ld8(ta, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = wm::__float_to_tf32(sU[(8 * group + i) * G::LDU + c_own] - v[i]);
+        tmem_st8(ta, v);
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncthreads();
+      if (*sAbort) break;
+      if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t ID = umma_idesc_tf32<128, C>();
+        const uint32_t p0 = smem_u32(sPc);
+#pragma unroll
+        for (int s = 0; s < C / 8; ++s)
+          umma_tf32_ts(tmem + G::TM_O, tmem + G::TM_B + 8 * s, umma_desc(p0 + 256 * s, (C / 4) * 128), ID, 1u);
+        umma_commit(barO);
+      }
+    }
+
+    // 7. O rows < n to global; S^T columns scaled by e^{Gamma_end}; S^T += B^T (scaled K)
+    if (!mbar_wait_abortable(barO, par, sAbort) && tid == 0) atomicOr(a.err, kErrWaitTimeout);
+    tc_fence_after();
+    if (!*sAbort) {
+      float v[8];
+      tmem_ld8(tmem + lane_base + G::TM_O + 8 * group, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int t = 8 * group + i;
+        if (t < n) Og[((c0 + t) * a.H + h) * DV + c_own] = __float2bfloat16_rn(v[i]);
+      }
+      float sv[32];
+      const uint32_t ts = tmem + lane_base + G::TM_S + 32 * group;
+      tmem_ld32(ts, sv);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) sv[i] *= sE[32 * group + i];
+      tmem_st32(ts, sv);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*sAbort) break;
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t ID = umma_idesc_tf32<128, DK>();
+      const uint32_t k0 = smem_u32(sKc);
+#pragma unroll
+      for (int s = 0; s < C / 8; ++s)
+        umma_tf32_ts(tmem + G::TM_S, tmem + G::TM_B + 8 * s, umma_desc(k0 + 256 * s, (C / 4) * 128), ID, 1u);
+      umma_commit(barS);
+    }
+  }
+
+  if (ci > 0 && !*sAbort && !mbar_wait_abortable(barS, static_cast<uint32_t>((ci - 1) & 1), sAbort) && tid == 0)
+    atomicOr(a.err, kErrWaitTimeout);
+  cp_async_wait<0>();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const bool ok = !*sAbort;
+  if (ok) {
+    float v[32];
+    tmem_ld32(tmem + lane_base + G::TM_S + 32 * group, v);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) __stcs(Sg + (32 * group + i) * DV + c_own, v[i]);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(G::TM_COLS) : "memory");
+  }
+  if (ok) clear_log_tile<OP, DK, DV, __nv_bfloat16>(a, sh, 0, DV);
+}
+
+// Grid (H, rows), 512 threads, KeyTcChunkGeom::BYTES of dynamic shared memory;
+// d_k = d_v = 128, bf16 inputs.  Instantiated in prefill.cu.
+template <int OP>
+cudaError_t launch_key_chunk_prefill_tc(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st);
 
 }  // namespace dl

@@ -97,9 +97,7 @@ def _prefill_then_decode(op, dims, dtype, kernel, H):
     o = h.prefill(*_prefill_args(op, d), cu_seqlens=torch.from_numpy(cu).cuda(),
                   slot_idx=torch.tensor(slots, dtype=torch.int32, device="cuda"), zero_state=True)
     assert h.log_len == 2                                # the handle's cycle is unchanged
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
-    auto_chunked = (dtype == torch.bfloat16 and sum(lens) >= 64 * rows       # the automatic rule
-                    and (op != "kda" or rows * H * (dv // 16) < 16 * sms))
+    auto_chunked = dtype == torch.bfloat16 and sum(lens) >= 64 * rows   # the automatic rule
     want = "chunked" if kernel == "chunked" or (kernel == "auto" and auto_chunked) else "recurrent"
     assert h.last_prefill_kernel == want
     got = o.float().cpu().numpy()
@@ -233,13 +231,14 @@ def test_chunked_prefill_refused_where_it_does_not_apply():
 
 
 @pytest.mark.parametrize("op,kernel", [(op, k) for op in OPS for k in ("recurrent", "chunked")])
-@pytest.mark.parametrize("d", [64, 128])
-def test_prefill_strong_decay(op, kernel, d):
+@pytest.mark.parametrize("d,H", [(64, 2), (128, 2), (128, 48)])
+def test_prefill_strong_decay(op, kernel, d, H):
     """Log-decays of -40 per token (on three keys for KDA/RWKV6, on every
     tenth token for GDN): cumulative decays far past fp32 range inside a
-    chunk, which no kernel may divide by."""
+    chunk, which no kernel may divide by.  H = 48 makes the chunked kernels
+    take whole-head tiles."""
     from recurrent_state_update_deltalog_b200 import DeltaLog
-    dtype, H, lens = torch.bfloat16, 2, [100, 37]
+    dtype, lens = torch.bfloat16, [100, 37]
     rows = len(lens)
     seq = sequence(51, op, rows, H, d, d, max(lens), bf16=True)
     seq["log_decay"] = seq["log_decay"].copy()
