@@ -251,12 +251,11 @@ int dl_read_state(dl_t h, float* S_out, void* stream);
  *   DL_PREFILL_CHUNKED: the chunk form on tensor cores (bf16-input handles
  *     only, DL_ERR_UNSUPPORTED otherwise): 32-token chunks, the WY form of
  *     the delta rule for GDN and KDA, per-key pair weights of KDA and RWKV6
- *     formed exactly on the SIMT lanes.  At d_k = d_v = 128, once rows x H
- *     reach half the SM count, each CTA keeps a whole head's state in tensor
- *     memory and runs the products with it as tcgen05 MMAs; otherwise
- *     64-column tiles (16-token chunks for per-key decay at d_k = 128) use
- *     warp-level MMAs.  The products with the state are tf32, inside the
- *     bf16-input tolerance. */
+ *     formed exactly on the SIMT lanes.  At d_k = d_v = 128 each CTA keeps
+ *     a whole head's state in tensor memory and runs the products with it as
+ *     tcgen05 MMAs; other shapes use 64-column tiles and warp-level MMAs.
+ *     The products with the state are tf32, inside the bf16-input
+ *     tolerance. */
 enum dl_option {
   DL_OPT_STEP_KERNEL = 0,
   DL_OPT_HOST_PREFETCH = 1,

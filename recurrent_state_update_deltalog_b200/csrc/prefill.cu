@@ -18,12 +18,6 @@ cudaError_t launch_prefill_op(const LaunchShape& s, const PrefillArgs& a, cudaSt
   DL_DISPATCH_DIMS(prefill_dims, s, a, st);
 }
 
-// Whole-head CTAs (VT = 128) for d_k = d_v = 128 once they cover at least
-// half the SMs (rows x heads), 64-column tiles below that.  Measured on B200
-// for the KDA kernel (H=32): whole-head CTAs 1.18x at B=64 L=512, 1.21x at
-// B=4 L=4096, but 0.83x at B=1 L=8192 (32 CTAs).
-inline bool whole_head_tiles(const LaunchShape& s) { return 2LL * s.units * s.H > s.sms; }
-
 template <int DK, int DV, int VT>
 cudaError_t launch_gdn_chunk_prefill(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st) {
   using G = ChunkGeom<DK, VT>;
@@ -47,9 +41,11 @@ cudaError_t launch_gdn_chunk_prefill_tc(const LaunchShape& s, const PrefillArgs&
 
 cudaError_t launch_gdn_chunk_prefill_dims(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st) {
   if (s.dk == 64 && s.dv == 64) return launch_gdn_chunk_prefill<64, 64, 64>(s, a, st);
-  if (s.dk == 128 && s.dv == 128)
-    return whole_head_tiles(s) ? launch_gdn_chunk_prefill_tc(s, a, st)
-                               : launch_gdn_chunk_prefill<128, 128, 64>(s, a, st);
+  // d_k = d_v = 128: whole heads with the state in tensor memory.  Measured on
+  // B200 against the warp-MMA kernel (64-column tiles, or 512-thread whole-head
+  // tiles), H = 32: 2.06x at B=64 L=512 and B=4 L=4096, and 1.55x at B=1 where
+  // it launches half the CTAs.
+  if (s.dk == 128 && s.dv == 128) return launch_gdn_chunk_prefill_tc(s, a, st);
   if (s.dk == 64 && s.dv == 128) return launch_gdn_chunk_prefill<64, 128, 64>(s, a, st);
   if (s.dk == 128 && s.dv == 64) return launch_gdn_chunk_prefill<128, 64, 64>(s, a, st);
   return cudaErrorInvalidValue;
@@ -80,9 +76,9 @@ cudaError_t launch_key_chunk_prefill_tc(const LaunchShape& s, const PrefillArgs&
 template <int OP>
 cudaError_t launch_key_chunk_prefill_dims(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st) {
   if (s.dk == 64 && s.dv == 64) return launch_key_chunk_prefill<OP, 64, 64, 64>(s, a, st);
-  if (s.dk == 128 && s.dv == 128)
-    return whole_head_tiles(s) ? launch_key_chunk_prefill_tc<OP>(s, a, st)
-                               : launch_key_chunk_prefill<OP, 128, 128, 64>(s, a, st);
+  // d_k = d_v = 128: whole heads with the state in tensor memory (KDA, H = 32:
+  // 1.68x the warp-MMA kernel at B=64 L=512, 1.40x at B=1 L=8192)
+  if (s.dk == 128 && s.dv == 128) return launch_key_chunk_prefill_tc<OP>(s, a, st);
   if (s.dk == 64 && s.dv == 128) return launch_key_chunk_prefill<OP, 64, 128, 64>(s, a, st);
   if (s.dk == 128 && s.dv == 64) return launch_key_chunk_prefill<OP, 128, 64, 64>(s, a, st);
   return cudaErrorInvalidValue;

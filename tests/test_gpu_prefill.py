@@ -61,9 +61,9 @@ def test_prefill_then_decode(op, dims, dtype, kernel):
 
 
 @pytest.mark.parametrize("op", OPS)
-def test_prefill_then_decode_whole_head_tiles(op):
-    """The same with 5 rows x 16 heads at d_k = d_v = 128: enough CTAs that the
-    chunked kernels take whole-head tiles (rows x heads above half the SMs)."""
+def test_prefill_then_decode_many_heads(op):
+    """The same with 5 rows x 16 heads at d_k = d_v = 128 (80 whole-head CTAs
+    of the tensor-memory kernels)."""
     _prefill_then_decode(op, (128, 128), torch.bfloat16, "chunked", H=16)
 
 
@@ -235,8 +235,7 @@ def test_chunked_prefill_refused_where_it_does_not_apply():
 def test_prefill_strong_decay(op, kernel, d, H):
     """Log-decays of -40 per token (on three keys for KDA/RWKV6, on every
     tenth token for GDN): cumulative decays far past fp32 range inside a
-    chunk, which no kernel may divide by.  H = 48 makes the chunked kernels
-    take whole-head tiles."""
+    chunk, which no kernel may divide by."""
     from recurrent_state_update_deltalog_b200 import DeltaLog
     dtype, lens = torch.bfloat16, [100, 37]
     rows = len(lens)
