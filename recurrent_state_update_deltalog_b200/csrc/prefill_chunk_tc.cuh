@@ -122,10 +122,15 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 
 constexpr size_t tc_align128(size_t x) { return (x + 127) & ~size_t(127); }
 
+template <int NT_>
 struct TcChunkGeom {
   static constexpr int DK = 128, DV = 128;   // a whole head per CTA
   static constexpr int C = 32;               // tokens per chunk
-  static constexpr int NT = 512, NW = 16;    // threads, warps (four per TMEM lane quarter)
+  // 256 threads (two CTAs per SM) or 512 (one CTA per SM, for launches with
+  // fewer CTAs than SMs)
+  static constexpr int NT = NT_, NW = NT / 32;
+  static constexpr int NG = NW / 4;          // column groups of the TMEM epilogues
+  static constexpr int MINB = NT == 256 ? 2 : 1;
   static constexpr int LDK = DK + 8;         // bf16 row stride of K and Q
   static constexpr int LDV = DV + 8;         // bf16 row stride of V
   static constexpr int LDA = C + 4;          // fp32 row stride of A and P (WMMA outputs)
@@ -133,8 +138,8 @@ struct TcChunkGeom {
   static constexpr size_t KQ_BYTES = tc_align128(size_t(C) * LDK * 2), V_BYTES = tc_align128(size_t(C) * LDV * 2);
   static constexpr size_t K_OFF = 0;                                  // [2][C][LDK] bf16
   static constexpr size_t Q_OFF = K_OFF + 2 * KQ_BYTES;               // [C][LDK] bf16
-  static constexpr size_t V_OFF = Q_OFF + KQ_BYTES;                   // [2][C][LDV] bf16
-  static constexpr size_t A_OFF = V_OFF + 2 * V_BYTES;                // [C][LDA] fp32
+  static constexpr size_t V_OFF = Q_OFF + KQ_BYTES;                   // [C][LDV] bf16
+  static constexpr size_t A_OFF = V_OFF + V_BYTES;                    // [C][LDA] fp32
   static constexpr size_t WC_OFF = tc_align128(A_OFF + size_t(C) * LDA * 4);   // W, K-major C x DK
   static constexpr size_t QC_OFF = WC_OFF + size_t(C) * DK * 4;       // e^G Q, K-major C x DK
   static constexpr size_t PC_OFF = QC_OFF + size_t(C) * DK * 4;       // P, K-major C x C
@@ -150,14 +155,14 @@ struct TcChunkGeom {
   static constexpr uint32_t TM_O = 160;      // O^T: C columns
 };
 
-template <int DUMMY = 0>
-__global__ void __launch_bounds__(512, 1) gdn_chunk_prefill_tc_kernel(const PrefillArgs a) {
-  using G = TcChunkGeom;
+template <int NT_>
+__global__ void __launch_bounds__(NT_, TcChunkGeom<NT_>::MINB) gdn_chunk_prefill_tc_kernel(const PrefillArgs a) {
+  using G = TcChunkGeom<NT_>;
   constexpr int C = G::C, DK = G::DK, DV = G::DV;
   extern __shared__ __align__(128) unsigned char smem[];
   auto kbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem + G::K_OFF + b * G::KQ_BYTES); };
   __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem + G::Q_OFF);
-  auto vbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem + G::V_OFF + b * G::V_BYTES); };
+  __nv_bfloat16* sV = reinterpret_cast<__nv_bfloat16*>(smem + G::V_OFF);
   float* sA = reinterpret_cast<float*>(smem + G::A_OFF);
   unsigned char* sWc = smem + G::WC_OFF;
   unsigned char* sQc = smem + G::QC_OFF;
@@ -178,6 +183,7 @@ __global__ void __launch_bounds__(512, 1) gdn_chunk_prefill_tc_kernel(const Pref
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int quarter = warp & 3, group = warp >> 2;   // TMEM lanes 32 quarter .., column group
+  constexpr int NG = G::NG;
   const int h = blockIdx.x;
   const int r = blockIdx.y;
 
@@ -215,14 +221,14 @@ __global__ void __launch_bounds__(512, 1) gdn_chunk_prefill_tc_kernel(const Pref
   const uint32_t lane_base = static_cast<uint32_t>(32 * quarter) << 16;
   const int c_own = 32 * quarter + lane;   // this thread's value column in TMEM epilogues
 
-  // S^T into tensor memory: this warp's 32 lanes (value columns), keys 32 group ..
-  {
+  // S^T into tensor memory: this warp's 32 lanes (value columns), key blocks 32 cb ..
+  for (int cb = group; cb < DK / 32; cb += NG) {
     float v[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = a.zero_state ? 0.f : __ldcs(Sg + (32 * group + i) * DV + c_own);
-    tmem_st32(tmem + lane_base + G::TM_S + 32 * group, v);
-    tmem_wait_st();
+    for (int i = 0; i < 32; ++i) v[i] = a.zero_state ? 0.f : __ldcs(Sg + (32 * cb + i) * DV + c_own);
+    tmem_st32(tmem + lane_base + G::TM_S + 32 * cb, v);
   }
+  tmem_wait_st();
 
   const __nv_bfloat16* Kg = static_cast<const __nv_bfloat16*>(a.k);
   const __nv_bfloat16* Qg = static_cast<const __nv_bfloat16*>(a.q);
@@ -249,20 +255,22 @@ __global__ void __launch_bounds__(512, 1) gdn_chunk_prefill_tc_kernel(const Pref
       }
     }
   };
-  auto stage_kv = [&](int b, long c) {
-    stage_rows(kbuf(b), Kg, c, DK, G::LDK);
-    stage_rows(vbuf(b), Vg, c, DV, G::LDV);
-  };
+
   float gn = 0.f, bnv = 0.f;   // warp 0, lane t: gate and beta of row t of the next chunk
   auto fetch_gates = [&](long c) {
     const int nv = static_cast<int>(t1 - c < C ? t1 - c : C);
     gn = lane < nv ? a.log_decay[(c + lane) * a.H + h] : 0.f;
     bnv = lane < nv ? a.beta[(c + lane) * a.H + h] : 0.f;
   };
+  // Copy groups, in commit order: K and V of chunk 0; then per chunk c: Q of c
+  // and K of c + 1 at its start, V of c + 1 once V of c has been consumed
+  // (V is single-buffered).  Groups may be empty.
   if (t0 < t1) {
-    stage_kv(0, t0);
+    stage_rows(kbuf(0), Kg, t0, DK, G::LDK);
     if (warp == 0) fetch_gates(t0);
   }
+  cp_async_commit();
+  if (t0 < t1) stage_rows(sV, Vg, t0, DV, G::LDV);
   cp_async_commit();
 
   // (r, k) of element e of a K-major operand with kt columns, enumerated in
@@ -284,10 +292,10 @@ __global__ void __launch_bounds__(512, 1) gdn_chunk_prefill_tc_kernel(const Pref
     __syncthreads();   // the previous chunk is done with every buffer
     stage_rows(sQ, Qg, c0, DK, G::LDK);
     cp_async_commit();
-    if (has_next) stage_kv(buf ^ 1, c0 + C);
+    if (has_next) stage_rows(kbuf(buf ^ 1), Kg, c0 + C, DK, G::LDK);
     cp_async_commit();
-    cp_async_wait<2>();   // K/V of this chunk have landed
-    __nv_bfloat16 *sK = kbuf(buf), *sV = vbuf(buf);
+    cp_async_wait<2>();   // K and V of this chunk have landed
+    __nv_bfloat16* sK = kbuf(buf);
 
     // 1. Gamma (inclusive prefix of the log-gates), beta and per-row factors
     if (warp == 0) {
@@ -325,6 +333,8 @@ __global__ void __launch_bounds__(512, 1) gdn_chunk_prefill_tc_kernel(const Pref
       sU[t * G::LDU + c] = sBeta[t] * __bfloat162float(sV[t * G::LDV + c]);
     }
     __syncthreads();
+    if (has_next) stage_rows(sV, Vg, c0 + C, DV, G::LDV);   // V of this chunk is consumed
+    cp_async_commit();
 
     // 3. (I + A) X = R, one right-hand-side column per thread
     if (tid < DK + DV) {
@@ -375,7 +385,7 @@ __global__ void __launch_bounds__(512, 1) gdn_chunk_prefill_tc_kernel(const Pref
     }
 
     // 5. P = Q K^T (.) [e^{G_t - G_s}]_{s <= t}, e^G Q and (e^{G_end - G} K)^T as operands
-    cp_async_wait<1>();   // Q of this chunk has landed
+    cp_async_wait<2>();   // Q of this chunk has landed (K and V of the next may be in flight)
     __syncthreads();
     lower_xyt<C, DK, G::LDK, G::LDA>(sQ, sK, sA);
     __syncthreads();
@@ -409,12 +419,14 @@ __global__ void __launch_bounds__(512, 1) gdn_chunk_prefill_tc_kernel(const Pref
     if (!mbar_wait_abortable(barB, par, sAbort) && tid == 0) atomicOr(a.err, kErrWaitTimeout);
     tc_fence_after();
     if (!*sAbort) {
-      float v[8];
-      const uint32_t ta = tmem + lane_base + G::TM_B + 8 * group;
-      tmem_ld8(ta, v);
+      for (int b8 = group; b8 < C / 8; b8 += NG) {
+        float v[8];
+        const uint32_t ta = tmem + lane_base + G::TM_B + 8 * b8;
+        tmem_ld8(ta, v);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = wm::__float_to_tf32(sU[(8 * group + i) * G::LDU + c_own] - v[i]);
-      tmem_st8(ta, v);
+        for (int i = 0; i < 8; ++i) v[i] = wm::__float_to_tf32(sU[(8 * b8 + i) * G::LDU + c_own] - v[i]);
+        tmem_st8(ta, v);
+      }
       tmem_wait_st();
     }
     tc_fence_before();
@@ -434,20 +446,24 @@ __global__ void __launch_bounds__(512, 1) gdn_chunk_prefill_tc_kernel(const Pref
     if (!mbar_wait_abortable(barO, par, sAbort) && tid == 0) atomicOr(a.err, kErrWaitTimeout);
     tc_fence_after();
     if (!*sAbort) {
-      float v[8];
-      tmem_ld8(tmem + lane_base + G::TM_O + 8 * group, v);
+      for (int b8 = group; b8 < C / 8; b8 += NG) {
+        float v[8];
+        tmem_ld8(tmem + lane_base + G::TM_O + 8 * b8, v);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int t = 8 * group + i;
-        if (t < n) Og[((c0 + t) * a.H + h) * DV + c_own] = __float2bfloat16_rn(v[i]);
+        for (int i = 0; i < 8; ++i) {
+          const int t = 8 * b8 + i;
+          if (t < n) Og[((c0 + t) * a.H + h) * DV + c_own] = __float2bfloat16_rn(v[i]);
+        }
       }
       const float dend = sEG[n - 1];
-      float sv[32];
-      const uint32_t ts = tmem + lane_base + G::TM_S + 32 * group;
-      tmem_ld32(ts, sv);
+      for (int cb = group; cb < DK / 32; cb += NG) {
+        float sv[32];
+        const uint32_t ts = tmem + lane_base + G::TM_S + 32 * cb;
+        tmem_ld32(ts, sv);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) sv[i] *= dend;
-      tmem_st32(ts, sv);
+        for (int i = 0; i < 32; ++i) sv[i] *= dend;
+        tmem_st32(ts, sv);
+      }
       tmem_wait_st();
     }
     tc_fence_before();
@@ -473,10 +489,12 @@ __global__ void __launch_bounds__(512, 1) gdn_chunk_prefill_tc_kernel(const Pref
   tc_fence_after();
   const bool ok = !*sAbort;
   if (ok) {
-    float v[32];
-    tmem_ld32(tmem + lane_base + G::TM_S + 32 * group, v);
+    for (int cb = group; cb < DK / 32; cb += NG) {
+      float v[32];
+      tmem_ld32(tmem + lane_base + G::TM_S + 32 * cb, v);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) __stcs(Sg + (32 * group + i) * DV + c_own, v[i]);
+      for (int i = 0; i < 32; ++i) __stcs(Sg + (32 * cb + i) * DV + c_own, v[i]);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -487,7 +505,8 @@ __global__ void __launch_bounds__(512, 1) gdn_chunk_prefill_tc_kernel(const Pref
   if (ok) clear_log_tile<OP_GDN, DK, DV, __nv_bfloat16>(a, sh, 0, DV);
 }
 
-// Grid (H, rows), 512 threads, TcChunkGeom::BYTES of dynamic shared memory;
+// Grid (H, rows), 256 threads (two CTAs per SM) once the launch has more CTAs
+// than SMs, else 512; TcChunkGeom<NT>::BYTES of dynamic shared memory;
 // d_k = d_v = 128, bf16 inputs.  Instantiated in prefill.cu.
 cudaError_t launch_gdn_chunk_prefill_tc(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st);
 
