@@ -72,15 +72,22 @@ cudaError_t launch_key_chunk_prefill(const LaunchShape& s, const PrefillArgs& a,
   return cudaGetLastError();
 }
 
-template <int OP>
-cudaError_t launch_key_chunk_prefill_tc(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st) {
-  using G = KeyTcChunkGeom;
-  auto kern = key_chunk_prefill_tc_kernel<OP>;
+template <int OP, int NT>
+cudaError_t launch_key_chunk_prefill_tc_nt(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st) {
+  using G = KeyTcChunkGeom<NT>;
+  auto kern = key_chunk_prefill_tc_kernel<OP, NT>;
   if (G::BYTES + 1024 > static_cast<size_t>(s.smem_block_optin)) return cudaErrorNotSupported;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(G::BYTES));
   if (e != cudaSuccess) return e;
   kern<<<dim3(s.H, s.units), G::NT, G::BYTES, st>>>(a);
   return cudaGetLastError();
+}
+
+// Two 256-thread CTAs per SM once the launch has more CTAs than SMs, as for GDN.
+template <int OP>
+cudaError_t launch_key_chunk_prefill_tc(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st) {
+  return static_cast<long long>(s.units) * s.H > s.sms ? launch_key_chunk_prefill_tc_nt<OP, 256>(s, a, st)
+                                                        : launch_key_chunk_prefill_tc_nt<OP, 512>(s, a, st);
 }
 
 template <int OP>

@@ -518,47 +518,54 @@ cudaError_t launch_gdn_chunk_prefill_tc(const LaunchShape& s, const PrefillArgs&
 // V^T, written straight into tensor memory.  The per-key decay of the state
 // update scales the columns of S^T.
 
+template <int NT_>
 struct KeyTcChunkGeom {
-  static constexpr int DK = 128, DV = 128, C = 32, NT = 512, NW = 16;
-  static constexpr int LDK = DK + 8, LDV = DV + 8, LDG = DK + 4, LDA = C + 4, LDU = DV + 4;
+  // 256 threads (two CTAs per SM) or 512 (one per SM, for launches with
+  // fewer CTAs than SMs)
+  static constexpr int DK = 128, DV = 128, C = 32, NT = NT_, NW = NT / 32;
+  static constexpr int NG = NW / 4;                 // column groups of the TMEM epilogues
+  static constexpr int MINB = NT == 256 ? 2 : 1;
+  static constexpr int LDK = DK + 8, LDV = DV + 8, LDG = DK + 4, LDA = C + 4;
   static constexpr size_t KQ_BYTES = tc_align128(size_t(C) * LDK * 2), V_BYTES = tc_align128(size_t(C) * LDV * 2);
   static constexpr size_t G_BYTES = tc_align128(size_t(C) * LDG * 4);
-  static constexpr size_t K_OFF = 0;                                   // [2][C][LDK] bf16
-  static constexpr size_t Q_OFF = K_OFF + 2 * KQ_BYTES;                // [2][C][LDK] bf16
-  static constexpr size_t V_OFF = Q_OFF + 2 * KQ_BYTES;                // [2][C][LDV] bf16
-  static constexpr size_t G_OFF = V_OFF + 2 * V_BYTES;                 // [2][C][LDG] gates, then Gamma
-  static constexpr size_t A_OFF = G_OFF + 2 * G_BYTES;                 // [C][LDA] A (KDA)
+  // single-buffered inputs: the next chunk's V streams in once the solve has
+  // consumed V, its K, Q and gates once the operands have been built
+  static constexpr size_t K_OFF = 0;                                   // [C][LDK] bf16
+  static constexpr size_t Q_OFF = K_OFF + KQ_BYTES;                    // [C][LDK] bf16
+  static constexpr size_t V_OFF = Q_OFF + KQ_BYTES;                    // [C][LDV] bf16
+  static constexpr size_t G_OFF = V_OFF + V_BYTES;                     // [C][LDG] gates, then Gamma
+  static constexpr size_t A_OFF = G_OFF + G_BYTES;                     // [C][LDA] A (KDA)
   static constexpr size_t P_OFF = tc_align128(A_OFF + size_t(C) * LDA * 4);   // [C][LDA] P
   static constexpr size_t WC_OFF = tc_align128(P_OFF + size_t(C) * LDA * 4);  // W, K-major C x DK
   static constexpr size_t QC_OFF = WC_OFF + size_t(C) * DK * 4;        // scaled queries, K-major C x DK
   static constexpr size_t PC_OFF = QC_OFF + size_t(C) * DK * 4;        // P, K-major C x C
   static constexpr size_t KC_OFF = PC_OFF + size_t(C) * C * 4;         // scaled keys^T, K-major DK x C
-  static constexpr size_t U_OFF = KC_OFF + size_t(DK) * C * 4;         // [C][LDU] U (KDA)
-  static constexpr size_t E_OFF = tc_align128(U_OFF + size_t(C) * LDU * 4);   // e^{G_end} [DK], u [DK], beta [C]
+  static constexpr size_t E_OFF = tc_align128(KC_OFF + size_t(DK) * C * 4);  // e^{G_end} [DK], u [DK], beta [C]
   static constexpr size_t BAR_OFF = tc_align128(E_OFF + (2 * DK + C) * 4);
   static constexpr size_t BYTES = BAR_OFF + 64;
-  static constexpr uint32_t TM_COLS = 256, TM_S = 0, TM_B = 128, TM_O = 160;
+  // tensor-memory columns: S^T, W S then B^T, O^T, U^T (KDA; the solve writes it)
+  static constexpr uint32_t TM_COLS = 256, TM_S = 0, TM_B = 128, TM_O = 160, TM_U = 192;
 };
 
-template <int OP>
-__global__ void __launch_bounds__(512, 1) key_chunk_prefill_tc_kernel(const PrefillArgs a) {
-  using G = KeyTcChunkGeom;
+template <int OP, int NT_>
+__global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_>::MINB) key_chunk_prefill_tc_kernel(const PrefillArgs a) {
+  using G = KeyTcChunkGeom<NT_>;
+  constexpr int NG = G::NG;
   constexpr int C = G::C, DK = G::DK, DV = G::DV;
   constexpr bool DELTA = OP == OP_KDA;
   constexpr float LOG2E = 1.4426950408889634f;
   static_assert(OP == OP_KDA || OP == OP_RWKV6, "per-key decay operators");
   extern __shared__ __align__(128) unsigned char smem[];
-  auto kbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem + G::K_OFF + b * G::KQ_BYTES); };
-  auto qbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem + G::Q_OFF + b * G::KQ_BYTES); };
-  auto vbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem + G::V_OFF + b * G::V_BYTES); };
-  auto gbuf = [&](int b) { return reinterpret_cast<float*>(smem + G::G_OFF + b * G::G_BYTES); };
+  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem + G::K_OFF);
+  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem + G::Q_OFF);
+  __nv_bfloat16* sV = reinterpret_cast<__nv_bfloat16*>(smem + G::V_OFF);
+  float* sG = reinterpret_cast<float*>(smem + G::G_OFF);
   float* sA = reinterpret_cast<float*>(smem + G::A_OFF);
   float* sP = reinterpret_cast<float*>(smem + G::P_OFF);
   unsigned char* sWc = smem + G::WC_OFF;
   unsigned char* sQc = smem + G::QC_OFF;
   unsigned char* sPc = smem + G::PC_OFF;
   unsigned char* sKc = smem + G::KC_OFF;
-  float* sU = reinterpret_cast<float*>(smem + G::U_OFF);
   float* sE = reinterpret_cast<float*>(smem + G::E_OFF);
   float* sBonus = sE + DK;
   float* sBeta = sE + 2 * DK;
@@ -612,13 +619,13 @@ __global__ void __launch_bounds__(512, 1) key_chunk_prefill_tc_kernel(const Pref
   const uint32_t tmem = *sTmem;
   const uint32_t lane_base = static_cast<uint32_t>(32 * quarter) << 16;
   const int c_own = 32 * quarter + lane;
-  {
+  for (int cb = group; cb < DK / 32; cb += NG) {
     float v[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = a.zero_state ? 0.f : __ldcs(Sg + (32 * group + i) * DV + c_own);
-    tmem_st32(tmem + lane_base + G::TM_S + 32 * group, v);
-    tmem_wait_st();
+    for (int i = 0; i < 32; ++i) v[i] = a.zero_state ? 0.f : __ldcs(Sg + (32 * cb + i) * DV + c_own);
+    tmem_st32(tmem + lane_base + G::TM_S + 32 * cb, v);
   }
+  tmem_wait_st();
 
   const __nv_bfloat16* Kg = static_cast<const __nv_bfloat16*>(a.k);
   const __nv_bfloat16* Qg = static_cast<const __nv_bfloat16*>(a.q);
@@ -644,15 +651,15 @@ __global__ void __launch_bounds__(512, 1) key_chunk_prefill_tc_kernel(const Pref
       }
     }
   };
-  auto stage = [&](int b, long c) {
-    stage_rows(kbuf(b), Kg, c, DK, G::LDK);
-    stage_rows(qbuf(b), Qg, c, DK, G::LDK);
-    stage_rows(vbuf(b), Vg, c, DV, G::LDV);
-    stage_rows(gbuf(b), a.log_decay, c, DK, G::LDG);
+  auto stage_kqg = [&](long c) {
+    stage_rows(sK, Kg, c, DK, G::LDK);
+    stage_rows(sQ, Qg, c, DK, G::LDK);
+    stage_rows(sG, a.log_decay, c, DK, G::LDG);
   };
   float bnext = 0.f;
   if (t0 < t1) {
-    stage(0, t0);
+    stage_kqg(t0);
+    stage_rows(sV, Vg, t0, DV, G::LDV);
     if (DELTA && tid < C && t0 + tid < t1) bnext = a.beta[(t0 + tid) * a.H + h];
   }
   cp_async_commit();
@@ -662,22 +669,18 @@ __global__ void __launch_bounds__(512, 1) key_chunk_prefill_tc_kernel(const Pref
     kk = (core % (kt >> 2)) * 4 + (within & 3);
   };
 
-  int buf = 0, ci = 0;
-  for (long c0 = t0; c0 < t1; c0 += C, buf ^= 1, ++ci) {
+  int ci = 0;
+  for (long c0 = t0; c0 < t1; c0 += C, ++ci) {
     const int n = static_cast<int>(t1 - c0 < C ? t1 - c0 : C);
     const bool has_next = c0 + C < t1;
     const uint32_t par = static_cast<uint32_t>(ci & 1);
-    __syncthreads();   // the previous chunk is done with buffer buf ^ 1 and every work buffer
-    if (has_next) stage(buf ^ 1, c0 + C);
-    cp_async_commit();
+    __syncthreads();   // the previous chunk is done with every work buffer
     if (DELTA && tid < C) {
       sBeta[tid] = bnext;
       bnext = has_next && c0 + C + tid < t1 ? a.beta[(c0 + C + tid) * a.H + h] : 0.f;
     }
-    cp_async_wait<1>();   // this chunk's inputs have landed
+    cp_async_wait<0>();   // this chunk's inputs have landed
     __syncthreads();
-    const __nv_bfloat16 *sK = kbuf(buf), *sQ = qbuf(buf), *sV = vbuf(buf);
-    float* sG = gbuf(buf);
 
     // 1. Gamma in log2 units, per key, in place; e^{Gamma_end}
     for (int j = tid; j < DK; j += G::NT) {
@@ -709,26 +712,21 @@ __global__ void __launch_bounds__(512, 1) key_chunk_prefill_tc_kernel(const Pref
             make_float4(bt * ex2_approx(g.x) * k4[0], bt * ex2_approx(g.y) * k4[1], bt * ex2_approx(g.z) * k4[2],
                         bt * ex2_approx(g.w) * k4[3]);
       }
-      for (int idx = tid; idx < C * DV / 4; idx += G::NT) {
-        const int t = idx / (DV / 4), c = 4 * (idx % (DV / 4));
-        float v4[4];
-        bf16x4_to_f32(sV + t * G::LDV + c, v4);
-        const float bt = sBeta[t];
-        *reinterpret_cast<float4*>(sU + t * G::LDU + c) = make_float4(bt * v4[0], bt * v4[1], bt * v4[2], bt * v4[3]);
-      }
     }
     __syncthreads();
 
     if (DELTA) {
-      // 3. (I + A) X = R, one right-hand-side column per thread; W to its operand layout
+      // 3. (I + A) X = R, one right-hand-side column per thread: W in shared
+      // memory, then its operand layout; U (right-hand side beta V read from V)
+      // into tensor memory, its column on this thread's TMEM lane
       if (tid < DK + DV) {
         const bool isw = tid < DK;
-        float* col = isw ? sWt + tid : sU + (tid - DK);
-        const int ld = isw ? LDW : G::LDU;
+        float* col = sWt + tid;
+        const int cu = tid - DK;
         float x[C];
 #pragma unroll
         for (int t = 0; t < C; ++t) {
-          float acc0 = col[t * ld], acc1 = 0.f;
+          float acc0 = isw ? col[t * LDW] : sBeta[t] * __bfloat162float(sV[t * G::LDV + cu]), acc1 = 0.f;
           const float* arow = sA + t * G::LDA;
 #pragma unroll
           for (int s = 0; s + 3 < t; s += 4) {
@@ -741,7 +739,11 @@ __global__ void __launch_bounds__(512, 1) key_chunk_prefill_tc_kernel(const Pref
 #pragma unroll
           for (int s = t & ~3; s < t; ++s) acc0 = fmaf(-arow[s], x[s], acc0);
           x[t] = acc0 + acc1;
-          col[t * ld] = x[t];
+          if (isw) col[t * LDW] = x[t];
+        }
+        if (!isw) {   // whole warps: the U columns are threads DK .. DK + DV - 1
+          tmem_st32(tmem + lane_base + G::TM_U, x);
+          tmem_wait_st();
         }
       }
       __syncthreads();
@@ -770,11 +772,13 @@ __global__ void __launch_bounds__(512, 1) key_chunk_prefill_tc_kernel(const Pref
         umma_commit(barB);
       }
     } else {
-      // B^T = V^T (bf16 values are tf32-exact), columns 8 group ..
-      float v[8];
+      // B^T = V^T (bf16 values are tf32-exact), column blocks 8 b8 ..
+      for (int b8 = group; b8 < C / 8; b8 += NG) {
+        float v[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = __bfloat162float(sV[(8 * group + i) * G::LDV + c_own]);
-      tmem_st8(tmem + lane_base + G::TM_B + 8 * group, v);
+        for (int i = 0; i < 8; ++i) v[i] = __bfloat162float(sV[(8 * b8 + i) * G::LDV + c_own]);
+        tmem_st8(tmem + lane_base + G::TM_B + 8 * b8, v);
+      }
       tmem_wait_st();
     }
 
@@ -800,6 +804,12 @@ __global__ void __launch_bounds__(512, 1) key_chunk_prefill_tc_kernel(const Pref
     fence_smem_to_async();
     tc_fence_before();
     __syncthreads();
+    // every read of this chunk's K, Q, V and gates is done: the next chunk's stream in
+    if (has_next) {
+      stage_kqg(c0 + C);
+      stage_rows(sV, Vg, c0 + C, DV, G::LDV);
+    }
+    cp_async_commit();
     if (tid == 0) {   // O^T = S^T (scaled Q)^T  (+ B^T P^T at once for RWKV6)
       tc_fence_after();
       constexpr uint32_t ID = umma_idesc_tf32<128, C>();
@@ -821,12 +831,15 @@ __global__ void __launch_bounds__(512, 1) key_chunk_prefill_tc_kernel(const Pref
       if (!mbar_wait_abortable(barB, par, sAbort) && tid == 0) atomicOr(a.err, kErrWaitTimeout);
       tc_fence_after();
       if (!*sAbort) {
-        float v[8];
-        const uint32_t ta = tmem + lane_base + G::TM_B + 8 * group;
-        tmem_ld8(ta, v);
+        for (int b8 = group; b8 < C / 8; b8 += NG) {
+          float v[8], u[8];
+          const uint32_t ta = tmem + lane_base + G::TM_B + 8 * b8;
+          tmem_ld8(ta, v);
+          tmem_ld8(tmem + lane_base + G::TM_U + 8 * b8, u);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = wm::__float_to_tf32(sU[(8 * group + i) * G::LDU + c_own] - v[i]);
-        tmem_st8(ta, v);
+          for (int i = 0; i < 8; ++i) v[i] = wm::__float_to_tf32(u[i] - v[i]);
+          tmem_st8(ta, v);
+        }
         tmem_wait_st();
       }
       tc_fence_before();
@@ -847,19 +860,23 @@ __global__ void __launch_bounds__(512, 1) key_chunk_prefill_tc_kernel(const Pref
     if (!mbar_wait_abortable(barO, par, sAbort) && tid == 0) atomicOr(a.err, kErrWaitTimeout);
     tc_fence_after();
     if (!*sAbort) {
-      float v[8];
-      tmem_ld8(tmem + lane_base + G::TM_O + 8 * group, v);
+      for (int b8 = group; b8 < C / 8; b8 += NG) {
+        float v[8];
+        tmem_ld8(tmem + lane_base + G::TM_O + 8 * b8, v);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int t = 8 * group + i;
-        if (t < n) Og[((c0 + t) * a.H + h) * DV + c_own] = __float2bfloat16_rn(v[i]);
+        for (int i = 0; i < 8; ++i) {
+          const int t = 8 * b8 + i;
+          if (t < n) Og[((c0 + t) * a.H + h) * DV + c_own] = __float2bfloat16_rn(v[i]);
+        }
       }
-      float sv[32];
-      const uint32_t ts = tmem + lane_base + G::TM_S + 32 * group;
-      tmem_ld32(ts, sv);
+      for (int cb = group; cb < DK / 32; cb += NG) {
+        float sv[32];
+        const uint32_t ts = tmem + lane_base + G::TM_S + 32 * cb;
+        tmem_ld32(ts, sv);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) sv[i] *= sE[32 * group + i];
-      tmem_st32(ts, sv);
+        for (int i = 0; i < 32; ++i) sv[i] *= sE[32 * cb + i];
+        tmem_st32(ts, sv);
+      }
       tmem_wait_st();
     }
     tc_fence_before();
@@ -884,10 +901,12 @@ __global__ void __launch_bounds__(512, 1) key_chunk_prefill_tc_kernel(const Pref
   tc_fence_after();
   const bool ok = !*sAbort;
   if (ok) {
-    float v[32];
-    tmem_ld32(tmem + lane_base + G::TM_S + 32 * group, v);
+    for (int cb = group; cb < DK / 32; cb += NG) {
+      float v[32];
+      tmem_ld32(tmem + lane_base + G::TM_S + 32 * cb, v);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) __stcs(Sg + (32 * group + i) * DV + c_own, v[i]);
+      for (int i = 0; i < 32; ++i) __stcs(Sg + (32 * cb + i) * DV + c_own, v[i]);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -898,7 +917,8 @@ __global__ void __launch_bounds__(512, 1) key_chunk_prefill_tc_kernel(const Pref
   if (ok) clear_log_tile<OP, DK, DV, __nv_bfloat16>(a, sh, 0, DV);
 }
 
-// Grid (H, rows), 512 threads, KeyTcChunkGeom::BYTES of dynamic shared memory;
+// Grid (H, rows), 256 threads (two CTAs per SM) once the launch has more CTAs
+// than SMs, else 512; KeyTcChunkGeom<NT>::BYTES of dynamic shared memory;
 // d_k = d_v = 128, bf16 inputs.  Instantiated in prefill.cu.
 template <int OP>
 cudaError_t launch_key_chunk_prefill_tc(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st);
