@@ -97,7 +97,7 @@ def _prefill_then_decode(op, dims, dtype, kernel, H):
     o = h.prefill(*_prefill_args(op, d), cu_seqlens=torch.from_numpy(cu).cuda(),
                   slot_idx=torch.tensor(slots, dtype=torch.int32, device="cuda"), zero_state=True)
     assert h.log_len == 2                                # the handle's cycle is unchanged
-    min_avg = 64 if (dk, dv) != (128, 128) else 32 if op == "kda" else 24   # the automatic rule
+    min_avg = 64 if (dk, dv) != (128, 128) else 24 if op == "kda" else 16   # the automatic rule
     auto_chunked = dtype == torch.bfloat16 and sum(lens) >= min_avg * rows
     want = "chunked" if kernel == "chunked" or (kernel == "auto" and auto_chunked) else "recurrent"
     assert h.last_prefill_kernel == want
