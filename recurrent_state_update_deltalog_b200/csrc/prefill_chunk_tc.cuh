@@ -122,6 +122,22 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 
 constexpr size_t tc_align128(size_t x) { return (x + 127) & ~size_t(127); }
 
+// K-major operand of R rows whose 8-row groups are adjacent (stride byte
+// offset 128) and whose 16-byte k-chunks are R/8 x 128 + 16 bytes apart
+// (leading byte offset): the 16-byte pad puts the 32 consecutive k of one
+// row on 32 different banks, so a warp can write a row, or a column-parallel
+// solve can update one, without bank conflicts.
+template <int R>
+__host__ __device__ constexpr uint32_t kmajor_pad_lbo() { return (R / 8) * 128 + 16; }
+template <int R>
+__device__ __forceinline__ uint32_t kmajor_pad_off(int r, int k) {
+  return static_cast<uint32_t>((r >> 3) * 128 + (k >> 2) * kmajor_pad_lbo<R>() + (r & 7) * 16 + (k & 3) * 4);
+}
+__device__ __forceinline__ uint64_t umma_desc_lbo(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3fff) | (static_cast<uint64_t>((lbo >> 4) & 0x3fff) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3fff) << 32) | (static_cast<uint64_t>(1) << 46);
+}
+
 template <int NT_>
 struct TcChunkGeom {
   static constexpr int DK = 128, DV = 128;   // a whole head per CTA
@@ -134,18 +150,18 @@ struct TcChunkGeom {
   static constexpr int LDK = DK + 8;         // bf16 row stride of K and Q
   static constexpr int LDV = DV + 8;         // bf16 row stride of V
   static constexpr int LDA = C + 4;          // fp32 row stride of A and P (WMMA outputs)
-  static constexpr int LDU = DV + 4;         // fp32 row stride of U
+  static constexpr uint32_t WQ_LBO = kmajor_pad_lbo<C>();             // W and e^G Q operand layout
+  static constexpr size_t WQ_BYTES = size_t(DK / 4) * WQ_LBO;
   static constexpr size_t KQ_BYTES = tc_align128(size_t(C) * LDK * 2), V_BYTES = tc_align128(size_t(C) * LDV * 2);
   static constexpr size_t K_OFF = 0;                                  // [2][C][LDK] bf16
   static constexpr size_t Q_OFF = K_OFF + 2 * KQ_BYTES;               // [C][LDK] bf16
   static constexpr size_t V_OFF = Q_OFF + KQ_BYTES;                   // [C][LDV] bf16
   static constexpr size_t A_OFF = V_OFF + V_BYTES;                    // [C][LDA] fp32
-  static constexpr size_t WC_OFF = tc_align128(A_OFF + size_t(C) * LDA * 4);   // W, K-major C x DK
-  static constexpr size_t QC_OFF = WC_OFF + size_t(C) * DK * 4;       // e^G Q, K-major C x DK
-  static constexpr size_t PC_OFF = QC_OFF + size_t(C) * DK * 4;       // P, K-major C x C
+  static constexpr size_t WC_OFF = tc_align128(A_OFF + size_t(C) * LDA * 4);   // W, padded K-major C x DK
+  static constexpr size_t QC_OFF = tc_align128(WC_OFF + WQ_BYTES);    // e^G Q, padded K-major C x DK
+  static constexpr size_t PC_OFF = tc_align128(QC_OFF + WQ_BYTES);    // P, K-major C x C
   static constexpr size_t KC_OFF = PC_OFF + size_t(C) * C * 4;        // (e^{..} K)^T, K-major DK x C
-  static constexpr size_t U_OFF = KC_OFF + size_t(DK) * C * 4;        // [C][LDU] fp32
-  static constexpr size_t G_OFF = tc_align128(U_OFF + size_t(C) * LDU * 4);    // 5 x [C] per-row factors
+  static constexpr size_t G_OFF = tc_align128(KC_OFF + size_t(DK) * C * 4);    // 5 x [C] per-row factors
   static constexpr size_t BAR_OFF = tc_align128(G_OFF + 5 * C * 4);            // 3 mbarriers, TMEM base, abort flag
   static constexpr size_t BYTES = BAR_OFF + 64;
   // tensor-memory columns
@@ -153,6 +169,7 @@ struct TcChunkGeom {
   static constexpr uint32_t TM_S = 0;        // S^T: 128 columns (keys)
   static constexpr uint32_t TM_B = 128;      // W S, then B^T: C columns (tokens)
   static constexpr uint32_t TM_O = 160;      // O^T: C columns
+  static constexpr uint32_t TM_U = 192;      // U^T: C columns (the solve writes it)
 };
 
 template <int NT_>
@@ -168,7 +185,6 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_>::MINB) gdn_chunk_prefill
   unsigned char* sQc = smem + G::QC_OFF;
   unsigned char* sPc = smem + G::PC_OFF;
   unsigned char* sKc = smem + G::KC_OFF;
-  float* sU = reinterpret_cast<float*>(smem + G::U_OFF);
   float* sG = reinterpret_cast<float*>(smem + G::G_OFF);
   float* sBeta = sG + C;
   float* sEG = sG + 2 * C;
@@ -280,9 +296,6 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_>::MINB) gdn_chunk_prefill
     rr = (core / (kt >> 2)) * 8 + (within >> 2);
     kk = (core % (kt >> 2)) * 4 + (within & 3);
   };
-  float* sWt = reinterpret_cast<float*>(smem + G::QC_OFF);   // W row-major [C][DK + 4] during the solve
-  constexpr int LDW = DK + 4;
-  static_assert(size_t(C) * LDW * 4 <= G::KC_OFF - G::QC_OFF, "row-major W fits the Q and P operand space");
 
   int buf = 0, ci = 0;
   for (long c0 = t0; c0 < t1; c0 += C, buf ^= 1, ++ci) {
@@ -324,27 +337,26 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_>::MINB) gdn_chunk_prefill
       float& x = sA[t * G::LDA + s];
       x = s < t ? sBeta[t] * expf(sG[t] - sG[s]) * x : 0.f;
     }
-    for (int idx = tid; idx < C * DK; idx += G::NT) {
-      const int t = idx / DK, j = idx % DK;
-      sWt[t * LDW + j] = sBEG[t] * __bfloat162float(sK[t * G::LDK + j]);
-    }
-    for (int idx = tid; idx < C * DV; idx += G::NT) {
-      const int t = idx / DV, c = idx % DV;
-      sU[t * G::LDU + c] = sBeta[t] * __bfloat162float(sV[t * G::LDV + c]);
+    for (int idx = tid; idx < C * DK / 4; idx += G::NT) {   // beta e^G K, four keys a thread
+      const int t = idx / (DK / 4), j = 4 * (idx % (DK / 4));
+      float k4[4];
+      bf16x4_to_f32(sK + t * G::LDK + j, k4);
+      const float f = sBEG[t];
+      *reinterpret_cast<float4*>(sWc + kmajor_pad_off<C>(t, j)) = make_float4(f * k4[0], f * k4[1], f * k4[2], f * k4[3]);
     }
     __syncthreads();
-    if (has_next) stage_rows(sV, Vg, c0 + C, DV, G::LDV);   // V of this chunk is consumed
-    cp_async_commit();
 
-    // 3. (I + A) X = R, one right-hand-side column per thread
+    // 3. (I + A) X = R, one right-hand-side column per thread: W in place in its
+    // operand layout (tf32-rounded); U (right-hand side beta V read from V) into
+    // tensor memory, its column on this thread's TMEM lane
     if (tid < DK + DV) {
       const bool isw = tid < DK;
-      float* col = isw ? sWt + tid : sU + (tid - DK);
-      const int ld = isw ? LDW : G::LDU;
+      const int cu = tid - DK;
       float x[C];
 #pragma unroll
       for (int t = 0; t < C; ++t) {
-        float acc0 = col[t * ld], acc1 = 0.f;
+        float acc0 = isw ? fp(sWc, kmajor_pad_off<C>(t, tid))[0] : sBeta[t] * __bfloat162float(sV[t * G::LDV + cu]);
+        float acc1 = 0.f;
         const float* arow = sA + t * G::LDA;
 #pragma unroll
         for (int s = 0; s + 3 < t; s += 4) {
@@ -357,17 +369,17 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_>::MINB) gdn_chunk_prefill
 #pragma unroll
         for (int s = t & ~3; s < t; ++s) acc0 = fmaf(-arow[s], x[s], acc0);
         x[t] = acc0 + acc1;
-        col[t * ld] = x[t];
+        if (isw) fp(sWc, kmajor_pad_off<C>(t, tid))[0] = wm::__float_to_tf32(x[t]);
+      }
+      if (!isw) {   // whole warps: the U columns are threads DK .. DK + DV - 1
+        tmem_st32(tmem + lane_base + G::TM_U, x);
+        tmem_wait_st();
       }
     }
-    __syncthreads();
-    // W into its K-major operand layout, tf32-rounded
-    for (int e = tid; e < C * DK; e += G::NT) {
-      int t, j;
-      kmajor_rk(e, DK, t, j);
-      fp(sWc, 4 * e)[0] = wm::__float_to_tf32(sWt[t * LDW + j]);
-    }
     fence_smem_to_async();
+    __syncthreads();
+    if (has_next) stage_rows(sV, Vg, c0 + C, DV, G::LDV);   // V of this chunk is consumed
+    cp_async_commit();
 
     // 4. the previous chunk's state update must be complete before S^T is read
     if (ci > 0 && !mbar_wait_abortable(barS, par ^ 1u, sAbort) && tid == 0) atomicOr(a.err, kErrWaitTimeout);
@@ -380,7 +392,8 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_>::MINB) gdn_chunk_prefill
       const uint32_t w0 = smem_u32(sWc);
 #pragma unroll
       for (int s = 0; s < DK / 8; ++s)
-        umma_tf32_ts(tmem + G::TM_B, tmem + G::TM_S + 8 * s, umma_desc(w0 + 256 * s, (DK / 4) * 128), ID, s > 0);
+        umma_tf32_ts(tmem + G::TM_B, tmem + G::TM_S + 8 * s, umma_desc_lbo(w0 + 2 * G::WQ_LBO * s, G::WQ_LBO, 128),
+                     ID, s > 0);
       umma_commit(barB);
     }
 
@@ -394,10 +407,14 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_>::MINB) gdn_chunk_prefill
       kmajor_rk(e, C, t, s);
       fp(sPc, 4 * e)[0] = s <= t ? wm::__float_to_tf32(expf(sG[t] - sG[s]) * sA[t * G::LDA + s]) : 0.f;
     }
-    for (int e = tid; e < C * DK; e += G::NT) {
-      int t, j;
-      kmajor_rk(e, DK, t, j);
-      fp(sQc, 4 * e)[0] = wm::__float_to_tf32(sEG[t] * __bfloat162float(sQ[t * G::LDK + j]));
+    for (int idx = tid; idx < C * DK / 4; idx += G::NT) {   // e^G Q, four keys a thread
+      const int t = idx / (DK / 4), j = 4 * (idx % (DK / 4));
+      float q4[4];
+      bf16x4_to_f32(sQ + t * G::LDK + j, q4);
+      const float f = sEG[t];
+      *reinterpret_cast<float4*>(sQc + kmajor_pad_off<C>(t, j)) =
+          make_float4(wm::__float_to_tf32(f * q4[0]), wm::__float_to_tf32(f * q4[1]), wm::__float_to_tf32(f * q4[2]),
+                      wm::__float_to_tf32(f * q4[3]));
     }
     for (int e = tid; e < DK * C; e += G::NT) {
       int j, t;
@@ -412,7 +429,8 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_>::MINB) gdn_chunk_prefill
       const uint32_t q0 = smem_u32(sQc);
 #pragma unroll
       for (int s = 0; s < DK / 8; ++s)
-        umma_tf32_ts(tmem + G::TM_O, tmem + G::TM_S + 8 * s, umma_desc(q0 + 256 * s, (DK / 4) * 128), ID, s > 0);
+        umma_tf32_ts(tmem + G::TM_O, tmem + G::TM_S + 8 * s, umma_desc_lbo(q0 + 2 * G::WQ_LBO * s, G::WQ_LBO, 128),
+                     ID, s > 0);
     }
 
     // 6. B^T = U^T - (W S)^T in tensor memory, tf32-rounded (columns 8 group ..)
@@ -420,11 +438,12 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_>::MINB) gdn_chunk_prefill
     tc_fence_after();
     if (!*sAbort) {
       for (int b8 = group; b8 < C / 8; b8 += NG) {
-        float v[8];
+        float v[8], u[8];
         const uint32_t ta = tmem + lane_base + G::TM_B + 8 * b8;
         tmem_ld8(ta, v);
+        tmem_ld8(tmem + lane_base + G::TM_U + 8 * b8, u);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = wm::__float_to_tf32(sU[(8 * b8 + i) * G::LDU + c_own] - v[i]);
+        for (int i = 0; i < 8; ++i) v[i] = wm::__float_to_tf32(u[i] - v[i]);
         tmem_st8(ta, v);
       }
       tmem_wait_st();
