@@ -545,6 +545,8 @@ struct KeyTcChunkGeom {
   static constexpr int NG = NW / 4;                 // column groups of the TMEM epilogues
   static constexpr int MINB = NT == 256 ? 2 : 1;
   static constexpr int LDK = DK + 8, LDV = DV + 8, LDG = DK + 4, LDA = C + 4;
+  static constexpr uint32_t WQ_LBO = kmajor_pad_lbo<C>();             // W and scaled-query operand layout
+  static constexpr size_t WQ_BYTES = size_t(DK / 4) * WQ_LBO;
   static constexpr size_t KQ_BYTES = tc_align128(size_t(C) * LDK * 2), V_BYTES = tc_align128(size_t(C) * LDV * 2);
   static constexpr size_t G_BYTES = tc_align128(size_t(C) * LDG * 4);
   // single-buffered inputs: the next chunk's V streams in once the solve has
@@ -555,9 +557,9 @@ struct KeyTcChunkGeom {
   static constexpr size_t G_OFF = V_OFF + V_BYTES;                     // [C][LDG] gates, then Gamma
   static constexpr size_t A_OFF = G_OFF + G_BYTES;                     // [C][LDA] A (KDA)
   static constexpr size_t P_OFF = tc_align128(A_OFF + size_t(C) * LDA * 4);   // [C][LDA] P
-  static constexpr size_t WC_OFF = tc_align128(P_OFF + size_t(C) * LDA * 4);  // W, K-major C x DK
-  static constexpr size_t QC_OFF = WC_OFF + size_t(C) * DK * 4;        // scaled queries, K-major C x DK
-  static constexpr size_t PC_OFF = QC_OFF + size_t(C) * DK * 4;        // P, K-major C x C
+  static constexpr size_t WC_OFF = tc_align128(P_OFF + size_t(C) * LDA * 4);  // W, padded K-major C x DK
+  static constexpr size_t QC_OFF = tc_align128(WC_OFF + WQ_BYTES);     // scaled queries, padded K-major C x DK
+  static constexpr size_t PC_OFF = tc_align128(QC_OFF + WQ_BYTES);     // P, K-major C x C
   static constexpr size_t KC_OFF = PC_OFF + size_t(C) * C * 4;         // scaled keys^T, K-major DK x C
   static constexpr size_t E_OFF = tc_align128(KC_OFF + size_t(DK) * C * 4);  // e^{G_end} [DK], u [DK], beta [C]
   static constexpr size_t BAR_OFF = tc_align128(E_OFF + (2 * DK + C) * 4);
@@ -594,9 +596,6 @@ __global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_>::MINB) key_chunk_pref
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(barB + 3);
   volatile int* sAbort = reinterpret_cast<volatile int*>(sTmem + 1);
   auto fp = [](unsigned char* base, uint32_t off) { return reinterpret_cast<float*>(base + off); };
-  float* sWt = reinterpret_cast<float*>(smem + G::QC_OFF);   // W row-major [C][DK + 4] during the solve
-  constexpr int LDW = DK + 4;
-  static_assert(size_t(C) * LDW * 4 <= G::KC_OFF - G::QC_OFF, "row-major W fits the Q and P operand space");
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int quarter = warp & 3, group = warp >> 2;
@@ -727,7 +726,7 @@ __global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_>::MINB) key_chunk_pref
         float k4[4];
         bf16x4_to_f32(sK + t * G::LDK + j, k4);
         const float bt = sBeta[t];
-        *reinterpret_cast<float4*>(sWt + t * LDW + j) =
+        *reinterpret_cast<float4*>(sWc + kmajor_pad_off<C>(t, j)) =
             make_float4(bt * ex2_approx(g.x) * k4[0], bt * ex2_approx(g.y) * k4[1], bt * ex2_approx(g.z) * k4[2],
                         bt * ex2_approx(g.w) * k4[3]);
       }
@@ -740,12 +739,12 @@ __global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_>::MINB) key_chunk_pref
       // into tensor memory, its column on this thread's TMEM lane
       if (tid < DK + DV) {
         const bool isw = tid < DK;
-        float* col = sWt + tid;
         const int cu = tid - DK;
         float x[C];
 #pragma unroll
         for (int t = 0; t < C; ++t) {
-          float acc0 = isw ? col[t * LDW] : sBeta[t] * __bfloat162float(sV[t * G::LDV + cu]), acc1 = 0.f;
+          float acc0 = isw ? fp(sWc, kmajor_pad_off<C>(t, tid))[0] : sBeta[t] * __bfloat162float(sV[t * G::LDV + cu]);
+          float acc1 = 0.f;
           const float* arow = sA + t * G::LDA;
 #pragma unroll
           for (int s = 0; s + 3 < t; s += 4) {
@@ -758,18 +757,12 @@ __global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_>::MINB) key_chunk_pref
 #pragma unroll
           for (int s = t & ~3; s < t; ++s) acc0 = fmaf(-arow[s], x[s], acc0);
           x[t] = acc0 + acc1;
-          if (isw) col[t * LDW] = x[t];
+          if (isw) fp(sWc, kmajor_pad_off<C>(t, tid))[0] = wm::__float_to_tf32(x[t]);
         }
         if (!isw) {   // whole warps: the U columns are threads DK .. DK + DV - 1
           tmem_st32(tmem + lane_base + G::TM_U, x);
           tmem_wait_st();
         }
-      }
-      __syncthreads();
-      for (int e = tid; e < C * DK; e += G::NT) {
-        int t, j;
-        kmajor_rk(e, DK, t, j);
-        fp(sWc, 4 * e)[0] = wm::__float_to_tf32(sWt[t * LDW + j]);
       }
       fence_smem_to_async();
     }
@@ -787,7 +780,8 @@ __global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_>::MINB) key_chunk_pref
         const uint32_t w0 = smem_u32(sWc);
 #pragma unroll
         for (int s = 0; s < DK / 8; ++s)
-          umma_tf32_ts(tmem + G::TM_B, tmem + G::TM_S + 8 * s, umma_desc(w0 + 256 * s, (DK / 4) * 128), ID, s > 0);
+          umma_tf32_ts(tmem + G::TM_B, tmem + G::TM_S + 8 * s,
+                       umma_desc_lbo(w0 + 2 * G::WQ_LBO * s, G::WQ_LBO, 128), ID, s > 0);
         umma_commit(barB);
       }
     } else {
@@ -807,12 +801,15 @@ __global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_>::MINB) key_chunk_pref
       kmajor_rk(e, C, t, s);
       fp(sPc, 4 * e)[0] = sP[t * G::LDA + s];   // tf32-rounded, zero above the diagonal
     }
-    for (int e = tid; e < C * DK; e += G::NT) {
-      int t, j;
-      kmajor_rk(e, DK, t, j);
+    for (int idx = tid; idx < C * DK / 4; idx += G::NT) {   // four keys a thread
+      const int t = idx / (DK / 4), j = 4 * (idx % (DK / 4));
       const int tg = DELTA ? t : t - 1;   // Gamma_t (KDA), Gamma_{t-1} (RWKV6)
-      const float g = tg >= 0 ? sG[tg * G::LDG + j] : 0.f;
-      fp(sQc, 4 * e)[0] = wm::__float_to_tf32(ex2_approx(g) * __bfloat162float(sQ[t * G::LDK + j]));
+      const float4 g = tg >= 0 ? *reinterpret_cast<const float4*>(sG + tg * G::LDG + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      float q4[4];
+      bf16x4_to_f32(sQ + t * G::LDK + j, q4);
+      *reinterpret_cast<float4*>(sQc + kmajor_pad_off<C>(t, j)) =
+          make_float4(wm::__float_to_tf32(ex2_approx(g.x) * q4[0]), wm::__float_to_tf32(ex2_approx(g.y) * q4[1]),
+                      wm::__float_to_tf32(ex2_approx(g.z) * q4[2]), wm::__float_to_tf32(ex2_approx(g.w) * q4[3]));
     }
     for (int e = tid; e < DK * C; e += G::NT) {
       int j, t;
@@ -835,7 +832,8 @@ __global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_>::MINB) key_chunk_pref
       const uint32_t q0 = smem_u32(sQc);
 #pragma unroll
       for (int s = 0; s < DK / 8; ++s)
-        umma_tf32_ts(tmem + G::TM_O, tmem + G::TM_S + 8 * s, umma_desc(q0 + 256 * s, (DK / 4) * 128), ID, s > 0);
+        umma_tf32_ts(tmem + G::TM_O, tmem + G::TM_S + 8 * s, umma_desc_lbo(q0 + 2 * G::WQ_LBO * s, G::WQ_LBO, 128),
+                     ID, s > 0);
       if (!DELTA) {
         const uint32_t p0 = smem_u32(sPc);
 #pragma unroll
