@@ -1,7 +1,8 @@
-// Chunked GDN prefill with the state in tensor memory: the WY chunk form of
-// gdn_chunk_prefill_kernel (prefill_chunk.cuh), with its three products with
-// the state issued as 5th-generation tensor-core MMAs (tcgen05, tf32 operands,
-// fp32 accumulation) on a whole 128 x 128 head per CTA.
+// Chunked prefill with the state in tensor memory, for d_k = d_v = 128: the
+// chunk forms of gdn_chunk_prefill_kernel (prefill_chunk.cuh) and of
+// key_chunk_prefill_kernel (prefill_chunk_key.cuh), with their three products
+// with the state issued as 5th-generation tensor-core MMAs (tcgen05, tf32
+// operands, fp32 accumulation) on a whole head per CTA.
 //
 // The state is kept transposed, S^T (value column c on TMEM lane c, key j on
 // column j), so that it serves directly as the A operand of
@@ -9,13 +10,17 @@
 //   O^T = S^T (e^{Gamma} Q)^T + B^T P^T
 //   S^T <- e^{Gamma_end} S^T + B^T (e^{Gamma_end - Gamma} K)
 // and receives the last as its accumulator; it never leaves tensor memory
-// between the prompt's first and last chunk.  W, the scaled queries, P and
-// the scaled keys are written by the SIMT lanes into shared memory in the
-// K-major no-swizzle operand layout (8-row x 16-byte core matrices).  One
-// thread issues the MMAs; their completion is tracked by mbarriers (bounded
-// waits: a wait that runs out raises DL_DEVERR_WAIT_TIMEOUT and the CTA
-// stops).  The state update of chunk i runs while chunk i + 1 computes its
-// gates, A and the triangular solve.
+// between the prompt's first and last chunk.  B^T, O^T and U^T live in
+// tensor memory too (the triangular solve writes U^T there: each U column is
+// a thread whose TMEM lane is that value column).  W, the scaled queries, P
+// and the scaled keys are written by the SIMT lanes into shared memory in
+// K-major no-swizzle operand layouts.  One thread issues the MMAs; their
+// completion is tracked by mbarriers (bounded waits: a wait that runs out
+// raises DL_DEVERR_WAIT_TIMEOUT and the CTA stops).  The state update of
+// chunk i runs while chunk i + 1 computes its gates, A and the solve.
+//
+// Two CTAs of 256 threads share an SM (and its 512 TMEM columns) when the
+// launch has more CTAs than SMs; one CTA of 512 threads otherwise.
 #pragma once
 
 #include "prefill_chunk.cuh"
@@ -25,14 +30,12 @@ namespace dl {
 
 // ---- tcgen05 / tensor-memory wrappers --------------------------------------
 
-// Byte offset of element (r, k) of an R x KT tf32 operand stored K-major with
-// no swizzle: 8-row x 4-element core matrices of 128 contiguous bytes, the
-// core matrices of one 8-row group adjacent along k, groups KT/4 x 128 bytes
-// apart.
-__device__ __forceinline__ uint32_t kmajor_off(int r, int k, int kt) {
-  return static_cast<uint32_t>((r >> 3) * (kt >> 2) * 128 + (k >> 2) * 128 + (r & 7) * 16 + (k & 3) * 4);
-}
-
+// K-major tf32 operands with no swizzle are made of 8-row x 4-element core
+// matrices of 128 contiguous bytes.  In the dense form used for P and the
+// scaled keys, the core matrices of one 8-row group are adjacent along k and
+// the groups KT/4 x 128 bytes apart: element (r, k) of an R x KT operand sits
+// at byte (r/8)(KT/4)128 + (k/4)128 + (r%8)16 + (k%4)4.
+//
 // Shared-memory matrix descriptor of such an operand: start address, leading
 // byte offset 128 (next core matrix along k), stride byte offset `sbo` (next
 // 8-row group), descriptor version 1, no swizzle.
