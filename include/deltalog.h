@@ -164,8 +164,10 @@ int dl_step_indexed(dl_t h, const int* slot_idx, int rows, const void* q, const 
  * Afterwards each named slot's base holds the state after its last token and
  * its log entries are cleared (dl_slot_load's convention), so dl_step
  * continues from it.  Other slots are untouched.  The outputs equal the
- * eager recurrence's token by token up to fp32 rounding.  With total == 0
- * the input pointers may be NULL. */
+ * eager recurrence's token by token up to fp32 rounding with the recurrent
+ * kernel, and up to the tf32 rounding of the products with the state with
+ * the chunked ones (DL_OPT_PREFILL_KERNEL).  With total == 0 the input
+ * pointers may be NULL. */
 #define DL_PREFILL_ZERO_STATE 1
 int dl_prefill(dl_t h, const int* slot_idx, int rows, const int* cu_seqlens, long long total, int flags,
                const void* q, const void* k, const void* v, const float* log_decay,
@@ -303,7 +305,9 @@ int dl_slot_read(dl_t h, int slot, float* S_out, void* stream);
 
 /* Bits of the device error word. */
 enum dl_device_error {
-  DL_DEVERR_WAIT_TIMEOUT = 1,  /* a bounded wait on a log copy gave up; that unit wrote nothing */
+  DL_DEVERR_WAIT_TIMEOUT = 1,  /* a bounded wait gave up (a log copy in a step: that unit wrote
+                                  nothing; a tensor-core MMA in a chunked prefill: that row
+                                  stopped and did not write its state) */
   DL_DEVERR_SLOT_INDEX = 2,    /* a slot index >= B (indexed steps, dl_prefill) */
   DL_DEVERR_SEQLEN = 4         /* dl_prefill: a row's cu_seqlens range is invalid */
 };
