@@ -220,12 +220,14 @@ int dl_read_state(dl_t h, float* S_out, void* stream);
 /* DL_OPT_HOST_PREFETCH (0 or 1, default 0): see dl_step_host.
  * DL_OPT_PDL (0 or 1, default 1): a register-tile step that follows an append
  * step of the same handle is launched as a programmatic dependent of the
- * previous kernel in the stream, so it starts streaming Sbar (which an append
- * never writes) and reading its inputs while that kernel drains; it reads the
- * log only once the previous kernel has completed.  Append steps allow their
+ * previous kernel in the stream, so its blocks become resident while that
+ * kernel drains.  Until that kernel has completed, the step reads nothing but
+ * Sbar (written only by this handle's own launches, and never by an append):
+ * its inputs, the slot map, the bonus and the log are read after it.  Kernels
+ * of the caller between two dl_step calls (producing the next token's inputs,
+ * say) are therefore safe with the option on.  Append steps allow their
  * successor to launch early; merge steps, dl_eager_step and dl_merge never
- * do.  Disable if other kernels in the stream trigger their dependents early
- * while still writing memory that a later dl_step reads as input. */
+ * do. */
 /* DL_OPT_VALUE_TILES (0 = automatic, 1, 2 or 4): value tiles per head of the
  * register-tile step kernel, i.e. how many CTAs split a head's d_v columns
  * (a split below 32 columns per tile falls back to fewer tiles; each tile
@@ -307,13 +309,17 @@ int dl_slot_read(dl_t h, int slot, float* S_out, void* stream);
 enum dl_device_error {
   DL_DEVERR_WAIT_TIMEOUT = 1,  /* a bounded wait gave up (a log copy in a step: that unit wrote
                                   nothing; a tensor-core MMA in a chunked prefill: that row
-                                  stopped and did not write its state) */
+                                  stopped and did not write its state).  A wait runs out only
+                                  when the hardware did not finish work it was given within a
+                                  second; treat the CUDA context as suspect afterwards */
   DL_DEVERR_SLOT_INDEX = 2,    /* a slot index >= B (indexed steps, dl_prefill) */
   DL_DEVERR_SEQLEN = 4         /* dl_prefill: a row's cu_seqlens range is invalid */
 };
 
-/* Read and clear the handle's device error word (synchronises `stream`).
- * Returns DL_OK, or DL_ERR_DEVICE with the word's bits in the message. */
+/* Read and clear the handle's device error word in one atomic step on
+ * `stream`, then synchronise `stream`.  Returns DL_OK, or DL_ERR_DEVICE with
+ * the word's bits in the message.  Bits raised later by work still running
+ * on other streams stay in the word for the next call. */
 int dl_check_device(dl_t h, void* stream);
 
 /* Static text for a status code, and the last error message of this thread. */

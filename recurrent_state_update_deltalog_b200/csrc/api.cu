@@ -391,6 +391,11 @@ int suggest_m(int op, int dk, int dv, int esize) {
   return best;
 }
 
+// Read and clear the device error word in one atomic step (err[0]) into its
+// snapshot (err[1]): bits that work on other streams raises meanwhile stay in
+// the word for the next check instead of being cleared unseen.
+__global__ void take_error_word(int* err) { err[1] = atomicExch(err, 0); }
+
 }  // namespace
 
 extern "C" {
@@ -471,7 +476,7 @@ int dl_create(dl_t* out, int B, int H, int d_k, int d_v, int M, int op, int in_d
       {&h->logB, nbh * h->Mcap * d_v * logb_alloc_esize(h)},
       {reinterpret_cast<void**>(&h->logLam), nbh * lam_unit_floats(h) * sizeof(float)},
       {reinterpret_cast<void**>(&h->u), static_cast<size_t>(H) * d_k * sizeof(float)},
-      {reinterpret_cast<void**>(&h->err), sizeof(int)},
+      {reinterpret_cast<void**>(&h->err), 2 * sizeof(int)},   // the word and a snapshot of it
       {&h->st[0].q, nbh * d_k * h->esize},
       {&h->st[0].k, nbh * d_k * h->esize},
       {&h->st[0].v, nbh * d_v * h->esize},
@@ -502,7 +507,7 @@ int dl_create(dl_t* out, int B, int H, int d_k, int d_v, int M, int op, int in_d
   }
   if (e == cudaSuccess) e = cudaMemset(h->Sbar, 0, state_bytes(h));
   if (e == cudaSuccess) e = cudaMemset(h->u, 0, static_cast<size_t>(H) * d_k * sizeof(float));
-  if (e == cudaSuccess) e = cudaMemset(h->err, 0, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(h->err, 0, 2 * sizeof(int));
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
     free_all(h);
@@ -837,9 +842,10 @@ int dl_check_device(dl_t h, void* stream) {
   if (!ds.ok()) return fail(DL_ERR_CUDA, "could not select the handle's device");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int flag = 0;
-  cudaError_t e = cudaMemcpyAsync(&flag, h->err, sizeof(int), cudaMemcpyDeviceToHost, s);
+  take_error_word<<<1, 1, 0, s>>>(h->err);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&flag, h->err + 1, sizeof(int), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e == cudaSuccess && flag) e = cudaMemsetAsync(h->err, 0, sizeof(int), s);
   if (e != cudaSuccess) return cuda_fail(e, "dl_check_device");
   return flag ? fail(DL_ERR_DEVICE, "device error word 0x%x", flag) : DL_OK;
 }

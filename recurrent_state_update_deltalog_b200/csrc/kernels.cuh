@@ -287,6 +287,20 @@ deltalog_step_kernel(const StepArgs a) {
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const int c4 = tid % TL::TPR, rg = tid / TL::TPR;
+  // Launch order.  When the host launches this step as a programmatic
+  // dependent (only after an append of the same handle), the kernel just
+  // before it in the stream may still be running, and its writes become
+  // visible only after griddep_wait.  That kernel need not be this handle's
+  // append: a caller's kernel that writes this token's inputs or slot map can
+  // sit in between.  So nothing but Sbar, which only this handle's own
+  // launches write (and appends never do), is read before the wait.  Mapped
+  // launches need the slot map to find their Sbar, and the per-key operators
+  // load their inputs ahead of the state tile (measured on B200: KDA and
+  // RWKV6 appends 5-6% faster than behind 32 KB of state loads), so both wait
+  // first; GDN streams its tile before the wait and loads its few input
+  // words after it.
+  constexpr bool WAIT_FIRST = MAP || OP != OP_GDN;
+  if constexpr (WAIT_FIRST) griddep_wait();
   const UnitIx ux = unit_of<NSPLIT, DVT, MAP>(a);
   if (!ux.ok) return;
   const long bu = ux.bu;      // batch unit: inputs and output
@@ -302,16 +316,10 @@ deltalog_step_kernel(const StepArgs a) {
   float* As = reinterpret_cast<float*>(s_dyn + LL::staged(n));      // merge only
   float* Bc = As + (n + 1) * DK;                                      // merge only
 
-  // 1. This head's Sbar tile into registers (all loads in flight) and the
-  // token's inputs.  Neither is written by the preceding kernel when this one
-  // is launched as a programmatic dependent: the host only does so after an
-  // append step, which writes nothing but the log, and the inputs come from
-  // work that completed before that step.  So these loads may overlap that
-  // kernel's tail; the log is read after griddep_wait.  An append lets the
-  // next step launch early; a merge, which writes Sbar, does not.
-  // Per-key operators load their inputs (d_k gates) ahead of the tile, so that
-  // ReplayPrep does not wait for them behind it (measured on B200: KDA and
-  // RWKV6 appends 5-6% faster); GDN's few input words go after it (1.7%).
+  // 1. The token's inputs and this head's Sbar tile into registers (all
+  // state loads in flight; order as above), then the log once the preceding
+  // kernel has completed.  An append lets the next step launch early; a
+  // merge, which writes Sbar, does not.
   const TI* qg = static_cast<const TI*>(a.q) + bu * DK;
   const TI* kg = static_cast<const TI*>(a.k) + bu * DK;
   float kr[TL::KPL], qr[TL::KPL], gt[TL::KPL], lt[TL::KPL], lp[TL::KPL];
@@ -337,7 +345,7 @@ deltalog_step_kernel(const StepArgs a) {
 #pragma unroll
   for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + (rg * TL::RPT + j) * DV + col0 + 4 * c4);
   if (MODE == MODE_APPEND) griddep_launch_dependents();
-  griddep_wait();
+  if constexpr (!WAIT_FIRST) griddep_wait();
   if (tid == 0) stage_log<OP, DK, DV, TI, BLOW>(s_dyn, &s_bar, a.logA, a.logLam, a.logB, sh, a.Mcap, n);
   if constexpr (!PERKEY) load_inputs();
 

@@ -165,7 +165,7 @@ struct TcChunkGeom {
   static constexpr size_t PC_OFF = tc_align128(QC_OFF + WQ_BYTES);    // P, K-major C x C
   static constexpr size_t KC_OFF = PC_OFF + size_t(C) * C * 4;        // (e^{..} K)^T, K-major DK x C
   static constexpr size_t G_OFF = tc_align128(KC_OFF + size_t(DK) * C * 4);    // 5 x [C] per-row factors
-  static constexpr size_t BAR_OFF = tc_align128(G_OFF + 5 * C * 4);            // 3 mbarriers, TMEM base, abort flag
+  static constexpr size_t BAR_OFF = tc_align128(G_OFF + 5 * C * 4);            // 3 mbarriers, TMEM base, abort flag, drain mbarrier
   static constexpr size_t BYTES = BAR_OFF + 64;
   // tensor-memory columns
   static constexpr uint32_t TM_COLS = 256;   // allocation (power of two)
@@ -198,6 +198,7 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_>::MINB) gdn_chunk_prefill
   uint64_t* barS = barB + 2;                                          // state update done
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(barB + 3);
   volatile int* sAbort = reinterpret_cast<volatile int*>(sTmem + 1);
+  uint64_t* barF = barB + 4;                                          // drain after an abort
   auto fp = [](unsigned char* base, uint32_t off) { return reinterpret_cast<float*>(base + off); };
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -224,6 +225,7 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_>::MINB) gdn_chunk_prefill
     mbar_init(barB, 1);
     mbar_init(barO, 1);
     mbar_init(barS, 1);
+    mbar_init(barF, 1);
     fence_mbar_init();
     *sAbort = 0;
   }
@@ -518,6 +520,14 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_>::MINB) gdn_chunk_prefill
       for (int i = 0; i < 32; ++i) __stcs(Sg + (32 * cb + i) * DV + c_own, v[i]);
     }
   }
+  if (!ok && tid == 0) {
+    // After a timed-out wait, MMAs this thread issued (and their arrivals on
+    // the barriers above) may still be pending: one more commit tracks all of
+    // them, and the tensor memory is freed only once it arrives (or its own
+    // bounded wait gives up).
+    umma_commit(barF);
+    mbar_wait_bounded(barF, 0);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -598,6 +608,7 @@ __global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_>::MINB) key_chunk_pref
   uint64_t* barS = barB + 2;
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(barB + 3);
   volatile int* sAbort = reinterpret_cast<volatile int*>(sTmem + 1);
+  uint64_t* barF = barB + 4;                                          // drain after an abort
   auto fp = [](unsigned char* base, uint32_t off) { return reinterpret_cast<float*>(base + off); };
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -623,6 +634,7 @@ __global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_>::MINB) key_chunk_pref
     mbar_init(barB, 1);
     mbar_init(barO, 1);
     mbar_init(barS, 1);
+    mbar_init(barF, 1);
     fence_mbar_init();
     *sAbort = 0;
   }
@@ -927,6 +939,14 @@ __global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_>::MINB) key_chunk_pref
 #pragma unroll
       for (int i = 0; i < 32; ++i) __stcs(Sg + (32 * cb + i) * DV + c_own, v[i]);
     }
+  }
+  if (!ok && tid == 0) {
+    // After a timed-out wait, MMAs this thread issued (and their arrivals on
+    // the barriers above) may still be pending: one more commit tracks all of
+    // them, and the tensor memory is freed only once it arrives (or its own
+    // bounded wait gives up).
+    umma_commit(barF);
+    mbar_wait_bounded(barF, 0);
   }
   tc_fence_before();
   __syncthreads();

@@ -349,6 +349,64 @@ def test_programmatic_launch_gives_identical_results(op):
     assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
 
 
+@pytest.mark.parametrize("mapped", [False, True])
+@pytest.mark.parametrize("op", OPS)
+def test_inputs_rewritten_in_place_before_each_step(op, mapped):
+    """A serving loop reuses one set of input buffers: a kernel of the caller
+    (here a torch copy, and for mapped steps a fresh slot permutation) writes
+    token t's q/k/v, gates and slot map in place right before dl_step.  With
+    programmatic launch on, the step may start while that copy drains, so it
+    must read none of them before the copy has completed.  The outputs and
+    states must equal those of plain launches and of untouched per-token
+    buffers bit for bit, and the oracle's."""
+    from recurrent_state_update_deltalog_b200 import DeltaLog
+    B, H, d, M, T = 96, 8, 128, 4, 11
+    S0, seq, u = make_inputs(op, B, H, d, d, T, torch.bfloat16)
+    dseq = to_device(seq, torch.bfloat16)
+    perms = [torch.from_numpy(np.random.default_rng(100 + t).permutation(B).astype(np.int32)).cuda()
+             for t in range(T)]
+
+    def token(t):   # inputs of token t in batch-row order (row r on slot perm[r])
+        args = step_args(op, dseq, t)
+        if not mapped:
+            return args
+        p = perms[t].long()
+        return tuple(x[p] if x is not None else None for x in args)
+
+    toks = [token(t) for t in range(T)]
+    res = []
+    for pdl, reuse in ((True, True), (False, True), (False, False)):
+        h = DeltaLog(B, H, d, d, M, op=op)
+        h.set_pdl(pdl)
+        h.load_state(torch.from_numpy(S0).cuda())
+        if u is not None:
+            h.set_bonus(torch.from_numpy(u).cuda())
+        bufs = [torch.empty_like(x) if x is not None else None for x in toks[0]]
+        ibuf = torch.empty(B, dtype=torch.int32, device="cuda")
+        outs = torch.empty((T, B, H, d), dtype=torch.bfloat16, device="cuda")
+        for t in range(T):
+            if reuse:
+                for b, x in zip(bufs, toks[t]):
+                    if b is not None:
+                        b.copy_(x)
+                ibuf.copy_(perms[t])
+                args, idx = bufs, ibuf
+            else:
+                args, idx = toks[t], perms[t]
+            h.step(*args, out=outs[t], **({"slot_idx": idx} if mapped else {}))
+        if mapped:   # back to slot order
+            outs = torch.stack([torch.empty_like(outs[t]).index_copy_(0, perms[t].long(), outs[t])
+                                for t in range(T)])
+        h.check_device()
+        res.append((outs.cpu(), h.read_state().cpu()))
+        h.close()
+    for o, s in res[1:]:
+        assert torch.equal(res[0][0], o) and torch.equal(res[0][1], s)
+    o_ref, S_ref, _ = run_oracle(op, S0, seq, u)
+    assert relerr(res[0][0].float().numpy(), o_ref) < TOL[torch.bfloat16]
+    assert relerr(res[0][1].numpy(), S_ref) < TOL[torch.bfloat16]
+
+
 # ---- per-slot admission (serving: admit / evict / flush one slot) ---------------
 
 def _oracle_step(op, S, seq, t, u):
