@@ -305,6 +305,53 @@ int dl_slot_load(dl_t h, int slot, const float* S, void* stream);
 int dl_slot_merge(dl_t h, int slot, void* stream);
 int dl_slot_read(dl_t h, int slot, float* S_out, void* stream);
 
+/* Allocation-free decode.  The pages have no counterpart to this call; it is
+ * an interface for callers that cannot allocate device memory.  Some callers
+ * cannot call cudaMalloc: a plugin inside an inference engine that hands out
+ * every byte of device memory from its own pool, a process whose device
+ * memory budget is fixed before it starts, or a latency-critical loop that
+ * cannot take an allocation's implicit device synchronisation.  They cannot
+ * create a handle, which allocates its base and log.  dl_decode_static runs T
+ * DeltaLog decode tokens for all B slots and H heads on a dense state S that
+ * the caller owns; the log lives in one fixed device array of
+ * DL_STATIC_SCRATCH_BYTES (16 MiB), which every device that loads this
+ * library holds until the process exits.  The call allocates nothing.
+ *   op, B, H, d_k, d_v, in_dtype   as for dl_create; 1 <= M <= DL_MAX_M;
+ *   S        device float [B][H][d_k][d_v], 16-byte aligned: the state before
+ *            the first token on entry, after the last token on return;
+ *   u        RWKV6 bonus [H][d_k] (device); ignored for GDN and KDA;
+ *   T        tokens; 0 is a no-op;
+ *   q (r for RWKV6), k, v, log_decay, beta, o   token-major: [T] followed
+ *            by the dl_step layout of each (o receives every token's output);
+ *   dev_err  NULL, or a device int (cleared by the caller) that the kernels
+ *            OR their DL_DEVERR_* bits into; with NULL the bits go to a word
+ *            inside the array, cleared at the start of each call and not
+ *            reported.
+ * Tokens 1..M-1 of every M-token cycle append to the log and token M merges
+ * into S (dl_step's schedule, cycles counted from the call's first token); a
+ * partial last cycle is folded into S at the end, so S is dense on return.
+ * The outputs and S equal those of a handle loaded with S that runs the same
+ * T dl_steps and then dl_merge.  The log of the B*H units must fit the
+ * array: per unit m (d_k es + d_v eb) bytes of factors and Lam bytes of
+ * snapshots, with m = max(M - 1, 1), es the input element size, eb = es for
+ * RWKV6 and 4 otherwise, Lam = 4 round4(m) for GDN and 4 m d_k otherwise,
+ * plus 256-byte alignment of each of the three regions and 256 bytes for the
+ * error word.  (GDN at d = 128, bf16, M = 8 takes 5,408 bytes a unit: about
+ * 3,100 units, e.g. B = 96 at H = 32.)  A larger request returns DL_ERR_ARG
+ * and says how many bytes it needs.
+ * The first call on a device looks the array's address up on that device
+ * (and may load the library's device code there): make it before any stream
+ * capture.  Every call uses the same array and finds the previous call's log
+ * in it; nothing of it is read before this call writes it, except the error
+ * word, which the call clears.  Calls whose work overlaps on the GPU (on
+ * different streams, or from several host threads) race on the array: the
+ * caller must order them.  Asynchronous on `stream`, on the current device. */
+#define DL_STATIC_SCRATCH_BYTES (16u << 20)
+int dl_decode_static(int op, int B, int H, int d_k, int d_v, int M, int in_dtype, float* S,
+                     const float* u, int T, const void* q, const void* k, const void* v,
+                     const float* log_decay, const float* beta, void* o, int* dev_err,
+                     void* stream);
+
 /* Bits of the device error word. */
 enum dl_device_error {
   DL_DEVERR_WAIT_TIMEOUT = 1,  /* a bounded wait gave up (a log copy in a step: that unit wrote

@@ -17,6 +17,7 @@ DL_OK = 0
 DL_MAX_M = 64
 DL_M_AUTO = 0
 DL_PREFILL_ZERO_STATE = 1
+DL_STATIC_SCRATCH_BYTES = 16 << 20
 DL_OPT_STEP_KERNEL = 0
 DL_OPT_HOST_PREFETCH = 1
 DL_OPT_PDL = 2
@@ -54,6 +55,7 @@ SIGNATURES = {
     "dl_slot_merge": (_I, [_P, _I, _P]),
     "dl_slot_read": (_I, [_P, _I, _P, _P]),
     "dl_check_device": (_I, [_P, _P]),
+    "dl_decode_static": (_I, [_I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "dl_strerror": (ctypes.c_char_p, [_I]),
     "dl_last_error": (ctypes.c_char_p, []),
 }

@@ -398,6 +398,12 @@ __global__ void take_error_word(int* err) { err[1] = atomicExch(err, 0); }
 
 }  // namespace
 
+namespace dl {
+// The last-error message of this thread, for entry points defined in other
+// translation units.
+int record_error(int code, const char* msg) { return fail(code, "%s", msg); }
+}  // namespace dl
+
 extern "C" {
 
 int dl_suggest_m(int op, int d_k, int d_v, int in_dtype, int* M) {
