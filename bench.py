@@ -8,7 +8,15 @@ decode sequence for all B slots: 256/M merge cycles, each M-1 append
 launches + 1 merge launch.  ``value`` = slot-tokens per second (B * tokens
 per step * steps / time) summed over all ranks, inputs resident in HBM.
 
-``--impl reference`` times the fp64 CPU oracle instead (rank 0 only).
+For the metric's headline the same line also carries, under "workloads",
+KDA (B=128, H=32, d=128) and RWKV6 (B=128, H=64, d=64) at M=8 with their
+eager-kernel and e2e figures, and under "sweep" the headline at M = 4 and 16
+(M = 1 is the "eager" key).  ``cpu_baseline`` times the fp64 oracle on the
+host cores (one spawned worker process per core, each on its own sample of
+the workload) and on one core alone.
+
+``--impl reference`` times that same oracle sample as the reference arm
+(rank 0 only).
 
 Prints ONE JSON line on rank 0.
 """
@@ -51,8 +59,11 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-eager", action="store_true")
-    ap.add_argument("--sweep", default="", help="extra M values to time, e.g. 1,4,16")
-    ap.add_argument("--kernel", choices=["auto", "register", "stream"], default="auto",
+    ap.add_argument("--sweep", default="",
+                    help="extra M values to time, e.g. 1,4,16 (default for the metric's headline: 4,16)")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time only the given workload (no other workloads of the metric, no M sweep)")
+    ap.add_argument("--kernel", choices=["auto", "register"], default="auto",
                     help="dl_step kernel variant")
     ap.add_argument("--tiles", type=int, default=0, choices=[0, 1, 2, 4],
                     help="value tiles per head of the register step kernel (0 = automatic)")
@@ -194,7 +205,7 @@ def measured_peak():
 
 
 # the sources that define the decode step kernels and their launch geometry
-STEP_KERNEL_SOURCES = ("kernels.cuh", "launch.cuh", "ptx.cuh", "stream.cuh")
+STEP_KERNEL_SOURCES = ("kernels.cuh", "launch.cuh", "ptx.cuh")
 
 
 def kernel_source_hash():
@@ -270,53 +281,136 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
-# reference arm: the fp64 CPU oracle
+# the fp64 CPU oracle on the host cores: cpu_baseline and the reference arm
 # ---------------------------------------------------------------------------
 
-def oracle_sample(a, slots, tokens, t0=0):
-    """Run the oracle on `slots` slots (all H heads) for `tokens` tokens; returns seconds."""
+ORACLE_UNITS_PER_WORKER = 64    # (slot, head) units each worker decodes per run
+ORACLE_MAX_WORKERS = 64         # host memory: ~150 MB of fp64 sample per worker
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def _oracle_worker(conn, seed, op, slots, H, d, tokens):
+    """One worker process: draws its own sample (slots x H heads x tokens of the
+    workload's distributions, with its own seed) once, then runs the fp64
+    oracle on it whenever it is told to and replies with the seconds taken."""
+    for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ[var] = "1"
     import numpy as np
     from oracle import eager
     from synthetic import bonus, initial_state, sequence
-    S0 = initial_state(a.seed, a.B, a.H, a.d, a.d, slots=range(slots))
-    seq = sequence(a.seed, a.op, slots, a.H, a.d, a.d, tokens, bf16=True, t0=t0)
-    u = bonus(a.seed, a.H, a.d) if a.op == "rwkv6" else None
-    t = time.perf_counter()
-    o, _, _ = eager(a.op, S0, seq, u=u)
-    el = time.perf_counter() - t
-    assert np.isfinite(o).all()
-    return el
+    S0 = initial_state(seed, slots, H, d, d)
+    seq = sequence(seed, op, slots, H, d, d, tokens, bf16=True)
+    u = bonus(seed, H, d) if op == "rwkv6" else None
+    conn.send("ready")
+    while conn.recv() == "run":
+        t = time.perf_counter()
+        o, _, _ = eager(op, S0, seq, u=u)
+        el = time.perf_counter() - t
+        conn.send((el, bool(np.isfinite(o).all())))
+    conn.close()
 
 
-def cpu_threads():
-    """Threads the oracle uses: its contractions are numpy einsum loops without
-    BLAS dispatch, and its elementwise work is numpy ufuncs -- one thread."""
-    return 1
+class OraclePool:
+    """Spawned worker processes, one per core used, each holding one sample of
+    the workload (ORACLE_UNITS_PER_WORKER units over one bench step of
+    tokens).  A run is every worker decoding its sample at once; its time is
+    wall-clock from the start signal to the last reply."""
+
+    def __init__(self, a, workers):
+        import multiprocessing as mp
+        ctx = mp.get_context("spawn")
+        self.workers = workers
+        self.slots = max(1, ORACLE_UNITS_PER_WORKER // a.H)
+        self.tokens = a.tokens
+        self.conns, self.procs = [], []
+        for w in range(workers):
+            parent, child = ctx.Pipe()
+            proc = ctx.Process(target=_oracle_worker, daemon=True,
+                               args=(child, a.seed + 1 + w, a.op, self.slots, a.H, a.d, self.tokens))
+            proc.start()
+            child.close()
+            self.conns.append(parent)
+            self.procs.append(proc)
+        for c in self.conns:
+            if c.recv() != "ready":
+                raise RuntimeError("oracle worker failed to start")
+
+    @property
+    def slot_tokens(self):
+        return self.workers * self.slots * self.tokens
+
+    def describe(self, a):
+        return (f"{self.workers} worker process(es), each {self.slots} slots x {a.H} heads x {self.tokens} "
+                f"tokens of {workload_name(a)} (fp64 eager recurrence; own seeded sample per worker)")
+
+    def run(self):
+        t = time.perf_counter()
+        for c in self.conns:
+            c.send("run")
+        res = [c.recv() for c in self.conns]
+        wall = time.perf_counter() - t
+        if not all(ok for _, ok in res):
+            raise RuntimeError("oracle produced non-finite outputs")
+        return wall
+
+    def close(self):
+        for c in self.conns:
+            try:
+                c.send("stop")
+                c.close()
+            except OSError:
+                pass
+        for proc in self.procs:
+            proc.join(timeout=30)
 
 
-def cpu_baseline(a, budget_s=10.0):
-    """Oracle throughput on a bounded sample of the workload: the first `slots`
-    slots (all H heads) over one bench step of tokens, grown to ~budget_s."""
-    tokens = a.tokens
-    probe = min(a.tokens, 32)
-    el = oracle_sample(a, 1, probe)
-    slots = int(max(1, min(a.B, budget_s / max(el * tokens / probe, 1e-3))))
-    el = oracle_sample(a, slots, tokens)
-    return {"value": slots * tokens / el, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"{slots} slots x {a.H} heads x {tokens} tokens of {workload_name(a)} "
-                      f"(fp64 eager recurrence)",
-            "seconds": round(el, 3)}
+def cpu_baseline(a):
+    """Oracle throughput on the host: every core (up to ORACLE_MAX_WORKERS)
+    decoding its own sample at once, and one core alone on the same sample."""
+    cores = min(host_cores(), ORACLE_MAX_WORKERS)
+    one = OraclePool(a, 1)
+    t1 = one.run()
+    one.close()
+    pool = OraclePool(a, cores)
+    tn = pool.run()
+    pool.close()
+    return {"value": pool.slot_tokens / tn, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(), "host_cores": host_cores(), "sample": pool.describe(a),
+            "seconds": round(tn, 3),
+            "single_core": {"value": one.slot_tokens / t1, "unit": UNIT, "seconds": round(t1, 3),
+                            "sample": one.describe(a)}}
 
 
 def run_reference(a, rank):
+    """The reference arm: the oracle as it stands on the host cores, each bench
+    step one run of the cpu_baseline sample (rank 0 alone; other ranks exit)."""
     if rank != 0:
         return
-    per_step_tokens = a.M * 4
+    cores = min(host_cores(), ORACLE_MAX_WORKERS)
+    pool = OraclePool(a, cores)
     for _ in range(a.warmup):
-        oracle_sample(a, 1, per_step_tokens)
-    times = [oracle_sample(a, 1, per_step_tokens, t0=i * per_step_tokens) for i in range(a.steps)]
+        pool.run()
+    times = [pool.run() for _ in range(a.steps)]
+    pool.close()
     total = sum(times)
-    value = per_step_tokens * a.steps / total
+    value = pool.slot_tokens * a.steps / total
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * total / a.steps,
@@ -324,8 +418,8 @@ def run_reference(a, rank):
         "data": "synthetic",
         "config": {"workload": workload_name(a), "op": a.op, "B": a.B, "H": a.H, "d_k": a.d,
                    "d_v": a.d, "M": a.M, "parallelism": "cpu"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-                         "sample": f"each step: 1 slot x {a.H} heads x {per_step_tokens} tokens"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "cpu_model": cpu_model(), "sample": "each step: " + pool.describe(a)},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -519,8 +613,7 @@ def run_gpu(a, rank, world, local_rank):
         count = sum(len(ns) for _, ns in launches)
         dur = sum(t for t, _ in launches) / count
         alg = sum(launch_bytes(op, "append", B, H, d, d, n, bb=bb) for _, ns in launches for n in ns) / count
-        dominant = ("deltalog_stream_kernel" if used_kernel[0] == "stream"
-                    else "deltalog_step_kernel") + " (append)"
+        dominant = "deltalog_step_kernel (append)"
     else:   # average over every launch of the step (graph replay or M = 1)
         dur = ms / (a.steps * a.tokens)
         alg = sb / a.tokens
@@ -549,8 +642,9 @@ def run_gpu(a, rank, world, local_rank):
             continue
         sms, _ = timed(mv)
         sbb = step_bytes(op, B, H, d, mv, a.tokens, bb=bb)
+        gbs = sbb / (sms / a.steps / 1e3) / 1e9
         sweep[str(mv)] = {"value": B * a.tokens * a.steps * world / (sms / 1e3),
-                          "gbs": sbb / (sms / a.steps / 1e3) / 1e9,
+                          "ms_per_step": sms / a.steps, "gbs": gbs, "frac": gbs / peak,
                           "write_bytes_per_token": write_bytes_per_token(op, B, H, d, mv, bb=bb)}
     if sweep:
         extra["sweep"] = sweep
@@ -613,7 +707,60 @@ def run_gpu(a, rank, world, local_rank):
         "e2e": e2e,
     }
     line.update(extra)
-    if not a.no_cpu and world == 1:
+    return line
+
+
+# The metric's workloads beside its headline (GDN B=256 H=32 d=128, M=8):
+# KDA and RWKV6 at their decode configurations, and the headline's M sweep.
+METRIC_HEADLINE = {"op": "gdn", "B": 256, "H": 32, "d": 128, "M": 8}
+METRIC_WORKLOADS = [{"op": "kda", "B": 128, "H": 32, "d": 128, "M": 8},
+                    {"op": "rwkv6", "B": 128, "H": 64, "d": 64, "M": 8}]
+METRIC_SWEEP = "4,16"
+
+
+def is_metric_headline(a):
+    """The plain headline configuration (no serving or tuning switches)."""
+    return (all(getattr(a, k) == v for k, v in METRIC_HEADLINE.items()) and not a.slot_map
+            and not a.admit_every and not a.graph and not a.log_b_bf16 and a.kernel == "auto"
+            and a.tiles == 0 and not a.no_pdl and not getattr(a, "m_auto", False))
+
+
+def workload_summary(line):
+    """The figures of one workload's line that the headline line carries."""
+    r = line["roofline"]
+    out = {"value": line["value"], "unit": line["unit"], "ms_per_step": line["ms_per_step"],
+           "step_gbs": r["step_gbs"], "step_frac": r["step_gbs"] / r["peak"],
+           "append_frac": r["frac"], "avg_append_us": r["avg_launch_us"],
+           "write_bytes_per_token": line["write_bytes_per_token"], "config": line["config"],
+           "clocks": line["clocks"]}
+    for key in ("eager", "speedup_vs_eager", "e2e"):
+        if line.get(key) is not None:
+            out[key] = line[key]
+    return out
+
+
+def run_decode(a, rank, world, local_rank):
+    """The decode bench: the headline line, plus (for the metric's headline) the
+    other workloads of the metric and the M sweep in extra keys of that line,
+    and the oracle on the host cores beside it."""
+    import copy
+    headline = is_metric_headline(a)
+    if headline and not a.sweep and not a.headline_only:
+        a.sweep = METRIC_SWEEP
+    line = run_gpu(a, rank, world, local_rank)
+    if headline and not a.headline_only:
+        extras = {}
+        for w in METRIC_WORKLOADS:
+            sub = copy.copy(a)
+            for k, v in w.items():
+                setattr(sub, k, v)
+            sub.sweep = ""
+            sub_line = run_gpu(sub, rank, world, local_rank)
+            if sub_line is not None:
+                extras[sub_line["config"]["workload"]] = workload_summary(sub_line)
+        if line is not None:
+            line["workloads"] = extras
+    if line is not None and not a.no_cpu and world == 1:
         line["cpu_baseline"] = cpu_baseline(a)
     return line
 
@@ -843,7 +990,7 @@ def main():
             if rank == 0:
                 run_pcie(a, local_rank)
         else:
-            line = run_gpu(a, rank, world, local_rank)
+            line = run_decode(a, rank, world, local_rank)
             if line is not None:
                 print(json.dumps(line), flush=True)
     finally:

@@ -78,10 +78,8 @@ enum dl_status {
  * 1 <= M <= DL_MAX_M, or M = DL_M_AUTO for dl_suggest_m's choice (read it
  * back with dl_merge_interval).  The base state starts at zero with an empty
  * log; the RWKV6 bonus starts at zero.  Pointers passed later must be aligned
- * to their element size (state pointers to 16 bytes); q, k, v, o (and
- * per-key log_decay) aligned to 16 bytes let dl_step use its streaming
- * kernel.  M = 1 makes every step a merge step (the deferred path then
- * performs the eager schedule). */
+ * to their element size (state pointers to 16 bytes).  M = 1 makes every step
+ * a merge step (the deferred path then performs the eager schedule). */
 #define DL_MAX_M 64
 #define DL_M_AUTO 0
 int dl_create(dl_t* out, int B, int H, int d_k, int d_v, int M, int op, int in_dtype);
@@ -129,13 +127,24 @@ int dl_step(dl_t h, const void* q, const void* k, const void* v,
  * layouts above, slot_idx is a device int32 array [rows].  A negative index
  * marks a padding row: nothing is read or written for it, o included.  An
  * index >= B is skipped the same way and sets DL_DEVERR_SLOT_INDEX in the
- * device error word (dl_check_device).  Rows must name distinct slots (undefined otherwise).
- * The step appends or merges every named slot exactly like dl_step.  A slot
- * that a step does not name receives no log entry, so from then on its state
- * is undefined until dl_slot_load; every live sequence must be in every step
- * (one handle per state pool and step sequence).  rows == 0 is a no-op.
- * DL_STEP_STREAM does not take an index map, and a map has at most 65535
- * rows (DL_ERR_UNSUPPORTED otherwise). */
+ * device error word (dl_check_device).  Rows must name distinct slots
+ * (undefined otherwise).  The step appends or merges every named slot
+ * exactly like dl_step.
+ * Held slots.  A live sequence that sits a token out (paused, waiting for a
+ * tool call, preempted to let others run) is named as s | DL_SLOT_HOLD: its
+ * row reads no input and writes no output, and its logical state stays
+ * exactly as it was.  On an append the slot receives a null entry (a_n = 0,
+ * b_n = 0 and Lam_n = Lam_{n-1}: nothing is added and its decay does not
+ * advance) and its base is not touched; on a merge step its log is folded
+ * into its base.  The serving integration the pages describe (DeltaLog
+ * technical summary, gist.science, section "Main contributions", item 3: the
+ * operators integrated into a vLLM-based serving stack) needs a sequence to
+ * stay in the pool while it is absent from a batch.  A slot that a step names neither way receives no
+ * log entry, so from then on its state is undefined until dl_slot_load: a
+ * handle's live slots must each be in every step, active or held.
+ * rows == 0 is a no-op.  A map has at most 65535 rows (DL_ERR_UNSUPPORTED
+ * otherwise). */
+#define DL_SLOT_HOLD 0x40000000
 int dl_step_indexed(dl_t h, const int* slot_idx, int rows, const void* q, const void* k,
                     const void* v, const float* log_decay, const float* beta, void* o,
                     void* stream);
@@ -195,7 +204,8 @@ int dl_eager_step(dl_t h, const void* q, const void* k, const void* v,
 
 /* dl_eager_step over batch rows on the slots slot_idx[0..rows), with the
  * conventions of dl_step_indexed (padding rows, index errors, distinct
- * slots).  Slots not named keep their state. */
+ * slots).  Slots not named, and held slots (DL_SLOT_HOLD), keep their
+ * state. */
 int dl_eager_step_indexed(dl_t h, const int* slot_idx, int rows, const void* q, const void* k,
                           const void* v, const float* log_decay, const float* beta, void* o,
                           void* stream);
@@ -208,14 +218,9 @@ int dl_merge(dl_t h, void* stream);
  * (device pointer) without changing the handle. */
 int dl_read_state(dl_t h, float* S_out, void* stream);
 
-/* Tuning options.  DL_OPT_STEP_KERNEL picks the kernel behind dl_step; all
- * variants compute the same result up to the order of fp32 summation.
- *   DL_STEP_AUTO (default): the fastest kernel measured for the launch
- *     (currently the register-tile kernel everywhere);
- *   DL_STEP_REGISTER: always the register-tile kernel (one CTA per slot-head);
- *   DL_STEP_STREAM: the persistent TMA-streaming kernel; needs q, k, v, o
- *     (and, for KDA/RWKV6, log_decay) 16-byte aligned and a shared-memory
- *     plan that fits the device, else dl_step returns DL_ERR_UNSUPPORTED.
+/* Tuning options.  DL_OPT_STEP_KERNEL picks the kernel behind dl_step:
+ *   DL_STEP_AUTO (default) and DL_STEP_REGISTER: the register-tile kernel
+ *     (one CTA per slot-head and value tile), the only step kernel.
  * Returns DL_ERR_ARG for an unknown option or value. */
 /* DL_OPT_HOST_PREFETCH (0 or 1, default 0): see dl_step_host.
  * DL_OPT_PDL (0 or 1, default 1): a register-tile step that follows an append
@@ -243,8 +248,7 @@ int dl_read_state(dl_t h, float* S_out, void* stream);
  * into Sbar at each merge (outputs no longer equal the eager recurrence's up
  * to fp32 rounding only).  bf16-input handles only (DL_ERR_UNSUPPORTED
  * otherwise); a no-op for RWKV6, whose log already holds raw bf16 v_i.
- * Changeable only while the log is empty (DL_ERR_STATE otherwise).  The
- * streaming kernel does not take it (DL_ERR_UNSUPPORTED). */
+ * Changeable only while the log is empty (DL_ERR_STATE otherwise). */
 /* DL_OPT_PREFILL_KERNEL picks the kernel behind dl_prefill:
  *   DL_PREFILL_AUTO (default): the chunked kernel for bf16-input handles
  *     whose prompts average at least 16 tokens (GDN, RWKV6) or 24 (KDA) at
@@ -260,20 +264,28 @@ int dl_read_state(dl_t h, float* S_out, void* stream);
  *     tcgen05 MMAs; other shapes use 64-column tiles and warp-level MMAs.
  *     The products with the state are tf32, inside the bf16-input
  *     tolerance. */
+/* DL_OPT_TEST_STALL_LOG (0 or 1, default 0; for tests of the error path
+ * only): register-tile steps arm their log barrier for the log's bytes but
+ * issue no copy, and bound the wait at 20 microseconds.  Every unit whose
+ * log is not empty then gives up, writes nothing (no output, no log entry,
+ * no state) and raises DL_DEVERR_WAIT_TIMEOUT; nothing is left in flight,
+ * so the context stays usable.  The handle's log is then out of step with
+ * its outputs: load a state (dl_load_state) or destroy it afterwards. */
 enum dl_option {
   DL_OPT_STEP_KERNEL = 0,
   DL_OPT_HOST_PREFETCH = 1,
   DL_OPT_PDL = 2,
   DL_OPT_VALUE_TILES = 3,
   DL_OPT_LOG_B_BF16 = 4,
-  DL_OPT_PREFILL_KERNEL = 5
+  DL_OPT_PREFILL_KERNEL = 5,
+  DL_OPT_TEST_STALL_LOG = 6
 };
 enum dl_prefill_kernel { DL_PREFILL_AUTO = 0, DL_PREFILL_RECURRENT = 1, DL_PREFILL_CHUNKED = 2 };
-enum dl_step_kernel { DL_STEP_AUTO = 0, DL_STEP_REGISTER = 1, DL_STEP_STREAM = 2 };
+enum dl_step_kernel { DL_STEP_AUTO = 0, DL_STEP_REGISTER = 1 };
 int dl_set_option(dl_t h, int option, int value);
 
 /* Which kernel the most recent dl_step / dl_step_host launched:
- * DL_STEP_REGISTER or DL_STEP_STREAM (DL_STEP_AUTO before the first step). */
+ * DL_STEP_REGISTER (DL_STEP_AUTO before the first step). */
 int dl_last_step_kernel(dl_t h, int* kind);
 
 /* Which kernel the most recent dl_prefill launched: DL_PREFILL_RECURRENT or

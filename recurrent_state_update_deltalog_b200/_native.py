@@ -18,14 +18,16 @@ DL_MAX_M = 64
 DL_M_AUTO = 0
 DL_PREFILL_ZERO_STATE = 1
 DL_STATIC_SCRATCH_BYTES = 16 << 20
+DL_SLOT_HOLD = 0x40000000
 DL_OPT_STEP_KERNEL = 0
 DL_OPT_HOST_PREFETCH = 1
 DL_OPT_PDL = 2
 DL_OPT_VALUE_TILES = 3
 DL_OPT_LOG_B_BF16 = 4
 DL_OPT_PREFILL_KERNEL = 5
+DL_OPT_TEST_STALL_LOG = 6
 DL_PREFILL_AUTO, DL_PREFILL_RECURRENT, DL_PREFILL_CHUNKED = 0, 1, 2
-DL_STEP_AUTO, DL_STEP_REGISTER, DL_STEP_STREAM = 0, 1, 2
+DL_STEP_AUTO, DL_STEP_REGISTER = 0, 1
 STATUS = {0: "DL_OK", -1: "DL_ERR_ARG", -2: "DL_ERR_UNSUPPORTED", -3: "DL_ERR_CUDA",
           -4: "DL_ERR_OOM", -5: "DL_ERR_DEVICE", -6: "DL_ERR_STATE"}
 

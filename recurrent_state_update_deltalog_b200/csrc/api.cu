@@ -13,6 +13,7 @@
 static_assert(DL_DEVERR_WAIT_TIMEOUT == dl::kErrWaitTimeout, "device error bits");
 static_assert(DL_DEVERR_SLOT_INDEX == dl::kErrSlotIndex, "device error bits");
 static_assert(DL_DEVERR_SEQLEN == dl::kErrSeqlen, "device error bits");
+static_assert(DL_SLOT_HOLD == dl::kSlotHold, "held-slot bit of the slot map");
 
 struct dl_handle {
   int B, H, dk, dv, M, op, dtype, device;
@@ -53,6 +54,7 @@ struct dl_handle {
   int log_b_bf16;           // DL_OPT_LOG_B_BF16
   int prefill_kernel;       // DL_OPT_PREFILL_KERNEL (DL_PREFILL_*)
   int last_prefill;         // DL_PREFILL_* used by the last dl_prefill
+  int stall_log;            // DL_OPT_TEST_STALL_LOG
 };
 
 namespace {
@@ -128,7 +130,7 @@ void free_all(dl_handle* h) {
 
 // Launch geometry and policies for the handle's current log length and
 // `units` launched (slot, head) units (0: every slot).
-dl::LaunchShape shape_of(const dl_handle* h, bool aligned16 = false, long units = 0) {
+dl::LaunchShape shape_of(const dl_handle* h, long units = 0) {
   dl::LaunchShape s;
   s.BH = static_cast<int>(units > 0 ? units : bh(h));
   s.H = h->H;
@@ -140,7 +142,6 @@ dl::LaunchShape shape_of(const dl_handle* h, bool aligned16 = false, long units 
   s.smem_sm = h->smem_sm;
   s.smem_reserved = h->smem_reserved;
   s.variant = h->step_kernel;
-  s.aligned16 = aligned16;
   // Programmatic launch only when the previous launch of this handle did not
   // write Sbar (an append): the step may then read Sbar before it completes.
   s.pdl = h->pdl && !h->wrote_state;
@@ -203,6 +204,7 @@ dl::StepArgs step_args(dl_handle* h, const void* q, const void* k, const void* v
   a.M = h->M;
   a.Mcap = h->Mcap;
   a.n = h->n;
+  a.stall_log = h->stall_log;
   return a;
 }
 
@@ -224,10 +226,7 @@ cudaError_t zero_slot_log(const dl_handle* h, int b, cudaStream_t s) {
 
 // `rows` batch rows of H units each are launched (B without an index map).
 cudaError_t launch_step(dl_handle* h, int mode, const dl::StepArgs& a, int rows, cudaStream_t s) {
-  // bulk-copy sources of the streaming kernel (GDN's scalar gate is a plain load)
-  const bool al = aligned(a.q, 16) && aligned(a.k, 16) && aligned(a.v, 16) && aligned(a.o, 16) &&
-                  (h->op == DL_GDN || aligned(a.log_decay, 16));
-  const dl::LaunchShape sh = shape_of(h, al, static_cast<long>(rows) * h->H);
+  const dl::LaunchShape sh = shape_of(h, static_cast<long>(rows) * h->H);
   int* used = &h->last_kernel;
   switch (h->op) {
     case DL_GDN: return dl::launch_step_op<dl::OP_GDN>(sh, mode, a, s, used);
@@ -237,7 +236,7 @@ cudaError_t launch_step(dl_handle* h, int mode, const dl::StepArgs& a, int rows,
 }
 
 cudaError_t launch_eager(const dl_handle* h, const dl::StepArgs& a, int rows, cudaStream_t s) {
-  dl::LaunchShape sh = shape_of(h, false, static_cast<long>(rows) * h->H);
+  dl::LaunchShape sh = shape_of(h, static_cast<long>(rows) * h->H);
   // the eager kernel has no per-tile ReplayPrep to repeat: two tiles for
   // d_v = 128 at every batch size measured (B = 1..1024)
   if (h->value_tiles == 0) sh.split = h->dv == 128 ? 2 : 1;
@@ -343,9 +342,6 @@ int do_step(dl_handle* h, const int* idx, int rows, const void* q, const void* k
   dl::StepArgs a = step_args(h, q, k, v, log_decay, beta, o);
   a.slot_idx = idx;
   cudaError_t e = launch_step(h, merge ? dl::MODE_MERGE : dl::MODE_APPEND, a, rows, s);
-  if (e == cudaErrorNotSupported)
-    return fail(DL_ERR_UNSUPPORTED, "the streaming step kernel cannot run this launch (alignment, shared memory "
-                                    "or a slot index map)");
   if (e != cudaSuccess) return cuda_fail(e, "deltalog step launch");
   h->n = merge ? 0 : h->n + 1;
   h->wrote_state = merge;
@@ -791,7 +787,7 @@ int dl_set_option(dl_t h, int option, int value) {
   if (!h) return fail(DL_ERR_ARG, "null handle");
   switch (option) {
     case DL_OPT_STEP_KERNEL:
-      if (value < DL_STEP_AUTO || value > DL_STEP_STREAM) return fail(DL_ERR_ARG, "bad step-kernel value %d", value);
+      if (value != DL_STEP_AUTO && value != DL_STEP_REGISTER) return fail(DL_ERR_ARG, "bad step-kernel value %d", value);
       h->step_kernel = value;
       return DL_OK;
     case DL_OPT_HOST_PREFETCH:
@@ -813,6 +809,10 @@ int dl_set_option(dl_t h, int option, int value) {
       if (value != h->log_b_bf16 && h->n != 0)
         return fail(DL_ERR_STATE, "change the b-log precision only with an empty log (call dl_merge)");
       h->log_b_bf16 = value;
+      return DL_OK;
+    case DL_OPT_TEST_STALL_LOG:
+      if (value != 0 && value != 1) return fail(DL_ERR_ARG, "bad stall-log value %d", value);
+      h->stall_log = value;
       return DL_OK;
     case DL_OPT_VALUE_TILES:
       if (value != 0 && value != 1 && value != 2 && value != 4)

@@ -50,7 +50,8 @@ struct StepArgs {
   const float* log_decay;  // [rows*H] (GDN) or [rows*H][DK]
   const float* beta;       // [rows*H] (GDN/KDA)
   void* o;                 // [rows*H][DV], input dtype
-  const int* slot_idx;     // [rows] pool slot of each batch row (< 0: padding), or null
+  const int* slot_idx;     // [rows] pool slot of each batch row (< 0: padding; kSlotHold
+                           // bit: the slot sits this token out), or null
   int slots;               // pool slots B (bound of slot_idx)
   void* logA;              // [BH][Mcap][DK], input dtype (a_i = k_i)
   void* logB;              // [BH][Mcap][DV], fp32 (GDN/KDA) or input dtype (RWKV6)
@@ -61,7 +62,12 @@ struct StepArgs {
   int M;                   // merge interval
   int Mcap;                // log capacity per (slot, head), >= 1
   int n;                   // entries in the log before this step (lockstep launches)
+  int stall_log;           // test only: arm the log barrier but issue no copy (see stage_log)
 };
+
+// Bound of the log wait when a test stalls the log on purpose: long enough
+// for nothing, short enough that the timeout path is quick.
+constexpr uint64_t kStallWaitNs = 20000;
 
 // Step kernel modes: every slot appends, or every slot merges.
 enum { MODE_APPEND = 0, MODE_MERGE = 1 };
@@ -69,17 +75,23 @@ enum { MODE_APPEND = 0, MODE_MERGE = 1 };
 // Device error bit: a slot index at or past the pool size (the row is skipped).
 constexpr int kErrSlotIndex = 2;
 
+// Slot-map bit of a held slot: the row names slot (index & ~kSlotHold), which
+// takes no input and writes no output this token but keeps its state exact
+// (an append gives it a null log entry; a merge folds its log).
+constexpr int kSlotHold = 0x40000000;
+
 // Which unit a CTA of a step kernel serves.  `bu` (row * H + head) indexes
 // inputs and outputs, `sh` (slot * H + head) the state and the log, `col0` is
 // the tile's first value column.  Unmapped launches: a 1-D grid of
 // B * H * NSPLIT CTAs and sh == bu.  Mapped launches (template switch, so the
 // unmapped kernels carry none of it): grid (H * NSPLIT, rows), row r on slot
 // slot_idx[r]; ok is false for a padding row (negative index) and for an
-// index past the pool, which also raises kErrSlotIndex.
+// index past the pool, which also raises kErrSlotIndex; hold is set for a
+// held slot.
 struct UnitIx {
   long bu, sh;
   int h, col0;
-  bool ok;
+  bool ok, hold;
 };
 
 template <int NSPLIT, int DVT, bool MAP>
@@ -89,9 +101,11 @@ __device__ __forceinline__ UnitIx unit_of(const StepArgs& a) {
     u.h = static_cast<int>(blockIdx.x) / NSPLIT;
     u.col0 = (static_cast<int>(blockIdx.x) % NSPLIT) * DVT;
     u.bu = static_cast<long>(blockIdx.y) * a.H + u.h;
-    const int slot = __ldg(a.slot_idx + blockIdx.y);
-    u.ok = slot >= 0 && slot < a.slots;
-    if (slot >= a.slots && threadIdx.x == 0) atomicOr(a.err, kErrSlotIndex);
+    const int raw = __ldg(a.slot_idx + blockIdx.y);
+    u.hold = raw >= 0 && (raw & kSlotHold);
+    const int slot = raw & ~kSlotHold;
+    u.ok = raw >= 0 && slot < a.slots;
+    if (raw >= 0 && slot >= a.slots && threadIdx.x == 0) atomicOr(a.err, kErrSlotIndex);
     u.sh = static_cast<long>(slot) * a.H + u.h;
   } else {
     u.bu = blockIdx.x / NSPLIT;
@@ -99,6 +113,7 @@ __device__ __forceinline__ UnitIx unit_of(const StepArgs& a) {
     u.h = static_cast<int>(u.bu % a.H);  // only RWKV6 reads it
     u.sh = u.bu;
     u.ok = true;
+    u.hold = false;
   }
   return u;
 }
@@ -224,17 +239,20 @@ __device__ __forceinline__ float4 load4f(const __nv_bfloat16* p) {
 }
 
 // Thread 0 starts the bulk copies of entries [0, n) of this (slot, head)'s log
-// into shared memory; completion arrives on `bar` (phase 0).
+// into shared memory; completion arrives on `bar` (phase 0).  With `stall`
+// (a test of the timeout path) the barrier expects the bytes but no copy is
+// issued: the wait runs out with nothing in flight.
 template <int OP, int DK, int DV, typename TI, bool BLOW>
 __device__ __forceinline__ void stage_log(unsigned char* smem, uint64_t* bar, const void* logA,
                                           const float* logLam, const void* logB, long sh, int Mcap,
-                                          int n) {
+                                          int n, bool stall = false) {
   using LL = LogLayout<OP, DK, DV, TI, BLOW>;
   using TB = typename LL::TB;
   mbar_init(bar, 1);
   fence_mbar_init();
   if (n == 0) return;
   mbar_arrive_expect_tx(bar, static_cast<uint32_t>(LL::staged(n)));
+  if (stall) return;
   bulk_g2s(smem, static_cast<const TI*>(logA) + sh * Mcap * DK, static_cast<uint32_t>(LL::a_bytes(n)), bar);
   if (LL::PERKEY)
     bulk_g2s(smem + LL::a_bytes(n), logLam + sh * Mcap * DK, static_cast<uint32_t>(LL::l_bytes(n)), bar);
@@ -246,15 +264,37 @@ __device__ __forceinline__ void stage_log(unsigned char* smem, uint64_t* bar, co
 // stop: the error word is raised, copies still in flight get one more bounded
 // wait (the CTA must not exit while they target its shared memory), and the
 // caller returns.
-__device__ __forceinline__ bool wait_log(uint64_t* bar, int n, int* err) {
-  int ok = n == 0 ? 1 : static_cast<int>(mbar_wait_bounded(bar, 0));
+__device__ __forceinline__ bool wait_log(uint64_t* bar, int n, int* err, uint64_t limit_ns = kWaitNs) {
+  int ok = n == 0 ? 1 : static_cast<int>(mbar_wait_bounded(bar, 0, limit_ns));
   if (__syncthreads_and(ok)) return true;
   if (threadIdx.x == 0) {
     atomicOr(err, kErrWaitTimeout);
-    mbar_wait_bounded(bar, 0);
+    mbar_wait_bounded(bar, 0, limit_ns);
   }
   __syncthreads();
   return false;
+}
+
+// A held slot's append: the null entry a_n = 0, b_n = 0, Lam_n = Lam_{n-1}
+// adds nothing to its state and does not advance its decay, so its logical
+// state stays exact without reading Sbar.  Each value tile writes its b_n
+// columns; the first tile writes a_n and the snapshot.
+template <int OP, int DK, int DV, typename TI, bool BLOW>
+__device__ __forceinline__ void hold_entry(const StepArgs& a, long sh, int col0, int dvt, int n) {
+  using TB = typename LogLayout<OP, DK, DV, TI, BLOW>::TB;
+  const int tid = threadIdx.x, nt = blockDim.x;
+  TB* dstB = static_cast<TB*>(a.logB) + (sh * a.Mcap + n) * DV + col0;
+  for (int c = tid; c < dvt; c += nt) dstB[c] = from_f<TB>(0.f);
+  if (col0 != 0) return;
+  TI* dstA = static_cast<TI*>(a.logA) + (sh * a.Mcap + n) * DK;
+  for (int j = tid; j < DK; j += nt) dstA[j] = from_f<TI>(0.f);
+  if constexpr (OP != OP_GDN) {
+    float* lam = a.logLam + sh * a.Mcap * DK;
+    for (int j = tid; j < DK; j += nt) lam[n * DK + j] = n > 0 ? lam[(n - 1) * DK + j] : 0.f;
+  } else if (tid == 0) {
+    float* lam = a.logLam + sh * gdn_lam_stride(a.Mcap);
+    lam[n] = n > 0 ? lam[n - 1] : 0.f;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -309,6 +349,14 @@ deltalog_step_kernel(const StepArgs a) {
   const int h = ux.h;
   const int n = a.n;
   constexpr bool MERGE = MODE == MODE_MERGE;
+  // A held slot: an append writes its null entry and stops; a merge runs with
+  // zero inputs (a null current entry) and writes no output, which folds the
+  // slot's log into its base at its unchanged logical state.
+  const bool hold = MAP && ux.hold;
+  if (!MERGE && hold) {
+    hold_entry<OP, DK, DV, TI, BLOW>(a, sh, col0, DVT, n);
+    return;
+  }
 
   const TI* sA = reinterpret_cast<const TI*>(s_dyn);
   const float* sL = reinterpret_cast<const float*>(s_dyn + LL::a_bytes(n));
@@ -326,6 +374,11 @@ deltalog_step_kernel(const StepArgs a) {
   float g_head = 0.f, vc = 0.f, betac = 0.f;
   const int c = tid;
   auto load_inputs = [&]() {
+    if (hold) {   // k = q = v = 0, gate 0, beta 0: a null current entry
+#pragma unroll
+      for (int m = 0; m < TL::KPL; ++m) kr[m] = qr[m] = gt[m] = 0.f;
+      return;
+    }
 #pragma unroll
     for (int m = 0; m < TL::KPL; ++m) {
       const int j = lane + 32 * m;
@@ -346,7 +399,8 @@ deltalog_step_kernel(const StepArgs a) {
   for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + (rg * TL::RPT + j) * DV + col0 + 4 * c4);
   if (MODE == MODE_APPEND) griddep_launch_dependents();
   if constexpr (!WAIT_FIRST) griddep_wait();
-  if (tid == 0) stage_log<OP, DK, DV, TI, BLOW>(s_dyn, &s_bar, a.logA, a.logLam, a.logB, sh, a.Mcap, n);
+  if (tid == 0)
+    stage_log<OP, DK, DV, TI, BLOW>(s_dyn, &s_bar, a.logA, a.logLam, a.logB, sh, a.Mcap, n, a.stall_log != 0);
   if constexpr (!PERKEY) load_inputs();
 
   // 2. Decay snapshots: Lam_{t-1} from the newest entry, Lam_t = Lam_{t-1} +
@@ -368,7 +422,7 @@ deltalog_step_kernel(const StepArgs a) {
     }
   }
   __syncthreads();                              // barrier init and s_lam visible
-  if (!wait_log(&s_bar, n, a.err)) return;
+  if (!wait_log(&s_bar, n, a.err, a.stall_log ? kStallWaitNs : kWaitNs)) return;
 
   // 3. ReplayPrep: per-entry coefficients once per (slot, head).  Warp w takes
   // entries i = w, w+NW, ...; i == n is the current token (kappa).
@@ -473,7 +527,7 @@ deltalog_step_kernel(const StepArgs a) {
       bt = vc;
     }
     oc = fmaf(s_kappa, bt, oc);
-    static_cast<TI*>(a.o)[bu * DV + col0 + c] = from_f<TI>(oc);
+    if (!hold) static_cast<TI*>(a.o)[bu * DV + col0 + c] = from_f<TI>(oc);
     if (MERGE) {
       Bc[c] = bt;
     } else {
@@ -533,7 +587,7 @@ eager_step_kernel(const StepArgs a) {
   const int lane = tid & 31, warp = tid >> 5;
   const int c4 = tid % TL::TPR, rg = tid / TL::TPR;
   const UnitIx ux = unit_of<NSPLIT, DVT, MAP>(a);
-  if (!ux.ok) return;
+  if (!ux.ok || ux.hold) return;   // the dense state of a held slot needs nothing
   const long bu = ux.bu;      // batch unit: inputs and output
   const long sh = ux.sh;      // pool unit: the state
   const int col0 = ux.col0;

@@ -4,12 +4,11 @@
 #pragma once
 
 #include "kernels.cuh"
-#include "stream.cuh"
 
 namespace dl {
 
 // Step-kernel variants (dl_set_option DL_OPT_STEP_KERNEL).
-enum { STEP_AUTO = 0, STEP_REGISTER = 1, STEP_STREAM = 2 };
+enum { STEP_AUTO = 0, STEP_REGISTER = 1 };
 
 struct LaunchShape {
   int BH;     // launched (slot or batch row) x heads
@@ -23,7 +22,6 @@ struct LaunchShape {
   int smem_sm;
   int smem_reserved;
   int variant;     // STEP_*
-  bool aligned16;  // q, k, v, o (and per-key log_decay) 16-byte aligned (bulk-copy sources)
   bool pdl;        // launch the step as a programmatic dependent of the previous kernel
   int split;       // value tiles per head for the register-tile step kernel (1, 2 or 4)
   int max_n;       // log length of the launched units (shared-memory sizing)
@@ -46,59 +44,6 @@ cudaError_t launch_maybe_pdl(void (*kern)(KArgs...), dim3 grid, int block, size_
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kern, args...);
-}
-
-// Ring/slot plan of the streaming kernel for one launch.
-struct StreamPlan {
-  bool ok;
-  int ctas_per_sm;
-  int ns;
-  size_t smem;
-};
-
-// Largest ring that fits: two CTAs per SM first (each one's finalize then
-// overlaps the other's streaming), else one CTA with a deeper ring.  A merge
-// launch keeps all of a unit's chunks resident until its write-back, so its
-// ring holds at least one chunk more than a unit.
-template <int OP, int DK, int DV, typename TI>
-StreamPlan plan_stream(const LaunchShape& s, int n, bool merge, size_t static_smem) {
-  using SG = StreamGeom<OP, DK, DV, TI>;
-  const int min_ns = merge ? SG::CPU + 1 : 2;
-  const int max_ns[2] = {6, kMaxStages};
-  for (int pass = 0; pass < 2; ++pass) {
-    const int ctas = pass == 0 ? 2 : 1;
-    for (int ns = max_ns[pass]; ns >= min_ns; --ns) {
-      const size_t dyn = SG::smem(n, merge, ns);
-      const size_t blk = dyn + static_smem;
-      if (blk > static_cast<size_t>(s.smem_block_optin)) continue;
-      if (static_cast<size_t>(ctas) * (blk + s.smem_reserved) > static_cast<size_t>(s.smem_sm)) continue;
-      return StreamPlan{true, ctas, ns, dyn};
-    }
-  }
-  return StreamPlan{false, 0, 0, 0};
-}
-
-template <int OP, int DK, int DV, typename TI, bool MERGE>
-cudaError_t stream_dims(const LaunchShape& s, const StepArgs& a, cudaStream_t st, bool* launched) {
-  auto kern = deltalog_stream_kernel<OP, DK, DV, TI, MERGE>;
-  *launched = false;
-  cudaFuncAttributes fa;
-  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
-  if (e != cudaSuccess) return e;
-  const StreamPlan p = plan_stream<OP, DK, DV, TI>(s, a.n, MERGE, fa.sharedSizeBytes);
-  if (!p.ok) return cudaSuccess;
-  if (p.smem + fa.sharedSizeBytes > 48 * 1024) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             s.smem_block_optin - static_cast<int>(fa.sharedSizeBytes));
-    if (e != cudaSuccess) return e;
-    // the whole unified L1/shared array as shared memory, so the planned CTAs fit
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e != cudaSuccess) return e;
-  }
-  const int grid = s.BH < p.ctas_per_sm * s.sms ? s.BH : p.ctas_per_sm * s.sms;
-  kern<<<grid, StreamGeom<OP, DK, DV, TI>::NT, p.smem, st>>>(a, StreamCfg{s.BH, p.ns});
-  *launched = true;
-  return cudaGetLastError();
 }
 
 // Opt a kernel into more than the default 48 KB of shared memory (static +
@@ -157,17 +102,6 @@ cudaError_t register_step(const LaunchShape& s, int mode, const StepArgs& a, cud
 
 template <int OP, int DK, int DV, typename TI>
 cudaError_t step_dims(const LaunchShape& s, int mode, const StepArgs& a, cudaStream_t st, int* used) {
-  // AUTO runs the register-tile kernel, the faster of the two on B200 for
-  // every operator's merge launches and for d_v = 64; STREAM is opt-in and
-  // takes no slot index map.
-  if (s.variant == STEP_STREAM && s.aligned16 && !a.slot_idx && !s.blow) {
-    bool launched = false;
-    cudaError_t e = mode == MODE_MERGE ? stream_dims<OP, DK, DV, TI, true>(s, a, st, &launched)
-                                       : stream_dims<OP, DK, DV, TI, false>(s, a, st, &launched);
-    if (launched) *used = STEP_STREAM;
-    if (e != cudaSuccess || launched) return e;
-  }
-  if (s.variant == STEP_STREAM) return cudaErrorNotSupported;
   *used = STEP_REGISTER;
   if constexpr (DV >= 128) {
     if (s.split == 4) return register_step<OP, DK, DV, TI, 4>(s, mode, a, st);

@@ -154,7 +154,6 @@ extern "C" int dl_decode_static(int op, int B, int H, int d_k, int d_v, int M, i
   sh.smem_sm = ds.smem_sm;
   sh.smem_reserved = ds.smem_reserved;
   sh.variant = dl::STEP_REGISTER;
-  sh.aligned16 = false;
   sh.units = sh.BH;
   sh.blow = false;
 

@@ -38,6 +38,8 @@ class DeltaLog:
     CUDA device that is current (or given) at construction.
     """
 
+    HOLD = N.DL_SLOT_HOLD   # slot-map bit of a slot that sits a token out
+
     def __init__(self, B, H, d_k, d_v, M, op="gdn", dtype=torch.bfloat16, device=None):
         if op not in OPS:
             raise ValueError(f"op must be one of {sorted(OPS)}")
@@ -118,7 +120,9 @@ class DeltaLog:
 
         With ``slot_idx`` (int32 [rows] on the device), inputs and output have
         ``rows`` batch rows and row r runs on slot ``slot_idx[r]`` (negative:
-        padding row, left untouched); every live slot must be named."""
+        padding row, left untouched); every live slot must be named, either
+        active or held (``slot | DeltaLog.HOLD``: no input read, no output
+        written, state kept exactly)."""
         rows = self._slot_map(slot_idx)
         out = self._alloc_out(True, rows) if out is None else out
         self._check_step(q, k, v, log_decay, beta, out, True, rows)
@@ -189,8 +193,8 @@ class DeltaLog:
         return out
 
     def set_step_kernel(self, kind):
-        """``"auto"`` (default), ``"register"`` or ``"stream"``: which kernel runs dl_step."""
-        vals = {"auto": N.DL_STEP_AUTO, "register": N.DL_STEP_REGISTER, "stream": N.DL_STEP_STREAM}
+        """``"auto"`` (default) or ``"register"``: which kernel runs dl_step."""
+        vals = {"auto": N.DL_STEP_AUTO, "register": N.DL_STEP_REGISTER}
         N.call("dl_set_option", self._h, N.DL_OPT_STEP_KERNEL, vals[kind])
 
     def set_host_prefetch(self, on):
@@ -218,16 +222,22 @@ class DeltaLog:
         """Store GDN/KDA log value factors b_i in bf16 (bf16 handles, empty log)."""
         N.call("dl_set_option", self._h, N.DL_OPT_LOG_B_BF16, 1 if on else 0)
 
+    def set_test_stall_log(self, on):
+        """Test of the error path only: steps arm their log barrier but copy
+        nothing, so every unit with a non-empty log times out (20 us), writes
+        nothing and raises DL_DEVERR_WAIT_TIMEOUT."""
+        N.call("dl_set_option", self._h, N.DL_OPT_TEST_STALL_LOG, 1 if on else 0)
+
     def set_value_tiles(self, n):
         """0 (automatic), 1, 2 or 4 value tiles (CTAs) per head in the register-tile step kernel."""
         N.call("dl_set_option", self._h, N.DL_OPT_VALUE_TILES, int(n))
 
     @property
     def last_step_kernel(self):
-        """Kernel used by the most recent step: ``"register"``, ``"stream"`` or ``None``."""
+        """Kernel used by the most recent step: ``"register"`` or ``None``."""
         k = ctypes.c_int()
         N.call("dl_last_step_kernel", self._h, ctypes.byref(k))
-        return {N.DL_STEP_REGISTER: "register", N.DL_STEP_STREAM: "stream"}.get(k.value)
+        return {N.DL_STEP_REGISTER: "register"}.get(k.value)
 
     @property
     def log_len(self):

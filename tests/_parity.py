@@ -49,7 +49,7 @@ def run_gpu(op, S0, seq, u, M, dtype, eager=False, record_merges=True, kernel="a
             log_b_bf16=False):
     """Run T steps through the library; returns (o[T,B,H,dv], {t: Sbar}, final logical S).
 
-    ``kernel`` selects the dl_step kernel ("auto", "register" or "stream")."""
+    ``kernel`` selects the dl_step kernel ("auto" or "register")."""
     from recurrent_state_update_deltalog_b200 import DeltaLog
     B, H, dk, dv = S0.shape
     T = seq["k"].shape[0]

@@ -14,7 +14,7 @@ pytestmark = pytest.mark.gpu
 OPS = ["gdn", "kda", "rwkv6"]
 
 
-KERNELS = ["register", "stream"]
+KERNELS = ["auto", "register"]
 
 
 def _check_run(op, B, H, dk, dv, M, T, dtype, eager=False, seed=0, kernel="auto", tiles=0):
@@ -49,36 +49,27 @@ def test_deferred_shapes(op, dims, dtype, kernel):
     _check_run(op, 3, 5, dims[0], dims[1], 4, 11, dtype, kernel=kernel)
 
 
-@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("op", OPS)
 @pytest.mark.parametrize("M", [1, 2, 3, 8, 16, 32, 33, 64])
-def test_deferred_every_M(op, M, kernel):
-    T = min(2 * M + 3, 70)
-    if kernel == "stream" and (M == 64 or (M >= 32 and op != "gdn")):
-        # A long per-key log does not fit the streaming kernel's shared memory
-        # next to its ring: forcing it is refused, AUTO falls back.
-        from recurrent_state_update_deltalog_b200 import DeltaLogError
-        with pytest.raises(DeltaLogError) as ei:
-            _check_run(op, 2, 3, 128, 128, M, T, torch.bfloat16, kernel="stream")
-        assert ei.value.status == -2
-        kernel = "auto"
-    _check_run(op, 2, 3, 128, 128, M, T, torch.bfloat16, kernel=kernel)
+def test_deferred_every_M(op, M):
+    _check_run(op, 2, 3, 128, 128, M, min(2 * M + 3, 70), torch.bfloat16)
 
 
 def test_step_kernel_selection_is_reported():
-    from recurrent_state_update_deltalog_b200 import DeltaLog
-    S0, seq, _ = make_inputs("gdn", 4, 8, 128, 128, 3, torch.bfloat16)
+    from recurrent_state_update_deltalog_b200 import DeltaLog, DeltaLogError
+    from recurrent_state_update_deltalog_b200 import _native as N
+    S0, seq, _ = make_inputs("gdn", 4, 8, 128, 128, 2, torch.bfloat16)
     dseq = to_device(seq, torch.bfloat16)
     h = DeltaLog(4, 8, 128, 128, 8, op="gdn")
     assert h.last_step_kernel is None
     h.step(*step_args("gdn", dseq, 0))
-    assert h.last_step_kernel in ("register", "stream")
-    h.set_step_kernel("stream")
-    h.step(*step_args("gdn", dseq, 1))
-    assert h.last_step_kernel == "stream"
-    h.set_step_kernel("register")
-    h.step(*step_args("gdn", dseq, 2))
     assert h.last_step_kernel == "register"
+    h.set_step_kernel("register")
+    h.step(*step_args("gdn", dseq, 1))
+    assert h.last_step_kernel == "register"
+    with pytest.raises(DeltaLogError) as ei:   # no other step kernel exists
+        N.call("dl_set_option", h._h, N.DL_OPT_STEP_KERNEL, 2)
+    assert ei.value.status == -1
     h.close()
 
 
@@ -100,11 +91,10 @@ def test_value_tiles_every_M(op, M, tiles):
 
 
 @pytest.mark.parametrize("op", OPS)
-def test_stream_kernel_many_units_per_cta(op):
-    """More units than persistent CTAs: every CTA walks several units and the
-    ring wraps many times (B*H = 2000 > 2 x SM count)."""
-    _check_run(op, 125, 16, 64, 64, 4, 9, torch.bfloat16, kernel="stream")
-    _check_run(op, 40, 16, 128, 128, 3, 7, torch.bfloat16, kernel="stream")
+def test_many_units_per_sm(op):
+    """More units than resident CTAs: several waves per launch (B*H = 2000)."""
+    _check_run(op, 125, 16, 64, 64, 4, 9, torch.bfloat16)
+    _check_run(op, 40, 16, 128, 128, 3, 7, torch.bfloat16)
 
 
 @pytest.mark.parametrize("op", OPS)
@@ -297,10 +287,9 @@ def test_extreme_gates_fp32(op):
     assert relerr(final, S_ref) < TOL[torch.float32]
 
 
-def test_unaligned_inputs_fall_back_or_refuse():
-    """q/k/v views offset by one element: AUTO runs the register kernel (same
-    result), STREAM refuses with DL_ERR_UNSUPPORTED."""
-    from recurrent_state_update_deltalog_b200 import DeltaLog, DeltaLogError
+def test_inputs_aligned_to_their_element_only():
+    """q/k/v views offset by one element (2-byte aligned) give the same result."""
+    from recurrent_state_update_deltalog_b200 import DeltaLog
     B, H, d, M, T = 2, 4, 64, 4, 6
     S0, seq, _ = make_inputs("gdn", B, H, d, d, T, torch.bfloat16)
     o_ref, S_ref, _ = run_oracle("gdn", S0, seq, None)
@@ -317,10 +306,6 @@ def test_unaligned_inputs_fall_back_or_refuse():
         outs.append(h.step(shifted["q"][t], shifted["k"][t], shifted["v"][t],
                            dseq["log_decay"][t], dseq["beta"][t]).float().cpu().numpy())
     assert relerr(np.stack(outs), o_ref) < 5e-3
-    h.set_step_kernel("stream")
-    with pytest.raises(DeltaLogError) as ei:
-        h.step(shifted["q"][0], shifted["k"][0], shifted["v"][0], dseq["log_decay"][0], dseq["beta"][0])
-    assert ei.value.status == -2
     h.close()
 
 
@@ -561,6 +546,83 @@ def test_slot_index_map_eager(op):
     _run_indexed(op, (128, 128), 1, torch.bfloat16, eager=True)
 
 
+def _run_hold(op, dims, M, dtype, eager=False, tiles=0, log_b_bf16=False):
+    """Slots that sit tokens out: named as slot | HOLD, across merge steps and
+    from the first or up to the last token.  The oracle does not advance a held
+    slot; its output row stays untouched and its state must equal the one it
+    paused with at every token, and every active output must match."""
+    from recurrent_state_update_deltalog_b200 import DeltaLog
+    B, H, T = 7, 3, 21
+    dk, dv = dims
+    S0, seq, u = make_inputs(op, B, H, dk, dv, T, dtype, seed=9)
+    tol = TOL[dtype]
+    rng = np.random.default_rng(21)
+    paused = {1: range(2, 9), 3: range(5, 7), 4: range(0, 3), 5: range(16, T), 0: (M - 1, 10)}
+    h = DeltaLog(B, H, dk, dv, M, op=op, dtype=dtype)
+    h.set_value_tiles(tiles)
+    h.set_log_b_bf16(log_b_bf16)
+    h.load_state(torch.from_numpy(S0).cuda())
+    if u is not None:
+        h.set_bonus(torch.from_numpy(u).cuda())
+    S_ref = S0.astype(np.float64)
+    try:
+        for t in range(T):
+            held = [b for b, r in paused.items() if t in r]
+            active = [b for b in range(B) if b not in held]
+            rows = list(rng.permutation(active)) + [b | DeltaLog.HOLD for b in held]
+            order = rng.permutation(len(rows))
+            idx = [int(rows[i]) for i in order]
+            plain = [b & ~DeltaLog.HOLD if b >= 0 else b for b in idx]
+            dseq = to_device(_batch(seq, t, plain), dtype)
+            sentinel = 7.0
+            out = torch.full((len(idx), H, dv), sentinel, dtype=dtype, device="cuda")
+            d_idx = torch.tensor(idx, dtype=torch.int32, device="cuda")
+            (h.eager_step if eager else h.step)(*step_args(op, dseq, 0), out=out, slot_idx=d_idx)
+            o_all, S_all = _oracle_step(op, S_ref, seq, t, u)
+            got = out.float().cpu().numpy()
+            act_rows = [r for r, b in enumerate(idx) if 0 <= b < B]
+            idle_rows = [r for r, b in enumerate(idx) if not 0 <= b < B]
+            assert np.all(got[idle_rows] == sentinel), t
+            assert relerr(got[act_rows], o_all[[idx[r] for r in act_rows]]) < tol, t
+            S_ref[active] = S_all[active]
+            for b in held:    # a held slot reads back exactly as it paused
+                assert relerr(h.slot_read(b).cpu().numpy(), S_ref[b]) < tol, (t, b)
+        assert (h.log_len == T % M) or eager
+        for b in range(B):
+            assert relerr(h.slot_read(b).cpu().numpy(), S_ref[b]) < tol, b
+        h.merge()
+        assert relerr(h.read_state().cpu().numpy(), S_ref) < tol
+        h.check_device()
+    finally:
+        h.close()
+
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("dims,M", [((64, 64), 3), ((128, 128), 4), ((128, 128), 8), ((64, 128), 5)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_held_slots(op, dims, M, dtype):
+    _run_hold(op, dims, M, dtype)
+
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("tiles", [2, 4])
+def test_held_slots_value_tiles(op, tiles):
+    """Held slots with each head split over several CTAs (each writes its
+    columns of the null entry; the first writes a_n and the snapshot)."""
+    _run_hold(op, (128, 128), 4, torch.bfloat16, tiles=tiles)
+
+
+@pytest.mark.parametrize("op", ["gdn", "kda"])
+def test_held_slots_bf16_log(op):
+    _run_hold(op, (128, 128), 8, torch.bfloat16, log_b_bf16=True)
+
+
+@pytest.mark.parametrize("op", OPS)
+def test_held_slots_eager(op):
+    """The dense kernel leaves a held slot's state as it is."""
+    _run_hold(op, (64, 64), 1, torch.bfloat16, eager=True)
+
+
 def test_slot_index_out_of_range_raises_device_flag():
     """An index past the pool skips its row and raises the device error word;
     the other rows are computed as usual."""
@@ -584,7 +646,10 @@ def test_slot_index_out_of_range_raises_device_flag():
 
 
 def test_slot_index_map_arguments():
+    import ctypes
+
     from recurrent_state_update_deltalog_b200 import DeltaLog, DeltaLogError
+    from recurrent_state_update_deltalog_b200 import _native as N
     h = DeltaLog(2, 2, 64, 64, 4, op="gdn", dtype=torch.float32)
     z = torch.zeros((3, 2, 64), device="cuda")
     g = torch.zeros((3, 2), device="cuda")
@@ -594,11 +659,10 @@ def test_slot_index_map_arguments():
     ge = torch.empty((0, 2), device="cuda")
     h.step(e, e, e, ge, ge, slot_idx=torch.empty(0, dtype=torch.int32, device="cuda"))  # no-op
     assert h.log_len == 0
-    h.set_step_kernel("stream")
-    one = torch.zeros((1, 2, 64), device="cuda")
-    with pytest.raises(DeltaLogError):
-        h.step(one, one, one, torch.zeros((1, 2), device="cuda"), torch.zeros((1, 2), device="cuda"),
-               slot_idx=torch.zeros(1, dtype=torch.int32, device="cuda"))
+    with pytest.raises(DeltaLogError):                 # a map pointer that is not 4-byte aligned
+        N.call("dl_step_indexed", h._h, ctypes.c_void_p(torch.zeros(2, dtype=torch.int32, device="cuda")
+                                                         .data_ptr() + 2), 1, None, None, None, None, None,
+               None, None)
     h.close()
 
 
@@ -668,9 +732,6 @@ def test_log_b_bf16_differs_from_fp32_log_and_option_rules():
         h.set_log_b_bf16(True)
     h.merge()
     h.set_log_b_bf16(True)
-    h.set_step_kernel("stream")
-    with pytest.raises(DeltaLogError):
-        h.step(*step_args(op, dseq, 1))
     h.close()
 
 
@@ -678,3 +739,51 @@ def test_log_b_bf16_differs_from_fp32_log_and_option_rules():
 def test_log_b_bf16_with_slot_map_and_admission(op):
     """The bf16 b-log under a slot index map with eviction and admission."""
     _run_indexed(op, (128, 128), 8, torch.bfloat16, log_b_bf16=True)
+
+
+# ---- failure paths made on purpose (no fault: a wait that nothing completes) ------
+
+@pytest.mark.parametrize("M", [4, 2])
+def test_stalled_log_wait_times_out_and_reports(M):
+    """With DL_OPT_TEST_STALL_LOG the log barrier expects bytes that no copy
+    delivers: every unit of the step gives up after its bounded wait, writes
+    nothing (output rows keep their sentinel; at M = 2 the step is a merge and
+    the base keeps its value) and dl_check_device reports the timeout bit.  The
+    context stays usable: a fresh handle then matches the oracle."""
+    from recurrent_state_update_deltalog_b200 import DeltaLog, DeltaLogError
+    op, B, H, d, T = "gdn", 3, 4, 64, 6
+    S0, seq, u = make_inputs(op, B, H, d, d, T, torch.bfloat16, seed=4)
+    dseq = to_device(seq, torch.bfloat16)
+    h = DeltaLog(B, H, d, d, M, op=op)
+    h.load_state(torch.from_numpy(S0).cuda())
+    h.step(*step_args(op, dseq, 0))                  # n = 0: no log to wait for
+    h.check_device()
+    h.set_test_stall_log(True)
+    out = torch.full((B, H, d), 7.0, dtype=torch.bfloat16, device="cuda")
+    h.step(*step_args(op, dseq, 1), out=out)         # n = 1: every unit stalls
+    with pytest.raises(DeltaLogError) as ei:
+        h.check_device()
+    assert ei.value.status == -5 and "0x1" in str(ei.value)
+    assert torch.all(out == 7.0)
+    if M == 2:   # the stalled merge left the base alone (step 0 only appended)
+        assert torch.equal(h.read_state().cpu(), torch.from_numpy(S0))
+    h.check_device()                                 # the word was cleared
+    h.close()
+    o, _, final = run_gpu(op, S0, seq, u, M, torch.bfloat16)
+    o_ref, S_ref, _ = run_oracle(op, S0, seq, u)
+    assert relerr(o, o_ref) < 5e-3 and relerr(final, S_ref) < 5e-3
+
+
+def test_create_too_large_returns_oom_and_leaks_nothing():
+    """A handle whose state cannot be allocated (4.4 TB) fails with DL_ERR_OOM,
+    frees what it took, and a small handle works afterwards."""
+    from recurrent_state_update_deltalog_b200 import DeltaLog, DeltaLogError
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    with pytest.raises(DeltaLogError) as ei:
+        DeltaLog(1 << 20, 64, 128, 128, 8, op="gdn")
+    assert ei.value.status == -4
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    _check_run("gdn", 2, 3, 64, 64, 4, 9, torch.bfloat16)

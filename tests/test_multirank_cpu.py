@@ -79,3 +79,18 @@ def test_job_aggregate_scales_with_replicas(world):
     import bench
     one = bench.job_tokens_per_s(128, 256, 10, 1, 20.0)
     assert bench.job_tokens_per_s(128, 256, 10, world, 20.0) == pytest.approx(world * one)
+
+
+def test_cpu_baseline_uses_every_core_and_reports_one_core():
+    """cpu_baseline runs the oracle on spawned worker processes (one per core)
+    and on one core alone, over the same per-worker sample."""
+    import argparse
+
+    import bench
+    a = argparse.Namespace(op="gdn", B=4, H=4, d=64, M=4, tokens=8, seed=0)
+    cb = bench.cpu_baseline(a)
+    cores = min(bench.host_cores(), bench.ORACLE_MAX_WORKERS)
+    assert cb["kind"] == "oracle" and cb["cores"] == cores and cb["value"] > 0
+    assert cb["cpu_model"] and cb["single_core"]["value"] > 0
+    assert f"{cores} worker process(es)" in cb["sample"]
+    assert cb["sample"].split(",", 1)[1] == cb["single_core"]["sample"].split(",", 1)[1]
