@@ -10,8 +10,8 @@ per step * steps / time) summed over all ranks, inputs resident in HBM.
 
 For the metric's headline the same line also carries, under "workloads",
 KDA (B=128, H=32, d=128) and RWKV6 (B=128, H=64, d=64) at M=8 with their
-eager-kernel and e2e figures, and under "sweep" the headline at M = 4 and 16
-(M = 1 is the "eager" key).  ``cpu_baseline`` times the fp64 oracle on the
+eager-kernel and e2e figures (and once more with fp16 per-key log-gates),
+and under "sweep" the headline at M = 4 and 16 (M = 1 is the "eager" key).  ``cpu_baseline`` times the fp64 oracle on the
 host cores (one spawned worker process per core, each on its own sample of
 the workload) and on one core alone.
 
@@ -79,6 +79,8 @@ def parse():
                          "of decode; one JSON line, ALU roofline")
     ap.add_argument("--log-b-bf16", action="store_true",
                     help="store GDN/KDA log value factors b_i in bf16 (DL_OPT_LOG_B_BF16)")
+    ap.add_argument("--log-lam-f16", action="store_true",
+                    help="store KDA/RWKV6 per-key decay metadata as fp16 log-gates (DL_OPT_LOG_LAM_F16)")
     ap.add_argument("--slot-map", action="store_true",
                     help="run every token through the slot index map: batch row r on slot perm_t[r], "
                          "a fresh random permutation of the B slots per pool token")
@@ -107,6 +109,7 @@ def parse():
 
 def workload_name(a):
     tail = "_logb_bf16" if getattr(a, "log_b_bf16", False) and a.op != "rwkv6" else ""
+    tail += "_lam_f16" if getattr(a, "log_lam_f16", False) and a.op != "gdn" else ""
     return f"{a.op}_decode_b{a.B}_h{a.H}_d{a.d}_m{a.M}_bf16{tail}"
 
 
@@ -114,16 +117,17 @@ def workload_name(a):
 # algorithmic bytes (what the method must move; no cache effects)
 # ---------------------------------------------------------------------------
 
-def entry_bytes(op, dk, dv, es=2, bb=None):
+def entry_bytes(op, dk, dv, es=2, bb=None, lb=4):
     """Bytes of one log entry: a_i (input dtype) + b_i + Lam_i.  bb: bytes of
-    one b_i element (default: the input dtype for RWKV6, fp32 otherwise)."""
+    one b_i element (default: the input dtype for RWKV6, fp32 otherwise); lb:
+    bytes of one per-key Lam element (4, or 2 for fp16 log-gates)."""
     a = dk * es
     b = dv * (bb or (es if op == "rwkv6" else 4))
-    lam = 4 if op == "gdn" else 4 * dk
+    lam = 4 if op == "gdn" else lb * dk
     return a + b + lam
 
 
-def launch_bytes(op, kind, B, H, dk, dv, n=0, es=2, bb=None):
+def launch_bytes(op, kind, B, H, dk, dv, n=0, es=2, bb=None, lb=4):
     """Algorithmic HBM bytes of one launch over all B*H (slot, head) units.
 
     kind: "append" (n entries in the log), "merge" (n entries before the step),
@@ -137,30 +141,30 @@ def launch_bytes(op, kind, B, H, dk, dv, n=0, es=2, bb=None):
     unit += (2 * dk + dv) * es + dv * es                      # q|r, k, v in; o out
     unit += {"gdn": 8, "kda": 4 * dk + 4, "rwkv6": 4 * dk}[op]  # gates
     if kind != "eager":
-        unit += n * entry_bytes(op, dk, dv, es, bb)
+        unit += n * entry_bytes(op, dk, dv, es, bb, lb)
     if kind == "append":
-        unit += entry_bytes(op, dk, dv, es, bb)
+        unit += entry_bytes(op, dk, dv, es, bb, lb)
     total = unit * B * H
     if op == "rwkv6":
         total += H * dk * 4
     return total
 
 
-def step_bytes(op, B, H, d, M, tokens, es=2, bb=None):
+def step_bytes(op, B, H, d, M, tokens, es=2, bb=None, lb=4):
     if M == 1:
         return tokens * launch_bytes(op, "eager", B, H, d, d, 0, es)
-    per_cycle = sum(launch_bytes(op, "append", B, H, d, d, n, es, bb) for n in range(M - 1))
-    per_cycle += launch_bytes(op, "merge", B, H, d, d, M - 1, es, bb)
+    per_cycle = sum(launch_bytes(op, "append", B, H, d, d, n, es, bb, lb) for n in range(M - 1))
+    per_cycle += launch_bytes(op, "merge", B, H, d, d, M - 1, es, bb, lb)
     return per_cycle * (tokens // M)
 
 
-def write_bytes_per_token(op, B, H, d, M, es=2, bb=None):
+def write_bytes_per_token(op, B, H, d, M, es=2, bb=None, lb=4):
     """Algorithmic HBM write bytes per slot-token (all heads), averaged over a cycle."""
     state_w = 4 * d * d
     io_w = d * es
     if M == 1:
         return H * (state_w + io_w)
-    ent = entry_bytes(op, d, d, es, bb)
+    ent = entry_bytes(op, d, d, es, bb, lb)
     per_cycle = (M - 1) * (io_w + ent) + (io_w + state_w)
     return H * per_cycle / M
 
@@ -441,6 +445,7 @@ def run_gpu(a, rank, world, local_rank):
     op, B, H, d, M = a.op, a.B, a.H, a.d, a.M
     seed = rank_seed(a.seed, rank)
     bb = 2 if a.log_b_bf16 else None           # b_i element bytes in the log
+    lb = 2 if a.log_lam_f16 and op != "gdn" else 4   # per-key Lam element bytes in the log
     es = 2
 
     # inputs: a pool of distinct tokens resident in HBM (> L2), cycled
@@ -478,6 +483,8 @@ def run_gpu(a, rank, world, local_rank):
         h.set_value_tiles(a.tiles)
         if a.log_b_bf16 and m > 1:
             h.set_log_b_bf16(True)
+        if a.log_lam_f16 and m > 1:
+            h.set_log_lam_f16(True)
         h.load_state(S0)
         if u is not None:
             h.set_bonus(u)
@@ -605,14 +612,14 @@ def run_gpu(a, rank, world, local_rank):
     # per-launch durations of the dominant (append) kernel, second pass
     launches = timed(M, per_launch=True)[1] if M > 1 and not a.graph else None
     value = job_tokens_per_s(B, a.tokens, a.steps, world, ms)
-    sb = step_bytes(op, B, H, d, M, a.tokens, bb=bb)
+    sb = step_bytes(op, B, H, d, M, a.tokens, bb=bb, lb=lb)
     result["value"] = value
     result["ms"] = ms
 
     if launches:
         count = sum(len(ns) for _, ns in launches)
         dur = sum(t for t, _ in launches) / count
-        alg = sum(launch_bytes(op, "append", B, H, d, d, n, bb=bb) for _, ns in launches for n in ns) / count
+        alg = sum(launch_bytes(op, "append", B, H, d, d, n, bb=bb, lb=lb) for _, ns in launches for n in ns) / count
         dominant = "deltalog_step_kernel (append)"
     else:   # average over every launch of the step (graph replay or M = 1)
         dur = ms / (a.steps * a.tokens)
@@ -641,11 +648,11 @@ def run_gpu(a, rank, world, local_rank):
         if a.tokens % mv:
             continue
         sms, _ = timed(mv)
-        sbb = step_bytes(op, B, H, d, mv, a.tokens, bb=bb)
+        sbb = step_bytes(op, B, H, d, mv, a.tokens, bb=bb, lb=lb)
         gbs = sbb / (sms / a.steps / 1e3) / 1e9
         sweep[str(mv)] = {"value": B * a.tokens * a.steps * world / (sms / 1e3),
                           "ms_per_step": sms / a.steps, "gbs": gbs, "frac": gbs / peak,
-                          "write_bytes_per_token": write_bytes_per_token(op, B, H, d, mv, bb=bb)}
+                          "write_bytes_per_token": write_bytes_per_token(op, B, H, d, mv, bb=bb, lb=lb)}
     if sweep:
         extra["sweep"] = sweep
 
@@ -695,6 +702,7 @@ def run_gpu(a, rank, world, local_rank):
                    "admit_every_tokens": a.admit_every or None,
                    "slot_map": "random permutation per token" if a.slot_map else None,
                    "log_b": "bf16" if (a.log_b_bf16 or op == "rwkv6") else "fp32",
+                   "log_lam": "fp32 scalar" if op == "gdn" else ("fp16 log-gates" if a.log_lam_f16 else "fp32"),
                    "input_pool_tokens": a.pool, "seed": a.seed,
                    "l2": (f"inputs larger than L2 (state {4 * B * H * d * d / 1e6:.0f} MB)"
                           if 4 * B * H * d * d > L2_BYTES else
@@ -702,7 +710,7 @@ def run_gpu(a, rank, world, local_rank):
                    "parallelism": "replicas" if world == 1 else f"replicas x{world} (B per rank)"},
         "roofline": roofline,
         "gpu_launches": a.steps * a.tokens,
-        "write_bytes_per_token": write_bytes_per_token(op, B, H, d, M, bb=bb),
+        "write_bytes_per_token": write_bytes_per_token(op, B, H, d, M, bb=bb, lb=lb),
         "clocks": clocks,
         "e2e": e2e,
     }
@@ -714,14 +722,17 @@ def run_gpu(a, rank, world, local_rank):
 # KDA and RWKV6 at their decode configurations, and the headline's M sweep.
 METRIC_HEADLINE = {"op": "gdn", "B": 256, "H": 32, "d": 128, "M": 8}
 METRIC_WORKLOADS = [{"op": "kda", "B": 128, "H": 32, "d": 128, "M": 8},
-                    {"op": "rwkv6", "B": 128, "H": 64, "d": 64, "M": 8}]
+                    {"op": "rwkv6", "B": 128, "H": 64, "d": 64, "M": 8},
+                    {"op": "kda", "B": 128, "H": 32, "d": 128, "M": 8, "log_lam_f16": True},
+                    {"op": "rwkv6", "B": 128, "H": 64, "d": 64, "M": 8, "log_lam_f16": True}]
 METRIC_SWEEP = "4,16"
 
 
 def is_metric_headline(a):
     """The plain headline configuration (no serving or tuning switches)."""
     return (all(getattr(a, k) == v for k, v in METRIC_HEADLINE.items()) and not a.slot_map
-            and not a.admit_every and not a.graph and not a.log_b_bf16 and a.kernel == "auto"
+            and not a.admit_every and not a.graph and not a.log_b_bf16 and not a.log_lam_f16
+            and a.kernel == "auto"
             and a.tiles == 0 and not a.no_pdl and not getattr(a, "m_auto", False))
 
 
@@ -755,6 +766,8 @@ def run_decode(a, rank, world, local_rank):
             for k, v in w.items():
                 setattr(sub, k, v)
             sub.sweep = ""
+            if sub.log_lam_f16:   # the same workload with compact snapshots: no second eager or e2e run
+                sub.no_eager = sub.no_e2e = True
             sub_line = run_gpu(sub, rank, world, local_rank)
             if sub_line is not None:
                 extras[sub_line["config"]["workload"]] = workload_summary(sub_line)

@@ -249,6 +249,21 @@ int dl_read_state(dl_t h, float* S_out, void* stream);
  * to fp32 rounding only).  bf16-input handles only (DL_ERR_UNSUPPORTED
  * otherwise); a no-op for RWKV6, whose log already holds raw bf16 v_i.
  * Changeable only while the log is empty (DL_ERR_STATE otherwise). */
+/* DL_OPT_LOG_LAM_F16 (0 or 1, default 0): store the per-key decay metadata of
+ * KDA/RWKV6 log entries as each step's log-gates in fp16 instead of fp32
+ * cumulative snapshots Lam_i: 1024 instead of 1280 bytes per entry for KDA
+ * at d = 128 (768 with DL_OPT_LOG_B_BF16), 384 instead of 512 for RWKV6 at
+ * d = 64.  The pages name the per-key metadata as the reason KDA and RWKV6
+ * gain less than GDN (DeltaLog technical summary, gist.science, section
+ * "Results").  Each kernel that reads a log rebuilds the fp32 snapshots
+ * Lam_i = g_0 + ... + g_i in entry order from the staged gates; the current
+ * token's own gate enters unrounded.  A rounded gate errs by at most 2^-11
+ * of itself, so a snapshot errs by at most 2^-11 |Lam_i| and a decay factor
+ * e^{Lam} by at most e^{Lam} |Lam| 2^-11 <= 2^-11/e of the state (outputs
+ * then match the eager recurrence to a few 1e-4, not to fp32 rounding).
+ * bf16-input handles only (DL_ERR_UNSUPPORTED otherwise); a no-op for GDN,
+ * whose snapshot is one scalar per entry.  Changeable only while the log is
+ * empty (DL_ERR_STATE otherwise). */
 /* DL_OPT_PREFILL_KERNEL picks the kernel behind dl_prefill:
  *   DL_PREFILL_AUTO (default): the chunked kernel for bf16-input handles
  *     whose prompts average at least 16 tokens (GDN, RWKV6) or 24 (KDA) at
@@ -278,7 +293,8 @@ enum dl_option {
   DL_OPT_VALUE_TILES = 3,
   DL_OPT_LOG_B_BF16 = 4,
   DL_OPT_PREFILL_KERNEL = 5,
-  DL_OPT_TEST_STALL_LOG = 6
+  DL_OPT_TEST_STALL_LOG = 6,
+  DL_OPT_LOG_LAM_F16 = 7
 };
 enum dl_prefill_kernel { DL_PREFILL_AUTO = 0, DL_PREFILL_RECURRENT = 1, DL_PREFILL_CHUNKED = 2 };
 enum dl_step_kernel { DL_STEP_AUTO = 0, DL_STEP_REGISTER = 1 };

@@ -26,6 +26,7 @@ DL_OPT_VALUE_TILES = 3
 DL_OPT_LOG_B_BF16 = 4
 DL_OPT_PREFILL_KERNEL = 5
 DL_OPT_TEST_STALL_LOG = 6
+DL_OPT_LOG_LAM_F16 = 7
 DL_PREFILL_AUTO, DL_PREFILL_RECURRENT, DL_PREFILL_CHUNKED = 0, 1, 2
 DL_STEP_AUTO, DL_STEP_REGISTER = 0, 1
 STATUS = {0: "DL_OK", -1: "DL_ERR_ARG", -2: "DL_ERR_UNSUPPORTED", -3: "DL_ERR_CUDA",

@@ -55,6 +55,7 @@ struct dl_handle {
   int prefill_kernel;       // DL_OPT_PREFILL_KERNEL (DL_PREFILL_*)
   int last_prefill;         // DL_PREFILL_* used by the last dl_prefill
   int stall_log;            // DL_OPT_TEST_STALL_LOG
+  int log_lam_f16;          // DL_OPT_LOG_LAM_F16
 };
 
 namespace {
@@ -103,6 +104,10 @@ size_t lam_per_entry(const dl_handle* h) { return h->op == DL_GDN ? 1 : static_c
 size_t lam_unit_floats(const dl_handle* h) {
   return h->op == DL_GDN ? static_cast<size_t>(dl::gdn_lam_stride(h->Mcap)) : static_cast<size_t>(h->Mcap) * h->dk;
 }
+// Bytes of one Lam element in the log: per-key snapshots are fp16 log-gates
+// with DL_OPT_LOG_LAM_F16 (the buffer is sized for fp32, so the option needs
+// no reallocation); GDN keeps fp32 scalars.
+size_t lam_esize(const dl_handle* h) { return h->op != DL_GDN && h->log_lam_f16 ? 2 : 4; }
 // Element size of b_i in the log: RWKV6 keeps raw v_i in the input dtype;
 // GDN/KDA keep fp32, or bf16 with DL_OPT_LOG_B_BF16.  The buffer is sized
 // for fp32 (logb_alloc_esize) so that the option needs no reallocation.
@@ -157,6 +162,7 @@ dl::LaunchShape shape_of(const dl_handle* h, long units = 0) {
   s.max_n = h->n;
   s.units = s.BH;
   s.blow = h->log_b_bf16 && h->op != DL_RWKV6;
+  s.lamc = h->log_lam_f16 && h->op != DL_GDN;
   return s;
 }
 
@@ -216,7 +222,7 @@ cudaError_t zero_slot_log(const dl_handle* h, int b, cudaStream_t s) {
   const size_t units = static_cast<size_t>(h->H), first = static_cast<size_t>(b) * units;
   const size_t a_unit = static_cast<size_t>(h->Mcap) * h->dk * h->esize;
   const size_t b_unit = static_cast<size_t>(h->Mcap) * h->dv * logb_esize(h);
-  const size_t l_unit = lam_unit_floats(h) * sizeof(float);
+  const size_t l_unit = lam_unit_floats(h) * lam_esize(h);
   cudaError_t e = cudaMemsetAsync(static_cast<char*>(h->logA) + first * a_unit, 0, units * a_unit, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(static_cast<char*>(h->logB) + first * b_unit, 0, units * b_unit, s);
   if (e == cudaSuccess)
@@ -616,6 +622,7 @@ int dl_prefill(dl_t h, const int* slot_idx, int rows, const int* cu_seqlens, lon
   a.Mcap = h->Mcap;
   a.n = h->n;
   a.b_esize = static_cast<int>(logb_esize(h));
+  a.lam_esize = static_cast<int>(lam_esize(h));
   a.zero_state = zero ? 1 : 0;
   cudaError_t e = launch_prefill(h, a, rows, s);
   if (e == cudaErrorNotSupported)
@@ -809,6 +816,13 @@ int dl_set_option(dl_t h, int option, int value) {
       if (value != h->log_b_bf16 && h->n != 0)
         return fail(DL_ERR_STATE, "change the b-log precision only with an empty log (call dl_merge)");
       h->log_b_bf16 = value;
+      return DL_OK;
+    case DL_OPT_LOG_LAM_F16:
+      if (value != 0 && value != 1) return fail(DL_ERR_ARG, "bad log-lam-f16 value %d", value);
+      if (value && h->dtype != DL_BF16) return fail(DL_ERR_UNSUPPORTED, "fp16 log-gates need bf16 inputs");
+      if (value != h->log_lam_f16 && h->n != 0)
+        return fail(DL_ERR_STATE, "change the snapshot precision only with an empty log (call dl_merge)");
+      h->log_lam_f16 = value;
       return DL_OK;
     case DL_OPT_TEST_STALL_LOG:
       if (value != 0 && value != 1) return fail(DL_ERR_ARG, "bad stall-log value %d", value);

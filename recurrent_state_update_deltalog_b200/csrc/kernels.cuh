@@ -28,6 +28,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -206,27 +207,56 @@ __host__ __device__ constexpr int gdn_lam_stride(int Mcap) { return (Mcap + 3) &
 // Shared-memory image of a (slot, head)'s log, staged by TMA bulk copies.
 // Byte layout (every region starts 16-byte aligned):
 //   A   n x DK input dtype     a_i = k_i
-//   L   n x DK fp32            Lam_i (KDA / RWKV6 only; GDN keeps n scalars apart)
+//   L   n x DK fp32 | fp16     Lam_i (KDA / RWKV6 only; GDN keeps n scalars
+//                              apart); LAMC: the step's log-gates g_i in fp16
 //   B   n x DV (fp32 | input)  b_i (RWKV6: raw v_i in the input dtype; BLOW:
 //                              GDN/KDA b_i rounded to bf16)
+// then, with LAMC, the fp32 snapshots rebuilt from the gates
+//   Lf  n x DK fp32            Lam_i = g_0 + ... + g_i, summed in entry order
 // followed, for merge-type launches, by the fp32 work arrays
 //   As  (n+1) x DK             ratio-scaled a_i, current entry last (ratio 1)
 //   Bc  DV                     the current entry's b_t
-template <int OP, int DK, int DV, typename TI, bool BLOW = false>
+// LAMC (compact per-key snapshots) stores each entry's own log-gate rather
+// than its cumulative snapshot.  A rounded gate errs by at most 2^-11 of
+// itself, so a rebuilt Lam_i errs by at most 2^-11 |Lam_i| and the decay
+// factor e^{Lam_i} by at most e^{Lam} |Lam| 2^-11 <= 2^-11 / e of the state:
+// rounding the snapshot itself would err by 2^-11 |Lam_i| in every ratio,
+// however close the two snapshots of the ratio are.
+template <int OP, int DK, int DV, typename TI, bool BLOW = false, bool LAMC = false>
 struct LogLayout {
   static_assert(!BLOW || (OP != OP_RWKV6 && std::is_same<TI, __nv_bfloat16>::value),
                 "a bf16 b-log is an option of bf16-input GDN/KDA handles");
+  static_assert(!LAMC || (OP != OP_GDN && std::is_same<TI, __nv_bfloat16>::value),
+                "compact snapshots are an option of bf16-input KDA/RWKV6 handles");
   using TB = typename std::conditional<OP == OP_RWKV6 || BLOW, TI, float>::type;
+  using TL = typename std::conditional<LAMC, __half, float>::type;   // L elements in the log
   static constexpr bool PERKEY = OP != OP_GDN;
   __host__ __device__ static constexpr size_t a_bytes(int n) { return size_t(n) * DK * sizeof(TI); }
-  __host__ __device__ static constexpr size_t l_bytes(int n) { return PERKEY ? size_t(n) * DK * 4 : 0; }
+  __host__ __device__ static constexpr size_t l_bytes(int n) { return PERKEY ? size_t(n) * DK * sizeof(TL) : 0; }
   __host__ __device__ static constexpr size_t b_bytes(int n) { return size_t(n) * DV * sizeof(TB); }
   __host__ __device__ static constexpr size_t staged(int n) { return a_bytes(n) + l_bytes(n) + b_bytes(n); }
+  __host__ __device__ static constexpr size_t table(int n) { return LAMC ? size_t(n) * DK * 4 : 0; }
   __host__ __device__ static constexpr size_t step_smem(int n, bool merge) {
-    return staged(n) + (merge ? size_t(n + 1) * DK * 4 + size_t(DV) * 4 : 0);
+    return staged(n) + table(n) + (merge ? size_t(n + 1) * DK * 4 + size_t(DV) * 4 : 0);
   }
-  __host__ __device__ static constexpr size_t materialize_smem(int n) { return staged(n) + size_t(n) * DK * 4; }
+  __host__ __device__ static constexpr size_t materialize_smem(int n) {
+    return staged(n) + table(n) + size_t(n) * DK * 4;
+  }
 };
+
+// LAMC: rebuild the fp32 snapshots Lam_i = g_0 + ... + g_i (i < n) from the
+// staged fp16 gates, one key per thread, always in entry order (so every
+// launch that reads a log sees the same values).  The caller synchronises.
+template <int DK>
+__device__ __forceinline__ void rebuild_snapshots(const __half* g, float* lam, int n) {
+  for (int j = threadIdx.x; j < DK; j += blockDim.x) {
+    float s = 0.f;
+    for (int i = 0; i < n; ++i) {
+      s += __half2float(g[i * DK + j]);
+      lam[i * DK + j] = s;
+    }
+  }
+}
 
 // Four consecutive log values as floats (fp32 or bf16 storage).
 __device__ __forceinline__ float4 load4f(const float* p) { return *reinterpret_cast<const float4*>(p); }
@@ -242,12 +272,13 @@ __device__ __forceinline__ float4 load4f(const __nv_bfloat16* p) {
 // into shared memory; completion arrives on `bar` (phase 0).  With `stall`
 // (a test of the timeout path) the barrier expects the bytes but no copy is
 // issued: the wait runs out with nothing in flight.
-template <int OP, int DK, int DV, typename TI, bool BLOW>
+template <int OP, int DK, int DV, typename TI, bool BLOW, bool LAMC>
 __device__ __forceinline__ void stage_log(unsigned char* smem, uint64_t* bar, const void* logA,
                                           const float* logLam, const void* logB, long sh, int Mcap,
                                           int n, bool stall = false) {
-  using LL = LogLayout<OP, DK, DV, TI, BLOW>;
+  using LL = LogLayout<OP, DK, DV, TI, BLOW, LAMC>;
   using TB = typename LL::TB;
+  using TLE = typename LL::TL;
   mbar_init(bar, 1);
   fence_mbar_init();
   if (n == 0) return;
@@ -255,7 +286,8 @@ __device__ __forceinline__ void stage_log(unsigned char* smem, uint64_t* bar, co
   if (stall) return;
   bulk_g2s(smem, static_cast<const TI*>(logA) + sh * Mcap * DK, static_cast<uint32_t>(LL::a_bytes(n)), bar);
   if (LL::PERKEY)
-    bulk_g2s(smem + LL::a_bytes(n), logLam + sh * Mcap * DK, static_cast<uint32_t>(LL::l_bytes(n)), bar);
+    bulk_g2s(smem + LL::a_bytes(n), reinterpret_cast<const TLE*>(logLam) + sh * Mcap * DK,
+             static_cast<uint32_t>(LL::l_bytes(n)), bar);
   bulk_g2s(smem + LL::a_bytes(n) + LL::l_bytes(n), static_cast<const TB*>(logB) + sh * Mcap * DV,
            static_cast<uint32_t>(LL::b_bytes(n)), bar);
 }
@@ -279,16 +311,19 @@ __device__ __forceinline__ bool wait_log(uint64_t* bar, int n, int* err, uint64_
 // adds nothing to its state and does not advance its decay, so its logical
 // state stays exact without reading Sbar.  Each value tile writes its b_n
 // columns; the first tile writes a_n and the snapshot.
-template <int OP, int DK, int DV, typename TI, bool BLOW>
+template <int OP, int DK, int DV, typename TI, bool BLOW, bool LAMC>
 __device__ __forceinline__ void hold_entry(const StepArgs& a, long sh, int col0, int dvt, int n) {
-  using TB = typename LogLayout<OP, DK, DV, TI, BLOW>::TB;
+  using TB = typename LogLayout<OP, DK, DV, TI, BLOW, LAMC>::TB;
   const int tid = threadIdx.x, nt = blockDim.x;
   TB* dstB = static_cast<TB*>(a.logB) + (sh * a.Mcap + n) * DV + col0;
   for (int c = tid; c < dvt; c += nt) dstB[c] = from_f<TB>(0.f);
   if (col0 != 0) return;
   TI* dstA = static_cast<TI*>(a.logA) + (sh * a.Mcap + n) * DK;
   for (int j = tid; j < DK; j += nt) dstA[j] = from_f<TI>(0.f);
-  if constexpr (OP != OP_GDN) {
+  if constexpr (LAMC) {   // a zero gate
+    __half* g = reinterpret_cast<__half*>(a.logLam) + (sh * a.Mcap + n) * DK;
+    for (int j = tid; j < DK; j += nt) g[j] = __float2half_rn(0.f);
+  } else if constexpr (OP != OP_GDN) {
     float* lam = a.logLam + sh * a.Mcap * DK;
     for (int j = tid; j < DK; j += nt) lam[n * DK + j] = n > 0 ? lam[(n - 1) * DK + j] : 0.f;
   } else if (tid == 0) {
@@ -304,12 +339,12 @@ __device__ __forceinline__ void hold_entry(const StepArgs& a, long sh, int col0,
 // tile recomputes the head's ReplayPrep coefficients and the first tile
 // appends the key-side entry.
 // ---------------------------------------------------------------------------
-template <int OP, int DK, int DV, typename TI, int MODE, int NSPLIT, bool MAP, bool BLOW>
+template <int OP, int DK, int DV, typename TI, int MODE, int NSPLIT, bool MAP, bool BLOW, bool LAMC>
 __global__ void __launch_bounds__(Tile<DK, DV / NSPLIT>::NT, Tile<DK, DV / NSPLIT>::MINB)
 deltalog_step_kernel(const StepArgs a) {
   constexpr int DVT = DV / NSPLIT;  // value-tile width owned by this CTA
   using TL = Tile<DK, DVT>;
-  using LL = LogLayout<OP, DK, DV, TI, BLOW>;
+  using LL = LogLayout<OP, DK, DV, TI, BLOW, LAMC>;
   using TB = typename LL::TB;
   constexpr bool DELTA = OP != OP_RWKV6;
   constexpr bool PERKEY = OP != OP_GDN;
@@ -354,14 +389,15 @@ deltalog_step_kernel(const StepArgs a) {
   // slot's log into its base at its unchanged logical state.
   const bool hold = MAP && ux.hold;
   if (!MERGE && hold) {
-    hold_entry<OP, DK, DV, TI, BLOW>(a, sh, col0, DVT, n);
+    hold_entry<OP, DK, DV, TI, BLOW, LAMC>(a, sh, col0, DVT, n);
     return;
   }
 
   const TI* sA = reinterpret_cast<const TI*>(s_dyn);
-  const float* sL = reinterpret_cast<const float*>(s_dyn + LL::a_bytes(n));
+  float* sLf = reinterpret_cast<float*>(s_dyn + LL::staged(n));       // LAMC: rebuilt snapshots
+  const float* sL = LAMC ? sLf : reinterpret_cast<const float*>(s_dyn + LL::a_bytes(n));
   const TB* sB = reinterpret_cast<const TB*>(s_dyn + LL::a_bytes(n) + LL::l_bytes(n));
-  float* As = reinterpret_cast<float*>(s_dyn + LL::staged(n));      // merge only
+  float* As = reinterpret_cast<float*>(s_dyn + LL::staged(n) + LL::table(n));   // merge only
   float* Bc = As + (n + 1) * DK;                                      // merge only
 
   // 1. The token's inputs and this head's Sbar tile into registers (all
@@ -400,19 +436,21 @@ deltalog_step_kernel(const StepArgs a) {
   if (MODE == MODE_APPEND) griddep_launch_dependents();
   if constexpr (!WAIT_FIRST) griddep_wait();
   if (tid == 0)
-    stage_log<OP, DK, DV, TI, BLOW>(s_dyn, &s_bar, a.logA, a.logLam, a.logB, sh, a.Mcap, n, a.stall_log != 0);
+    stage_log<OP, DK, DV, TI, BLOW, LAMC>(s_dyn, &s_bar, a.logA, a.logLam, a.logB, sh, a.Mcap, n,
+                                          a.stall_log != 0);
   if constexpr (!PERKEY) load_inputs();
 
   // 2. Decay snapshots: Lam_{t-1} from the newest entry, Lam_t = Lam_{t-1} +
-  // log-gate; GDN's scalar snapshots of every entry.
-  if (PERKEY) {
+  // log-gate; GDN's scalar snapshots of every entry.  (LAMC rebuilds the
+  // snapshots from the staged gates below, once the log has arrived.)
+  if (PERKEY && !LAMC) {
     const float* lamp = a.logLam + (sh * a.Mcap + (n > 0 ? n - 1 : 0)) * DK;
 #pragma unroll
     for (int m = 0; m < TL::KPL; ++m) {
       lp[m] = n > 0 ? lamp[lane + 32 * m] : 0.f;
       lt[m] = lp[m] + gt[m];
     }
-  } else {
+  } else if (!PERKEY) {
     if (tid < n) s_lam[tid] = a.logLam[sh * gdn_lam_stride(a.Mcap) + tid];
     const float lprev = n > 0 ? a.logLam[sh * gdn_lam_stride(a.Mcap) + (n - 1)] : 0.f;
 #pragma unroll
@@ -423,6 +461,15 @@ deltalog_step_kernel(const StepArgs a) {
   }
   __syncthreads();                              // barrier init and s_lam visible
   if (!wait_log(&s_bar, n, a.err, a.stall_log ? kStallWaitNs : kWaitNs)) return;
+  if constexpr (LAMC) {
+    rebuild_snapshots<DK>(reinterpret_cast<const __half*>(s_dyn + LL::a_bytes(n)), sLf, n);
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < TL::KPL; ++m) {
+      lp[m] = n > 0 ? sLf[(n - 1) * DK + lane + 32 * m] : 0.f;
+      lt[m] = lp[m] + gt[m];
+    }
+  }
 
   // 3. ReplayPrep: per-entry coefficients once per (slot, head).  Warp w takes
   // entries i = w, w+NW, ...; i == n is the current token (kappa).
@@ -486,7 +533,11 @@ deltalog_step_kernel(const StepArgs a) {
       for (int m = 0; m < TL::KPL; ++m) {
         const int j = lane + 32 * m;
         dstA[j] = kg[j];
-        if (PERKEY) a.logLam[(sh * a.Mcap + n) * DK + j] = lt[m];
+        if (LAMC) {
+          reinterpret_cast<__half*>(a.logLam)[(sh * a.Mcap + n) * DK + j] = __float2half_rn(gt[m]);
+        } else if (PERKEY) {
+          a.logLam[(sh * a.Mcap + n) * DK + j] = lt[m];
+        }
       }
       if (!PERKEY && lane == 0) a.logLam[sh * gdn_lam_stride(a.Mcap) + n] = lt[0];
     }
@@ -687,11 +738,11 @@ eager_step_kernel(const StepArgs a) {
 // otherwise).  Lam_last = Lam_{n-1}, the newest snapshot; a unit with an
 // empty log is copied through.
 // ---------------------------------------------------------------------------
-template <int OP, int DK, int DV, typename TI, bool BLOW>
+template <int OP, int DK, int DV, typename TI, bool BLOW, bool LAMC>
 __global__ void __launch_bounds__(Tile<DK, DV>::NT, Tile<DK, DV>::MINB)
 materialize_kernel(const MaterializeArgs a) {
   using TL = Tile<DK, DV>;
-  using LL = LogLayout<OP, DK, DV, TI, BLOW>;
+  using LL = LogLayout<OP, DK, DV, TI, BLOW, LAMC>;
   using TB = typename LL::TB;
   constexpr bool PERKEY = OP != OP_GDN;
   __shared__ __align__(16) float s_dec[DK];
@@ -717,27 +768,36 @@ materialize_kernel(const MaterializeArgs a) {
   const int n = a.n;
 
   const TI* sA = reinterpret_cast<const TI*>(s_dyn);
-  const float* sL = reinterpret_cast<const float*>(s_dyn + LL::a_bytes(n));
+  float* sLf = reinterpret_cast<float*>(s_dyn + LL::staged(n));       // LAMC: rebuilt snapshots
+  const float* sL = LAMC ? sLf : reinterpret_cast<const float*>(s_dyn + LL::a_bytes(n));
   const TB* sB = reinterpret_cast<const TB*>(s_dyn + LL::a_bytes(n) + LL::l_bytes(n));
-  float* As = reinterpret_cast<float*>(s_dyn + LL::staged(n));
+  float* As = reinterpret_cast<float*>(s_dyn + LL::staged(n) + LL::table(n));
 
   const float* Sp = a.Sin + sh * (DK * DV);
   float4 st[TL::RPT];
 #pragma unroll
   for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + (rg * TL::RPT + j) * DV + 4 * c4);
-  if (tid == 0) stage_log<OP, DK, DV, TI, BLOW>(s_dyn, &s_bar, a.logA, a.logLam, a.logB, sh, a.Mcap, n);
+  if (tid == 0) stage_log<OP, DK, DV, TI, BLOW, LAMC>(s_dyn, &s_bar, a.logA, a.logLam, a.logB, sh, a.Mcap, n);
 
   float ll[TL::KPL];
+  if constexpr (!LAMC) {
 #pragma unroll
-  for (int m = 0; m < TL::KPL; ++m) {
-    const int j = lane + 32 * m;
-    ll[m] = n == 0 ? 0.f
-            : PERKEY ? a.logLam[(sh * a.Mcap + (n - 1)) * DK + j]
-                     : a.logLam[sh * gdn_lam_stride(a.Mcap) + (n - 1)];
+    for (int m = 0; m < TL::KPL; ++m) {
+      const int j = lane + 32 * m;
+      ll[m] = n == 0 ? 0.f
+              : PERKEY ? a.logLam[(sh * a.Mcap + (n - 1)) * DK + j]
+                       : a.logLam[sh * gdn_lam_stride(a.Mcap) + (n - 1)];
+    }
   }
   if (!PERKEY && tid < n) s_lam[tid] = a.logLam[sh * gdn_lam_stride(a.Mcap) + tid];
   __syncthreads();
   if (!wait_log(&s_bar, n, a.err)) return;
+  if constexpr (LAMC) {
+    rebuild_snapshots<DK>(reinterpret_cast<const __half*>(s_dyn + LL::a_bytes(n)), sLf, n);
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < TL::KPL; ++m) ll[m] = n == 0 ? 0.f : sLf[(n - 1) * DK + lane + 32 * m];
+  }
 
   for (int i = warp; i < n; i += TL::NW) {
 #pragma unroll

@@ -27,6 +27,7 @@ struct LaunchShape {
   int max_n;       // log length of the launched units (shared-memory sizing)
   int units;       // materialisation: units in the launch
   bool blow;       // GDN/KDA b_i stored in bf16 (bf16-input handles only)
+  bool lamc;       // KDA/RWKV6 snapshots stored as fp16 log-gates (bf16-input handles only)
 };
 
 // Launch with the programmatic-stream-serialisation attribute when `pdl`.
@@ -66,38 +67,57 @@ dim3 step_grid(const LaunchShape& s) {
   return dim3(s.BH * NSPLIT);
 }
 
-template <int OP, int DK, int DV, typename TI, int MODE, int NSPLIT, bool MAP, bool BLOW>
+template <int OP, int DK, int DV, typename TI, int MODE, int NSPLIT, bool MAP, bool BLOW, bool LAMC>
 cudaError_t register_step_mode(const LaunchShape& s, const StepArgs& a, cudaStream_t st) {
   using TL = Tile<DK, DV / NSPLIT>;
-  using LL = LogLayout<OP, DK, DV, TI, BLOW>;
+  using LL = LogLayout<OP, DK, DV, TI, BLOW, LAMC>;
   const size_t smem = LL::step_smem(a.n, MODE == MODE_MERGE);
-  auto kern = deltalog_step_kernel<OP, DK, DV, TI, MODE, NSPLIT, MAP, BLOW>;
+  auto kern = deltalog_step_kernel<OP, DK, DV, TI, MODE, NSPLIT, MAP, BLOW, LAMC>;
   cudaError_t e = allow_smem(kern, smem, LL::step_smem(kMaxM - 1, MODE != MODE_APPEND));
   if (e != cudaSuccess) return e;
   return launch_maybe_pdl(kern, step_grid<NSPLIT, MAP>(s), TL::NT, smem, st, s.pdl, a);
 }
 
-template <int OP, int DK, int DV, typename TI, int NSPLIT, bool BLOW>
+template <int OP, int DK, int DV, typename TI, int NSPLIT, bool BLOW, bool LAMC>
 cudaError_t register_step_log(const LaunchShape& s, int mode, const StepArgs& a, cudaStream_t st) {
   if (a.slot_idx) {
-    if (mode == MODE_MERGE) return register_step_mode<OP, DK, DV, TI, MODE_MERGE, NSPLIT, true, BLOW>(s, a, st);
-    return register_step_mode<OP, DK, DV, TI, MODE_APPEND, NSPLIT, true, BLOW>(s, a, st);
+    if (mode == MODE_MERGE) return register_step_mode<OP, DK, DV, TI, MODE_MERGE, NSPLIT, true, BLOW, LAMC>(s, a, st);
+    return register_step_mode<OP, DK, DV, TI, MODE_APPEND, NSPLIT, true, BLOW, LAMC>(s, a, st);
   }
-  if (mode == MODE_MERGE) return register_step_mode<OP, DK, DV, TI, MODE_MERGE, NSPLIT, false, BLOW>(s, a, st);
-  return register_step_mode<OP, DK, DV, TI, MODE_APPEND, NSPLIT, false, BLOW>(s, a, st);
+  if (mode == MODE_MERGE) return register_step_mode<OP, DK, DV, TI, MODE_MERGE, NSPLIT, false, BLOW, LAMC>(s, a, st);
+  return register_step_mode<OP, DK, DV, TI, MODE_APPEND, NSPLIT, false, BLOW, LAMC>(s, a, st);
 }
 
-// A bf16 b-log exists for bf16-input GDN/KDA handles; other instantiations
-// are never built.
+// A bf16 b-log exists for bf16-input GDN/KDA handles, compact fp16
+// snapshots for bf16-input KDA/RWKV6 handles; other instantiations are never
+// built.
 template <int OP, typename TI>
 constexpr bool kHasBlow = OP != OP_RWKV6 && std::is_same<TI, __nv_bfloat16>::value;
+template <int OP, typename TI>
+constexpr bool kHasLamc = OP != OP_GDN && std::is_same<TI, __nv_bfloat16>::value;
+
+// Calls FN<BLOW, LAMC>() for the handle's log storage.
+template <int OP, typename TI, typename FN>
+cudaError_t with_log_kind(const LaunchShape& s, FN fn) {
+  if constexpr (kHasLamc<OP, TI>) {
+    if (s.lamc) {
+      if constexpr (kHasBlow<OP, TI>) {
+        if (s.blow) return fn(std::true_type{}, std::true_type{});
+      }
+      return fn(std::false_type{}, std::true_type{});
+    }
+  }
+  if constexpr (kHasBlow<OP, TI>) {
+    if (s.blow) return fn(std::true_type{}, std::false_type{});
+  }
+  return fn(std::false_type{}, std::false_type{});
+}
 
 template <int OP, int DK, int DV, typename TI, int NSPLIT>
 cudaError_t register_step(const LaunchShape& s, int mode, const StepArgs& a, cudaStream_t st) {
-  if constexpr (kHasBlow<OP, TI>) {
-    if (s.blow) return register_step_log<OP, DK, DV, TI, NSPLIT, true>(s, mode, a, st);
-  }
-  return register_step_log<OP, DK, DV, TI, NSPLIT, false>(s, mode, a, st);
+  return with_log_kind<OP, TI>(s, [&](auto blow, auto lamc) {
+    return register_step_log<OP, DK, DV, TI, NSPLIT, decltype(blow)::value, decltype(lamc)::value>(s, mode, a, st);
+  });
 }
 
 template <int OP, int DK, int DV, typename TI>
@@ -129,10 +149,10 @@ cudaError_t eager_dims(const LaunchShape& s, const StepArgs& a, cudaStream_t st)
   return a.slot_idx ? eager_map<OP, DK, DV, TI, true>(s, a, st) : eager_map<OP, DK, DV, TI, false>(s, a, st);
 }
 
-template <int OP, int DK, int DV, typename TI, bool BLOW>
+template <int OP, int DK, int DV, typename TI, bool BLOW, bool LAMC>
 cudaError_t materialize_log(const LaunchShape& s, const MaterializeArgs& a, cudaStream_t st) {
-  using LL = LogLayout<OP, DK, DV, TI, BLOW>;
-  auto kern = materialize_kernel<OP, DK, DV, TI, BLOW>;
+  using LL = LogLayout<OP, DK, DV, TI, BLOW, LAMC>;
+  auto kern = materialize_kernel<OP, DK, DV, TI, BLOW, LAMC>;
   const size_t smem = LL::materialize_smem(s.max_n);
   cudaError_t e = allow_smem(kern, smem, LL::materialize_smem(kMaxM - 1));
   if (e != cudaSuccess) return e;
@@ -143,10 +163,9 @@ cudaError_t materialize_log(const LaunchShape& s, const MaterializeArgs& a, cuda
 
 template <int OP, int DK, int DV, typename TI>
 cudaError_t materialize_dims(const LaunchShape& s, const MaterializeArgs& a, cudaStream_t st) {
-  if constexpr (kHasBlow<OP, TI>) {
-    if (s.blow) return materialize_log<OP, DK, DV, TI, true>(s, a, st);
-  }
-  return materialize_log<OP, DK, DV, TI, false>(s, a, st);
+  return with_log_kind<OP, TI>(s, [&](auto blow, auto lamc) {
+    return materialize_log<OP, DK, DV, TI, decltype(blow)::value, decltype(lamc)::value>(s, a, st);
+  });
 }
 
 #define DL_DISPATCH_DIMS(FN, ...)                                                          \

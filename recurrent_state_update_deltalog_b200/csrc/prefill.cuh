@@ -44,12 +44,14 @@ struct PrefillArgs {
   long total;              // tokens in the packed batch
   int H, slots, Mcap, n;
   int b_esize;             // bytes of one b_i element in the log (2 or 4)
+  int lam_esize;           // bytes of one per-key Lam element in the log (4, or 2 for fp16 log-gates)
   int zero_state;          // 1: every row starts from S = 0; 0: from Sbar
 };
 
 // Clear entries [0, n) of unit `sh`'s log: the b_i columns of this value tile,
 // and (first tile only) a_i and Lam_i.  Zero entries add nothing to S_t, and
-// Lam_i = 0 restarts the unit's cumulative decay at the hand-off.
+// Lam_i = 0 (or zero log-gates, with fp16 per-key snapshots) restarts the
+// unit's cumulative decay at the hand-off.
 template <int OP, int DK, int DV, typename TI>
 __device__ __forceinline__ void clear_log_tile(const PrefillArgs& a, long sh, int col0, int ncols) {
   const int n = a.n;
@@ -66,7 +68,9 @@ __device__ __forceinline__ void clear_log_tile(const PrefillArgs& a, long sh, in
   if (OP == OP_GDN) {
     for (int idx = threadIdx.x; idx < n; idx += blockDim.x) a.logLam[sh * gdn_lam_stride(a.Mcap) + idx] = 0.f;
   } else {
-    for (int idx = threadIdx.x; idx < n * DK; idx += blockDim.x) a.logLam[sh * a.Mcap * DK + idx] = 0.f;
+    const int halves = a.lam_esize / 2;
+    unsigned short* lam = reinterpret_cast<unsigned short*>(a.logLam) + sh * a.Mcap * DK * halves;
+    for (int idx = threadIdx.x; idx < n * DK * halves; idx += blockDim.x) lam[idx] = 0;
   }
 }
 

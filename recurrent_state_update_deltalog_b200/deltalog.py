@@ -228,6 +228,10 @@ class DeltaLog:
         nothing and raises DL_DEVERR_WAIT_TIMEOUT."""
         N.call("dl_set_option", self._h, N.DL_OPT_TEST_STALL_LOG, 1 if on else 0)
 
+    def set_log_lam_f16(self, on):
+        """Store KDA/RWKV6 per-key decay metadata as fp16 log-gates (bf16 handles, empty log)."""
+        N.call("dl_set_option", self._h, N.DL_OPT_LOG_LAM_F16, 1 if on else 0)
+
     def set_value_tiles(self, n):
         """0 (automatic), 1, 2 or 4 value tiles (CTAs) per head in the register-tile step kernel."""
         N.call("dl_set_option", self._h, N.DL_OPT_VALUE_TILES, int(n))

@@ -46,7 +46,7 @@ def step_args(op, dseq, t):
 
 
 def run_gpu(op, S0, seq, u, M, dtype, eager=False, record_merges=True, kernel="auto", tiles=0,
-            log_b_bf16=False):
+            log_b_bf16=False, log_lam_f16=False):
     """Run T steps through the library; returns (o[T,B,H,dv], {t: Sbar}, final logical S).
 
     ``kernel`` selects the dl_step kernel ("auto" or "register")."""
@@ -59,6 +59,8 @@ def run_gpu(op, S0, seq, u, M, dtype, eager=False, record_merges=True, kernel="a
     h.set_value_tiles(tiles)
     if log_b_bf16:
         h.set_log_b_bf16(True)
+    if log_lam_f16:
+        h.set_log_lam_f16(True)
     try:
         h.load_state(torch.from_numpy(S0).cuda())
         if u is not None:

@@ -85,3 +85,18 @@ def _count_chunk_flops(op, d, C):
 @pytest.mark.parametrize("d,C", [(64, 32), (128, 16), (128, 32), (8, 4)])
 def test_chunk_prefill_flops(op, d, C):
     assert bench.chunk_prefill_flops(op, d, C) == _count_chunk_flops(op, d, C)
+
+
+@pytest.mark.parametrize("op,d", [("kda", 128), ("rwkv6", 64)])
+@pytest.mark.parametrize("M", [4, 8, 16])
+def test_step_bytes_with_f16_log_gates(op, d, M):
+    """fp16 per-key log-gates: every entry carries 2 d bytes less (the Lam_i
+    term 4 d becomes 2 d), appended once and replayed (M - 1) / 2 times on
+    average per token; nothing else changes.  KDA d = 128: 1280 -> 1024 bytes
+    per entry; RWKV6 d = 64: 512 -> 384."""
+    B, H, tokens = 3, 5, 4 * M
+    full = bench.step_bytes(op, B, H, d, M, tokens) / tokens
+    half = bench.step_bytes(op, B, H, d, M, tokens, lb=2) / tokens
+    saved_per_entry = 2 * d
+    assert full - half == pytest.approx(B * H * saved_per_entry * ((M - 1) / M + (M - 1) / 2), rel=1e-12)
+    assert bench.entry_bytes(op, d, d, lb=2) == {"kda": 1024, "rwkv6": 384}[op]

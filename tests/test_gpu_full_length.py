@@ -46,8 +46,9 @@ def _device_draws(gen, op, B, H, d):
 
 
 def _full_length(op, B, H, d, T, variants, n_units=24, seed=0):
-    """Run every variant ("eager", or a merge interval M) over T tokens of the
-    full batch; return the sampled units' outputs and states next to the oracle's."""
+    """Run every variant ("eager", a merge interval M, or (M, "lam_f16") for
+    fp16 per-key log-gates) over T tokens of the full batch; compare the
+    sampled units' outputs and states with the oracle's."""
     from recurrent_state_update_deltalog_b200 import DeltaLog
     rng = np.random.default_rng(1234)
     flat = np.unique(np.concatenate([rng.choice(B * H, size=n_units, replace=False), [0, B * H - 1]]))
@@ -71,13 +72,18 @@ def _full_length(op, B, H, d, T, variants, n_units=24, seed=0):
     S0 = torch.randn((B, H, d, d), generator=gen, device="cuda") * 0.02
     S0[bi, hi] = torch.from_numpy(S0_s).cuda()
 
+    def interval(v):
+        return 1 if v == "eager" else v[0] if isinstance(v, tuple) else v
+
     def record_steps(v):
-        every = 32 if v in ("eager", 1) else v
+        every = 32 if interval(v) == 1 else interval(v)
         return [t for t in range(T) if (t + 1) % every == 0]
 
     handles, outs, states = {}, {}, {}
     for v in variants:
-        h = DeltaLog(B, H, d, d, 1 if v == "eager" else v, op=op, dtype=BF16)
+        h = DeltaLog(B, H, d, d, interval(v), op=op, dtype=BF16)
+        if isinstance(v, tuple) and "lam_f16" in v:
+            h.set_log_lam_f16(True)
         h.load_state(S0)
         if u is not None:
             h.set_bonus(torch.from_numpy(u).cuda())
@@ -131,14 +137,14 @@ def test_gdn_b256_h32_d128_256_tokens():
 
 
 def test_kda_b128_h32_d128_256_tokens():
-    _full_length("kda", 128, 32, 128, 256, ["eager", 8])
+    _full_length("kda", 128, 32, 128, 256, ["eager", 8, (8, "lam_f16")])
 
 
 def test_rwkv6_b128_h64_d64_256_tokens():
-    _full_length("rwkv6", 128, 64, 64, 256, ["eager", 8])
+    _full_length("rwkv6", 128, 64, 64, 256, ["eager", 8, (8, "lam_f16")])
 
 
 @pytest.mark.parametrize("op", ["gdn", "kda"])
 def test_b1024_h32_d128_512_tokens(op):
     """The largest point of the B x M sweep: 2.15 GB of state per handle, 65,536 CTAs a launch."""
-    _full_length(op, 1024, 32, 128, 512, ["eager", 8, 32])
+    _full_length(op, 1024, 32, 128, 512, ["eager", 8, 32] + ([(32, "lam_f16")] if op == "kda" else []))

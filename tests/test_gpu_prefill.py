@@ -67,7 +67,7 @@ def test_prefill_then_decode_many_heads(op):
     _prefill_then_decode(op, (128, 128), torch.bfloat16, "chunked", H=16)
 
 
-def _prefill_then_decode(op, dims, dtype, kernel, H):
+def _prefill_then_decode(op, dims, dtype, kernel, H, log_lam_f16=False):
     from recurrent_state_update_deltalog_b200 import DeltaLog
     dk, dv = dims
     B, M, T_dec = 8, 4, 7
@@ -83,6 +83,7 @@ def _prefill_then_decode(op, dims, dtype, kernel, H):
     S_pool = initial_state(5, B, H, dk, dv)             # other slots keep this
     h = DeltaLog(B, H, dk, dv, M, op=op, dtype=dtype)
     h.set_prefill_kernel(kernel)
+    h.set_log_lam_f16(log_lam_f16)
     h.load_state(torch.from_numpy(S_pool).cuda())
     if u is not None:
         h.set_bonus(torch.from_numpy(u).cuda())
@@ -127,11 +128,25 @@ def _prefill_then_decode(op, dims, dtype, kernel, H):
 def test_prefill_continues_logical_state(op, kernel):
     """Without DL_PREFILL_ZERO_STATE a prompt continues from the slot's
     logical state (base + log), e.g. the second chunk of a long prompt."""
+    _prefill_continues(op, kernel)
+
+
+@pytest.mark.parametrize("op", ["kda", "rwkv6"])
+@pytest.mark.parametrize("kernel", ["recurrent", "chunked"])
+def test_prefill_with_f16_log_gates(op, kernel):
+    """The hand-off folds (continued prompts) and clears (new prompts) a log
+    whose per-key snapshots are fp16 log-gates."""
+    _prefill_continues(op, kernel, log_lam_f16=True)
+    _prefill_then_decode(op, (128, 128), torch.bfloat16, kernel, H=3, log_lam_f16=True)
+
+
+def _prefill_continues(op, kernel, log_lam_f16=False):
     from recurrent_state_update_deltalog_b200 import DeltaLog
     dtype, dk, dv, B, H, M = torch.bfloat16, 128, 128, 4, 2, 8
     S0, warm, u = make_inputs(op, B, H, dk, dv, 5, dtype, seed=31)
     h = DeltaLog(B, H, dk, dv, M, op=op, dtype=dtype)
     h.set_prefill_kernel(kernel)
+    h.set_log_lam_f16(log_lam_f16)
     h.load_state(torch.from_numpy(S0).cuda())
     if u is not None:
         h.set_bonus(torch.from_numpy(u).cuda())
