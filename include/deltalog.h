@@ -107,7 +107,10 @@ int dl_merge_interval(dl_t h, int* M);
 int dl_destroy(dl_t h);
 
 /* Copy the dense state S [B][H][d_k][d_v] (device pointer) into Sbar and empty
- * the log: the next step starts a new merge cycle. */
+ * the log: the next step starts a new merge cycle.  Sbar is the dense base
+ * that holds the history up to the last merge point (DeltaLog technical
+ * summary, gist.science, section "Method -- core mechanism: base + log",
+ * item 1). */
 int dl_load_state(dl_t h, const float* S, void* stream);
 
 /* RWKV6 only: copy the bonus u [H][d_k] (device pointer). */
@@ -117,6 +120,13 @@ int dl_set_bonus(dl_t h, const float* u, void* stream);
  * With n entries in the log before the call (every slot holds n; see
  * dl_slot_load): if n + 1 < M the step appends (Sbar is read, never
  * written); if n + 1 == M it merges (Sbar <- S_t and the log empties).
+ * These are the append and merge phases of the DeltaLog technical summary
+ * (gist.science, section "Method -- core mechanism: base + log": for M-1
+ * steps only compact factors and the current log-decay snapshot are
+ * appended; every M steps base plus replayed log is written into the base
+ * and the log reset).  Every step's output is computed from base + replayed
+ * log, so it is the eager recurrence's (arXiv 2608.15533 abstract, fugumt.com:
+ * the model observes the same dense state as in eager decoding).
  * Writes o [B][H][d_v].  All pointers are device pointers. */
 int dl_step(dl_t h, const void* q, const void* k, const void* v,
             const float* log_decay, const float* beta, void* o, void* stream);
@@ -196,9 +206,11 @@ int dl_prefill(dl_t h, const int* slot_idx, int rows, const int* cu_seqlens, lon
 int dl_step_host(dl_t h, const void* q, const void* k, const void* v,
                  const float* log_decay, const float* beta, void* o, void* stream);
 
-/* Eager dense baseline: read S_{t-1} from Sbar, write S_t back, every token.
- * Requires every slot's log to be empty (DL_ERR_STATE otherwise; call
- * dl_merge). */
+/* Eager dense baseline: read S_{t-1} from Sbar, write S_t back, every token:
+ * the dense materialisation after every token that the DeltaLog technical
+ * summary describes as the state-update tax (gist.science, section
+ * "Problem: the state-update tax in linear-attention decoding").  Requires
+ * every slot's log to be empty (DL_ERR_STATE otherwise; call dl_merge). */
 int dl_eager_step(dl_t h, const void* q, const void* k, const void* v,
                   const float* log_decay, const float* beta, void* o, void* stream);
 
@@ -211,11 +223,16 @@ int dl_eager_step_indexed(dl_t h, const int* slot_idx, int rows, const void* q, 
                           void* stream);
 
 /* Fold every slot's log into Sbar now (no output) and empty them; a no-op
- * when all logs are empty.  For an explicit flush or a checkpoint. */
+ * when all logs are empty.  For an explicit flush or a checkpoint.  This is
+ * the merge phase without a token (DeltaLog technical summary, gist.science,
+ * section "Method -- core mechanism: base + log": the accumulated logical
+ * state, base plus replayed log entries, written into the base). */
 int dl_merge(dl_t h, void* stream);
 
 /* Write the logical state (Sbar + replayed log) to S_out [B][H][d_k][d_v]
- * (device pointer) without changing the handle. */
+ * (device pointer) without changing the handle: the dense state the model
+ * observes, equal to the eager decoder's (arXiv 2608.15533 abstract,
+ * fugumt.com). */
 int dl_read_state(dl_t h, float* S_out, void* stream);
 
 /* Tuning options.  DL_OPT_STEP_KERNEL picks the kernel behind dl_step:
