@@ -435,10 +435,12 @@ deltalog_step_kernel(const StepArgs a) {
     }
   };
   if constexpr (PERKEY) load_inputs();
-  float* Sp = a.Sbar + sh * (DK * DV);
+  // This thread's rows of the tile, addressed from one register with
+  // immediate row offsets (rows are DV floats apart).
+  float* Sp = a.Sbar + sh * (DK * DV) + (rg * TL::RPT) * DV + col0 + 4 * c4;
   float4 st[TL::RPT];
 #pragma unroll
-  for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + (rg * TL::RPT + j) * DV + col0 + 4 * c4);
+  for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + j * DV);
   if (MODE == MODE_APPEND) griddep_launch_dependents();
   if constexpr (!WAIT_FIRST) griddep_wait();
   if (tid == 0)
@@ -616,8 +618,14 @@ deltalog_step_kernel(const StepArgs a) {
         fma4(st[j4 + 3], a4.w, b4);
       }
     }
+    // Re-derive the store addresses from the one base register rather than
+    // keep the load addresses live across the kernel (measured with ptxas:
+    // the merge variants drop from 128 registers with 32 bytes of spills to
+    // 114-118 registers and none).
+    float* Sw = Sp;
+    asm volatile("" : "+l"(Sw));
 #pragma unroll
-    for (int j = 0; j < TL::RPT; ++j) st_state(Sp + (rg * TL::RPT + j) * DV + col0 + 4 * c4, st[j]);
+    for (int j = 0; j < TL::RPT; ++j) st_state(Sw + j * DV, st[j]);
   }
 }
 
@@ -650,10 +658,10 @@ eager_step_kernel(const StepArgs a) {
   const int col0 = ux.col0;
   const int h = ux.h;
 
-  float* Sp = a.Sbar + sh * (DK * DV);
+  float* Sp = a.Sbar + sh * (DK * DV) + (rg * TL::RPT) * DV + col0 + 4 * c4;   // this thread's rows
   float4 st[TL::RPT];
 #pragma unroll
-  for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + (rg * TL::RPT + j) * DV + col0 + 4 * c4);
+  for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + j * DV);
 
   const int c = tid;
   float vc = 0.f, betac = 0.f;
@@ -729,13 +737,15 @@ eager_step_kernel(const StepArgs a) {
   __syncthreads();
 
   const float4 b4 = *reinterpret_cast<const float4*>(&s_b[4 * c4]);
+  float* Sw = Sp;
+  asm volatile("" : "+l"(Sw));   // store addresses from one register (see the step kernel)
 #pragma unroll
   for (int j = 0; j < TL::RPT; ++j) {
     const int row = rg * TL::RPT + j;
     float4 x = st[j];
     scale4(x, s_dec[row]);
     fma4(x, s_k[row], b4);
-    st_state(Sp + row * DV + col0 + 4 * c4, x);
+    st_state(Sw + j * DV, x);
   }
 }
 
@@ -779,10 +789,10 @@ materialize_kernel(const MaterializeArgs a) {
   const TB* sB = reinterpret_cast<const TB*>(s_dyn + LL::a_bytes(n) + LL::l_bytes(n));
   float* As = reinterpret_cast<float*>(s_dyn + LL::staged(n) + LL::table(n));
 
-  const float* Sp = a.Sin + sh * (DK * DV);
+  const float* Sp = a.Sin + sh * (DK * DV) + (rg * TL::RPT) * DV + 4 * c4;   // this thread's rows
   float4 st[TL::RPT];
 #pragma unroll
-  for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + (rg * TL::RPT + j) * DV + 4 * c4);
+  for (int j = 0; j < TL::RPT; ++j) st[j] = ld_state(Sp + j * DV);
   if (tid == 0) stage_log<OP, DK, DV, TI, BLOW, LAMC>(s_dyn, &s_bar, a.logA, a.logLam, a.logB, sh, a.Mcap, n);
 
   float ll[TL::KPL];
@@ -835,8 +845,10 @@ materialize_kernel(const MaterializeArgs a) {
       fma4(st[j4 + 3], a4.w, b4);
     }
   }
+  float* Sw = Sq + (rg * TL::RPT) * DV + 4 * c4;
+  asm volatile("" : "+l"(Sw));   // store addresses from one register (see the step kernel)
 #pragma unroll
-  for (int j = 0; j < TL::RPT; ++j) st_state(Sq + (rg * TL::RPT + j) * DV + 4 * c4, st[j]);
+  for (int j = 0; j < TL::RPT; ++j) st_state(Sw + j * DV, st[j]);
 }
 
 }  // namespace dl
