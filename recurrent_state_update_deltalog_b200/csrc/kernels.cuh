@@ -256,9 +256,18 @@ template <int DK>
 __device__ __forceinline__ void rebuild_snapshots(const __half* g, float* lam, int n) {
   for (int j = threadIdx.x; j < DK; j += blockDim.x) {
     float s = 0.f;
-    for (int i = 0; i < n; ++i) {
-      s += __half2float(g[i * DK + j]);
-      lam[i * DK + j] = s;
+    for (int i0 = 0; i0 < n; i0 += 8) {
+      // eight gates in flight at once; the sums stay in entry order
+      float gi[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) gi[u] = i0 + u < n ? __half2float(g[(i0 + u) * DK + j]) : 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (i0 + u < n) {
+          s += gi[u];
+          lam[(i0 + u) * DK + j] = s;
+        }
+      }
     }
   }
 }
