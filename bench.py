@@ -916,8 +916,7 @@ def run_prefill(a, rank, world, local_rank):
     tok_s = B * L / (ms / 1e3)
     sm = (clocks or {}).get("sm_mhz") or 1965.0
     if h.last_prefill_kernel == "chunked":
-        # the bench's heads are square (d_k = d_v = d): 32-token chunks in every
-        # chunked kernel that serves them (16 only for d_k = 128, d_v = 64 heads)
+        # every chunked kernel takes 32-token chunks
         C = 32
         per_th = chunk_prefill_flops(op, d, C)
         bf16, kind = measured_bf16_tflops()

@@ -284,25 +284,18 @@ int dl_read_state(dl_t h, float* S_out, void* stream);
 /* DL_OPT_PREFILL_KERNEL picks the kernel behind dl_prefill:
  *   DL_PREFILL_AUTO (default): the chunked kernel for bf16-input handles
  *     whose prompts average at least 16 tokens (GDN, RWKV6) or 24 (KDA) at
- *     d_k = d_v = 128, 64 at other shapes; the recurrent kernel otherwise;
+ *     d_k = d_v = 128, and 32 (GDN, RWKV6) or 64 (KDA) at the other shapes;
+ *     the recurrent kernel otherwise;
  *   DL_PREFILL_RECURRENT: the recurrence token by token, state in registers
  *     (every operator and dtype; outputs equal the eager recurrence's up to
  *     fp32 rounding);
  *   DL_PREFILL_CHUNKED: the chunk form on tensor cores (bf16-input handles
  *     only, DL_ERR_UNSUPPORTED otherwise): 32-token chunks, the WY form of
  *     the delta rule for GDN and KDA, per-key pair weights of KDA and RWKV6
- *     formed exactly on the SIMT lanes.  At d_k = d_v = 128 each CTA keeps
- *     a whole head's state in tensor memory and runs the products with it as
- *     tcgen05 MMAs; other shapes use 64-column tiles and warp-level MMAs.
- *     The products with the state are tf32, inside the bf16-input
- *     tolerance. */
-/* DL_OPT_TEST_STALL_LOG (0 or 1, default 0; for tests of the error path
- * only): register-tile steps arm their log barrier for the log's bytes but
- * issue no copy, and bound the wait at 20 microseconds.  Every unit whose
- * log is not empty then gives up, writes nothing (no output, no log entry,
- * no state) and raises DL_DEVERR_WAIT_TIMEOUT; nothing is left in flight,
- * so the context stays usable.  The handle's log is then out of step with
- * its outputs: load a state (dl_load_state) or destroy it afterwards. */
+ *     formed exactly on the SIMT lanes.  Each CTA keeps a whole head's state
+ *     in tensor memory and runs the products with it as tcgen05 MMAs, for
+ *     every head shape.  The products with the state are tf32, inside the
+ *     bf16-input tolerance. */
 enum dl_option {
   DL_OPT_STEP_KERNEL = 0,
   DL_OPT_HOST_PREFETCH = 1,

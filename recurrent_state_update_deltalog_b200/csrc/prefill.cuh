@@ -263,14 +263,14 @@ prefill_kernel(const PrefillArgs a) {
   clear_log_tile<OP, DK, DV, TI>(a, sh, col0, CW);
 }
 
-// Chunked tensor-core GDN prefill (bf16 inputs; prefill_chunk.cuh), any
-// supported d_k x d_v.  cudaErrorNotSupported when its shared memory does not
-// fit the device.
+// Chunked GDN prefill with the state in tensor memory (bf16 inputs;
+// prefill_chunk_tc.cuh), any supported d_k x d_v: grid (H, rows).
+// cudaErrorNotSupported when its shared memory does not fit the device.
 cudaError_t launch_gdn_chunk_prefill_dims(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st);
 
-// Chunked tensor-core KDA / RWKV6 prefill (bf16 inputs; prefill_chunk_key.cuh):
-// grid (H * d_v/64, rows), 256 threads.  cudaErrorNotSupported when its shared
-// memory does not fit the device.
+// Chunked KDA / RWKV6 prefill with the state in tensor memory (bf16 inputs;
+// prefill_chunk_tc.cuh): grid (H, rows).  cudaErrorNotSupported when its
+// shared memory does not fit the device.
 template <int OP>
 cudaError_t launch_key_chunk_prefill_dims(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st);
 extern template cudaError_t launch_key_chunk_prefill_dims<OP_KDA>(const LaunchShape&, const PrefillArgs&, cudaStream_t);

@@ -1,19 +1,21 @@
-// Chunked prefill with the state in tensor memory, for d_k = d_v = 128: the
-// chunk forms of gdn_chunk_prefill_kernel (prefill_chunk.cuh) and of
-// key_chunk_prefill_kernel (prefill_chunk_key.cuh), with their three products
-// with the state issued as 5th-generation tensor-core MMAs (tcgen05, tf32
-// operands, fp32 accumulation) on a whole head per CTA.
+// Chunked prefill with the state in tensor memory: the chunk forms of
+// prefill_chunk.cuh with their three products with the state issued as
+// 5th-generation tensor-core MMAs (tcgen05, tf32 operands, fp32 accumulation)
+// on a whole head per CTA, for every head shape (d_k, d_v in {64, 128}).
 //
 // The state is kept transposed, S^T (value column c on TMEM lane c, key j on
 // column j), so that it serves directly as the A operand of
-//   B^T = U^T - S^T W^T                  (M = 128 value columns, N = C tokens)
+//   B^T = U^T - S^T W^T                  (M = 128 lanes, N = C tokens)
 //   O^T = S^T (e^{Gamma} Q)^T + B^T P^T
 //   S^T <- e^{Gamma_end} S^T + B^T (e^{Gamma_end - Gamma} K)
 // and receives the last as its accumulator; it never leaves tensor memory
-// between the prompt's first and last chunk.  B^T, O^T and U^T live in
-// tensor memory too (the triangular solve writes U^T there: each U column is
-// a thread whose TMEM lane is that value column).  W, the scaled queries, P
-// and the scaled keys are written by the SIMT lanes into shared memory in
+// between the prompt's first and last chunk.  A d_v = 64 head uses lanes
+// 0 .. 63 of the M = 128 products and keeps lanes 64 .. 127 zero: each row of
+// an MMA result depends only on the same row of its tensor-memory operand,
+// and every element-wise pass stays on its own lane.  B^T, O^T and U^T live
+// in tensor memory too (the triangular solve writes U^T there: each U column
+// is a thread whose TMEM lane is that value column).  W, the scaled queries,
+// P and the scaled keys are written by the SIMT lanes into shared memory in
 // K-major no-swizzle operand layouts.  One thread issues the MMAs; their
 // completion is tracked by mbarriers (bounded waits: a wait that runs out
 // raises DL_DEVERR_WAIT_TIMEOUT and the CTA stops).  The state update of
@@ -24,7 +26,6 @@
 #pragma once
 
 #include "prefill_chunk.cuh"
-#include "prefill_chunk_key.cuh"
 
 namespace dl {
 
@@ -141,9 +142,14 @@ __device__ __forceinline__ uint64_t umma_desc_lbo(uint32_t addr, uint32_t lbo, u
          (static_cast<uint64_t>((sbo >> 4) & 0x3fff) << 32) | (static_cast<uint64_t>(1) << 46);
 }
 
-template <int NT_>
+template <int NT_, int DK_ = 128, int DV_ = 128>
 struct TcChunkGeom {
-  static constexpr int DK = 128, DV = 128;   // a whole head per CTA
+  // a whole head per CTA; value columns sit on tensor-memory lanes 0 .. DV-1
+  // of the 128 an M = 128 MMA covers (a d_v = 64 head leaves the upper 64
+  // lanes zero: every MMA row and every element-wise pass stays within its own
+  // lane, so padding never reaches a value column)
+  static constexpr int DK = DK_, DV = DV_;
+  static_assert((DK == 64 || DK == 128) && (DV == 64 || DV == 128), "head shape");
   static constexpr int C = 32;               // tokens per chunk
   // 256 threads (two CTAs per SM) or 512 (one CTA per SM, for launches with
   // fewer CTAs than SMs)
@@ -169,15 +175,15 @@ struct TcChunkGeom {
   static constexpr size_t BYTES = BAR_OFF + 64;
   // tensor-memory columns
   static constexpr uint32_t TM_COLS = 256;   // allocation (power of two)
-  static constexpr uint32_t TM_S = 0;        // S^T: 128 columns (keys)
-  static constexpr uint32_t TM_B = 128;      // W S, then B^T: C columns (tokens)
-  static constexpr uint32_t TM_O = 160;      // O^T: C columns
-  static constexpr uint32_t TM_U = 192;      // U^T: C columns (the solve writes it)
+  static constexpr uint32_t TM_S = 0;        // S^T: DK columns (keys)
+  static constexpr uint32_t TM_B = DK;       // W S, then B^T: C columns (tokens)
+  static constexpr uint32_t TM_O = DK + 32;  // O^T: C columns
+  static constexpr uint32_t TM_U = DK + 64;  // U^T: C columns (the solve writes it)
 };
 
-template <int NT_>
-__global__ void __launch_bounds__(NT_, TcChunkGeom<NT_>::MINB) gdn_chunk_prefill_tc_kernel(const PrefillArgs a) {
-  using G = TcChunkGeom<NT_>;
+template <int NT_, int DK_, int DV_>
+__global__ void __launch_bounds__(NT_, TcChunkGeom<NT_, DK_, DV_>::MINB) gdn_chunk_prefill_tc_kernel(const PrefillArgs a) {
+  using G = TcChunkGeom<NT_, DK_, DV_>;
   constexpr int C = G::C, DK = G::DK, DV = G::DV;
   extern __shared__ __align__(128) unsigned char smem[];
   auto kbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem + G::K_OFF + b * G::KQ_BYTES); };
@@ -241,12 +247,13 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_>::MINB) gdn_chunk_prefill
   const uint32_t tmem = *sTmem;
   const uint32_t lane_base = static_cast<uint32_t>(32 * quarter) << 16;
   const int c_own = 32 * quarter + lane;   // this thread's value column in TMEM epilogues
+  const bool own_col = c_own < DV;         // false on the padding lanes of a d_v = 64 head
 
   // S^T into tensor memory: this warp's 32 lanes (value columns), key blocks 32 cb ..
   for (int cb = group; cb < DK / 32; cb += NG) {
     float v[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = a.zero_state ? 0.f : __ldcs(Sg + (32 * cb + i) * DV + c_own);
+    for (int i = 0; i < 32; ++i) v[i] = a.zero_state || !own_col ? 0.f : __ldcs(Sg + (32 * cb + i) * DV + c_own);
     tmem_st32(tmem + lane_base + G::TM_S + 32 * cb, v);
   }
   tmem_wait_st();
@@ -354,13 +361,18 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_>::MINB) gdn_chunk_prefill
     // 3. (I + A) X = R, one right-hand-side column per thread: W in place in its
     // operand layout (tf32-rounded); U (right-hand side beta V read from V) into
     // tensor memory, its column on this thread's TMEM lane
-    if (tid < DK + DV) {
-      const bool isw = tid < DK;
-      const int cu = tid - DK;
+    // W column j on thread j; U^T lane c on thread 128 + c, which belongs to
+    // the warp whose tensor-memory sub-partition holds lane c (lanes past d_v
+    // are padding and solve a zero right-hand side)
+    const bool isw = tid < DK, isu = tid >= 128 && tid < 256;
+    if (isw || isu) {
+      const int cu = tid - 128;
+      const bool live = isw || cu < DV;
       float x[C];
 #pragma unroll
       for (int t = 0; t < C; ++t) {
-        float acc0 = isw ? fp(sWc, kmajor_pad_off<C>(t, tid))[0] : sBeta[t] * __bfloat162float(sV[t * G::LDV + cu]);
+        float acc0 = isw ? fp(sWc, kmajor_pad_off<C>(t, tid))[0]
+                         : live ? sBeta[t] * __bfloat162float(sV[t * G::LDV + cu]) : 0.f;
         float acc1 = 0.f;
         const float* arow = sA + t * G::LDA;
 #pragma unroll
@@ -376,7 +388,7 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_>::MINB) gdn_chunk_prefill
         x[t] = acc0 + acc1;
         if (isw) fp(sWc, kmajor_pad_off<C>(t, tid))[0] = wm::__float_to_tf32(x[t]);
       }
-      if (!isw) {   // whole warps: the U columns are threads DK .. DK + DV - 1
+      if (isu) {   // whole warps: threads 128 .. 255
         tmem_st32(tmem + lane_base + G::TM_U, x);
         tmem_wait_st();
       }
@@ -476,7 +488,7 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_>::MINB) gdn_chunk_prefill
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int t = 8 * b8 + i;
-          if (t < n) Og[((c0 + t) * a.H + h) * DV + c_own] = __float2bfloat16_rn(v[i]);
+          if (t < n && own_col) Og[((c0 + t) * a.H + h) * DV + c_own] = __float2bfloat16_rn(v[i]);
         }
       }
       const float dend = sEG[n - 1];
@@ -516,8 +528,10 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_>::MINB) gdn_chunk_prefill
     for (int cb = group; cb < DK / 32; cb += NG) {
       float v[32];
       tmem_ld32(tmem + lane_base + G::TM_S + 32 * cb, v);
+      if (own_col) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) __stcs(Sg + (32 * cb + i) * DV + c_own, v[i]);
+        for (int i = 0; i < 32; ++i) __stcs(Sg + (32 * cb + i) * DV + c_own, v[i]);
+      }
     }
   }
   if (!ok && tid == 0) {
@@ -538,23 +552,25 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_>::MINB) gdn_chunk_prefill
 }
 
 // Grid (H, rows), 256 threads (two CTAs per SM) once the launch has more CTAs
-// than SMs, else 512; TcChunkGeom<NT>::BYTES of dynamic shared memory;
-// d_k = d_v = 128, bf16 inputs.  Instantiated in prefill.cu.
+// than SMs, else 512; TcChunkGeom<NT, DK, DV>::BYTES of dynamic shared memory;
+// bf16 inputs.  Instantiated in prefill.cu.
+template <int DK, int DV>
 cudaError_t launch_gdn_chunk_prefill_tc(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st);
 
 // ---- KDA and RWKV6 (per-key decay) ---------------------------------------------
 //
-// The chunk form of key_chunk_prefill_kernel (prefill_chunk_key.cuh) with the
-// same tensor-memory state: A and P pair by pair on the SIMT lanes, the three
-// products with the state on tcgen05.  RWKV6 has no W S product: its B^T is
+// The per-key chunk form (prefill_chunk.cuh) with the same tensor-memory
+// state: A and P pair by pair on the SIMT lanes, the three products with the
+// state on tcgen05.  RWKV6 has no W S product: its B^T is
 // V^T, written straight into tensor memory.  The per-key decay of the state
 // update scales the columns of S^T.
 
-template <int NT_>
+template <int NT_, int DK_ = 128, int DV_ = 128>
 struct KeyTcChunkGeom {
   // 256 threads (two CTAs per SM) or 512 (one per SM, for launches with
-  // fewer CTAs than SMs)
-  static constexpr int DK = 128, DV = 128, C = 32, NT = NT_, NW = NT / 32;
+  // fewer CTAs than SMs); value columns on lanes 0 .. DV-1 as in TcChunkGeom
+  static constexpr int DK = DK_, DV = DV_, C = 32, NT = NT_, NW = NT / 32;
+  static_assert((DK == 64 || DK == 128) && (DV == 64 || DV == 128), "head shape");
   static constexpr int NG = NW / 4;                 // column groups of the TMEM epilogues
   static constexpr int MINB = NT == 256 ? 2 : 1;
   static constexpr int LDK = DK + 8, LDV = DV + 8, LDG = DK + 4, LDA = C + 4;
@@ -578,12 +594,13 @@ struct KeyTcChunkGeom {
   static constexpr size_t BAR_OFF = tc_align128(E_OFF + (2 * DK + C) * 4);
   static constexpr size_t BYTES = BAR_OFF + 64;
   // tensor-memory columns: S^T, W S then B^T, O^T, U^T (KDA; the solve writes it)
-  static constexpr uint32_t TM_COLS = 256, TM_S = 0, TM_B = 128, TM_O = 160, TM_U = 192;
+  static constexpr uint32_t TM_COLS = 256, TM_S = 0, TM_B = DK, TM_O = DK + 32, TM_U = DK + 64;
 };
 
-template <int OP, int NT_>
-__global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_>::MINB) key_chunk_prefill_tc_kernel(const PrefillArgs a) {
-  using G = KeyTcChunkGeom<NT_>;
+template <int OP, int NT_, int DK_, int DV_>
+__global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_, DK_, DV_>::MINB)
+key_chunk_prefill_tc_kernel(const PrefillArgs a) {
+  using G = KeyTcChunkGeom<NT_, DK_, DV_>;
   constexpr int NG = G::NG;
   constexpr int C = G::C, DK = G::DK, DV = G::DV;
   constexpr bool DELTA = OP == OP_KDA;
@@ -652,10 +669,11 @@ __global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_>::MINB) key_chunk_pref
   const uint32_t tmem = *sTmem;
   const uint32_t lane_base = static_cast<uint32_t>(32 * quarter) << 16;
   const int c_own = 32 * quarter + lane;
+  const bool own_col = c_own < DV;
   for (int cb = group; cb < DK / 32; cb += NG) {
     float v[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = a.zero_state ? 0.f : __ldcs(Sg + (32 * cb + i) * DV + c_own);
+    for (int i = 0; i < 32; ++i) v[i] = a.zero_state || !own_col ? 0.f : __ldcs(Sg + (32 * cb + i) * DV + c_own);
     tmem_st32(tmem + lane_base + G::TM_S + 32 * cb, v);
   }
   tmem_wait_st();
@@ -752,13 +770,16 @@ __global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_>::MINB) key_chunk_pref
       // 3. (I + A) X = R, one right-hand-side column per thread: W in shared
       // memory, then its operand layout; U (right-hand side beta V read from V)
       // into tensor memory, its column on this thread's TMEM lane
-      if (tid < DK + DV) {
-        const bool isw = tid < DK;
-        const int cu = tid - DK;
+      // W column j on thread j; U^T lane c on thread 128 + c (see the GDN kernel)
+      const bool isw = tid < DK, isu = tid >= 128 && tid < 256;
+      if (isw || isu) {
+        const int cu = tid - 128;
+        const bool live = isw || cu < DV;
         float x[C];
 #pragma unroll
         for (int t = 0; t < C; ++t) {
-          float acc0 = isw ? fp(sWc, kmajor_pad_off<C>(t, tid))[0] : sBeta[t] * __bfloat162float(sV[t * G::LDV + cu]);
+          float acc0 = isw ? fp(sWc, kmajor_pad_off<C>(t, tid))[0]
+                           : live ? sBeta[t] * __bfloat162float(sV[t * G::LDV + cu]) : 0.f;
           float acc1 = 0.f;
           const float* arow = sA + t * G::LDA;
 #pragma unroll
@@ -774,7 +795,7 @@ __global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_>::MINB) key_chunk_pref
           x[t] = acc0 + acc1;
           if (isw) fp(sWc, kmajor_pad_off<C>(t, tid))[0] = wm::__float_to_tf32(x[t]);
         }
-        if (!isw) {   // whole warps: the U columns are threads DK .. DK + DV - 1
+        if (isu) {   // whole warps: threads 128 .. 255
           tmem_st32(tmem + lane_base + G::TM_U, x);
           tmem_wait_st();
         }
@@ -804,7 +825,7 @@ __global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_>::MINB) key_chunk_pref
       for (int b8 = group; b8 < C / 8; b8 += NG) {
         float v[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = __bfloat162float(sV[(8 * b8 + i) * G::LDV + c_own]);
+        for (int i = 0; i < 8; ++i) v[i] = own_col ? __bfloat162float(sV[(8 * b8 + i) * G::LDV + c_own]) : 0.f;
         tmem_st8(tmem + lane_base + G::TM_B + 8 * b8, v);
       }
       tmem_wait_st();
@@ -898,7 +919,7 @@ __global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_>::MINB) key_chunk_pref
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int t = 8 * b8 + i;
-          if (t < n) Og[((c0 + t) * a.H + h) * DV + c_own] = __float2bfloat16_rn(v[i]);
+          if (t < n && own_col) Og[((c0 + t) * a.H + h) * DV + c_own] = __float2bfloat16_rn(v[i]);
         }
       }
       for (int cb = group; cb < DK / 32; cb += NG) {
@@ -936,8 +957,10 @@ __global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_>::MINB) key_chunk_pref
     for (int cb = group; cb < DK / 32; cb += NG) {
       float v[32];
       tmem_ld32(tmem + lane_base + G::TM_S + 32 * cb, v);
+      if (own_col) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) __stcs(Sg + (32 * cb + i) * DV + c_own, v[i]);
+        for (int i = 0; i < 32; ++i) __stcs(Sg + (32 * cb + i) * DV + c_own, v[i]);
+      }
     }
   }
   if (!ok && tid == 0) {
@@ -958,9 +981,9 @@ __global__ void __launch_bounds__(NT_, KeyTcChunkGeom<NT_>::MINB) key_chunk_pref
 }
 
 // Grid (H, rows), 256 threads (two CTAs per SM) once the launch has more CTAs
-// than SMs, else 512; KeyTcChunkGeom<NT>::BYTES of dynamic shared memory;
-// d_k = d_v = 128, bf16 inputs.  Instantiated in prefill.cu.
-template <int OP>
+// than SMs, else 512; KeyTcChunkGeom<NT, DK, DV>::BYTES of dynamic shared
+// memory; bf16 inputs.  Instantiated in prefill.cu.
+template <int OP, int DK, int DV>
 cudaError_t launch_key_chunk_prefill_tc(const LaunchShape& s, const PrefillArgs& a, cudaStream_t st);
 
 }  // namespace dl
