@@ -63,6 +63,17 @@ __device__ __forceinline__ void umma_tf32_ts(uint32_t d, uint32_t a, uint64_t bd
       : "memory");
 }
 
+// D[tmem] (+)= A[smem desc] B[smem desc]; one thread issues.
+__device__ __forceinline__ void umma_tf32_ss(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+      ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
+      : "memory");
+}
+
 // Arrive once on `bar` when every MMA this thread issued so far has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -160,7 +171,10 @@ struct TcChunkGeom {
   static constexpr int LDV = DV + 8;         // bf16 row stride of V
   static constexpr int LDA = C + 4;          // fp32 row stride of A and P (WMMA outputs)
   static constexpr uint32_t WQ_LBO = kmajor_pad_lbo<C>();             // W and e^G Q operand layout
-  static constexpr size_t WQ_BYTES = size_t(DK / 4) * WQ_LBO;
+  // the W and e^G Q buffers also hold the solve's right-hand sides R_W^T and
+  // R_U^T, dense K-major 128 x C operands
+  static constexpr size_t WQ_BYTES = size_t(DK / 4) * WQ_LBO > size_t(128) * C * 4 ? size_t(DK / 4) * WQ_LBO
+                                                                                    : size_t(128) * C * 4;
   static constexpr size_t KQ_BYTES = tc_align128(size_t(C) * LDK * 2), V_BYTES = tc_align128(size_t(C) * LDV * 2);
   static constexpr size_t K_OFF = 0;                                  // [2][C][LDK] bf16
   static constexpr size_t Q_OFF = K_OFF + 2 * KQ_BYTES;               // [C][LDK] bf16
@@ -171,14 +185,17 @@ struct TcChunkGeom {
   static constexpr size_t PC_OFF = tc_align128(QC_OFF + WQ_BYTES);    // P, K-major C x C
   static constexpr size_t KC_OFF = PC_OFF + size_t(C) * C * 4;        // (e^{..} K)^T, K-major DK x C
   static constexpr size_t G_OFF = tc_align128(KC_OFF + size_t(DK) * C * 4);    // 5 x [C] per-row factors
-  static constexpr size_t BAR_OFF = tc_align128(G_OFF + 5 * C * 4);            // 3 mbarriers, TMEM base, abort flag, drain mbarrier
+  static constexpr size_t T_OFF = tc_align128(G_OFF + 5 * C * 4);              // [C][LDA] T = (I + A)^-1
+  static constexpr size_t X_OFF = T_OFF + size_t(C) * LDA * 4;                 // [16][17] A21 T11
+  static constexpr size_t BAR_OFF = tc_align128(X_OFF + 16 * 17 * 4);          // 4 mbarriers, TMEM base, abort flag, drain
   static constexpr size_t BYTES = BAR_OFF + 64;
   // tensor-memory columns
   static constexpr uint32_t TM_COLS = 256;   // allocation (power of two)
   static constexpr uint32_t TM_S = 0;        // S^T: DK columns (keys)
   static constexpr uint32_t TM_B = DK;       // W S, then B^T: C columns (tokens)
   static constexpr uint32_t TM_O = DK + 32;  // O^T: C columns
-  static constexpr uint32_t TM_U = DK + 64;  // U^T: C columns (the solve writes it)
+  static constexpr uint32_t TM_U = DK + 64;  // U^T: C columns (the solve's product writes it)
+  static constexpr uint32_t TM_W = DK + 96;  // W^T: C columns (the solve's product, then W's operand)
 };
 
 template <int NT_, int DK_, int DV_>
@@ -199,12 +216,15 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_, DK_, DV_>::MINB) gdn_chu
   float* sEG = sG + 2 * C;
   float* sBEG = sG + 3 * C;
   float* sEnd = sG + 4 * C;
+  float* sT = reinterpret_cast<float*>(smem + G::T_OFF);
+  float* sX = reinterpret_cast<float*>(smem + G::X_OFF);
   uint64_t* barB = reinterpret_cast<uint64_t*>(smem + G::BAR_OFF);   // W S done
   uint64_t* barO = barB + 1;                                          // O^T done
   uint64_t* barS = barB + 2;                                          // state update done
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(barB + 3);
   volatile int* sAbort = reinterpret_cast<volatile int*>(sTmem + 1);
   uint64_t* barF = barB + 4;                                          // drain after an abort
+  uint64_t* barT = barB + 5;                                          // the solve's products done
   auto fp = [](unsigned char* base, uint32_t off) { return reinterpret_cast<float*>(base + off); };
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -232,6 +252,7 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_, DK_, DV_>::MINB) gdn_chu
     mbar_init(barO, 1);
     mbar_init(barS, 1);
     mbar_init(barF, 1);
+    mbar_init(barT, 1);
     fence_mbar_init();
     *sAbort = 0;
   }
@@ -341,7 +362,7 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_, DK_, DV_>::MINB) gdn_chu
     }
     __syncthreads();
 
-    // 2. A = strictly lower (beta_t e^{G_t - G_s} k_t . k_s); right-hand sides
+    // 2. A = strictly lower (beta_t e^{G_t - G_s} k_t . k_s)
     lower_xyt<C, DK, G::LDK, G::LDA>(sK, sK, sA);
     __syncthreads();
     for (int idx = tid; idx < C * C; idx += G::NT) {
@@ -349,51 +370,117 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_, DK_, DV_>::MINB) gdn_chu
       float& x = sA[t * G::LDA + s];
       x = s < t ? sBeta[t] * expf(sG[t] - sG[s]) * x : 0.f;
     }
-    for (int idx = tid; idx < C * DK / 4; idx += G::NT) {   // beta e^G K, four keys a thread
-      const int t = idx / (DK / 4), j = 4 * (idx % (DK / 4));
-      float k4[4];
-      bf16x4_to_f32(sK + t * G::LDK + j, k4);
-      const float f = sBEG[t];
-      *reinterpret_cast<float4*>(sWc + kmajor_pad_off<C>(t, j)) = make_float4(f * k4[0], f * k4[1], f * k4[2], f * k4[3]);
-    }
     __syncthreads();
 
-    // 3. (I + A) X = R, one right-hand-side column per thread: W in place in its
-    // operand layout (tf32-rounded); U (right-hand side beta V read from V) into
-    // tensor memory, its column on this thread's TMEM lane
-    // W column j on thread j; U^T lane c on thread 128 + c, which belongs to
-    // the warp whose tensor-memory sub-partition holds lane c (lanes past d_v
-    // are padding and solve a zero right-hand side)
-    const bool isw = tid < DK, isu = tid >= 128 && tid < 256;
-    if (isw || isu) {
-      const int cu = tid - 128;
-      const bool live = isw || cu < DV;
-      float x[C];
+    // 3. (I + A) W = diag(beta e^G) K and (I + A) U = diag(beta) V as
+    // W^T = R_W^T T^T and U^T = R_U^T T^T with T = (I + A)^{-1}: T on the SIMT
+    // lanes in 16 x 16 blocks (T11, T22 column by column on warp 0, then
+    // T21 = -T22 (A21 T11)), the two products on the tensor cores.  Meanwhile
+    // the other warps write the right-hand sides as dense K-major 128 x C
+    // operands, R_W^T into the e^G Q buffer and R_U^T into the W buffer
+    // (rows past d_k or d_v are zero).
+    if (warp == 0) {
+      const int c = lane, r0 = c & ~15;   // column c of the diagonal block at rows r0 ..
+      float x[16];
 #pragma unroll
-      for (int t = 0; t < C; ++t) {
-        float acc0 = isw ? fp(sWc, kmajor_pad_off<C>(t, tid))[0]
-                         : live ? sBeta[t] * __bfloat162float(sV[t * G::LDV + cu]) : 0.f;
-        float acc1 = 0.f;
-        const float* arow = sA + t * G::LDA;
+      for (int i = 0; i < 16; ++i) {
+        const int t = r0 + i;
+        const float* arow = sA + t * G::LDA + r0;
+        float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-        for (int s = 0; s + 3 < t; s += 4) {
-          const float4 a4 = *reinterpret_cast<const float4*>(arow + s);
-          acc0 = fmaf(-a4.x, x[s], acc0);
-          acc1 = fmaf(-a4.y, x[s + 1], acc1);
-          acc0 = fmaf(-a4.z, x[s + 2], acc0);
-          acc1 = fmaf(-a4.w, x[s + 3], acc1);
+        for (int k = 0; k + 1 < i; k += 2) {
+          acc0 = fmaf(-arow[k], x[k], acc0);
+          acc1 = fmaf(-arow[k + 1], x[k + 1], acc1);
         }
-#pragma unroll
-        for (int s = t & ~3; s < t; ++s) acc0 = fmaf(-arow[s], x[s], acc0);
-        x[t] = acc0 + acc1;
-        if (isw) fp(sWc, kmajor_pad_off<C>(t, tid))[0] = wm::__float_to_tf32(x[t]);
+        if (i & 1) acc0 = fmaf(-arow[i - 1], x[i - 1], acc0);
+        x[i] = t == c ? 1.f : t < c ? 0.f : acc0 + acc1;
+        sT[t * G::LDA + c] = x[i];
+        sT[(t ^ 16) * G::LDA + c] = 0.f;   // the other block row of column c: T12 = 0, T21 filled below
       }
-      if (isu) {   // whole warps: threads 128 .. 255
-        tmem_st32(tmem + lane_base + G::TM_U, x);
-        tmem_wait_st();
+    } else {   // four tokens of one key (one 16-byte run of the layout) a thread
+      for (int e = 4 * (tid - 32); e < 128 * C; e += 4 * (G::NT - 32)) {
+        int rr, s;
+        kmajor_rk(e, C, rr, s);
+        float4 w = make_float4(0.f, 0.f, 0.f, 0.f), u = w;
+        if (rr < DK) {
+          const __nv_bfloat16* kc = sK + s * G::LDK + rr;
+          w = make_float4(wm::__float_to_tf32(sBEG[s] * __bfloat162float(kc[0])),
+                          wm::__float_to_tf32(sBEG[s + 1] * __bfloat162float(kc[G::LDK])),
+                          wm::__float_to_tf32(sBEG[s + 2] * __bfloat162float(kc[2 * G::LDK])),
+                          wm::__float_to_tf32(sBEG[s + 3] * __bfloat162float(kc[3 * G::LDK])));
+        }
+        if (rr < DV) {
+          const __nv_bfloat16* vc = sV + s * G::LDV + rr;
+          u = make_float4(wm::__float_to_tf32(sBeta[s] * __bfloat162float(vc[0])),
+                          wm::__float_to_tf32(sBeta[s + 1] * __bfloat162float(vc[G::LDV])),
+                          wm::__float_to_tf32(sBeta[s + 2] * __bfloat162float(vc[2 * G::LDV])),
+                          wm::__float_to_tf32(sBeta[s + 3] * __bfloat162float(vc[3 * G::LDV])));
+        }
+        *reinterpret_cast<float4*>(sQc + 4 * e) = w;
+        *reinterpret_cast<float4*>(sWc + 4 * e) = u;
+      }
+    }
+    __syncthreads();
+    // The blocks hold explicit zeros above their diagonals, so both products
+    // run over all 16 terms.
+    if (tid < 256) {   // X = A21 T11
+      const int i = 16 + (tid >> 4), j = tid & 15;
+      float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+      for (int l = 0; l < 16; l += 2) {
+        acc0 = fmaf(sA[i * G::LDA + l], sT[l * G::LDA + j], acc0);
+        acc1 = fmaf(sA[i * G::LDA + l + 1], sT[(l + 1) * G::LDA + j], acc1);
+      }
+      sX[(i - 16) * 17 + j] = acc0 + acc1;
+    }
+    __syncthreads();
+    if (tid < 256) {   // T21 = -T22 X
+      const int i = 16 + (tid >> 4), j = tid & 15;
+      float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; k += 2) {
+        acc0 = fmaf(sT[i * G::LDA + 16 + k], sX[k * 17 + j], acc0);
+        acc1 = fmaf(sT[i * G::LDA + 17 + k], sX[(k + 1) * 17 + j], acc1);
+      }
+      sT[i * G::LDA + j] = -(acc0 + acc1);
+    }
+    __syncthreads();
+    for (int e = 4 * tid; e < C * C; e += 4 * G::NT) {   // T as the B operand (N = t, K = s), tf32
+      int t, s;
+      kmajor_rk(e, C, t, s);
+      const float* tr = sT + t * G::LDA + s;
+      *reinterpret_cast<float4*>(sPc + 4 * e) = make_float4(wm::__float_to_tf32(tr[0]), wm::__float_to_tf32(tr[1]),
+                                                            wm::__float_to_tf32(tr[2]), wm::__float_to_tf32(tr[3]));
+    }
+    fence_smem_to_async();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t ID = umma_idesc_tf32<128, C>();
+      const uint32_t t0 = smem_u32(sPc), rw = smem_u32(sQc), ru = smem_u32(sWc);
+#pragma unroll
+      for (int s = 0; s < C / 8; ++s)
+        umma_tf32_ss(tmem + G::TM_W, umma_desc(rw + 256 * s, (C / 4) * 128), umma_desc(t0 + 256 * s, (C / 4) * 128),
+                     ID, s > 0);
+#pragma unroll
+      for (int s = 0; s < C / 8; ++s)
+        umma_tf32_ss(tmem + G::TM_U, umma_desc(ru + 256 * s, (C / 4) * 128), umma_desc(t0 + 256 * s, (C / 4) * 128),
+                     ID, s > 0);
+      umma_commit(barT);
+    }
+    if (!mbar_wait_abortable(barT, par, sAbort) && tid == 0) atomicOr(a.err, kErrWaitTimeout);
+    tc_fence_after();
+    if (!*sAbort && c_own < DK) {   // W^T (key j on lane j) into W's padded operand layout, tf32
+      for (int b8 = group; b8 < C / 8; b8 += NG) {
+        float v[8];
+        tmem_ld8(tmem + lane_base + G::TM_W + 8 * b8, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) fp(sWc, kmajor_pad_off<C>(8 * b8 + i, c_own))[0] = wm::__float_to_tf32(v[i]);
       }
     }
     fence_smem_to_async();
+    tc_fence_before();
     __syncthreads();
     if (has_next) stage_rows(sV, Vg, c0 + C, DV, G::LDV);   // V of this chunk is consumed
     cp_async_commit();
@@ -419,10 +506,14 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_, DK_, DV_>::MINB) gdn_chu
     __syncthreads();
     lower_xyt<C, DK, G::LDK, G::LDA>(sQ, sK, sA);
     __syncthreads();
-    for (int e = tid; e < C * C; e += G::NT) {
+    for (int e = 4 * tid; e < C * C; e += 4 * G::NT) {   // four columns s of one row t a thread
       int t, s;
       kmajor_rk(e, C, t, s);
-      fp(sPc, 4 * e)[0] = s <= t ? wm::__float_to_tf32(expf(sG[t] - sG[s]) * sA[t * G::LDA + s]) : 0.f;
+      float p[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        p[i] = s + i <= t ? wm::__float_to_tf32(expf(sG[t] - sG[s + i]) * sA[t * G::LDA + s + i]) : 0.f;
+      *reinterpret_cast<float4*>(sPc + 4 * e) = make_float4(p[0], p[1], p[2], p[3]);
     }
     for (int idx = tid; idx < C * DK / 4; idx += G::NT) {   // e^G Q, four keys a thread
       const int t = idx / (DK / 4), j = 4 * (idx % (DK / 4));
@@ -433,10 +524,15 @@ __global__ void __launch_bounds__(NT_, TcChunkGeom<NT_, DK_, DV_>::MINB) gdn_chu
           make_float4(wm::__float_to_tf32(f * q4[0]), wm::__float_to_tf32(f * q4[1]), wm::__float_to_tf32(f * q4[2]),
                       wm::__float_to_tf32(f * q4[3]));
     }
-    for (int e = tid; e < DK * C; e += G::NT) {
+    for (int e = 4 * tid; e < DK * C; e += 4 * G::NT) {   // four tokens t of one key j a thread
       int j, t;
       kmajor_rk(e, C, j, t);
-      fp(sKc, 4 * e)[0] = wm::__float_to_tf32(sEnd[t] * __bfloat162float(sK[t * G::LDK + j]));
+      const __nv_bfloat16* kc = sK + t * G::LDK + j;
+      *reinterpret_cast<float4*>(sKc + 4 * e) =
+          make_float4(wm::__float_to_tf32(sEnd[t] * __bfloat162float(kc[0])),
+                      wm::__float_to_tf32(sEnd[t + 1] * __bfloat162float(kc[G::LDK])),
+                      wm::__float_to_tf32(sEnd[t + 2] * __bfloat162float(kc[2 * G::LDK])),
+                      wm::__float_to_tf32(sEnd[t + 3] * __bfloat162float(kc[3 * G::LDK])));
     }
     fence_smem_to_async();
     __syncthreads();
@@ -832,10 +928,11 @@ key_chunk_prefill_tc_kernel(const PrefillArgs a) {
     }
 
     // 5. P, the scaled queries and the scaled keys^T into their operand layouts
-    for (int e = tid; e < C * C; e += G::NT) {
+    for (int e = 4 * tid; e < C * C; e += 4 * G::NT) {   // tf32-rounded, zero above the diagonal
       int t, s;
       kmajor_rk(e, C, t, s);
-      fp(sPc, 4 * e)[0] = sP[t * G::LDA + s];   // tf32-rounded, zero above the diagonal
+      const float* pr = sP + t * G::LDA + s;
+      *reinterpret_cast<float4*>(sPc + 4 * e) = make_float4(pr[0], pr[1], pr[2], pr[3]);
     }
     for (int idx = tid; idx < C * DK / 4; idx += G::NT) {   // four keys a thread
       const int t = idx / (DK / 4), j = 4 * (idx % (DK / 4));
@@ -847,11 +944,16 @@ key_chunk_prefill_tc_kernel(const PrefillArgs a) {
           make_float4(wm::__float_to_tf32(ex2_approx(g.x) * q4[0]), wm::__float_to_tf32(ex2_approx(g.y) * q4[1]),
                       wm::__float_to_tf32(ex2_approx(g.z) * q4[2]), wm::__float_to_tf32(ex2_approx(g.w) * q4[3]));
     }
-    for (int e = tid; e < DK * C; e += G::NT) {
+    for (int e = 4 * tid; e < DK * C; e += 4 * G::NT) {   // four tokens t of one key j a thread
       int j, t;
       kmajor_rk(e, C, j, t);
-      fp(sKc, 4 * e)[0] = wm::__float_to_tf32(ex2_approx(sG[(C - 1) * G::LDG + j] - sG[t * G::LDG + j]) *
-                                               __bfloat162float(sK[t * G::LDK + j]));
+      const float gend = sG[(C - 1) * G::LDG + j];
+      float k4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        k4[i] = wm::__float_to_tf32(ex2_approx(gend - sG[(t + i) * G::LDG + j]) *
+                                    __bfloat162float(sK[(t + i) * G::LDK + j]));
+      *reinterpret_cast<float4*>(sKc + 4 * e) = make_float4(k4[0], k4[1], k4[2], k4[3]);
     }
     fence_smem_to_async();
     tc_fence_before();
