@@ -140,41 +140,124 @@ __device__ __forceinline__ void strict_pair(int p, int& t, int& s) {
   s = p - t * (t - 1) / 2;
 }
 
+// tf32 warp-MMA fragments (16 x 16 x 8) for the split-precision products
+using TfA = wm::fragment<wm::matrix_a, 16, 16, 8, wm::precision::tf32, wm::row_major>;
+using TfBc = wm::fragment<wm::matrix_b, 16, 16, 8, wm::precision::tf32, wm::col_major>;
+using AccTf = wm::fragment<wm::accumulator, 16, 16, 8, float>;
+
+// x = hi + lo with hi and lo both tf32 (hi the rounding of x)
+template <typename Frag>
+__device__ __forceinline__ void split_tf32(Frag& hi, Frag& lo) {
+#pragma unroll
+  for (int i = 0; i < hi.num_elements; ++i) {
+    const float x = hi.x[i];
+    hi.x[i] = wm::__float_to_tf32(x);
+    lo.x[i] = wm::__float_to_tf32(x - hi.x[i]);
+  }
+}
+
+// acc = X Y^T over columns [k0, k0 + KN) of fp32 X, Y [16][ldm], on one
+// warp, to about fp32 accuracy: with X = Xh + Xl and Y = Yh + Yl split into
+// tf32 parts, the sum Xl Yh + Xh Yl + Xh Yh (the Xl Yl term is below fp32
+// rounding).
+template <int KN>
+__device__ __forceinline__ void xyt_split_tf32(const float* X, const float* Y, int ldm, int k0, AccTf& acc) {
+  wm::fill_fragment(acc, 0.f);
+#pragma unroll
+  for (int k = k0; k < k0 + KN; k += 8) {
+    TfA xh, xl;
+    TfBc yh, yl;
+    wm::load_matrix_sync(xh, X + k, ldm);
+    wm::load_matrix_sync(yh, Y + k, ldm);
+    split_tf32(xh, xl);
+    split_tf32(yh, yl);
+    wm::mma_sync(acc, xl, yh, acc);
+    wm::mma_sync(acc, xh, yl, acc);
+    wm::mma_sync(acc, xh, yh, acc);
+  }
+}
+
 // A (KDA: beta_t-weighted, strictly lower) and P (lower; RWKV6: strictly
-// lower plus the bonus diagonal) of one chunk, pair by pair with one exp2 per
-// (pair, key) from Gamma in log2 units; the upper triangles zero.  P is stored
-// tf32-rounded.  When twice the strict pairs plus the diagonal make exactly
-// one item per thread, each strict pair is split between two adjacent lanes,
-// one half of the keys each.
-template <int OP, int DK, int C, int NT, int LDK, int LDG, int LDA>
+// lower plus the bonus diagonal) of one 32-token chunk, Gamma in log2 units;
+// the upper triangles zero, P tf32-rounded.
+//
+// Pairs inside one half of the chunk (t, s < 16 or t, s >= 16) take one
+// exp2 per (pair, key) on the SIMT lanes: 480 items, each strict pair split
+// into two halves of the keys on adjacent lanes, and the 32 diagonal pairs.
+// Pairs across the halves (t >= 16 > s) go through token 15:
+// 2^{Gamma_t - Gamma_s} = 2^{Gamma_t - Gamma_15} 2^{Gamma_15 - Gamma_s}, both
+// exponents <= 0 (Gamma_{t-1} in place of Gamma_t for RWKV6's P), so that
+// 16 x 16 block is a product of rows each scaled once: Ks (keys s < 16), Kt
+// (beta_t-weighted keys t >= 16, KDA) and Qt (queries t >= 16), fp32
+// [16][LDX], on warp MMAs in split tf32: four warps a product (KDA: warps
+// 0-3 A, 4-7 P; RWKV6: warps 0-3 P), each over a quarter of the keys, their
+// partial 16 x 16 blocks in sXA and sXP (fp32 [4][16][16]) and summed at the
+// end.  No cumulative decay is divided by.  Two block barriers inside; the
+// caller synchronises after the call.
+template <int OP, int DK, int C, int NT, int LDK, int LDG, int LDA, int LDX>
 __device__ __forceinline__ void key_pair_phase(const __nv_bfloat16* sK, const __nv_bfloat16* sQ, const float* sG,
-                                               const float* sBeta, const float* sBonus, float* sA, float* sP) {
+                                               const float* sBeta, const float* sBonus, float* sKs, float* sKt,
+                                               float* sQt, float* sXA, float* sXP, float* sA, float* sP) {
+  static_assert(C == 32, "two halves of 16 tokens");
+  static_assert(LDX % 4 == 0 && LDA % 4 == 0, "warp-MMA leading dimensions");
   constexpr bool DELTA = OP == OP_KDA;
-  const int tid = threadIdx.x;
-  constexpr int NSTRICT = C * (C - 1) / 2;
-  constexpr bool SPLIT = 2 * NSTRICT + C == NT;
-  constexpr int NITEMS = SPLIT ? NT : NSTRICT + C;
-  for (int p = tid; p < NITEMS; p += NT) {
-    const int nstr = SPLIT ? 2 * NSTRICT : NSTRICT;   // strict items come first
-    const bool strict = p < nstr;
-    int t, s;
-    if (strict) {
-      strict_pair(SPLIT ? p >> 1 : p, t, s);
-    } else {
-      t = s = p - nstr;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  // the scaled rows (four keys an item)
+  for (int idx = tid; idx < 16 * DK / 4; idx += NT) {
+    const int i = idx / (DK / 4), j = 4 * (idx % (DK / 4)), t = 16 + i;
+    const float4 gm = *reinterpret_cast<const float4*>(sG + 15 * LDG + j);
+    const float4 gs = *reinterpret_cast<const float4*>(sG + i * LDG + j);
+    const float4 gt = *reinterpret_cast<const float4*>(sG + (DELTA ? t : t - 1) * LDG + j);
+    const float es[4] = {ex2_approx(gm.x - gs.x), ex2_approx(gm.y - gs.y), ex2_approx(gm.z - gs.z),
+                         ex2_approx(gm.w - gs.w)};
+    const float et[4] = {ex2_approx(gt.x - gm.x), ex2_approx(gt.y - gm.y), ex2_approx(gt.z - gm.z),
+                         ex2_approx(gt.w - gm.w)};
+    float ks[4], kt[4], qt[4];
+    bf16x4_to_f32(sK + i * LDK + j, ks);
+    bf16x4_to_f32(sQ + t * LDK + j, qt);
+    *reinterpret_cast<float4*>(sKs + i * LDX + j) = make_float4(ks[0] * es[0], ks[1] * es[1], ks[2] * es[2], ks[3] * es[3]);
+    *reinterpret_cast<float4*>(sQt + i * LDX + j) = make_float4(qt[0] * et[0], qt[1] * et[1], qt[2] * et[2], qt[3] * et[3]);
+    if (DELTA) {
+      bf16x4_to_f32(sK + t * LDK + j, kt);
+      const float bt = sBeta[t];
+      *reinterpret_cast<float4*>(sKt + i * LDX + j) =
+          make_float4(bt * kt[0] * et[0], bt * kt[1] * et[1], bt * kt[2] * et[2], bt * kt[3] * et[3]);
     }
-    const int j0 = SPLIT && strict ? (p & 1) * (DK / 2) : 0;
-    const int j1 = SPLIT && strict ? j0 + DK / 2 : DK;
-    const __nv_bfloat16* kt = sK + t * LDK;
-    const __nv_bfloat16* ks = sK + s * LDK;
-    const __nv_bfloat16* qt = sQ + t * LDK;
+  }
+  __syncthreads();
+
+  // the block across the halves (rows 16.., columns ..15), partial sums
+  static_assert(NT >= 256, "eight warps for the two products");
+  if (warp < (DELTA ? 8 : 4)) {
+    const bool isA = DELTA && warp < 4;
+    const int w4 = warp & 3;
+    AccTf acc;
+    xyt_split_tf32<DK / 4>(isA ? sKt : sQt, sKs, LDX, w4 * (DK / 4), acc);
+    wm::store_matrix_sync((isA ? sXA : sXP) + w4 * 256, acc, 16, wm::mem_row_major);
+  }
+
+  constexpr int NSTR = 2 * 120;                 // strict pairs inside the halves
+  constexpr int NI = 2 * NSTR + C;
+  static_assert(NI % NT == 0 && (2 * NSTR) % 32 == 0, "items: whole rounds, warp-uniform kinds");
+#pragma unroll 1
+  for (int it = 0; it < NI / NT; ++it) {
+    const int p = it * NT + tid;
     float accA = 0.f, accP = 0.f;
-    if (strict) {
-      // exponent rows: Gamma_t (KDA) or Gamma_{t-1} (RWKV6), against Gamma_s
+    int t, s;
+    const bool strict = p < 2 * NSTR;
+    if (strict) {   // strict pair inside a half, keys [j0, j0 + DK / 2)
+      const int q = p >> 1, b = q >= 120 ? 1 : 0;
+      strict_pair(q - 120 * b, t, s);
+      t += 16 * b;
+      s += 16 * b;
+      const int j0 = (p & 1) * (DK / 2);
+      const __nv_bfloat16* kt = sK + t * LDK;
+      const __nv_bfloat16* ks = sK + s * LDK;
+      const __nv_bfloat16* qt = sQ + t * LDK;
       const float* gt = sG + (OP == OP_RWKV6 ? t - 1 : t) * LDG;
       const float* gs = sG + s * LDG;
 #pragma unroll 2
-      for (int j = j0; j < j1; j += 8) {
+      for (int j = j0; j < j0 + DK / 2; j += 8) {
         float fks[8], fqt[8], fkt[8];
         bf16x8_to_f32(ks + j, fks);
         bf16x8_to_f32(qt + j, fqt);
@@ -192,8 +275,10 @@ __device__ __forceinline__ void key_pair_phase(const __nv_bfloat16* sK, const __
           accP = fmaf(fqt[e], m, accP);
         }
       }
-    } else {
-      // diagonal: q_t . k_t (KDA), (u (.) k_t) . r_t (RWKV6)
+    } else {   // diagonal: q_t . k_t (KDA), (u (.) k_t) . r_t (RWKV6)
+      t = s = p - 2 * NSTR;
+      const __nv_bfloat16* kt = sK + t * LDK;
+      const __nv_bfloat16* qt = sQ + t * LDK;
 #pragma unroll 2
       for (int j = 0; j < DK; j += 8) {
         float fkt[8], fqt[8];
@@ -203,15 +288,14 @@ __device__ __forceinline__ void key_pair_phase(const __nv_bfloat16* sK, const __
         for (int e = 0; e < 8; ++e) accP = fmaf(fqt[e], OP == OP_RWKV6 ? sBonus[j + e] * fkt[e] : fkt[e], accP);
       }
     }
-    if (SPLIT) {   // one item per thread: every lane of the warp reaches the shuffles
-      const float oA = __shfl_xor_sync(0xffffffffu, accA, 1), oP = __shfl_xor_sync(0xffffffffu, accP, 1);
-      if (strict) {
-        accA += oA;
-        accP += oP;
-      }
+    // every lane of the warp reaches the shuffles (whole rounds of items)
+    const float oA = __shfl_xor_sync(0xffffffffu, accA, 1), oP = __shfl_xor_sync(0xffffffffu, accP, 1);
+    if (strict) {
+      accA += oA;
+      accP += oP;
     }
-    if (!SPLIT || !strict || (p & 1) == 0) {
-      if (DELTA && strict) sA[t * LDA + s] = sBeta[t] * accA;
+    if (!strict || (p & 1) == 0) {
+      if (DELTA && s < t) sA[t * LDA + s] = sBeta[t] * accA;
       sP[t * LDA + s] = wm::__float_to_tf32(accP);
     }
   }
@@ -219,6 +303,12 @@ __device__ __forceinline__ void key_pair_phase(const __nv_bfloat16* sK, const __
     const int t = idx / C, s = idx % C;
     if (s > t) sP[t * LDA + s] = 0.f;
     if (DELTA && s >= t) sA[t * LDA + s] = 0.f;
+  }
+  __syncthreads();   // the partial blocks are stored
+  for (int idx = tid; idx < 256; idx += NT) {
+    const int r = idx >> 4, c = idx & 15;
+    sP[(16 + r) * LDA + c] = wm::__float_to_tf32((sXP[idx] + sXP[256 + idx]) + (sXP[512 + idx] + sXP[768 + idx]));
+    if (DELTA) sA[(16 + r) * LDA + c] = (sXA[idx] + sXA[256 + idx]) + (sXA[512 + idx] + sXA[768 + idx]);
   }
 }
 

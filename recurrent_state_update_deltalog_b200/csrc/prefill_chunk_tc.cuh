@@ -656,8 +656,9 @@ cudaError_t launch_gdn_chunk_prefill_tc(const LaunchShape& s, const PrefillArgs&
 // ---- KDA and RWKV6 (per-key decay) ---------------------------------------------
 //
 // The per-key chunk form (prefill_chunk.cuh) with the same tensor-memory
-// state: A and P pair by pair on the SIMT lanes, the three products with the
-// state on tcgen05.  RWKV6 has no W S product: its B^T is
+// state: A and P on the SIMT lanes (pairs across the chunk's halves as
+// products of rows scaled once each), the blocked solve of the GDN kernel,
+// its two products and the three products with the state on tcgen05.  RWKV6 has no W S product: its B^T is
 // V^T, written straight into tensor memory.  The per-key decay of the state
 // update scales the columns of S^T.
 
@@ -670,8 +671,13 @@ struct KeyTcChunkGeom {
   static constexpr int NG = NW / 4;                 // column groups of the TMEM epilogues
   static constexpr int MINB = NT == 256 ? 2 : 1;
   static constexpr int LDK = DK + 8, LDV = DV + 8, LDG = DK + 4, LDA = C + 4;
+  static constexpr int LDX = DK + 4;                                   // fp32 rows scaled through token 15
   static constexpr uint32_t WQ_LBO = kmajor_pad_lbo<C>();             // W and scaled-query operand layout
-  static constexpr size_t WQ_BYTES = size_t(DK / 4) * WQ_LBO;
+  // the W and scaled-query buffers also hold the solve's right-hand sides
+  // R_W^T and R_U^T (dense K-major 128 x C) and, before them, the scaled rows
+  // of the pair phase (two [16][LDX] arrays in the scaled-query buffer)
+  static constexpr size_t WQ_MIN = size_t(128) * C * 4 > size_t(32) * LDX * 4 ? size_t(128) * C * 4 : size_t(32) * LDX * 4;
+  static constexpr size_t WQ_BYTES = size_t(DK / 4) * WQ_LBO > WQ_MIN ? size_t(DK / 4) * WQ_LBO : WQ_MIN;
   static constexpr size_t KQ_BYTES = tc_align128(size_t(C) * LDK * 2), V_BYTES = tc_align128(size_t(C) * LDV * 2);
   static constexpr size_t G_BYTES = tc_align128(size_t(C) * LDG * 4);
   // single-buffered inputs: the next chunk's V streams in once the solve has
@@ -687,10 +693,13 @@ struct KeyTcChunkGeom {
   static constexpr size_t PC_OFF = tc_align128(QC_OFF + WQ_BYTES);     // P, K-major C x C
   static constexpr size_t KC_OFF = PC_OFF + size_t(C) * C * 4;         // scaled keys^T, K-major DK x C
   static constexpr size_t E_OFF = tc_align128(KC_OFF + size_t(DK) * C * 4);  // e^{G_end} [DK], u [DK], beta [C]
-  static constexpr size_t BAR_OFF = tc_align128(E_OFF + (2 * DK + C) * 4);
+  static constexpr size_t T_OFF = tc_align128(E_OFF + (2 * DK + C) * 4);     // [C][LDA] T = (I + A)^-1 (KDA)
+  static constexpr size_t X_OFF = T_OFF + size_t(C) * LDA * 4;               // [16][17] A21 T11
+  static constexpr size_t BAR_OFF = tc_align128(X_OFF + 16 * 17 * 4);
   static constexpr size_t BYTES = BAR_OFF + 64;
-  // tensor-memory columns: S^T, W S then B^T, O^T, U^T (KDA; the solve writes it)
-  static constexpr uint32_t TM_COLS = 256, TM_S = 0, TM_B = DK, TM_O = DK + 32, TM_U = DK + 64;
+  // tensor-memory columns: S^T, W S then B^T, O^T, and the solve's products
+  // U^T and W^T (KDA)
+  static constexpr uint32_t TM_COLS = 256, TM_S = 0, TM_B = DK, TM_O = DK + 32, TM_U = DK + 64, TM_W = DK + 96;
 };
 
 template <int OP, int NT_, int DK_, int DV_>
@@ -716,12 +725,15 @@ key_chunk_prefill_tc_kernel(const PrefillArgs a) {
   float* sE = reinterpret_cast<float*>(smem + G::E_OFF);
   float* sBonus = sE + DK;
   float* sBeta = sE + 2 * DK;
+  float* sT = reinterpret_cast<float*>(smem + G::T_OFF);
+  float* sX = reinterpret_cast<float*>(smem + G::X_OFF);
   uint64_t* barB = reinterpret_cast<uint64_t*>(smem + G::BAR_OFF);
   uint64_t* barO = barB + 1;
   uint64_t* barS = barB + 2;
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(barB + 3);
   volatile int* sAbort = reinterpret_cast<volatile int*>(sTmem + 1);
   uint64_t* barF = barB + 4;                                          // drain after an abort
+  uint64_t* barT = barB + 5;                                          // the solve's products (KDA)
   auto fp = [](unsigned char* base, uint32_t off) { return reinterpret_cast<float*>(base + off); };
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -748,6 +760,7 @@ key_chunk_prefill_tc_kernel(const PrefillArgs a) {
     mbar_init(barO, 1);
     mbar_init(barS, 1);
     mbar_init(barF, 1);
+    mbar_init(barT, 1);
     fence_mbar_init();
     *sAbort = 0;
   }
@@ -841,59 +854,113 @@ key_chunk_prefill_tc_kernel(const PrefillArgs a) {
     }
     __syncthreads();
 
-    // 2. A and P pair by pair; right-hand sides (KDA)
-    key_pair_phase<OP, DK, C, G::NT, G::LDK, G::LDG, G::LDA>(sK, sQ, sG, sBeta, sBonus, sA, sP);
-    for (int idx = tid; idx < C * C; idx += G::NT) {
-      const int t = idx / C, s = idx % C;
-      if (s > t) sP[t * G::LDA + s] = 0.f;
-      if (DELTA && s >= t) sA[t * G::LDA + s] = 0.f;
-    }
-    if (DELTA) {
-      for (int idx = tid; idx < C * DK / 4; idx += G::NT) {
-        const int t = idx / (DK / 4), j = 4 * (idx % (DK / 4));
-        const float4 g = *reinterpret_cast<const float4*>(sG + t * G::LDG + j);
-        float k4[4];
-        bf16x4_to_f32(sK + t * G::LDK + j, k4);
-        const float bt = sBeta[t];
-        *reinterpret_cast<float4*>(sWc + kmajor_pad_off<C>(t, j)) =
-            make_float4(bt * ex2_approx(g.x) * k4[0], bt * ex2_approx(g.y) * k4[1], bt * ex2_approx(g.z) * k4[2],
-                        bt * ex2_approx(g.w) * k4[3]);
-      }
-    }
+    // 2. A and P; the rows scaled through token 15 sit in the scaled-query and
+    // W buffers, free until the solve, the partial products in the T and P
+    // operand buffers, free until then too
+    key_pair_phase<OP, DK, C, G::NT, G::LDK, G::LDG, G::LDA, G::LDX>(
+        sK, sQ, sG, sBeta, sBonus, fp(sQc, 0), fp(sQc, 16 * G::LDX * 4), fp(sWc, 0), sT, fp(sPc, 0), sA, sP);
     __syncthreads();
 
     if (DELTA) {
-      // 3. (I + A) X = R, one right-hand-side column per thread: W in shared
-      // memory, then its operand layout; U (right-hand side beta V read from V)
-      // into tensor memory, its column on this thread's TMEM lane
-      // W column j on thread j; U^T lane c on thread 128 + c (see the GDN kernel)
-      const bool isw = tid < DK, isu = tid >= 128 && tid < 256;
-      if (isw || isu) {
-        const int cu = tid - 128;
-        const bool live = isw || cu < DV;
-        float x[C];
+      // 3. (I + A) W = diag(beta) (2^Gamma (.) K) and (I + A) U = diag(beta) V as
+      // W^T = R_W^T T^T and U^T = R_U^T T^T with T = (I + A)^{-1}, as in the GDN
+      // kernel: T11 and T22 column by column on warp 0 while the other warps
+      // write R_W^T (into the scaled-query buffer) and R_U^T (into the W buffer)
+      // as dense K-major 128 x C operands, then T21 = -T22 (A21 T11), then the
+      // two products on the tensor cores.
+      if (warp == 0) {
+        const int c = lane, r0 = c & ~15;
+        float x[16];
 #pragma unroll
-        for (int t = 0; t < C; ++t) {
-          float acc0 = isw ? fp(sWc, kmajor_pad_off<C>(t, tid))[0]
-                           : live ? sBeta[t] * __bfloat162float(sV[t * G::LDV + cu]) : 0.f;
-          float acc1 = 0.f;
-          const float* arow = sA + t * G::LDA;
+        for (int i = 0; i < 16; ++i) {
+          const int t = r0 + i;
+          const float* arow = sA + t * G::LDA + r0;
+          float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-          for (int s = 0; s + 3 < t; s += 4) {
-            const float4 a4 = *reinterpret_cast<const float4*>(arow + s);
-            acc0 = fmaf(-a4.x, x[s], acc0);
-            acc1 = fmaf(-a4.y, x[s + 1], acc1);
-            acc0 = fmaf(-a4.z, x[s + 2], acc0);
-            acc1 = fmaf(-a4.w, x[s + 3], acc1);
+          for (int k = 0; k + 1 < i; k += 2) {
+            acc0 = fmaf(-arow[k], x[k], acc0);
+            acc1 = fmaf(-arow[k + 1], x[k + 1], acc1);
           }
-#pragma unroll
-          for (int s = t & ~3; s < t; ++s) acc0 = fmaf(-arow[s], x[s], acc0);
-          x[t] = acc0 + acc1;
-          if (isw) fp(sWc, kmajor_pad_off<C>(t, tid))[0] = wm::__float_to_tf32(x[t]);
+          if (i & 1) acc0 = fmaf(-arow[i - 1], x[i - 1], acc0);
+          x[i] = t == c ? 1.f : t < c ? 0.f : acc0 + acc1;
+          sT[t * G::LDA + c] = x[i];
+          sT[(t ^ 16) * G::LDA + c] = 0.f;
         }
-        if (isu) {   // whole warps: threads 128 .. 255
-          tmem_st32(tmem + lane_base + G::TM_U, x);
-          tmem_wait_st();
+      } else {   // four tokens of one key a thread
+        for (int e = 4 * (tid - 32); e < 128 * C; e += 4 * (G::NT - 32)) {
+          int rr, s;
+          kmajor_rk(e, C, rr, s);
+          float w[4] = {0.f, 0.f, 0.f, 0.f}, u[4] = {0.f, 0.f, 0.f, 0.f};
+          if (rr < DK) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              w[i] = wm::__float_to_tf32(sBeta[s + i] * ex2_approx(sG[(s + i) * G::LDG + rr]) *
+                                         __bfloat162float(sK[(s + i) * G::LDK + rr]));
+          }
+          if (rr < DV) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              u[i] = wm::__float_to_tf32(sBeta[s + i] * __bfloat162float(sV[(s + i) * G::LDV + rr]));
+          }
+          *reinterpret_cast<float4*>(sQc + 4 * e) = make_float4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<float4*>(sWc + 4 * e) = make_float4(u[0], u[1], u[2], u[3]);
+        }
+      }
+      __syncthreads();
+      if (tid < 256) {   // X = A21 T11 (zeros above the diagonals: 16 terms)
+        const int i = 16 + (tid >> 4), j = tid & 15;
+        float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+        for (int l = 0; l < 16; l += 2) {
+          acc0 = fmaf(sA[i * G::LDA + l], sT[l * G::LDA + j], acc0);
+          acc1 = fmaf(sA[i * G::LDA + l + 1], sT[(l + 1) * G::LDA + j], acc1);
+        }
+        sX[(i - 16) * 17 + j] = acc0 + acc1;
+      }
+      __syncthreads();
+      if (tid < 256) {   // T21 = -T22 X
+        const int i = 16 + (tid >> 4), j = tid & 15;
+        float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; k += 2) {
+          acc0 = fmaf(sT[i * G::LDA + 16 + k], sX[k * 17 + j], acc0);
+          acc1 = fmaf(sT[i * G::LDA + 17 + k], sX[(k + 1) * 17 + j], acc1);
+        }
+        sT[i * G::LDA + j] = -(acc0 + acc1);
+      }
+      __syncthreads();
+      for (int e = 4 * tid; e < C * C; e += 4 * G::NT) {   // T as the B operand (N = t, K = s), tf32
+        int t, s;
+        kmajor_rk(e, C, t, s);
+        const float* tr = sT + t * G::LDA + s;
+        *reinterpret_cast<float4*>(sPc + 4 * e) = make_float4(wm::__float_to_tf32(tr[0]), wm::__float_to_tf32(tr[1]),
+                                                              wm::__float_to_tf32(tr[2]), wm::__float_to_tf32(tr[3]));
+      }
+      fence_smem_to_async();
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t ID = umma_idesc_tf32<128, C>();
+        const uint32_t t0 = smem_u32(sPc), rw = smem_u32(sQc), ru = smem_u32(sWc);
+#pragma unroll
+        for (int s = 0; s < C / 8; ++s)
+          umma_tf32_ss(tmem + G::TM_W, umma_desc(rw + 256 * s, (C / 4) * 128), umma_desc(t0 + 256 * s, (C / 4) * 128),
+                       ID, s > 0);
+#pragma unroll
+        for (int s = 0; s < C / 8; ++s)
+          umma_tf32_ss(tmem + G::TM_U, umma_desc(ru + 256 * s, (C / 4) * 128), umma_desc(t0 + 256 * s, (C / 4) * 128),
+                       ID, s > 0);
+        umma_commit(barT);
+      }
+      if (!mbar_wait_abortable(barT, par, sAbort) && tid == 0) atomicOr(a.err, kErrWaitTimeout);
+      tc_fence_after();
+      if (!*sAbort && c_own < DK) {   // W^T (key j on lane j) into W's padded operand layout, tf32
+        for (int b8 = group; b8 < C / 8; b8 += NG) {
+          float v[8];
+          tmem_ld8(tmem + lane_base + G::TM_W + 8 * b8, v);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) fp(sWc, kmajor_pad_off<C>(8 * b8 + i, c_own))[0] = wm::__float_to_tf32(v[i]);
         }
       }
       fence_smem_to_async();

@@ -23,6 +23,10 @@ Expanding the per-token recurrences over C tokens gives these equations;
 this test checks that they hold (to fp64 rounding) for chunk sizes from 1 to
 past the prompt length, including a ragged last chunk, on the bench's input
 recipe and on strongly decaying gates.  It shares nothing with the CUDA code.
+
+Two rearrangements that the tensor-memory kernels make are checked as well:
+the pairs across the two halves of a 32-token chunk as a product of rows
+scaled once each through token 15, and (I + A)^{-1} by 16 x 16 blocks.
 """
 import numpy as np
 import pytest
@@ -113,3 +117,70 @@ def test_chunk_form_strong_decay(op):
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(S))
     assert np.abs(o - o_ref).max() <= 1e-12 * np.abs(o_ref).max()
     assert np.abs(S - S_ref).max() <= 1e-12 * np.abs(S_ref).max()
+
+
+def _pair_weights(K, Q, G, Gq, be):
+    """A and P of one chunk pair by pair (per-key weights e^{Gq_t - G_s})."""
+    n = len(K)
+    A, P = np.zeros((n, n)), np.zeros((n, n))
+    for t in range(n):
+        for s in range(t):
+            P[t, s] = np.sum(Q[t] * K[s] * np.exp(Gq[t] - G[s]))
+            if be is not None:
+                A[t, s] = be[t] * np.sum(K[t] * K[s] * np.exp(G[t] - G[s]))
+    return A, P
+
+
+@pytest.mark.parametrize("op", ["kda", "rwkv6"])
+@pytest.mark.parametrize("strong", [False, True])
+def test_pairs_across_halves_through_token_15(op, strong):
+    """The tensor-memory kernels form the 16 x 16 block of pairs t >= 16 > s of a
+    32-token chunk as a product of rows scaled once each, through token 15:
+    e^{G_t - G_s} = e^{G_t - G_15} e^{G_15 - G_s}.  Both exponents are <= 0 (no
+    cumulative decay is divided by) and the block equals the pair-by-pair one."""
+    d, C = 16, 32
+    seq = sequence(11, op, 1, 1, d, d, C, bf16=True)
+    one = _unit(seq, 0, 0)
+    g = one["log_decay"].astype(np.float64).copy()
+    if strong:
+        g[:, :5] = -40.0
+    G = np.cumsum(g, axis=0)
+    Gq = G if op == "kda" else np.vstack([np.zeros((1, d)), G[:-1]])   # Gamma_{t-1} for RWKV6's P
+    K = one["k"].astype(np.float64)
+    Q = one["r" if op == "rwkv6" else "q"].astype(np.float64)
+    be = one["beta"].astype(np.float64) if op == "kda" else None
+    A, P = _pair_weights(K, Q, G, Gq, be)
+
+    lo, hi = slice(0, 16), slice(16, 32)
+    ds, dt, dq = G[15] - G[lo], G[hi] - G[15], Gq[hi] - G[15]
+    assert ds.max() <= 0 and dt.max() <= 0 and dq.max() <= 0
+    Ks, Kt, Qt = K[lo] * np.exp(ds), K[hi] * np.exp(dt), Q[hi] * np.exp(dq)
+    scale = max(np.abs(P).max(), 1e-300)
+    assert np.abs(Qt @ Ks.T - P[hi, lo]).max() <= 1e-12 * scale
+    if be is not None:
+        assert np.abs(be[hi, None] * (Kt @ Ks.T) - A[hi, lo]).max() <= 1e-12 * np.abs(A).max()
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_blocked_inverse_of_unit_lower(seed):
+    """(I + A)^{-1} for a strictly lower 32 x 32 A as the kernels form it: the
+    diagonal blocks T11, T22 column by column by forward substitution, then
+    T21 = -T22 (A21 T11); T12 = 0.  Checked against a dense inverse, and
+    W = T R against a triangular solve."""
+    rng = np.random.default_rng(seed)
+    n = 32
+    A = np.tril(rng.standard_normal((n, n)) * 0.3, -1)
+    T = np.zeros((n, n))
+    for c in range(n):
+        r0 = c & ~15
+        x = np.zeros(16)
+        for i in range(16):
+            t = r0 + i
+            x[i] = 1.0 if t == c else 0.0 if t < c else -A[t, r0:r0 + i] @ x[:i]
+        T[r0:r0 + 16, c] = x
+    T[16:, :16] = -T[16:, 16:] @ (A[16:, :16] @ T[:16, :16])
+    I = np.eye(n)
+    ref = np.linalg.inv(I + A)
+    assert np.abs(T - ref).max() <= 1e-10 * np.abs(ref).max()
+    R = rng.standard_normal((n, 8))
+    assert np.allclose(T @ R, np.linalg.solve(I + A, R), rtol=0, atol=1e-10 * np.abs(R).max() * np.abs(ref).max())
