@@ -13,10 +13,11 @@
 // 0 .. 63 of the M = 128 products and keeps lanes 64 .. 127 zero: each row of
 // an MMA result depends only on the same row of its tensor-memory operand,
 // and every element-wise pass stays on its own lane.  B^T, O^T and U^T live
-// in tensor memory too (the triangular solve writes U^T there: each U column
-// is a thread whose TMEM lane is that value column).  W, the scaled queries,
-// P and the scaled keys are written by the SIMT lanes into shared memory in
-// K-major no-swizzle operand layouts.  One thread issues the MMAs; their
+// in tensor memory too.  The triangular solve forms T = (I + A)^{-1} in
+// 16 x 16 blocks on the SIMT lanes and W^T, U^T as two tcgen05 products with
+// T^T, into tensor memory.  W, the scaled queries, P, T, the solve's
+// right-hand sides and the scaled keys are written by the SIMT lanes into
+// shared memory in K-major no-swizzle operand layouts.  One thread issues the MMAs; their
 // completion is tracked by mbarriers (bounded waits: a wait that runs out
 // raises DL_DEVERR_WAIT_TIMEOUT and the CTA stops).  The state update of
 // chunk i runs while chunk i + 1 computes its gates, A and the solve.
@@ -140,8 +141,8 @@ constexpr size_t tc_align128(size_t x) { return (x + 127) & ~size_t(127); }
 // K-major operand of R rows whose 8-row groups are adjacent (stride byte
 // offset 128) and whose 16-byte k-chunks are R/8 x 128 + 16 bytes apart
 // (leading byte offset): the 16-byte pad puts the 32 consecutive k of one
-// row on 32 different banks, so a warp can write a row, or a column-parallel
-// solve can update one, without bank conflicts.
+// row on 32 different banks, so a warp writes a row (one k a lane, as the
+// copy of W^T out of tensor memory does) without bank conflicts.
 template <int R>
 __host__ __device__ constexpr uint32_t kmajor_pad_lbo() { return (R / 8) * 128 + 16; }
 template <int R>
