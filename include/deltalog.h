@@ -283,8 +283,8 @@ int dl_read_state(dl_t h, float* S_out, void* stream);
  * empty (DL_ERR_STATE otherwise). */
 /* DL_OPT_PREFILL_KERNEL picks the kernel behind dl_prefill:
  *   DL_PREFILL_AUTO (default): the chunked kernel for bf16-input handles
- *     whose prompts average at least 16 tokens (GDN, RWKV6) or 24 (KDA) at
- *     d_k = d_v = 128, and 32 (GDN, RWKV6) or 64 (KDA) at the other shapes;
+ *     whose prompts average at least 16 tokens at d_k = d_v = 128 and 32
+ *     at the other shapes;
  *     the recurrent kernel otherwise;
  *   DL_PREFILL_RECURRENT: the recurrence token by token, state in registers
  *     (every operator and dtype; outputs equal the eager recurrence's up to

@@ -305,17 +305,15 @@ cudaError_t materialize_slots(const dl_handle* h, const int* slot_idx, int rows,
 // The chunked prefills (state in tensor memory) serve bf16-input handles.
 // AUTO picks them once the prompts average enough tokens to fill their
 // 32-token chunks.  Measured on B200 against the recurrent kernel (bf16):
-//   d = 128, H = 32: GDN L=16 1.32, L=24 1.86, L=32 2.43, B=64 L=512 3.2;
-//               KDA L=16 0.94, L=24 1.37, L=32 1.77, B=64 L=512 2.09;
-//   d = 64:     GDN (H=32) L=32 1.15, B=64 L=512 1.58; KDA (H=32) L=32
-//               0.93, B=64 L=512 1.18; RWKV6 (H=64) L=32 1.05, L=64 1.18,
-//               B=64 L=512 1.38, B=4 L=4096 3.44.
-// Thresholds: 16 tokens (GDN, RWKV6) and 24 (KDA) at d_k = d_v = 128; 32
-// (GDN, RWKV6) and 64 (KDA) at the other shapes.
+//   d = 128, H = 32: GDN L=8 0.90, L=16 1.32, L=24 1.86, B=64 L=512 4.2;
+//               KDA L=16 1.05, B=64 L=512 2.4; RWKV6 L=8 0.69;
+//   d = 64:     GDN (H=32) L=16 0.73, L=32 1.15; KDA (H=32) L=32 1.10;
+//               RWKV6 (H=64) L=16 0.65, L=32 1.05, B=64 L=512 1.6.
+// Thresholds: 16 tokens at d_k = d_v = 128, 32 at the other shapes.
 bool chunked_prefill(const dl_handle* h, int rows, long long total) {
   if (h->prefill_kernel != DL_PREFILL_AUTO) return h->prefill_kernel == DL_PREFILL_CHUNKED;
   const bool big = h->dk == 128 && h->dv == 128;
-  const long long min_avg = h->op == DL_KDA ? (big ? 24 : 64) : (big ? 16 : 32);
+  const long long min_avg = big ? 16 : 32;
   return h->dtype == DL_BF16 && total >= min_avg * rows;
 }
 

@@ -99,7 +99,7 @@ def _prefill_then_decode(op, dims, dtype, kernel, H, log_lam_f16=False):
                   slot_idx=torch.tensor(slots, dtype=torch.int32, device="cuda"), zero_state=True)
     assert h.log_len == 2                                # the handle's cycle is unchanged
     big = (dk, dv) == (128, 128)   # the automatic rule
-    min_avg = (24 if big else 64) if op == "kda" else (16 if big else 32)
+    min_avg = 16 if big else 32
     auto_chunked = dtype == torch.bfloat16 and sum(lens) >= min_avg * rows
     want = "chunked" if kernel == "chunked" or (kernel == "auto" and auto_chunked) else "recurrent"
     assert h.last_prefill_kernel == want
