@@ -23,6 +23,8 @@ Prints ONE JSON line on rank 0.
 from __future__ import annotations
 
 import argparse
+import contextlib
+import gc
 import hashlib
 import json
 import os
@@ -40,6 +42,21 @@ L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0   # burst cuBLAS bf16 GEMM, an earlier B200 measurement
 
+
+
+@contextlib.contextmanager
+def no_gc():
+    """The Python collector off inside a timed region: a full collection can
+    stall the launching thread for milliseconds, long enough to drain the
+    GPU's queue of short launches."""
+    was = gc.isenabled()
+    gc.collect()
+    gc.disable()
+    try:
+        yield
+    finally:
+        if was:
+            gc.enable()
 
 def parse():
     ap = argparse.ArgumentParser()
@@ -563,11 +580,12 @@ def run_gpu(a, rank, world, local_rank):
                 run_graph_step(graphs, cyc)
             start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             barrier()
-            start.record(stream)
-            for _ in range(a.steps):
-                run_graph_step(graphs, cyc)
-            stop.record(stream)
-            barrier()
+            with no_gc():
+                start.record(stream)
+                for _ in range(a.steps):
+                    run_graph_step(graphs, cyc)
+                stop.record(stream)
+                barrier()
             ms = start.elapsed_time(stop)
             if not eager:
                 used_kernel[0] = h.last_step_kernel
@@ -584,11 +602,12 @@ def run_gpu(a, rank, world, local_rank):
               for _ in range(nev)]
         start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
-        start.record(stream)
-        for _ in range(steps):
-            run_step(h, m, eager, ev if per_launch else None, rec)
-        stop.record(stream)
-        barrier()
+        with no_gc():
+            start.record(stream)
+            for _ in range(steps):
+                run_step(h, m, eager, ev if per_launch else None, rec)
+            stop.record(stream)
+            barrier()
         ms = start.elapsed_time(stop)
         launches = None
         if per_launch:
@@ -673,11 +692,12 @@ def run_gpu(a, rank, world, local_rank):
             host_step()
         start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
-        start.record(stream)
-        for _ in range(a.steps):
-            host_step()
-        stop.record(stream)
-        barrier()
+        with no_gc():
+            start.record(stream)
+            for _ in range(a.steps):
+                host_step()
+            stop.record(stream)
+            barrier()
         e_ms = max_over_ranks(start.elapsed_time(stop))
         h.close()
         h2d = sum(host[nm][0].numel() * host[nm].element_size() for nm in names) * a.tokens
@@ -858,10 +878,11 @@ def eager_tokenwise(a, seq, names, first, u, stream, dev):
     eager_all()
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    eager_all()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
+    with no_gc():
+        e0.record(stream)
+        eager_all()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
     eager_ms = e0.elapsed_time(e1)
     return {"value": B * L / (eager_ms / 1e3), "unit": "tokens/s", "ms": eager_ms}
 
@@ -905,11 +926,12 @@ def run_prefill(a, rank, world, local_rank):
     sampler = ClockSampler(local_rank)
     sampler.start()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(a.steps):
-        once()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
+    with no_gc():
+        e0.record(stream)
+        for _ in range(a.steps):
+            once()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
     clocks = sampler.stop()
     ms = e0.elapsed_time(e1) / a.steps
     h.check_device()
