@@ -181,83 +181,117 @@ __device__ __forceinline__ void xyt_split_tf32(const float* X, const float* Y, i
 // lower plus the bonus diagonal) of one 32-token chunk, Gamma in log2 units;
 // the upper triangles zero, P tf32-rounded.
 //
-// Pairs inside one half of the chunk (t, s < 16 or t, s >= 16) take one
-// exp2 per (pair, key) on the SIMT lanes: 480 items, each strict pair split
-// into two halves of the keys on adjacent lanes, and the 32 diagonal pairs.
-// Pairs across the halves (t >= 16 > s) go through token 15:
-// 2^{Gamma_t - Gamma_s} = 2^{Gamma_t - Gamma_15} 2^{Gamma_15 - Gamma_s}, both
-// exponents <= 0 (Gamma_{t-1} in place of Gamma_t for RWKV6's P), so that
-// 16 x 16 block is a product of rows each scaled once: Ks (keys s < 16), Kt
-// (beta_t-weighted keys t >= 16, KDA) and Qt (queries t >= 16), fp32
-// [16][LDX], on warp MMAs in split tf32: four warps a product (KDA: warps
-// 0-3 A, 4-7 P; RWKV6: warps 0-3 P), each over a quarter of the keys, their
-// partial 16 x 16 blocks in sXA and sXP (fp32 [4][16][16]) and summed at the
-// end.  No cumulative decay is divided by.  Two block barriers inside; the
-// caller synchronises after the call.
+// A pair (t, s) with a token r between them (s <= r < t) factors as
+// 2^{Gamma_t - Gamma_s} = 2^{Gamma_t - Gamma_r} 2^{Gamma_r - Gamma_s}, both
+// exponents <= 0 (Gamma_{t-1} in place of Gamma_t for RWKV6's P, with
+// r <= t - 1), so a block of such pairs is a product of rows each scaled once
+// and no cumulative decay is divided by.  Blocks, by level:
+//   1. t >= 16 > s through token 15 (a 16 x 16 block);
+//   2. (256 threads) inside each half, t in its second quarter and s in its
+//      first, through token 7 or 23 (two 8 x 8 blocks, the diagonal blocks
+//      of one 16 x 16 product).
+// Each level's rows (Ks: keys s; Kt: beta_t-weighted keys t, KDA; Qt:
+// queries t; fp32 [16][LDX]) are products on warp MMAs in split tf32, four
+// warps a product (KDA: warps 0-3 A, 4-7 P; RWKV6: warps 0-3 P), each over a
+// quarter of the keys, with partial blocks in sXA and sXP (fp32 [4][16][16]).
+// The strict pairs left inside the quarters (112; 240 inside the halves at
+// 512 threads) and the 32 diagonal pairs take one exp2 per (pair, key) on the
+// SIMT lanes, a strict pair split over two adjacent lanes by keys: one item a
+// thread.  The second level pays at two CTAs an SM (B=64 L=512 on B200: KDA
+// +8%, RWKV6 +9% at d = 64 and +15% at d = 128) and costs 4% at one
+// 512-thread CTA an SM, whose threads the first level's items already fill.
+// Two block barriers inside (four with the second level); the caller
+// synchronises after the call.
 template <int OP, int DK, int C, int NT, int LDK, int LDG, int LDA, int LDX>
 __device__ __forceinline__ void key_pair_phase(const __nv_bfloat16* sK, const __nv_bfloat16* sQ, const float* sG,
                                                const float* sBeta, const float* sBonus, float* sKs, float* sKt,
                                                float* sQt, float* sXA, float* sXP, float* sA, float* sP) {
-  static_assert(C == 32, "two halves of 16 tokens");
+  static_assert(C == 32, "halves of 16 tokens, quarters of 8");
   static_assert(LDX % 4 == 0 && LDA % 4 == 0, "warp-MMA leading dimensions");
+  static_assert(NT == 256 || NT == 512, "eight or sixteen warps");
   constexpr bool DELTA = OP == OP_KDA;
   const int tid = threadIdx.x, warp = tid >> 5;
-  // the scaled rows (four keys an item)
-  for (int idx = tid; idx < 16 * DK / 4; idx += NT) {
-    const int i = idx / (DK / 4), j = 4 * (idx % (DK / 4)), t = 16 + i;
-    const float4 gm = *reinterpret_cast<const float4*>(sG + 15 * LDG + j);
-    const float4 gs = *reinterpret_cast<const float4*>(sG + i * LDG + j);
-    const float4 gt = *reinterpret_cast<const float4*>(sG + (DELTA ? t : t - 1) * LDG + j);
-    const float es[4] = {ex2_approx(gm.x - gs.x), ex2_approx(gm.y - gs.y), ex2_approx(gm.z - gs.z),
-                         ex2_approx(gm.w - gs.w)};
-    const float et[4] = {ex2_approx(gt.x - gm.x), ex2_approx(gt.y - gm.y), ex2_approx(gt.z - gm.z),
-                         ex2_approx(gt.w - gm.w)};
-    float ks[4], kt[4], qt[4];
-    bf16x4_to_f32(sK + i * LDK + j, ks);
-    bf16x4_to_f32(sQ + t * LDK + j, qt);
-    *reinterpret_cast<float4*>(sKs + i * LDX + j) = make_float4(ks[0] * es[0], ks[1] * es[1], ks[2] * es[2], ks[3] * es[3]);
-    *reinterpret_cast<float4*>(sQt + i * LDX + j) = make_float4(qt[0] * et[0], qt[1] * et[1], qt[2] * et[2], qt[3] * et[3]);
-    if (DELTA) {
-      bf16x4_to_f32(sK + t * LDK + j, kt);
-      const float bt = sBeta[t];
-      *reinterpret_cast<float4*>(sKt + i * LDX + j) =
-          make_float4(bt * kt[0] * et[0], bt * kt[1] * et[1], bt * kt[2] * et[2], bt * kt[3] * et[3]);
+
+  // the rows of one level: row i pairs key s, token t and reference r
+  auto scale_rows = [&](int level) {
+    for (int idx = tid; idx < 16 * DK / 4; idx += NT) {
+      const int i = idx / (DK / 4), j = 4 * (idx % (DK / 4));
+      const int s = level == 1 ? i : 16 * (i >> 3) + (i & 7);
+      const int t = level == 1 ? 16 + i : s + 8;
+      const int r = level == 1 ? 15 : 16 * (i >> 3) + 7;
+      const float4 gm = *reinterpret_cast<const float4*>(sG + r * LDG + j);
+      const float4 gs = *reinterpret_cast<const float4*>(sG + s * LDG + j);
+      const float4 gt = *reinterpret_cast<const float4*>(sG + (DELTA ? t : t - 1) * LDG + j);
+      const float es[4] = {ex2_approx(gm.x - gs.x), ex2_approx(gm.y - gs.y), ex2_approx(gm.z - gs.z),
+                           ex2_approx(gm.w - gs.w)};
+      const float et[4] = {ex2_approx(gt.x - gm.x), ex2_approx(gt.y - gm.y), ex2_approx(gt.z - gm.z),
+                           ex2_approx(gt.w - gm.w)};
+      float ks[4], kt[4], qt[4];
+      bf16x4_to_f32(sK + s * LDK + j, ks);
+      bf16x4_to_f32(sQ + t * LDK + j, qt);
+      *reinterpret_cast<float4*>(sKs + i * LDX + j) =
+          make_float4(ks[0] * es[0], ks[1] * es[1], ks[2] * es[2], ks[3] * es[3]);
+      *reinterpret_cast<float4*>(sQt + i * LDX + j) =
+          make_float4(qt[0] * et[0], qt[1] * et[1], qt[2] * et[2], qt[3] * et[3]);
+      if (DELTA) {
+        bf16x4_to_f32(sK + t * LDK + j, kt);
+        const float bt = sBeta[t];
+        *reinterpret_cast<float4*>(sKt + i * LDX + j) =
+            make_float4(bt * kt[0] * et[0], bt * kt[1] * et[1], bt * kt[2] * et[2], bt * kt[3] * et[3]);
+      }
     }
-  }
+  };
+  // the level's 16 x 16 products, partial sums a quarter of the keys each
+  auto products = [&]() {
+    if (warp < (DELTA ? 8 : 4)) {
+      const bool isA = DELTA && warp < 4;
+      const int w4 = warp & 3;
+      AccTf acc;
+      xyt_split_tf32<DK / 4>(isA ? sKt : sQt, sKs, LDX, w4 * (DK / 4), acc);
+      wm::store_matrix_sync((isA ? sXA : sXP) + w4 * 256, acc, 16, wm::mem_row_major);
+    }
+  };
+  // entry e of the 16 x 16 product into (t, s)
+  auto sum_entry = [&](int e, int t, int s) {
+    sP[t * LDA + s] = wm::__float_to_tf32((sXP[e] + sXP[256 + e]) + (sXP[512 + e] + sXP[768 + e]));
+    if (DELTA) sA[t * LDA + s] = (sXA[e] + sXA[256 + e]) + (sXA[512 + e] + sXA[768 + e]);
+  };
+
+  constexpr bool TWO = NT == 256;             // the second level of blocks
+  scale_rows(1);
   __syncthreads();
-
-  // the block across the halves (rows 16.., columns ..15), partial sums
-  static_assert(NT >= 256, "eight warps for the two products");
-  if (warp < (DELTA ? 8 : 4)) {
-    const bool isA = DELTA && warp < 4;
-    const int w4 = warp & 3;
-    AccTf acc;
-    xyt_split_tf32<DK / 4>(isA ? sKt : sQt, sKs, LDX, w4 * (DK / 4), acc);
-    wm::store_matrix_sync((isA ? sXA : sXP) + w4 * 256, acc, 16, wm::mem_row_major);
+  products();
+  if (TWO) {
+    __syncthreads();
+    for (int idx = tid; idx < 256; idx += NT) sum_entry(idx, 16 + (idx >> 4), idx & 15);
+    scale_rows(2);
+    __syncthreads();
+    products();
   }
 
-  constexpr int NSTR = 2 * 120;                 // strict pairs inside the halves
-  constexpr int NI = 2 * NSTR + C;
-  static_assert(NI % NT == 0 && (2 * NSTR) % 32 == 0, "items: whole rounds, warp-uniform kinds");
-#pragma unroll 1
-  for (int it = 0; it < NI / NT; ++it) {
-    const int p = it * NT + tid;
+  // the strict pairs left (two lanes each) and the diagonal, one item a thread
+  constexpr int BS = TWO ? 8 : 16;              // the blocks they sit in
+  constexpr int NPB = BS * (BS - 1) / 2, KS = 2;
+  constexpr int NSPLIT = (C / BS) * NPB * KS, NI = NSPLIT + C;
+  static_assert(NI == NT && NSPLIT % 32 == 0, "one round, warp-uniform kinds");
+  {
+    const int p = tid;
     float accA = 0.f, accP = 0.f;
-    int t, s;
-    const bool strict = p < 2 * NSTR;
-    if (strict) {   // strict pair inside a half, keys [j0, j0 + DK / 2)
-      const int q = p >> 1, b = q >= 120 ? 1 : 0;
-      strict_pair(q - 120 * b, t, s);
-      t += 16 * b;
-      s += 16 * b;
-      const int j0 = (p & 1) * (DK / 2);
+    int t = 0, s = 0;
+    const bool split = p < NSPLIT;
+    if (split) {   // strict pair inside a block, keys [j0, j0 + DK / KS)
+      const int q = p / KS, b = q / NPB;
+      strict_pair(q - NPB * b, t, s);
+      t += BS * b;
+      s += BS * b;
+      const int j0 = (p % KS) * (DK / KS);
       const __nv_bfloat16* kt = sK + t * LDK;
       const __nv_bfloat16* ks = sK + s * LDK;
       const __nv_bfloat16* qt = sQ + t * LDK;
       const float* gt = sG + (OP == OP_RWKV6 ? t - 1 : t) * LDG;
       const float* gs = sG + s * LDG;
 #pragma unroll 2
-      for (int j = j0; j < j0 + DK / 2; j += 8) {
+      for (int j = j0; j < j0 + DK / KS; j += 8) {
         float fks[8], fqt[8], fkt[8];
         bf16x8_to_f32(ks + j, fks);
         bf16x8_to_f32(qt + j, fqt);
@@ -276,7 +310,7 @@ __device__ __forceinline__ void key_pair_phase(const __nv_bfloat16* sK, const __
         }
       }
     } else {   // diagonal: q_t . k_t (KDA), (u (.) k_t) . r_t (RWKV6)
-      t = s = p - 2 * NSTR;
+      t = s = p - NSPLIT;
       const __nv_bfloat16* kt = sK + t * LDK;
       const __nv_bfloat16* qt = sQ + t * LDK;
 #pragma unroll 2
@@ -288,27 +322,33 @@ __device__ __forceinline__ void key_pair_phase(const __nv_bfloat16* sK, const __
         for (int e = 0; e < 8; ++e) accP = fmaf(fqt[e], OP == OP_RWKV6 ? sBonus[j + e] * fkt[e] : fkt[e], accP);
       }
     }
-    // every lane of the warp reaches the shuffles (whole rounds of items)
-    const float oA = __shfl_xor_sync(0xffffffffu, accA, 1), oP = __shfl_xor_sync(0xffffffffu, accP, 1);
-    if (strict) {
-      accA += oA;
-      accP += oP;
+    // every lane of the warp reaches the shuffles
+#pragma unroll
+    for (int o = 1; o < KS; o <<= 1) {
+      const float oA = __shfl_xor_sync(0xffffffffu, accA, o), oP = __shfl_xor_sync(0xffffffffu, accP, o);
+      if (split) {
+        accA += oA;
+        accP += oP;
+      }
     }
-    if (!strict || (p & 1) == 0) {
+    if (!split || p % KS == 0) {
       if (DELTA && s < t) sA[t * LDA + s] = sBeta[t] * accA;
       sP[t * LDA + s] = wm::__float_to_tf32(accP);
     }
+  }
+  __syncthreads();   // the last level's partial blocks are stored
+  if (TWO) {
+    for (int idx = tid; idx < 128; idx += NT) {   // the two 8 x 8 diagonal blocks of that product
+      const int b = idx >> 6, r = (idx >> 3) & 7, c = idx & 7;
+      sum_entry((8 * b + r) * 16 + 8 * b + c, 16 * b + 8 + r, 16 * b + c);
+    }
+  } else {
+    for (int idx = tid; idx < 256; idx += NT) sum_entry(idx, 16 + (idx >> 4), idx & 15);
   }
   for (int idx = tid; idx < C * C; idx += NT) {
     const int t = idx / C, s = idx % C;
     if (s > t) sP[t * LDA + s] = 0.f;
     if (DELTA && s >= t) sA[t * LDA + s] = 0.f;
-  }
-  __syncthreads();   // the partial blocks are stored
-  for (int idx = tid; idx < 256; idx += NT) {
-    const int r = idx >> 4, c = idx & 15;
-    sP[(16 + r) * LDA + c] = wm::__float_to_tf32((sXP[idx] + sXP[256 + idx]) + (sXP[512 + idx] + sXP[768 + idx]));
-    if (DELTA) sA[(16 + r) * LDA + c] = (sXA[idx] + sXA[256 + idx]) + (sXA[512 + idx] + sXA[768 + idx]);
   }
 }
 

@@ -25,8 +25,9 @@ past the prompt length, including a ragged last chunk, on the bench's input
 recipe and on strongly decaying gates.  It shares nothing with the CUDA code.
 
 Two rearrangements that the tensor-memory kernels make are checked as well:
-the pairs across the two halves of a 32-token chunk as a product of rows
-scaled once each through token 15, and (I + A)^{-1} by 16 x 16 blocks.
+blocks of pairs of a 32-token chunk as products of rows scaled once each
+through a token between them (tokens 15, 7 and 23), and (I + A)^{-1} by
+16 x 16 blocks.
 """
 import numpy as np
 import pytest
@@ -133,11 +134,14 @@ def _pair_weights(K, Q, G, Gq, be):
 
 @pytest.mark.parametrize("op", ["kda", "rwkv6"])
 @pytest.mark.parametrize("strong", [False, True])
-def test_pairs_across_halves_through_token_15(op, strong):
-    """The tensor-memory kernels form the 16 x 16 block of pairs t >= 16 > s of a
-    32-token chunk as a product of rows scaled once each, through token 15:
-    e^{G_t - G_s} = e^{G_t - G_15} e^{G_15 - G_s}.  Both exponents are <= 0 (no
-    cumulative decay is divided by) and the block equals the pair-by-pair one."""
+def test_pair_blocks_through_a_reference_token(op, strong):
+    """The tensor-memory kernels form blocks of pairs of a 32-token chunk as
+    products of rows scaled once each, through a token r between s and t:
+    e^{G_t - G_s} = e^{G_t - G_r} e^{G_r - G_s}.  The 16 x 16 block t >= 16 > s
+    goes through token 15; inside each half, the 8 x 8 block of its second
+    quarter against its first goes through token 7 or 23.  Every exponent is
+    <= 0 (no cumulative decay is divided by) and each block equals the
+    pair-by-pair one."""
     d, C = 16, 32
     seq = sequence(11, op, 1, 1, d, d, C, bf16=True)
     one = _unit(seq, 0, 0)
@@ -151,14 +155,19 @@ def test_pairs_across_halves_through_token_15(op, strong):
     be = one["beta"].astype(np.float64) if op == "kda" else None
     A, P = _pair_weights(K, Q, G, Gq, be)
 
-    lo, hi = slice(0, 16), slice(16, 32)
-    ds, dt, dq = G[15] - G[lo], G[hi] - G[15], Gq[hi] - G[15]
-    assert ds.max() <= 0 and dt.max() <= 0 and dq.max() <= 0
-    Ks, Kt, Qt = K[lo] * np.exp(ds), K[hi] * np.exp(dt), Q[hi] * np.exp(dq)
-    scale = max(np.abs(P).max(), 1e-300)
-    assert np.abs(Qt @ Ks.T - P[hi, lo]).max() <= 1e-12 * scale
-    if be is not None:
-        assert np.abs(be[hi, None] * (Kt @ Ks.T) - A[hi, lo]).max() <= 1e-12 * np.abs(A).max()
+    # level 1: t >= 16 > s through token 15; level 2: second quarter against
+    # first quarter of each half, through token 7 or 23
+    blocks = [(slice(16, 32), slice(0, 16), 15), (slice(8, 16), slice(0, 8), 7), (slice(24, 32), slice(16, 24), 23)]
+    for hi, lo, r in blocks:
+        ds, dt, dq = G[r] - G[lo], G[hi] - G[r], Gq[hi] - G[r]
+        assert ds.max() <= 0 and dt.max() <= 0 and dq.max() <= 0
+        Ks, Kt, Qt = K[lo] * np.exp(ds), K[hi] * np.exp(dt), Q[hi] * np.exp(dq)
+        assert np.abs(Qt @ Ks.T - P[hi, lo]).max() <= 1e-12 * max(np.abs(P).max(), 1e-300), r
+        if be is not None:
+            assert np.abs(be[hi, None] * (Kt @ Ks.T) - A[hi, lo]).max() <= 1e-12 * np.abs(A).max(), r
+    # what is left pair by pair: the strict pairs inside the four quarters
+    left = sum(1 for t in range(C) for s_ in range(t) if t // 8 == s_ // 8)
+    assert left == 4 * 28
 
 
 @pytest.mark.parametrize("seed", [0, 1, 2])
