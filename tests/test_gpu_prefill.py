@@ -248,11 +248,14 @@ def test_chunked_prefill_refused_where_it_does_not_apply():
 
 
 @pytest.mark.parametrize("op,kernel", [(op, k) for op in OPS for k in ("recurrent", "chunked")])
-@pytest.mark.parametrize("d,H", [(64, 2), (128, 2), (128, 48)])
+@pytest.mark.parametrize("d,H", [(64, 2), (128, 2), (128, 48), (128, 96), (64, 80)])
 def test_prefill_strong_decay(op, kernel, d, H):
     """Log-decays of -40 per token (on three keys for KDA/RWKV6, on every
     tenth token for GDN): cumulative decays far past fp32 range inside a
-    chunk, which no kernel may divide by."""
+    chunk, which no kernel may divide by.  Two rows of H = 96 or 80 heads
+    launch more CTAs than the GPU has SMs, so the chunked kernels run their
+    256-thread variant (for KDA and RWKV6, with both levels of pair blocks);
+    the smaller cases run the 512-thread one."""
     from recurrent_state_update_deltalog_b200 import DeltaLog
     dtype, lens = torch.bfloat16, [100, 37]
     rows = len(lens)
