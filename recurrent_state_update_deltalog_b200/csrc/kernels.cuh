@@ -157,6 +157,16 @@ __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return
 __device__ __forceinline__ float4 ld_state(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }
 __device__ __forceinline__ void st_state(float* p, float4 v) { __stcs(reinterpret_cast<float4*>(p), v); }
 
+// e^x as 2^(x log2 e) on the SFU (ex2.approx): relative error about 2^-22,
+// plus the rounding of x log2 e (2^-24 |x| in the exponent); results below
+// the normal range flush to zero.  The ratios exp(Lam_t - Lam_i) <= 1 of the
+// replay take it: a few instructions each on every CTA's serial path.
+__device__ __forceinline__ float exp_sfu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x * 1.4426950408889634f));
+  return y;
+}
+
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
   for (int m = 16; m > 0; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
@@ -498,12 +508,12 @@ deltalog_step_kernel(const StepArgs a) {
         const int j = lane + 32 * m;
         const float ai = to_f(sA[i * DK + j]);
         const float lam_i = PERKEY ? sL[i * DK + j] : s_lam[i];
-        const float r_t = expf(lt[m] - lam_i);                 // ratio to Lam_t
+        const float r_t = exp_sfu(lt[m] - lam_i);              // ratio to Lam_t
         if (DELTA) {
           dk = fmaf(r_t * ai, kr[m], dk);
           dq = fmaf(r_t * ai, qr[m], dq);
         } else {
-          const float r_p = expf(lp[m] - lam_i);               // RWKV6 reads S_{t-1}
+          const float r_p = exp_sfu(lp[m] - lam_i);            // RWKV6 reads S_{t-1}
           dq = fmaf(r_p * ai, qr[m], dq);
         }
         if (MERGE) As[i * DK + j] = r_t * ai;
@@ -535,12 +545,12 @@ deltalog_step_kernel(const StepArgs a) {
 #pragma unroll
     for (int m = 0; m < TL::KPL; ++m) {
       const int j = lane + 32 * m;
-      const float et = expf(lt[m]);
+      const float et = exp_sfu(lt[m]);
       if (DELTA) {
         s_kt[j] = et * kr[m];
         s_qt[j] = et * qr[m];
       } else {
-        s_qt[j] = expf(lp[m]) * qr[m];
+        s_qt[j] = exp_sfu(lp[m]) * qr[m];
       }
       if (MERGE) s_dec[j] = et;
     }
