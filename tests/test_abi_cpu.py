@@ -135,8 +135,8 @@ def test_suggest_m_near_stationary_point(lib, op, dk, dv, dtype):
 
 
 @pytest.mark.parametrize("op,d,band", [
-    (0, 128, (7, 12)), (1, 128, (7, 12)), (2, 64, (6, 11)),
-    (0, 64, (8, 12)), (1, 64, (5, 9)), (2, 128, (7, 12)),
+    (0, 128, (9, 12)), (1, 128, (7, 11)), (2, 64, (8, 9)),
+    (0, 64, (9, 12)), (1, 64, (5, 8)), (2, 128, (8, 12)),
 ])
 def test_suggest_m_inside_measured_band(lib, op, d, band):
     """Within the band of M whose measured B200 throughput is within 1% of
