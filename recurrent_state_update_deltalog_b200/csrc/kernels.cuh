@@ -195,22 +195,27 @@ constexpr int kMaxM = 64;
 
 template <int DK, int DV>
 struct Tile {
-  static constexpr int NT = 2 * DV;      // threads per CTA
+  // The whole 64 x 64 tile (a d = 64 head, one value tile) runs on 64 threads
+  // with 16 rows each ("slim"); every other tile on 2 DV threads with DK / 8
+  // rows each.
+  static constexpr bool SLIM = DK == 64 && DV == 64;
+  static constexpr int NT = SLIM ? 64 : 2 * DV;   // threads per CTA
   static constexpr int TPR = DV / 4;     // threads that cover one state row with float4s
-  static constexpr int RG = NT / TPR;    // row groups (= 8)
+  static constexpr int RG = NT / TPR;    // row groups (8; 4 for the slim tile)
   static constexpr int RPT = DK / RG;    // rows held by each thread
   static constexpr int NW = NT / 32;     // warps
   static constexpr int KPL = DK / 32;    // keys per lane in warp-wide key loops
-  // CTAs per SM the register budget is sized for: d_k = 64 tiles keep only
-  // 32 state registers per thread, so eight 128-thread CTAs (64 registers
-  // each) fit and keep 128 KB of state loads in flight per SM.
+  // CTAs per SM the register budget is sized for.  128-thread tiles at d_k =
+  // 64 keep 32 state registers per thread, so eight CTAs (64 registers each)
+  // fit; the slim tile keeps 64 and fits eight at 128 registers.
   static constexpr int MINB = NT >= 256 ? 2 : (NT >= 128 ? (DK == 64 ? 8 : 4) : 8);
-  // Append launches of 128-thread tiles at d_k = 128 fit five CTAs per SM (96
-  // registers, no spills) and so keep 160 KB of state loads in flight per SM
-  // instead of 128 KB; measured on B200, GDN B=256 appends 86.9 -> 83.8 us.
-  // Six (80 registers) spill and lose; merge launches need their 128.
-  static constexpr int MINB_APPEND = (NT == 128 && DK == 128) ? 5 : MINB;
-  static_assert(DV % 32 == 0 && DK % 32 == 0 && RG == 8 && RPT % 4 == 0, "tile shape");
+  // Append launches keep more state loads in flight per SM: 128-thread tiles
+  // at d_k = 128 fit five CTAs (96 registers, no spills), 160 KB instead of
+  // 128 KB; measured on B200, GDN B=256 appends 86.9 -> 83.8 us.  Six (80
+  // registers) spill and lose; merge launches need their 128.  The slim tile
+  // fits ten (102 registers), also 160 KB.
+  static constexpr int MINB_APPEND = (NT == 128 && DK == 128) ? 5 : (SLIM ? 10 : MINB);
+  static_assert(DV % 32 == 0 && DK % 32 == 0 && (RG == 8 || (SLIM && RG == 4)) && RPT % 4 == 0, "tile shape");
   static_assert(NT >= kMaxM - 1 && DV <= NT, "one thread per log entry / value column in setup phases");
 };
 
